@@ -1,0 +1,208 @@
+/*
+ * rdt.h — C ABI of librdt: the looped Recurrent Block of the OpenMythos
+ * Recurrent-Depth Transformer on one B200 (sm_100a).
+ *
+ * Conventions (all entry points):
+ *  - Every pointer argument named as "device" is a device pointer owned by the
+ *    caller.  The library allocates nothing on these paths; scratch memory is the
+ *    caller's workspace `ws` of at least rdt_workspace_size() bytes, 256-byte aligned.
+ *  - Matrices are row-major.  Weight matrices use the nn.Linear layout
+ *    [out_features, in_features] and are stored in the model dtype
+ *    (cfg->dtype: 0 = fp32, 1 = bf16).  Vectors marked "fp32" are always fp32.
+ *  - Activations are sequence-major rows: row = b * seq + i for sequence b,
+ *    position i.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All calls only
+ *    enqueue work on it and return, except rdt_read_device_status (synchronises).
+ *  - Arguments are validated on the host before anything is launched; a bad
+ *    argument returns RDT_ERR_INVALID_ARG (or RDT_ERR_UNSUPPORTED for a valid but
+ *    unimplemented shape) with nothing enqueued.  No C++ exception crosses the ABI.
+ *  - Kernels that detect an inconsistency on the device (an index out of range)
+ *    record it in a status word inside the workspace instead of trapping; read it
+ *    with rdt_read_device_status.
+ *
+ * Page references (titles and sections of the extracted web pages):
+ *  "OpenMythos 분석" (zero.shotlearni.ng): Core Structure, Recurrent Block, latent
+ *  reasoning, Repeating the parameter reduces expressiveness, MoE, MLA, RoPE &
+ *  generation cache, ACT.  "OpenMythos" README mirror (runchr.com): 사용법,
+ *  모델 변형, Attention 구현, 동적 시스템 관점, 해결책.
+ */
+#ifndef RDT_H_
+#define RDT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RDT_API __attribute__((visibility("default")))
+#else
+#define RDT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RDT_OK = 0,
+  RDT_ERR_INVALID_ARG = 1,     /* null pointer, bad size, inconsistent config       */
+  RDT_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. MLA decode)        */
+  RDT_ERR_WORKSPACE = 3,       /* ws too small or misaligned                          */
+  RDT_ERR_CUDA = 4,            /* a CUDA runtime call failed                          */
+  RDT_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait gave up                  */
+  RDT_ERR_DEVICE_BOUNDS = 6    /* a device-side index check failed                   */
+} rdt_status;
+
+/* Mirror of MythosConfig (README mirror, 사용법) narrowed to the recurrent block,
+ * plus the constants the pages leave open. */
+typedef struct {
+  int dim;                 /* D                                                    */
+  int n_heads;             /* H; GQA head_dim = D / H                              */
+  int n_kv_heads;          /* Hkv (GQA); H divisible by Hkv                       */
+  int attn_type;           /* 0 = GQA, 1 = MLA                                     */
+  int kv_lora_rank;        /* MLA latent width                                     */
+  int q_lora_rank;         /* MLA query latent width                               */
+  int qk_rope_head_dim;    /* MLA rotary part of the score dim                     */
+  int qk_nope_head_dim;    /* MLA non-rotary part of the score dim                 */
+  int v_head_dim;          /* MLA value head dim                                   */
+  int n_experts;           /* E routed experts (0: dense FFN block)                */
+  int n_shared_experts;    /* S always-on experts                                  */
+  int top_k;               /* experts per token (n_experts_per_tok)                */
+  int expert_dim;          /* F hidden width of routed and shared experts          */
+  int lora_rank;           /* r of the depth-wise LoRA                             */
+  int max_loop_iters;      /* rows of the LoRA scale table                          */
+  int loop_dim;            /* channels carrying the loop-index embedding (even)    */
+  float rope_theta;        /* RoPE base (10000)                                    */
+  float loop_theta;        /* loop-embedding base (10000)                          */
+  float norm_eps;          /* RMSNorm epsilon (1e-6)                                */
+  int dtype;               /* 0 = fp32, 1 = bf16 (storage of matrices, e, GEMM inputs) */
+} rdt_config;
+
+/* Recurrent-block (or dense prelude/coda block) weights: device pointers.
+ * Model-dtype matrices unless marked fp32.  Unused fields may be NULL
+ * (e.g. the MLA fields for GQA, routing fields for a dense block). */
+typedef struct {
+  const float* rec_norm_w;   /* [D] fp32  RecurrentBlock.norm on h_loop + e         */
+  const float* attn_norm_w;  /* [D] fp32  pre-attention RMSNorm                      */
+  const float* ffn_norm_w;   /* [D] fp32  pre-FFN RMSNorm                            */
+  /* GQA */
+  const void* w_qkv;         /* [(H + 2 Hkv) hd, D]: q heads, then k heads, then v    */
+  const void* w_o;           /* [D, H hd] (GQA) or [D, H v_head_dim] (MLA)            */
+  /* MLA (DeepSeek-V2 layout) */
+  const void* w_q_down;      /* [q_lora_rank, D]                                      */
+  const float* q_norm_w;     /* [q_lora_rank] fp32                                    */
+  const void* w_q_up;        /* [H (nope + rope), q_lora_rank], per head [nope|rope]  */
+  const void* w_kv_down;     /* [kv_lora_rank + rope, D]: c_kv then k_rope            */
+  const float* kv_norm_w;    /* [kv_lora_rank] fp32                                   */
+  const void* w_kv_up;       /* [H (nope + v), kv_lora_rank], per head [k_nope|v]     */
+  /* MoE ("OpenMythos 분석", MoE) */
+  const void* w_router;      /* [E, D]                                                */
+  const float* router_bias;  /* [E] fp32, used for selection only                     */
+  const void* w13;           /* [E + S][2F][D]: rows [0,F) = W1 (gate), [F,2F) = W3    */
+  const void* w2;            /* [E + S][D][F]; experts 0..E-1 routed, E.. shared      */
+  /* depth-wise LoRA ("Repeating the parameter ...") */
+  const void* lora_down;     /* [r, D]                                                */
+  const void* lora_B;        /* [r, D]                                                */
+  const float* lora_scale;   /* [max_loop_iters, r] fp32                              */
+  /* LTI injection ("latent reasoning") and ACT halting head ("ACT") */
+  const float* log_A;        /* [D] fp32                                              */
+  const float* log_dt;       /* [1] fp32                                              */
+  const float* inj_B;        /* [D] fp32                                              */
+  const float* halt_w;       /* [D] fp32                                              */
+  const float* halt_b;       /* [1] fp32                                              */
+} rdt_weights;
+
+/* One K/V cache per recurrent loop iteration (cache key recurrent_loop_t,
+ * "OpenMythos 분석", Recurrent Block / RoPE & generation cache).
+ * GQA: k, v [n_loops][batch][Hkv][t_max][hd], model dtype, post-RoPE keys. */
+typedef struct {
+  void* k;
+  void* v;
+  int n_loops;   /* loop caches held (>= the n_loops of a call that uses it) */
+  int batch;     /* sequences held                                          */
+  int t_max;     /* positions per sequence                                  */
+} rdt_kv_cache;
+
+/* Optional per-loop trace of a row range (tests; NULL in production).
+ * Each non-NULL buffer is device memory sized [n_loops][n_rows][...]. */
+typedef struct {
+  int row0, n_rows;
+  float* h_in;           /* [L][n_rows][D]  state entering loop t                    */
+  float* f;              /* [L][n_rows][D]  router input RMSNorm_ffn(x1), as stored   */
+  float* biased_logits;  /* [L][n_rows][E]  router logits + router_bias              */
+  float* p;              /* [L][n_rows]     halting probability (ACT on)             */
+} rdt_trace;
+
+enum {
+  RDT_FLAG_TRANSFORMER_OFF = 1   /* debug: Transformer(h, e) term = 0 (pure LTI)      */
+};
+
+/* Bytes of workspace needed by rdt_recurrent_forward / rdt_recurrent_decode_step /
+ * rdt_block_forward / rdt_head for `batch` x `seq` rows attending to at most
+ * `max_keys` keys per sequence (prefill: start_pos + seq; decode: cache t_max).
+ * Returns 0 for an invalid config. */
+RDT_API size_t rdt_workspace_size(const rdt_config* cfg, int batch, int seq, int max_keys);
+
+/* RecurrentBlock.forward ("OpenMythos 분석", Recurrent Block; update rule
+ * h_{t+1} = A h_t + B e + Transformer(h_t, e), README mirror 동적 시스템 관점).
+ *  h0 [N, D] fp32, e [N, D] model dtype, N = batch * seq; positions start_pos + i.
+ *  act_threshold <= 0 turns ACT off (h_out = state after the last loop).
+ *  halt_logit_offset: NULL or [N] fp32 added to the halting logit (workload hook).
+ *  Outputs: h_out [N, D] fp32 (ACT-weighted state), halt_weights [n_loops, N] fp32,
+ *  expert_ids [n_loops, N, top_k] int32 (-1 for halted rows).
+ *  cache: NULL, or per-loop caches that receive this call's K/V at positions
+ *  start_pos..start_pos+seq-1 (and supply earlier keys when start_pos > 0).
+ *  trace: NULL or a row-range trace.  flags: RDT_FLAG_*.
+ *  Weights of a MoE block are required (n_experts >= 1, top_k >= 1). */
+RDT_API rdt_status rdt_recurrent_forward(const rdt_config* cfg, const rdt_weights* w,
+                                 const float* h0, const void* e,
+                                 int batch, int seq, int start_pos, int n_loops,
+                                 float act_threshold, const float* halt_logit_offset,
+                                 float* h_out, float* halt_weights, int32_t* expert_ids,
+                                 const rdt_kv_cache* cache, const rdt_trace* trace, int flags,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* One KV-cached decode step of the recurrent block ("OpenMythos 분석", RoPE &
+ * generation cache): one new token per sequence b at position cache_len[b]
+ * (device int32 [batch]); loop t reads and extends loop cache t (GQA only).
+ * The new K/V are written at cache_len[b]; the caller advances cache_len.
+ * Outputs as rdt_recurrent_forward with N = batch. */
+RDT_API rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_weights* w,
+                                     const float* h0, const void* e, int batch,
+                                     const int32_t* cache_len, int n_loops, float act_threshold,
+                                     float* h_out, float* halt_weights, int32_t* expert_ids,
+                                     const rdt_kv_cache* cache,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/* One pre-norm TransformerBlock: x_out = x1 + FFN(RMSNorm(x1)), x1 = x_in + Attn(RMSNorm(x_in)).
+ * FFN is the MoE when cfg->n_experts > 0, else the dense SwiGLU in w13/w2 expert 0
+ * with hidden cfg->expert_dim (prelude/coda: Expert(dim, dim*4//3), "OpenMythos 분석", MoE).
+ * x_in, x_out [N, D] fp32 (may not alias). */
+RDT_API rdt_status rdt_block_forward(const rdt_config* cfg, const rdt_weights* w,
+                             const float* x_in, float* x_out, int batch, int seq, int start_pos,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* Token embedding gather ("OpenMythos 분석", Core Structure: self.embed(input_ids)):
+ * out[i] = table[ids[i]] widened to fp32.  table [vocab, D] model dtype; ids int32 [n]. */
+RDT_API rdt_status rdt_embed(const rdt_config* cfg, const void* table, int vocab, const int32_t* ids, int n,
+                     float* out, void* stream);
+
+/* LM head: logits = RMSNorm(x) W_head^T ("OpenMythos 분석", Core Structure:
+ * self.head(self.norm(x))).  x [n, D] fp32, norm_w [D] fp32, head [vocab, D] model dtype,
+ * logits [n, vocab] fp32. */
+RDT_API rdt_status rdt_head(const rdt_config* cfg, const float* x, int n, const float* norm_w,
+                    const void* head, int vocab, float* logits,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read and clear the device status word in `ws`. */
+RDT_API rdt_status rdt_read_device_status(void* ws, void* stream);
+
+/* Static description of a status code. */
+RDT_API const char* rdt_status_string(rdt_status s);
+
+/* Library build identifier (kernel set and target), static string. */
+RDT_API const char* rdt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RDT_H_ */

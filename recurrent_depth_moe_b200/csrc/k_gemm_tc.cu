@@ -1,0 +1,467 @@
+// Tensor-core GEMM for sm_100a: tcgen05.mma with TMEM accumulators, operands staged
+// by TMA (no multicast) into 128-byte-swizzled shared memory, persistent CTAs.
+//
+//   C[M, N] = A[M, K] . B[N, K]^T, bf16 operands, fp32 accumulation.
+//   Tile: 128 rows x 256 MMA columns x 64-deep K stages (4 stages, 48 KB each).
+//   Grouped mode (MoE experts): the m-tiles come from a device tile list
+//   {group, row0, rows}; B is the group's weight slab.  SwiGLU: the 256 MMA columns
+//   are 128 gate rows (W1) and the matching 128 up rows (W3) of the expert, so the
+//   epilogue forms silu(gate) * up for 128 output columns in registers.
+//
+// Warp roles (192 threads): warp 0 lane 0 issues TMA loads; warp 1 owns TMEM
+// (alloc / dealloc) and lane 0 issues the MMAs; warps 2..5 are the epilogue, each
+// reading its 32-lane quarter of the accumulator with tcgen05.ld.  The accumulator
+// is double-buffered in TMEM (2 x 256 columns) so the epilogue of one tile overlaps
+// the MMAs of the next.  Every mbarrier wait is bounded: on timeout the CTA records
+// RDT_ERR_DEVICE_TIMEOUT in the status word and leaves its loops.
+#include "common.cuh"
+#include "kernels.h"
+
+#include <cuda.h>
+#include <mutex>
+
+namespace rdt {
+namespace tc {
+
+constexpr int BM = 128, BK = 64, BN_MMA = 256, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;            // 16 KB
+constexpr int B_HALF = 128 * BK * 2;            // 16 KB (one 128-row TMA box)
+constexpr int STAGE_BYTES = A_BYTES + 2 * B_HALF;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr long long TIMEOUT_CYCLES = 4000000000LL;   // ~2 s at 2 GHz
+constexpr int TMEM_COLS = 512;
+
+struct TcArgs {
+  GemmParams p;
+  int n_n;             // n tiles
+  int m_tiles;         // dense: m tiles; grouped: read from *p.n_tiles
+  int b_rows_group;    // rows of B per group (grouped)
+  int n_out_tile;      // output columns per tile (128 SwiGLU, 256 otherwise)
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false on timeout or when another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(b, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(b, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > TIMEOUT_CYCLES) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// K-major, 128-byte-swizzled operand tile: 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t smem_desc(const void* p) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_u32(p) >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;                  // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset: 8 rows x 128 B
+  d |= (uint64_t)1 << 46;                  // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                  // SWIZZLE_128B
+  return d;
+}
+
+// kind::f16 instruction descriptor: bf16 A/B, fp32 D, both K-major, M = 128, N = 256.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z)); }
+
+__device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * q + 2 * j], v[8 * q + 2 * j + 1]);
+      w[j] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    reinterpret_cast<uint4*>(dst)[q] = u;
+  }
+}
+
+__device__ __forceinline__ int rope_pair_tc(const GemmParams& p, int c) {
+  for (int q = 0; q < p.n_rope; ++q) {
+    const RopeDesc& r = p.rope[q];
+    int rel = c - r.col0;
+    if (rel < 0 || rel >= r.n_heads * r.head_stride) continue;
+    int o = rel % r.head_stride - r.off;
+    if (o >= 0 && o < r.dim) return o >> 1;
+  }
+  return -1;
+}
+
+struct TileInfo { int group, row0, rows, n0; };
+
+__device__ __forceinline__ TileInfo decode_tile(const TcArgs& a, int t) {
+  TileInfo ti;
+  const int m_i = t / a.n_n, n_i = t % a.n_n;
+  if (a.p.tiles) {
+    ti.group = a.p.tiles[4 * m_i];
+    ti.row0 = a.p.tiles[4 * m_i + 1];
+    ti.rows = a.p.tiles[4 * m_i + 2];
+  } else {
+    ti.group = 0;
+    ti.row0 = m_i * BM;
+    ti.rows = min(BM, a.p.M - ti.row0);
+  }
+  ti.n0 = n_i * a.n_out_tile;
+  return ti;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = (uint32_t*)(done + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  const GemmParams& p = args.p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int m_tiles = p.tiles ? min(*p.n_tiles, p.max_tiles) : args.m_tiles;
+  const int total = m_tiles * args.n_n;
+  const int nk = p.K / BK;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer ----------------
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+      const TileInfo ti = decode_tile(args, t);
+      int b0, b1;
+      if (EPI == EPI_SWIGLU_T) {
+        b0 = ti.group * args.b_rows_group + ti.n0;
+        b1 = ti.group * args.b_rows_group + p.up_off + ti.n0;
+      } else {
+        b0 = ti.group * args.b_rows_group + ti.n0;
+        b1 = b0 + 128;
+      }
+      for (int ks = 0; ks < nk; ++ks) {
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+        uint8_t* sa = smem + stage * STAGE_BYTES;
+        mbar_expect_tx(&full[stage], STAGE_BYTES);
+        tma_load_2d(sa, &tmA, &full[stage], ks * BK, ti.row0);
+        tma_load_2d(sa + A_BYTES, &tmB, &full[stage], ks * BK, b0);
+        tma_load_2d(sa + A_BYTES + B_HALF, &tmB, &full[stage], ks * BK, b1);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    constexpr uint32_t IDESC = idesc_bf16(BM, BN_MMA);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      if (!(ok = mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t d = tmem + acc * BN_MMA;
+      for (int ks = 0; ks < nk; ++ks) {
+        if (!(ok = mbar_wait(&full[stage], phase, abort_flag))) break;
+        tc_fence_after();
+        uint8_t* sa = smem + stage * STAGE_BYTES;
+        const uint64_t ad = smem_desc(sa), bd = smem_desc(sa + A_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k)
+          umma_bf16(d, ad + 2 * k, bd + 2 * k, IDESC, (ks | k) != 0);
+        umma_commit(&empty[stage]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+      }
+      if (!ok) break;
+      umma_commit(&tfull[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+    // all issued MMAs complete before TMEM is released
+    umma_commit(done);
+    mbar_wait(done, 0, abort_flag);
+  } else if (warp >= 2) {
+    // ---------------- epilogue ----------------
+    const int quarter = warp & 3;
+    const int rl = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const TileInfo ti = decode_tile(args, t);
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN_MMA;
+      const bool valid = rl < ti.rows;
+      const long long r = (long long)ti.row0 + rl;
+      if (EPI == EPI_SWIGLU_T) {
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          float g[32], u[32];
+          tmem_ld32(tbase + c, g);
+          tmem_ld32(tbase + 128 + c, u);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j]) * u[j];
+          if (valid) store_bf16x32((bf16*)p.C + r * p.ldc + ti.n0 + c, g);
+        }
+      } else {
+        const float rs = (EPI == EPI_GATE_F32 && valid) ? p.row_scale[r] : 0.f;
+        const int pos = (EPI == EPI_ROPE_T && valid) ? p.pos[r] : 0;
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 32) {
+          float v[32];
+          tmem_ld32(tbase + c, v);
+          if (!valid) continue;
+          const int col = ti.n0 + c;
+          if (EPI == EPI_STORE_T) {
+            store_bf16x32((bf16*)p.C + r * p.ldc + col, v);
+          } else if (EPI == EPI_ROPE_T) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              int m = rope_pair_tc(p, col + j);
+              if (m >= 0) {
+                float2 cs = p.rope_tab[(long long)pos * p.rope_half + m];
+                float r0 = v[j] * cs.x - v[j + 1] * cs.y, r1 = v[j] * cs.y + v[j + 1] * cs.x;
+                v[j] = r0;
+                v[j + 1] = r1;
+              }
+            }
+            store_bf16x32((bf16*)p.C + r * p.ldc + col, v);
+          } else {
+            float* dst = (float*)p.C + r * p.ldc + col;
+            if (EPI == EPI_RESID_F32) {
+              const float4* rs4 = (const float4*)(p.resid + r * p.ld_resid + col);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                float4 a = rs4[q];
+                ((float4*)dst)[q] = make_float4(a.x + v[4 * q], a.y + v[4 * q + 1], a.z + v[4 * q + 2], a.w + v[4 * q + 3]);
+              }
+            } else if (EPI == EPI_GATE_F32) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                ((float4*)dst)[q] = make_float4(rs * v[4 * q], rs * v[4 * q + 1], rs * v[4 * q + 2], rs * v[4 * q + 3]);
+            } else {
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                ((float4*)dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) record_status(p.st, ST_TIMEOUT, 501, blockIdx.x);
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)ptr;
+  });
+  return fn;
+}
+
+// 2-D bf16 map over [rows, cols] (row stride ld elements), box = 64 columns x box_rows rows, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsigned long long cols,
+              unsigned long long ld, unsigned box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+inline bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+}  // namespace
+
+bool gemm_tc_supports(const GemmParams& p, int epi) {
+  if (epi < EPI_STORE_F32 || epi > EPI_GATE_F32) return false;
+  if (p.K < tc::BK || p.K % tc::BK) return false;
+  if (epi == EPI_SWIGLU_T ? (p.N % 128) : (p.N % 256)) return false;
+  if (p.lda % 8 || p.ldb % 8 || !al16(p.A) || !al16(p.B) || !al16(p.C)) return false;
+  if (epi == EPI_STORE_F32 || epi == EPI_RESID_F32 || epi == EPI_GATE_F32) {
+    if (p.ldc % 4) return false;
+  } else if (p.ldc % 8) {
+    return false;
+  }
+  if (epi == EPI_RESID_F32 && (p.ld_resid % 4 || !al16(p.resid))) return false;
+  if (p.tiles && (p.b_group_stride % p.ldb || p.b_rows <= 0)) return false;
+  return encode_fn() != nullptr;
+}
+
+int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
+  tc::TcArgs a;
+  a.p = p;
+  a.n_out_tile = (epi == EPI_SWIGLU_T) ? 128 : 256;
+  a.n_n = p.N / a.n_out_tile;
+  a.m_tiles = p.tiles ? 0 : (p.M + tc::BM - 1) / tc::BM;
+  a.b_rows_group = p.tiles ? (int)(p.b_group_stride / p.ldb) : 0;
+  // B map extent: the caller's b_rows (all groups' rows), else N rows (SwiGLU: gate then up rows)
+  CUtensorMap mA, mB;
+  if (!make_map(&mA, p.A, (unsigned long long)p.M, p.K, p.lda, 128)) return -1;
+  unsigned long long brows = p.b_rows > 0 ? (unsigned long long)p.b_rows
+                                          : (unsigned long long)((epi == EPI_SWIGLU_T) ? p.up_off + p.N : p.N);
+  if (!make_map(&mB, p.B, brows, p.K, p.ldb, 128)) return -1;
+  int grid;
+  if (p.tiles) {
+    grid = sm_count();
+  } else {
+    long long tiles = (long long)a.m_tiles * a.n_n;
+    grid = (int)std::min<long long>(tiles, sm_count());
+  }
+  if (grid <= 0) return 0;
+#define RDT_TC_CASE(E)                                                                              \
+  case E: {                                                                                         \
+    static bool attr = false;                                                                       \
+    if (!attr) {                                                                                    \
+      if (cudaFuncSetAttribute(tc::k_gemm_tc<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
+                               tc::SMEM_BYTES) != cudaSuccess)                                      \
+        return -1;                                                                                  \
+      attr = true;                                                                                  \
+    }                                                                                               \
+    tc::k_gemm_tc<E><<<grid, 192, tc::SMEM_BYTES, s>>>(mA, mB, a);                                  \
+    break;                                                                                          \
+  }
+  switch (epi) {
+    RDT_TC_CASE(EPI_STORE_F32)
+    RDT_TC_CASE(EPI_STORE_T)
+    RDT_TC_CASE(EPI_RESID_F32)
+    RDT_TC_CASE(EPI_ROPE_T)
+    RDT_TC_CASE(EPI_SWIGLU_T)
+    RDT_TC_CASE(EPI_GATE_F32)
+    default: return -1;
+  }
+#undef RDT_TC_CASE
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace rdt

@@ -1,0 +1,416 @@
+// Row-wise kernels of the recurrent block: loop prologue (S1), norms, tables, the
+// fused combine + depth-wise LoRA + LTI injection + ACT step (S9), running-row
+// compaction, K/V cache writes and the MLA latent preparation.
+//
+// All are HBM-bound row kernels: one CTA per row, 256 threads, the row staged in
+// dynamic shared memory so every input element is read once and every output
+// element written once.
+#include "common.cuh"
+#include "kernels.h"
+#include <math.h>
+
+namespace rdt {
+
+// ------------------------------------------------------------------------------------------
+// tables (double precision, rounded once to fp32)
+// ------------------------------------------------------------------------------------------
+
+// A = exp(-exp(clamp(log_dt + log_A, -20, 20))) ("OpenMythos 분석", latent reasoning).
+__global__ void k_lti_A(const float* log_A, const float* log_dt, float* A, int D) {
+  int d = blockIdx.x * blockDim.x + threadIdx.x;
+  if (d >= D) return;
+  double z = (double)log_dt[0] + (double)log_A[d];
+  z = fmin(fmax(z, -20.0), 20.0);
+  A[d] = (float)exp(-exp(z));
+}
+
+// Loop-index embedding of loop t: emb[j] = sin(t w_j), emb[half + j] = cos(t w_j),
+// w_j = theta^(-2j / loop_dim) ("OpenMythos 분석", Repeating the parameter ...).
+__global__ void k_loop_emb(float* emb, int loop_dim, int t, float theta) {
+  int half = loop_dim / 2;
+  for (int j = threadIdx.x; j < half; j += blockDim.x) {
+    double w = pow((double)theta, -2.0 * j / loop_dim);
+    double ang = (double)t * w;
+    emb[j] = (float)sin(ang);
+    emb[half + j] = (float)cos(ang);
+  }
+}
+
+// RoPE phasors: tab[p * half + m] = (cos, sin)(p * theta^(-2m / dim)).
+__global__ void k_rope_table(float2* tab, int n_pos, int dim, float theta) {
+  int half = dim / 2;
+  long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)n_pos * half) return;
+  int p = (int)(idx / half), m = (int)(idx % half);
+  double ang = (double)p * pow((double)theta, -2.0 * m / dim);
+  tab[idx] = make_float2((float)cos(ang), (float)sin(ang));
+}
+
+// pos[row] = start_pos + row % seq
+__global__ void k_positions(int* pos, int N, int seq, int start_pos) {
+  int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r < N) pos[r] = start_pos + r % seq;
+}
+
+// decode: the new token of sequence b sits at cache_len[b]; out-of-range lengths are
+// recorded in the status word and clamped so no table or cache access leaves its buffer.
+__global__ void k_positions_decode(int* pos, const int* cache_len, int B, int t_max, DevStatus* st) {
+  int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= B) return;
+  int p = cache_len[r];
+  if (p < 0 || p >= t_max) {
+    record_status(st, ST_BOUNDS, 102, p);
+    p = p < 0 ? 0 : t_max - 1;
+  }
+  pos[r] = p;
+}
+
+// ------------------------------------------------------------------------------------------
+// S1: combined = RMSNorm_rec(h + emb_t + e); a = RMSNorm_attn(combined)
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void k_loop_prologue(const float* __restrict__ h, const T* __restrict__ e,
+                                const float* __restrict__ emb, int loop_dim,
+                                const float* __restrict__ w_rec, const float* __restrict__ w_attn,
+                                float* __restrict__ combined, T* __restrict__ a, int D, float eps) {
+  extern __shared__ float xs[];
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  const float* hr = h + row * D;
+  const T* er = e + row * D;
+  float ss = 0.f;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float x = hr[d] + to_f(er[d]);
+    if (d < loop_dim) x += emb[d];
+    xs[d] = x;
+    ss += x * x;
+  }
+  ss = block_sum(ss, red);
+  float inv = rsqrtf(ss / D + eps);
+  float ss2 = 0.f;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float c = xs[d] * inv * w_rec[d];
+    xs[d] = c;
+    combined[row * D + d] = c;
+    ss2 += c * c;
+  }
+  ss2 = block_sum(ss2, red);
+  float inv2 = rsqrtf(ss2 / D + eps);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) a[row * D + d] = from_f<T>(xs[d] * inv2 * w_attn[d]);
+}
+
+// out = RMSNorm(x) * w over rows of width D (fp32 in, model dtype out).
+// in_ld / out_ld are the row strides (elements); x may be a column slice.
+template <typename TI, typename TO>
+__global__ void k_rmsnorm(const TI* __restrict__ x, long long in_ld, const float* __restrict__ w,
+                          TO* __restrict__ out, long long out_ld, int D, float eps) {
+  extern __shared__ float xs[];
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  float ss = 0.f;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float v = to_f(x[row * in_ld + d]);
+    xs[d] = v;
+    ss += v * v;
+  }
+  ss = block_sum(ss, red);
+  float inv = rsqrtf(ss / D + eps);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) out[row * out_ld + d] = from_f<TO>(xs[d] * inv * w[d]);
+}
+
+// ------------------------------------------------------------------------------------------
+// MLA latent preparation: ckv = RMSNorm_kv(kv_raw[:, :kvr]) (model dtype);
+// krope = RoPE(kv_raw[:, kvr:]) (model dtype).
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void k_mla_kv_prep(const float* __restrict__ kv_raw, int kvr, int dr,
+                              const float* __restrict__ kv_norm_w, float eps,
+                              const int* __restrict__ pos, const float2* __restrict__ rope_tab,
+                              T* __restrict__ ckv, T* __restrict__ krope) {
+  __shared__ float red[32];
+  const long long row = blockIdx.x;
+  const float* x = kv_raw + row * (kvr + dr);
+  float ss = 0.f;
+  for (int d = threadIdx.x; d < kvr; d += blockDim.x) ss += x[d] * x[d];
+  ss = block_sum(ss, red);
+  float inv = rsqrtf(ss / kvr + eps);
+  for (int d = threadIdx.x; d < kvr; d += blockDim.x) ckv[row * kvr + d] = from_f<T>(x[d] * inv * kv_norm_w[d]);
+  const int p = pos[row];
+  for (int m = threadIdx.x; m < dr / 2; m += blockDim.x) {
+    float2 cs = rope_tab[(long long)p * (dr / 2) + m];
+    float x0 = x[kvr + 2 * m], x1 = x[kvr + 2 * m + 1];
+    krope[row * dr + 2 * m] = from_f<T>(x0 * cs.x - x1 * cs.y);
+    krope[row * dr + 2 * m + 1] = from_f<T>(x0 * cs.y + x1 * cs.x);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// GQA K/V rows -> per-loop cache [B][Hkv][t_max][hd] at position pos[row].
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void k_kv_to_cache(const T* __restrict__ qkv, long long ld, int k_col, int v_col,
+                              int Hkv, int hd, const int* __restrict__ pos, int seq, int t_max,
+                              T* __restrict__ kc, T* __restrict__ vc, DevStatus* st) {
+  const long long row = blockIdx.x;
+  const int b = (int)(row / seq);
+  const int p = pos[row];
+  if (p < 0 || p >= t_max) {
+    if (threadIdx.x == 0) record_status(st, ST_BOUNDS, 101, p);
+    return;
+  }
+  for (int i = threadIdx.x; i < Hkv * hd; i += blockDim.x) {
+    int g = i / hd, d = i % hd;
+    long long dst = (((long long)b * Hkv + g) * t_max + p) * hd + d;
+    kc[dst] = qkv[row * ld + k_col + i];
+    vc[dst] = qkv[row * ld + v_col + i];
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// S9: combine + depth-wise LoRA + LTI injection + freeze + ACT, one CTA per row.
+//   trans = x1 + sum_j y[slot_of[i][j]]                (routed, gate already applied; shared)
+//   trans += ((trans Wd^T) * scale[min(t, mli-1)]) B_lora
+//   h_new = A h + B_inj e + trans;  rows halted before loop t keep h (frozen)
+//   ACT: p = sigmoid(h_new . w_halt + b_halt + off); w = remainder if cum + p >= thr or
+//   last loop, else p; cum += p; h_out += w h_new.   ACT off: w = [t == L-1].
+// block_only: out = trans (one plain block, no LoRA / injection / ACT).
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void k_combine_inject_act(CombineParams p) {
+  extern __shared__ float sm[];
+  float* tr = sm;                 // [D] trans, then h_new
+  float* zq = sm + p.D;           // [r] LoRA projections
+  __shared__ float red[32];
+  const int i = blockIdx.x;
+  const int D = p.D;
+  const int kS = p.k + p.S;
+  if (!p.block_only && p.halted[i]) {   // frozen row
+    if (threadIdx.x == 0) p.halt_w_out[(long long)p.t * p.N + i] = 0.f;
+    for (int j = threadIdx.x; j < p.k; j += blockDim.x) p.ids_out[((long long)p.t * p.N + i) * p.k + j] = -1;
+    return;
+  }
+  const float* x1 = p.x1 + (long long)i * D;
+  if (p.transformer_off) {
+    for (int d = threadIdx.x; d < D; d += blockDim.x) tr[d] = 0.f;
+  } else {
+    for (int d = threadIdx.x; d < D; d += blockDim.x) tr[d] = x1[d];
+    for (int j = 0; j < kS; ++j) {
+      int slot = p.slot_of[(long long)i * kS + j];
+      if (slot < 0 || slot >= p.max_slots) {
+        if (threadIdx.x == 0) record_status(p.st, ST_BOUNDS, 201, slot);
+        continue;
+      }
+      const float* yr = p.y + (long long)slot * D;
+      for (int d = threadIdx.x; d < D; d += blockDim.x) tr[d] += yr[d];
+    }
+  }
+  __syncthreads();
+  if (p.block_only) {
+    for (int d = threadIdx.x; d < D; d += blockDim.x) p.out[(long long)i * D + d] = tr[d];
+    return;
+  }
+  if (!p.transformer_off && p.r > 0) {
+    const T* Wd = (const T*)p.lora_down;
+    const T* Bl = (const T*)p.lora_B;
+    const float* sc = p.lora_scale + (long long)min(p.t, p.max_loop_iters - 1) * p.r;
+    for (int q = 0; q < p.r; ++q) {
+      float part = 0.f;
+      for (int d = threadIdx.x; d < D; d += blockDim.x) part += tr[d] * to_f(Wd[(long long)q * D + d]);
+      part = block_sum(part, red);
+      if (threadIdx.x == 0) zq[q] = part * sc[q];
+    }
+    __syncthreads();
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+      float acc = 0.f;
+      for (int q = 0; q < p.r; ++q) acc += zq[q] * to_f(Bl[(long long)q * D + d]);
+      tr[d] += acc;
+    }
+  }
+  const float* hr = p.h + (long long)i * D;
+  const T* er = (const T*)p.e + (long long)i * D;
+  float zh = 0.f;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float hn = p.A[d] * hr[d] + p.inj_B[d] * to_f(er[d]) + tr[d];
+    tr[d] = hn;
+    if (p.act_on) zh += hn * p.halt_wv[d];
+  }
+  float w;
+  const bool last = (p.t == p.n_loops - 1);
+  if (p.act_on) {
+    zh = block_sum(zh, red);
+    float z = zh + p.halt_b[0] + (p.halt_off ? p.halt_off[i] : 0.f);
+    float prob = 1.f / (1.f + expf(-z));
+    float cum = p.cum[i];
+    bool stop = (cum + prob >= p.thr) || last;
+    w = stop ? fmaxf(1.f - cum, 0.f) : prob;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      p.cum[i] = cum + prob;
+      if (stop) p.halted[i] = 1;
+      if (p.p_out) p.p_out[i] = prob;
+    }
+  } else {
+    w = last ? 1.f : 0.f;
+  }
+  float* ho = p.h_out + (long long)i * D;
+  float* hw = p.h_state + (long long)i * D;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float hn = tr[d];
+    ho[d] += w * hn;
+    hw[d] = hn;
+  }
+  if (threadIdx.x == 0) p.halt_w_out[(long long)p.t * p.N + i] = w;
+  for (int j = threadIdx.x; j < p.k; j += blockDim.x)
+    p.ids_out[((long long)p.t * p.N + i) * p.k + j] = p.transformer_off ? -1 : p.ids[(long long)i * p.k + j];
+}
+
+// ------------------------------------------------------------------------------------------
+// running-row compaction (single CTA, ordered): run_list = rows with halted == 0.
+// ------------------------------------------------------------------------------------------
+__global__ void k_compact(const int* __restrict__ halted, int N, int* __restrict__ run_list,
+                          int* __restrict__ run_idx, int* __restrict__ n_run) {
+  __shared__ int warp_tot[32];
+  __shared__ int base;
+  if (threadIdx.x == 0) base = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int c0 = 0; c0 < N; c0 += blockDim.x) {
+    int i = c0 + threadIdx.x;
+    int run = (i < N && !halted[i]) ? 1 : 0;
+    unsigned m = __ballot_sync(0xffffffffu, run);
+    int pre = __popc(m & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[wid] = __popc(m);
+    __syncthreads();
+    int off = 0;
+    for (int w2 = 0; w2 < wid; ++w2) off += warp_tot[w2];
+    int total = 0;
+    for (int w2 = 0; w2 < nw; ++w2) total += warp_tot[w2];
+    if (i < N) {
+      int idx = base + off + pre;
+      run_idx[i] = run ? idx : -1;
+      if (run) run_list[idx] = i;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) base += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *n_run = base;
+}
+
+__global__ void k_iota(int* run_list, int* run_idx, int* n_run, int N) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < N) { run_list[i] = i; run_idx[i] = i; }
+  if (i == 0) *n_run = N;
+}
+
+// embedding gather: out[i] = table[ids[i]] (fp32)
+template <typename T>
+__global__ void k_embed(const T* __restrict__ table, int vocab, const int* __restrict__ ids, int D,
+                        float* __restrict__ out, DevStatus* st) {
+  const long long i = blockIdx.x;
+  int id = ids[i];
+  if (id < 0 || id >= vocab) {
+    if (threadIdx.x == 0) record_status(st, ST_BOUNDS, 301, id);
+    id = 0;
+  }
+  for (int d = threadIdx.x; d < D; d += blockDim.x) out[i * D + d] = to_f(table[(long long)id * D + d]);
+}
+
+// trace: copy rows [row0, row0 + n) of a [*, W] fp32 or model-dtype matrix (+ optional
+// per-column bias) into a fp32 destination.
+template <typename T>
+__global__ void k_trace_rows(const T* __restrict__ src, int W, int row0, const float* __restrict__ bias,
+                             float* __restrict__ dst) {
+  const long long r = blockIdx.x;
+  for (int c = threadIdx.x; c < W; c += blockDim.x)
+    dst[r * W + c] = to_f(src[(row0 + r) * (long long)W + c]) + (bias ? bias[c] : 0.f);
+}
+
+// ------------------------------------------------------------------------------------------
+// launchers
+// ------------------------------------------------------------------------------------------
+static inline int nthreads_for(int D) { return D >= 2048 ? 256 : 128; }
+
+void launch_lti_A(const float* log_A, const float* log_dt, float* A, int D, cudaStream_t s) {
+  k_lti_A<<<(D + 255) / 256, 256, 0, s>>>(log_A, log_dt, A, D);
+}
+void launch_loop_emb(float* emb, int loop_dim, int t, float theta, cudaStream_t s) {
+  if (loop_dim >= 2) k_loop_emb<<<1, 128, 0, s>>>(emb, loop_dim, t, theta);
+}
+void launch_rope_table(float2* tab, int n_pos, int dim, float theta, cudaStream_t s) {
+  long long n = (long long)n_pos * (dim / 2);
+  if (n > 0) k_rope_table<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(tab, n_pos, dim, theta);
+}
+void launch_positions(int* pos, int N, int seq, int start_pos, cudaStream_t s) {
+  k_positions<<<(N + 255) / 256, 256, 0, s>>>(pos, N, seq, start_pos);
+}
+void launch_positions_decode(int* pos, const int* cache_len, int B, int t_max, DevStatus* st, cudaStream_t s) {
+  k_positions_decode<<<(B + 255) / 256, 256, 0, s>>>(pos, cache_len, B, t_max, st);
+}
+void launch_loop_prologue(int dtype, const float* h, const void* e, const float* emb, int loop_dim,
+                          const float* w_rec, const float* w_attn, float* combined, void* a,
+                          int N, int D, float eps, cudaStream_t s) {
+  size_t smem = (size_t)D * sizeof(float);
+  if (dtype == 0)
+    k_loop_prologue<float><<<N, nthreads_for(D), smem, s>>>(h, (const float*)e, emb, loop_dim, w_rec, w_attn,
+                                                           combined, (float*)a, D, eps);
+  else
+    k_loop_prologue<bf16><<<N, nthreads_for(D), smem, s>>>(h, (const bf16*)e, emb, loop_dim, w_rec, w_attn,
+                                                          combined, (bf16*)a, D, eps);
+}
+void launch_rmsnorm(int in_f32, int dtype, const void* x, long long in_ld, const float* w, void* out,
+                    long long out_ld, int rows, int D, float eps, cudaStream_t s) {
+  size_t smem = (size_t)D * sizeof(float);
+  int nt = nthreads_for(D);
+  if (in_f32) {
+    if (dtype == 0) k_rmsnorm<float, float><<<rows, nt, smem, s>>>((const float*)x, in_ld, w, (float*)out, out_ld, D, eps);
+    else k_rmsnorm<float, bf16><<<rows, nt, smem, s>>>((const float*)x, in_ld, w, (bf16*)out, out_ld, D, eps);
+  } else {
+    if (dtype == 0) k_rmsnorm<float, float><<<rows, nt, smem, s>>>((const float*)x, in_ld, w, (float*)out, out_ld, D, eps);
+    else k_rmsnorm<bf16, bf16><<<rows, nt, smem, s>>>((const bf16*)x, in_ld, w, (bf16*)out, out_ld, D, eps);
+  }
+}
+void launch_mla_kv_prep(int dtype, const float* kv_raw, int kvr, int dr, const float* kv_norm_w, float eps,
+                        const int* pos, const float2* rope_tab, void* ckv, void* krope, int N, cudaStream_t s) {
+  if (dtype == 0)
+    k_mla_kv_prep<float><<<N, 64, 0, s>>>(kv_raw, kvr, dr, kv_norm_w, eps, pos, rope_tab, (float*)ckv, (float*)krope);
+  else
+    k_mla_kv_prep<bf16><<<N, 64, 0, s>>>(kv_raw, kvr, dr, kv_norm_w, eps, pos, rope_tab, (bf16*)ckv, (bf16*)krope);
+}
+void launch_kv_to_cache(int dtype, const void* qkv, long long ld, int k_col, int v_col, int Hkv, int hd,
+                        const int* pos, int N, int seq, int t_max, void* kc, void* vc, DevStatus* st,
+                        cudaStream_t s) {
+  if (dtype == 0)
+    k_kv_to_cache<float><<<N, 128, 0, s>>>((const float*)qkv, ld, k_col, v_col, Hkv, hd, pos, seq, t_max,
+                                           (float*)kc, (float*)vc, st);
+  else
+    k_kv_to_cache<bf16><<<N, 128, 0, s>>>((const bf16*)qkv, ld, k_col, v_col, Hkv, hd, pos, seq, t_max,
+                                          (bf16*)kc, (bf16*)vc, st);
+}
+void launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s) {
+  size_t smem = (size_t)(p.D + 64) * sizeof(float);
+  int nt = nthreads_for(p.D);
+  if (dtype == 0) k_combine_inject_act<float><<<n_rows, nt, smem, s>>>(p);
+  else k_combine_inject_act<bf16><<<n_rows, nt, smem, s>>>(p);
+}
+void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* n_run, cudaStream_t s) {
+  k_compact<<<1, 1024, 0, s>>>(halted, N, run_list, run_idx, n_run);
+}
+void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s) {
+  k_iota<<<(N + 255) / 256, 256, 0, s>>>(run_list, run_idx, n_run, N);
+}
+void launch_embed(int dtype, const void* table, int vocab, const int* ids, int n, int D, float* out,
+                  DevStatus* st, cudaStream_t s) {
+  if (dtype == 0) k_embed<float><<<n, 128, 0, s>>>((const float*)table, vocab, ids, D, out, st);
+  else k_embed<bf16><<<n, 128, 0, s>>>((const bf16*)table, vocab, ids, D, out, st);
+}
+void launch_trace_rows(int src_is_model_dtype, int dtype, const void* src, int W, int row0, int n,
+                       const float* bias, float* dst, cudaStream_t s) {
+  if (n <= 0) return;
+  if (!src_is_model_dtype || dtype == 0)
+    k_trace_rows<float><<<n, 128, 0, s>>>((const float*)src, W, row0, bias, dst);
+  else
+    k_trace_rows<bf16><<<n, 128, 0, s>>>((const bf16*)src, W, row0, bias, dst);
+}
+
+}  // namespace rdt

@@ -1,0 +1,130 @@
+// Internal launcher declarations of librdt (host side).  Not part of the ABI.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rdt {
+
+struct DevStatus;
+
+// ------------------------------------------------------------------------------------------
+// GEMM: C[M, N] = A[M, K] . B[N, K]^T with A, B K-contiguous (nn.Linear layout for B).
+// Grouped mode: tiles[4 * i] = {group, row0, rows, 0}; B advanced by group * b_group_stride.
+// ------------------------------------------------------------------------------------------
+enum Epi {
+  EPI_STORE_F32 = 0,   // C fp32 = acc
+  EPI_STORE_T = 1,     // C model dtype = acc
+  EPI_RESID_F32 = 2,   // C fp32 = resid + acc
+  EPI_ROPE_T = 3,      // C model dtype = RoPE(acc) on the described column ranges
+  EPI_SWIGLU_T = 4,    // C model dtype = silu(acc(B rows c)) * acc(B rows up_off + c)
+  EPI_GATE_F32 = 5     // C fp32 = row_scale[row] * acc
+};
+
+struct RopeDesc {        // columns col0 + h * head_stride + off + [0, dim), h < n_heads
+  int col0, n_heads, head_stride, off, dim;
+};
+
+struct GemmParams {
+  const void* A; long long lda;
+  const void* B; long long ldb; long long b_group_stride;
+  int M, N, K;
+  const int* tiles; const int* n_tiles; int max_tiles;  // grouped mode when tiles != nullptr
+  int up_off;                                            // SWIGLU: W3 row offset in a group
+  void* C; long long ldc;
+  const float* resid; long long ld_resid;
+  const float* row_scale;
+  const int* pos; const float2* rope_tab; int rope_half; int n_rope; RopeDesc rope[2];
+  long long b_rows;                                      // rows of the B tensor (0: derive from N)
+  int impl;                                              // -1 auto, else a GemmImpl
+  DevStatus* st;
+};
+
+// Which implementation handles a GEMM (decided on the host from shape and dtype).
+enum GemmImpl { GEMM_SIMT = 0, GEMM_TC = 1 };
+int gemm_tile_m(GemmImpl impl);
+GemmImpl gemm_pick(int dtype, const GemmParams& p, int epi);
+int launch_gemm(int dtype, int epi, const GemmParams& p, cudaStream_t s);   // returns 0 on success
+
+// ------------------------------------------------------------------------------------------
+// attention
+// ------------------------------------------------------------------------------------------
+struct AttnParams {
+  const void* q; long long q_row; int q_head;           // q[row, h, 0 : dn + dr]
+  const void* k1; long long k1_b, k1_j, k1_g;           // per-kv-head key part, dim dn
+  const void* k2; long long k2_b, k2_j;                 // head-shared key part, dim dr (MLA)
+  const void* v; long long v_b, v_j, v_g;               // dim dv
+  void* o; long long o_row; int o_head;
+  int B, T, H, G;                                       // G = H / Hkv
+  int dn, dr, dv;
+  const int* q_pos;                                     // [B * T] absolute positions
+  int key_pos0;                                         // absolute position of key index 0
+  const int* n_keys_dev;                                // per sequence (decode) or nullptr
+  int n_keys;                                           // keys per sequence (prefill)
+  float scale;
+  // split-KV decode scratch
+  float* part_o; float* part_ml; int n_split;
+};
+int launch_attention(int dtype, const AttnParams& p, cudaStream_t s);
+int launch_attention_decode(int dtype, const AttnParams& p, cudaStream_t s);
+
+// ------------------------------------------------------------------------------------------
+// MoE routing and permutation
+// ------------------------------------------------------------------------------------------
+struct RouteParams {
+  const float* logits; const float* bias;       // [N, E], [E]
+  int N, E, k, S;
+  const int* run_list; const int* n_run;
+  int* ids; float* gates; int* rank; int* counts;   // [N, k], [N, k], [N, k], [E]
+  int* offsets;                                  // [E + S + 1]
+  int* tiles; int* n_tiles; int max_tiles; int tile_m;
+  int* slot_of; int* tok_of; float* gate_of;     // [N, k + S], [M], [M]
+  const void* f; void* xg; int D;                // gather source rows / destination
+  int max_slots;
+  DevStatus* st;
+};
+void launch_router_topk(const RouteParams& p, cudaStream_t s);
+void launch_route_scan(const RouteParams& p, cudaStream_t s);
+void launch_route_scatter(int dtype, const RouteParams& p, cudaStream_t s);
+
+// ------------------------------------------------------------------------------------------
+// row kernels
+// ------------------------------------------------------------------------------------------
+struct CombineParams {
+  int N, D, k, S, r, t, n_loops, max_loop_iters, max_slots;
+  int act_on, transformer_off, block_only;
+  float thr;
+  const float* x1; const float* y; const int* slot_of; const int* ids;
+  const void* lora_down; const void* lora_B; const float* lora_scale;
+  const float* A; const float* inj_B; const void* e;
+  const float* h; float* h_state; float* h_out;
+  const float* halt_wv; const float* halt_b; const float* halt_off;
+  float* cum; int* halted;
+  float* halt_w_out; int* ids_out; float* p_out;
+  float* out;   // block_only
+  DevStatus* st;
+};
+
+void launch_lti_A(const float* log_A, const float* log_dt, float* A, int D, cudaStream_t s);
+void launch_loop_emb(float* emb, int loop_dim, int t, float theta, cudaStream_t s);
+void launch_rope_table(float2* tab, int n_pos, int dim, float theta, cudaStream_t s);
+void launch_positions(int* pos, int N, int seq, int start_pos, cudaStream_t s);
+void launch_positions_decode(int* pos, const int* cache_len, int B, int t_max, DevStatus* st, cudaStream_t s);
+void launch_loop_prologue(int dtype, const float* h, const void* e, const float* emb, int loop_dim,
+                          const float* w_rec, const float* w_attn, float* combined, void* a,
+                          int N, int D, float eps, cudaStream_t s);
+void launch_rmsnorm(int in_f32, int dtype, const void* x, long long in_ld, const float* w, void* out,
+                    long long out_ld, int rows, int D, float eps, cudaStream_t s);
+void launch_mla_kv_prep(int dtype, const float* kv_raw, int kvr, int dr, const float* kv_norm_w, float eps,
+                        const int* pos, const float2* rope_tab, void* ckv, void* krope, int N, cudaStream_t s);
+void launch_kv_to_cache(int dtype, const void* qkv, long long ld, int k_col, int v_col, int Hkv, int hd,
+                        const int* pos, int N, int seq, int t_max, void* kc, void* vc, DevStatus* st,
+                        cudaStream_t s);
+void launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s);
+void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* n_run, cudaStream_t s);
+void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s);
+void launch_embed(int dtype, const void* table, int vocab, const int* ids, int n, int D, float* out,
+                  DevStatus* st, cudaStream_t s);
+void launch_trace_rows(int src_is_model_dtype, int dtype, const void* src, int W, int row0, int n,
+                       const float* bias, float* dst, cudaStream_t s);
+
+}  // namespace rdt

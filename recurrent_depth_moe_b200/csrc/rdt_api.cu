@@ -1,0 +1,552 @@
+// librdt C ABI: host validation, workspace carving and per-loop orchestration of
+// the recurrent block.  Host code only enqueues kernels on the caller's stream;
+// nothing here allocates device memory or synchronises (except
+// rdt_read_device_status).
+#include "../../include/rdt.h"
+#include "common.cuh"
+#include "kernels.h"
+
+#include <string.h>
+#include <algorithm>
+
+using namespace rdt;
+
+namespace {
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct Layout {
+  // byte offsets into the workspace
+  size_t status, h, combined, a, qkv, cq_raw, cq, q, kv_raw, ckv, krope, kvu, attn, x1, f, logits;
+  size_t ids, gates, rank, counts, offsets, tiles, ntiles, slot_of, tok_of, gate_of, xg, u, y;
+  size_t run_list, run_idx, nrun, cum, halted, Avec, emb, rope, pos, p_buf, part_o, part_ml, xn;
+  size_t total;
+  int max_tiles, max_slots, rope_dim, rope_pos, n_split;
+};
+
+int esize(const rdt_config* c) { return c->dtype == 0 ? 4 : 2; }
+
+rdt_status check_config(const rdt_config* c) {
+  if (!c) return RDT_ERR_INVALID_ARG;
+  if (c->dim <= 0 || c->n_heads <= 0 || (c->dtype != 0 && c->dtype != 1)) return RDT_ERR_INVALID_ARG;
+  if (c->attn_type == 0) {
+    if (c->n_kv_heads <= 0 || c->dim % c->n_heads || c->n_heads % c->n_kv_heads) return RDT_ERR_INVALID_ARG;
+    int hd = c->dim / c->n_heads;
+    if (hd % 2 || hd > 192) return RDT_ERR_UNSUPPORTED;
+  } else if (c->attn_type == 1) {
+    if (c->kv_lora_rank <= 0 || c->q_lora_rank <= 0 || c->qk_rope_head_dim <= 0 || c->qk_nope_head_dim < 0 ||
+        c->v_head_dim <= 0 || c->qk_rope_head_dim % 2)
+      return RDT_ERR_INVALID_ARG;
+    if (c->qk_rope_head_dim + c->qk_nope_head_dim > 192 || c->v_head_dim > 128) return RDT_ERR_UNSUPPORTED;
+  } else {
+    return RDT_ERR_INVALID_ARG;
+  }
+  if (c->n_experts < 0 || c->n_shared_experts < 0 || c->top_k < 0 || c->top_k > c->n_experts) return RDT_ERR_INVALID_ARG;
+  if (c->n_experts > 256 || c->top_k > 32 || c->n_experts + c->n_shared_experts > 1024 ||
+      c->top_k + c->n_shared_experts > 64)
+    return RDT_ERR_UNSUPPORTED;
+  if (c->n_experts + c->n_shared_experts < 1 || c->expert_dim <= 0) return RDT_ERR_INVALID_ARG;
+  if (c->lora_rank < 0 || c->lora_rank > 64 || c->max_loop_iters < 1) return RDT_ERR_INVALID_ARG;
+  if (c->loop_dim < 0 || c->loop_dim % 2 || c->loop_dim > c->dim) return RDT_ERR_INVALID_ARG;
+  if (!(c->norm_eps >= 0.f) || !(c->rope_theta > 0.f) || !(c->loop_theta > 0.f)) return RDT_ERR_INVALID_ARG;
+  return RDT_OK;
+}
+
+void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
+  const size_t N = (size_t)B * T, D = c->dim, es = esize(c);
+  const int k = c->top_k, S = c->n_shared_experts, E = c->n_experts, F = c->expert_dim;
+  const size_t M = N * (size_t)(k + S);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
+  memset(L, 0, sizeof(*L));
+  L->status = take(sizeof(DevStatus));
+  L->h = take(N * D * 4);
+  L->combined = take(N * D * 4);
+  L->a = take(N * D * es);
+  int H = c->n_heads, dv = 0;
+  if (c->attn_type == 0) {
+    int hd = c->dim / H;
+    L->qkv = take(N * (size_t)(H + 2 * c->n_kv_heads) * hd * es);
+    dv = hd;
+    L->rope_dim = hd;
+  } else {
+    int dn = c->qk_nope_head_dim, dr = c->qk_rope_head_dim;
+    dv = c->v_head_dim;
+    L->cq_raw = take(N * c->q_lora_rank * 4);
+    L->cq = take(N * c->q_lora_rank * es);
+    L->q = take(N * (size_t)H * (dn + dr) * es);
+    L->kv_raw = take(N * (size_t)(c->kv_lora_rank + dr) * 4);
+    L->ckv = take(N * c->kv_lora_rank * es);
+    L->krope = take(N * dr * es);
+    L->kvu = take(N * (size_t)H * (dn + dv) * es);
+    L->rope_dim = dr;
+  }
+  L->attn = take(N * (size_t)H * dv * es);
+  L->x1 = take(N * D * 4);
+  L->f = take(N * D * es);
+  L->xn = take(N * D * es);
+  L->logits = take(N * (size_t)std::max(E, 1) * 4);
+  L->ids = take(N * std::max(k, 1) * 4);
+  L->gates = take(N * std::max(k, 1) * 4);
+  L->rank = take(N * std::max(k, 1) * 4);
+  L->counts = take((size_t)std::max(E, 1) * 4);
+  L->offsets = take((size_t)(E + S + 1) * 4);
+  L->max_tiles = (int)((M + 63) / 64) + E + S + 1;
+  L->tiles = take((size_t)L->max_tiles * 16);
+  L->ntiles = take(16);
+  L->max_slots = (int)M;
+  L->slot_of = take(N * (k + S) * 4);
+  L->tok_of = take(M * 4);
+  L->gate_of = take(M * 4);
+  L->xg = take(M * D * es);
+  L->u = take(M * (size_t)F * es);
+  L->y = take(M * D * 4);
+  L->run_list = take(N * 4);
+  L->run_idx = take(N * 4);
+  L->nrun = take(16);
+  L->cum = take(N * 4);
+  L->halted = take(N * 4);
+  L->p_buf = take(N * 4);
+  L->Avec = take(D * 4);
+  L->emb = take((size_t)std::max(c->loop_dim, 2) * 4);
+  L->rope_pos = std::max(max_keys, T);
+  L->rope = take((size_t)L->rope_pos * (L->rope_dim / 2) * 8);
+  L->pos = take(N * 4);
+  L->n_split = 0;
+  L->part_o = take(16);
+  L->part_ml = take(16);
+  L->total = off;
+}
+
+template <typename P> P at(void* ws, size_t off) { return (P)((char*)ws + off); }
+
+struct Ctx {
+  const rdt_config* c;
+  const rdt_weights* w;
+  Layout L;
+  void* ws;
+  cudaStream_t s;
+  DevStatus* st;
+  int dtype;
+};
+
+#define RDT_TRY(x)                          \
+  do {                                      \
+    if ((x) != 0) return RDT_ERR_CUDA;      \
+  } while (0)
+
+GemmParams gemm_base(const Ctx& x) {
+  GemmParams g;
+  memset(&g, 0, sizeof(g));
+  g.st = x.st;
+  g.impl = -1;
+  return g;
+}
+
+// Attention sub-block (S2 + S3 + S4): x1 = combined + Attn(a).  rows = N (all rows:
+// halted rows keep contributing keys/values).
+rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const void* a, float* x1,
+                           const rdt_kv_cache* cache, int loop_t, int start_pos, bool decode) {
+  const rdt_config* c = x.c;
+  const rdt_weights* w = x.w;
+  const int N = B * T, D = c->dim, H = c->n_heads, es = esize(c);
+  const int* pos = at<const int*>(x.ws, x.L.pos);
+  const float2* tab = at<const float2*>(x.ws, x.L.rope);
+  void* attn = at<void*>(x.ws, x.L.attn);
+  AttnParams ap;
+  memset(&ap, 0, sizeof(ap));
+  ap.B = B; ap.T = T; ap.H = H; ap.q_pos = pos;
+  int dv;
+  if (c->attn_type == 0) {
+    const int Hkv = c->n_kv_heads, hd = D / H, W = (H + 2 * Hkv) * hd;
+    void* qkv = at<void*>(x.ws, x.L.qkv);
+    GemmParams g = gemm_base(x);
+    g.A = a; g.lda = D; g.B = w->w_qkv; g.ldb = D; g.M = N; g.N = W; g.K = D;
+    g.C = qkv; g.ldc = W; g.pos = pos; g.rope_tab = tab; g.rope_half = hd / 2; g.n_rope = 2;
+    g.rope[0] = RopeDesc{0, H, hd, 0, hd};
+    g.rope[1] = RopeDesc{H * hd, Hkv, hd, 0, hd};
+    RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, x.s));
+    ap.q = qkv; ap.q_row = W; ap.q_head = hd; ap.dn = hd; ap.dr = 0; ap.dv = hd; ap.G = H / Hkv;
+    ap.scale = 1.f / sqrtf((float)hd);
+    const bool use_cache = cache && cache->k;
+    if (use_cache) {
+      size_t per_loop = (size_t)cache->batch * Hkv * cache->t_max * hd * es;
+      char* kc = (char*)cache->k + per_loop * loop_t;
+      char* vc = (char*)cache->v + per_loop * loop_t;
+      launch_kv_to_cache(x.dtype, qkv, W, H * hd, (H + Hkv) * hd, Hkv, hd, pos, N, T, cache->t_max, kc, vc, x.st, x.s);
+      if (decode || start_pos > 0) {
+        long long sj = hd, sg = (long long)cache->t_max * hd, sb = (long long)Hkv * sg;
+        ap.k1 = kc; ap.k1_b = sb; ap.k1_j = sj; ap.k1_g = sg;
+        ap.v = vc; ap.v_b = sb; ap.v_j = sj; ap.v_g = sg;
+        ap.key_pos0 = 0;
+        ap.n_keys = decode ? cache->t_max : start_pos + T;
+      }
+    }
+    if (!ap.k1) {
+      ap.k1 = (const char*)qkv + (size_t)H * hd * es; ap.k1_b = (long long)T * W; ap.k1_j = W; ap.k1_g = hd;
+      ap.v = (const char*)qkv + (size_t)(H + Hkv) * hd * es; ap.v_b = (long long)T * W; ap.v_j = W; ap.v_g = hd;
+      ap.key_pos0 = start_pos; ap.n_keys = T;
+    }
+    dv = hd;
+  } else {
+    if (cache && cache->k) return RDT_ERR_UNSUPPORTED;   // MLA latent-cache decode not built
+    const int dn = c->qk_nope_head_dim, dr = c->qk_rope_head_dim, kvr = c->kv_lora_rank, ql = c->q_lora_rank;
+    dv = c->v_head_dim;
+    float* cq_raw = at<float*>(x.ws, x.L.cq_raw);
+    void* cq = at<void*>(x.ws, x.L.cq);
+    void* q = at<void*>(x.ws, x.L.q);
+    float* kv_raw = at<float*>(x.ws, x.L.kv_raw);
+    void* ckv = at<void*>(x.ws, x.L.ckv);
+    void* krope = at<void*>(x.ws, x.L.krope);
+    void* kvu = at<void*>(x.ws, x.L.kvu);
+    GemmParams g = gemm_base(x);
+    g.A = a; g.lda = D; g.B = w->w_q_down; g.ldb = D; g.M = N; g.N = ql; g.K = D; g.C = cq_raw; g.ldc = ql;
+    RDT_TRY(launch_gemm(x.dtype, EPI_STORE_F32, g, x.s));
+    launch_rmsnorm(1, x.dtype, cq_raw, ql, w->q_norm_w, cq, ql, N, ql, c->norm_eps, x.s);
+    g = gemm_base(x);
+    g.A = cq; g.lda = ql; g.B = w->w_q_up; g.ldb = ql; g.M = N; g.N = H * (dn + dr); g.K = ql;
+    g.C = q; g.ldc = H * (dn + dr); g.pos = pos; g.rope_tab = tab; g.rope_half = dr / 2; g.n_rope = 1;
+    g.rope[0] = RopeDesc{0, H, dn + dr, dn, dr};
+    RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, x.s));
+    g = gemm_base(x);
+    g.A = a; g.lda = D; g.B = w->w_kv_down; g.ldb = D; g.M = N; g.N = kvr + dr; g.K = D; g.C = kv_raw; g.ldc = kvr + dr;
+    RDT_TRY(launch_gemm(x.dtype, EPI_STORE_F32, g, x.s));
+    launch_mla_kv_prep(x.dtype, kv_raw, kvr, dr, w->kv_norm_w, c->norm_eps, pos, tab, ckv, krope, N, x.s);
+    g = gemm_base(x);
+    g.A = ckv; g.lda = kvr; g.B = w->w_kv_up; g.ldb = kvr; g.M = N; g.N = H * (dn + dv); g.K = kvr;
+    g.C = kvu; g.ldc = H * (dn + dv);
+    RDT_TRY(launch_gemm(x.dtype, EPI_STORE_T, g, x.s));
+    const long long kvw = (long long)H * (dn + dv);
+    ap.q = q; ap.q_row = H * (dn + dr); ap.q_head = dn + dr; ap.dn = dn; ap.dr = dr; ap.dv = dv; ap.G = 1;
+    ap.k1 = kvu; ap.k1_b = (long long)T * kvw; ap.k1_j = kvw; ap.k1_g = dn + dv;
+    ap.k2 = krope; ap.k2_b = (long long)T * dr; ap.k2_j = dr;
+    ap.v = (const char*)kvu + (size_t)dn * es; ap.v_b = (long long)T * kvw; ap.v_j = kvw; ap.v_g = dn + dv;
+    ap.key_pos0 = start_pos; ap.n_keys = T;
+    ap.scale = 1.f / sqrtf((float)(dn + dr));
+  }
+  ap.o = attn; ap.o_row = (long long)H * dv; ap.o_head = dv;
+  RDT_TRY(launch_attention(x.dtype, ap, x.s));
+  GemmParams g = gemm_base(x);
+  g.A = attn; g.lda = (long long)H * dv; g.B = w->w_o; g.ldb = (long long)H * dv; g.M = N; g.N = D; g.K = H * dv;
+  g.C = x1; g.ldc = D; g.resid = combined; g.ld_resid = D;
+  RDT_TRY(launch_gemm(x.dtype, EPI_RESID_F32, g, x.s));
+  return RDT_OK;
+}
+
+// MoE FFN (S5 .. S8) on the running rows: y[slot] = gate * Expert_e(f[token]).
+rdt_status moe_block(Ctx& x, int N, const float* x1) {
+  const rdt_config* c = x.c;
+  const rdt_weights* w = x.w;
+  const int D = c->dim, E = c->n_experts, k = c->top_k, S = c->n_shared_experts, F = c->expert_dim;
+  void* f = at<void*>(x.ws, x.L.f);
+  launch_rmsnorm(1, x.dtype, x1, D, w->ffn_norm_w, f, D, N, D, c->norm_eps, x.s);
+  float* logits = at<float*>(x.ws, x.L.logits);
+  GemmParams g = gemm_base(x);
+  g.A = f; g.lda = D; g.B = w->w_router; g.ldb = D; g.M = N; g.N = E; g.K = D; g.C = logits; g.ldc = E;
+  RDT_TRY(launch_gemm(x.dtype, EPI_STORE_F32, g, x.s));
+  RouteParams rp;
+  memset(&rp, 0, sizeof(rp));
+  rp.logits = logits; rp.bias = w->router_bias; rp.N = N; rp.E = E; rp.k = k; rp.S = S;
+  rp.run_list = at<int*>(x.ws, x.L.run_list); rp.n_run = at<int*>(x.ws, x.L.nrun);
+  rp.ids = at<int*>(x.ws, x.L.ids); rp.gates = at<float*>(x.ws, x.L.gates); rp.rank = at<int*>(x.ws, x.L.rank);
+  rp.counts = at<int*>(x.ws, x.L.counts); rp.offsets = at<int*>(x.ws, x.L.offsets);
+  rp.tiles = at<int*>(x.ws, x.L.tiles); rp.n_tiles = at<int*>(x.ws, x.L.ntiles); rp.max_tiles = x.L.max_tiles;
+  rp.slot_of = at<int*>(x.ws, x.L.slot_of); rp.tok_of = at<int*>(x.ws, x.L.tok_of);
+  rp.gate_of = at<float*>(x.ws, x.L.gate_of); rp.f = f; rp.xg = at<void*>(x.ws, x.L.xg); rp.D = D;
+  rp.max_slots = x.L.max_slots; rp.st = x.st;
+  // expert GEMMs pick their tile height from the implementation that will run them
+  GemmParams up = gemm_base(x);
+  up.A = rp.xg; up.lda = D; up.B = w->w13; up.ldb = D; up.b_group_stride = (long long)2 * F * D;
+  up.M = x.L.max_slots; up.N = F; up.K = D; up.up_off = F; up.b_rows = (long long)(E + S) * 2 * F;
+  up.tiles = rp.tiles; up.n_tiles = rp.n_tiles; up.max_tiles = x.L.max_tiles;
+  up.C = at<void*>(x.ws, x.L.u); up.ldc = F;
+  GemmParams dn = gemm_base(x);
+  dn.A = up.C; dn.lda = F; dn.B = w->w2; dn.ldb = F; dn.b_group_stride = (long long)D * F;
+  dn.M = x.L.max_slots; dn.N = D; dn.K = F; dn.b_rows = (long long)(E + S) * D; dn.tiles = rp.tiles; dn.n_tiles = rp.n_tiles; dn.max_tiles = x.L.max_tiles;
+  dn.C = at<float*>(x.ws, x.L.y); dn.ldc = D; dn.row_scale = rp.gate_of;
+  // both expert GEMMs consume the same tile list, so they must share one tile height
+  GemmImpl iu = gemm_pick(x.dtype, up, EPI_SWIGLU_T), id = gemm_pick(x.dtype, dn, EPI_GATE_F32);
+  if (iu != id) iu = id = GEMM_SIMT;
+  up.impl = dn.impl = (int)iu;
+  rp.tile_m = gemm_tile_m(iu);
+  if (cudaMemsetAsync(rp.counts, 0, sizeof(int) * std::max(E, 1), x.s) != cudaSuccess) return RDT_ERR_CUDA;
+  launch_router_topk(rp, x.s);
+  launch_route_scan(rp, x.s);
+  launch_route_scatter(x.dtype, rp, x.s);
+  RDT_TRY(launch_gemm(x.dtype, EPI_SWIGLU_T, up, x.s));
+  RDT_TRY(launch_gemm(x.dtype, EPI_GATE_F32, dn, x.s));
+  return RDT_OK;
+}
+
+CombineParams combine_base(Ctx& x, int N) {
+  const rdt_config* c = x.c;
+  const rdt_weights* w = x.w;
+  CombineParams cp;
+  memset(&cp, 0, sizeof(cp));
+  cp.N = N; cp.D = c->dim; cp.k = c->top_k; cp.S = c->n_shared_experts; cp.r = c->lora_rank;
+  cp.max_loop_iters = c->max_loop_iters; cp.max_slots = x.L.max_slots;
+  cp.x1 = at<float*>(x.ws, x.L.x1); cp.y = at<float*>(x.ws, x.L.y); cp.slot_of = at<int*>(x.ws, x.L.slot_of);
+  cp.ids = at<int*>(x.ws, x.L.ids);
+  cp.lora_down = w->lora_down; cp.lora_B = w->lora_B; cp.lora_scale = w->lora_scale;
+  cp.A = at<float*>(x.ws, x.L.Avec); cp.inj_B = w->inj_B;
+  cp.h = at<float*>(x.ws, x.L.h); cp.h_state = at<float*>(x.ws, x.L.h);
+  cp.halt_wv = w->halt_w; cp.halt_b = w->halt_b;
+  cp.cum = at<float*>(x.ws, x.L.cum); cp.halted = at<int*>(x.ws, x.L.halted);
+  cp.p_out = at<float*>(x.ws, x.L.p_buf);
+  cp.st = x.st;
+  return cp;
+}
+
+rdt_status check_block_weights(const rdt_config* c, const rdt_weights* w, bool moe) {
+  if (!w || !w->attn_norm_w || !w->ffn_norm_w || !w->w_o || !w->w13 || !w->w2) return RDT_ERR_INVALID_ARG;
+  if (c->attn_type == 0 && !w->w_qkv) return RDT_ERR_INVALID_ARG;
+  if (c->attn_type == 1 && (!w->w_q_down || !w->q_norm_w || !w->w_q_up || !w->w_kv_down || !w->kv_norm_w || !w->w_kv_up))
+    return RDT_ERR_INVALID_ARG;
+  if (moe && (!w->w_router || !w->router_bias || c->n_experts < 1 || c->top_k < 1)) return RDT_ERR_INVALID_ARG;
+  return RDT_OK;
+}
+
+rdt_status check_ws(void* ws, size_t ws_bytes, const Layout& L) {
+  if (!ws || ((uintptr_t)ws & 255)) return RDT_ERR_WORKSPACE;
+  if (ws_bytes < L.total) return RDT_ERR_WORKSPACE;
+  return RDT_OK;
+}
+
+// Shared loop driver of prefill (decode = false) and decode (decode = true).
+rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float* h0, const void* e, int B, int T,
+                         int start_pos, const int32_t* cache_len, int n_loops, float thr, const float* halt_off,
+                         float* h_out, float* halt_weights, int32_t* expert_ids, const rdt_kv_cache* cache,
+                         const rdt_trace* trace, int flags, void* ws, size_t ws_bytes, cudaStream_t s, bool decode) {
+  rdt_status st = check_config(c);
+  if (st != RDT_OK) return st;
+  if ((st = check_block_weights(c, w, true)) != RDT_OK) return st;
+  if (!w->rec_norm_w || !w->log_A || !w->log_dt || !w->inj_B) return RDT_ERR_INVALID_ARG;
+  if (c->lora_rank > 0 && (!w->lora_down || !w->lora_B || !w->lora_scale)) return RDT_ERR_INVALID_ARG;
+  if (!h0 || !e || !h_out || !halt_weights || !expert_ids) return RDT_ERR_INVALID_ARG;
+  if (B <= 0 || T <= 0 || n_loops <= 0 || start_pos < 0) return RDT_ERR_INVALID_ARG;
+  if (thr != thr) return RDT_ERR_INVALID_ARG;   // NaN threshold
+  const bool act_on = thr > 0.f;
+  if (act_on && (!w->halt_w || !w->halt_b)) return RDT_ERR_INVALID_ARG;
+  if ((long long)B * T > (1LL << 30)) return RDT_ERR_UNSUPPORTED;
+  int max_keys = start_pos + T;
+  if (cache) {
+    if (!cache->k || !cache->v || cache->t_max <= 0 || cache->batch < B || cache->n_loops < n_loops)
+      return RDT_ERR_INVALID_ARG;
+    if (c->attn_type != 0) return RDT_ERR_UNSUPPORTED;
+    if (!decode && start_pos + T > cache->t_max) return RDT_ERR_INVALID_ARG;
+    max_keys = std::max(max_keys, cache->t_max);
+  }
+  if (decode && (!cache || !cache_len)) return RDT_ERR_INVALID_ARG;
+  if (trace && (trace->row0 < 0 || trace->n_rows < 0 || trace->row0 + trace->n_rows > B * T)) return RDT_ERR_INVALID_ARG;
+  Ctx x;
+  x.c = c; x.w = w; x.ws = ws; x.s = s; x.dtype = c->dtype;
+  make_layout(c, B, T, max_keys, &x.L);
+  if ((st = check_ws(ws, ws_bytes, x.L)) != RDT_OK) return st;
+  x.st = at<DevStatus*>(ws, x.L.status);
+  const int N = B * T, D = c->dim, E = c->n_experts;
+  const bool transformer_off = (flags & RDT_FLAG_TRANSFORMER_OFF) != 0;
+  float* h = at<float*>(ws, x.L.h);
+  float* combined = at<float*>(ws, x.L.combined);
+  void* a = at<void*>(ws, x.L.a);
+  float* x1 = at<float*>(ws, x.L.x1);
+  float* emb = at<float*>(ws, x.L.emb);
+  int* pos = at<int*>(ws, x.L.pos);
+  // per-call set-up
+  if (cudaMemsetAsync(x.st, 0, sizeof(DevStatus), s) != cudaSuccess) return RDT_ERR_CUDA;
+  if (cudaMemcpyAsync(h, h0, (size_t)N * D * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return RDT_ERR_CUDA;
+  if (cudaMemsetAsync(h_out, 0, (size_t)N * D * 4, s) != cudaSuccess) return RDT_ERR_CUDA;
+  if (cudaMemsetAsync(at<void*>(ws, x.L.cum), 0, (size_t)N * 4, s) != cudaSuccess) return RDT_ERR_CUDA;
+  if (cudaMemsetAsync(at<void*>(ws, x.L.halted), 0, (size_t)N * 4, s) != cudaSuccess) return RDT_ERR_CUDA;
+  launch_lti_A(w->log_A, w->log_dt, at<float*>(ws, x.L.Avec), D, s);
+  launch_rope_table(at<float2*>(ws, x.L.rope), x.L.rope_pos, x.L.rope_dim, c->rope_theta, s);
+  if (decode) launch_positions_decode(pos, cache_len, B, cache->t_max, x.st, s);
+  else launch_positions(pos, N, T, start_pos, s);
+  launch_iota(at<int*>(ws, x.L.run_list), at<int*>(ws, x.L.run_idx), at<int*>(ws, x.L.nrun), N, s);
+  CombineParams cp = combine_base(x, N);
+  cp.n_loops = n_loops; cp.act_on = act_on; cp.thr = thr; cp.e = e; cp.h_out = h_out;
+  cp.halt_off = halt_off; cp.halt_w_out = halt_weights; cp.ids_out = expert_ids;
+  cp.transformer_off = transformer_off;
+  for (int t = 0; t < n_loops; ++t) {
+    if (trace && trace->h_in)
+      launch_trace_rows(0, x.dtype, h, D, trace->row0, trace->n_rows, nullptr,
+                        trace->h_in + (size_t)t * trace->n_rows * D, s);
+    launch_loop_emb(emb, c->loop_dim, t, c->loop_theta, s);
+    launch_loop_prologue(x.dtype, h, e, emb, c->loop_dim, w->rec_norm_w, w->attn_norm_w, combined, a, N, D,
+                         c->norm_eps, s);
+    if (!transformer_off) {
+      if ((st = attention_block(x, B, T, combined, a, x1, cache, t, start_pos, decode)) != RDT_OK) return st;
+      if ((st = moe_block(x, N, x1)) != RDT_OK) return st;
+      if (trace && trace->f)
+        launch_trace_rows(1, x.dtype, at<void*>(ws, x.L.f), D, trace->row0, trace->n_rows, nullptr,
+                          trace->f + (size_t)t * trace->n_rows * D, s);
+      if (trace && trace->biased_logits)
+        launch_trace_rows(0, x.dtype, at<float*>(ws, x.L.logits), E, trace->row0, trace->n_rows, w->router_bias,
+                          trace->biased_logits + (size_t)t * trace->n_rows * E, s);
+    }
+    cp.t = t;
+    launch_combine(x.dtype, cp, N, s);
+    if (trace && trace->p && act_on)
+      launch_trace_rows(0, x.dtype, at<float*>(ws, x.L.p_buf), 1, trace->row0, trace->n_rows, nullptr,
+                        trace->p + (size_t)t * trace->n_rows, s);
+    if (act_on && t + 1 < n_loops)
+      launch_compact(at<int*>(ws, x.L.halted), N, at<int*>(ws, x.L.run_list), at<int*>(ws, x.L.run_idx),
+                     at<int*>(ws, x.L.nrun), s);
+  }
+  if (cudaGetLastError() != cudaSuccess) return RDT_ERR_CUDA;
+  return RDT_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------------------------------
+// GEMM dispatch
+// ------------------------------------------------------------------------------------------
+namespace rdt {
+int launch_gemm_simt(int dtype, int epi, const GemmParams& p, cudaStream_t s);
+int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s);
+bool gemm_tc_supports(const GemmParams& p, int epi);
+int launch_attention_simt(int dtype, const AttnParams& p, cudaStream_t s);
+
+int gemm_tile_m(GemmImpl impl) { return impl == GEMM_TC ? 128 : 64; }
+GemmImpl gemm_pick(int dtype, const GemmParams& p, int epi) {
+  if (p.impl == GEMM_SIMT) return GEMM_SIMT;
+  if (dtype == 1 && gemm_tc_supports(p, epi)) return GEMM_TC;
+  return GEMM_SIMT;
+}
+int launch_gemm(int dtype, int epi, const GemmParams& p, cudaStream_t s) {
+  if (gemm_pick(dtype, p, epi) == GEMM_TC) return launch_gemm_tc(epi, p, s);
+  return launch_gemm_simt(dtype, epi, p, s);
+}
+int launch_attention(int dtype, const AttnParams& p, cudaStream_t s) { return launch_attention_simt(dtype, p, s); }
+}  // namespace rdt
+
+// ------------------------------------------------------------------------------------------
+// C ABI
+// ------------------------------------------------------------------------------------------
+extern "C" {
+
+size_t rdt_workspace_size(const rdt_config* cfg, int batch, int seq, int max_keys) {
+  if (check_config(cfg) != RDT_OK || batch <= 0 || seq <= 0) return 0;
+  Layout L;
+  make_layout(cfg, batch, seq, std::max(max_keys, seq), &L);
+  return L.total;
+}
+
+rdt_status rdt_recurrent_forward(const rdt_config* cfg, const rdt_weights* w, const float* h0, const void* e,
+                                 int batch, int seq, int start_pos, int n_loops, float act_threshold,
+                                 const float* halt_logit_offset, float* h_out, float* halt_weights,
+                                 int32_t* expert_ids, const rdt_kv_cache* cache, const rdt_trace* trace, int flags,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  return run_recurrent(cfg, w, h0, e, batch, seq, start_pos, nullptr, n_loops, act_threshold, halt_logit_offset,
+                       h_out, halt_weights, expert_ids, cache, trace, flags, ws, ws_bytes, (cudaStream_t)stream,
+                       false);
+}
+
+rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_weights* w, const float* h0, const void* e,
+                                     int batch, const int32_t* cache_len, int n_loops, float act_threshold,
+                                     float* h_out, float* halt_weights, int32_t* expert_ids,
+                                     const rdt_kv_cache* cache, void* ws, size_t ws_bytes, void* stream) {
+  return run_recurrent(cfg, w, h0, e, batch, 1, 0, cache_len, n_loops, act_threshold, nullptr, h_out, halt_weights,
+                       expert_ids, cache, nullptr, 0, ws, ws_bytes, (cudaStream_t)stream, true);
+}
+
+rdt_status rdt_block_forward(const rdt_config* cfg, const rdt_weights* w, const float* x_in, float* x_out, int batch,
+                             int seq, int start_pos, void* ws, size_t ws_bytes, void* stream) {
+  rdt_status st = check_config(cfg);
+  if (st != RDT_OK) return st;
+  const bool moe = cfg->n_experts > 0;
+  if ((st = check_block_weights(cfg, w, moe)) != RDT_OK) return st;
+  if (!x_in || !x_out || x_in == x_out || batch <= 0 || seq <= 0 || start_pos < 0) return RDT_ERR_INVALID_ARG;
+  if (!moe && cfg->n_shared_experts != 1) return RDT_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  Ctx x;
+  x.c = cfg; x.w = w; x.ws = ws; x.s = s; x.dtype = cfg->dtype;
+  make_layout(cfg, batch, seq, start_pos + seq, &x.L);
+  if ((st = check_ws(ws, ws_bytes, x.L)) != RDT_OK) return st;
+  x.st = at<DevStatus*>(ws, x.L.status);
+  const int N = batch * seq, D = cfg->dim, F = cfg->expert_dim;
+  if (cudaMemsetAsync(x.st, 0, sizeof(DevStatus), s) != cudaSuccess) return RDT_ERR_CUDA;
+  launch_rope_table(at<float2*>(ws, x.L.rope), x.L.rope_pos, x.L.rope_dim, cfg->rope_theta, s);
+  launch_positions(at<int*>(ws, x.L.pos), N, seq, start_pos, s);
+  void* a = at<void*>(ws, x.L.a);
+  float* x1 = at<float*>(ws, x.L.x1);
+  launch_rmsnorm(1, x.dtype, x_in, D, w->attn_norm_w, a, D, N, D, cfg->norm_eps, s);
+  if ((st = attention_block(x, batch, seq, x_in, a, x1, nullptr, 0, start_pos, false)) != RDT_OK) return st;
+  if (moe) {
+    launch_iota(at<int*>(ws, x.L.run_list), at<int*>(ws, x.L.run_idx), at<int*>(ws, x.L.nrun), N, s);
+    if ((st = moe_block(x, N, x1)) != RDT_OK) return st;
+    CombineParams cp = combine_base(x, N);
+    cp.block_only = 1; cp.out = x_out;
+    launch_combine(x.dtype, cp, N, s);
+  } else {
+    void* f = at<void*>(ws, x.L.f);
+    launch_rmsnorm(1, x.dtype, x1, D, w->ffn_norm_w, f, D, N, D, cfg->norm_eps, s);
+    GemmParams up = gemm_base(x);
+    up.A = f; up.lda = D; up.B = w->w13; up.ldb = D; up.M = N; up.N = F; up.K = D; up.up_off = F;
+    up.C = at<void*>(ws, x.L.u); up.ldc = F;
+    if (launch_gemm(x.dtype, EPI_SWIGLU_T, up, s)) return RDT_ERR_CUDA;
+    GemmParams dn = gemm_base(x);
+    dn.A = up.C; dn.lda = F; dn.B = w->w2; dn.ldb = F; dn.M = N; dn.N = D; dn.K = F;
+    dn.C = x_out; dn.ldc = D; dn.resid = x1; dn.ld_resid = D;
+    if (launch_gemm(x.dtype, EPI_RESID_F32, dn, s)) return RDT_ERR_CUDA;
+  }
+  if (cudaGetLastError() != cudaSuccess) return RDT_ERR_CUDA;
+  return RDT_OK;
+}
+
+rdt_status rdt_embed(const rdt_config* cfg, const void* table, int vocab, const int32_t* ids, int n, float* out,
+                     void* stream) {
+  if (!cfg || cfg->dim <= 0 || (cfg->dtype != 0 && cfg->dtype != 1) || !table || !ids || !out || vocab <= 0 || n <= 0)
+    return RDT_ERR_INVALID_ARG;
+  launch_embed(cfg->dtype, table, vocab, ids, n, cfg->dim, out, nullptr, (cudaStream_t)stream);
+  return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
+}
+
+rdt_status rdt_head(const rdt_config* cfg, const float* xin, int n, const float* norm_w, const void* head, int vocab,
+                    float* logits, void* ws, size_t ws_bytes, void* stream) {
+  rdt_status st = check_config(cfg);
+  if (st != RDT_OK) return st;
+  if (!xin || n <= 0 || !norm_w || !head || vocab <= 0 || !logits) return RDT_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  Layout L;
+  make_layout(cfg, 1, n, n, &L);
+  if ((st = check_ws(ws, ws_bytes, L)) != RDT_OK) return st;
+  void* xn = at<void*>(ws, L.xn);
+  launch_rmsnorm(1, cfg->dtype, xin, cfg->dim, norm_w, xn, cfg->dim, n, cfg->dim, cfg->norm_eps, s);
+  GemmParams g;
+  memset(&g, 0, sizeof(g));
+  g.impl = -1;
+  g.A = xn; g.lda = cfg->dim; g.B = head; g.ldb = cfg->dim; g.M = n; g.N = vocab; g.K = cfg->dim;
+  g.C = logits; g.ldc = vocab; g.st = at<DevStatus*>(ws, L.status);
+  if (launch_gemm(cfg->dtype, EPI_STORE_F32, g, s)) return RDT_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
+}
+
+rdt_status rdt_read_device_status(void* ws, void* stream) {
+  if (!ws) return RDT_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  DevStatus hs;
+  if (cudaMemcpyAsync(&hs, ws, sizeof(hs), cudaMemcpyDeviceToHost, s) != cudaSuccess) return RDT_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return RDT_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(hs), s) != cudaSuccess) return RDT_ERR_CUDA;
+  if (hs.code == ST_TIMEOUT) return RDT_ERR_DEVICE_TIMEOUT;
+  if (hs.code == ST_BOUNDS) return RDT_ERR_DEVICE_BOUNDS;
+  return RDT_OK;
+}
+
+const char* rdt_status_string(rdt_status s) {
+  switch (s) {
+    case RDT_OK: return "ok";
+    case RDT_ERR_INVALID_ARG: return "invalid argument";
+    case RDT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RDT_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case RDT_ERR_CUDA: return "CUDA runtime error";
+    case RDT_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case RDT_ERR_DEVICE_BOUNDS: return "device-side bounds check failed";
+  }
+  return "unknown status";
+}
+
+const char* rdt_version(void) { return "librdt 0.1 sm_100a"; }
+
+}  // extern "C"

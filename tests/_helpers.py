@@ -1,0 +1,122 @@
+"""Shared helpers of the parity tests: device copies of seeded inputs, metrics,
+and the teacher-forced router check."""
+from __future__ import annotations
+
+import math
+
+import torch
+
+import rdt_inputs as RI
+from oracle import rdt_oracle as O
+
+F64 = torch.float64
+
+
+def to_dev(w, device="cuda"):
+    if isinstance(w, dict):
+        return {k: to_dev(v, device) for k, v in w.items()}
+    if isinstance(w, list):
+        return [to_dev(v, device) for v in w]
+    return w.to(device).contiguous()
+
+
+def to_cpu(w):
+    if isinstance(w, dict):
+        return {k: to_cpu(v) for k, v in w.items()}
+    if isinstance(w, list):
+        return [to_cpu(v) for v in w]
+    return w.detach().cpu()
+
+
+def max_rel(g: torch.Tensor, o: torch.Tensor) -> float:
+    """fp32-mode metric: max |g - o| / max |o| over the tensor."""
+    g, o = g.detach().cpu().double(), o.detach().cpu().double()
+    return float((g - o).abs().max() / o.abs().max().clamp_min(1e-30))
+
+
+def rel_l2(g: torch.Tensor, o: torch.Tensor) -> float:
+    """bf16-mode metric: ||g - o||_2 / ||o||_2."""
+    g, o = g.detach().cpu().double(), o.detach().cpu().double()
+    return float((g - o).norm() / o.norm().clamp_min(1e-30))
+
+
+FP32_TOL = 1e-4      # max relative error, fp32 mode
+BF16_TOL = 2e-2      # relative L2, bf16 mode
+ID_MARGIN = 1e-3     # router ties below this biased-logit margin may differ
+
+
+def topk_margin(biased: torch.Tensor, k: int) -> torch.Tensor:
+    """k-th minus (k+1)-th largest biased logit per row (inf when k = E)."""
+    s = torch.sort(biased, dim=-1, descending=True).values
+    if s.shape[-1] <= k:
+        return torch.full(s.shape[:-1], math.inf, dtype=s.dtype)
+    return s[..., k - 1] - s[..., k]
+
+
+def teacher_forced_ids(cfg, W, trace, ids_gpu: torch.Tensor, n_loops: int):
+    """Recompute top-k in fp64 on the kernel's own router input (trace.f) and compare
+    with the kernel's ids wherever the margin is >= ID_MARGIN.
+    Returns (n_compared, n_mismatch, n_skipped)."""
+    k = cfg.n_experts_per_tok
+    Wr = W["w_router"].detach().cpu().double()
+    bias = W["router_bias"].detach().cpu().double()
+    r0, n = trace.row0, trace.n_rows
+    compared = mism = skipped = 0
+    for t in range(n_loops):
+        ids_t = ids_gpu[t, r0:r0 + n].cpu().long()
+        run = ids_t[:, 0] >= 0
+        if not run.any():
+            continue
+        f = trace.f[t].cpu().double()[run]
+        biased = f @ Wr.T + bias
+        want = O.topk_lower_index(biased, k)
+        marg = topk_margin(biased, k)
+        ok = marg >= ID_MARGIN
+        got = ids_t[run]
+        compared += int(ok.sum())
+        skipped += int((~ok).sum())
+        # compare as sets in the kernel's order: the kernel emits descending biased order too
+        mism += int((got[ok] != want[ok]).any(dim=-1).sum())
+    return compared, mism, skipped
+
+
+DECISION_MARGIN = 5e-2   # bf16: rows may take another route / halting loop only at oracle near-ties
+MAX_DIVERGENT = 0.05     # ... and at most this fraction of rows may do so
+
+
+def divergent_rows(ids_g, hw_g, ids_o, hw_o, record, thr, k):
+    """Rows whose end-to-end decisions (expert ids at any loop, or the halting loop)
+    differ between the kernel and the oracle.  Each must be a near-tie in the oracle:
+    top-k margin < DECISION_MARGIN at the first loop whose ids differ, or
+    |cum + p - thr| < DECISION_MARGIN at the loop where halting differs.
+    Returns (mask of divergent rows, list of offending rows that were not near-ties)."""
+    ids_g = ids_g.cpu().long()
+    L, N = hw_o.shape
+    hl_g, hl_o = halting_loop(hw_g), halting_loop(hw_o)
+    div = torch.zeros(N, dtype=torch.bool)
+    bad = []
+    for i in range(N):
+        d_ids = (ids_g[:, i] != ids_o[:, i]).any(-1)
+        if d_ids.any():
+            div[i] = True
+            t = int(torch.nonzero(d_ids)[0])
+            if ids_o[t, i, 0] >= 0 and ids_g[t, i, 0] >= 0:
+                m = float(topk_margin(record[t]["biased"][i:i + 1], k)[0])
+                if m >= DECISION_MARGIN:
+                    bad.append((i, t, "route", m))
+            continue
+        if hl_g[i] != hl_o[i]:
+            div[i] = True
+            t = int(min(hl_g[i], hl_o[i]))
+            if thr > 0 and "cum" in record[t]:
+                m = abs(float(record[t]["cum"][i]) - thr)
+                if m >= DECISION_MARGIN:
+                    bad.append((i, t, "halt", m))
+    return div, bad
+
+
+def halting_loop(hw: torch.Tensor) -> torch.Tensor:
+    """Index of the last loop with a non-zero ACT weight, per position."""
+    L = hw.shape[0]
+    nz = (hw.cpu() > 0).to(torch.int64) * torch.arange(L)[:, None]
+    return nz.max(dim=0).values

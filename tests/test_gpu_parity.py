@@ -1,0 +1,247 @@
+"""GPU (librdt) against the CPU oracle on the same seeded inputs.
+
+fp32 mode: max relative error <= 1e-4, ids exact.  bf16 mode: relative L2 <= 2e-2 on
+h_out (and logits), ids teacher-forced with the 1e-3 margin rule."""
+import math
+
+import pytest
+import torch
+
+import rdt_inputs as RI
+from oracle import rdt_oracle as O
+from tests._helpers import (BF16_TOL, FP32_TOL, MAX_DIVERGENT, divergent_rows, halting_loop, max_rel, rel_l2,
+                            teacher_forced_ids, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+R = pytest.importorskip("recurrent_depth_moe_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    R.load_library()
+
+
+def _recurrent_case(name, n_loops=None, seq=None, batch=None, **wkw):
+    wl = RI.get_workload(name)
+    cfg = wl.cfg
+    B = batch or wl.batch
+    T = seq or wl.seq
+    L = n_loops or wl.n_loops
+    W = RI.block_weights(cfg, wl.seed, **wkw)
+    h0, e = RI.recurrent_inputs(cfg, B, T, wl.seed)
+    return wl, cfg, W, h0, e, B, T, L
+
+
+@pytest.mark.parametrize("name", ["tiny_gqa_fp32", "tiny_mla_fp32", "mid_gqa_fp32"])
+def test_recurrent_fp32_matches_oracle(name):
+    wl, cfg, W, h0, e, B, T, L = _recurrent_case(name, attn_std=0.08, halt_w_std=0.2, lora_scale_std=1.0)
+    thr = wl.act_threshold
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    tr = R.Trace.alloc(cfg, L, 0, B * T)
+    h_out, hw, ids = blk.forward(h0.cuda(), e.cuda(), B, T, L, thr, trace=tr)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    o_h, o_hw, o_ids, _ = O.recurrent_forward(cfg, W, h0, e, B, L, thr)
+    assert max_rel(h_out, o_h) <= FP32_TOL
+    assert max_rel(hw, o_hw) <= FP32_TOL
+    assert torch.equal(ids.cpu().long(), o_ids)
+
+
+def test_tiny_gqa_fp32_model_logits():
+    """The usage script's tiny GQA model end to end: logits (2, 16, 1000)."""
+    wl = RI.get_workload("tiny_gqa_fp32")
+    cfg = wl.cfg
+    MW = RI.model_weights(cfg, wl.seed)
+    ids = torch.randint(0, cfg.vocab_size, (wl.batch, wl.seq), generator=torch.Generator().manual_seed(wl.seed))
+    logits, rec = R.model_forward(cfg, to_dev(MW), ids.cuda(), wl.n_loops, wl.act_threshold)
+    o_logits, o_rec, _ = O.model_forward(cfg, MW, ids, wl.n_loops, wl.act_threshold)
+    assert tuple(logits.shape) == (2, 16, 1000)
+    assert max_rel(logits, o_logits) <= FP32_TOL
+    assert max_rel(rec[0], o_rec[0]) <= FP32_TOL
+    assert torch.equal(rec[2].cpu().long(), o_rec[2])
+
+
+def test_tiny_mla_fp32_model_logits():
+    wl = RI.get_workload("tiny_mla_fp32")
+    cfg = wl.cfg
+    MW = RI.model_weights(cfg, wl.seed)
+    ids = torch.randint(0, cfg.vocab_size, (wl.batch, wl.seq), generator=torch.Generator().manual_seed(wl.seed))
+    logits, rec = R.model_forward(cfg, to_dev(MW), ids.cuda(), wl.n_loops, wl.act_threshold)
+    o_logits, o_rec, _ = O.model_forward(cfg, MW, ids, wl.n_loops, wl.act_threshold)
+    assert max_rel(logits, o_logits) <= FP32_TOL
+    assert max_rel(rec[1], o_rec[1]) <= FP32_TOL
+    assert torch.equal(rec[2].cpu().long(), o_rec[2])
+
+
+def _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, o_hw, o_ids, record, thr, L):
+    """bf16 parity: rows whose routing or halting diverged end to end must be oracle
+    near-ties (and few); the rest meet the relative-L2 bound; ids are exact teacher-forced."""
+    div, bad = divergent_rows(ids, hw, o_ids, o_hw, record, thr, cfg.n_experts_per_tok)
+    assert not bad, f"decisions differ away from near-ties: {bad[:5]}"
+    assert div.float().mean() <= MAX_DIVERGENT, f"{int(div.sum())} of {div.numel()} rows diverged"
+    keep = ~div
+    err = rel_l2(h_out.cpu()[keep], o_h[keep])
+    assert err <= BF16_TOL, f"relative L2 {err:.3e} on {int(keep.sum())} rows"
+    n, nbad, skipped = teacher_forced_ids(cfg, W, tr, ids, L)
+    assert n > 0 and nbad == 0, f"{nbad} of {n} teacher-forced id rows differ ({skipped} near-ties skipped)"
+    return keep
+
+
+def _teacher_forced_states(cfg, W, tr, e, B, L, ids, hw):
+    """One loop of the oracle from the kernel's own state entering loop t, against the
+    kernel's state entering loop t + 1 (no compounding across loops).  Rows running in
+    loop t are compared, except where the kernel's route differs from the oracle's at a
+    near-tie (margin < DECISION_MARGIN).  Returns the per-loop relative L2 errors."""
+    from tests._helpers import DECISION_MARGIN, topk_margin
+    hl = halting_loop(hw)
+    errs = []
+    for t in range(L - 1):
+        h_in = tr.h_in[t].cpu()
+        got = tr.h_in[t + 1].cpu().double()
+        h_new, o_ids, biased = _one_loop(cfg, W, h_in, e, B, t)
+        rows = hl >= t
+        diff = (ids[t].cpu().long() != o_ids).any(-1) & rows
+        near = topk_margin(biased, cfg.n_experts_per_tok) < DECISION_MARGIN
+        assert not (diff & ~near).any(), f"loop {t}: routes differ away from near-ties"
+        keep = rows & ~diff
+        errs.append(rel_l2(got[keep], h_new[keep]))
+    return errs
+
+
+def _one_loop(cfg, W, h, e, B, t):
+    """Oracle state update of loop t from state h (Transformer + LoRA + injection).
+    Returns (h_new, expert ids, biased router logits)."""
+    emb = O.loop_embedding(t, cfg.loop_dim, cfg.dim, cfg.loop_theta)
+    hd = h.double()
+    comb = O.rmsnorm(hd + emb + e.double(), W["rec_norm_w"], cfg.norm_eps)
+    T = h.shape[0] // B
+    pos = torch.arange(h.shape[0]) % T
+    trans, _, info = O.transformer_block(cfg, W, comb, B, pos, True)
+    trans = trans + O.lora_delta(cfg, W, trans, t)
+    A = O.lti_A(W["log_A"], W["log_dt"])
+    return A * hd + W["inj_B"].double() * e.double() + trans, info["ids"], info["biased"]
+
+
+@pytest.mark.parametrize("name", ["tiny_mla_bf16", "mid_gqa_bf16"])
+def test_recurrent_bf16_matches_oracle(name):
+    wl, cfg, W, h0, e, B, T, L = _recurrent_case(name, attn_std=0.08, halt_w_std=0.2, lora_scale_std=1.0)
+    thr = wl.act_threshold
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    tr = R.Trace.alloc(cfg, L, 0, B * T)
+    h_out, hw, ids = blk.forward(h0.cuda(), e.cuda(), B, T, L, thr, trace=tr)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    rec = []
+    o_h, o_hw, o_ids, _ = O.recurrent_forward(cfg, W, h0, e, B, L, thr, record=rec)
+    _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, o_hw, o_ids, rec, thr, L)
+    errs = _teacher_forced_states(cfg, W, tr, e, B, L, ids, hw)
+    assert max(errs) <= BF16_TOL, f"per-loop teacher-forced relative L2 {errs}"
+
+
+def test_tiny_mla_bf16_model_logits():
+    wl = RI.get_workload("tiny_mla_bf16")
+    cfg = wl.cfg
+    MW = RI.model_weights(cfg, wl.seed)
+    ids = torch.randint(0, cfg.vocab_size, (wl.batch, wl.seq), generator=torch.Generator().manual_seed(wl.seed))
+    logits, rec = R.model_forward(cfg, to_dev(MW), ids.cuda(), wl.n_loops, wl.act_threshold)
+    o_logits, o_rec, _ = O.model_forward(cfg, MW, ids, wl.n_loops, wl.act_threshold)
+    keep = halting_loop(rec[1]) == halting_loop(o_rec[1])
+    assert (~keep).float().mean() <= 0.01
+    assert rel_l2(rec[0].cpu()[keep], o_rec[0][keep]) <= BF16_TOL
+    lg = logits.reshape(-1, cfg.vocab_size).cpu()[keep]
+    assert rel_l2(lg, o_logits.reshape(-1, cfg.vocab_size)[keep]) <= BF16_TOL
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_lti_closed_form_on_gpu(dtype):
+    """Transformer term off: h_L = a^L h0 + b e (1 - a^L)/(1 - a) (README mirror, 동적 시스템 관점)."""
+    wl = RI.get_workload("mid_gqa_fp32")
+    cfg = wl.cfg.replace(dtype=dtype)
+    W = RI.block_weights(cfg, 3)
+    h0, e = RI.recurrent_inputs(cfg, 1, 40, 3)
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    L = 9
+    h, hw, ids = blk.forward(h0.cuda(), e.cuda(), 1, 40, L, 0.0, flags=R.RDT_FLAG_TRANSFORMER_OFF)
+    a = torch.exp(-torch.exp(W["log_A"].double()))
+    closed = a ** L * h0.double() + W["inj_B"].double() * e.double() * (1 - a ** L) / (1 - a)
+    assert max_rel(h, closed) <= 1e-5
+    assert (ids.cpu() == -1).all() and torch.equal(hw.cpu()[-1], torch.ones(40))
+
+
+@pytest.mark.parametrize("name", ["mid_gqa_fp32", "mid_gqa_bf16"])
+def test_causality_bit_exact_on_gpu(name):
+    """Perturbing later positions leaves earlier rows bit-identical (fixed reduction order,
+    no split across rows)."""
+    wl, cfg, W, h0, e, B, T, L = _recurrent_case(name, attn_std=0.08, halt_w_std=0.2)
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    out1 = [t.clone() for t in blk.forward(h0.cuda(), e.cuda(), B, T, L, wl.act_threshold)]
+    h0b, eb = h0.clone(), e.clone()
+    cut = 150
+    for b in range(B):
+        h0b[b * T + cut:(b + 1) * T] += 0.5
+        eb[b * T + cut:(b + 1) * T] = (eb[b * T + cut:(b + 1) * T].float() * -1.0).to(eb.dtype)
+    out2 = blk.forward(h0b.cuda(), eb.cuda(), B, T, L, wl.act_threshold)
+    for b in range(B):
+        sl = slice(b * T, b * T + cut)
+        assert torch.equal(out1[0][sl], out2[0][sl])
+        assert torch.equal(out1[1][:, sl], out2[1][:, sl])
+        assert torch.equal(out1[2][:, sl], out2[2][:, sl])
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_decode_step_matches_oracle_and_prefill(dtype):
+    """Prefill T tokens filling per-loop caches, then one decode step at position T:
+    equals the oracle decode step, and the prefill of T + 1 tokens."""
+    wl = RI.get_workload("mid_gqa_fp32")
+    cfg = wl.cfg.replace(dtype=dtype)
+    W = RI.block_weights(cfg, 7, attn_std=0.08, halt_w_std=0.2)
+    B, T, L, thr = 3, 37, 3, 0.99
+    h0, e = RI.recurrent_inputs(cfg, B, T + 1, 7)
+    keep = torch.tensor([b * (T + 1) + i for b in range(B) for i in range(T)])
+    last = torch.tensor([b * (T + 1) + T for b in range(B)])
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    t_max = 64
+    k = torch.zeros(L, B, cfg.n_kv_heads, t_max, cfg.head_dim, dtype=cfg.torch_dtype, device="cuda")
+    cache = R.KVCache(k, torch.zeros_like(k))
+    blk.forward(h0[keep].cuda(), e[keep].cuda(), B, T, L, thr, cache=cache)
+    clen = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    d_h, d_hw, d_ids = blk.decode_step(h0[last].cuda(), e[last].cuda(), clen, cache, L, thr)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    full = O.recurrent_forward(cfg, W, h0, e, B, L, thr)
+    if dtype == "fp32":
+        assert max_rel(d_h, full[0][last]) <= FP32_TOL
+        assert torch.equal(d_ids.cpu().long(), full[2][:, last])
+    else:
+        assert rel_l2(d_h, full[0][last]) <= BF16_TOL
+    # GPU prefill of T + 1 tokens gives the same last rows as GPU prefill + decode
+    p_h, p_hw, p_ids = blk.forward(h0.cuda(), e.cuda(), B, T + 1, L, thr)
+    tol = 1e-5 if dtype == "fp32" else 1e-2
+    assert rel_l2(d_h, p_h[last.cuda()]) <= tol
+
+
+def test_invalid_arguments_return_errors():
+    wl = RI.get_workload("tiny_gqa_fp32")
+    cfg = wl.cfg
+    W = to_dev(RI.block_weights(cfg, 0))
+    blk = R.RecurrentBlock(cfg, W)
+    h0, e = RI.recurrent_inputs(cfg, 1, 8, 0)
+    h0, e = h0.cuda(), e.cuda()
+    with pytest.raises(R.RdtError) as ei:
+        blk.forward(h0, e, 1, 8, 0, 0.0)                 # n_loops = 0
+    assert ei.value.code == 1
+    with pytest.raises(R.RdtError) as ei:
+        blk.forward(h0, e, 1, 8, 2, float("nan"))        # NaN threshold
+    assert ei.value.code == 1
+    small = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(R.RdtError) as ei:
+        blk.forward(h0, e, 1, 8, 2, 0.0, workspace=small)
+    assert ei.value.code == 3
+    bad = dict(W)
+    bad.pop("w_router")
+    with pytest.raises(R.RdtError) as ei:
+        R.RecurrentBlock(cfg, bad).forward(h0, e, 1, 8, 2, 0.0)
+    assert ei.value.code == 1
