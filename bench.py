@@ -1,0 +1,331 @@
+"""Benchmark of the looped Recurrent Block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one full recurrent-block forward (all loops, every kernel of the path) over
+one batch of the 1B-shaped prefill workload (dim 2048, 16 heads GQA with 4 kv heads,
+64 routed + 1 shared SwiGLU experts, top-4, expert_dim 2048, lora_rank 16, 16 loops,
+batch 4 x seq 4096, bf16).  Weights and inputs are seeded synthetic draws.
+
+Multi-GPU (torchrun, one process per GPU): each rank runs an independent replica on
+its own batch (sequences shard with no exchange); the time is the max over ranks.
+
+Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle instead (on
+bounded samples of the same workload, host cores only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import rdt_inputs as RI  # noqa: E402
+
+METRIC = "recurrent-block token·loops/s prefill; decode tokens/s; % roofline, 1×B200"
+UNIT = "token·loops/s"
+WORKLOAD = "rdt1b_prefill"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def workload_desc(wl):
+    c = wl.cfg
+    return (f"{wl.name}: 1B-shaped recurrent block prefill, dim {c.dim}, {c.n_heads} heads GQA ({c.n_kv_heads} kv), "
+            f"{c.n_experts} routed + {c.n_shared_experts} shared SwiGLU experts top-{c.n_experts_per_tok}, "
+            f"expert_dim {c.expert_dim}, lora_rank {c.lora_rank}, {wl.n_loops} loops, batch {wl.batch} x seq {wl.seq}, "
+            f"{c.dtype}, ACT {wl.act_threshold} (halting bias {wl.halt_b})")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.idx), "-lms", "200"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def expert_up_flops(wl, n_running: int) -> float:
+    c = wl.cfg
+    rows = n_running * (c.n_experts_per_tok + c.n_shared_experts)
+    return 2.0 * rows * c.dim * 2 * c.expert_dim
+
+
+# ------------------------------------------------------------------------------------------
+# CPU oracle sample (reference arm and cpu_baseline)
+# ------------------------------------------------------------------------------------------
+
+def oracle_sample(wl, W_cpu, h0, e, positions: int, loops: int):
+    """Time the CPU oracle on sequence 0, positions [0, positions), `loops` loops.
+    Causal prefix slices are exact (attention is causal, routing per token)."""
+    from oracle import rdt_oracle as O
+    t0 = time.perf_counter()
+    O.recurrent_forward(wl.cfg, W_cpu, h0[:positions], e[:positions], 1, loops, wl.act_threshold)
+    dt = time.perf_counter() - t0
+    return positions * loops / dt, dt
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    torch.manual_seed(0)
+    W = RI.block_weights(wl.cfg, wl.seed, device="cpu", halt_b=wl.halt_b)
+    h0, e = RI.recurrent_inputs(wl.cfg, 1, 64, wl.seed)
+    pos, loops = 32, 4
+    for _ in range(args.warmup):
+        oracle_sample(wl, W, h0, e, pos, 1)
+    rates, total = [], 0.0
+    for _ in range(args.steps):
+        r, dt = oracle_sample(wl, W, h0, e, pos, loops)
+        rates.append(r)
+        total += dt
+    value = args.steps * pos * loops / total
+    cores = torch.get_num_threads()
+    sample = f"sequence 0, positions 0-{pos - 1}, loops 0-{loops - 1} of {wl.name} (fp64 oracle, per step)"
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": workload_desc(wl), "batch": wl.batch, "seq_len": wl.seq, "n_loops": wl.n_loops},
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------
+
+def run_ours(args, wl, rank, world, local_rank):
+    import recurrent_depth_moe_b200 as R
+    from recurrent_depth_moe_b200 import _native as NAT
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = wl.cfg
+    B, T, L = wl.batch, wl.seq, wl.n_loops
+    N = B * T
+    # weights: identical replica on every rank; inputs: a different batch per rank
+    W = RI.block_weights(cfg, wl.seed, device=dev, halt_b=wl.halt_b)
+    h0, e = RI.recurrent_inputs(cfg, B, T, wl.seed + 101 * rank, device=dev)
+    blk = R.RecurrentBlock(cfg, W)
+    ws = blk.workspace(B, T, T)
+    out = (torch.empty(N, cfg.dim, dtype=torch.float32, device=dev),
+           torch.empty(L, N, dtype=torch.float32, device=dev),
+           torch.empty(L, N, cfg.n_experts_per_tok, dtype=torch.int32, device=dev))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        blk.forward(h0, e, B, T, L, wl.act_threshold, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0, "device status word set during warm-up"
+
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local_rank
+    clocks = ClockSampler(gpu_index)
+    clocks.start()
+    time.sleep(0.3)
+    NAT.profile_start()
+    n0 = NAT.launch_count()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    launches = NAT.launch_count() - n0
+    prof = NAT.profile_stop()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1) / args.steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # executed token-loops of one step (positions that halt early run fewer loops)
+    hw = out[1]
+    last = ((hw > 0).to(torch.int64) * torch.arange(L, device=dev)[:, None]).max(dim=0).values
+    executed = float((last + 1).sum().item())
+    tl = torch.tensor([executed], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(tl, op=torch.distributed.ReduceOp.SUM)
+    value = float(tl.item()) / (ms_max / 1e3)
+
+    # end to end through the public API: pinned host inputs -> device -> forward -> host outputs
+    h0_h = h0.cpu().pin_memory()
+    e_h = e.cpu().pin_memory()
+    h0_d, e_d = torch.empty_like(h0), torch.empty_like(e)
+    outs_h = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in out]
+    h2d = h0_h.numel() * h0_h.element_size() + e_h.numel() * e_h.element_size()
+    d2h = sum(o.numel() * o.element_size() for o in out)
+
+    def e2e_step():
+        h0_d.copy_(h0_h, non_blocking=True)
+        e_d.copy_(e_h, non_blocking=True)
+        blk.forward(h0_d, e_d, B, T, L, wl.act_threshold, out=out, workspace=ws)
+        for oh, od in zip(outs_h, out):
+            oh.copy_(od, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = float(tl.item()) / (float(te.item()) / 1e3)
+
+    if rank != 0:
+        return
+    pk, pk_kind = peaks()
+    up = prof.get("expert_up_swiglu", (0, 0.0))
+    n_running = N  # per loop; all rows run when nothing halts early
+    achieved_tflops = None
+    if up[0]:
+        avg_ms = up[1] / up[0]
+        # rows actually routed per launch: executed token-loops / loops = mean running rows
+        mean_running = executed / L
+        achieved_tflops = expert_up_flops(wl, mean_running) / (avg_ms / 1e3) / 1e12
+    peak_t = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    roofline = {"bound": "tensor", "kernel": "expert_up_swiglu (tcgen05 grouped GEMM, SwiGLU epilogue)",
+                "achieved": achieved_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                "frac": (achieved_tflops / peak_t) if achieved_tflops else None,
+                "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)",
+                "traffic": None,
+                "flops_per_launch": expert_up_flops(wl, executed / L)}
+    breakdown = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps} for k, v in sorted(prof.items())}
+    res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded N(0,0.02) weights, unit-RMS h0/e rows)",
+           "config": {"workload": workload_desc(wl), "batch": B * world, "seq_len": T, "n_loops": L,
+                      "parallelism": f"replicas x{world} (sequence-sharded, no collective)",
+                      "l2": "inputs larger than L2 (1.65 GB of expert weights + 0.5 GB activations per loop)"},
+           "executed_token_loops_per_step": executed * world,
+           "roofline": roofline, "gpu_launches": launches,
+           "kernel_ms_per_step": breakdown,
+           "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+           "clocks": clk}
+    if world == 1 and not args.no_cpu_baseline:
+        W_cpu = {k: v.cpu() for k, v in W.items()}
+        h0_c, e_c = h0[:64].cpu(), e[:64].cpu()
+        pos, loops = 64, 8
+        rate, dt = oracle_sample(wl, W_cpu, h0_c, e_c, pos, loops)
+        res["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+                               "sample": f"sequence 0, positions 0-{pos - 1}, loops 0-{loops - 1} "
+                                         f"(fp64 oracle, {dt:.1f} s)"}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        log("warm-up raised to 3 steps")
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = RI.get_workload(WORKLOAD)
+    if args.impl == "reference":
+        run_reference(args, wl, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    from recurrent_depth_moe_b200 import build as BLD
+    if rank == 0:
+        BLD.build()
+    if world > 1:
+        torch.distributed.barrier()
+    try:
+        run_ours(args, wl, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -202,6 +202,26 @@ RDT_API const char* rdt_status_string(rdt_status s);
 /* Library build identifier (kernel set and target), static string. */
 RDT_API const char* rdt_version(void);
 
+/* ---- measurement support (benchmarks; no effect on results) ---------------- */
+
+/* Number of kernels this library has enqueued since it was loaded (host counter). */
+RDT_API unsigned long long rdt_launch_count(void);
+
+/* Per-kernel-class device time: while profiling is on, every library call records a
+ * CUDA event pair on its stream around each kernel class it launches. */
+typedef struct {
+  char name[32];      /* kernel class, e.g. "expert_up_swiglu"          */
+  int launches;       /* timed launches of that class                    */
+  double total_ms;    /* summed event-to-event device time               */
+} rdt_kernel_time;
+
+/* Start (or restart) collection.  Creates the event pool on first use. */
+RDT_API rdt_status rdt_profile_start(void);
+
+/* Stop collection, wait for the recorded events and write up to max_entries
+ * per-class totals to out.  Returns the number written, or -1 on a CUDA error. */
+RDT_API int rdt_profile_stop(rdt_kernel_time* out, int max_entries);
+
 #ifdef __cplusplus
 }
 #endif

@@ -122,7 +122,7 @@ WORKLOADS = {
     "rdt1b_prefill": Workload("rdt1b_prefill", RDTConfig(
         dim=2048, n_heads=16, n_kv_heads=4, max_seq_len=4096, max_loop_iters=16,
         n_experts=64, n_shared_experts=1, n_experts_per_tok=4, expert_dim=2048, lora_rank=16,
-        dtype="bf16"), batch=4, seq=4096, n_loops=16, seed=2, act_threshold=0.99, halt_b=-6.0,
+        dtype="bf16"), batch=4, seq=4096, n_loops=16, seed=2, act_threshold=0.99, halt_b=-30.0,
         device_weights=True),
     # 3B-shaped KV-cached decode (mythos_3b: dim 3072, 64 experts, expert_dim 4096, 16 loops).
     "rdt3b_decode": Workload("rdt3b_decode", RDTConfig(

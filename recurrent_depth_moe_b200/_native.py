@@ -50,8 +50,13 @@ class rdt_trace(ctypes.Structure):
                 ("biased_logits", c_void_p), ("p", c_void_p)]
 
 
+class rdt_kernel_time(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", c_int), ("total_ms", ctypes.c_double)]
+
+
 EXPORTS = ("rdt_workspace_size", "rdt_recurrent_forward", "rdt_recurrent_decode_step", "rdt_block_forward",
-           "rdt_embed", "rdt_head", "rdt_read_device_status", "rdt_status_string", "rdt_version")
+           "rdt_embed", "rdt_head", "rdt_read_device_status", "rdt_status_string", "rdt_version",
+           "rdt_launch_count", "rdt_profile_start", "rdt_profile_stop")
 
 _lib = None
 
@@ -87,6 +92,12 @@ def load(path: str = LIB_PATH):
     lib.rdt_status_string.restype = c_char_p
     lib.rdt_version.argtypes = []
     lib.rdt_version.restype = c_char_p
+    lib.rdt_launch_count.argtypes = []
+    lib.rdt_launch_count.restype = ctypes.c_ulonglong
+    lib.rdt_profile_start.argtypes = []
+    lib.rdt_profile_start.restype = c_int
+    lib.rdt_profile_stop.argtypes = [POINTER(rdt_kernel_time), c_int]
+    lib.rdt_profile_stop.restype = c_int
     _lib = lib
     return lib
 
@@ -94,3 +105,20 @@ def load(path: str = LIB_PATH):
 def check(fn: str, code: int):
     if code != RDT_OK:
         raise RdtError(fn, code)
+
+
+def launch_count() -> int:
+    return int(load().rdt_launch_count())
+
+
+def profile_start():
+    check("rdt_profile_start", load().rdt_profile_start())
+
+
+def profile_stop() -> dict:
+    """{kernel class: (launches, total_ms)} recorded since profile_start()."""
+    buf = (rdt_kernel_time * 32)()
+    n = load().rdt_profile_stop(buf, 32)
+    if n < 0:
+        raise RdtError("rdt_profile_stop", RDT_ERR_CUDA)
+    return {buf[i].name.decode(): (buf[i].launches, buf[i].total_ms) for i in range(n)}

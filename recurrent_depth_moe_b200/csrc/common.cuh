@@ -8,6 +8,9 @@ namespace rdt {
 
 typedef __nv_bfloat16 bf16;
 
+// Host-side count of kernels this library enqueued (every launch site calls it).
+void note_launch();
+
 // ------------------------------------------------------------------------------------------
 // storage conversions (model dtype = float or bf16)
 // ------------------------------------------------------------------------------------------

@@ -76,8 +76,8 @@ int launch_attention_simt(int dtype, const AttnParams& p, cudaStream_t s) {
   long long warps = (long long)p.B * p.T * p.H;
   unsigned blocks = (unsigned)((warps + 7) / 8);
   if (blocks == 0) return 0;
-  if (dtype == 0) k_attn_simt<float><<<blocks, 256, 0, s>>>(p);
-  else k_attn_simt<bf16><<<blocks, 256, 0, s>>>(p);
+  if (dtype == 0) { k_attn_simt<float><<<blocks, 256, 0, s>>>(p); note_launch(); }
+  else { k_attn_simt<bf16><<<blocks, 256, 0, s>>>(p); note_launch(); }
   return 0;
 }
 

@@ -130,12 +130,12 @@ int launch_gemm_simt(int dtype, int epi, const GemmParams& p, cudaStream_t s) {
   if (grid.x == 0 || grid.y == 0) return 0;
 #define RDT_SIMT_CASE(TA, TO)                                                              \
   switch (epi) {                                                                           \
-    case EPI_STORE_F32: k_gemm_simt<TA, float, EPI_STORE_F32><<<grid, 256, 0, s>>>(p); break; \
-    case EPI_STORE_T: k_gemm_simt<TA, TO, EPI_STORE_T><<<grid, 256, 0, s>>>(p); break;        \
-    case EPI_RESID_F32: k_gemm_simt<TA, float, EPI_RESID_F32><<<grid, 256, 0, s>>>(p); break; \
-    case EPI_ROPE_T: k_gemm_simt<TA, TO, EPI_ROPE_T><<<grid, 256, 0, s>>>(p); break;          \
-    case EPI_SWIGLU_T: k_gemm_simt<TA, TO, EPI_SWIGLU_T><<<grid, 256, 0, s>>>(p); break;      \
-    case EPI_GATE_F32: k_gemm_simt<TA, float, EPI_GATE_F32><<<grid, 256, 0, s>>>(p); break;   \
+    case EPI_STORE_F32: { k_gemm_simt<TA, float, EPI_STORE_F32><<<grid, 256, 0, s>>>(p); note_launch(); } break; \
+    case EPI_STORE_T: { k_gemm_simt<TA, TO, EPI_STORE_T><<<grid, 256, 0, s>>>(p); note_launch(); } break;        \
+    case EPI_RESID_F32: { k_gemm_simt<TA, float, EPI_RESID_F32><<<grid, 256, 0, s>>>(p); note_launch(); } break; \
+    case EPI_ROPE_T: { k_gemm_simt<TA, TO, EPI_ROPE_T><<<grid, 256, 0, s>>>(p); note_launch(); } break;          \
+    case EPI_SWIGLU_T: { k_gemm_simt<TA, TO, EPI_SWIGLU_T><<<grid, 256, 0, s>>>(p); note_launch(); } break;      \
+    case EPI_GATE_F32: { k_gemm_simt<TA, float, EPI_GATE_F32><<<grid, 256, 0, s>>>(p); note_launch(); } break;   \
     default: return -1;                                                                    \
   }
   if (dtype == 0) { RDT_SIMT_CASE(float, float) } else { RDT_SIMT_CASE(bf16, bf16) }

@@ -448,7 +448,7 @@ int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
         return -1;                                                                                  \
       attr = true;                                                                                  \
     }                                                                                               \
-    tc::k_gemm_tc<E><<<grid, 192, tc::SMEM_BYTES, s>>>(mA, mB, a);                                  \
+    { tc::k_gemm_tc<E><<<grid, 192, tc::SMEM_BYTES, s>>>(mA, mB, a); note_launch(); }                                  \
     break;                                                                                          \
   }
   switch (epi) {

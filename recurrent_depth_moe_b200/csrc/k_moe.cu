@@ -178,17 +178,17 @@ __global__ void __launch_bounds__(128) k_route_scatter(RouteParams p) {
 }
 
 void launch_router_topk(const RouteParams& p, cudaStream_t s) {
-  k_router_topk<<<(p.N + 7) / 8, 256, 0, s>>>(p);
+  { k_router_topk<<<(p.N + 7) / 8, 256, 0, s>>>(p); note_launch(); }
 }
 void launch_route_scan(const RouteParams& p, cudaStream_t s) {
   int nseg = p.E + p.S;
   int threads = 32;
   while (threads < nseg) threads <<= 1;
-  k_route_scan<<<1, threads, 0, s>>>(p);
+  { k_route_scan<<<1, threads, 0, s>>>(p); note_launch(); }
 }
 void launch_route_scatter(int dtype, const RouteParams& p, cudaStream_t s) {
-  if (dtype == 0) k_route_scatter<float><<<p.N, 128, 0, s>>>(p);
-  else k_route_scatter<bf16><<<p.N, 128, 0, s>>>(p);
+  if (dtype == 0) { k_route_scatter<float><<<p.N, 128, 0, s>>>(p); note_launch(); }
+  else { k_route_scatter<bf16><<<p.N, 128, 0, s>>>(p); note_launch(); }
 }
 
 }  // namespace rdt

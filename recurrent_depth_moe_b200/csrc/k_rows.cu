@@ -332,85 +332,85 @@ __global__ void k_trace_rows(const T* __restrict__ src, int W, int row0, const f
 static inline int nthreads_for(int D) { return D >= 2048 ? 256 : 128; }
 
 void launch_lti_A(const float* log_A, const float* log_dt, float* A, int D, cudaStream_t s) {
-  k_lti_A<<<(D + 255) / 256, 256, 0, s>>>(log_A, log_dt, A, D);
+  { k_lti_A<<<(D + 255) / 256, 256, 0, s>>>(log_A, log_dt, A, D); note_launch(); }
 }
 void launch_loop_emb(float* emb, int loop_dim, int t, float theta, cudaStream_t s) {
-  if (loop_dim >= 2) k_loop_emb<<<1, 128, 0, s>>>(emb, loop_dim, t, theta);
+  if (loop_dim >= 2) { k_loop_emb<<<1, 128, 0, s>>>(emb, loop_dim, t, theta); note_launch(); }
 }
 void launch_rope_table(float2* tab, int n_pos, int dim, float theta, cudaStream_t s) {
   long long n = (long long)n_pos * (dim / 2);
-  if (n > 0) k_rope_table<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(tab, n_pos, dim, theta);
+  if (n > 0) { k_rope_table<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(tab, n_pos, dim, theta); note_launch(); }
 }
 void launch_positions(int* pos, int N, int seq, int start_pos, cudaStream_t s) {
-  k_positions<<<(N + 255) / 256, 256, 0, s>>>(pos, N, seq, start_pos);
+  { k_positions<<<(N + 255) / 256, 256, 0, s>>>(pos, N, seq, start_pos); note_launch(); }
 }
 void launch_positions_decode(int* pos, const int* cache_len, int B, int t_max, DevStatus* st, cudaStream_t s) {
-  k_positions_decode<<<(B + 255) / 256, 256, 0, s>>>(pos, cache_len, B, t_max, st);
+  { k_positions_decode<<<(B + 255) / 256, 256, 0, s>>>(pos, cache_len, B, t_max, st); note_launch(); }
 }
 void launch_loop_prologue(int dtype, const float* h, const void* e, const float* emb, int loop_dim,
                           const float* w_rec, const float* w_attn, float* combined, void* a,
                           int N, int D, float eps, cudaStream_t s) {
   size_t smem = (size_t)D * sizeof(float);
   if (dtype == 0)
-    k_loop_prologue<float><<<N, nthreads_for(D), smem, s>>>(h, (const float*)e, emb, loop_dim, w_rec, w_attn,
-                                                           combined, (float*)a, D, eps);
+    { k_loop_prologue<float><<<N, nthreads_for(D), smem, s>>>(h, (const float*)e, emb, loop_dim, w_rec, w_attn,
+                                                           combined, (float*)a, D, eps); note_launch(); }
   else
-    k_loop_prologue<bf16><<<N, nthreads_for(D), smem, s>>>(h, (const bf16*)e, emb, loop_dim, w_rec, w_attn,
-                                                          combined, (bf16*)a, D, eps);
+    { k_loop_prologue<bf16><<<N, nthreads_for(D), smem, s>>>(h, (const bf16*)e, emb, loop_dim, w_rec, w_attn,
+                                                          combined, (bf16*)a, D, eps); note_launch(); }
 }
 void launch_rmsnorm(int in_f32, int dtype, const void* x, long long in_ld, const float* w, void* out,
                     long long out_ld, int rows, int D, float eps, cudaStream_t s) {
   size_t smem = (size_t)D * sizeof(float);
   int nt = nthreads_for(D);
   if (in_f32) {
-    if (dtype == 0) k_rmsnorm<float, float><<<rows, nt, smem, s>>>((const float*)x, in_ld, w, (float*)out, out_ld, D, eps);
-    else k_rmsnorm<float, bf16><<<rows, nt, smem, s>>>((const float*)x, in_ld, w, (bf16*)out, out_ld, D, eps);
+    if (dtype == 0) { k_rmsnorm<float, float><<<rows, nt, smem, s>>>((const float*)x, in_ld, w, (float*)out, out_ld, D, eps); note_launch(); }
+    else { k_rmsnorm<float, bf16><<<rows, nt, smem, s>>>((const float*)x, in_ld, w, (bf16*)out, out_ld, D, eps); note_launch(); }
   } else {
-    if (dtype == 0) k_rmsnorm<float, float><<<rows, nt, smem, s>>>((const float*)x, in_ld, w, (float*)out, out_ld, D, eps);
-    else k_rmsnorm<bf16, bf16><<<rows, nt, smem, s>>>((const bf16*)x, in_ld, w, (bf16*)out, out_ld, D, eps);
+    if (dtype == 0) { k_rmsnorm<float, float><<<rows, nt, smem, s>>>((const float*)x, in_ld, w, (float*)out, out_ld, D, eps); note_launch(); }
+    else { k_rmsnorm<bf16, bf16><<<rows, nt, smem, s>>>((const bf16*)x, in_ld, w, (bf16*)out, out_ld, D, eps); note_launch(); }
   }
 }
 void launch_mla_kv_prep(int dtype, const float* kv_raw, int kvr, int dr, const float* kv_norm_w, float eps,
                         const int* pos, const float2* rope_tab, void* ckv, void* krope, int N, cudaStream_t s) {
   if (dtype == 0)
-    k_mla_kv_prep<float><<<N, 64, 0, s>>>(kv_raw, kvr, dr, kv_norm_w, eps, pos, rope_tab, (float*)ckv, (float*)krope);
+    { k_mla_kv_prep<float><<<N, 64, 0, s>>>(kv_raw, kvr, dr, kv_norm_w, eps, pos, rope_tab, (float*)ckv, (float*)krope); note_launch(); }
   else
-    k_mla_kv_prep<bf16><<<N, 64, 0, s>>>(kv_raw, kvr, dr, kv_norm_w, eps, pos, rope_tab, (bf16*)ckv, (bf16*)krope);
+    { k_mla_kv_prep<bf16><<<N, 64, 0, s>>>(kv_raw, kvr, dr, kv_norm_w, eps, pos, rope_tab, (bf16*)ckv, (bf16*)krope); note_launch(); }
 }
 void launch_kv_to_cache(int dtype, const void* qkv, long long ld, int k_col, int v_col, int Hkv, int hd,
                         const int* pos, int N, int seq, int t_max, void* kc, void* vc, DevStatus* st,
                         cudaStream_t s) {
   if (dtype == 0)
-    k_kv_to_cache<float><<<N, 128, 0, s>>>((const float*)qkv, ld, k_col, v_col, Hkv, hd, pos, seq, t_max,
-                                           (float*)kc, (float*)vc, st);
+    { k_kv_to_cache<float><<<N, 128, 0, s>>>((const float*)qkv, ld, k_col, v_col, Hkv, hd, pos, seq, t_max,
+                                           (float*)kc, (float*)vc, st); note_launch(); }
   else
-    k_kv_to_cache<bf16><<<N, 128, 0, s>>>((const bf16*)qkv, ld, k_col, v_col, Hkv, hd, pos, seq, t_max,
-                                          (bf16*)kc, (bf16*)vc, st);
+    { k_kv_to_cache<bf16><<<N, 128, 0, s>>>((const bf16*)qkv, ld, k_col, v_col, Hkv, hd, pos, seq, t_max,
+                                          (bf16*)kc, (bf16*)vc, st); note_launch(); }
 }
 void launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s) {
   size_t smem = (size_t)(p.D + 64) * sizeof(float);
   int nt = nthreads_for(p.D);
-  if (dtype == 0) k_combine_inject_act<float><<<n_rows, nt, smem, s>>>(p);
-  else k_combine_inject_act<bf16><<<n_rows, nt, smem, s>>>(p);
+  if (dtype == 0) { k_combine_inject_act<float><<<n_rows, nt, smem, s>>>(p); note_launch(); }
+  else { k_combine_inject_act<bf16><<<n_rows, nt, smem, s>>>(p); note_launch(); }
 }
 void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* n_run, cudaStream_t s) {
-  k_compact<<<1, 1024, 0, s>>>(halted, N, run_list, run_idx, n_run);
+  { k_compact<<<1, 1024, 0, s>>>(halted, N, run_list, run_idx, n_run); note_launch(); }
 }
 void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s) {
-  k_iota<<<(N + 255) / 256, 256, 0, s>>>(run_list, run_idx, n_run, N);
+  { k_iota<<<(N + 255) / 256, 256, 0, s>>>(run_list, run_idx, n_run, N); note_launch(); }
 }
 void launch_embed(int dtype, const void* table, int vocab, const int* ids, int n, int D, float* out,
                   DevStatus* st, cudaStream_t s) {
-  if (dtype == 0) k_embed<float><<<n, 128, 0, s>>>((const float*)table, vocab, ids, D, out, st);
-  else k_embed<bf16><<<n, 128, 0, s>>>((const bf16*)table, vocab, ids, D, out, st);
+  if (dtype == 0) { k_embed<float><<<n, 128, 0, s>>>((const float*)table, vocab, ids, D, out, st); note_launch(); }
+  else { k_embed<bf16><<<n, 128, 0, s>>>((const bf16*)table, vocab, ids, D, out, st); note_launch(); }
 }
 void launch_trace_rows(int src_is_model_dtype, int dtype, const void* src, int W, int row0, int n,
                        const float* bias, float* dst, cudaStream_t s) {
   if (n <= 0) return;
   if (!src_is_model_dtype || dtype == 0)
-    k_trace_rows<float><<<n, 128, 0, s>>>((const float*)src, W, row0, bias, dst);
+    { k_trace_rows<float><<<n, 128, 0, s>>>((const float*)src, W, row0, bias, dst); note_launch(); }
   else
-    k_trace_rows<bf16><<<n, 128, 0, s>>>((const bf16*)src, W, row0, bias, dst);
+    { k_trace_rows<bf16><<<n, 128, 0, s>>>((const bf16*)src, W, row0, bias, dst); note_launch(); }
 }
 
 }  // namespace rdt

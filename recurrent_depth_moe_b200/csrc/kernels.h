@@ -7,6 +7,20 @@ namespace rdt {
 
 struct DevStatus;
 
+// Kernel classes for event timing (ProfScope records a CUDA event pair around the
+// launches in its scope on the given stream when profiling is on).
+enum ProfClass {
+  PC_PROLOGUE = 0, PC_QKV, PC_ATTN, PC_OPROJ, PC_FFN_NORM, PC_ROUTER_GEMM, PC_ROUTE, PC_EXPERT_UP,
+  PC_EXPERT_DOWN, PC_COMBINE, PC_OTHER, PC_COUNT
+};
+struct ProfScope {
+  ProfScope(int cls, cudaStream_t s);
+  ~ProfScope();
+  int cls_;
+  cudaStream_t s_;
+  void* a_;
+};
+
 // ------------------------------------------------------------------------------------------
 // GEMM: C[M, N] = A[M, K] . B[N, K]^T with A, B K-contiguous (nn.Linear layout for B).
 // Grouped mode: tiles[4 * i] = {group, row0, rows, 0}; B advanced by group * b_group_stride.

@@ -165,7 +165,7 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
     g.C = qkv; g.ldc = W; g.pos = pos; g.rope_tab = tab; g.rope_half = hd / 2; g.n_rope = 2;
     g.rope[0] = RopeDesc{0, H, hd, 0, hd};
     g.rope[1] = RopeDesc{H * hd, Hkv, hd, 0, hd};
-    RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, x.s));
+    { ProfScope ps(PC_QKV, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, x.s)); }
     ap.q = qkv; ap.q_row = W; ap.q_head = hd; ap.dn = hd; ap.dr = 0; ap.dv = hd; ap.G = H / Hkv;
     ap.scale = 1.f / sqrtf((float)hd);
     const bool use_cache = cache && cache->k;
@@ -173,7 +173,7 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
       size_t per_loop = (size_t)cache->batch * Hkv * cache->t_max * hd * es;
       char* kc = (char*)cache->k + per_loop * loop_t;
       char* vc = (char*)cache->v + per_loop * loop_t;
-      launch_kv_to_cache(x.dtype, qkv, W, H * hd, (H + Hkv) * hd, Hkv, hd, pos, N, T, cache->t_max, kc, vc, x.st, x.s);
+      { ProfScope ps(PC_OTHER, x.s); launch_kv_to_cache(x.dtype, qkv, W, H * hd, (H + Hkv) * hd, Hkv, hd, pos, N, T, cache->t_max, kc, vc, x.st, x.s); }
       if (decode || start_pos > 0) {
         long long sj = hd, sg = (long long)cache->t_max * hd, sb = (long long)Hkv * sg;
         ap.k1 = kc; ap.k1_b = sb; ap.k1_j = sj; ap.k1_g = sg;
@@ -225,11 +225,11 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
     ap.scale = 1.f / sqrtf((float)(dn + dr));
   }
   ap.o = attn; ap.o_row = (long long)H * dv; ap.o_head = dv;
-  RDT_TRY(launch_attention(x.dtype, ap, x.s));
+  { ProfScope ps(PC_ATTN, x.s); RDT_TRY(launch_attention(x.dtype, ap, x.s)); }
   GemmParams g = gemm_base(x);
   g.A = attn; g.lda = (long long)H * dv; g.B = w->w_o; g.ldb = (long long)H * dv; g.M = N; g.N = D; g.K = H * dv;
   g.C = x1; g.ldc = D; g.resid = combined; g.ld_resid = D;
-  RDT_TRY(launch_gemm(x.dtype, EPI_RESID_F32, g, x.s));
+  { ProfScope ps(PC_OPROJ, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_RESID_F32, g, x.s)); }
   return RDT_OK;
 }
 
@@ -239,11 +239,11 @@ rdt_status moe_block(Ctx& x, int N, const float* x1) {
   const rdt_weights* w = x.w;
   const int D = c->dim, E = c->n_experts, k = c->top_k, S = c->n_shared_experts, F = c->expert_dim;
   void* f = at<void*>(x.ws, x.L.f);
-  launch_rmsnorm(1, x.dtype, x1, D, w->ffn_norm_w, f, D, N, D, c->norm_eps, x.s);
+  { ProfScope ps(PC_FFN_NORM, x.s); launch_rmsnorm(1, x.dtype, x1, D, w->ffn_norm_w, f, D, N, D, c->norm_eps, x.s); }
   float* logits = at<float*>(x.ws, x.L.logits);
   GemmParams g = gemm_base(x);
   g.A = f; g.lda = D; g.B = w->w_router; g.ldb = D; g.M = N; g.N = E; g.K = D; g.C = logits; g.ldc = E;
-  RDT_TRY(launch_gemm(x.dtype, EPI_STORE_F32, g, x.s));
+  { ProfScope ps(PC_ROUTER_GEMM, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_STORE_F32, g, x.s)); }
   RouteParams rp;
   memset(&rp, 0, sizeof(rp));
   rp.logits = logits; rp.bias = w->router_bias; rp.N = N; rp.E = E; rp.k = k; rp.S = S;
@@ -270,11 +270,14 @@ rdt_status moe_block(Ctx& x, int N, const float* x1) {
   up.impl = dn.impl = (int)iu;
   rp.tile_m = gemm_tile_m(iu);
   if (cudaMemsetAsync(rp.counts, 0, sizeof(int) * std::max(E, 1), x.s) != cudaSuccess) return RDT_ERR_CUDA;
-  launch_router_topk(rp, x.s);
-  launch_route_scan(rp, x.s);
-  launch_route_scatter(x.dtype, rp, x.s);
-  RDT_TRY(launch_gemm(x.dtype, EPI_SWIGLU_T, up, x.s));
-  RDT_TRY(launch_gemm(x.dtype, EPI_GATE_F32, dn, x.s));
+  {
+    ProfScope ps(PC_ROUTE, x.s);
+    launch_router_topk(rp, x.s);
+    launch_route_scan(rp, x.s);
+    launch_route_scatter(x.dtype, rp, x.s);
+  }
+  { ProfScope ps(PC_EXPERT_UP, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_SWIGLU_T, up, x.s)); }
+  { ProfScope ps(PC_EXPERT_DOWN, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_GATE_F32, dn, x.s)); }
   return RDT_OK;
 }
 
@@ -370,9 +373,12 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
     if (trace && trace->h_in)
       launch_trace_rows(0, x.dtype, h, D, trace->row0, trace->n_rows, nullptr,
                         trace->h_in + (size_t)t * trace->n_rows * D, s);
-    launch_loop_emb(emb, c->loop_dim, t, c->loop_theta, s);
-    launch_loop_prologue(x.dtype, h, e, emb, c->loop_dim, w->rec_norm_w, w->attn_norm_w, combined, a, N, D,
-                         c->norm_eps, s);
+    {
+      ProfScope ps(PC_PROLOGUE, s);
+      launch_loop_emb(emb, c->loop_dim, t, c->loop_theta, s);
+      launch_loop_prologue(x.dtype, h, e, emb, c->loop_dim, w->rec_norm_w, w->attn_norm_w, combined, a, N, D,
+                           c->norm_eps, s);
+    }
     if (!transformer_off) {
       if ((st = attention_block(x, B, T, combined, a, x1, cache, t, start_pos, decode)) != RDT_OK) return st;
       if ((st = moe_block(x, N, x1)) != RDT_OK) return st;
@@ -384,13 +390,15 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
                           trace->biased_logits + (size_t)t * trace->n_rows * E, s);
     }
     cp.t = t;
-    launch_combine(x.dtype, cp, N, s);
+    { ProfScope ps(PC_COMBINE, s); launch_combine(x.dtype, cp, N, s); }
     if (trace && trace->p && act_on)
       launch_trace_rows(0, x.dtype, at<float*>(ws, x.L.p_buf), 1, trace->row0, trace->n_rows, nullptr,
                         trace->p + (size_t)t * trace->n_rows, s);
-    if (act_on && t + 1 < n_loops)
+    if (act_on && t + 1 < n_loops) {
+      ProfScope ps(PC_OTHER, s);
       launch_compact(at<int*>(ws, x.L.halted), N, at<int*>(ws, x.L.run_list), at<int*>(ws, x.L.run_idx),
                      at<int*>(ws, x.L.nrun), s);
+    }
   }
   if (cudaGetLastError() != cudaSuccess) return RDT_ERR_CUDA;
   return RDT_OK;
@@ -406,6 +414,8 @@ int launch_gemm_simt(int dtype, int epi, const GemmParams& p, cudaStream_t s);
 int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s);
 bool gemm_tc_supports(const GemmParams& p, int epi);
 int launch_attention_simt(int dtype, const AttnParams& p, cudaStream_t s);
+bool attention_fa_supports(int dtype, const AttnParams& p);
+int launch_attention_fa(const AttnParams& p, cudaStream_t s);
 
 int gemm_tile_m(GemmImpl impl) { return impl == GEMM_TC ? 128 : 64; }
 GemmImpl gemm_pick(int dtype, const GemmParams& p, int epi) {
@@ -417,7 +427,10 @@ int launch_gemm(int dtype, int epi, const GemmParams& p, cudaStream_t s) {
   if (gemm_pick(dtype, p, epi) == GEMM_TC) return launch_gemm_tc(epi, p, s);
   return launch_gemm_simt(dtype, epi, p, s);
 }
-int launch_attention(int dtype, const AttnParams& p, cudaStream_t s) { return launch_attention_simt(dtype, p, s); }
+int launch_attention(int dtype, const AttnParams& p, cudaStream_t s) {
+  if (attention_fa_supports(dtype, p)) return launch_attention_fa(p, s);
+  return launch_attention_simt(dtype, p, s);
+}
 }  // namespace rdt
 
 // ------------------------------------------------------------------------------------------

@@ -9,8 +9,7 @@ import torch
 
 import rdt_inputs as RI
 from oracle import rdt_oracle as O
-from tests._helpers import (BF16_TOL, FP32_TOL, MAX_DIVERGENT, divergent_rows, halting_loop, max_rel, rel_l2,
-                            teacher_forced_ids, to_dev)
+from tests._helpers import (BF16_TOL, FP32_TOL, halting_loop, max_rel, rel_l2, teacher_forced_ids, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -76,18 +75,15 @@ def test_tiny_mla_fp32_model_logits():
     assert torch.equal(rec[2].cpu().long(), o_rec[2])
 
 
-def _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, o_hw, o_ids, record, thr, L):
-    """bf16 parity: rows whose routing or halting diverged end to end must be oracle
-    near-ties (and few); the rest meet the relative-L2 bound; ids are exact teacher-forced."""
-    div, bad = divergent_rows(ids, hw, o_ids, o_hw, record, thr, cfg.n_experts_per_tok)
-    assert not bad, f"decisions differ away from near-ties: {bad[:5]}"
-    assert div.float().mean() <= MAX_DIVERGENT, f"{int(div.sum())} of {div.numel()} rows diverged"
-    keep = ~div
-    err = rel_l2(h_out.cpu()[keep], o_h[keep])
-    assert err <= BF16_TOL, f"relative L2 {err:.3e} on {int(keep.sum())} rows"
+def _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, L):
+    """bf16 parity, end to end: relative L2 over every row; ids exact teacher-forced
+    (the kernel's own router input) wherever the top-k margin is >= 1e-3.  End-to-end
+    routes are not compared: a near-tie flip at one position changes that position's
+    state, hence its keys and values, hence every later position's attention."""
+    err = rel_l2(h_out, o_h)
+    assert err <= BF16_TOL, f"relative L2 {err:.3e}"
     n, nbad, skipped = teacher_forced_ids(cfg, W, tr, ids, L)
     assert n > 0 and nbad == 0, f"{nbad} of {n} teacher-forced id rows differ ({skipped} near-ties skipped)"
-    return keep
 
 
 def _teacher_forced_states(cfg, W, tr, e, B, L, ids, hw):
@@ -125,18 +121,21 @@ def _one_loop(cfg, W, h, e, B, t):
     return A * hd + W["inj_B"].double() * e.double() + trans, info["ids"], info["biased"]
 
 
+STRONG = dict(attn_std=0.08, halt_w_std=0.2, lora_scale_std=1.0)   # peaky attention, visible LoRA and ACT
+
+
+@pytest.mark.parametrize("variant", ["literal", "strong"])
 @pytest.mark.parametrize("name", ["tiny_mla_bf16", "mid_gqa_bf16"])
-def test_recurrent_bf16_matches_oracle(name):
-    wl, cfg, W, h0, e, B, T, L = _recurrent_case(name, attn_std=0.08, halt_w_std=0.2, lora_scale_std=1.0)
+def test_recurrent_bf16_matches_oracle(name, variant):
+    wl, cfg, W, h0, e, B, T, L = _recurrent_case(name, **(STRONG if variant == "strong" else {}))
     thr = wl.act_threshold
     blk = R.RecurrentBlock(cfg, to_dev(W))
     tr = R.Trace.alloc(cfg, L, 0, B * T)
     h_out, hw, ids = blk.forward(h0.cuda(), e.cuda(), B, T, L, thr, trace=tr)
     torch.cuda.synchronize()
     assert blk.read_status() == 0
-    rec = []
-    o_h, o_hw, o_ids, _ = O.recurrent_forward(cfg, W, h0, e, B, L, thr, record=rec)
-    _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, o_hw, o_ids, rec, thr, L)
+    o_h, o_hw, o_ids, _ = O.recurrent_forward(cfg, W, h0, e, B, L, thr)
+    _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, L)
     errs = _teacher_forced_states(cfg, W, tr, e, B, L, ids, hw)
     assert max(errs) <= BF16_TOL, f"per-loop teacher-forced relative L2 {errs}"
 
@@ -148,11 +147,8 @@ def test_tiny_mla_bf16_model_logits():
     ids = torch.randint(0, cfg.vocab_size, (wl.batch, wl.seq), generator=torch.Generator().manual_seed(wl.seed))
     logits, rec = R.model_forward(cfg, to_dev(MW), ids.cuda(), wl.n_loops, wl.act_threshold)
     o_logits, o_rec, _ = O.model_forward(cfg, MW, ids, wl.n_loops, wl.act_threshold)
-    keep = halting_loop(rec[1]) == halting_loop(o_rec[1])
-    assert (~keep).float().mean() <= 0.01
-    assert rel_l2(rec[0].cpu()[keep], o_rec[0][keep]) <= BF16_TOL
-    lg = logits.reshape(-1, cfg.vocab_size).cpu()[keep]
-    assert rel_l2(lg, o_logits.reshape(-1, cfg.vocab_size)[keep]) <= BF16_TOL
+    assert rel_l2(rec[0], o_rec[0]) <= BF16_TOL
+    assert rel_l2(logits, o_logits) <= BF16_TOL
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
