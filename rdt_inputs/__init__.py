@@ -141,6 +141,15 @@ WORKLOADS = {
         dim=512, n_heads=4, n_kv_heads=2, max_seq_len=512, max_loop_iters=2,
         n_experts=8, n_shared_experts=1, n_experts_per_tok=2, expert_dim=256, lora_rank=8,
         dtype="bf16"), batch=2, seq=200, n_loops=3, seed=5, act_threshold=0.99),
+    # Test-only: router widths of the 1B / 10B shapes (fused tensor-core routing), ragged expert segments.
+    "mid_e64_bf16": Workload("mid_e64_bf16", RDTConfig(
+        dim=512, n_heads=4, n_kv_heads=2, max_seq_len=512, max_loop_iters=2,
+        n_experts=64, n_shared_experts=1, n_experts_per_tok=4, expert_dim=128, lora_rank=16,
+        dtype="bf16"), batch=2, seq=200, n_loops=3, seed=6, act_threshold=0.99),
+    "mid_e128_bf16": Workload("mid_e128_bf16", RDTConfig(
+        dim=512, n_heads=4, n_kv_heads=1, max_seq_len=512, max_loop_iters=2,
+        n_experts=128, n_shared_experts=1, n_experts_per_tok=8, expert_dim=128, lora_rank=16,
+        dtype="bf16"), batch=1, seq=300, n_loops=2, seed=7, act_threshold=0.9),
     "mid_gqa_fp32": Workload("mid_gqa_fp32", RDTConfig(
         dim=512, n_heads=4, n_kv_heads=2, max_seq_len=512, max_loop_iters=2,
         n_experts=8, n_shared_experts=1, n_experts_per_tok=2, expert_dim=256, lora_rank=8,

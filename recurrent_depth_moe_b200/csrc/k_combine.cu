@@ -1,0 +1,171 @@
+// S9 as a warp-per-row kernel for row widths that are multiples of 128: the fused
+// combine + depth-wise LoRA + LTI injection + freeze + ACT step of one loop.
+//
+// Lane l holds columns 4l + 128j (j < D/128) of its row in registers, so every global
+// access is a coalesced 16-byte vector and every input is read exactly once:
+//   trans  = x1 + sum_{j < k+S} y[slot_of[i][j]]          (gates already applied)
+//   z_q    = (trans . Wd_q) * scale[min(t, mli-1)]_q       (warp reductions, q < r)
+//   trans += sum_q z_q B_q                                 ("OpenMythos 분석", Recurrent Block)
+//   h_new  = A h + B_inj e + trans                         (LTIInjection, latent reasoning)
+//   rows halted before loop t keep h (frozen)
+//   ACT:  p = sigmoid(h_new . w_halt + b + off); w = remainder if cum + p >= thr or
+//         last loop, else p; cum += p; h_out += w h_new    ("OpenMythos 분석", ACT)
+// The LoRA matrices (2 r D elements) are shared by all rows and stay in L1/L2.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rdt {
+
+template <typename T> struct Vec4;
+template <> struct Vec4<float> {
+  static __device__ __forceinline__ float4 load(const float* p) { return __ldg(reinterpret_cast<const float4*>(p)); }
+};
+template <> struct Vec4<bf16> {
+  static __device__ __forceinline__ float4 load(const bf16* p) {
+    uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&u.x), b = *reinterpret_cast<__nv_bfloat162*>(&u.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+  }
+};
+
+__device__ __forceinline__ float4 f4_add(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+__device__ __forceinline__ float f4_dot(float4 a, float4 b) { return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w; }
+
+template <typename T, int VPL>
+__global__ void __launch_bounds__(256) k_combine_warp(CombineParams p) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (i >= p.N) return;
+  const int D = p.D;
+  const int kS = p.k + p.S;
+  if (!p.block_only && p.halted[i]) {   // frozen row: no update, zero weight, no experts
+    if (lane == 0) p.halt_w_out[(long long)p.t * p.N + i] = 0.f;
+    if (lane < p.k) p.ids_out[((long long)p.t * p.N + i) * p.k + lane] = -1;
+    return;
+  }
+  float4 tr[VPL];
+  const long long rowD = (long long)i * D;
+  if (p.transformer_off) {
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) tr[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else {
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) tr[j] = __ldg(reinterpret_cast<const float4*>(p.x1 + rowD + 4 * lane + 128 * j));
+    for (int s = 0; s < kS; ++s) {
+      const int slot = p.slot_of[(long long)i * kS + s];
+      if (slot < 0 || slot >= p.max_slots) {
+        if (lane == 0) record_status(p.st, ST_BOUNDS, 202, slot);
+        continue;
+      }
+      const float* yr = p.y + (long long)slot * D + 4 * lane;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) tr[j] = f4_add(tr[j], __ldg(reinterpret_cast<const float4*>(yr + 128 * j)));
+    }
+  }
+  if (p.block_only) {
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) *reinterpret_cast<float4*>(p.out + rowD + 4 * lane + 128 * j) = tr[j];
+    return;
+  }
+  if (!p.transformer_off && p.r > 0) {
+    const T* Wd = (const T*)p.lora_down;
+    const T* Bl = (const T*)p.lora_B;
+    const float* sc = p.lora_scale + (long long)min(p.t, p.max_loop_iters - 1) * p.r;
+    __shared__ float zs[8][64];
+    float* z = zs[threadIdx.x >> 5];
+    for (int q = 0; q < p.r; ++q) {
+      float part = 0.f;
+      const T* w = Wd + (long long)q * D + 4 * lane;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) part += f4_dot(tr[j], Vec4<T>::load(w + 128 * j));
+      part = warp_sum(part) * sc[q];
+      if (lane == 0) z[q] = part;
+    }
+    __syncwarp();
+    // every z_q is complete, so the delta can be added to the row in place
+    for (int q = 0; q < p.r; ++q) {
+      const T* b = Bl + (long long)q * D + 4 * lane;
+      const float zq = z[q];
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) {
+        float4 v = Vec4<T>::load(b + 128 * j);
+        tr[j].x += zq * v.x; tr[j].y += zq * v.y; tr[j].z += zq * v.z; tr[j].w += zq * v.w;
+      }
+    }
+  }
+  // h_new = A h + B e + trans (in place in tr)
+  const T* er = (const T*)p.e + rowD + 4 * lane;
+  float zh = 0.f;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int d = 4 * lane + 128 * j;
+    float4 hv = __ldg(reinterpret_cast<const float4*>(p.h + rowD + d));
+    float4 av = __ldg(reinterpret_cast<const float4*>(p.A + d));
+    float4 bv = __ldg(reinterpret_cast<const float4*>(p.inj_B + d));
+    float4 ev = Vec4<T>::load(er + 128 * j);
+    tr[j].x += av.x * hv.x + bv.x * ev.x;
+    tr[j].y += av.y * hv.y + bv.y * ev.y;
+    tr[j].z += av.z * hv.z + bv.z * ev.z;
+    tr[j].w += av.w * hv.w + bv.w * ev.w;
+    if (p.act_on) zh += f4_dot(tr[j], __ldg(reinterpret_cast<const float4*>(p.halt_wv + d)));
+  }
+  const bool last = (p.t == p.n_loops - 1);
+  float w;
+  if (p.act_on) {
+    zh = warp_sum(zh);
+    const float zz = zh + p.halt_b[0] + (p.halt_off ? p.halt_off[i] : 0.f);
+    const float prob = 1.f / (1.f + expf(-zz));
+    const float cum = p.cum[i];
+    const bool stop = (cum + prob >= p.thr) || last;
+    w = stop ? fmaxf(1.f - cum, 0.f) : prob;
+    __syncwarp();
+    if (lane == 0) {
+      p.cum[i] = cum + prob;
+      if (stop) p.halted[i] = 1;
+      if (p.p_out) p.p_out[i] = prob;
+    }
+  } else {
+    w = last ? 1.f : 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int d = 4 * lane + 128 * j;
+    float4* ho = reinterpret_cast<float4*>(p.h_out + rowD + d);
+    if (w != 0.f) {
+      float4 o = *ho;
+      o.x += w * tr[j].x; o.y += w * tr[j].y; o.z += w * tr[j].z; o.w += w * tr[j].w;
+      *ho = o;
+    }
+    *reinterpret_cast<float4*>(p.h_state + rowD + d) = tr[j];
+  }
+  if (lane == 0) p.halt_w_out[(long long)p.t * p.N + i] = w;
+  if (lane < p.k)
+    p.ids_out[((long long)p.t * p.N + i) * p.k + lane] = p.transformer_off ? -1 : p.ids[(long long)i * p.k + lane];
+}
+
+// Returns false when the shape needs the CTA-per-row kernel instead.
+static inline bool al(const void* q, int b) { return ((uintptr_t)q % b) == 0; }
+
+bool launch_combine_warp(int dtype, const CombineParams& p, int n_rows, cudaStream_t s) {
+  if (p.D % 128 || p.r > 64 || p.k > 32) return false;
+  const int ev = dtype == 0 ? 16 : 8;   // bytes of a 4-element vector in the model dtype
+  if (!al(p.x1, 16) || !al(p.y, 16) || !al(p.h, 16) || !al(p.h_state, 16) || !al(p.h_out, 16) || !al(p.A, 16) ||
+      !al(p.inj_B, 16) || !al(p.e, ev) || (p.act_on && !al(p.halt_wv, 16)) || (p.out && !al(p.out, 16)) ||
+      (p.r > 0 && (!al(p.lora_down, ev) || !al(p.lora_B, ev))))
+    return false;
+  const int vpl = p.D / 128;
+  const unsigned blocks = (unsigned)((n_rows + 7) / 8);
+#define RDT_CW(V)                                                                                   \
+  case V:                                                                                           \
+    if (dtype == 0) { k_combine_warp<float, V><<<blocks, 256, 0, s>>>(p); note_launch(); }          \
+    else { k_combine_warp<bf16, V><<<blocks, 256, 0, s>>>(p); note_launch(); }                      \
+    return true;
+  switch (vpl) {
+    RDT_CW(1) RDT_CW(2) RDT_CW(4) RDT_CW(8) RDT_CW(12) RDT_CW(16) RDT_CW(24) RDT_CW(32)
+    default: return false;
+  }
+#undef RDT_CW
+}
+
+}  // namespace rdt

@@ -2,41 +2,49 @@
 // by TMA (no multicast) into 128-byte-swizzled shared memory, persistent CTAs.
 //
 //   C[M, N] = A[M, K] . B[N, K]^T, bf16 operands, fp32 accumulation.
-//   Tile: 128 rows x 256 MMA columns x 64-deep K stages (4 stages, 48 KB each).
+//   Tile: 128 rows x BN MMA columns (BN = 64, 128 or 256) x 64-deep K stages.
 //   Grouped mode (MoE experts): the m-tiles come from a device tile list
 //   {group, row0, rows}; B is the group's weight slab.  SwiGLU: the 256 MMA columns
 //   are 128 gate rows (W1) and the matching 128 up rows (W3) of the expert, so the
 //   epilogue forms silu(gate) * up for 128 output columns in registers.
+//   Router (BN = E): each epilogue thread owns one token's E logits and performs the
+//   softmax, the biased top-k (ties -> lower expert index), the gate renormalisation
+//   and the per-expert histogram ("OpenMythos 분석", MoE) without a second pass.
 //
 // Warp roles (192 threads): warp 0 lane 0 issues TMA loads; warp 1 owns TMEM
 // (alloc / dealloc) and lane 0 issues the MMAs; warps 2..5 are the epilogue, each
 // reading its 32-lane quarter of the accumulator with tcgen05.ld.  The accumulator
-// is double-buffered in TMEM (2 x 256 columns) so the epilogue of one tile overlaps
+// is double-buffered in TMEM (2 x BN columns) so the epilogue of one tile overlaps
 // the MMAs of the next.  Every mbarrier wait is bounded: on timeout the CTA records
 // RDT_ERR_DEVICE_TIMEOUT in the status word and leaves its loops.
 #include "common.cuh"
 #include "kernels.h"
 
 #include <cuda.h>
+#include <algorithm>
 #include <mutex>
 
 namespace rdt {
 namespace tc {
 
-constexpr int BM = 128, BK = 64, BN_MMA = 256, STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;            // 16 KB
-constexpr int B_HALF = 128 * BK * 2;            // 16 KB (one 128-row TMA box)
-constexpr int STAGE_BYTES = A_BYTES + 2 * B_HALF;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
 constexpr long long TIMEOUT_CYCLES = 4000000000LL;   // ~2 s at 2 GHz
-constexpr int TMEM_COLS = 512;
+
+template <int BN> struct Shape {
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;   // power of two >= 32
+  static constexpr int B_BOX = BN > 128 ? 128 : BN;             // rows per TMA box
+};
 
 struct TcArgs {
   GemmParams p;
   int n_n;             // n tiles
   int m_tiles;         // dense: m tiles; grouped: read from *p.n_tiles
   int b_rows_group;    // rows of B per group (grouped)
-  int n_out_tile;      // output columns per tile (128 SwiGLU, 256 otherwise)
+  int n_out_tile;      // output columns per tile
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -94,7 +102,7 @@ __device__ __forceinline__ uint64_t smem_desc(const void* p) {
   return d;
 }
 
-// kind::f16 instruction descriptor: bf16 A/B, fp32 D, both K-major, M = 128, N = 256.
+// kind::f16 instruction descriptor: bf16 A/B, fp32 D, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
@@ -146,7 +154,10 @@ __device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
   }
 }
 
-__device__ __forceinline__ int rope_pair_tc(const GemmParams& p, int c) {
+// RoPE pair index of the first column of a 32-column chunk, or -1 when the chunk is
+// not rotated.  Descriptors are 32-column aligned (checked on the host), so a chunk is
+// either entirely inside one head's rotated range or entirely outside.
+__device__ __forceinline__ int rope_chunk(const GemmParams& p, int c) {
   for (int q = 0; q < p.n_rope; ++q) {
     const RopeDesc& r = p.rope[q];
     int rel = c - r.col0;
@@ -175,12 +186,67 @@ __device__ __forceinline__ TileInfo decode_tile(const TcArgs& a, int t) {
   return ti;
 }
 
-template <int EPI>
+// Router epilogue for one row held by this thread: E logits in TMEM columns [0, E).
+template <int E>
+__device__ __forceinline__ void route_row(const GemmParams& p, uint32_t tbase, bool valid, long long r) {
+  float lg[E];
+#pragma unroll
+  for (int c = 0; c < E; c += 32) {
+    float v[32];
+    tmem_ld32(tbase + c, v);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) lg[c + j] = v[j];
+  }
+  if (!valid) return;
+  float* lrow = (float*)p.C + r * p.ldc;
+#pragma unroll
+  for (int c = 0; c < E; c += 4) *reinterpret_cast<float4*>(lrow + c) = make_float4(lg[c], lg[c + 1], lg[c + 2], lg[c + 3]);
+  if (p.run_idx && p.run_idx[r] < 0) return;      // halted row: logits only
+  float mx = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < E; ++e) mx = fmaxf(mx, lg[e]);
+  float sum = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) sum += __expf(lg[e] - mx);
+  uint32_t taken[E / 32];
+#pragma unroll
+  for (int w = 0; w < E / 32; ++w) taken[w] = 0u;
+  int sel[32];
+  float sc[32];
+  float gsum = 0.f;
+  for (int j = 0; j < p.topk; ++j) {
+    float bv = -INFINITY;
+    int be = -1;
+    float braw = 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float b = lg[e] + p.bias[e];
+      const bool free = !((taken[e >> 5] >> (e & 31)) & 1u);
+      if (free && (be < 0 || b > bv)) { bv = b; be = e; braw = lg[e]; }   // strict >: lower index wins ties
+    }
+    if (be < 0) { record_status(p.st, ST_BOUNDS, 502, j); be = 0; }
+#pragma unroll
+    for (int w = 0; w < E / 32; ++w)
+      if ((be >> 5) == w) taken[w] |= 1u << (be & 31);
+    sel[j] = be;
+    sc[j] = __expf(braw - mx) / sum;
+    gsum += sc[j];
+  }
+  for (int j = 0; j < p.topk; ++j) {
+    const long long o = r * p.topk + j;
+    p.ids[o] = sel[j];
+    p.gates[o] = sc[j] / gsum;
+    p.rank[o] = atomicAdd(&p.counts[sel[j]], 1);
+  }
+}
+
+template <int EPI, int BN>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const TcArgs args) {
+  using S = Shape<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = (uint64_t*)(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = (uint64_t*)(smem + STAGES * S::STAGE_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -205,7 +271,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(TMEM_COLS)
+                 "r"(S::TMEM_COLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -223,27 +289,28 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t phase = 0;
     for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
       const TileInfo ti = decode_tile(args, t);
+      const int gb = ti.group * args.b_rows_group;
       int b0, b1;
       if (EPI == EPI_SWIGLU_T) {
-        b0 = ti.group * args.b_rows_group + ti.n0;
-        b1 = ti.group * args.b_rows_group + p.up_off + ti.n0;
+        b0 = gb + ti.n0;
+        b1 = gb + p.up_off + ti.n0;
       } else {
-        b0 = ti.group * args.b_rows_group + ti.n0;
-        b1 = b0 + 128;
+        b0 = gb + ti.n0;
+        b1 = b0 + S::B_BOX;
       }
       for (int ks = 0; ks < nk; ++ks) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
-        uint8_t* sa = smem + stage * STAGE_BYTES;
-        mbar_expect_tx(&full[stage], STAGE_BYTES);
+        uint8_t* sa = smem + stage * S::STAGE_BYTES;
+        mbar_expect_tx(&full[stage], S::STAGE_BYTES);
         tma_load_2d(sa, &tmA, &full[stage], ks * BK, ti.row0);
         tma_load_2d(sa + A_BYTES, &tmB, &full[stage], ks * BK, b0);
-        tma_load_2d(sa + A_BYTES + B_HALF, &tmB, &full[stage], ks * BK, b1);
+        if (BN > 128) tma_load_2d(sa + A_BYTES + S::B_BOX * BK * 2, &tmB, &full[stage], ks * BK, b1);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
-    constexpr uint32_t IDESC = idesc_bf16(BM, BN_MMA);
+    constexpr uint32_t IDESC = idesc_bf16(BM, BN);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
@@ -252,11 +319,11 @@ __global__ void __launch_bounds__(192, 1)
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       if (!(ok = mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag))) break;
       tc_fence_after();
-      const uint32_t d = tmem + acc * BN_MMA;
+      const uint32_t d = tmem + acc * BN;
       for (int ks = 0; ks < nk; ++ks) {
         if (!(ok = mbar_wait(&full[stage], phase, abort_flag))) break;
         tc_fence_after();
-        uint8_t* sa = smem + stage * STAGE_BYTES;
+        uint8_t* sa = smem + stage * S::STAGE_BYTES;
         const uint64_t ad = smem_desc(sa), bd = smem_desc(sa + A_BYTES);
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)
@@ -281,15 +348,17 @@ __global__ void __launch_bounds__(192, 1)
       const TileInfo ti = decode_tile(args, t);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN_MMA;
+      const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN;
       const bool valid = rl < ti.rows;
       const long long r = (long long)ti.row0 + rl;
-      if (EPI == EPI_SWIGLU_T) {
+      if (EPI == EPI_ROUTER) {
+        if (BN == 64 || BN == 128) route_row<(BN == 128 ? 128 : 64)>(p, tbase, valid, r);
+      } else if (EPI == EPI_SWIGLU_T) {
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
+        for (int c = 0; c < BN / 2; c += 32) {
           float g[32], u[32];
           tmem_ld32(tbase + c, g);
-          tmem_ld32(tbase + 128 + c, u);
+          tmem_ld32(tbase + BN / 2 + c, u);
 #pragma unroll
           for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j]) * u[j];
           if (valid) store_bf16x32((bf16*)p.C + r * p.ldc + ti.n0 + c, g);
@@ -298,7 +367,7 @@ __global__ void __launch_bounds__(192, 1)
         const float rs = (EPI == EPI_GATE_F32 && valid) ? p.row_scale[r] : 0.f;
         const int pos = (EPI == EPI_ROPE_T && valid) ? p.pos[r] : 0;
 #pragma unroll 1
-        for (int c = 0; c < 256; c += 32) {
+        for (int c = 0; c < BN; c += 32) {
           float v[32];
           tmem_ld32(tbase + c, v);
           if (!valid) continue;
@@ -306,14 +375,17 @@ __global__ void __launch_bounds__(192, 1)
           if (EPI == EPI_STORE_T) {
             store_bf16x32((bf16*)p.C + r * p.ldc + col, v);
           } else if (EPI == EPI_ROPE_T) {
+            const int m0 = rope_chunk(p, col);
+            if (m0 >= 0) {
+              const float4* cs4 = reinterpret_cast<const float4*>(p.rope_tab + (long long)pos * p.rope_half + m0);
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              int m = rope_pair_tc(p, col + j);
-              if (m >= 0) {
-                float2 cs = p.rope_tab[(long long)pos * p.rope_half + m];
-                float r0 = v[j] * cs.x - v[j + 1] * cs.y, r1 = v[j] * cs.y + v[j + 1] * cs.x;
-                v[j] = r0;
-                v[j + 1] = r1;
+              for (int q = 0; q < 8; ++q) {
+                const float4 cs = cs4[q];   // (cos, sin) of pairs m0 + 2q and m0 + 2q + 1
+                float a0 = v[4 * q], a1 = v[4 * q + 1], b0 = v[4 * q + 2], b1 = v[4 * q + 3];
+                v[4 * q] = a0 * cs.x - a1 * cs.y;
+                v[4 * q + 1] = a0 * cs.y + a1 * cs.x;
+                v[4 * q + 2] = b0 * cs.z - b1 * cs.w;
+                v[4 * q + 3] = b0 * cs.w + b1 * cs.z;
               }
             }
             store_bf16x32((bf16*)p.C + r * p.ldc + col, v);
@@ -348,7 +420,7 @@ __global__ void __launch_bounds__(192, 1)
   if (*abort_flag && threadIdx.x == 0) record_status(p.st, ST_TIMEOUT, 501, blockIdx.x);
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(S::TMEM_COLS) : "memory");
   }
 }
 
@@ -401,27 +473,71 @@ int sm_count() {
 }
 
 inline bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+// MMA tile width for an epilogue and output width N (0 = unsupported).
+int pick_bn(const GemmParams& p, int epi) {
+  if (epi == EPI_SWIGLU_T) return (p.N % 128 == 0) ? 256 : 0;
+  if (epi == EPI_ROUTER) return (p.N == 64 || p.N == 128) ? p.N : 0;
+  if (p.N % 256 == 0) return 256;
+  if (p.N % 128 == 0) return 128;
+  if (p.N % 64 == 0) return 64;
+  return 0;
+}
+
+template <int EPI, int BN>
+int launch_tc(const CUtensorMap& mA, const CUtensorMap& mB, const tc::TcArgs& a, int grid, cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(tc::k_gemm_tc<EPI, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::Shape<BN>::SMEM_BYTES) != cudaSuccess)
+      return -1;
+    attr = true;
+  }
+  { tc::k_gemm_tc<EPI, BN><<<grid, 192, tc::Shape<BN>::SMEM_BYTES, s>>>(mA, mB, a); note_launch(); }
+  return 0;
+}
+
+template <int EPI>
+int launch_tc_bn(int bn, const CUtensorMap& mA, const CUtensorMap& mB, const tc::TcArgs& a, int grid, cudaStream_t s) {
+  switch (bn) {
+    case 64: return launch_tc<EPI, 64>(mA, mB, a, grid, s);
+    case 128: return launch_tc<EPI, 128>(mA, mB, a, grid, s);
+    case 256: return launch_tc<EPI, 256>(mA, mB, a, grid, s);
+  }
+  return -1;
+}
 }  // namespace
 
 bool gemm_tc_supports(const GemmParams& p, int epi) {
-  if (epi < EPI_STORE_F32 || epi > EPI_GATE_F32) return false;
+  if (epi < EPI_STORE_F32 || epi > EPI_ROUTER) return false;
   if (p.K < tc::BK || p.K % tc::BK) return false;
-  if (epi == EPI_SWIGLU_T ? (p.N % 128) : (p.N % 256)) return false;
+  if (!pick_bn(p, epi)) return false;
   if (p.lda % 8 || p.ldb % 8 || !al16(p.A) || !al16(p.B) || !al16(p.C)) return false;
-  if (epi == EPI_STORE_F32 || epi == EPI_RESID_F32 || epi == EPI_GATE_F32) {
+  if (epi == EPI_STORE_F32 || epi == EPI_RESID_F32 || epi == EPI_GATE_F32 || epi == EPI_ROUTER) {
     if (p.ldc % 4) return false;
   } else if (p.ldc % 8) {
     return false;
   }
   if (epi == EPI_RESID_F32 && (p.ld_resid % 4 || !al16(p.resid))) return false;
+  if (epi == EPI_ROPE_T) {
+    if (p.rope_half % 2 || !al16(p.rope_tab)) return false;
+    for (int q = 0; q < p.n_rope; ++q) {
+      const RopeDesc& r = p.rope[q];
+      if (r.col0 % 32 || r.head_stride % 32 || r.off % 32 || r.dim % 32) return false;
+    }
+  }
+  if (epi == EPI_ROUTER && (!p.bias || !p.ids || !p.gates || !p.rank || !p.counts || p.topk < 1 || p.topk > 32))
+    return false;
   if (p.tiles && (p.b_group_stride % p.ldb || p.b_rows <= 0)) return false;
   return encode_fn() != nullptr;
 }
 
 int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
+  const int bn = pick_bn(p, epi);
+  if (!bn) return -1;
   tc::TcArgs a;
   a.p = p;
-  a.n_out_tile = (epi == EPI_SWIGLU_T) ? 128 : 256;
+  a.n_out_tile = (epi == EPI_SWIGLU_T) ? bn / 2 : bn;
   a.n_n = p.N / a.n_out_tile;
   a.m_tiles = p.tiles ? 0 : (p.M + tc::BM - 1) / tc::BM;
   a.b_rows_group = p.tiles ? (int)(p.b_group_stride / p.ldb) : 0;
@@ -430,7 +546,7 @@ int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
   if (!make_map(&mA, p.A, (unsigned long long)p.M, p.K, p.lda, 128)) return -1;
   unsigned long long brows = p.b_rows > 0 ? (unsigned long long)p.b_rows
                                           : (unsigned long long)((epi == EPI_SWIGLU_T) ? p.up_off + p.N : p.N);
-  if (!make_map(&mB, p.B, brows, p.K, p.ldb, 128)) return -1;
+  if (!make_map(&mB, p.B, brows, p.K, p.ldb, bn > 128 ? 128 : bn)) return -1;
   int grid;
   if (p.tiles) {
     grid = sm_count();
@@ -439,28 +555,19 @@ int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
     grid = (int)std::min<long long>(tiles, sm_count());
   }
   if (grid <= 0) return 0;
-#define RDT_TC_CASE(E)                                                                              \
-  case E: {                                                                                         \
-    static bool attr = false;                                                                       \
-    if (!attr) {                                                                                    \
-      if (cudaFuncSetAttribute(tc::k_gemm_tc<E>, cudaFuncAttributeMaxDynamicSharedMemorySize,       \
-                               tc::SMEM_BYTES) != cudaSuccess)                                      \
-        return -1;                                                                                  \
-      attr = true;                                                                                  \
-    }                                                                                               \
-    { tc::k_gemm_tc<E><<<grid, 192, tc::SMEM_BYTES, s>>>(mA, mB, a); note_launch(); }                                  \
-    break;                                                                                          \
-  }
+  int rc;
   switch (epi) {
-    RDT_TC_CASE(EPI_STORE_F32)
-    RDT_TC_CASE(EPI_STORE_T)
-    RDT_TC_CASE(EPI_RESID_F32)
-    RDT_TC_CASE(EPI_ROPE_T)
-    RDT_TC_CASE(EPI_SWIGLU_T)
-    RDT_TC_CASE(EPI_GATE_F32)
+    case EPI_STORE_F32: rc = launch_tc_bn<EPI_STORE_F32>(bn, mA, mB, a, grid, s); break;
+    case EPI_STORE_T: rc = launch_tc_bn<EPI_STORE_T>(bn, mA, mB, a, grid, s); break;
+    case EPI_RESID_F32: rc = launch_tc_bn<EPI_RESID_F32>(bn, mA, mB, a, grid, s); break;
+    case EPI_ROPE_T: rc = launch_tc_bn<EPI_ROPE_T>(bn, mA, mB, a, grid, s); break;
+    case EPI_SWIGLU_T: rc = launch_tc<EPI_SWIGLU_T, 256>(mA, mB, a, grid, s); break;
+    case EPI_GATE_F32: rc = launch_tc_bn<EPI_GATE_F32>(bn, mA, mB, a, grid, s); break;
+    case EPI_ROUTER: rc = (bn == 64) ? launch_tc<EPI_ROUTER, 64>(mA, mB, a, grid, s)
+                                     : launch_tc<EPI_ROUTER, 128>(mA, mB, a, grid, s); break;
     default: return -1;
   }
-#undef RDT_TC_CASE
+  if (rc) return rc;
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

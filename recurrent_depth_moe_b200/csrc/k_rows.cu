@@ -387,7 +387,10 @@ void launch_kv_to_cache(int dtype, const void* qkv, long long ld, int k_col, int
     { k_kv_to_cache<bf16><<<N, 128, 0, s>>>((const bf16*)qkv, ld, k_col, v_col, Hkv, hd, pos, seq, t_max,
                                           (bf16*)kc, (bf16*)vc, st); note_launch(); }
 }
+bool launch_combine_warp(int dtype, const CombineParams& p, int n_rows, cudaStream_t s);
+
 void launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s) {
+  if (launch_combine_warp(dtype, p, n_rows, s)) return;
   size_t smem = (size_t)(p.D + 64) * sizeof(float);
   int nt = nthreads_for(p.D);
   if (dtype == 0) { k_combine_inject_act<float><<<n_rows, nt, smem, s>>>(p); note_launch(); }

@@ -31,7 +31,8 @@ enum Epi {
   EPI_RESID_F32 = 2,   // C fp32 = resid + acc
   EPI_ROPE_T = 3,      // C model dtype = RoPE(acc) on the described column ranges
   EPI_SWIGLU_T = 4,    // C model dtype = silu(acc(B rows c)) * acc(B rows up_off + c)
-  EPI_GATE_F32 = 5     // C fp32 = row_scale[row] * acc
+  EPI_GATE_F32 = 5,    // C fp32 = row_scale[row] * acc
+  EPI_ROUTER = 6       // C fp32 = logits; plus softmax / biased top-k / gates / expert histogram
 };
 
 struct RopeDesc {        // columns col0 + h * head_stride + off + [0, dim), h < n_heads
@@ -50,6 +51,9 @@ struct GemmParams {
   const int* pos; const float2* rope_tab; int rope_half; int n_rope; RopeDesc rope[2];
   long long b_rows;                                      // rows of the B tensor (0: derive from N)
   int impl;                                              // -1 auto, else a GemmImpl
+  // EPI_ROUTER: route the running rows (run_idx >= 0) from their logits row
+  const float* bias; const int* run_idx; int topk;
+  int* ids; float* gates; int* rank; int* counts;
   DevStatus* st;
 };
 

@@ -241,9 +241,6 @@ rdt_status moe_block(Ctx& x, int N, const float* x1) {
   void* f = at<void*>(x.ws, x.L.f);
   { ProfScope ps(PC_FFN_NORM, x.s); launch_rmsnorm(1, x.dtype, x1, D, w->ffn_norm_w, f, D, N, D, c->norm_eps, x.s); }
   float* logits = at<float*>(x.ws, x.L.logits);
-  GemmParams g = gemm_base(x);
-  g.A = f; g.lda = D; g.B = w->w_router; g.ldb = D; g.M = N; g.N = E; g.K = D; g.C = logits; g.ldc = E;
-  { ProfScope ps(PC_ROUTER_GEMM, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_STORE_F32, g, x.s)); }
   RouteParams rp;
   memset(&rp, 0, sizeof(rp));
   rp.logits = logits; rp.bias = w->router_bias; rp.N = N; rp.E = E; rp.k = k; rp.S = S;
@@ -270,9 +267,16 @@ rdt_status moe_block(Ctx& x, int N, const float* x1) {
   up.impl = dn.impl = (int)iu;
   rp.tile_m = gemm_tile_m(iu);
   if (cudaMemsetAsync(rp.counts, 0, sizeof(int) * std::max(E, 1), x.s) != cudaSuccess) return RDT_ERR_CUDA;
+  // router logits; on the tensor-core path the GEMM epilogue also routes the running rows
+  GemmParams g = gemm_base(x);
+  g.A = f; g.lda = D; g.B = w->w_router; g.ldb = D; g.M = N; g.N = E; g.K = D; g.C = logits; g.ldc = E;
+  g.bias = w->router_bias; g.run_idx = at<int*>(x.ws, x.L.run_idx); g.topk = k;
+  g.ids = rp.ids; g.gates = rp.gates; g.rank = rp.rank; g.counts = rp.counts;
+  const bool fused_route = gemm_pick(x.dtype, g, EPI_ROUTER) == GEMM_TC;
+  { ProfScope ps(PC_ROUTER_GEMM, x.s); RDT_TRY(launch_gemm(x.dtype, fused_route ? EPI_ROUTER : EPI_STORE_F32, g, x.s)); }
   {
     ProfScope ps(PC_ROUTE, x.s);
-    launch_router_topk(rp, x.s);
+    if (!fused_route) launch_router_topk(rp, x.s);
     launch_route_scan(rp, x.s);
     launch_route_scatter(x.dtype, rp, x.s);
   }
