@@ -19,6 +19,7 @@
 // RDT_ERR_DEVICE_TIMEOUT in the status word and leaves its loops.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 #include <cuda.h>
 #include <algorithm>
@@ -29,7 +30,6 @@ namespace tc {
 
 constexpr int BM = 128, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
-constexpr long long TIMEOUT_CYCLES = 4000000000LL;   // ~2 s at 2 GHz
 
 template <int BN> struct Shape {
   static constexpr int B_BYTES = BN * BK * 2;
@@ -46,97 +46,6 @@ struct TcArgs {
   int b_rows_group;    // rows of B per group (grouped)
   int n_out_tile;      // output columns per tile
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, int count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-// Bounded wait: false on timeout or when another role already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try_wait(b, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(b, parity)) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > TIMEOUT_CYCLES) {
-      *abort_flag = 1;
-      return false;
-    }
-  }
-  return true;
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
-          smem_u32(dst)),
-      "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-
-// K-major, 128-byte-swizzled operand tile: 8-row groups 1024 bytes apart.
-__device__ __forceinline__ uint64_t smem_desc(const void* p) {
-  uint64_t d = 0;
-  d |= (uint64_t)((smem_u32(p) >> 4) & 0x3FFF);
-  d |= (uint64_t)1 << 16;                  // leading byte offset (unused for swizzled K-major)
-  d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset: 8 rows x 128 B
-  d |= (uint64_t)1 << 46;                  // descriptor version (sm_100)
-  d |= (uint64_t)2 << 61;                  // SWIZZLE_128B
-  return d;
-}
-
-// kind::f16 instruction descriptor: bf16 A/B, fp32 D, both K-major.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(accum)
-      : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z)); }
 
@@ -389,6 +298,15 @@ __global__ void __launch_bounds__(192, 1)
               }
             }
             store_bf16x32((bf16*)p.C + r * p.ldc + col, v);
+            if (p.vt && col >= p.vt_col0 && col < p.vt_col0 + p.vt_heads * p.vt_hd) {
+              // transposed copy of the values: for each dim, the warp's 32 rows are 32
+              // consecutive positions, so every store instruction writes 64 contiguous bytes
+              const int vc = col - p.vt_col0, g = vc / p.vt_hd, d0 = vc % p.vt_hd;
+              const long long b = r / p.vt_T, tpos = r % p.vt_T;
+              bf16* vt = (bf16*)p.vt + ((b * p.vt_heads + g) * p.vt_hd + d0) * p.vt_ld + tpos;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) vt[(long long)j * p.vt_ld] = __float2bfloat16_rn(v[j]);
+            }
           } else {
             float* dst = (float*)p.C + r * p.ldc + col;
             if (EPI == EPI_RESID_F32) {
@@ -473,7 +391,15 @@ int sm_count() {
 }
 
 inline bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+}  // namespace
 
+bool tc_make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsigned long long cols,
+                 unsigned long long ld, unsigned box_rows) {
+  return make_map(m, base, rows, cols, ld, box_rows);
+}
+int tc_sm_count() { return sm_count(); }
+
+namespace {
 // MMA tile width for an epilogue and output width N (0 = unsupported).
 int pick_bn(const GemmParams& p, int epi) {
   if (epi == EPI_SWIGLU_T) return (p.N % 128 == 0) ? 256 : 0;

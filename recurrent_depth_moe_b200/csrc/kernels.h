@@ -54,6 +54,9 @@ struct GemmParams {
   // EPI_ROUTER: route the running rows (run_idx >= 0) from their logits row
   const float* bias; const int* run_idx; int topk;
   int* ids; float* gates; int* rank; int* counts;
+  // EPI_ROPE_T (optional): also store the value columns [vt_col0, vt_col0 + vt_heads * vt_hd)
+  // transposed: vt[((b * vt_heads + g) * vt_hd + d) * vt_ld + t] for row = b * vt_T + t
+  void* vt; int vt_col0, vt_heads, vt_hd, vt_T; long long vt_ld;
   DevStatus* st;
 };
 
@@ -81,6 +84,8 @@ struct AttnParams {
   float scale;
   // split-KV decode scratch
   float* part_o; float* part_ml; int n_split;
+  // tensor-core prefill: values transposed, vt[((b * Hkv + g) * dv + d) * vt_ld + j]
+  const void* vt; long long vt_ld;
 };
 int launch_attention(int dtype, const AttnParams& p, cudaStream_t s);
 int launch_attention_decode(int dtype, const AttnParams& p, cudaStream_t s);

@@ -19,7 +19,7 @@ struct Layout {
   // byte offsets into the workspace
   size_t status, h, combined, a, qkv, cq_raw, cq, q, kv_raw, ckv, krope, kvu, attn, x1, f, logits;
   size_t ids, gates, rank, counts, offsets, tiles, ntiles, slot_of, tok_of, gate_of, xg, u, y;
-  size_t run_list, run_idx, nrun, cum, halted, Avec, emb, rope, pos, p_buf, part_o, part_ml, xn;
+  size_t run_list, run_idx, nrun, cum, halted, Avec, emb, rope, pos, p_buf, part_o, part_ml, xn, vt;
   size_t total;
   int max_tiles, max_slots, rope_dim, rope_pos, n_split;
 };
@@ -67,6 +67,7 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
   if (c->attn_type == 0) {
     int hd = c->dim / H;
     L->qkv = take(N * (size_t)(H + 2 * c->n_kv_heads) * hd * es);
+    L->vt = take(N * (size_t)c->n_kv_heads * hd * es);   // values transposed per sequence
     dv = hd;
     L->rope_dim = hd;
   } else {
@@ -165,6 +166,14 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
     g.C = qkv; g.ldc = W; g.pos = pos; g.rope_tab = tab; g.rope_half = hd / 2; g.n_rope = 2;
     g.rope[0] = RopeDesc{0, H, hd, 0, hd};
     g.rope[1] = RopeDesc{H * hd, Hkv, hd, 0, hd};
+    // the tensor-core attention reads V transposed; the QKV epilogue writes that copy
+    const bool kv_from_qkv = !(cache && cache->k && (decode || start_pos > 0));
+    bool want_vt = x.dtype == 1 && hd == 128 && T % 8 == 0 && kv_from_qkv && !decode;
+    if (want_vt) {
+      g.vt = at<void*>(x.ws, x.L.vt); g.vt_col0 = (H + Hkv) * hd; g.vt_heads = Hkv; g.vt_hd = hd; g.vt_T = T; g.vt_ld = T;
+      if (gemm_pick(x.dtype, g, EPI_ROPE_T) != GEMM_TC) { g.vt = nullptr; want_vt = false; }
+    }
+    ap.vt = want_vt ? g.vt : nullptr; ap.vt_ld = T;
     { ProfScope ps(PC_QKV, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, x.s)); }
     ap.q = qkv; ap.q_row = W; ap.q_head = hd; ap.dn = hd; ap.dr = 0; ap.dv = hd; ap.G = H / Hkv;
     ap.scale = 1.f / sqrtf((float)hd);
@@ -420,6 +429,8 @@ bool gemm_tc_supports(const GemmParams& p, int epi);
 int launch_attention_simt(int dtype, const AttnParams& p, cudaStream_t s);
 bool attention_fa_supports(int dtype, const AttnParams& p);
 int launch_attention_fa(const AttnParams& p, cudaStream_t s);
+bool attention_tc_supports(int dtype, const AttnParams& p);
+int launch_attention_tc(const AttnParams& p, cudaStream_t s);
 
 int gemm_tile_m(GemmImpl impl) { return impl == GEMM_TC ? 128 : 64; }
 GemmImpl gemm_pick(int dtype, const GemmParams& p, int epi) {
@@ -432,6 +443,7 @@ int launch_gemm(int dtype, int epi, const GemmParams& p, cudaStream_t s) {
   return launch_gemm_simt(dtype, epi, p, s);
 }
 int launch_attention(int dtype, const AttnParams& p, cudaStream_t s) {
+  if (attention_tc_supports(dtype, p)) return launch_attention_tc(p, s);
   if (attention_fa_supports(dtype, p)) return launch_attention_fa(p, s);
   return launch_attention_simt(dtype, p, s);
 }
