@@ -250,6 +250,14 @@ def run_ours(args, wl, rank, world, local_rank):
         torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
     e2e_value = float(tl.item()) / (float(te.item()) / 1e3)
 
+    # host copy for the CPU-oracle baseline, then free the prefill workload before the
+    # decode one (23 GB of weights and caches)
+    W_cpu = {k: v.cpu() for k, v in W.items()} if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    h0_c, e_c = h0[:64].cpu(), e[:64].cpu()
+    del blk, ws, W, out, h0_d, e_d
+    torch.cuda.empty_cache()
+    decode_res = None if args.no_decode else run_decode(args, rank, world, local_rank)
+
     if rank != 0:
         return
     pk, pk_kind = peaks()
@@ -281,15 +289,107 @@ def run_ours(args, wl, rank, world, local_rank):
            "kernel_ms_per_step": breakdown,
            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
            "clocks": clk}
+    if not args.no_decode:
+        res["decode"] = decode_res
     if world == 1 and not args.no_cpu_baseline:
-        W_cpu = {k: v.cpu() for k, v in W.items()}
-        h0_c, e_c = h0[:64].cpu(), e[:64].cpu()
         pos, loops = 64, 8
         rate, dt = oracle_sample(wl, W_cpu, h0_c, e_c, pos, loops)
         res["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
                                "sample": f"sequence 0, positions 0-{pos - 1}, loops 0-{loops - 1} "
                                          f"(fp64 oracle, {dt:.1f} s)"}
     print(json.dumps(res), flush=True)
+
+
+def decode_algorithmic_bytes(cfg, ids: torch.Tensor, lens: torch.Tensor) -> float:
+    """HBM bytes one decode step must move at minimum: every expert a loop touches is
+    streamed once (routed experts by the realised routing, plus the shared ones), the
+    attention / router / LoRA weights once per loop, each sequence's cache of that loop
+    read once (cache_len + 1 keys and values) and one new K/V row written."""
+    D, F, E, S = cfg.dim, cfg.expert_dim, cfg.n_experts, cfg.n_shared_experts
+    hd, H, Hkv = cfg.head_dim, cfg.n_heads, cfg.n_kv_heads
+    expert_bytes = 3 * D * F * 2
+    attn_bytes = ((H + 2 * Hkv) * hd * D + D * H * hd) * 2
+    small = (E * D + 2 * cfg.lora_rank * D) * 2
+    L = ids.shape[0]
+    kv = float((lens.double() + 1).sum()) * Hkv * hd * 2 * 2
+    total = 0.0
+    for t in range(L):
+        distinct = int(torch.unique(ids[t][ids[t] >= 0]).numel())
+        total += (distinct + S) * expert_bytes + attn_bytes + small + kv
+    return total
+
+
+def run_decode(args, rank, world, local_rank):
+    """3B-shaped KV-cached decode: 64 sequences with 4096-token random caches per loop,
+    one new token per sequence per step over `decode_steps` steps."""
+    import recurrent_depth_moe_b200 as R
+    from recurrent_depth_moe_b200 import _native as NAT
+    dev = torch.device("cuda", local_rank)
+    wl = RI.get_workload("rdt3b_decode")
+    cfg = wl.cfg
+    B, L, steps = wl.batch, wl.n_loops, args.decode_steps
+    t_max = wl.cache_len + steps + args.warmup
+    W = RI.block_weights(cfg, wl.seed, device=dev)
+    k, v = RI.random_kv_cache(cfg, L, B, t_max, wl.cache_len, wl.seed + 31 * rank, device=dev)
+    h0s, es = [], []
+    for st in range(steps + args.warmup):
+        h, e = RI.decode_inputs(cfg, B, st, wl.seed + 31 * rank, device=dev)
+        h0s.append(h)
+        es.append(e)
+    blk = R.RecurrentBlock(cfg, W)
+    cache = R.KVCache(k, v)
+    ws = blk.workspace(B, 1, t_max)
+    clen = torch.full((B,), wl.cache_len, dtype=torch.int32, device=dev)
+    out = (torch.empty(B, cfg.dim, dtype=torch.float32, device=dev), torch.empty(L, B, dtype=torch.float32, device=dev),
+           torch.empty(L, B, cfg.n_experts_per_tok, dtype=torch.int32, device=dev))
+    for st in range(args.warmup):
+        blk.decode_step(h0s[st], es[st], clen, cache, L, wl.act_threshold, out=out, workspace=ws)
+        clen.add_(1)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0, "device status word set during decode warm-up"
+    lens0 = clen.clone()
+    stream = torch.cuda.current_stream()
+    NAT.profile_start()
+    n0 = NAT.launch_count()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for st in range(steps):
+        blk.decode_step(h0s[args.warmup + st], es[args.warmup + st], clen, cache, L, wl.act_threshold, out=out,
+                        workspace=ws)
+        clen.add_(1)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    launches = NAT.launch_count() - n0
+    prof = NAT.profile_stop()
+    ms = e0.elapsed_time(e1) / steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+    # algorithmic bytes of the last timed step (its routing and cache lengths)
+    bytes_step = decode_algorithmic_bytes(cfg, out[2].cpu(), (clen - 1).cpu())
+    pk, pk_kind = peaks()
+    gbs = bytes_step / (ms / 1e3) / 1e9
+    res = {"metric": "decode tokens/s", "value": B * world / (ms_max / 1e3), "unit": "tokens/s",
+           "ms_per_step": ms_max, "steps": steps,
+           "workload": (f"{wl.name}: 3B-shaped KV-cached decode, dim {cfg.dim}, {cfg.n_heads} heads GQA "
+                        f"({cfg.n_kv_heads} kv), {cfg.n_experts} routed + {cfg.n_shared_experts} shared experts "
+                        f"top-{cfg.n_experts_per_tok}, expert_dim {cfg.expert_dim}, {L} loops, batch {B} sequences "
+                        f"with {wl.cache_len}-token random caches per loop, 1 new token per step, bf16, ACT off"),
+           "roofline": {"bound": "hbm", "kernel": "whole decode step (expert weights + caches streamed)",
+                        "achieved": gbs, "peak": pk.get("hbm_gbs"), "unit": "GB/s",
+                        "frac": gbs / pk.get("hbm_gbs"), "peak_kind": f"{pk_kind} HBM copy bandwidth",
+                        "algorithmic_bytes_per_step": bytes_step, "traffic": None},
+           "gpu_launches": launches,
+           "kernel_ms_per_step": {k2: {"launches": v2[0], "ms_per_step": v2[1] / steps} for k2, v2 in sorted(prof.items())}}
+    del k, v, cache, W, blk, ws
+    torch.cuda.empty_cache()
+    return res
 
 
 def main():
@@ -299,6 +399,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=128)
+    ap.add_argument("--batch", type=int, default=None, help="override the sequences per step (small profiling cases)")
+    ap.add_argument("--loops", type=int, default=None, help="override n_loops (small profiling cases)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         log("warm-up raised to 3 steps")
@@ -307,6 +411,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = RI.get_workload(WORKLOAD)
+    if args.batch or args.loops:
+        import dataclasses
+        wl = dataclasses.replace(wl, batch=args.batch or wl.batch, n_loops=args.loops or wl.n_loops)
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
         return

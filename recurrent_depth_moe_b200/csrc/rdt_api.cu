@@ -11,6 +11,10 @@
 
 using namespace rdt;
 
+namespace rdt {
+int decode_split_count(int t_max);
+}
+
 namespace {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -113,9 +117,10 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
   L->rope_pos = std::max(max_keys, T);
   L->rope = take((size_t)L->rope_pos * (L->rope_dim / 2) * 8);
   L->pos = take(N * 4);
-  L->n_split = 0;
-  L->part_o = take(16);
-  L->part_ml = take(16);
+  // decode layouts (one row per sequence) hold the split-KV attention partials
+  L->n_split = (T == 1) ? decode_split_count(std::max(max_keys, 1)) : 0;
+  L->part_o = take(L->n_split ? (size_t)B * H * L->n_split * 128 * 4 : 16);
+  L->part_ml = take(L->n_split ? (size_t)B * H * L->n_split * 2 * 4 : 16);
   L->total = off;
 }
 
@@ -189,6 +194,9 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
         ap.v = vc; ap.v_b = sb; ap.v_j = sj; ap.v_g = sg;
         ap.key_pos0 = 0;
         ap.n_keys = decode ? cache->t_max : start_pos + T;
+        if (decode && x.L.n_split) {
+          ap.part_o = at<float*>(x.ws, x.L.part_o); ap.part_ml = at<float*>(x.ws, x.L.part_ml); ap.n_split = x.L.n_split;
+        }
       }
     }
     if (!ap.k1) {
@@ -443,6 +451,7 @@ int launch_gemm(int dtype, int epi, const GemmParams& p, cudaStream_t s) {
   return launch_gemm_simt(dtype, epi, p, s);
 }
 int launch_attention(int dtype, const AttnParams& p, cudaStream_t s) {
+  if (p.part_o && p.T == 1 && launch_attention_decode(dtype, p, s) == 0) return 0;
   if (attention_tc_supports(dtype, p)) return launch_attention_tc(p, s);
   if (attention_fa_supports(dtype, p)) return launch_attention_fa(p, s);
   return launch_attention_simt(dtype, p, s);

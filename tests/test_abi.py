@@ -46,8 +46,8 @@ def test_workspace_size_host_logic(lib):
         cs = api.config_struct(wl.cfg)
         n = api.workspace_size(cs, wl.batch, wl.seq, wl.seq + wl.cache_len)
         assert n > 0 and n % 256 == 0
-        # monotone in the row count
-        assert api.workspace_size(cs, wl.batch, wl.seq * 2, wl.seq * 2 + wl.cache_len) > n
+        # monotone in the number of sequences
+        assert api.workspace_size(cs, wl.batch * 2, wl.seq, wl.seq + wl.cache_len) > n
     bad = api.config_struct(RI.get_workload("tiny_gqa_fp32").cfg)
     bad.n_kv_heads = 3                       # 8 heads not divisible by 3
     assert api.workspace_size(bad, 2, 16, 16) == 0

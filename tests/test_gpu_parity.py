@@ -241,3 +241,40 @@ def test_invalid_arguments_return_errors():
     with pytest.raises(R.RdtError) as ei:
         R.RecurrentBlock(cfg, bad).forward(h0, e, 1, 8, 2, 0.0)
     assert ei.value.code == 1
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_decode_random_cache_ragged_lengths(dtype):
+    """Decode step against random per-loop caches (the 3B decode workload's structure:
+    GQA group 3, one cache per loop) with a different cache length per sequence."""
+    cfg = RI.RDTConfig(dim=768, n_heads=6, n_kv_heads=2, max_seq_len=160, max_loop_iters=3, n_experts=8,
+                       n_shared_experts=1, n_experts_per_tok=2, expert_dim=128, lora_rank=8, dtype=dtype)
+    W = RI.block_weights(cfg, 21, attn_std=0.05)
+    B, L, t_max = 4, 3, 160
+    lens = [37, 100, 64, 5]
+    k, v = RI.random_kv_cache(cfg, L, B, t_max, max(lens), 22)
+    for b, n in enumerate(lens):                       # positions >= len are not part of the cache
+        k[:, b, :, n:] = 0
+        v[:, b, :, n:] = 0
+    h0, e = RI.decode_inputs(cfg, B, 0, 23)
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    cache = R.KVCache(k.cuda(), v.cuda())
+    clen = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    d_h, d_hw, d_ids = blk.decode_step(h0.cuda(), e.cuda(), clen, cache, L, 0.0)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    caches = [[{"k": k[t, b, :, :lens[b]].permute(1, 0, 2), "v": v[t, b, :, :lens[b]].permute(1, 0, 2),
+                "pos": torch.arange(lens[b])} for b in range(B)] for t in range(L)]
+    o_h, o_hw, o_ids, new_kv = O.decode_step(cfg, W, h0, e, caches, lens, L, 0.0)
+    if dtype == "fp32":
+        assert max_rel(d_h, o_h) <= FP32_TOL
+        assert torch.equal(d_ids.cpu().long(), o_ids)
+    else:
+        assert rel_l2(d_h, o_h) <= BF16_TOL
+    # the new keys / values were appended at cache_len[b] in every loop cache
+    kc = cache.k.cpu()
+    for t in range(L):
+        for b in range(B):
+            got = kc[t, b, :, lens[b]].double()
+            want = new_kv[t][b][0][0].double()
+            assert rel_l2(got, want) <= (1e-5 if dtype == "fp32" else 2e-2)
