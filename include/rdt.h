@@ -173,6 +173,31 @@ RDT_API rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_we
                                      const rdt_kv_cache* cache,
                                      void* ws, size_t ws_bytes, void* stream);
 
+/* Decode step without a caller workspace, for callers that cannot allocate device
+ * memory (a warm serving loop that must not allocate, a host runtime without a CUDA
+ * allocator of its own, a memory-pool budget with no room for a per-call workspace).
+ * The paper has no counterpart: this is a library convenience around
+ * rdt_recurrent_decode_step, which it runs unchanged.
+ *  - Scratch: a static device array of RDT_STATIC_SCRATCH_BYTES inside librdt, held
+ *    by every GPU that loads the library until the process exits.  Nothing is
+ *    allocated by this call (no cudaMalloc / cudaFree / allocating library routine).
+ *  - Arguments, layouts and outputs are those of rdt_recurrent_decode_step; the
+ *    caller still provides inputs, outputs, weights and the caches.
+ *  - Sizes whose workspace (rdt_workspace_size(cfg, batch, 1, cache->t_max)) exceeds
+ *    RDT_STATIC_SCRATCH_BYTES are rejected with RDT_ERR_WORKSPACE, nothing enqueued.
+ *  - The first call on each device resolves the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call before
+ *    any stream capture.
+ *  - All calls share the one array: calls that overlap on the GPU (different streams,
+ *    or other host threads) race and corrupt each other.  Each call initialises every
+ *    part of the array it reads, so leftover contents of earlier calls do not matter. */
+#define RDT_STATIC_SCRATCH_BYTES (32u << 20)
+RDT_API rdt_status rdt_recurrent_decode_step_static(const rdt_config* cfg, const rdt_weights* w,
+                                                    const float* h0, const void* e, int batch,
+                                                    const int32_t* cache_len, int n_loops, float act_threshold,
+                                                    float* h_out, float* halt_weights, int32_t* expert_ids,
+                                                    const rdt_kv_cache* cache, void* stream);
+
 /* One pre-norm TransformerBlock: x_out = x1 + FFN(RMSNorm(x1)), x1 = x_in + Attn(RMSNorm(x_in)).
  * FFN is the MoE when cfg->n_experts > 0, else the dense SwiGLU in w13/w2 expert 0
  * with hidden cfg->expert_dim (prelude/coda: Expert(dim, dim*4//3), "OpenMythos 분석", MoE).
