@@ -30,7 +30,50 @@ template <> struct Vec4<bf16> {
 };
 
 __device__ __forceinline__ float4 f4_add(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+template <typename T> __device__ __forceinline__ void store4(T* p, float4 v);
+template <> __device__ __forceinline__ void store4<float>(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
+}
 __device__ __forceinline__ float f4_dot(float4 a, float4 b) { return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w; }
+
+// Prologue of the next loop for one row held by a warp (x = state, in registers):
+//   combined = RMSNorm_rec(x + emb + e) * w_rec ; a = RMSNorm_attn(combined) * w_attn
+template <typename T, int VPL>
+__device__ __forceinline__ void next_prologue(const CombineParams& p, float4 (&x)[VPL], long long rowD, int lane) {
+  const T* er = (const T*)p.e + rowD + 4 * lane;
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int d = 4 * lane + 128 * j;
+    float4 ev = Vec4<T>::load(er + 128 * j);
+    x[j] = f4_add(x[j], ev);
+    if (d < p.loop_dim) x[j] = f4_add(x[j], __ldg(reinterpret_cast<const float4*>(p.next_emb + d)));
+    ss += f4_dot(x[j], x[j]);
+  }
+  const float inv = rsqrtf(warp_sum(ss) / p.D + p.eps);
+  float ss2 = 0.f;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int d = 4 * lane + 128 * j;
+    const float4 wv = __ldg(reinterpret_cast<const float4*>(p.w_rec + d));
+    x[j] = make_float4(x[j].x * inv * wv.x, x[j].y * inv * wv.y, x[j].z * inv * wv.z, x[j].w * inv * wv.w);
+    *reinterpret_cast<float4*>(p.combined_out + rowD + d) = x[j];
+    ss2 += f4_dot(x[j], x[j]);
+  }
+  const float inv2 = rsqrtf(warp_sum(ss2) / p.D + p.eps);
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int d = 4 * lane + 128 * j;
+    const float4 wv = __ldg(reinterpret_cast<const float4*>(p.w_attn + d));
+    store4<T>((T*)p.a_out + rowD + d,
+              make_float4(x[j].x * inv2 * wv.x, x[j].y * inv2 * wv.y, x[j].z * inv2 * wv.z, x[j].w * inv2 * wv.w));
+  }
+}
 
 template <typename T, int VPL>
 __global__ void __launch_bounds__(256) k_combine_warp(CombineParams p) {
@@ -39,13 +82,18 @@ __global__ void __launch_bounds__(256) k_combine_warp(CombineParams p) {
   if (i >= p.N) return;
   const int D = p.D;
   const int kS = p.k + p.S;
+  const long long rowD = (long long)i * D;
+  float4 tr[VPL];
   if (!p.block_only && p.halted[i]) {   // frozen row: no update, zero weight, no experts
     if (lane == 0) p.halt_w_out[(long long)p.t * p.N + i] = 0.f;
     if (lane < p.k) p.ids_out[((long long)p.t * p.N + i) * p.k + lane] = -1;
+    if (p.next_emb) {                   // its keys / values are still recomputed next loop
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) tr[j] = __ldg(reinterpret_cast<const float4*>(p.h + rowD + 4 * lane + 128 * j));
+      next_prologue<T, VPL>(p, tr, rowD, lane);
+    }
     return;
   }
-  float4 tr[VPL];
-  const long long rowD = (long long)i * D;
   if (p.transformer_off) {
 #pragma unroll
     for (int j = 0; j < VPL; ++j) tr[j] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -58,9 +106,9 @@ __global__ void __launch_bounds__(256) k_combine_warp(CombineParams p) {
         if (lane == 0) record_status(p.st, ST_BOUNDS, 202, slot);
         continue;
       }
-      const float* yr = p.y + (long long)slot * D + 4 * lane;
+      const T* yr = (const T*)p.y + (long long)slot * D + 4 * lane;
 #pragma unroll
-      for (int j = 0; j < VPL; ++j) tr[j] = f4_add(tr[j], __ldg(reinterpret_cast<const float4*>(yr + 128 * j)));
+      for (int j = 0; j < VPL; ++j) tr[j] = f4_add(tr[j], Vec4<T>::load(yr + 128 * j));
     }
   }
   if (p.block_only) {
@@ -142,17 +190,62 @@ __global__ void __launch_bounds__(256) k_combine_warp(CombineParams p) {
   if (lane == 0) p.halt_w_out[(long long)p.t * p.N + i] = w;
   if (lane < p.k)
     p.ids_out[((long long)p.t * p.N + i) * p.k + lane] = p.transformer_off ? -1 : p.ids[(long long)i * p.k + lane];
+  if (p.next_emb) next_prologue<T, VPL>(p, tr, rowD, lane);
+}
+
+// out = RMSNorm(x) * w for fp32 rows of width D = 128 * VPL, one warp per row.
+template <typename T, int VPL>
+__global__ void __launch_bounds__(256) k_rmsnorm_warp(const float* __restrict__ x, const float* __restrict__ w,
+                                                      T* __restrict__ out, int N, int D, float eps) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (i >= N) return;
+  const long long rowD = (long long)i * D;
+  float4 v[VPL];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    v[j] = __ldg(reinterpret_cast<const float4*>(x + rowD + 4 * lane + 128 * j));
+    ss += f4_dot(v[j], v[j]);
+  }
+  const float inv = rsqrtf(warp_sum(ss) / D + eps);
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    const int d = 4 * lane + 128 * j;
+    const float4 wv = __ldg(reinterpret_cast<const float4*>(w + d));
+    store4<T>(out + rowD + d, make_float4(v[j].x * inv * wv.x, v[j].y * inv * wv.y, v[j].z * inv * wv.z,
+                                          v[j].w * inv * wv.w));
+  }
 }
 
 // Returns false when the shape needs the CTA-per-row kernel instead.
 static inline bool al(const void* q, int b) { return ((uintptr_t)q % b) == 0; }
 
+bool launch_rmsnorm_warp(int dtype, const float* x, const float* w, void* out, int N, int D, float eps,
+                         cudaStream_t s) {
+  if (D % 128 || !al(x, 16) || !al(w, 16) || !al(out, dtype == 0 ? 16 : 8)) return false;
+  const unsigned blocks = (unsigned)((N + 7) / 8);
+#define RDT_RW(V)                                                                                             \
+  case V:                                                                                                     \
+    if (dtype == 0) { k_rmsnorm_warp<float, V><<<blocks, 256, 0, s>>>(x, w, (float*)out, N, D, eps); note_launch(); } \
+    else { k_rmsnorm_warp<bf16, V><<<blocks, 256, 0, s>>>(x, w, (bf16*)out, N, D, eps); note_launch(); }    \
+    return true;
+  switch (D / 128) {
+    RDT_RW(1) RDT_RW(2) RDT_RW(4) RDT_RW(8) RDT_RW(12) RDT_RW(16) RDT_RW(24) RDT_RW(32)
+    default: return false;
+  }
+#undef RDT_RW
+}
+
 bool launch_combine_warp(int dtype, const CombineParams& p, int n_rows, cudaStream_t s) {
   if (p.D % 128 || p.r > 64 || p.k > 32) return false;
   const int ev = dtype == 0 ? 16 : 8;   // bytes of a 4-element vector in the model dtype
-  if (!al(p.x1, 16) || !al(p.y, 16) || !al(p.h, 16) || !al(p.h_state, 16) || !al(p.h_out, 16) || !al(p.A, 16) ||
+  if (!al(p.x1, 16) || !al(p.y, ev) || !al(p.h, 16) || !al(p.h_state, 16) || !al(p.h_out, 16) || !al(p.A, 16) ||
       !al(p.inj_B, 16) || !al(p.e, ev) || (p.act_on && !al(p.halt_wv, 16)) || (p.out && !al(p.out, 16)) ||
       (p.r > 0 && (!al(p.lora_down, ev) || !al(p.lora_B, ev))))
+    return false;
+  if (p.next_emb && (p.loop_dim % 4 || !al(p.next_emb, 16) || !al(p.w_rec, 16) || !al(p.w_attn, 16) ||
+                     !al(p.combined_out, 16) || !al(p.a_out, ev)))
     return false;
   const int vpl = p.D / 128;
   const unsigned blocks = (unsigned)((n_rows + 7) / 8);

@@ -117,8 +117,8 @@ __global__ void __launch_bounds__(256) k_gemm_simt(GemmParams p) {
           ((float*)p.C)[r * p.ldc + c] = p.resid[r * p.ld_resid + c] + v;
         } else if (EPI == EPI_SWIGLU_T) {
           ((TC*)p.C)[r * p.ldc + c] = from_f<TC>(silu_f(v) * acu[i][j]);
-        } else if (EPI == EPI_GATE_F32) {
-          ((float*)p.C)[r * p.ldc + c] = p.row_scale[r] * v;
+        } else if (EPI == EPI_GATE_T) {
+          ((TC*)p.C)[r * p.ldc + c] = from_f<TC>(p.row_scale[r] * v);
         }
       }
     }
@@ -135,7 +135,7 @@ int launch_gemm_simt(int dtype, int epi, const GemmParams& p, cudaStream_t s) {
     case EPI_RESID_F32: { k_gemm_simt<TA, float, EPI_RESID_F32><<<grid, 256, 0, s>>>(p); note_launch(); } break; \
     case EPI_ROPE_T: { k_gemm_simt<TA, TO, EPI_ROPE_T><<<grid, 256, 0, s>>>(p); note_launch(); } break;          \
     case EPI_SWIGLU_T: { k_gemm_simt<TA, TO, EPI_SWIGLU_T><<<grid, 256, 0, s>>>(p); note_launch(); } break;      \
-    case EPI_GATE_F32: { k_gemm_simt<TA, float, EPI_GATE_F32><<<grid, 256, 0, s>>>(p); note_launch(); } break;   \
+    case EPI_GATE_T: { k_gemm_simt<TA, TO, EPI_GATE_T><<<grid, 256, 0, s>>>(p); note_launch(); } break;   \
     default: return -1;                                                                    \
   }
   if (dtype == 0) { RDT_SIMT_CASE(float, float) } else { RDT_SIMT_CASE(bf16, bf16) }

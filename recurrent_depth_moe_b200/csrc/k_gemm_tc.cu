@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(192, 1)
           if (valid) store_bf16x32((bf16*)p.C + r * p.ldc + ti.n0 + c, g);
         }
       } else {
-        const float rs = (EPI == EPI_GATE_F32 && valid) ? p.row_scale[r] : 0.f;
+        const float rs = (EPI == EPI_GATE_T && valid) ? p.row_scale[r] : 0.f;
         const int pos = (EPI == EPI_ROPE_T && valid) ? p.pos[r] : 0;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -282,6 +282,10 @@ __global__ void __launch_bounds__(192, 1)
           if (!valid) continue;
           const int col = ti.n0 + c;
           if (EPI == EPI_STORE_T) {
+            store_bf16x32((bf16*)p.C + r * p.ldc + col, v);
+          } else if (EPI == EPI_GATE_T) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) v[q] *= rs;
             store_bf16x32((bf16*)p.C + r * p.ldc + col, v);
           } else if (EPI == EPI_ROPE_T) {
             const int m0 = rope_chunk(p, col);
@@ -316,10 +320,6 @@ __global__ void __launch_bounds__(192, 1)
                 float4 a = rs4[q];
                 ((float4*)dst)[q] = make_float4(a.x + v[4 * q], a.y + v[4 * q + 1], a.z + v[4 * q + 2], a.w + v[4 * q + 3]);
               }
-            } else if (EPI == EPI_GATE_F32) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                ((float4*)dst)[q] = make_float4(rs * v[4 * q], rs * v[4 * q + 1], rs * v[4 * q + 2], rs * v[4 * q + 3]);
             } else {
 #pragma unroll
               for (int q = 0; q < 8; ++q)
@@ -439,7 +439,7 @@ bool gemm_tc_supports(const GemmParams& p, int epi) {
   if (p.K < tc::BK || p.K % tc::BK) return false;
   if (!pick_bn(p, epi)) return false;
   if (p.lda % 8 || p.ldb % 8 || !al16(p.A) || !al16(p.B) || !al16(p.C)) return false;
-  if (epi == EPI_STORE_F32 || epi == EPI_RESID_F32 || epi == EPI_GATE_F32 || epi == EPI_ROUTER) {
+  if (epi == EPI_STORE_F32 || epi == EPI_RESID_F32 || epi == EPI_ROUTER) {
     if (p.ldc % 4) return false;
   } else if (p.ldc % 8) {
     return false;
@@ -488,7 +488,7 @@ int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
     case EPI_RESID_F32: rc = launch_tc_bn<EPI_RESID_F32>(bn, mA, mB, a, grid, s); break;
     case EPI_ROPE_T: rc = launch_tc_bn<EPI_ROPE_T>(bn, mA, mB, a, grid, s); break;
     case EPI_SWIGLU_T: rc = launch_tc<EPI_SWIGLU_T, 256>(mA, mB, a, grid, s); break;
-    case EPI_GATE_F32: rc = launch_tc_bn<EPI_GATE_F32>(bn, mA, mB, a, grid, s); break;
+    case EPI_GATE_T: rc = launch_tc_bn<EPI_GATE_T>(bn, mA, mB, a, grid, s); break;
     case EPI_ROUTER: rc = (bn == 64) ? launch_tc<EPI_ROUTER, 64>(mA, mB, a, grid, s)
                                      : launch_tc<EPI_ROUTER, 128>(mA, mB, a, grid, s); break;
     default: return -1;

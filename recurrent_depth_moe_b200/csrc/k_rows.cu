@@ -200,8 +200,8 @@ __global__ void k_combine_inject_act(CombineParams p) {
         if (threadIdx.x == 0) record_status(p.st, ST_BOUNDS, 201, slot);
         continue;
       }
-      const float* yr = p.y + (long long)slot * D;
-      for (int d = threadIdx.x; d < D; d += blockDim.x) tr[d] += yr[d];
+      const T* yr = (const T*)p.y + (long long)slot * D;
+      for (int d = threadIdx.x; d < D; d += blockDim.x) tr[d] += to_f(yr[d]);
     }
   }
   __syncthreads();
@@ -358,8 +358,13 @@ void launch_loop_prologue(int dtype, const float* h, const void* e, const float*
     { k_loop_prologue<bf16><<<N, nthreads_for(D), smem, s>>>(h, (const bf16*)e, emb, loop_dim, w_rec, w_attn,
                                                           combined, (bf16*)a, D, eps); note_launch(); }
 }
+bool launch_rmsnorm_warp(int dtype, const float* x, const float* w, void* out, int N, int D, float eps,
+                         cudaStream_t s);
+
 void launch_rmsnorm(int in_f32, int dtype, const void* x, long long in_ld, const float* w, void* out,
                     long long out_ld, int rows, int D, float eps, cudaStream_t s) {
+  if (in_f32 && in_ld == D && out_ld == D && launch_rmsnorm_warp(dtype, (const float*)x, w, out, rows, D, eps, s))
+    return;
   size_t smem = (size_t)D * sizeof(float);
   int nt = nthreads_for(D);
   if (in_f32) {
@@ -389,12 +394,13 @@ void launch_kv_to_cache(int dtype, const void* qkv, long long ld, int k_col, int
 }
 bool launch_combine_warp(int dtype, const CombineParams& p, int n_rows, cudaStream_t s);
 
-void launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s) {
-  if (launch_combine_warp(dtype, p, n_rows, s)) return;
+bool launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s) {
+  if (launch_combine_warp(dtype, p, n_rows, s)) return p.next_emb != nullptr;
   size_t smem = (size_t)(p.D + 64) * sizeof(float);
   int nt = nthreads_for(p.D);
   if (dtype == 0) { k_combine_inject_act<float><<<n_rows, nt, smem, s>>>(p); note_launch(); }
   else { k_combine_inject_act<bf16><<<n_rows, nt, smem, s>>>(p); note_launch(); }
+  return false;
 }
 void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* n_run, cudaStream_t s) {
   { k_compact<<<1, 1024, 0, s>>>(halted, N, run_list, run_idx, n_run); note_launch(); }

@@ -31,7 +31,7 @@ enum Epi {
   EPI_RESID_F32 = 2,   // C fp32 = resid + acc
   EPI_ROPE_T = 3,      // C model dtype = RoPE(acc) on the described column ranges
   EPI_SWIGLU_T = 4,    // C model dtype = silu(acc(B rows c)) * acc(B rows up_off + c)
-  EPI_GATE_F32 = 5,    // C fp32 = row_scale[row] * acc
+  EPI_GATE_T = 5,      // C model dtype = row_scale[row] * acc
   EPI_ROUTER = 6       // C fp32 = logits; plus softmax / biased top-k / gates / expert histogram
 };
 
@@ -116,7 +116,7 @@ struct CombineParams {
   int N, D, k, S, r, t, n_loops, max_loop_iters, max_slots;
   int act_on, transformer_off, block_only;
   float thr;
-  const float* x1; const float* y; const int* slot_of; const int* ids;
+  const float* x1; const void* y; const int* slot_of; const int* ids;   // y in the model dtype
   const void* lora_down; const void* lora_B; const float* lora_scale;
   const float* A; const float* inj_B; const void* e;
   const float* h; float* h_state; float* h_out;
@@ -124,6 +124,10 @@ struct CombineParams {
   float* cum; int* halted;
   float* halt_w_out; int* ids_out; float* p_out;
   float* out;   // block_only
+  // fused prologue of loop t + 1 (warp-per-row kernel only; next_emb == nullptr: off):
+  // combined = RMSNorm_rec(h_new + emb + e), a = RMSNorm_attn(combined)
+  const float* next_emb; int loop_dim; const float* w_rec; const float* w_attn; float eps;
+  float* combined_out; void* a_out;
   DevStatus* st;
 };
 
@@ -142,7 +146,8 @@ void launch_mla_kv_prep(int dtype, const float* kv_raw, int kvr, int dr, const f
 void launch_kv_to_cache(int dtype, const void* qkv, long long ld, int k_col, int v_col, int Hkv, int hd,
                         const int* pos, int N, int seq, int t_max, void* kc, void* vc, DevStatus* st,
                         cudaStream_t s);
-void launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s);
+// returns true when the fused next-loop prologue ran (p.next_emb set and supported)
+bool launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s);
 void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* n_run, cudaStream_t s);
 void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s);
 void launch_embed(int dtype, const void* table, int vocab, const int* ids, int n, int D, float* out,

@@ -105,7 +105,7 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
   L->gate_of = take(M * 4);
   L->xg = take(M * D * es);
   L->u = take(M * (size_t)F * es);
-  L->y = take(M * D * 4);
+  L->y = take(M * D * es);   // gate-scaled expert outputs, model dtype
   L->run_list = take(N * 4);
   L->run_idx = take(N * 4);
   L->nrun = take(16);
@@ -113,7 +113,7 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
   L->halted = take(N * 4);
   L->p_buf = take(N * 4);
   L->Avec = take(D * 4);
-  L->emb = take((size_t)std::max(c->loop_dim, 2) * 4);
+  L->emb = take((size_t)2 * std::max(c->loop_dim, 2) * 4);   // loop embeddings of loops t and t + 1
   L->rope_pos = std::max(max_keys, T);
   L->rope = take((size_t)L->rope_pos * (L->rope_dim / 2) * 8);
   L->pos = take(N * 4);
@@ -277,9 +277,9 @@ rdt_status moe_block(Ctx& x, int N, const float* x1) {
   GemmParams dn = gemm_base(x);
   dn.A = up.C; dn.lda = F; dn.B = w->w2; dn.ldb = F; dn.b_group_stride = (long long)D * F;
   dn.M = x.L.max_slots; dn.N = D; dn.K = F; dn.b_rows = (long long)(E + S) * D; dn.tiles = rp.tiles; dn.n_tiles = rp.n_tiles; dn.max_tiles = x.L.max_tiles;
-  dn.C = at<float*>(x.ws, x.L.y); dn.ldc = D; dn.row_scale = rp.gate_of;
+  dn.C = at<void*>(x.ws, x.L.y); dn.ldc = D; dn.row_scale = rp.gate_of;
   // both expert GEMMs consume the same tile list, so they must share one tile height
-  GemmImpl iu = gemm_pick(x.dtype, up, EPI_SWIGLU_T), id = gemm_pick(x.dtype, dn, EPI_GATE_F32);
+  GemmImpl iu = gemm_pick(x.dtype, up, EPI_SWIGLU_T), id = gemm_pick(x.dtype, dn, EPI_GATE_T);
   if (iu != id) iu = id = GEMM_SIMT;
   up.impl = dn.impl = (int)iu;
   rp.tile_m = gemm_tile_m(iu);
@@ -298,7 +298,7 @@ rdt_status moe_block(Ctx& x, int N, const float* x1) {
     launch_route_scatter(x.dtype, rp, x.s);
   }
   { ProfScope ps(PC_EXPERT_UP, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_SWIGLU_T, up, x.s)); }
-  { ProfScope ps(PC_EXPERT_DOWN, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_GATE_F32, dn, x.s)); }
+  { ProfScope ps(PC_EXPERT_DOWN, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_GATE_T, dn, x.s)); }
   return RDT_OK;
 }
 
@@ -309,7 +309,7 @@ CombineParams combine_base(Ctx& x, int N) {
   memset(&cp, 0, sizeof(cp));
   cp.N = N; cp.D = c->dim; cp.k = c->top_k; cp.S = c->n_shared_experts; cp.r = c->lora_rank;
   cp.max_loop_iters = c->max_loop_iters; cp.max_slots = x.L.max_slots;
-  cp.x1 = at<float*>(x.ws, x.L.x1); cp.y = at<float*>(x.ws, x.L.y); cp.slot_of = at<int*>(x.ws, x.L.slot_of);
+  cp.x1 = at<float*>(x.ws, x.L.x1); cp.y = at<void*>(x.ws, x.L.y); cp.slot_of = at<int*>(x.ws, x.L.slot_of);
   cp.ids = at<int*>(x.ws, x.L.ids);
   cp.lora_down = w->lora_down; cp.lora_B = w->lora_B; cp.lora_scale = w->lora_scale;
   cp.A = at<float*>(x.ws, x.L.Avec); cp.inj_B = w->inj_B;
@@ -390,14 +390,19 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
   cp.n_loops = n_loops; cp.act_on = act_on; cp.thr = thr; cp.e = e; cp.h_out = h_out;
   cp.halt_off = halt_off; cp.halt_w_out = halt_weights; cp.ids_out = expert_ids;
   cp.transformer_off = transformer_off;
+  cp.loop_dim = c->loop_dim; cp.w_rec = w->rec_norm_w; cp.w_attn = w->attn_norm_w; cp.eps = c->norm_eps;
+  cp.combined_out = combined; cp.a_out = a;
+  const int emb_stride = std::max(c->loop_dim, 2);
+  bool prologue_done = false;   // set when the previous loop's combine kernel computed this loop's prologue
   for (int t = 0; t < n_loops; ++t) {
+    float* emb_t = emb + (size_t)(t & 1) * emb_stride;
     if (trace && trace->h_in)
       launch_trace_rows(0, x.dtype, h, D, trace->row0, trace->n_rows, nullptr,
                         trace->h_in + (size_t)t * trace->n_rows * D, s);
-    {
+    if (!prologue_done) {
       ProfScope ps(PC_PROLOGUE, s);
-      launch_loop_emb(emb, c->loop_dim, t, c->loop_theta, s);
-      launch_loop_prologue(x.dtype, h, e, emb, c->loop_dim, w->rec_norm_w, w->attn_norm_w, combined, a, N, D,
+      launch_loop_emb(emb_t, c->loop_dim, t, c->loop_theta, s);
+      launch_loop_prologue(x.dtype, h, e, emb_t, c->loop_dim, w->rec_norm_w, w->attn_norm_w, combined, a, N, D,
                            c->norm_eps, s);
     }
     if (!transformer_off) {
@@ -411,7 +416,14 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
                           trace->biased_logits + (size_t)t * trace->n_rows * E, s);
     }
     cp.t = t;
-    { ProfScope ps(PC_COMBINE, s); launch_combine(x.dtype, cp, N, s); }
+    cp.next_emb = nullptr;
+    if (t + 1 < n_loops && c->loop_dim >= 0) {
+      // the combine kernel of loop t also produces combined / a of loop t + 1
+      float* emb_n = emb + (size_t)((t + 1) & 1) * emb_stride;
+      launch_loop_emb(emb_n, c->loop_dim, t + 1, c->loop_theta, s);
+      cp.next_emb = emb_n;
+    }
+    { ProfScope ps(PC_COMBINE, s); prologue_done = launch_combine(x.dtype, cp, N, s); }
     if (trace && trace->p && act_on)
       launch_trace_rows(0, x.dtype, at<float*>(ws, x.L.p_buf), 1, trace->row0, trace->n_rows, nullptr,
                         trace->p + (size_t)t * trace->n_rows, s);
