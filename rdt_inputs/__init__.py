@@ -150,6 +150,11 @@ WORKLOADS = {
         dim=512, n_heads=4, n_kv_heads=1, max_seq_len=512, max_loop_iters=2,
         n_experts=128, n_shared_experts=1, n_experts_per_tok=8, expert_dim=128, lora_rank=16,
         dtype="bf16"), batch=1, seq=300, n_loops=2, seed=7, act_threshold=0.9),
+    # Test-only: several query-tile pairs with a ragged last tile (tensor-core attention), GQA group 4.
+    "mid_t392_bf16": Workload("mid_t392_bf16", RDTConfig(
+        dim=512, n_heads=4, n_kv_heads=1, max_seq_len=512, max_loop_iters=2,
+        n_experts=8, n_shared_experts=1, n_experts_per_tok=2, expert_dim=128, lora_rank=8,
+        dtype="bf16"), batch=2, seq=392, n_loops=2, seed=8, act_threshold=0.99),
     "mid_gqa_fp32": Workload("mid_gqa_fp32", RDTConfig(
         dim=512, n_heads=4, n_kv_heads=2, max_seq_len=512, max_loop_iters=2,
         n_experts=8, n_shared_experts=1, n_experts_per_tok=2, expert_dim=256, lora_rank=8,

@@ -1,20 +1,21 @@
 // Causal GQA prefill attention on the sm_100a tensor cores (S3 of the recurrent block),
 // head dim 128, bf16 operands, fp32 softmax and accumulation.
 //
-// One CTA per (sequence, head, 128-query tile), heaviest tiles first.
-//   warp 0      TMA: Q once; K and V^T tiles of 128 keys into a 2-stage ring
-//   warp 1      TMEM owner; lane 0 issues  S_j = Q K_j^T  (into one of two TMEM S
-//               buffers, so QK^T of tile j+1 overlaps the softmax of tile j) and
-//               O += P_j V_j  (TMEM O accumulator)
-//   warps 2..5  softmax: thread = query row = TMEM lane.  Reads its S row, masks
-//               (key j visible iff key_pos0 + j <= q_pos, "OpenMythos 분석", Core
-//               Structure causal mask), keeps a running max m and sum l in the log2
-//               domain, writes P = exp2(s - m) as bf16 into 128B-swizzled shared
-//               memory (the A operand of the PV MMA).  The running max is raised only
-//               when it grows by more than 2^8, and only then is the O row rescaled in
-//               TMEM, so probabilities stay <= 256 and most tiles skip the rescale.
-// V is consumed transposed (V^T[b][g][dim][t], written by the QKV GEMM epilogue) so
-// both MMAs read K-major operands.  Every wait is bounded (RDT_ERR_DEVICE_TIMEOUT).
+// One CTA per (sequence, head, pair of 128-query tiles), heaviest pairs first.
+//   warp 0      TMA: both Q tiles once; K and V^T tiles of 64 keys into a 3-stage ring
+//   warp 1      TMEM owner; lane 0 issues, per key tile j and query tile q,
+//               S_qj = Q_q K_j^T (two TMEM S buffers per query tile) and
+//               O_q += P_qj V_j (one TMEM O accumulator per query tile)
+//   warps 2..5  softmax of query tile 0; warps 6..9 softmax of query tile 1.
+//               Thread = query row = TMEM lane: reads its S row, masks (key j visible
+//               iff key_pos0 + j <= q_pos, "OpenMythos 분석", Core Structure causal
+//               mask), keeps a running max m and sum l in the log2 domain, writes
+//               P = exp2(s - m) as bf16 into 128B-swizzled shared memory (the A operand
+//               of the PV MMA).  The running max is raised only when it grows by more
+//               than 2^8, and only then is the O row rescaled in TMEM.
+// The two query tiles share every K / V tile and their softmax groups overlap each
+// other and the tensor core.  V is consumed transposed (V^T[b][g][dim][t], written by
+// the QKV GEMM epilogue) so both MMAs read K-major operands.  Every wait is bounded.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_common.cuh"
@@ -23,16 +24,20 @@ namespace rdt {
 
 bool tc_make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsigned long long cols,
                  unsigned long long ld, unsigned box_rows);
-int tc_sm_count();
 
 namespace fat {
 
-constexpr int BQ = 128, BKV = 128, HD = 128;
-constexpr int TILE = 128 * 128 * 2;   // 32 KB: two 64-column swizzle atoms of 16 KB
-constexpr int HALF = TILE / 2;
-constexpr int SMEM = TILE /*Q*/ + 2 * TILE /*K*/ + 2 * TILE /*V^T*/ + TILE /*P*/ + 1024 + 256;
-constexpr int TMEM_COLS = 512;        // S0 [0,128), S1 [128,256), O [256,384)
-constexpr float RESCALE_LOG2 = 8.f;   // lazy rescale threshold (factor 256)
+constexpr int BQ = 128, BKV = 64, HD = 128, NQ = 2, STAGES = 3;
+constexpr int QTILE = BQ * HD * 2;      // 32 KB: two 64-dim swizzle atoms of 16 KB
+constexpr int QHALF = QTILE / 2;
+constexpr int KTILE = BKV * HD * 2;     // 16 KB: two atoms [64 keys][64 dims] of 8 KB
+constexpr int KHALF = KTILE / 2;
+constexpr int VTILE = HD * BKV * 2;     // 16 KB: one atom [128 dims][64 keys]
+constexpr int PTILE = BQ * BKV * 2;     // 16 KB: one atom [128 queries][64 keys]
+constexpr int SMEM = NQ * QTILE + STAGES * (KTILE + VTILE) + NQ * PTILE + 1024 + 512;
+constexpr int TMEM_COLS = 512;          // S[q][buf] at (2q + buf) * 64; O[q] at 256 + 128 q
+constexpr float RESCALE_LOG2 = 8.f;     // lazy rescale threshold (factor 256)
+constexpr int THREADS = 64 + NQ * 128;
 
 struct Args {
   int B, T, H, G, Hkv;
@@ -42,52 +47,65 @@ struct Args {
   bf16* o;
   long long o_row;         // output row stride (elements); head h at column h * 128
   int q_col0, k_col0;      // qkv columns of query head 0 and key head 0
-  DevStatus* st;
 };
 
 using namespace rdt::tc;
 
-__global__ void __launch_bounds__(192, 1)
-    k_attn_tc(const __grid_constant__ CUtensorMap tmQK, const __grid_constant__ CUtensorMap tmVt, const Args a) {
+__device__ __forceinline__ int visible_tiles(const Args& a, long long row_last, int q_rows) {
+  if (q_rows <= 0) return 0;
+  int n_vis = min(a.n_keys, a.q_pos[row_last] - a.key_pos0 + 1);
+  return n_vis > 0 ? (n_vis + BKV - 1) / BKV : 0;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmVt, const Args a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + TILE;            // 2 stages
-  uint8_t* sV = sK + 2 * TILE;        // 2 stages
-  uint8_t* sP = sV + 2 * TILE;
-  uint64_t* bars = (uint64_t*)(sP + TILE);
+  uint8_t* sQ = smem;                          // [NQ] query tiles
+  uint8_t* sK = sQ + NQ * QTILE;               // [STAGES]
+  uint8_t* sV = sK + STAGES * KTILE;           // [STAGES]
+  uint8_t* sP = sV + STAGES * VTILE;           // [NQ]
+  uint64_t* bars = (uint64_t*)(sP + NQ * PTILE);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;       // [2]
-  uint64_t* kv_empty = bars + 3;      // [2]
-  uint64_t* s_full = bars + 5;        // [2]
-  uint64_t* p_full = bars + 7;
-  uint64_t* pv_done = bars + 8;
-  uint64_t* done = bars + 9;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 10);
+  uint64_t* kv_full = bars + 1;                // [STAGES]
+  uint64_t* kv_empty = kv_full + STAGES;       // [STAGES]
+  uint64_t* s_full = kv_empty + STAGES;        // [NQ][2]
+  uint64_t* p_full = s_full + 2 * NQ;          // [NQ]
+  uint64_t* pv_done = p_full + NQ;             // [NQ]
+  uint64_t* done = pv_done + NQ;
+  uint32_t* tmem_slot = (uint32_t*)(done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int n_qt = (a.T + BQ - 1) / BQ;
+  const int n_pairs = (n_qt + NQ - 1) / NQ;
   const int BH = a.B * a.H;
-  const int qt = n_qt - 1 - (int)(blockIdx.x / BH);
+  const int pair = n_pairs - 1 - (int)(blockIdx.x / BH);    // heaviest pairs first
   const int bh = blockIdx.x % BH;
   const int b = bh / a.H, h = bh % a.H, g = h / a.G;
-  const int q0 = qt * BQ;
-  const int q_rows = min(BQ, a.T - q0);
-  const long long row0 = (long long)b * a.T + q0;
-  int n_vis = min(a.n_keys, a.q_pos[row0 + q_rows - 1] - a.key_pos0 + 1);
-  if (n_vis < 0) n_vis = 0;
-  const int nt = (n_vis + BKV - 1) / BKV;
+  int q0[NQ], q_rows[NQ], nt[NQ];
+  int nt_max = 0;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    q0[q] = (pair * NQ + q) * BQ;
+    q_rows[q] = max(0, min(BQ, a.T - q0[q]));
+    nt[q] = visible_tiles(a, (long long)b * a.T + q0[q] + q_rows[q] - 1, q_rows[q]);
+    nt_max = max(nt_max, nt[q]);
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
-      mbar_init(&s_full[s], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
+    for (int q = 0; q < NQ; ++q) {
+      mbar_init(&s_full[2 * q], 1);
+      mbar_init(&s_full[2 * q + 1], 1);
+      mbar_init(&p_full[q], 128);
+      mbar_init(&pv_done[q], 1);
+    }
     mbar_init(done, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -105,92 +123,112 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
-    mbar_expect_tx(q_full, TILE);
+    int qbytes = 0;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) qbytes += q_rows[q] > 0 ? QTILE : 0;
+    mbar_expect_tx(q_full, qbytes);
     const int qx = a.q_col0 + h * HD;
-    tma_load_2d(sQ, &tmQK, q_full, qx, (int)row0);
-    tma_load_2d(sQ + HALF, &tmQK, q_full, qx + 64, (int)row0);
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      if (q_rows[q] <= 0) continue;
+      const int qy = b * a.T + q0[q];
+      tma_load_2d(sQ + q * QTILE, &tmQ, q_full, qx, qy);
+      tma_load_2d(sQ + q * QTILE + QHALF, &tmQ, q_full, qx + 64, qy);
+    }
     const int kx = a.k_col0 + g * HD;
     const int vy = (b * a.Hkv + g) * HD;
-    for (int j = 0; j < nt; ++j) {
-      const int st = j & 1;
-      if (!mbar_wait(&kv_empty[st], ((j >> 1) & 1) ^ 1, abort_flag)) break;
-      mbar_expect_tx(&kv_full[st], 2 * TILE);
+    for (int j = 0; j < nt_max; ++j) {
+      const int st = j % STAGES;
+      if (!mbar_wait(&kv_empty[st], ((j / STAGES) & 1) ^ 1, abort_flag)) break;
+      mbar_expect_tx(&kv_full[st], KTILE + VTILE);
       const int ky = b * a.T + j * BKV;
-      tma_load_2d(sK + st * TILE, &tmQK, &kv_full[st], kx, ky);
-      tma_load_2d(sK + st * TILE + HALF, &tmQK, &kv_full[st], kx + 64, ky);
-      tma_load_2d(sV + st * TILE, &tmVt, &kv_full[st], j * BKV, vy);
-      tma_load_2d(sV + st * TILE + HALF, &tmVt, &kv_full[st], j * BKV + 64, vy);
+      tma_load_2d(sK + st * KTILE, &tmK, &kv_full[st], kx, ky);
+      tma_load_2d(sK + st * KTILE + KHALF, &tmK, &kv_full[st], kx + 64, ky);
+      tma_load_2d(sV + st * VTILE, &tmVt, &kv_full[st], j * BKV, vy);
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
-    constexpr uint32_t IDESC = idesc_bf16(128, 128);
-    const uint32_t tO = tmem + 256;
+    constexpr uint32_t IDESC_S = idesc_bf16(128, BKV);
+    constexpr uint32_t IDESC_O = idesc_bf16(128, HD);
     bool ok = mbar_wait(q_full, 0, abort_flag);
     auto issue_pv = [&](int jj) -> bool {
-      if (!mbar_wait(p_full, jj & 1, abort_flag)) return false;
-      tc_fence_after();
-      const int st = jj & 1;
+      const int st = jj % STAGES;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t ad = smem_desc(sP + (kk >> 2) * HALF) + 2 * (kk & 3);
-        const uint64_t bd = smem_desc(sV + st * TILE + (kk >> 2) * HALF) + 2 * (kk & 3);
-        umma_bf16(tO, ad, bd, IDESC, (jj > 0 || kk > 0) ? 1u : 0u);
+      for (int q = 0; q < NQ; ++q) {
+        if (jj >= nt[q]) continue;
+        if (!mbar_wait(&p_full[q], jj & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t tO = tmem + 256 + q * 128;
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          const uint64_t ad = smem_desc(sP + q * PTILE) + 2 * kk;
+          const uint64_t bd = smem_desc(sV + st * VTILE) + 2 * kk;
+          umma_bf16(tO, ad, bd, IDESC_O, (jj > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&pv_done[q]);
       }
-      umma_commit(pv_done);
       umma_commit(&kv_empty[st]);
       return true;
     };
-    for (int j = 0; j < nt && ok; ++j) {
-      const int st = j & 1;
-      if (!(ok = mbar_wait(&kv_full[st], (j >> 1) & 1, abort_flag))) break;
+    for (int j = 0; j < nt_max && ok; ++j) {
+      const int st = j % STAGES;
+      if (!(ok = mbar_wait(&kv_full[st], (j / STAGES) & 1, abort_flag))) break;
       tc_fence_after();
-      const uint32_t tS = tmem + st * 128;
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t ad = smem_desc(sQ + (kk >> 2) * HALF) + 2 * (kk & 3);
-        const uint64_t bd = smem_desc(sK + st * TILE + (kk >> 2) * HALF) + 2 * (kk & 3);
-        umma_bf16(tS, ad, bd, IDESC, kk > 0 ? 1u : 0u);
+      for (int q = 0; q < NQ; ++q) {
+        if (j >= nt[q]) continue;
+        const uint32_t tS = tmem + (2 * q + (j & 1)) * BKV;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint64_t ad = smem_desc(sQ + q * QTILE + (kk >> 2) * QHALF) + 2 * (kk & 3);
+          const uint64_t bd = smem_desc(sK + st * KTILE + (kk >> 2) * KHALF) + 2 * (kk & 3);
+          umma_bf16(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[2 * q + (j & 1)]);
       }
-      umma_commit(&s_full[st]);
       if (j >= 1) ok = issue_pv(j - 1);
     }
-    if (ok && nt > 0) issue_pv(nt - 1);
+    if (ok && nt_max > 0) issue_pv(nt_max - 1);
     umma_commit(done);
     mbar_wait(done, 0, abort_flag);
   } else if (warp >= 2) {
-    // ---------------- softmax ----------------
+    // ---------------- softmax of query tile q ----------------
+    const int q = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int rl = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const bool row_valid = rl < q_rows;
+    const long long row0 = (long long)b * a.T + q0[q];
+    const bool row_valid = rl < q_rows[q];
     const int my_pos = row_valid ? a.q_pos[row0 + rl] : -1;
+    const int n_vis = row_valid ? min(a.n_keys, a.q_pos[row0 + q_rows[q] - 1] - a.key_pos0 + 1) : 0;
+    const int ntq = nt[q];
+    const uint32_t tO = tmem + lane_base + 256 + q * 128;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint8_t* prow0 = sP + rl * 128;           // keys 0..63 of this row
-    uint8_t* prow1 = sP + HALF + rl * 128;    // keys 64..127
-    for (int j = 0; j < nt; ++j) {
-      const int st = j & 1;
-      if (!(ok = mbar_wait(&s_full[st], (j >> 1) & 1, abort_flag))) break;
+    uint8_t* prow = sP + q * PTILE + rl * 128;
+    for (int j = 0; j < ntq; ++j) {
+      if (!(ok = mbar_wait(&s_full[2 * q + (j & 1)], (j >> 1) & 1, abort_flag))) break;
       tc_fence_after();
-      float s[128];
+      float s[BKV];
 #pragma unroll
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; c < BKV; c += 32) {
         float v[32];
-        tmem_ld32(tmem + lane_base + st * 128 + c, v);
+        tmem_ld32(tmem + lane_base + (2 * q + (j & 1)) * BKV + c, v);
 #pragma unroll
-        for (int q = 0; q < 32; ++q) s[c + q] = v[q];
+        for (int e = 0; e < 32; ++e) s[c + e] = v[e];
       }
       const int k0 = j * BKV;
       const int kp0 = a.key_pos0 + k0;
       const bool need_mask = (kp0 + BKV - 1 > my_pos) || (k0 + BKV > n_vis);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < BKV; ++c)
+          if (kp0 + c > my_pos || k0 + c >= n_vis) s[c] = -INFINITY;
+      }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float x = s[c] * a.sl2;
-        if (need_mask && (kp0 + c > my_pos || k0 + c >= n_vis)) x = -INFINITY;
-        s[c] = x;
-        mx = fmaxf(mx, x);
-      }
+      for (int c = 0; c < BKV; ++c) mx = fmaxf(mx, s[c]);
+      mx *= a.sl2;                               // the scale is positive: max commutes with it
       float alpha = 1.f;
       if (j == 0) {
         m_used = mx;
@@ -200,12 +238,11 @@ __global__ void __launch_bounds__(192, 1)
         l *= alpha;
       }
       const float base = (m_used == -INFINITY) ? 0.f : m_used;
-      // P_j into registers (packed bf16) before the shared buffer is free again
-      uint32_t pk[64];
+      uint32_t pk[BKV / 2];
       float sum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = exp2f(s[c] - base), p1 = exp2f(s[c + 1] - base);
+      for (int c = 0; c < BKV; c += 2) {
+        const float p0 = exp2f(fmaf(s[c], a.sl2, -base)), p1 = exp2f(fmaf(s[c + 1], a.sl2, -base));
         sum += p0 + p1;
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[c >> 1] = *reinterpret_cast<uint32_t*>(&h2);
@@ -213,51 +250,50 @@ __global__ void __launch_bounds__(192, 1)
       l += sum;
       if (j >= 1) {
         // PV of tile j-1 done: O is stable and the P buffer is free
-        if (!(ok = mbar_wait(pv_done, (j - 1) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(&pv_done[q], (j - 1) & 1, abort_flag))) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < 128; c += 32) {
+          for (int c = 0; c < HD; c += 32) {
             float v[32];
-            tmem_ld32(tmem + lane_base + 256 + c, v);
+            tmem_ld32(tO + c, v);
 #pragma unroll
-            for (int q = 0; q < 32; ++q) v[q] *= alpha;
-            tmem_st32(tmem + lane_base + 256 + c, v);
+            for (int e = 0; e < 32; ++e) v[e] *= alpha;
+            tmem_st32(tO + c, v);
           }
           tmem_st_wait();
         }
       }
-      // 16-byte chunk c (8 keys) of a 128-byte row goes to chunk c ^ (row & 7)
+      // 16-byte chunk c (8 keys) of the 128-byte row goes to chunk c ^ (row & 7)
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint8_t* rowp = (c < 8) ? prow0 : prow1;
-        const int ch = (c & 7) ^ (rl & 7);
-        *reinterpret_cast<uint4*>(rowp + ch * 16) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      for (int c = 0; c < BKV / 8; ++c) {
+        const int ch = c ^ (rl & 7);
+        *reinterpret_cast<uint4*>(prow + ch * 16) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
       fence_async_smem();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[q]);
     }
     // final: O / l
-    if (ok && nt > 0 && mbar_wait(pv_done, (nt - 1) & 1, abort_flag)) {
+    if (ok && ntq > 0 && mbar_wait(&pv_done[q], (ntq - 1) & 1, abort_flag)) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       bf16* orow = a.o + (row0 + rl) * a.o_row + (long long)h * HD;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; c < HD; c += 32) {
         float v[32];
-        tmem_ld32(tmem + lane_base + 256 + c, v);
+        tmem_ld32(tO + c, v);
         if (row_valid) {
 #pragma unroll
-          for (int q = 0; q < 32; q += 8) {
+          for (int e0 = 0; e0 < 32; e0 += 8) {
             uint4 u;
             uint32_t* w = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(v[q + 2 * e] * inv, v[q + 2 * e + 1] * inv);
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(v[e0 + 2 * e] * inv, v[e0 + 2 * e + 1] * inv);
               w[e] = *reinterpret_cast<uint32_t*>(&h2);
             }
-            *reinterpret_cast<uint4*>(orow + c + q) = u;
+            *reinterpret_cast<uint4*>(orow + c + e0) = u;
           }
         }
       }
@@ -265,7 +301,6 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (*abort_flag && threadIdx.x == 0) record_status(a.st, ST_TIMEOUT, 601, blockIdx.x);
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
@@ -293,9 +328,11 @@ int launch_attention_tc(const AttnParams& p, cudaStream_t s) {
   const int Hkv = p.H / p.G;
   // Q and K live in the qkv rows [B*T, q_row]; k1 points at key head 0 inside those rows
   const long long k_col0 = ((const bf16*)p.k1 - (const bf16*)p.q);
-  CUtensorMap mQK, mVt;
-  if (!tc_make_map(&mQK, p.q, (unsigned long long)p.B * p.T, (unsigned long long)p.q_row, p.q_row, 128)) return -1;
-  if (!tc_make_map(&mVt, p.vt, (unsigned long long)p.B * Hkv * 128, (unsigned long long)p.T, p.vt_ld, 128))
+  CUtensorMap mQ, mK, mVt;
+  const unsigned long long rows = (unsigned long long)p.B * p.T;
+  if (!tc_make_map(&mQ, p.q, rows, (unsigned long long)p.q_row, p.q_row, fat::BQ)) return -1;
+  if (!tc_make_map(&mK, p.q, rows, (unsigned long long)p.q_row, p.q_row, fat::BKV)) return -1;
+  if (!tc_make_map(&mVt, p.vt, (unsigned long long)p.B * Hkv * fat::HD, (unsigned long long)p.T, p.vt_ld, fat::HD))
     return -1;
   fat::Args a;
   a.B = p.B; a.T = p.T; a.H = p.H; a.G = p.G; a.Hkv = Hkv;
@@ -303,10 +340,10 @@ int launch_attention_tc(const AttnParams& p, cudaStream_t s) {
   a.sl2 = p.scale * 1.4426950408889634f;
   a.o = (bf16*)p.o; a.o_row = p.o_row;
   a.q_col0 = 0; a.k_col0 = (int)k_col0;
-  a.st = nullptr;
-  const long long blocks = (long long)((p.T + fat::BQ - 1) / fat::BQ) * p.B * p.H;
+  const int n_qt = (p.T + fat::BQ - 1) / fat::BQ;
+  const long long blocks = (long long)((n_qt + fat::NQ - 1) / fat::NQ) * p.B * p.H;
   if (blocks <= 0) return 0;
-  { fat::k_attn_tc<<<(unsigned)blocks, 192, fat::SMEM, s>>>(mQK, mVt, a); note_launch(); }
+  { fat::k_attn_tc<<<(unsigned)blocks, fat::THREADS, fat::SMEM, s>>>(mQ, mK, mVt, a); note_launch(); }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -76,7 +76,7 @@ __device__ __forceinline__ void next_prologue(const CombineParams& p, float4 (&x
 }
 
 template <typename T, int VPL>
-__global__ void __launch_bounds__(256) k_combine_warp(CombineParams p) {
+__global__ void __launch_bounds__(256, (VPL >= 24 ? 1 : 2)) k_combine_warp(CombineParams p) {
   const int lane = threadIdx.x & 31;
   const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (i >= p.N) return;

@@ -125,7 +125,7 @@ STRONG = dict(attn_std=0.08, halt_w_std=0.2, lora_scale_std=1.0)   # peaky atten
 
 
 @pytest.mark.parametrize("variant", ["literal", "strong"])
-@pytest.mark.parametrize("name", ["tiny_mla_bf16", "mid_gqa_bf16", "mid_e64_bf16", "mid_e128_bf16"])
+@pytest.mark.parametrize("name", ["tiny_mla_bf16", "mid_gqa_bf16", "mid_e64_bf16", "mid_e128_bf16", "mid_t392_bf16"])
 def test_recurrent_bf16_matches_oracle(name, variant):
     wl, cfg, W, h0, e, B, T, L = _recurrent_case(name, **(STRONG if variant == "strong" else {}))
     thr = wl.act_threshold
