@@ -51,10 +51,17 @@ def peaks():
 
 def workload_desc(wl):
     c = wl.cfg
-    return (f"{wl.name}: 1B-shaped recurrent block prefill, dim {c.dim}, {c.n_heads} heads GQA ({c.n_kv_heads} kv), "
+    shape = {"rdt1b_prefill": "1B-shaped recurrent block prefill",
+             "rdt10b_prefill_zipf": "10B-shaped load-imbalanced recurrent block prefill"}.get(wl.name, wl.name)
+    extra = ""
+    if wl.zipf_s:
+        extra += f", Zipf(s={wl.zipf_s}) router bias"
+    if wl.halt_spread:
+        extra += f", halting spread over {wl.halt_spread[0]}-{wl.halt_spread[1]} loops"
+    return (f"{wl.name}: {shape}, dim {c.dim}, {c.n_heads} heads GQA ({c.n_kv_heads} kv), "
             f"{c.n_experts} routed + {c.n_shared_experts} shared SwiGLU experts top-{c.n_experts_per_tok}, "
             f"expert_dim {c.expert_dim}, lora_rank {c.lora_rank}, {wl.n_loops} loops, batch {wl.batch} x seq {wl.seq}, "
-            f"{c.dtype}, ACT {wl.act_threshold} (halting bias {wl.halt_b})")
+            f"{c.dtype}, ACT {wl.act_threshold} (halting bias {wl.halt_b}){extra}")
 
 
 class ClockSampler:
@@ -128,11 +135,32 @@ def oracle_sample(wl, W_cpu, h0, e, positions: int, loops: int):
     return positions * loops / dt, dt
 
 
+def workload_weights(wl, device):
+    """Weights of a prefill workload (Zipf router bias and halting spread where the
+    workload names them) and its per-position halting-logit offsets (or None)."""
+    cfg = wl.cfg
+    if wl.zipf_s or wl.halt_spread:
+        bias = RI.zipf_router_bias(cfg.n_experts, cfg.dim, wl.zipf_s, wl.seed) if wl.zipf_s else None
+        W = RI.block_weights(cfg, wl.seed, device=device, router_bias=bias,
+                             halt_w_std=0.0 if wl.halt_spread else None, halt_b=0.0 if wl.halt_spread else wl.halt_b)
+    else:
+        W = RI.block_weights(cfg, wl.seed, device=device, halt_b=wl.halt_b)
+    off = None
+    if wl.halt_spread:
+        off, _ = RI.halting_offsets_spread(wl.batch * wl.seq, wl.halt_spread[0], wl.halt_spread[1],
+                                           wl.act_threshold, wl.seed)
+        off = off.to(device)
+    return W, off
+
+
 def run_reference(args, wl, rank, world):
     if rank != 0:
         return
     torch.manual_seed(0)
-    W = RI.block_weights(wl.cfg, wl.seed, device="cpu", halt_b=wl.halt_b)
+    W, _ = workload_weights(wl, "cpu") if wl.cfg.n_experts <= 64 else (None, None)
+    if W is None:   # the 10B shape's expert weights (18 GB) do not fit a host sample
+        print(json.dumps({"impl": "reference", "unavailable": "10B-shaped weights exceed the host sample budget"}))
+        return
     h0, e = RI.recurrent_inputs(wl.cfg, 1, 64, wl.seed)
     pos, loops = 32, 4
     for _ in range(args.warmup):
@@ -167,7 +195,7 @@ def run_ours(args, wl, rank, world, local_rank):
     B, T, L = wl.batch, wl.seq, wl.n_loops
     N = B * T
     # weights: identical replica on every rank; inputs: a different batch per rank
-    W = RI.block_weights(cfg, wl.seed, device=dev, halt_b=wl.halt_b)
+    W, halt_off = workload_weights(wl, dev)
     h0, e = RI.recurrent_inputs(cfg, B, T, wl.seed + 101 * rank, device=dev)
     blk = R.RecurrentBlock(cfg, W)
     ws = blk.workspace(B, T, T)
@@ -177,7 +205,7 @@ def run_ours(args, wl, rank, world, local_rank):
     stream = torch.cuda.current_stream()
 
     def step():
-        blk.forward(h0, e, B, T, L, wl.act_threshold, out=out, workspace=ws)
+        blk.forward(h0, e, B, T, L, wl.act_threshold, halt_logit_offset=halt_off, out=out, workspace=ws)
 
     for _ in range(args.warmup):
         step()
@@ -231,7 +259,7 @@ def run_ours(args, wl, rank, world, local_rank):
     def e2e_step():
         h0_d.copy_(h0_h, non_blocking=True)
         e_d.copy_(e_h, non_blocking=True)
-        blk.forward(h0_d, e_d, B, T, L, wl.act_threshold, out=out, workspace=ws)
+        blk.forward(h0_d, e_d, B, T, L, wl.act_threshold, halt_logit_offset=halt_off, out=out, workspace=ws)
         for oh, od in zip(outs_h, out):
             oh.copy_(od, non_blocking=True)
 
@@ -252,7 +280,8 @@ def run_ours(args, wl, rank, world, local_rank):
 
     # host copy for the CPU-oracle baseline, then free the prefill workload before the
     # decode one (23 GB of weights and caches)
-    W_cpu = {k: v.cpu() for k, v in W.items()} if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and cfg.n_experts <= 64
+    W_cpu = {k: v.cpu() for k, v in W.items()} if want_cpu else None
     h0_c, e_c = h0[:64].cpu(), e[:64].cpu()
     del blk, ws, W, out, h0_d, e_d
     torch.cuda.empty_cache()
@@ -283,7 +312,7 @@ def run_ours(args, wl, rank, world, local_rank):
            "data": "synthetic (seeded N(0,0.02) weights, unit-RMS h0/e rows)",
            "config": {"workload": workload_desc(wl), "batch": B * world, "seq_len": T, "n_loops": L,
                       "parallelism": f"replicas x{world} (sequence-sharded, no collective)",
-                      "l2": "inputs larger than L2 (1.65 GB of expert weights + 0.5 GB activations per loop)"},
+                      "l2": f"inputs larger than L2 ({3 * cfg.dim * cfg.expert_dim * (cfg.n_experts + cfg.n_shared_experts) * 2 / 1e9:.2f} GB of expert weights streamed per loop)"},
            "executed_token_loops_per_step": executed * world,
            "roofline": roofline, "gpu_launches": launches,
            "kernel_ms_per_step": breakdown,
@@ -291,7 +320,7 @@ def run_ours(args, wl, rank, world, local_rank):
            "clocks": clk}
     if not args.no_decode:
         res["decode"] = decode_res
-    if world == 1 and not args.no_cpu_baseline:
+    if W_cpu is not None:
         pos, loops = 64, 8
         rate, dt = oracle_sample(wl, W_cpu, h0_c, e_c, pos, loops)
         res["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
@@ -401,6 +430,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=128)
+    ap.add_argument("--workload", default=WORKLOAD, choices=["rdt1b_prefill", "rdt10b_prefill_zipf"])
     ap.add_argument("--batch", type=int, default=None, help="override the sequences per step (small profiling cases)")
     ap.add_argument("--loops", type=int, default=None, help="override n_loops (small profiling cases)")
     args = ap.parse_args()
@@ -410,7 +440,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    wl = RI.get_workload(WORKLOAD)
+    wl = RI.get_workload(args.workload)
     if args.batch or args.loops:
         import dataclasses
         wl = dataclasses.replace(wl, batch=args.batch or wl.batch, n_loops=args.loops or wl.n_loops)

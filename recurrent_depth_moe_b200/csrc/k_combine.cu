@@ -14,6 +14,8 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#include <algorithm>
+
 namespace rdt {
 
 template <typename T> struct Vec4;
@@ -75,11 +77,20 @@ __device__ __forceinline__ void next_prologue(const CombineParams& p, float4 (&x
   }
 }
 
+// Plain 4-element load usable on shared or global memory (generic address).
+template <typename T> __device__ __forceinline__ float4 ld4(const T* p);
+template <> __device__ __forceinline__ float4 ld4<float>(const float* p) { return *reinterpret_cast<const float4*>(p); }
+template <> __device__ __forceinline__ float4 ld4<bf16>(const bf16* p) {
+  uint2 u = *reinterpret_cast<const uint2*>(p);
+  float2 fa = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.x));
+  float2 fb = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u.y));
+  return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+// One row (one warp) of S9; Wd / Bl point at the LoRA matrices (shared or global).
 template <typename T, int VPL>
-__global__ void __launch_bounds__(256, (VPL >= 24 ? 1 : 2)) k_combine_warp(CombineParams p) {
-  const int lane = threadIdx.x & 31;
-  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (i >= p.N) return;
+__device__ __forceinline__ void combine_row(const CombineParams& p, int i, int lane, float* z, const T* Wd,
+                                            const T* Bl) {
   const int D = p.D;
   const int kS = p.k + p.S;
   const long long rowD = (long long)i * D;
@@ -100,15 +111,26 @@ __global__ void __launch_bounds__(256, (VPL >= 24 ? 1 : 2)) k_combine_warp(Combi
   } else {
 #pragma unroll
     for (int j = 0; j < VPL; ++j) tr[j] = __ldg(reinterpret_cast<const float4*>(p.x1 + rowD + 4 * lane + 128 * j));
-    for (int s = 0; s < kS; ++s) {
-      const int slot = p.slot_of[(long long)i * kS + s];
-      if (slot < 0 || slot >= p.max_slots) {
-        if (lane == 0) record_status(p.st, ST_BOUNDS, 202, slot);
-        continue;
+    // slot rows two at a time, so two rows' loads are in flight per memory round trip
+    const int* so = p.slot_of + (long long)i * kS;
+    for (int s = 0; s < kS; s += 2) {
+      int s0 = so[s], s1 = (s + 1 < kS) ? so[s + 1] : -2;
+      if (s0 < 0 || s0 >= p.max_slots) {
+        if (lane == 0) record_status(p.st, ST_BOUNDS, 202, s0);
+        s0 = -1;
       }
-      const T* yr = (const T*)p.y + (long long)slot * D + 4 * lane;
+      if (s1 != -2 && (s1 < 0 || s1 >= p.max_slots)) {
+        if (lane == 0) record_status(p.st, ST_BOUNDS, 202, s1);
+        s1 = -1;
+      }
+      const T* y0 = (const T*)p.y + (long long)max(s0, 0) * D + 4 * lane;
+      const T* y1 = (const T*)p.y + (long long)max(s1, 0) * D + 4 * lane;
 #pragma unroll
-      for (int j = 0; j < VPL; ++j) tr[j] = f4_add(tr[j], Vec4<T>::load(yr + 128 * j));
+      for (int j = 0; j < VPL; ++j) {
+        const float4 a0 = s0 >= 0 ? Vec4<T>::load(y0 + 128 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 a1 = s1 >= 0 ? Vec4<T>::load(y1 + 128 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        tr[j] = f4_add(tr[j], f4_add(a0, a1));
+      }
     }
   }
   if (p.block_only) {
@@ -117,30 +139,27 @@ __global__ void __launch_bounds__(256, (VPL >= 24 ? 1 : 2)) k_combine_warp(Combi
     return;
   }
   if (!p.transformer_off && p.r > 0) {
-    const T* Wd = (const T*)p.lora_down;
-    const T* Bl = (const T*)p.lora_B;
     const float* sc = p.lora_scale + (long long)min(p.t, p.max_loop_iters - 1) * p.r;
-    __shared__ float zs[8][64];
-    float* z = zs[threadIdx.x >> 5];
     for (int q = 0; q < p.r; ++q) {
       float part = 0.f;
       const T* w = Wd + (long long)q * D + 4 * lane;
 #pragma unroll
-      for (int j = 0; j < VPL; ++j) part += f4_dot(tr[j], Vec4<T>::load(w + 128 * j));
+      for (int j = 0; j < VPL; ++j) part += f4_dot(tr[j], ld4<T>(w + 128 * j));
       part = warp_sum(part) * sc[q];
       if (lane == 0) z[q] = part;
     }
     __syncwarp();
     // every z_q is complete, so the delta can be added to the row in place
     for (int q = 0; q < p.r; ++q) {
-      const T* b = Bl + (long long)q * D + 4 * lane;
+      const T* bq = Bl + (long long)q * D + 4 * lane;
       const float zq = z[q];
 #pragma unroll
       for (int j = 0; j < VPL; ++j) {
-        float4 v = Vec4<T>::load(b + 128 * j);
+        float4 v = ld4<T>(bq + 128 * j);
         tr[j].x += zq * v.x; tr[j].y += zq * v.y; tr[j].z += zq * v.z; tr[j].w += zq * v.w;
       }
     }
+    __syncwarp();
   }
   // h_new = A h + B e + trans (in place in tr)
   const T* er = (const T*)p.e + rowD + 4 * lane;
@@ -193,6 +212,34 @@ __global__ void __launch_bounds__(256, (VPL >= 24 ? 1 : 2)) k_combine_warp(Combi
   if (p.next_emb) next_prologue<T, VPL>(p, tr, rowD, lane);
 }
 
+// Persistent: WARPS warps per CTA, one CTA per SM, rows strided over the grid.  With
+// LSMEM the LoRA matrices (2 r D elements) are staged in shared memory once per CTA,
+// so the rank-r projections read shared memory instead of making 2 r round trips to L2.
+template <typename T, int VPL, int WARPS, bool LSMEM>
+__global__ void __launch_bounds__(WARPS * 32, 1) k_combine_warp(CombineParams p) {
+  extern __shared__ __align__(16) uint8_t csm[];
+  __shared__ float zs[WARPS][64];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const T* Wd = (const T*)p.lora_down;
+  const T* Bl = (const T*)p.lora_B;
+  if (LSMEM && p.r > 0 && !p.transformer_off && !p.block_only) {
+    const size_t bytes = (size_t)p.r * p.D * sizeof(T);
+    const int4* gs0 = reinterpret_cast<const int4*>(p.lora_down);
+    const int4* gs1 = reinterpret_cast<const int4*>(p.lora_B);
+    int4* d0 = reinterpret_cast<int4*>(csm);
+    int4* d1 = reinterpret_cast<int4*>(csm + bytes);
+    for (size_t v = threadIdx.x; v < bytes / 16; v += blockDim.x) {
+      d0[v] = __ldg(gs0 + v);
+      d1[v] = __ldg(gs1 + v);
+    }
+    __syncthreads();
+    Wd = reinterpret_cast<const T*>(csm);
+    Bl = reinterpret_cast<const T*>(csm + bytes);
+  }
+  for (int i = blockIdx.x * WARPS + warp; i < p.N; i += gridDim.x * WARPS)
+    combine_row<T, VPL>(p, i, lane, zs[warp], Wd, Bl);
+}
+
 // out = RMSNorm(x) * w for fp32 rows of width D = 128 * VPL, one warp per row.
 template <typename T, int VPL>
 __global__ void __launch_bounds__(256) k_rmsnorm_warp(const float* __restrict__ x, const float* __restrict__ w,
@@ -237,6 +284,39 @@ bool launch_rmsnorm_warp(int dtype, const float* x, const float* w, void* out, i
 #undef RDT_RW
 }
 
+int combine_sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <typename T, int VPL>
+bool launch_combine_vpl(const CombineParams& p, int n_rows, cudaStream_t s) {
+  constexpr int WARPS = VPL >= 24 ? 8 : 16;
+  const size_t lbytes = (size_t)2 * p.r * p.D * sizeof(T);
+  const bool lsmem = p.r > 0 && lbytes <= 160 * 1024 && (((size_t)p.r * p.D * sizeof(T)) % 16) == 0 &&
+                     ((uintptr_t)p.lora_down % 16) == 0 && ((uintptr_t)p.lora_B % 16) == 0;
+  const int grid = std::max(1, std::min((n_rows + WARPS - 1) / WARPS, combine_sm_count()));
+  if (lsmem) {
+    static bool attr = false;
+    if (!attr) {
+      if (cudaFuncSetAttribute(k_combine_warp<T, VPL, WARPS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               160 * 1024) != cudaSuccess)
+        return false;
+      attr = true;
+    }
+    { k_combine_warp<T, VPL, WARPS, true><<<grid, WARPS * 32, lbytes, s>>>(p); note_launch(); }
+  } else {
+    { k_combine_warp<T, VPL, WARPS, false><<<grid, WARPS * 32, 0, s>>>(p); note_launch(); }
+  }
+  return true;
+}
+
 bool launch_combine_warp(int dtype, const CombineParams& p, int n_rows, cudaStream_t s) {
   if (p.D % 128 || p.r > 64 || p.k > 32) return false;
   const int ev = dtype == 0 ? 16 : 8;   // bytes of a 4-element vector in the model dtype
@@ -247,14 +327,10 @@ bool launch_combine_warp(int dtype, const CombineParams& p, int n_rows, cudaStre
   if (p.next_emb && (p.loop_dim % 4 || !al(p.next_emb, 16) || !al(p.w_rec, 16) || !al(p.w_attn, 16) ||
                      !al(p.combined_out, 16) || !al(p.a_out, ev)))
     return false;
-  const int vpl = p.D / 128;
-  const unsigned blocks = (unsigned)((n_rows + 7) / 8);
-#define RDT_CW(V)                                                                                   \
-  case V:                                                                                           \
-    if (dtype == 0) { k_combine_warp<float, V><<<blocks, 256, 0, s>>>(p); note_launch(); }          \
-    else { k_combine_warp<bf16, V><<<blocks, 256, 0, s>>>(p); note_launch(); }                      \
-    return true;
-  switch (vpl) {
+#define RDT_CW(V)                                                                             \
+  case V:                                                                                     \
+    return dtype == 0 ? launch_combine_vpl<float, V>(p, n_rows, s) : launch_combine_vpl<bf16, V>(p, n_rows, s);
+  switch (p.D / 128) {
     RDT_CW(1) RDT_CW(2) RDT_CW(4) RDT_CW(8) RDT_CW(12) RDT_CW(16) RDT_CW(24) RDT_CW(32)
     default: return false;
   }
