@@ -31,6 +31,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 import rdt_inputs as RI  # noqa: E402
+from recurrent_depth_moe_b200 import replicas as REP  # noqa: E402
 
 METRIC = "recurrent-block token·loops/s prefill; decode tokens/s; % roofline, 1×B200"
 UNIT = "token·loops/s"
@@ -196,7 +197,7 @@ def run_ours(args, wl, rank, world, local_rank):
     N = B * T
     # weights: identical replica on every rank; inputs: a different batch per rank
     W, halt_off = workload_weights(wl, dev)
-    h0, e = RI.recurrent_inputs(cfg, B, T, wl.seed + 101 * rank, device=dev)
+    h0, e = RI.recurrent_inputs(cfg, B, T, REP.replica_input_seed(wl.seed, rank), device=dev)
     blk = R.RecurrentBlock(cfg, W)
     ws = blk.workspace(B, T, T)
     out = (torch.empty(N, cfg.dim, dtype=torch.float32, device=dev),
@@ -234,19 +235,14 @@ def run_ours(args, wl, rank, world, local_rank):
     prof = NAT.profile_stop()
     clk = clocks.stop()
     ms = ev0.elapsed_time(ev1) / args.steps
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = REP.max_over_ranks(ms, device=dev)
 
     # executed token-loops of one step (positions that halt early run fewer loops)
     hw = out[1]
     last = ((hw > 0).to(torch.int64) * torch.arange(L, device=dev)[:, None]).max(dim=0).values
     executed = float((last + 1).sum().item())
-    tl = torch.tensor([executed], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(tl, op=torch.distributed.ReduceOp.SUM)
-    value = float(tl.item()) / (ms_max / 1e3)
+    executed_all = REP.sum_over_ranks(executed, device=dev)
+    value = executed_all / (ms_max / 1e3)
 
     # end to end through the public API: pinned host inputs -> device -> forward -> host outputs
     h0_h = h0.cpu().pin_memory()
@@ -273,10 +269,8 @@ def run_ours(args, wl, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = float(tl.item()) / (float(te.item()) / 1e3)
+    e2e_ms = REP.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
+    e2e_value = executed_all / (e2e_ms / 1e3)
 
     # host copy for the CPU-oracle baseline, then free the prefill workload before the
     # decode one (23 GB of weights and caches)
@@ -313,7 +307,7 @@ def run_ours(args, wl, rank, world, local_rank):
            "config": {"workload": workload_desc(wl), "batch": B * world, "seq_len": T, "n_loops": L,
                       "parallelism": f"replicas x{world} (sequence-sharded, no collective)",
                       "l2": f"inputs larger than L2 ({3 * cfg.dim * cfg.expert_dim * (cfg.n_experts + cfg.n_shared_experts) * 2 / 1e9:.2f} GB of expert weights streamed per loop)"},
-           "executed_token_loops_per_step": executed * world,
+           "executed_token_loops_per_step": executed_all,
            "roofline": roofline, "gpu_launches": launches,
            "kernel_ms_per_step": breakdown,
            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -359,10 +353,10 @@ def run_decode(args, rank, world, local_rank):
     B, L, steps = wl.batch, wl.n_loops, args.decode_steps
     t_max = wl.cache_len + steps + args.warmup
     W = RI.block_weights(cfg, wl.seed, device=dev)
-    k, v = RI.random_kv_cache(cfg, L, B, t_max, wl.cache_len, wl.seed + 31 * rank, device=dev)
+    k, v = RI.random_kv_cache(cfg, L, B, t_max, wl.cache_len, REP.replica_input_seed(wl.seed, rank), device=dev)
     h0s, es = [], []
     for st in range(steps + args.warmup):
-        h, e = RI.decode_inputs(cfg, B, st, wl.seed + 31 * rank, device=dev)
+        h, e = RI.decode_inputs(cfg, B, st, REP.replica_input_seed(wl.seed, rank), device=dev)
         h0s.append(h)
         es.append(e)
     blk = R.RecurrentBlock(cfg, W)
@@ -396,10 +390,7 @@ def run_decode(args, rank, world, local_rank):
     launches = NAT.launch_count() - n0
     prof = NAT.profile_stop()
     ms = e0.elapsed_time(e1) / steps
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = REP.max_over_ranks(ms, device=dev)
     # algorithmic bytes of the last timed step (its routing and cache lengths)
     bytes_step = decode_algorithmic_bytes(cfg, out[2].cpu(), (clen - 1).cpu())
     pk, pk_kind = peaks()
