@@ -43,40 +43,6 @@ template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float4 v) {
 }
 __device__ __forceinline__ float f4_dot(float4 a, float4 b) { return a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w; }
 
-// Prologue of the next loop for one row held by a warp (x = state, in registers):
-//   combined = RMSNorm_rec(x + emb + e) * w_rec ; a = RMSNorm_attn(combined) * w_attn
-template <typename T, int VPL>
-__device__ __forceinline__ void next_prologue(const CombineParams& p, float4 (&x)[VPL], long long rowD, int lane) {
-  const T* er = (const T*)p.e + rowD + 4 * lane;
-  float ss = 0.f;
-#pragma unroll
-  for (int j = 0; j < VPL; ++j) {
-    const int d = 4 * lane + 128 * j;
-    float4 ev = Vec4<T>::load(er + 128 * j);
-    x[j] = f4_add(x[j], ev);
-    if (d < p.loop_dim) x[j] = f4_add(x[j], __ldg(reinterpret_cast<const float4*>(p.next_emb + d)));
-    ss += f4_dot(x[j], x[j]);
-  }
-  const float inv = rsqrtf(warp_sum(ss) / p.D + p.eps);
-  float ss2 = 0.f;
-#pragma unroll
-  for (int j = 0; j < VPL; ++j) {
-    const int d = 4 * lane + 128 * j;
-    const float4 wv = __ldg(reinterpret_cast<const float4*>(p.w_rec + d));
-    x[j] = make_float4(x[j].x * inv * wv.x, x[j].y * inv * wv.y, x[j].z * inv * wv.z, x[j].w * inv * wv.w);
-    *reinterpret_cast<float4*>(p.combined_out + rowD + d) = x[j];
-    ss2 += f4_dot(x[j], x[j]);
-  }
-  const float inv2 = rsqrtf(warp_sum(ss2) / p.D + p.eps);
-#pragma unroll
-  for (int j = 0; j < VPL; ++j) {
-    const int d = 4 * lane + 128 * j;
-    const float4 wv = __ldg(reinterpret_cast<const float4*>(p.w_attn + d));
-    store4<T>((T*)p.a_out + rowD + d,
-              make_float4(x[j].x * inv2 * wv.x, x[j].y * inv2 * wv.y, x[j].z * inv2 * wv.z, x[j].w * inv2 * wv.w));
-  }
-}
-
 // Plain 4-element load usable on shared or global memory (generic address).
 template <typename T> __device__ __forceinline__ float4 ld4(const T* p);
 template <> __device__ __forceinline__ float4 ld4<float>(const float* p) { return *reinterpret_cast<const float4*>(p); }
@@ -87,76 +53,164 @@ template <> __device__ __forceinline__ float4 ld4<bf16>(const bf16* p) {
   return make_float4(fa.x, fa.y, fb.x, fb.y);
 }
 
-// One row (one warp) of S9; Wd / Bl point at the LoRA matrices (shared or global).
-template <typename T, int VPL>
-__device__ __forceinline__ void combine_row(const CombineParams& p, int i, int lane, float* z, const T* Wd,
-                                            const T* Bl) {
+// A row is processed by a group of WPR warps; warp wr of the group owns the float4
+// columns 4 lane + 128 j for j in [wr VQ, (wr + 1) VQ), VQ = VPL / WPR.  Row-wide sums go
+// through shared memory: each warp reduces its part, lane 0 stores it in slot `slot` of
+// the group's scratch, one named barrier (id bar, WPR warps) and every lane adds the
+// WPR partials.  Slots are never reused within a row, and the next row's first barrier
+// orders them against the previous row, so one barrier per reduction phase suffices.
+template <int WPR>
+struct Group {
+  float* red;   // [WPR][32] partial sums of this group
+  int wr, bar;
+  __device__ __forceinline__ void sync() const {
+    if (WPR > 1) asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(WPR * 32) : "memory");
+  }
+  // Finish `n` warp-reduced partials held (identically) by every lane in v[0..n).
+  template <int NMAX>
+  __device__ __forceinline__ void reduce(float (&v)[NMAX], int n, int slot0, int lane) const {
+    if (WPR == 1) return;
+    if (lane == 0)
+      for (int q = 0; q < n; ++q) red[wr * 32 + slot0 + q] = v[q];
+    sync();
+    for (int q = 0; q < n; ++q) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < WPR; ++w) t += red[w * 32 + slot0 + q];
+      v[q] = t;
+    }
+  }
+  __device__ __forceinline__ float reduce1(float v, int slot, int lane) const {
+    float a[1] = {v};
+    reduce<1>(a, 1, slot, lane);
+    return a[0];
+  }
+};
+
+// Prologue of the next loop for the group's row (x = this warp's part of the state):
+//   combined = RMSNorm_rec(x + emb + e) * w_rec ; a = RMSNorm_attn(combined) * w_attn
+template <typename T, int VQ, int WPR>
+__device__ __forceinline__ void next_prologue(const CombineParams& p, float4 (&x)[VQ], long long rowD, int lane,
+                                              int j0, const Group<WPR>& g) {
+  const T* er = (const T*)p.e + rowD + 4 * lane;
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < VQ; ++j) {
+    const int d = 4 * lane + 128 * (j0 + j);
+    float4 ev = Vec4<T>::load(er + 128 * (j0 + j));
+    x[j] = f4_add(x[j], ev);
+    if (d < p.loop_dim) x[j] = f4_add(x[j], __ldg(reinterpret_cast<const float4*>(p.next_emb + d)));
+    ss += f4_dot(x[j], x[j]);
+  }
+  ss = g.reduce1(warp_sum(ss), 17, lane);
+  const float inv = rsqrtf(ss / p.D + p.eps);
+  float ss2 = 0.f;
+#pragma unroll
+  for (int j = 0; j < VQ; ++j) {
+    const int d = 4 * lane + 128 * (j0 + j);
+    const float4 wv = __ldg(reinterpret_cast<const float4*>(p.w_rec + d));
+    x[j] = make_float4(x[j].x * inv * wv.x, x[j].y * inv * wv.y, x[j].z * inv * wv.z, x[j].w * inv * wv.w);
+    *reinterpret_cast<float4*>(p.combined_out + rowD + d) = x[j];
+    ss2 += f4_dot(x[j], x[j]);
+  }
+  ss2 = g.reduce1(warp_sum(ss2), 18, lane);
+  const float inv2 = rsqrtf(ss2 / p.D + p.eps);
+#pragma unroll
+  for (int j = 0; j < VQ; ++j) {
+    const int d = 4 * lane + 128 * (j0 + j);
+    const float4 wv = __ldg(reinterpret_cast<const float4*>(p.w_attn + d));
+    store4<T>((T*)p.a_out + rowD + d,
+              make_float4(x[j].x * inv2 * wv.x, x[j].y * inv2 * wv.y, x[j].z * inv2 * wv.z, x[j].w * inv2 * wv.w));
+  }
+}
+
+// One row of S9 by a group of WPR warps; Wd / Bl point at the LoRA matrices (shared or global).
+template <typename T, int VPL, int WPR>
+__device__ __forceinline__ void combine_row(const CombineParams& p, int i, int lane, const Group<WPR>& g,
+                                            float* z, const T* Wd, const T* Bl) {
+  constexpr int VQ = VPL / WPR;
+  const int j0 = g.wr * VQ;
   const int D = p.D;
   const int kS = p.k + p.S;
   const long long rowD = (long long)i * D;
-  float4 tr[VPL];
+  const bool lead = (g.wr == 0);
+  float4 tr[VQ];
   if (!p.block_only && p.halted[i]) {   // frozen row: no update, zero weight, no experts
-    if (lane == 0) p.halt_w_out[(long long)p.t * p.N + i] = 0.f;
-    if (lane < p.k) p.ids_out[((long long)p.t * p.N + i) * p.k + lane] = -1;
+    if (lead && lane == 0) p.halt_w_out[(long long)p.t * p.N + i] = 0.f;
+    if (lead && lane < p.k) p.ids_out[((long long)p.t * p.N + i) * p.k + lane] = -1;
     if (p.next_emb) {                   // its keys / values are still recomputed next loop
 #pragma unroll
-      for (int j = 0; j < VPL; ++j) tr[j] = __ldg(reinterpret_cast<const float4*>(p.h + rowD + 4 * lane + 128 * j));
-      next_prologue<T, VPL>(p, tr, rowD, lane);
+      for (int j = 0; j < VQ; ++j)
+        tr[j] = __ldg(reinterpret_cast<const float4*>(p.h + rowD + 4 * lane + 128 * (j0 + j)));
+      next_prologue<T, VQ, WPR>(p, tr, rowD, lane, j0, g);
     }
     return;
   }
   if (p.transformer_off) {
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) tr[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < VQ; ++j) tr[j] = make_float4(0.f, 0.f, 0.f, 0.f);
   } else {
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) tr[j] = __ldg(reinterpret_cast<const float4*>(p.x1 + rowD + 4 * lane + 128 * j));
+    for (int j = 0; j < VQ; ++j)
+      tr[j] = __ldg(reinterpret_cast<const float4*>(p.x1 + rowD + 4 * lane + 128 * (j0 + j)));
     // slot rows two at a time, so two rows' loads are in flight per memory round trip
     const int* so = p.slot_of + (long long)i * kS;
     for (int s = 0; s < kS; s += 2) {
       int s0 = so[s], s1 = (s + 1 < kS) ? so[s + 1] : -2;
       if (s0 < 0 || s0 >= p.max_slots) {
-        if (lane == 0) record_status(p.st, ST_BOUNDS, 202, s0);
+        if (lead && lane == 0) record_status(p.st, ST_BOUNDS, 202, s0);
         s0 = -1;
       }
       if (s1 != -2 && (s1 < 0 || s1 >= p.max_slots)) {
-        if (lane == 0) record_status(p.st, ST_BOUNDS, 202, s1);
+        if (lead && lane == 0) record_status(p.st, ST_BOUNDS, 202, s1);
         s1 = -1;
       }
       const T* y0 = (const T*)p.y + (long long)max(s0, 0) * D + 4 * lane;
       const T* y1 = (const T*)p.y + (long long)max(s1, 0) * D + 4 * lane;
 #pragma unroll
-      for (int j = 0; j < VPL; ++j) {
-        const float4 a0 = s0 >= 0 ? Vec4<T>::load(y0 + 128 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 a1 = s1 >= 0 ? Vec4<T>::load(y1 + 128 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j = 0; j < VQ; ++j) {
+        const int c = 128 * (j0 + j);
+        const float4 a0 = s0 >= 0 ? Vec4<T>::load(y0 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 a1 = s1 >= 0 ? Vec4<T>::load(y1 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
         tr[j] = f4_add(tr[j], f4_add(a0, a1));
       }
     }
   }
   if (p.block_only) {
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) *reinterpret_cast<float4*>(p.out + rowD + 4 * lane + 128 * j) = tr[j];
+    for (int j = 0; j < VQ; ++j) *reinterpret_cast<float4*>(p.out + rowD + 4 * lane + 128 * (j0 + j)) = tr[j];
     return;
   }
   if (!p.transformer_off && p.r > 0) {
     const float* sc = p.lora_scale + (long long)min(p.t, p.max_loop_iters - 1) * p.r;
-    for (int q = 0; q < p.r; ++q) {
-      float part = 0.f;
-      const T* w = Wd + (long long)q * D + 4 * lane;
+    float zq[16];
+    // rank in chunks of 16: partial projections of this warp's columns, then the group sum
+    for (int q0 = 0; q0 < p.r; q0 += 16) {
+      const int nq = min(16, p.r - q0);
 #pragma unroll
-      for (int j = 0; j < VPL; ++j) part += f4_dot(tr[j], ld4<T>(w + 128 * j));
-      part = warp_sum(part) * sc[q];
-      if (lane == 0) z[q] = part;
+      for (int q = 0; q < 16; ++q) {
+        float part = 0.f;
+        if (q < nq) {
+          const T* w = Wd + (long long)(q0 + q) * D + 4 * lane;
+#pragma unroll
+          for (int j = 0; j < VQ; ++j) part += f4_dot(tr[j], ld4<T>(w + 128 * (j0 + j)));
+        }
+        zq[q] = warp_sum(part);
+      }
+      g.reduce<16>(zq, nq, 0, lane);
+      if (lane == 0)
+        for (int q = 0; q < nq; ++q) z[q0 + q] = zq[q] * sc[q0 + q];
+      if (q0 + 16 < p.r) g.sync();   // slots 0..15 are rewritten by the next chunk
     }
     __syncwarp();
     // every z_q is complete, so the delta can be added to the row in place
     for (int q = 0; q < p.r; ++q) {
       const T* bq = Bl + (long long)q * D + 4 * lane;
-      const float zq = z[q];
+      const float zv = z[q];
 #pragma unroll
-      for (int j = 0; j < VPL; ++j) {
-        float4 v = ld4<T>(bq + 128 * j);
-        tr[j].x += zq * v.x; tr[j].y += zq * v.y; tr[j].z += zq * v.z; tr[j].w += zq * v.w;
+      for (int j = 0; j < VQ; ++j) {
+        float4 v = ld4<T>(bq + 128 * (j0 + j));
+        tr[j].x += zv * v.x; tr[j].y += zv * v.y; tr[j].z += zv * v.z; tr[j].w += zv * v.w;
       }
     }
     __syncwarp();
@@ -165,12 +219,12 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
   const T* er = (const T*)p.e + rowD + 4 * lane;
   float zh = 0.f;
 #pragma unroll
-  for (int j = 0; j < VPL; ++j) {
-    const int d = 4 * lane + 128 * j;
+  for (int j = 0; j < VQ; ++j) {
+    const int d = 4 * lane + 128 * (j0 + j);
     float4 hv = __ldg(reinterpret_cast<const float4*>(p.h + rowD + d));
     float4 av = __ldg(reinterpret_cast<const float4*>(p.A + d));
     float4 bv = __ldg(reinterpret_cast<const float4*>(p.inj_B + d));
-    float4 ev = Vec4<T>::load(er + 128 * j);
+    float4 ev = Vec4<T>::load(er + 128 * (j0 + j));
     tr[j].x += av.x * hv.x + bv.x * ev.x;
     tr[j].y += av.y * hv.y + bv.y * ev.y;
     tr[j].z += av.z * hv.z + bv.z * ev.z;
@@ -180,14 +234,14 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
   const bool last = (p.t == p.n_loops - 1);
   float w;
   if (p.act_on) {
-    zh = warp_sum(zh);
+    zh = g.reduce1(warp_sum(zh), 16, lane);
     const float zz = zh + p.halt_b[0] + (p.halt_off ? p.halt_off[i] : 0.f);
     const float prob = 1.f / (1.f + expf(-zz));
     const float cum = p.cum[i];
     const bool stop = (cum + prob >= p.thr) || last;
     w = stop ? fmaxf(1.f - cum, 0.f) : prob;
-    __syncwarp();
-    if (lane == 0) {
+    g.sync();   // every warp has read cum before the lead updates it
+    if (lead && lane == 0) {
       p.cum[i] = cum + prob;
       if (stop) p.halted[i] = 1;
       if (p.p_out) p.p_out[i] = prob;
@@ -196,8 +250,8 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
     w = last ? 1.f : 0.f;
   }
 #pragma unroll
-  for (int j = 0; j < VPL; ++j) {
-    const int d = 4 * lane + 128 * j;
+  for (int j = 0; j < VQ; ++j) {
+    const int d = 4 * lane + 128 * (j0 + j);
     float4* ho = reinterpret_cast<float4*>(p.h_out + rowD + d);
     if (w != 0.f) {
       float4 o = *ho;
@@ -206,20 +260,26 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
     }
     *reinterpret_cast<float4*>(p.h_state + rowD + d) = tr[j];
   }
-  if (lane == 0) p.halt_w_out[(long long)p.t * p.N + i] = w;
-  if (lane < p.k)
+  if (lead && lane == 0) p.halt_w_out[(long long)p.t * p.N + i] = w;
+  if (lead && lane < p.k)
     p.ids_out[((long long)p.t * p.N + i) * p.k + lane] = p.transformer_off ? -1 : p.ids[(long long)i * p.k + lane];
-  if (p.next_emb) next_prologue<T, VPL>(p, tr, rowD, lane);
+  if (p.next_emb) next_prologue<T, VQ, WPR>(p, tr, rowD, lane, j0, g);
 }
 
-// Persistent: WARPS warps per CTA, one CTA per SM, rows strided over the grid.  With
-// LSMEM the LoRA matrices (2 r D elements) are staged in shared memory once per CTA,
-// so the rank-r projections read shared memory instead of making 2 r round trips to L2.
-template <typename T, int VPL, int WARPS, bool LSMEM>
-__global__ void __launch_bounds__(WARPS * 32, 1) k_combine_warp(CombineParams p) {
+// Persistent: GROUPS row groups of WPR warps per CTA, one CTA per SM, rows strided over
+// the grid.  With LSMEM the LoRA matrices (2 r D elements) are staged in shared memory once
+// per CTA, so the rank-r projections read shared memory instead of L2.
+template <typename T, int VPL, int WPR, int GROUPS, bool LSMEM>
+__global__ void __launch_bounds__(GROUPS * WPR * 32, 1) k_combine_warp(CombineParams p) {
   extern __shared__ __align__(16) uint8_t csm[];
-  __shared__ float zs[WARPS][64];
+  __shared__ float zs[GROUPS][64];
+  __shared__ float red[GROUPS][WPR * 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int grp = warp / WPR;
+  Group<WPR> g;
+  g.red = red[grp];
+  g.wr = warp % WPR;
+  g.bar = 1 + grp;
   const T* Wd = (const T*)p.lora_down;
   const T* Bl = (const T*)p.lora_B;
   if (LSMEM && p.r > 0 && !p.transformer_off && !p.block_only) {
@@ -236,8 +296,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) k_combine_warp(CombineParams p)
     Wd = reinterpret_cast<const T*>(csm);
     Bl = reinterpret_cast<const T*>(csm + bytes);
   }
-  for (int i = blockIdx.x * WARPS + warp; i < p.N; i += gridDim.x * WARPS)
-    combine_row<T, VPL>(p, i, lane, zs[warp], Wd, Bl);
+  for (int i = blockIdx.x * GROUPS + grp; i < p.N; i += gridDim.x * GROUPS)
+    combine_row<T, VPL, WPR>(p, i, lane, g, zs[grp], Wd, Bl);
 }
 
 // out = RMSNorm(x) * w for fp32 rows of width D = 128 * VPL, one warp per row.
@@ -297,22 +357,25 @@ int combine_sm_count() {
 
 template <typename T, int VPL>
 bool launch_combine_vpl(const CombineParams& p, int n_rows, cudaStream_t s) {
-  constexpr int WARPS = VPL >= 24 ? 8 : 16;
+  // rows split over 4 warps when the width allows (32 warps per SM, 16-register rows)
+  constexpr int WPR = (VPL % 4 == 0) ? 4 : ((VPL % 2 == 0) ? 2 : 1);
+  constexpr int GROUPS = 8;
   const size_t lbytes = (size_t)2 * p.r * p.D * sizeof(T);
   const bool lsmem = p.r > 0 && lbytes <= 160 * 1024 && (((size_t)p.r * p.D * sizeof(T)) % 16) == 0 &&
                      ((uintptr_t)p.lora_down % 16) == 0 && ((uintptr_t)p.lora_B % 16) == 0;
-  const int grid = std::max(1, std::min((n_rows + WARPS - 1) / WARPS, combine_sm_count()));
+  const int grid = std::max(1, std::min((n_rows + GROUPS - 1) / GROUPS, combine_sm_count()));
+  constexpr int THREADS = GROUPS * WPR * 32;
   if (lsmem) {
     static bool attr = false;
     if (!attr) {
-      if (cudaFuncSetAttribute(k_combine_warp<T, VPL, WARPS, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               160 * 1024) != cudaSuccess)
+      if (cudaFuncSetAttribute(k_combine_warp<T, VPL, WPR, GROUPS, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) != cudaSuccess)
         return false;
       attr = true;
     }
-    { k_combine_warp<T, VPL, WARPS, true><<<grid, WARPS * 32, lbytes, s>>>(p); note_launch(); }
+    { k_combine_warp<T, VPL, WPR, GROUPS, true><<<grid, THREADS, lbytes, s>>>(p); note_launch(); }
   } else {
-    { k_combine_warp<T, VPL, WARPS, false><<<grid, WARPS * 32, 0, s>>>(p); note_launch(); }
+    { k_combine_warp<T, VPL, WPR, GROUPS, false><<<grid, THREADS, 0, s>>>(p); note_launch(); }
   }
   return true;
 }
