@@ -45,7 +45,7 @@ extern "C" {
 typedef enum {
   RDT_OK = 0,
   RDT_ERR_INVALID_ARG = 1,     /* null pointer, bad size, inconsistent config       */
-  RDT_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. MLA decode)        */
+  RDT_ERR_UNSUPPORTED = 2,     /* valid but not implemented                          */
   RDT_ERR_WORKSPACE = 3,       /* ws too small or misaligned                          */
   RDT_ERR_CUDA = 4,            /* a CUDA runtime call failed                          */
   RDT_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait gave up                  */
@@ -112,8 +112,13 @@ typedef struct {
 } rdt_weights;
 
 /* One K/V cache per recurrent loop iteration (cache key recurrent_loop_t,
- * "OpenMythos 분석", Recurrent Block / RoPE & generation cache).
- * GQA: k, v [n_loops][batch][Hkv][t_max][hd], model dtype, post-RoPE keys. */
+ * "OpenMythos 분석", Recurrent Block / RoPE & generation cache), model dtype,
+ * caller-owned device memory; a sequence's positions beyond its length are never read.
+ * GQA: k, v [n_loops][batch][Hkv][t_max][hd], post-RoPE keys and values.
+ * MLA ("OpenMythos 분석", MLA: the cache keeps the latent, not per-head K/V):
+ *      k = c_kv   [n_loops][batch][t_max][kv_lora_rank], before its RMSNorm;
+ *      v = k_rope [n_loops][batch][t_max][qk_rope_head_dim], rotated, one for all heads.
+ *      Each call rebuilds [k_nope | v] of the cached positions from c_kv. */
 typedef struct {
   void* k;
   void* v;
@@ -163,7 +168,7 @@ RDT_API rdt_status rdt_recurrent_forward(const rdt_config* cfg, const rdt_weight
 
 /* One KV-cached decode step of the recurrent block ("OpenMythos 분석", RoPE &
  * generation cache): one new token per sequence b at position cache_len[b]
- * (device int32 [batch]); loop t reads and extends loop cache t (GQA only).
+ * (device int32 [batch]); loop t reads and extends loop cache t (GQA or MLA).
  * The new K/V are written at cache_len[b]; the caller advances cache_len.
  * Outputs as rdt_recurrent_forward with N = batch. */
 RDT_API rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_weights* w,

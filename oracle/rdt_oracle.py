@@ -399,7 +399,8 @@ def decode_step(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, caches: list, c
     """One KV-cached decode step of the recurrent block ("OpenMythos 분석", "RoPE &
     generation cache"): one new token per sequence b at position cache_len[b]; loop t
     attends to its own loop cache (keys 0..cache_len[b]-1) plus the new token.
-    caches[t][b] = {"k": [C_b, Hkv, hd], "v": ..., "pos": [C_b]} (GQA).
+    caches[t][b] = {"k": [C_b, Hkv, hd], "v": ..., "pos": [C_b]} (GQA), or
+    {"c_kv": [C_b, kv_lora_rank], "k_rope": [C_b, qk_rope_head_dim], "pos": [C_b]} (MLA).
     Returns (h_out [B, D], halt_weights [L, B], expert_ids [L, B, k], new_kv)."""
     B = h0.shape[0]
     h = _d(h0).clone()

@@ -304,6 +304,22 @@ def random_kv_cache(cfg: RDTConfig, n_loops: int, batch: int, t_max: int, filled
     return k, v
 
 
+def random_latent_cache(cfg: RDTConfig, n_loops: int, batch: int, t_max: int, filled: int,
+                        seed: int, device="cpu"):
+    """One random MLA latent cache per recurrent loop: c_kv [n_loops, B, t_max, kv_lora_rank]
+    and k_rope [n_loops, B, t_max, qk_rope_head_dim] (model dtype), N(0,1) in positions
+    [0, filled), zero beyond."""
+    g = _gen(seed + 37, device)
+    ckv = torch.zeros(n_loops, batch, t_max, cfg.kv_lora_rank, dtype=cfg.torch_dtype, device=device)
+    kr = torch.zeros(n_loops, batch, t_max, cfg.qk_rope_head_dim, dtype=cfg.torch_dtype, device=device)
+    for t in range(n_loops):
+        ckv[t, :, :filled] = torch.randn(batch, filled, cfg.kv_lora_rank, generator=g,
+                                         device=device).to(cfg.torch_dtype)
+        kr[t, :, :filled] = torch.randn(batch, filled, cfg.qk_rope_head_dim, generator=g,
+                                        device=device).to(cfg.torch_dtype)
+    return ckv, kr
+
+
 def halting_offsets_spread(n: int, lo: int, hi: int, threshold: float, seed: int):
     """Per-position halting-logit offsets that make position i halt after exactly
     k_i loops, k_i ~ U{lo..hi}: with a zero halting weight and bias, the halting

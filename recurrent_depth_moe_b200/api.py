@@ -101,14 +101,25 @@ def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
 
 @dataclass
 class KVCache:
-    """One GQA K/V cache per recurrent loop: k, v [n_loops, batch, Hkv, t_max, hd]."""
+    """One attention cache per recurrent loop.
+    GQA: k, v [n_loops, batch, Hkv, t_max, hd] (post-RoPE keys, values).
+    MLA: k = c_kv [n_loops, batch, t_max, kv_lora_rank] (before its RMSNorm),
+         v = k_rope [n_loops, batch, t_max, qk_rope_head_dim] (rotated, shared by all heads)."""
     k: torch.Tensor
     v: torch.Tensor
 
+    @property
+    def t_max(self) -> int:
+        return self.k.shape[3] if self.k.dim() == 5 else self.k.shape[2]
+
     def struct(self) -> N.rdt_kv_cache:
+        if self.k.dim() not in (4, 5) or self.k.shape[:2] != self.v.shape[:2]:
+            raise ValueError("cache tensors must be [n_loops, batch, ...] with matching leading dims")
+        if not (self.k.is_contiguous() and self.v.is_contiguous()):
+            raise ValueError("cache tensors must be contiguous")
         s = N.rdt_kv_cache()
         s.k, s.v = self.k.data_ptr(), self.v.data_ptr()
-        s.n_loops, s.batch, s.t_max = self.k.shape[0], self.k.shape[1], self.k.shape[3]
+        s.n_loops, s.batch, s.t_max = self.k.shape[0], self.k.shape[1], self.t_max
         return s
 
 
@@ -170,7 +181,7 @@ class RecurrentBlock:
             out = (torch.empty(Nr, cfg.dim, dtype=torch.float32, device=h0.device),
                    torch.empty(n_loops, Nr, dtype=torch.float32, device=h0.device),
                    torch.empty(n_loops, Nr, cfg.n_experts_per_tok, dtype=torch.int32, device=h0.device))
-        max_keys = start_pos + seq if cache is None else max(start_pos + seq, cache.k.shape[3])
+        max_keys = start_pos + seq if cache is None else max(start_pos + seq, cache.t_max)
         ws = workspace if workspace is not None else self.workspace(batch, seq, max_keys)
         cs = cache.struct() if cache is not None else None
         ts = trace.struct() if trace is not None else None
@@ -197,7 +208,7 @@ class RecurrentBlock:
             out = (torch.empty(B, cfg.dim, dtype=torch.float32, device=h0.device),
                    torch.empty(n_loops, B, dtype=torch.float32, device=h0.device),
                    torch.empty(n_loops, B, cfg.n_experts_per_tok, dtype=torch.int32, device=h0.device))
-        ws = workspace if workspace is not None else self.workspace(B, 1, cache.k.shape[3])
+        ws = workspace if workspace is not None else self.workspace(B, 1, cache.t_max)
         cs = cache.struct()
         rc = lib.rdt_recurrent_decode_step(ctypes.byref(self.cs), ctypes.byref(self.w.struct), h0.data_ptr(),
                                            e.data_ptr(), B, cache_len.data_ptr(), n_loops, float(act_threshold),

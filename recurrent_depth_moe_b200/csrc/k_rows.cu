@@ -145,6 +145,27 @@ __global__ void k_mla_kv_prep(const float* __restrict__ kv_raw, int kvr, int dr,
 }
 
 // ------------------------------------------------------------------------------------------
+// MLA latent cache of one loop: c_kv [B][t_max][kvr] (raw, before its RMSNorm) and the
+// rotated k_rope [B][t_max][dr] shared by all heads ("OpenMythos 분석", MLA: the cache
+// holds c_kv and k_rope), written at position pos[row].
+// ------------------------------------------------------------------------------------------
+template <typename T>
+__global__ void k_mla_to_cache(const float* __restrict__ kv_raw, const T* __restrict__ krope, int kvr, int dr,
+                               const int* __restrict__ pos, int seq, int t_max, T* __restrict__ ckv_c,
+                               T* __restrict__ kr_c, DevStatus* st) {
+  const long long row = blockIdx.x;
+  const int b = (int)(row / seq);
+  const int p = pos[row];
+  if (p < 0 || p >= t_max) {
+    if (threadIdx.x == 0) record_status(st, ST_BOUNDS, 103, p);
+    return;
+  }
+  const long long dst = (long long)b * t_max + p;
+  for (int d = threadIdx.x; d < kvr; d += blockDim.x) ckv_c[dst * kvr + d] = from_f<T>(kv_raw[row * (kvr + dr) + d]);
+  for (int d = threadIdx.x; d < dr; d += blockDim.x) kr_c[dst * dr + d] = krope[row * dr + d];
+}
+
+// ------------------------------------------------------------------------------------------
 // GQA K/V rows -> per-loop cache [B][Hkv][t_max][hd] at position pos[row].
 // ------------------------------------------------------------------------------------------
 template <typename T>
@@ -393,6 +414,12 @@ void launch_kv_to_cache(int dtype, const void* qkv, long long ld, int k_col, int
                                           (bf16*)kc, (bf16*)vc, st); note_launch(); }
 }
 bool launch_combine_warp(int dtype, const CombineParams& p, int n_rows, cudaStream_t s);
+
+void launch_mla_to_cache(int dtype, const float* kv_raw, const void* krope, int kvr, int dr, const int* pos, int N,
+                         int seq, int t_max, void* ckv_c, void* kr_c, DevStatus* st, cudaStream_t s) {
+  if (dtype == 0) { k_mla_to_cache<float><<<N, 64, 0, s>>>(kv_raw, (const float*)krope, kvr, dr, pos, seq, t_max, (float*)ckv_c, (float*)kr_c, st); note_launch(); }
+  else { k_mla_to_cache<bf16><<<N, 64, 0, s>>>(kv_raw, (const bf16*)krope, kvr, dr, pos, seq, t_max, (bf16*)ckv_c, (bf16*)kr_c, st); note_launch(); }
+}
 
 bool launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s) {
   if (launch_combine_warp(dtype, p, n_rows, s)) return p.next_emb != nullptr;

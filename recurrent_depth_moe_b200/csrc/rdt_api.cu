@@ -24,6 +24,7 @@ struct Layout {
   size_t status, h, combined, a, qkv, cq_raw, cq, q, kv_raw, ckv, krope, kvu, attn, x1, f, logits;
   size_t ids, gates, rank, counts, offsets, tiles, ntiles, slot_of, tok_of, gate_of, xg, u, y;
   size_t run_list, run_idx, nrun, cum, halted, Avec, emb, rope, pos, p_buf, part_o, part_ml, xn, vt;
+  size_t mla_ckv_all, mla_kvu_all;   // MLA with earlier cached keys: rebuilt per-head keys / values
   size_t total;
   int max_tiles, max_slots, rope_dim, rope_pos, n_split;
 };
@@ -85,6 +86,10 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
     L->krope = take(N * dr * es);
     L->kvu = take(N * (size_t)H * (dn + dv) * es);
     L->rope_dim = dr;
+    if (max_keys > T) {   // earlier positions come from the latent cache
+      L->mla_ckv_all = take((size_t)B * max_keys * c->kv_lora_rank * es);
+      L->mla_kvu_all = take((size_t)B * max_keys * H * (dn + dv) * es);
+    }
   }
   L->attn = take(N * (size_t)H * dv * es);
   L->x1 = take(N * D * 4);
@@ -206,7 +211,6 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
     }
     dv = hd;
   } else {
-    if (cache && cache->k) return RDT_ERR_UNSUPPORTED;   // MLA latent-cache decode not built
     const int dn = c->qk_nope_head_dim, dr = c->qk_rope_head_dim, kvr = c->kv_lora_rank, ql = c->q_lora_rank;
     dv = c->v_head_dim;
     float* cq_raw = at<float*>(x.ws, x.L.cq_raw);
@@ -239,6 +243,31 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
     ap.k2 = krope; ap.k2_b = (long long)T * dr; ap.k2_j = dr;
     ap.v = (const char*)kvu + (size_t)dn * es; ap.v_b = (long long)T * kvw; ap.v_j = kvw; ap.v_g = dn + dv;
     ap.key_pos0 = start_pos; ap.n_keys = T;
+    if (cache && cache->k) {
+      // latent cache of loop t: c_kv [B][t_max][kvr] (raw) and k_rope [B][t_max][dr]
+      const int tm = cache->t_max;
+      char* ckv_c = (char*)cache->k + (size_t)loop_t * cache->batch * tm * kvr * es;
+      char* kr_c = (char*)cache->v + (size_t)loop_t * cache->batch * tm * dr * es;
+      { ProfScope ps(PC_OTHER, x.s); launch_mla_to_cache(x.dtype, kv_raw, krope, kvr, dr, pos, N, T, tm, ckv_c, kr_c, x.st, x.s); }
+      if (decode || start_pos > 0) {
+        // keys / values of every cached position: [k_nope | v] = RMSNorm(c_kv) W_kvu^T
+        if (!x.L.mla_kvu_all) return RDT_ERR_WORKSPACE;
+        void* ckv_all = at<void*>(x.ws, x.L.mla_ckv_all);
+        void* kvu_all = at<void*>(x.ws, x.L.mla_kvu_all);
+        const int rows = B * tm;
+        ProfScope ps(PC_OTHER, x.s);
+        launch_rmsnorm(0, x.dtype, ckv_c, kvr, w->kv_norm_w, ckv_all, kvr, rows, kvr, c->norm_eps, x.s);
+        GemmParams g2 = gemm_base(x);
+        g2.A = ckv_all; g2.lda = kvr; g2.B = w->w_kv_up; g2.ldb = kvr; g2.M = rows; g2.N = H * (dn + dv); g2.K = kvr;
+        g2.C = kvu_all; g2.ldc = kvw;
+        RDT_TRY(launch_gemm(x.dtype, EPI_STORE_T, g2, x.s));
+        ap.k1 = kvu_all; ap.k1_b = (long long)tm * kvw; ap.k1_j = kvw; ap.k1_g = dn + dv;
+        ap.k2 = kr_c; ap.k2_b = (long long)tm * dr; ap.k2_j = dr;
+        ap.v = (const char*)kvu_all + (size_t)dn * es; ap.v_b = (long long)tm * kvw; ap.v_j = kvw; ap.v_g = dn + dv;
+        ap.key_pos0 = 0;
+        ap.n_keys = decode ? tm : start_pos + T;
+      }
+    }
     ap.scale = 1.f / sqrtf((float)(dn + dr));
   }
   ap.o = attn; ap.o_row = (long long)H * dv; ap.o_head = dv;
@@ -356,7 +385,6 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
   if (cache) {
     if (!cache->k || !cache->v || cache->t_max <= 0 || cache->batch < B || cache->n_loops < n_loops)
       return RDT_ERR_INVALID_ARG;
-    if (c->attn_type != 0) return RDT_ERR_UNSUPPORTED;
     if (!decode && start_pos + T > cache->t_max) return RDT_ERR_INVALID_ARG;
     max_keys = std::max(max_keys, cache->t_max);
   }

@@ -1,0 +1,130 @@
+"""MLA with a latent cache on the GPU: prefill fills one (c_kv, k_rope) cache per loop,
+a decode step or a later prefill chunk reads it back and rebuilds the per-head keys and
+values ("OpenMythos 분석", MLA; "RoPE & generation cache").  Compared with the oracle's
+decode step (which takes the same latent cache), with its prefill of the whole sequence,
+and with the GPU's own prefill."""
+import pytest
+import torch
+
+import rdt_inputs as RI
+from oracle import rdt_oracle as O
+from tests._helpers import BF16_TOL, FP32_TOL, max_rel, rel_l2, to_dev
+
+pytestmark = pytest.mark.gpu
+
+R = pytest.importorskip("recurrent_depth_moe_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    R.load_library()
+
+
+def _tiny(dtype):
+    return RI.get_workload("tiny_mla_fp32").cfg.replace(dtype=dtype)
+
+
+def _mid(dtype):
+    # wider latent (128) and head dims (nope 64, rope 32, v 64): GEMMs large enough for the tensor-core path
+    return RI.RDTConfig(dim=512, n_heads=4, n_kv_heads=4, max_seq_len=256, max_loop_iters=4, n_experts=8,
+                        n_shared_experts=1, n_experts_per_tok=2, expert_dim=128, lora_rank=8, attn_type="mla",
+                        kv_lora_rank=128, q_lora_rank=192, qk_rope_head_dim=32, qk_nope_head_dim=64,
+                        v_head_dim=64, dtype=dtype)
+
+
+def _latent_cache(cfg, L, B, t_max):
+    z = lambda w: torch.zeros(L, B, t_max, w, dtype=cfg.torch_dtype, device="cuda")
+    return R.KVCache(z(cfg.kv_lora_rank), z(cfg.qk_rope_head_dim))
+
+
+def _close(got, want, dtype):
+    if dtype == "fp32":
+        assert max_rel(got, want) <= FP32_TOL
+    else:
+        assert rel_l2(got, want) <= BF16_TOL
+
+
+@pytest.mark.parametrize("make", [_tiny, _mid])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_mla_prefill_then_decode_matches_oracle_and_prefill(make, dtype):
+    cfg = make(dtype)
+    W = RI.block_weights(cfg, 51, attn_std=0.08, halt_w_std=0.2)
+    B, T, L, thr, t_max = 3, 37, 3, 0.99, 64
+    h0, e = RI.recurrent_inputs(cfg, B, T + 1, 52)
+    keep = torch.tensor([b * (T + 1) + i for b in range(B) for i in range(T)])
+    last = torch.tensor([b * (T + 1) + T for b in range(B)])
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    cache = _latent_cache(cfg, L, B, t_max)
+    blk.forward(h0[keep].cuda(), e[keep].cuda(), B, T, L, thr, cache=cache)
+    clen = torch.full((B,), T, dtype=torch.int32, device="cuda")
+    d_h, d_hw, d_ids = blk.decode_step(h0[last].cuda(), e[last].cuda(), clen, cache, L, thr)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    full = O.recurrent_forward(cfg, W, h0, e, B, L, thr)
+    _close(d_h, full[0][last], dtype)
+    assert max_rel(d_hw, full[1][:, last]) <= (FP32_TOL if dtype == "fp32" else 2e-2)
+    if dtype == "fp32":
+        assert torch.equal(d_ids.cpu().long(), full[2][:, last])
+    # the cache now holds the latent entries of all T + 1 positions of every loop
+    for t in range(L):
+        for b in range(B):
+            c_kv, k_rope = full[3][t][b]
+            _close(cache.k[t, b, :T + 1], c_kv, dtype)
+            _close(cache.v[t, b, :T + 1], k_rope, dtype)
+    assert not cache.k[:, :, T + 1:].any()              # nothing written past the new token
+    p_h, p_hw, p_ids = blk.forward(h0.cuda(), e.cuda(), B, T + 1, L, thr)
+    assert rel_l2(d_h, p_h[last.cuda()]) <= (1e-5 if dtype == "fp32" else 1e-2)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_mla_decode_random_latent_cache_ragged_lengths(dtype):
+    """Decode against random per-loop latent caches with a different length per sequence."""
+    cfg = _mid(dtype)
+    W = RI.block_weights(cfg, 53, attn_std=0.05)
+    B, L, t_max = 4, 3, 160
+    lens = [37, 100, 64, 5]
+    ckv, kr = RI.random_latent_cache(cfg, L, B, t_max, max(lens), 54)
+    for b, n in enumerate(lens):                       # positions >= len are not part of the cache
+        ckv[:, b, n:] = 0
+        kr[:, b, n:] = 0
+    h0, e = RI.decode_inputs(cfg, B, 0, 55)
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    cache = R.KVCache(ckv.cuda(), kr.cuda())
+    clen = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    d_h, d_hw, d_ids = blk.decode_step(h0.cuda(), e.cuda(), clen, cache, L, 0.0)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    caches = [[{"c_kv": ckv[t, b, :lens[b]], "k_rope": kr[t, b, :lens[b]], "pos": torch.arange(lens[b])}
+               for b in range(B)] for t in range(L)]
+    o_h, o_hw, o_ids, new_kv = O.decode_step(cfg, W, h0, e, caches, lens, L, 0.0)
+    _close(d_h, o_h, dtype)
+    if dtype == "fp32":
+        assert torch.equal(d_ids.cpu().long(), o_ids)
+    for t in range(L):
+        for b in range(B):
+            _close(cache.k[t, b, lens[b]], new_kv[t][b][0][0], dtype)
+            _close(cache.v[t, b, lens[b]], new_kv[t][b][1][0], dtype)
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_mla_chunked_prefill_reads_the_latent_cache(dtype):
+    """A second prefill chunk at start_pos = T1 attends to the first chunk through the
+    latent cache: its rows equal the oracle's prefill of the whole T1 + T2 tokens."""
+    cfg = _mid(dtype)
+    W = RI.block_weights(cfg, 56, attn_std=0.08, halt_w_std=0.2)
+    B, T1, T2, L, thr, t_max = 2, 40, 24, 3, 0.99, 80
+    h0, e = RI.recurrent_inputs(cfg, B, T1 + T2, 57)
+    first = torch.tensor([b * (T1 + T2) + i for b in range(B) for i in range(T1)])
+    second = torch.tensor([b * (T1 + T2) + T1 + i for b in range(B) for i in range(T2)])
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    cache = _latent_cache(cfg, L, B, t_max)
+    blk.forward(h0[first].cuda(), e[first].cuda(), B, T1, L, thr, cache=cache)
+    c_h, c_hw, c_ids = blk.forward(h0[second].cuda(), e[second].cuda(), B, T2, L, thr, start_pos=T1, cache=cache)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    full = O.recurrent_forward(cfg, W, h0, e, B, L, thr)
+    _close(c_h, full[0][second], dtype)
+    if dtype == "fp32":
+        assert torch.equal(c_ids.cpu().long(), full[2][:, second])

@@ -395,6 +395,29 @@ def test_decode_step_equals_prefill_of_one_more_token(act):
     assert torch.equal(dec[2], full[2][:, last])
 
 
+@pytest.mark.parametrize("act", [0.0, 0.99])
+def test_mla_decode_from_latent_cache_equals_prefill(act):
+    """MLA: a decode step that reads only the latent cache (c_kv, k_rope) of the T earlier
+    positions gives the prefill of T+1 tokens ("OpenMythos 분석", MLA: the cache holds the
+    latent; "RoPE & generation cache")."""
+    cfg = RI.get_workload("tiny_mla_fp32").cfg
+    W = weights(cfg, seed=4, attn_std=0.1, halt_w_std=0.3)
+    B, T, L = 2, 6, 5
+    h0, e = RI.recurrent_inputs(cfg, B, T + 1, 17)
+    full = O.recurrent_forward(cfg, W, h0, e, B, L, act)
+    keep = torch.tensor([b * (T + 1) + i for b in range(B) for i in range(T)])
+    pre = O.recurrent_forward(cfg, W, h0[keep], e[keep], B, L, act)
+    caches = [[{"c_kv": pre[3][t][b][0], "k_rope": pre[3][t][b][1], "pos": torch.arange(T)} for b in range(B)]
+              for t in range(L)]
+    assert caches[0][0]["c_kv"].shape == (T, cfg.kv_lora_rank)
+    assert caches[0][0]["k_rope"].shape == (T, cfg.qk_rope_head_dim)
+    last = torch.tensor([b * (T + 1) + T for b in range(B)])
+    dec = O.decode_step(cfg, W, h0[last], e[last], caches, [T] * B, L, act)
+    assert torch.allclose(dec[0], full[0][last], atol=1e-12)
+    assert torch.allclose(dec[1], full[1][:, last], atol=1e-12)
+    assert torch.equal(dec[2], full[2][:, last])
+
+
 def test_mla_absorbed_form_matches():
     """Scores via the absorbed form q_nope^T (W_uk c_kv) == q_nope . k_nope (DeepSeek-V2)."""
     wl = RI.get_workload("tiny_mla_fp32")
