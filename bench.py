@@ -280,6 +280,8 @@ def run_ours(args, wl, rank, world, local_rank):
     del blk, ws, W, out, h0_d, e_d
     torch.cuda.empty_cache()
     decode_res = None if args.no_decode else run_decode(args, rank, world, local_rank)
+    mla_res = None if args.no_decode or args.no_mla_decode else run_decode(args, rank, world, local_rank,
+                                                                             "rdt3b_mla_decode")
 
     if rank != 0:
         return
@@ -314,6 +316,8 @@ def run_ours(args, wl, rank, world, local_rank):
            "clocks": clk}
     if not args.no_decode:
         res["decode"] = decode_res
+        if mla_res is not None:
+            res["decode_mla"] = mla_res
     if W_cpu is not None:
         pos, loops = 64, 8
         rate, dt = oracle_sample(wl, W_cpu, h0_c, e_c, pos, loops)
@@ -323,18 +327,36 @@ def run_ours(args, wl, rank, world, local_rank):
     print(json.dumps(res), flush=True)
 
 
+def attn_weight_bytes(cfg) -> int:
+    """bf16 bytes of one loop's attention weights."""
+    D, H = cfg.dim, cfg.n_heads
+    if cfg.attn_type == "gqa":
+        hd, Hkv = cfg.head_dim, cfg.n_kv_heads
+        return ((H + 2 * Hkv) * hd * D + D * H * hd) * 2
+    dn, dr, dv, kvr, ql = (cfg.qk_nope_head_dim, cfg.qk_rope_head_dim, cfg.v_head_dim, cfg.kv_lora_rank,
+                           cfg.q_lora_rank)
+    return (ql * D + H * (dn + dr) * ql + (kvr + dr) * D + H * (dn + dv) * kvr + D * H * dv) * 2
+
+
+def cache_bytes_per_key(cfg) -> int:
+    """bf16 bytes one cached position holds per loop: K and V of every kv head (GQA), or
+    the latent c_kv plus one k_rope shared by all heads (MLA)."""
+    if cfg.attn_type == "gqa":
+        return 2 * cfg.n_kv_heads * cfg.head_dim * 2
+    return (cfg.kv_lora_rank + cfg.qk_rope_head_dim) * 2
+
+
 def decode_algorithmic_bytes(cfg, ids: torch.Tensor, lens: torch.Tensor) -> float:
     """HBM bytes one decode step must move at minimum: every expert a loop touches is
     streamed once (routed experts by the realised routing, plus the shared ones), the
     attention / router / LoRA weights once per loop, each sequence's cache of that loop
-    read once (cache_len + 1 keys and values) and one new K/V row written."""
+    read once (cache_len + 1 positions) and one new cache row written."""
     D, F, E, S = cfg.dim, cfg.expert_dim, cfg.n_experts, cfg.n_shared_experts
-    hd, H, Hkv = cfg.head_dim, cfg.n_heads, cfg.n_kv_heads
     expert_bytes = 3 * D * F * 2
-    attn_bytes = ((H + 2 * Hkv) * hd * D + D * H * hd) * 2
+    attn_bytes = attn_weight_bytes(cfg)
     small = (E * D + 2 * cfg.lora_rank * D) * 2
     L = ids.shape[0]
-    kv = float((lens.double() + 1).sum()) * Hkv * hd * 2 * 2
+    kv = float((lens.double() + 1).sum()) * cache_bytes_per_key(cfg)
     total = 0.0
     for t in range(L):
         distinct = int(torch.unique(ids[t][ids[t] >= 0]).numel())
@@ -342,18 +364,20 @@ def decode_algorithmic_bytes(cfg, ids: torch.Tensor, lens: torch.Tensor) -> floa
     return total
 
 
-def run_decode(args, rank, world, local_rank):
-    """3B-shaped KV-cached decode: 64 sequences with 4096-token random caches per loop,
-    one new token per sequence per step over `decode_steps` steps."""
+def run_decode(args, rank, world, local_rank, name="rdt3b_decode"):
+    """3B-shaped KV-cached decode: 64 sequences with 4096-token random caches per loop
+    (GQA K/V, or the MLA latent cache), one new token per sequence per step over
+    `decode_steps` steps."""
     import recurrent_depth_moe_b200 as R
     from recurrent_depth_moe_b200 import _native as NAT
     dev = torch.device("cuda", local_rank)
-    wl = RI.get_workload("rdt3b_decode")
+    wl = RI.get_workload(name)
     cfg = wl.cfg
     B, L, steps = wl.batch, wl.n_loops, args.decode_steps
     t_max = wl.cache_len + steps + args.warmup
     W = RI.block_weights(cfg, wl.seed, device=dev)
-    k, v = RI.random_kv_cache(cfg, L, B, t_max, wl.cache_len, REP.replica_input_seed(wl.seed, rank), device=dev)
+    make_cache = RI.random_kv_cache if cfg.attn_type == "gqa" else RI.random_latent_cache
+    k, v = make_cache(cfg, L, B, t_max, wl.cache_len, REP.replica_input_seed(wl.seed, rank), device=dev)
     h0s, es = [], []
     for st in range(steps + args.warmup):
         h, e = RI.decode_inputs(cfg, B, st, REP.replica_input_seed(wl.seed, rank), device=dev)
@@ -395,12 +419,31 @@ def run_decode(args, rank, world, local_rank):
     bytes_step = decode_algorithmic_bytes(cfg, out[2].cpu(), (clen - 1).cpu())
     pk, pk_kind = peaks()
     gbs = bytes_step / (ms / 1e3) / 1e9
+    # attention alone: the cache bytes of all timed steps over the attention kernels' time
+    keys_read = float(steps * (lens0.double() + 1).sum() + B * steps * (steps - 1) / 2) * L
+    attn_ms = prof.get("attention", (0, 0.0))[1] / steps
+    attn_bytes = keys_read / steps * cache_bytes_per_key(cfg)
+    attn_gbs = attn_bytes / (attn_ms / 1e3) / 1e9 if attn_ms else None
+    if cfg.attn_type == "gqa":
+        attn_desc = f"{cfg.n_heads} heads GQA ({cfg.n_kv_heads} kv, head dim {cfg.head_dim})"
+        attn_kernel = "k_attn_decode_mma + k_attn_decode_combine (split-KV, mma.sync)"
+    else:
+        attn_desc = (f"{cfg.n_heads} heads MLA (kv_lora_rank {cfg.kv_lora_rank}, q_lora_rank {cfg.q_lora_rank}, "
+                     f"rope {cfg.qk_rope_head_dim}, nope {cfg.qk_nope_head_dim}, v {cfg.v_head_dim}; latent cache, "
+                     f"absorbed)")
+        attn_kernel = "k_mla_q_absorb + k_mla_attn + k_mla_out (split-KV latent attention, mma.sync)"
     res = {"metric": "decode tokens/s", "value": B * world / (ms_max / 1e3), "unit": "tokens/s",
            "ms_per_step": ms_max, "steps": steps,
-           "workload": (f"{wl.name}: 3B-shaped KV-cached decode, dim {cfg.dim}, {cfg.n_heads} heads GQA "
-                        f"({cfg.n_kv_heads} kv), {cfg.n_experts} routed + {cfg.n_shared_experts} shared experts "
+           "workload": (f"{wl.name}: 3B-shaped KV-cached decode, dim {cfg.dim}, {attn_desc}, "
+                        f"{cfg.n_experts} routed + {cfg.n_shared_experts} shared experts "
                         f"top-{cfg.n_experts_per_tok}, expert_dim {cfg.expert_dim}, {L} loops, batch {B} sequences "
                         f"with {wl.cache_len}-token random caches per loop, 1 new token per step, bf16, ACT off"),
+           "cache_bytes_per_token_loop": cache_bytes_per_key(cfg),
+           "attention_roofline": {"bound": "hbm", "kernel": attn_kernel, "achieved": attn_gbs,
+                                  "peak": pk.get("hbm_gbs"), "unit": "GB/s",
+                                  "frac": attn_gbs / pk.get("hbm_gbs") if attn_gbs else None,
+                                  "ms_per_step": attn_ms, "cache_bytes_per_step": attn_bytes,
+                                  "peak_kind": f"{pk_kind} HBM copy bandwidth"},
            "roofline": {"bound": "hbm", "kernel": "whole decode step (expert weights + caches streamed)",
                         "achieved": gbs, "peak": pk.get("hbm_gbs"), "unit": "GB/s",
                         "frac": gbs / pk.get("hbm_gbs"), "peak_kind": f"{pk_kind} HBM copy bandwidth",
@@ -421,6 +464,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=128)
+    ap.add_argument("--no-mla-decode", action="store_true", help="skip the multi-latent-attention decode line")
+    ap.add_argument("--decode-only", default=None,
+                    choices=["rdt3b_decode", "rdt3b_mla_decode", "mla_decode_attn_small"],
+                    help="profiling: run only this decode workload and print its line")
     ap.add_argument("--workload", default=WORKLOAD, choices=["rdt1b_prefill", "rdt10b_prefill_zipf"])
     ap.add_argument("--batch", type=int, default=None, help="override the sequences per step (small profiling cases)")
     ap.add_argument("--loops", type=int, default=None, help="override n_loops (small profiling cases)")
@@ -449,7 +496,12 @@ def main():
     if world > 1:
         torch.distributed.barrier()
     try:
-        run_ours(args, wl, rank, world, local_rank)
+        if args.decode_only:
+            res = run_decode(args, rank, world, local_rank, args.decode_only)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+        else:
+            run_ours(args, wl, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -130,6 +130,25 @@ WORKLOADS = {
         n_experts=64, n_shared_experts=1, n_experts_per_tok=4, expert_dim=4096, lora_rank=16,
         dtype="bf16"), batch=64, seq=1, n_loops=16, seed=3, act_threshold=0.0, kind="decode",
         cache_len=4096, decode_steps=128, device_weights=True),
+    # The same decode with multi-latent attention: the pages fix MLA dims only for the tiny
+    # model, so the latent widths are DeepSeek-V2's (the MLA design the pages cite):
+    # kv_lora_rank 512, q_lora_rank 1536, rope 64, nope 128, v 128.  Per loop and token the
+    # latent cache holds (512 + 64) x 2 bytes against 2 x 8 x 128 x 2 for the GQA cache.
+    "rdt3b_mla_decode": Workload("rdt3b_mla_decode", RDTConfig(
+        dim=3072, n_heads=24, n_kv_heads=24, max_seq_len=4096 + 128, max_loop_iters=16,
+        n_experts=64, n_shared_experts=1, n_experts_per_tok=4, expert_dim=4096, lora_rank=16,
+        attn_type="mla", kv_lora_rank=512, q_lora_rank=1536, qk_rope_head_dim=64, qk_nope_head_dim=128,
+        v_head_dim=128, dtype="bf16"), batch=64, seq=1, n_loops=16, seed=5, act_threshold=0.0, kind="decode",
+        cache_len=4096, decode_steps=128, device_weights=True),
+    # Profiling case for the latent attention: the attention of rdt3b_mla_decode (same
+    # heads, latent widths, batch and cache length) with a small MoE and 2 loops, so that
+    # well under 1 GB is held on the device.
+    "mla_decode_attn_small": Workload("mla_decode_attn_small", RDTConfig(
+        dim=3072, n_heads=24, n_kv_heads=24, max_seq_len=4096 + 128, max_loop_iters=2,
+        n_experts=8, n_shared_experts=1, n_experts_per_tok=2, expert_dim=128, lora_rank=16,
+        attn_type="mla", kv_lora_rank=512, q_lora_rank=1536, qk_rope_head_dim=64, qk_nope_head_dim=128,
+        v_head_dim=128, dtype="bf16"), batch=64, seq=1, n_loops=2, seed=6, act_threshold=0.0, kind="decode",
+        cache_len=4096, decode_steps=8, device_weights=True),
     # 10B-shaped prefill, load-imbalanced (mythos_10b: dim 4096, 128 experts, expert_dim 5632, 24 loops).
     "rdt10b_prefill_zipf": Workload("rdt10b_prefill_zipf", RDTConfig(
         dim=4096, n_heads=32, n_kv_heads=8, max_seq_len=8192, max_loop_iters=24,

@@ -90,6 +90,24 @@ struct AttnParams {
 int launch_attention(int dtype, const AttnParams& p, cudaStream_t s);
 int launch_attention_decode(int dtype, const AttnParams& p, cudaStream_t s);
 
+// MLA decode on the latent cache, weight-absorbed (bf16): q absorption, split-KV latent
+// attention over all heads of a sequence, range merge + value absorption into o.
+struct MlaDecodeParams {
+  int B, H, dn, dr, dv, kvr;
+  const void* q; long long q_row; int q_head;   // [B][H][dn + dr]: q_nope, rotated q_rope
+  const void* w_kvu; const float* kv_norm_w;    // [H (dn + dv)][kvr], [kvr]
+  float eps, scale;
+  const void* ckv; const void* krope; int t_max;  // this loop's cache: [B][t_max][kvr], [B][t_max][dr]
+  const int* q_pos;                             // [B] new-token position = cache_len[b]
+  void* qa;                                     // scratch [B][H][kvr]
+  float* part_o; float* part_ml; int n_split;   // [B][H][n_split][kvr], [B][H][n_split][2]
+  void* o; long long o_row;                     // attention output [B][H dv]
+};
+bool mla_decode_supports(int attn_type, int dtype, int H, int kvr, int dr, int dn, int dv);
+int mla_decode_splits(int B, int t_max);
+int launch_mla_decode(const MlaDecodeParams& p, cudaStream_t s);
+int tc_sm_count();
+
 // ------------------------------------------------------------------------------------------
 // MoE routing and permutation
 // ------------------------------------------------------------------------------------------

@@ -25,6 +25,8 @@ struct Layout {
   size_t ids, gates, rank, counts, offsets, tiles, ntiles, slot_of, tok_of, gate_of, xg, u, y;
   size_t run_list, run_idx, nrun, cum, halted, Avec, emb, rope, pos, p_buf, part_o, part_ml, xn, vt;
   size_t mla_ckv_all, mla_kvu_all;   // MLA with earlier cached keys: rebuilt per-head keys / values
+  size_t mla_qa;                     // MLA absorbed decode: absorbed queries (0 = path not used)
+  int part_dim;                      // split-KV partial width (head dim, or kv_lora_rank)
   size_t total;
   int max_tiles, max_slots, rope_dim, rope_pos, n_split;
 };
@@ -86,7 +88,10 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
     L->krope = take(N * dr * es);
     L->kvu = take(N * (size_t)H * (dn + dv) * es);
     L->rope_dim = dr;
-    if (max_keys > T) {   // earlier positions come from the latent cache
+    if (T == 1 && mla_decode_supports(1, c->dtype, H, c->kv_lora_rank, dr, dn, dv)) {
+      // decode on the latent cache in the absorbed form: nothing per head is rebuilt
+      L->mla_qa = take((size_t)B * H * c->kv_lora_rank * es);
+    } else if (max_keys > T) {   // earlier positions come from the latent cache
       L->mla_ckv_all = take((size_t)B * max_keys * c->kv_lora_rank * es);
       L->mla_kvu_all = take((size_t)B * max_keys * H * (dn + dv) * es);
     }
@@ -124,7 +129,12 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
   L->pos = take(N * 4);
   // decode layouts (one row per sequence) hold the split-KV attention partials
   L->n_split = (T == 1) ? decode_split_count(std::max(max_keys, 1)) : 0;
-  L->part_o = take(L->n_split ? (size_t)B * H * L->n_split * 128 * 4 : 16);
+  L->part_dim = 128;
+  if (L->mla_qa) {
+    L->n_split = mla_decode_splits(B, std::max(max_keys, 1));
+    L->part_dim = c->kv_lora_rank;
+  }
+  L->part_o = take(L->n_split ? (size_t)B * H * L->n_split * L->part_dim * 4 : 16);
   L->part_ml = take(L->n_split ? (size_t)B * H * L->n_split * 2 * 4 : 16);
   L->total = off;
 }
@@ -168,6 +178,7 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
   memset(&ap, 0, sizeof(ap));
   ap.B = B; ap.T = T; ap.H = H; ap.q_pos = pos;
   int dv;
+  bool absorbed = false;   // MLA decode ran in the absorbed form (attention output written)
   if (c->attn_type == 0) {
     const int Hkv = c->n_kv_heads, hd = D / H, W = (H + 2 * Hkv) * hd;
     void* qkv = at<void*>(x.ws, x.L.qkv);
@@ -220,23 +231,29 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
     void* ckv = at<void*>(x.ws, x.L.ckv);
     void* krope = at<void*>(x.ws, x.L.krope);
     void* kvu = at<void*>(x.ws, x.L.kvu);
-    GemmParams g = gemm_base(x);
-    g.A = a; g.lda = D; g.B = w->w_q_down; g.ldb = D; g.M = N; g.N = ql; g.K = D; g.C = cq_raw; g.ldc = ql;
-    RDT_TRY(launch_gemm(x.dtype, EPI_STORE_F32, g, x.s));
-    launch_rmsnorm(1, x.dtype, cq_raw, ql, w->q_norm_w, cq, ql, N, ql, c->norm_eps, x.s);
-    g = gemm_base(x);
-    g.A = cq; g.lda = ql; g.B = w->w_q_up; g.ldb = ql; g.M = N; g.N = H * (dn + dr); g.K = ql;
-    g.C = q; g.ldc = H * (dn + dr); g.pos = pos; g.rope_tab = tab; g.rope_half = dr / 2; g.n_rope = 1;
-    g.rope[0] = RopeDesc{0, H, dn + dr, dn, dr};
-    RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, x.s));
-    g = gemm_base(x);
-    g.A = a; g.lda = D; g.B = w->w_kv_down; g.ldb = D; g.M = N; g.N = kvr + dr; g.K = D; g.C = kv_raw; g.ldc = kvr + dr;
-    RDT_TRY(launch_gemm(x.dtype, EPI_STORE_F32, g, x.s));
-    launch_mla_kv_prep(x.dtype, kv_raw, kvr, dr, w->kv_norm_w, c->norm_eps, pos, tab, ckv, krope, N, x.s);
-    g = gemm_base(x);
-    g.A = ckv; g.lda = kvr; g.B = w->w_kv_up; g.ldb = kvr; g.M = N; g.N = H * (dn + dv); g.K = kvr;
-    g.C = kvu; g.ldc = H * (dn + dv);
-    RDT_TRY(launch_gemm(x.dtype, EPI_STORE_T, g, x.s));
+    {
+      ProfScope ps_proj(PC_QKV, x.s);   // the projections, up to the attention proper
+      GemmParams g = gemm_base(x);
+      g.A = a; g.lda = D; g.B = w->w_q_down; g.ldb = D; g.M = N; g.N = ql; g.K = D; g.C = cq_raw; g.ldc = ql;
+      RDT_TRY(launch_gemm(x.dtype, EPI_STORE_F32, g, x.s));
+      launch_rmsnorm(1, x.dtype, cq_raw, ql, w->q_norm_w, cq, ql, N, ql, c->norm_eps, x.s);
+      g = gemm_base(x);
+      g.A = cq; g.lda = ql; g.B = w->w_q_up; g.ldb = ql; g.M = N; g.N = H * (dn + dr); g.K = ql;
+      g.C = q; g.ldc = H * (dn + dr); g.pos = pos; g.rope_tab = tab; g.rope_half = dr / 2; g.n_rope = 1;
+      g.rope[0] = RopeDesc{0, H, dn + dr, dn, dr};
+      RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, x.s));
+      g = gemm_base(x);
+      g.A = a; g.lda = D; g.B = w->w_kv_down; g.ldb = D; g.M = N; g.N = kvr + dr; g.K = D; g.C = kv_raw; g.ldc = kvr + dr;
+      RDT_TRY(launch_gemm(x.dtype, EPI_STORE_F32, g, x.s));
+      launch_mla_kv_prep(x.dtype, kv_raw, kvr, dr, w->kv_norm_w, c->norm_eps, pos, tab, ckv, krope, N, x.s);
+      absorbed = T == 1 && cache && cache->k && x.L.mla_qa;   // one row per sequence, keys from the cache
+      if (!absorbed) {   // per-head [k_nope | v] of this call's rows
+        g = gemm_base(x);
+        g.A = ckv; g.lda = kvr; g.B = w->w_kv_up; g.ldb = kvr; g.M = N; g.N = H * (dn + dv); g.K = kvr;
+        g.C = kvu; g.ldc = H * (dn + dv);
+        RDT_TRY(launch_gemm(x.dtype, EPI_STORE_T, g, x.s));
+      }
+    }
     const long long kvw = (long long)H * (dn + dv);
     ap.q = q; ap.q_row = H * (dn + dr); ap.q_head = dn + dr; ap.dn = dn; ap.dr = dr; ap.dv = dv; ap.G = 1;
     ap.k1 = kvu; ap.k1_b = (long long)T * kvw; ap.k1_j = kvw; ap.k1_g = dn + dv;
@@ -249,7 +266,20 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
       char* ckv_c = (char*)cache->k + (size_t)loop_t * cache->batch * tm * kvr * es;
       char* kr_c = (char*)cache->v + (size_t)loop_t * cache->batch * tm * dr * es;
       { ProfScope ps(PC_OTHER, x.s); launch_mla_to_cache(x.dtype, kv_raw, krope, kvr, dr, pos, N, T, tm, ckv_c, kr_c, x.st, x.s); }
-      if (decode || start_pos > 0) {
+      if (absorbed) {
+        MlaDecodeParams mp;
+        memset(&mp, 0, sizeof(mp));
+        mp.B = B; mp.H = H; mp.dn = dn; mp.dr = dr; mp.dv = dv; mp.kvr = kvr;
+        mp.q = q; mp.q_row = (long long)H * (dn + dr); mp.q_head = dn + dr;
+        mp.w_kvu = w->w_kv_up; mp.kv_norm_w = w->kv_norm_w; mp.eps = c->norm_eps;
+        mp.scale = 1.f / sqrtf((float)(dn + dr));
+        mp.ckv = ckv_c; mp.krope = kr_c; mp.t_max = tm; mp.q_pos = pos;
+        mp.qa = at<void*>(x.ws, x.L.mla_qa);
+        mp.part_o = at<float*>(x.ws, x.L.part_o); mp.part_ml = at<float*>(x.ws, x.L.part_ml); mp.n_split = x.L.n_split;
+        mp.o = attn; mp.o_row = (long long)H * dv;
+        ProfScope ps(PC_ATTN, x.s);
+        if (launch_mla_decode(mp, x.s) != 0) return RDT_ERR_CUDA;
+      } else if (decode || start_pos > 0) {
         // keys / values of every cached position: [k_nope | v] = RMSNorm(c_kv) W_kvu^T
         if (!x.L.mla_kvu_all) return RDT_ERR_WORKSPACE;
         void* ckv_all = at<void*>(x.ws, x.L.mla_ckv_all);
@@ -271,7 +301,7 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
     ap.scale = 1.f / sqrtf((float)(dn + dr));
   }
   ap.o = attn; ap.o_row = (long long)H * dv; ap.o_head = dv;
-  { ProfScope ps(PC_ATTN, x.s); RDT_TRY(launch_attention(x.dtype, ap, x.s)); }
+  if (!absorbed) { ProfScope ps(PC_ATTN, x.s); RDT_TRY(launch_attention(x.dtype, ap, x.s)); }
   GemmParams g = gemm_base(x);
   g.A = attn; g.lda = (long long)H * dv; g.B = w->w_o; g.ldb = (long long)H * dv; g.M = N; g.N = D; g.K = H * dv;
   g.C = x1; g.ldc = D; g.resid = combined; g.ld_resid = D;

@@ -113,3 +113,32 @@ def test_rdt10b_zipf_prefill_properties():
     # the Zipf bias makes the load imbalanced: popular experts take far more than E / k share
     counts = torch.bincount(ids_c[0][ids_c[0] >= 0].flatten(), minlength=cfg.n_experts).double()
     assert counts.max() / counts.mean() > 3.0
+
+
+def test_rdt3b_mla_decode_sequence_matches_oracle():
+    """3B-shaped decode with multi-latent attention at full size (64 sequences, per-loop
+    4096-token random latent caches, kv_lora_rank 512): sequence 37 against the oracle
+    decode step, and the new latent entries of every loop."""
+    wl = RI.get_workload("rdt3b_mla_decode")
+    cfg, B, L = wl.cfg, wl.batch, wl.n_loops
+    dev = torch.device("cuda")
+    t_max = wl.cache_len + 8
+    W = RI.block_weights(cfg, wl.seed, device=dev)
+    ckv, kr = RI.random_latent_cache(cfg, L, B, t_max, wl.cache_len, wl.seed, device=dev)
+    h0, e = RI.decode_inputs(cfg, B, 0, wl.seed, device=dev)
+    blk = R.RecurrentBlock(cfg, W)
+    cache = R.KVCache(ckv, kr)
+    clen = torch.full((B,), wl.cache_len, dtype=torch.int32, device=dev)
+    d_h, d_hw, d_ids = blk.decode_step(h0, e, clen, cache, L, wl.act_threshold)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    assert torch.isfinite(d_h).all()
+    Wc = _cpu(W)
+    b = 37
+    caches = [[{"c_kv": ckv[t, b, :wl.cache_len].cpu(), "k_rope": kr[t, b, :wl.cache_len].cpu(),
+                "pos": torch.arange(wl.cache_len)}] for t in range(L)]
+    o_h, o_hw, o_ids, new_kv = O.decode_step(cfg, Wc, h0[b:b + 1].cpu(), e[b:b + 1].cpu(), caches, [wl.cache_len],
+                                             L, wl.act_threshold)
+    assert rel_l2(d_h[b:b + 1], o_h) <= BF16_TOL
+    for t in range(L):
+        assert rel_l2(ckv[t, b, wl.cache_len], new_kv[t][0][0][0]) <= BF16_TOL

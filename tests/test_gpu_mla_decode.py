@@ -1,8 +1,9 @@
-"""MLA with a latent cache on the GPU: prefill fills one (c_kv, k_rope) cache per loop,
-a decode step or a later prefill chunk reads it back and rebuilds the per-head keys and
-values ("OpenMythos 분석", MLA; "RoPE & generation cache").  Compared with the oracle's
-decode step (which takes the same latent cache), with its prefill of the whole sequence,
-and with the GPU's own prefill."""
+"""MLA with a latent cache on the GPU: prefill fills one (c_kv, k_rope) cache per loop; a
+single-row call (decode step, or one token at start_pos > 0) reads it in the
+weight-absorbed form (bf16) or by rebuilding the per-head keys and values (fp32), and a
+later prefill chunk rebuilds them ("OpenMythos 분석", MLA; "RoPE & generation cache").
+Compared with the oracle's decode step (which takes the same latent cache), with its
+prefill of the whole sequence, and with the GPU's own prefill."""
 import pytest
 import torch
 
@@ -128,3 +129,61 @@ def test_mla_chunked_prefill_reads_the_latent_cache(dtype):
     _close(c_h, full[0][second], dtype)
     if dtype == "fp32":
         assert torch.equal(c_ids.cpu().long(), full[2][:, second])
+
+
+def _wide(H):
+    # DeepSeek-V2 latent widths (kv_lora_rank 512, rope 64); H 16 fills one 16-row MMA
+    # tile, H 24 two tiles with 8 padded rows
+    return RI.RDTConfig(dim=1536, n_heads=H, n_kv_heads=H, max_seq_len=1024, max_loop_iters=4, n_experts=8,
+                        n_shared_experts=1, n_experts_per_tok=2, expert_dim=128, lora_rank=8, attn_type="mla",
+                        kv_lora_rank=512, q_lora_rank=256, qk_rope_head_dim=64, qk_nope_head_dim=128,
+                        v_head_dim=128, dtype="bf16")
+
+
+@pytest.mark.parametrize("H", [16, 24])
+def test_mla_absorbed_decode_wide_latent_ragged(H):
+    """Absorbed decode at kv_lora_rank 512 against the oracle's decode step, with ragged
+    cache lengths: several key ranges, a tile-aligned length + 1, an empty cache (the new
+    token alone) and a single cached token."""
+    cfg = _wide(H)
+    W = RI.block_weights(cfg, 60 + H, attn_std=0.05)
+    B, L, t_max = 5, 2, 720
+    lens = [300, 700, 64, 0, 1]
+    ckv, kr = RI.random_latent_cache(cfg, L, B, t_max, max(lens), 61)
+    for b, n in enumerate(lens):
+        ckv[:, b, n:] = 0
+        kr[:, b, n:] = 0
+    h0, e = RI.decode_inputs(cfg, B, 0, 62)
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    cache = R.KVCache(ckv.cuda(), kr.cuda())
+    clen = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    d_h, d_hw, d_ids = blk.decode_step(h0.cuda(), e.cuda(), clen, cache, L, 0.0)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    caches = [[{"c_kv": ckv[t, b, :lens[b]], "k_rope": kr[t, b, :lens[b]], "pos": torch.arange(lens[b])}
+               for b in range(B)] for t in range(L)]
+    o_h, o_hw, o_ids, new_kv = O.decode_step(cfg, W, h0, e, caches, lens, L, 0.0)
+    for b in range(B):                                  # every sequence on its own, not just on average
+        assert rel_l2(d_h[b], o_h[b]) <= BF16_TOL, b
+    for t in range(L):                                  # the new token's latent entry, every loop
+        for b in range(B):
+            assert rel_l2(cache.k[t, b, lens[b]], new_kv[t][b][0][0]) <= BF16_TOL
+
+
+def test_mla_single_token_prefill_through_the_cache():
+    """rdt_recurrent_forward with one token at start_pos > 0 reads the latent cache the
+    same way as the decode step."""
+    cfg = _mid("bf16")
+    W = RI.block_weights(cfg, 63, attn_std=0.08, halt_w_std=0.2)
+    B, T, L, thr, t_max = 2, 20, 3, 0.99, 32
+    h0, e = RI.recurrent_inputs(cfg, B, T + 1, 64)
+    keep = torch.tensor([b * (T + 1) + i for b in range(B) for i in range(T)])
+    last = torch.tensor([b * (T + 1) + T for b in range(B)])
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    cache = _latent_cache(cfg, L, B, t_max)
+    blk.forward(h0[keep].cuda(), e[keep].cuda(), B, T, L, thr, cache=cache)
+    s_h, s_hw, s_ids = blk.forward(h0[last].cuda(), e[last].cuda(), B, 1, L, thr, start_pos=T, cache=cache)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    full = O.recurrent_forward(cfg, W, h0, e, B, L, thr)
+    assert rel_l2(s_h, full[0][last]) <= BF16_TOL
