@@ -225,10 +225,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < BKV; ++c)
           if (kp0 + c > my_pos || k0 + c >= n_vis) s[c] = -INFINITY;
       }
-      float mx = -INFINITY;
+      // row max as 8 independent chains and a tree (max is exact in any order)
+      float mp[8];
 #pragma unroll
-      for (int c = 0; c < BKV; ++c) mx = fmaxf(mx, s[c]);
-      mx *= a.sl2;                               // the scale is positive: max commutes with it
+      for (int k = 0; k < 8; ++k) mp[k] = s[k];
+#pragma unroll
+      for (int c = 8; c < BKV; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
+#pragma unroll
+      for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int k = 0; k < w; ++k) mp[k] = fmaxf(mp[k], mp[k + w]);
+      const float mx = mp[0] * a.sl2;            // the scale is positive: max commutes with it
       float alpha = 1.f;
       if (j == 0) {
         m_used = mx;
@@ -239,15 +246,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       const float base = (m_used == -INFINITY) ? 0.f : m_used;
       uint32_t pk[BKV / 2];
-      float sum = 0.f;
+      float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 partial sums, then a tree
 #pragma unroll
       for (int c = 0; c < BKV; c += 2) {
         const float p0 = exp2f(fmaf(s[c], a.sl2, -base)), p1 = exp2f(fmaf(s[c + 1], a.sl2, -base));
-        sum += p0 + p1;
+        sp[(c >> 1) & 7] += p0 + p1;
         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
         pk[c >> 1] = *reinterpret_cast<uint32_t*>(&h2);
       }
-      l += sum;
+#pragma unroll
+      for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int k = 0; k < w; ++k) sp[k] += sp[k + w];
+      l += sp[0];
       if (j >= 1) {
         // PV of tile j-1 done: O is stable and the P buffer is free
         if (!(ok = mbar_wait(&pv_done[q], (j - 1) & 1, abort_flag))) break;

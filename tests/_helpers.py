@@ -91,3 +91,31 @@ def halting_loop(hw: torch.Tensor) -> torch.Tensor:
     L = hw.shape[0]
     nz = (hw.cpu() > 0).to(torch.int64) * torch.arange(L)[:, None]
     return nz.max(dim=0).values
+
+
+HALT_MARGIN = 2e-2   # bf16: a position may halt at another loop only where the oracle's cum + p is this close to thr
+
+
+def same_halting_rows(hw_gpu: torch.Tensor, hw_oracle: torch.Tensor, record: list, thr: float,
+                      seq: int = 0) -> torch.Tensor:
+    """ACT halts a position when cum + p reaches the threshold ("OpenMythos 분석", ACT), a
+    decision taken on a float: within rounding of the threshold bf16 and fp64 may halt one
+    loop apart, as a top-k near-tie may route apart.  Asserts that every position whose
+    halting loop differs had, in the oracle, cum + p within HALT_MARGIN of thr at the
+    earlier of the two loops.  Returns the mask of positions whose result is still
+    determined: a halted row is frozen but its keys and values are recomputed every loop,
+    so a position that halts at another loop changes what every later position of its
+    sequence attends to.  With seq > 0 (rows sequence-major, seq positions each) those
+    later positions are left out as well; with seq = 0 only the position itself."""
+    hg, ho = halting_loop(hw_gpu), halting_loop(hw_oracle)
+    diff = hg != ho
+    if diff.any():
+        t_first = torch.minimum(hg, ho)[diff]
+        cum = torch.stack([r["cum"] for r in record])            # [L, N] oracle cum after loop t
+        near = (cum[t_first, torch.nonzero(diff)[:, 0]] - thr).abs() < HALT_MARGIN
+        assert near.all(), f"{int((~near).sum())} positions halt at another loop away from the threshold"
+    if seq <= 0:
+        return ~diff
+    d = diff.view(-1, seq).to(torch.int64)
+    downstream = torch.cumsum(d, dim=1) > 0                     # at or after the first disagreement
+    return ~downstream.reshape(-1)
