@@ -211,6 +211,21 @@ RDT_API rdt_status rdt_block_forward(const rdt_config* cfg, const rdt_weights* w
                              const float* x_in, float* x_out, int batch, int seq, int start_pos,
                              void* ws, size_t ws_bytes, void* stream);
 
+/* rdt_block_forward with a KV cache for the block (a prelude or coda layer of the
+ * generation loop, "OpenMythos 분석", RoPE & generation cache: one cache per layer).
+ *  cache: NULL (same as rdt_block_forward), or the block's cache in the layout of
+ *         rdt_kv_cache with n_loops >= 1 (slot 0 is used).
+ *  cache_len: NULL for a prefill at positions start_pos..start_pos+seq-1 (written to
+ *         the cache; earlier positions are read from it when start_pos > 0), or device
+ *         int32 [batch] for a decode step (seq = 1): the new token of sequence b is at
+ *         position cache_len[b], written there, and attends to positions 0..cache_len[b].
+ *  Workspace: rdt_workspace_size(cfg, batch, seq, max(start_pos + seq, cache->t_max)).
+ *  Invalid: decode without a cache or with seq != 1; a prefill past cache->t_max. */
+RDT_API rdt_status rdt_block_forward_cached(const rdt_config* cfg, const rdt_weights* w,
+                                            const float* x_in, float* x_out, int batch, int seq, int start_pos,
+                                            const int32_t* cache_len, const rdt_kv_cache* cache,
+                                            void* ws, size_t ws_bytes, void* stream);
+
 /* Token embedding gather ("OpenMythos 분석", Core Structure: self.embed(input_ids)):
  * out[i] = table[ids[i]] widened to fp32.  table [vocab, D] model dtype; ids int32 [n]. */
 RDT_API rdt_status rdt_embed(const rdt_config* cfg, const void* table, int vocab, const int32_t* ids, int n,
@@ -222,6 +237,25 @@ RDT_API rdt_status rdt_embed(const rdt_config* cfg, const void* table, int vocab
 RDT_API rdt_status rdt_head(const rdt_config* cfg, const float* x, int n, const float* norm_w,
                     const void* head, int vocab, float* logits,
                     void* ws, size_t ws_bytes, void* stream);
+
+/* rdt_head on n rows of x spaced x_ld floats apart (x_ld >= dim), e.g. the last
+ * position of each sequence of a prefill (x_ld = seq * dim).  logits [n, vocab]. */
+RDT_API rdt_status rdt_head_rows(const rdt_config* cfg, const float* x, long long x_ld, int n,
+                                 const float* norm_w, const void* head, int vocab, float* logits,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/* Greedy next token of generation (the pages print the generation loop but not its
+ * sampling rule; the plainest reading is the most likely token): for each row b < n,
+ * tokens[b * out_ld] = argmax_v logits[b * vocab + v], ties to the lowest index; NaN
+ * is never chosen (a row of NaN gives 0).  logits fp32 and tokens int32, device. */
+RDT_API rdt_status rdt_greedy_tokens(const float* logits, int n, int vocab, int32_t* tokens, int out_ld,
+                                     void* stream);
+
+/* out[i] = x[i] in the model dtype (fp32 copy, or bf16 round-to-nearest-even), i < n:
+ * the recurrent block's injected input e is the prelude output in the model dtype
+ * ("OpenMythos 분석", Core Structure: e = x after the prelude).  Device pointers. */
+RDT_API rdt_status rdt_to_model_dtype(const rdt_config* cfg, const float* x, void* out, long long n,
+                                      void* stream);
 
 /* Synchronise `stream`, read and clear the device status word in `ws`. */
 RDT_API rdt_status rdt_read_device_status(void* ws, void* stream);

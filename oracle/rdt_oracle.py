@@ -394,6 +394,30 @@ def model_forward(cfg, MW: dict, ids: torch.Tensor, n_loops: int, act_threshold:
     return logits.reshape(B, T, -1), rec, e
 
 
+def greedy(logits: torch.Tensor) -> torch.Tensor:
+    """The most likely next token per row, ties to the lowest index (the pages print the
+    generation loop but not its sampling rule; greedy is the plainest reading).
+    torch.argmax returns the first maximal index."""
+    return torch.argmax(logits, dim=-1)
+
+
+def generate(cfg, MW: dict, prompt_ids: torch.Tensor, max_new_tokens: int, n_loops: int,
+             act_threshold: float = 0.0):
+    """OpenMythos.generate ("OpenMythos 분석", RoPE & generation cache), by its definition:
+    every new token is the greedy choice from the last position of a full forward pass
+    over all tokens so far.  No cache: the library's cached steps (prompt at start_pos 0,
+    then one token at position prompt_len + step - 1) must reproduce this.
+    Returns (ids [B, T0 + n] int64, step logits [n, B, V])."""
+    ids = prompt_ids.clone().to(torch.int64)
+    step_logits = []
+    for _ in range(max_new_tokens):
+        logits, _, _ = model_forward(cfg, MW, ids, n_loops, act_threshold)
+        last = logits[:, -1]
+        step_logits.append(last)
+        ids = torch.cat([ids, greedy(last)[:, None]], dim=1)
+    return ids, torch.stack(step_logits)
+
+
 def decode_step(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, caches: list, cache_len: list,
                 n_loops: int, act_threshold: float = 0.0):
     """One KV-cached decode step of the recurrent block ("OpenMythos 분석", "RoPE &

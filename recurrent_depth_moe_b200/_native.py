@@ -55,7 +55,8 @@ class rdt_kernel_time(ctypes.Structure):
 
 
 EXPORTS = ("rdt_workspace_size", "rdt_recurrent_forward", "rdt_recurrent_decode_step", "rdt_block_forward",
-           "rdt_embed", "rdt_head", "rdt_read_device_status", "rdt_status_string", "rdt_version",
+           "rdt_block_forward_cached", "rdt_embed", "rdt_head", "rdt_head_rows", "rdt_greedy_tokens",
+           "rdt_to_model_dtype", "rdt_read_device_status", "rdt_status_string", "rdt_version",
            "rdt_launch_count", "rdt_profile_start", "rdt_profile_stop")
 
 _lib = None
@@ -82,6 +83,15 @@ def load(path: str = LIB_PATH):
     lib.rdt_block_forward.argtypes = [POINTER(rdt_config), POINTER(rdt_weights), P, P, c_int, c_int, c_int, P,
                                       c_size_t, P]
     lib.rdt_block_forward.restype = c_int
+    lib.rdt_block_forward_cached.argtypes = [POINTER(rdt_config), POINTER(rdt_weights), P, P, c_int, c_int, c_int,
+                                             P, POINTER(rdt_kv_cache), P, c_size_t, P]
+    lib.rdt_block_forward_cached.restype = c_int
+    lib.rdt_head_rows.argtypes = [POINTER(rdt_config), P, ctypes.c_longlong, c_int, P, P, c_int, P, P, c_size_t, P]
+    lib.rdt_head_rows.restype = c_int
+    lib.rdt_greedy_tokens.argtypes = [P, c_int, c_int, P, c_int, P]
+    lib.rdt_greedy_tokens.restype = c_int
+    lib.rdt_to_model_dtype.argtypes = [POINTER(rdt_config), P, P, ctypes.c_longlong, P]
+    lib.rdt_to_model_dtype.restype = c_int
     lib.rdt_embed.argtypes = [POINTER(rdt_config), P, c_int, P, c_int, P, P]
     lib.rdt_embed.restype = c_int
     lib.rdt_head.argtypes = [POINTER(rdt_config), P, c_int, P, P, c_int, P, P, c_size_t, P]

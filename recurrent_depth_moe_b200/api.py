@@ -222,6 +222,40 @@ class RecurrentBlock:
         return lib.rdt_read_device_status(self._ws.data_ptr(), _stream()) if self._ws is not None else N.RDT_OK
 
 
+class Block:
+    """One pre-norm prelude/coda block (dense SwiGLU FFN) or MoE block bound to its weights."""
+
+    def __init__(self, cfg, weights: dict, dense: bool = True):
+        _require_cuda()
+        self.cfg = cfg
+        self.cs = dense_config_struct(cfg) if dense else config_struct(cfg)
+        self.w = Weights(weights, _DT[cfg.dtype][1])
+
+    def workspace(self, batch: int, seq: int, max_keys: int) -> torch.Tensor:
+        return alloc_workspace(workspace_size(self.cs, batch, seq, max_keys))
+
+    def forward(self, x: torch.Tensor, batch: int, seq: int, start_pos: int = 0, cache: Optional[KVCache] = None,
+                cache_len: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """rdt_block_forward_cached: prefill at start_pos (cache_len None) or one decode
+        step at positions cache_len[b] (seq 1); cache None = no cache."""
+        lib = N.load()
+        _check_act(x, "x", torch.float32, (batch * seq, self.cfg.dim))
+        if cache_len is not None:
+            _check_act(cache_len, "cache_len", torch.int32, (batch,))
+        out = torch.empty_like(x) if out is None else out
+        max_keys = start_pos + seq if cache is None else max(start_pos + seq, cache.t_max)
+        ws = workspace if workspace is not None else self.workspace(batch, seq, max_keys)
+        cs = cache.struct() if cache is not None else None
+        rc = lib.rdt_block_forward_cached(ctypes.byref(self.cs), ctypes.byref(self.w.struct), x.data_ptr(),
+                                          out.data_ptr(), batch, seq, start_pos,
+                                          None if cache_len is None else cache_len.data_ptr(),
+                                          None if cs is None else ctypes.byref(cs), ws.data_ptr(), ws.numel(),
+                                          _stream())
+        N.check("rdt_block_forward_cached", rc)
+        return out
+
+
 def block_forward(cfg, weights: dict, x: torch.Tensor, batch: int, seq: int, start_pos: int = 0,
                   dense: bool = True) -> torch.Tensor:
     """rdt_block_forward: one pre-norm prelude/coda block (dense SwiGLU FFN) or a MoE block."""
@@ -237,6 +271,28 @@ def block_forward(cfg, weights: dict, x: torch.Tensor, batch: int, seq: int, sta
     return out
 
 
+def to_model_dtype(cfg, x: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """rdt_to_model_dtype: the prelude output as the recurrent block's injected input e."""
+    lib = _require_cuda()
+    if not x.is_cuda or not x.is_contiguous() or x.dtype != torch.float32:
+        raise ValueError("x: expected a contiguous CUDA float32 tensor")
+    out = torch.empty(x.shape, dtype=_DT[cfg.dtype][1], device=x.device) if out is None else out
+    rc = lib.rdt_to_model_dtype(ctypes.byref(config_struct(cfg)), x.data_ptr(), out.data_ptr(), x.numel(), _stream())
+    N.check("rdt_to_model_dtype", rc)
+    return out
+
+
+def greedy_tokens(logits: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """rdt_greedy_tokens: argmax per row of fp32 logits [n, V], ties to the lowest index."""
+    lib = _require_cuda()
+    _check_act(logits, "logits", torch.float32, tuple(logits.shape))
+    n, V = logits.shape
+    out = torch.empty(n, dtype=torch.int32, device=logits.device) if out is None else out
+    rc = lib.rdt_greedy_tokens(logits.data_ptr(), n, V, out.data_ptr(), 1, _stream())
+    N.check("rdt_greedy_tokens", rc)
+    return out
+
+
 def embed(cfg, table: torch.Tensor, ids: torch.Tensor) -> torch.Tensor:
     lib = _require_cuda()
     cs = config_struct(cfg)
@@ -248,14 +304,25 @@ def embed(cfg, table: torch.Tensor, ids: torch.Tensor) -> torch.Tensor:
     return out
 
 
-def head(cfg, x: torch.Tensor, norm_w: torch.Tensor, head_w: torch.Tensor) -> torch.Tensor:
+def head(cfg, x: torch.Tensor, norm_w: torch.Tensor, head_w: torch.Tensor, last_of: int = 0,
+         out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """rdt_head / rdt_head_rows: logits of every row of x [n, D], or with last_of = T of
+    the last row of each T-row sequence (x [B * T, D] -> logits [B, V])."""
     lib = _require_cuda()
     cs = config_struct(cfg)
-    n = x.shape[0]
-    out = torch.empty(n, head_w.shape[0], dtype=torch.float32, device="cuda")
-    ws = alloc_workspace(workspace_size(cs, 1, n, n))
-    rc = lib.rdt_head(ctypes.byref(cs), x.data_ptr(), n, norm_w.data_ptr(), head_w.data_ptr(), head_w.shape[0],
-                      out.data_ptr(), ws.data_ptr(), ws.numel(), _stream())
+    if not x.is_cuda or not x.is_contiguous() or x.dtype != torch.float32 or x.shape[-1] != cfg.dim:
+        raise ValueError("x: expected a contiguous CUDA float32 [n, dim] tensor")
+    n = x.shape[0] // last_of if last_of else x.shape[0]
+    V = head_w.shape[0]
+    out = torch.empty(n, V, dtype=torch.float32, device="cuda") if out is None else out
+    ws = workspace if workspace is not None else alloc_workspace(workspace_size(cs, 1, n, n))
+    if last_of:
+        ptr = x.data_ptr() + (last_of - 1) * cfg.dim * 4
+        rc = lib.rdt_head_rows(ctypes.byref(cs), ptr, last_of * cfg.dim, n, norm_w.data_ptr(), head_w.data_ptr(), V,
+                               out.data_ptr(), ws.data_ptr(), ws.numel(), _stream())
+    else:
+        rc = lib.rdt_head(ctypes.byref(cs), x.data_ptr(), n, norm_w.data_ptr(), head_w.data_ptr(), V,
+                          out.data_ptr(), ws.data_ptr(), ws.numel(), _stream())
     N.check("rdt_head", rc)
     return out
 
@@ -268,11 +335,127 @@ def model_forward(cfg, MW: dict, ids: torch.Tensor, n_loops: int, act_threshold:
     x = embed(cfg, MW["embed"], ids)
     for W in MW["prelude"]:
         x = block_forward(cfg, W, x, B, T)
-    e = x.to(_DT[cfg.dtype][1]).contiguous()
+    e = to_model_dtype(cfg, x)
     rb = RecurrentBlock(cfg, MW["recurrent"])
-    rec = rb.forward(x.contiguous(), e, B, T, n_loops, act_threshold)
+    rec = rb.forward(x, e, B, T, n_loops, act_threshold)
     x = rec[0]
     for W in MW["coda"]:
         x = block_forward(cfg, W, x, B, T)
     logits = head(cfg, x, MW["norm_w"], MW["head"])
     return logits.reshape(B, T, -1), rec
+
+
+def _layer_cache(cfg, n_loops: int, batch: int, t_max: int) -> KVCache:
+    """Zeroed per-loop (or, with n_loops 1, per-layer) cache in the layout of rdt_kv_cache."""
+    dt = _DT[cfg.dtype][1]
+    if cfg.attn_type == "gqa":
+        z = torch.zeros(n_loops, batch, cfg.n_kv_heads, t_max, cfg.head_dim, dtype=dt, device="cuda")
+        return KVCache(z, torch.zeros_like(z))
+    return KVCache(torch.zeros(n_loops, batch, t_max, cfg.kv_lora_rank, dtype=dt, device="cuda"),
+                   torch.zeros(n_loops, batch, t_max, cfg.qk_rope_head_dim, dtype=dt, device="cuda"))
+
+
+class Generator:
+    """OpenMythos.generate on the library's entry points ("OpenMythos 분석", RoPE &
+    generation cache): step 0 runs the whole prompt at start_pos 0 and fills one cache per
+    prelude / coda layer and per recurrent loop; every later step runs the last token
+    alone at position prompt_len + step - 1 against those caches.  The next token is the
+    greedy choice (rdt_greedy_tokens).  All buffers are allocated once per generator, so
+    the decode steps allocate nothing."""
+
+    def __init__(self, cfg, MW: dict, batch: int, prompt_len: int, max_new_tokens: int, n_loops: int,
+                 act_threshold: float = 0.0):
+        _require_cuda()
+        self.cfg, self.MW = cfg, MW
+        self.B, self.T0, self.new, self.L, self.thr = batch, prompt_len, max_new_tokens, n_loops, act_threshold
+        self.t_max = prompt_len + max_new_tokens
+        B, D, T0 = batch, cfg.dim, prompt_len
+        self.pre = [Block(cfg, W) for W in MW["prelude"]]
+        self.coda = [Block(cfg, W) for W in MW["coda"]]
+        self.rb = RecurrentBlock(cfg, MW["recurrent"])
+        self.pre_cache = [_layer_cache(cfg, 1, B, self.t_max) for _ in self.pre]
+        self.coda_cache = [_layer_cache(cfg, 1, B, self.t_max) for _ in self.coda]
+        self.rec_cache = _layer_cache(cfg, n_loops, B, self.t_max)
+        sizes = [workspace_size(b.cs, B, s, self.t_max) for b in self.pre + self.coda for s in (T0, 1)]
+        self.ws_block = alloc_workspace(max(sizes + [256]))
+        self.ws_rec_prefill = self.rb.workspace(B, T0, self.t_max)
+        self.ws_rec_decode = self.rb.workspace(B, 1, self.t_max)
+        cs = config_struct(cfg)
+        self.ws_head = alloc_workspace(workspace_size(cs, 1, B, B))
+        V = MW["head"].shape[0]
+        dt = _DT[cfg.dtype][1]
+        self.xa = torch.empty(B * T0, D, dtype=torch.float32, device="cuda")
+        self.xb = torch.empty_like(self.xa)
+        self.e = torch.empty(B * T0, D, dtype=dt, device="cuda")
+        self.rec_out = (torch.empty(B * T0, D, dtype=torch.float32, device="cuda"),
+                        torch.empty(n_loops, B * T0, dtype=torch.float32, device="cuda"),
+                        torch.empty(n_loops, B * T0, cfg.n_experts_per_tok, dtype=torch.int32, device="cuda"))
+        self.logits = torch.empty(B, V, dtype=torch.float32, device="cuda")
+        self.tokens = torch.empty(max_new_tokens, B, dtype=torch.int32, device="cuda")
+        self.dec_out = (torch.empty(B, D, dtype=torch.float32, device="cuda"),
+                        torch.empty(n_loops, B, dtype=torch.float32, device="cuda"),
+                        torch.empty(n_loops, B, cfg.n_experts_per_tok, dtype=torch.int32, device="cuda"))
+        self.cache_len = torch.empty(B, dtype=torch.int32, device="cuda")
+
+    def _run_blocks(self, blocks, caches, x, y, seq, start_pos, cache_len):
+        for blk, c in zip(blocks, caches):
+            blk.forward(x, self.B, seq, start_pos, cache=c, cache_len=cache_len, out=y, workspace=self.ws_block)
+            x, y = y, x
+        return x, y
+
+    def prefill(self, prompt_ids: torch.Tensor) -> torch.Tensor:
+        """Step 0: the prompt [B, T0] (int32, CUDA); returns the first new token [B]."""
+        B, T0, D = self.B, self.T0, self.cfg.dim
+        lib = N.load()
+        ids = prompt_ids.reshape(-1)
+        if not ids.is_cuda or ids.dtype != torch.int32 or ids.numel() != B * T0 or not ids.is_contiguous():
+            raise ValueError("prompt_ids: expected a contiguous CUDA int32 [batch, prompt_len] tensor")
+        x, y = self.xa, self.xb
+        rc = lib.rdt_embed(ctypes.byref(config_struct(self.cfg)), self.MW["embed"].data_ptr(),
+                           self.MW["embed"].shape[0], ids.data_ptr(), B * T0, x.data_ptr(), _stream())
+        N.check("rdt_embed", rc)
+        x, y = self._run_blocks(self.pre, self.pre_cache, x, y, T0, 0, None)
+        to_model_dtype(self.cfg, x, out=self.e)
+        self.rb.forward(x, self.e, B, T0, self.L, self.thr, start_pos=0, cache=self.rec_cache, out=self.rec_out,
+                        workspace=self.ws_rec_prefill)
+        x, y = self._run_blocks(self.coda, self.coda_cache, self.rec_out[0], y, T0, 0, None)
+        head(self.cfg, x, self.MW["norm_w"], self.MW["head"], last_of=T0, out=self.logits, workspace=self.ws_head)
+        greedy_tokens(self.logits, out=self.tokens[0])
+        return self.tokens[0]
+
+    def decode(self, step: int) -> torch.Tensor:
+        """Step `step` >= 1: the token of step - 1 at position prompt_len + step - 1."""
+        B, D = self.B, self.cfg.dim
+        lib = N.load()
+        self.cache_len.fill_(self.T0 + step - 1)
+        x, y = self.xa[:B], self.xb[:B]
+        rc = lib.rdt_embed(ctypes.byref(config_struct(self.cfg)), self.MW["embed"].data_ptr(),
+                           self.MW["embed"].shape[0], self.tokens[step - 1].data_ptr(), B, x.data_ptr(), _stream())
+        N.check("rdt_embed", rc)
+        x, y = self._run_blocks(self.pre, self.pre_cache, x, y, 1, 0, self.cache_len)
+        e = self.e[:B]
+        to_model_dtype(self.cfg, x, out=e)
+        out = self.dec_out
+        self.rb.decode_step(x, e, self.cache_len, self.rec_cache, self.L, self.thr, out=out,
+                            workspace=self.ws_rec_decode)
+        x, y = self._run_blocks(self.coda, self.coda_cache, out[0], y, 1, 0, self.cache_len)
+        head(self.cfg, x, self.MW["norm_w"], self.MW["head"], out=self.logits, workspace=self.ws_head)
+        greedy_tokens(self.logits, out=self.tokens[step])
+        return self.tokens[step]
+
+    def run(self, prompt_ids: torch.Tensor) -> torch.Tensor:
+        """Prompt [B, T0] -> the generated tokens [B, max_new_tokens] (int32, CUDA)."""
+        self.prefill(prompt_ids)
+        for step in range(1, self.new):
+            self.decode(step)
+        return self.tokens.t()
+
+
+def generate(cfg, MW: dict, prompt_ids: torch.Tensor, max_new_tokens: int, n_loops: int,
+             act_threshold: float = 0.0) -> torch.Tensor:
+    """Greedy generation: returns [B, T0 + max_new_tokens] token ids (int32, CUDA)."""
+    B, T0 = prompt_ids.shape
+    ids = prompt_ids.to(device="cuda", dtype=torch.int32).contiguous()
+    gen = Generator(cfg, MW, B, T0, max_new_tokens, n_loops, act_threshold)
+    new = gen.run(ids)
+    return torch.cat([ids, new], dim=1)

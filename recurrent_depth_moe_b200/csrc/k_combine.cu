@@ -53,6 +53,32 @@ template <> __device__ __forceinline__ float4 ld4<bf16>(const bf16* p) {
   return make_float4(fa.x, fa.y, fb.x, fb.y);
 }
 
+// Warp sums of 16 values at once (a transposed butterfly, 16 shuffles instead of 80):
+// at each step a lane keeps one half of its values, sends the other half to its partner
+// and adds the partner's copy of the half it kept.  Lanes 2q and 2q + 1 end with the sum
+// of v[q] over the warp.
+__device__ __forceinline__ float warp_sum16(const float (&v)[16], int lane) {
+  float a[8], b[4], c[2];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const bool hi = lane & 16;
+    a[i] = (hi ? v[i + 8] : v[i]) + __shfl_xor_sync(0xffffffffu, hi ? v[i] : v[i + 8], 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const bool hi = lane & 8;
+    b[i] = (hi ? a[i + 4] : a[i]) + __shfl_xor_sync(0xffffffffu, hi ? a[i] : a[i + 4], 8);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const bool hi = lane & 4;
+    c[i] = (hi ? b[i + 2] : b[i]) + __shfl_xor_sync(0xffffffffu, hi ? b[i] : b[i + 2], 4);
+  }
+  const bool hi = lane & 2;
+  float d = (hi ? c[1] : c[0]) + __shfl_xor_sync(0xffffffffu, hi ? c[0] : c[1], 2);
+  return d + __shfl_xor_sync(0xffffffffu, d, 1);
+}
+
 // A row is processed by a group of WPR warps; warp wr of the group owns the float4
 // columns 4 lane + 128 j for j in [wr VQ, (wr + 1) VQ), VQ = VPL / WPR.  Row-wide sums go
 // through shared memory: each warp reduces its part, lane 0 stores it in slot `slot` of
@@ -153,18 +179,19 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
 #pragma unroll
     for (int j = 0; j < VQ; ++j)
       tr[j] = __ldg(reinterpret_cast<const float4*>(p.x1 + rowD + 4 * lane + 128 * (j0 + j)));
+    // the row's slot indices in one warp load; lane s holds slot s (invalid ones -> -1)
+    int my_slot = -2;
+    if (lane < kS) {
+      my_slot = __ldg(p.slot_of + (long long)i * kS + lane);
+      if (my_slot < 0 || my_slot >= p.max_slots) {
+        if (lead) record_status(p.st, ST_BOUNDS, 202, my_slot);
+        my_slot = -1;
+      }
+    }
     // slot rows two at a time, so two rows' loads are in flight per memory round trip
-    const int* so = p.slot_of + (long long)i * kS;
     for (int s = 0; s < kS; s += 2) {
-      int s0 = so[s], s1 = (s + 1 < kS) ? so[s + 1] : -2;
-      if (s0 < 0 || s0 >= p.max_slots) {
-        if (lead && lane == 0) record_status(p.st, ST_BOUNDS, 202, s0);
-        s0 = -1;
-      }
-      if (s1 != -2 && (s1 < 0 || s1 >= p.max_slots)) {
-        if (lead && lane == 0) record_status(p.st, ST_BOUNDS, 202, s1);
-        s1 = -1;
-      }
+      const int s0 = __shfl_sync(0xffffffffu, my_slot, s);
+      const int s1 = (s + 1 < kS) ? __shfl_sync(0xffffffffu, my_slot, s + 1) : -1;
       const T* y0 = (const T*)p.y + (long long)max(s0, 0) * D + 4 * lane;
       const T* y1 = (const T*)p.y + (long long)max(s1, 0) * D + 4 * lane;
 #pragma unroll
@@ -183,24 +210,34 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
   }
   if (!p.transformer_off && p.r > 0) {
     const float* sc = p.lora_scale + (long long)min(p.t, p.max_loop_iters - 1) * p.r;
-    float zq[16];
-    // rank in chunks of 16: partial projections of this warp's columns, then the group sum
+    // rank in chunks of 16: partial projections of this warp's columns, one transposed warp
+    // reduction, then the group sum; lane q of every warp ends with z[q0 + q]
     for (int q0 = 0; q0 < p.r; q0 += 16) {
       const int nq = min(16, p.r - q0);
+      float part[16];
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        float part = 0.f;
+        part[q] = 0.f;
         if (q < nq) {
           const T* w = Wd + (long long)(q0 + q) * D + 4 * lane;
 #pragma unroll
-          for (int j = 0; j < VQ; ++j) part += f4_dot(tr[j], ld4<T>(w + 128 * (j0 + j)));
+          for (int j = 0; j < VQ; ++j) part[q] += f4_dot(tr[j], ld4<T>(w + 128 * (j0 + j)));
         }
-        zq[q] = warp_sum(part);
       }
-      g.reduce<16>(zq, nq, 0, lane);
-      if (lane == 0)
-        for (int q = 0; q < nq; ++q) z[q0 + q] = zq[q] * sc[q0 + q];
-      if (q0 + 16 < p.r) g.sync();   // slots 0..15 are rewritten by the next chunk
+      const float ws = warp_sum16(part, lane);           // sum of part[lane >> 1]
+      if (WPR == 1) {
+        if ((lane & 1) == 0 && (lane >> 1) < nq) z[q0 + (lane >> 1)] = ws * sc[q0 + (lane >> 1)];
+      } else {
+        if ((lane & 1) == 0) g.red[g.wr * 32 + (lane >> 1)] = ws;
+        g.sync();
+        if (g.wr == 0 && lane < nq) {
+          float t = 0.f;
+#pragma unroll
+          for (int w = 0; w < WPR; ++w) t += g.red[w * 32 + lane];
+          z[q0 + lane] = t * sc[q0 + lane];
+        }
+        g.sync();   // z complete; slots 0..15 free for the next chunk
+      }
     }
     __syncwarp();
     // every z_q is complete, so the delta can be added to the row in place

@@ -9,6 +9,8 @@
 #include "kernels.h"
 #include <math.h>
 
+#include <algorithm>
+
 namespace rdt {
 
 // ------------------------------------------------------------------------------------------
@@ -435,6 +437,51 @@ void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* 
 void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s) {
   { k_iota<<<(N + 255) / 256, 256, 0, s>>>(run_list, run_idx, n_run, N); note_launch(); }
 }
+// Greedy choice of the next token: CTA per row, argmax over the vocabulary with ties to
+// the lowest index; NaN compares below every number (a row of NaN gives 0).
+__global__ void __launch_bounds__(256) k_greedy(const float* __restrict__ logits, int vocab,
+                                               int* __restrict__ tokens, int out_ld) {
+  __shared__ float bv_s[8];
+  __shared__ int bi_s[8];
+  const float* row = logits + (long long)blockIdx.x * vocab;
+  float bv = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int v = threadIdx.x; v < vocab; v += 256) {
+    float x = row[v];
+    if (x != x) continue;
+    if (x > bv || (x == bv && v < bi)) { bv = x; bi = v; }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+  }
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) { bv_s[w] = bv; bi_s[w] = bi; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int k = 1; k < 8; ++k)
+      if (bv_s[k] > bv_s[0] || (bv_s[k] == bv_s[0] && bi_s[k] < bi_s[0])) { bv_s[0] = bv_s[k]; bi_s[0] = bi_s[k]; }
+    tokens[(long long)blockIdx.x * out_ld] = bi_s[0] == 0x7fffffff ? 0 : bi_s[0];
+  }
+}
+
+__global__ void k_to_model_dtype(const float* __restrict__ x, bf16* __restrict__ out, long long n) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+    out[i] = __float2bfloat16_rn(x[i]);
+}
+
+void launch_greedy(const float* logits, int n, int vocab, int* tokens, int out_ld, cudaStream_t s) {
+  k_greedy<<<n, 256, 0, s>>>(logits, vocab, tokens, out_ld);
+  note_launch();
+}
+void launch_to_model_dtype(const float* x, void* out, long long n, cudaStream_t s) {
+  const long long blocks = std::min<long long>((n + 255) / 256, 148LL * 16);
+  k_to_model_dtype<<<(unsigned)blocks, 256, 0, s>>>(x, (bf16*)out, n);
+  note_launch();
+}
+
 void launch_embed(int dtype, const void* table, int vocab, const int* ids, int n, int D, float* out,
                   DevStatus* st, cudaStream_t s) {
   if (dtype == 0) { k_embed<float><<<n, 128, 0, s>>>((const float*)table, vocab, ids, D, out, st); note_launch(); }

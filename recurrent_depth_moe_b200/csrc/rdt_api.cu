@@ -558,28 +558,39 @@ rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_weights* w
                        expert_ids, cache, nullptr, 0, ws, ws_bytes, (cudaStream_t)stream, true);
 }
 
-rdt_status rdt_block_forward(const rdt_config* cfg, const rdt_weights* w, const float* x_in, float* x_out, int batch,
-                             int seq, int start_pos, void* ws, size_t ws_bytes, void* stream) {
+rdt_status rdt_block_forward_cached(const rdt_config* cfg, const rdt_weights* w, const float* x_in, float* x_out,
+                                    int batch, int seq, int start_pos, const int32_t* cache_len,
+                                    const rdt_kv_cache* cache, void* ws, size_t ws_bytes, void* stream) {
   rdt_status st = check_config(cfg);
   if (st != RDT_OK) return st;
   const bool moe = cfg->n_experts > 0;
   if ((st = check_block_weights(cfg, w, moe)) != RDT_OK) return st;
   if (!x_in || !x_out || x_in == x_out || batch <= 0 || seq <= 0 || start_pos < 0) return RDT_ERR_INVALID_ARG;
   if (!moe && cfg->n_shared_experts != 1) return RDT_ERR_INVALID_ARG;
+  const bool decode = cache_len != nullptr;
+  int max_keys = start_pos + seq;
+  if (cache) {
+    if (!cache->k || !cache->v || cache->t_max <= 0 || cache->batch < batch || cache->n_loops < 1)
+      return RDT_ERR_INVALID_ARG;
+    if (!decode && start_pos + seq > cache->t_max) return RDT_ERR_INVALID_ARG;
+    max_keys = std::max(max_keys, cache->t_max);
+  }
+  if (decode && (!cache || seq != 1)) return RDT_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   Ctx x;
   x.c = cfg; x.w = w; x.ws = ws; x.s = s; x.dtype = cfg->dtype;
-  make_layout(cfg, batch, seq, start_pos + seq, &x.L);
+  make_layout(cfg, batch, seq, max_keys, &x.L);
   if ((st = check_ws(ws, ws_bytes, x.L)) != RDT_OK) return st;
   x.st = at<DevStatus*>(ws, x.L.status);
   const int N = batch * seq, D = cfg->dim, F = cfg->expert_dim;
   if (cudaMemsetAsync(x.st, 0, sizeof(DevStatus), s) != cudaSuccess) return RDT_ERR_CUDA;
   launch_rope_table(at<float2*>(ws, x.L.rope), x.L.rope_pos, x.L.rope_dim, cfg->rope_theta, s);
-  launch_positions(at<int*>(ws, x.L.pos), N, seq, start_pos, s);
+  if (decode) launch_positions_decode(at<int*>(ws, x.L.pos), cache_len, batch, cache->t_max, x.st, s);
+  else launch_positions(at<int*>(ws, x.L.pos), N, seq, start_pos, s);
   void* a = at<void*>(ws, x.L.a);
   float* x1 = at<float*>(ws, x.L.x1);
   launch_rmsnorm(1, x.dtype, x_in, D, w->attn_norm_w, a, D, N, D, cfg->norm_eps, s);
-  if ((st = attention_block(x, batch, seq, x_in, a, x1, nullptr, 0, start_pos, false)) != RDT_OK) return st;
+  if ((st = attention_block(x, batch, seq, x_in, a, x1, cache, 0, start_pos, decode)) != RDT_OK) return st;
   if (moe) {
     launch_iota(at<int*>(ws, x.L.run_list), at<int*>(ws, x.L.run_idx), at<int*>(ws, x.L.nrun), N, s);
     if ((st = moe_block(x, N, x1)) != RDT_OK) return st;
@@ -602,6 +613,30 @@ rdt_status rdt_block_forward(const rdt_config* cfg, const rdt_weights* w, const 
   return RDT_OK;
 }
 
+rdt_status rdt_block_forward(const rdt_config* cfg, const rdt_weights* w, const float* x_in, float* x_out, int batch,
+                             int seq, int start_pos, void* ws, size_t ws_bytes, void* stream) {
+  return rdt_block_forward_cached(cfg, w, x_in, x_out, batch, seq, start_pos, nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+rdt_status rdt_greedy_tokens(const float* logits, int n, int vocab, int32_t* tokens, int out_ld, void* stream) {
+  if (!logits || !tokens || n <= 0 || vocab <= 0 || out_ld < 1) return RDT_ERR_INVALID_ARG;
+  launch_greedy(logits, n, vocab, tokens, out_ld, (cudaStream_t)stream);
+  return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
+}
+
+rdt_status rdt_to_model_dtype(const rdt_config* cfg, const float* x, void* out, long long n, void* stream) {
+  if (!cfg || (cfg->dtype != 0 && cfg->dtype != 1) || !x || !out || n < 0) return RDT_ERR_INVALID_ARG;
+  if (n == 0) return RDT_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cfg->dtype == 0) {
+    if (x != out && cudaMemcpyAsync(out, x, (size_t)n * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+      return RDT_ERR_CUDA;
+  } else {
+    launch_to_model_dtype(x, out, n, s);
+  }
+  return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
+}
+
 rdt_status rdt_embed(const rdt_config* cfg, const void* table, int vocab, const int32_t* ids, int n, float* out,
                      void* stream) {
   if (!cfg || cfg->dim <= 0 || (cfg->dtype != 0 && cfg->dtype != 1) || !table || !ids || !out || vocab <= 0 || n <= 0)
@@ -610,17 +645,17 @@ rdt_status rdt_embed(const rdt_config* cfg, const void* table, int vocab, const 
   return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
 }
 
-rdt_status rdt_head(const rdt_config* cfg, const float* xin, int n, const float* norm_w, const void* head, int vocab,
-                    float* logits, void* ws, size_t ws_bytes, void* stream) {
+rdt_status rdt_head_rows(const rdt_config* cfg, const float* xin, long long x_ld, int n, const float* norm_w,
+                         const void* head, int vocab, float* logits, void* ws, size_t ws_bytes, void* stream) {
   rdt_status st = check_config(cfg);
   if (st != RDT_OK) return st;
-  if (!xin || n <= 0 || !norm_w || !head || vocab <= 0 || !logits) return RDT_ERR_INVALID_ARG;
+  if (!xin || n <= 0 || x_ld < cfg->dim || !norm_w || !head || vocab <= 0 || !logits) return RDT_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
   Layout L;
   make_layout(cfg, 1, n, n, &L);
   if ((st = check_ws(ws, ws_bytes, L)) != RDT_OK) return st;
   void* xn = at<void*>(ws, L.xn);
-  launch_rmsnorm(1, cfg->dtype, xin, cfg->dim, norm_w, xn, cfg->dim, n, cfg->dim, cfg->norm_eps, s);
+  launch_rmsnorm(1, cfg->dtype, xin, x_ld, norm_w, xn, cfg->dim, n, cfg->dim, cfg->norm_eps, s);
   GemmParams g;
   memset(&g, 0, sizeof(g));
   g.impl = -1;
@@ -628,6 +663,11 @@ rdt_status rdt_head(const rdt_config* cfg, const float* xin, int n, const float*
   g.C = logits; g.ldc = vocab; g.st = at<DevStatus*>(ws, L.status);
   if (launch_gemm(cfg->dtype, EPI_STORE_F32, g, s)) return RDT_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
+}
+
+rdt_status rdt_head(const rdt_config* cfg, const float* xin, int n, const float* norm_w, const void* head, int vocab,
+                    float* logits, void* ws, size_t ws_bytes, void* stream) {
+  return rdt_head_rows(cfg, xin, cfg ? cfg->dim : 0, n, norm_w, head, vocab, logits, ws, ws_bytes, stream);
 }
 
 rdt_status rdt_read_device_status(void* ws, void* stream) {

@@ -488,3 +488,26 @@ def test_mla_latent_cache_entries():
     assert torch.allclose(c_kv, kv_raw[:, :cfg.kv_lora_rank], atol=1e-15)
     want = _rope_complex(kv_raw[:, None, cfg.kv_lora_rank:].contiguous(), torch.arange(T) + 4, 10000.0)[:, 0]
     assert torch.allclose(k_rope, want, atol=1e-13)
+
+
+# 9. generation
+def test_generate_is_causally_consistent():
+    """Causality makes a greedy generation checkable in one pass: the forward pass over the
+    final sequence has, at each position T0 - 1 + s, the logits of step s and the token
+    generated at step s as its argmax (a wrong start position, a non-causal mask or an
+    off-by-one in the loop fails this)."""
+    wl = RI.get_workload("tiny_gqa_fp32")
+    cfg = wl.cfg
+    MW = RI.model_weights(cfg, 3)
+    prompt = torch.randint(0, cfg.vocab_size, (2, 6), generator=torch.Generator().manual_seed(4))
+    ids, step_logits = O.generate(cfg, MW, prompt, 4, n_loops=3)
+    assert torch.equal(ids[:, :6], prompt)
+    full, _, _ = O.model_forward(cfg, MW, ids[:, :-1], 3, 0.0)
+    for s in range(4):
+        assert torch.allclose(full[:, 5 + s], step_logits[s], atol=1e-10)
+        assert torch.equal(torch.argmax(full[:, 5 + s], -1), ids[:, 6 + s])
+
+
+def test_greedy_ties_go_to_the_lowest_index():
+    x = torch.tensor([[0.5, 2.0, 2.0, -1.0], [3.0, 3.0, 3.0, 3.0]], dtype=torch.float64)
+    assert O.greedy(x).tolist() == [1, 0]
