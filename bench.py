@@ -282,6 +282,7 @@ def run_ours(args, wl, rank, world, local_rank):
     decode_res = None if args.no_decode else run_decode(args, rank, world, local_rank)
     mla_res = None if args.no_decode or args.no_mla_decode else run_decode(args, rank, world, local_rank,
                                                                              "rdt3b_mla_decode")
+    gen_res = None if args.no_decode or args.no_generate else run_generate(args, rank, world, local_rank)
 
     if rank != 0:
         return
@@ -318,6 +319,8 @@ def run_ours(args, wl, rank, world, local_rank):
         res["decode"] = decode_res
         if mla_res is not None:
             res["decode_mla"] = mla_res
+        if gen_res is not None:
+            res["generate"] = gen_res
     if W_cpu is not None:
         pos, loops = 64, 8
         rate, dt = oracle_sample(wl, W_cpu, h0_c, e_c, pos, loops)
@@ -455,6 +458,87 @@ def run_decode(args, rank, world, local_rank, name="rdt3b_decode"):
     return res
 
 
+def run_generate(args, rank, world, local_rank):
+    """1B-shaped greedy generation through the library's Generator: the prompt pass
+    (embedding, prelude, 16-loop recurrent prefill filling the caches, coda, head of the
+    last positions), then one decode step per new token.  End to end: the prompt ids are
+    copied in from pinned host memory and the generated ids copied out, inside the timed
+    region."""
+    import recurrent_depth_moe_b200 as R
+    from recurrent_depth_moe_b200 import _native as NAT
+    dev = torch.device("cuda", local_rank)
+    wl = RI.get_workload("rdt1b_generate")
+    cfg = wl.cfg
+    B, T0, new, L = wl.batch, wl.seq, args.generate_new or wl.decode_steps, wl.n_loops
+    MW = RI.model_weights(cfg, wl.seed, device=dev, halt_b=wl.halt_b)
+    g = torch.Generator().manual_seed(REP.replica_input_seed(wl.seed, rank))
+    prompts = [torch.randint(0, cfg.vocab_size, (B, T0), generator=g, dtype=torch.int32).pin_memory()
+               for _ in range(2)]
+    gen = R.Generator(cfg, MW, B, T0, new, L, wl.act_threshold)
+    ids_d = torch.empty(B, T0, dtype=torch.int32, device=dev)
+    out_h = torch.empty(new, B, dtype=torch.int32).pin_memory()
+    stream = torch.cuda.current_stream()
+
+    def one(prompt):
+        ids_d.copy_(prompt, non_blocking=True)
+        gen.prefill(ids_d)
+        for step in range(1, new):
+            gen.decode(step)
+        out_h.copy_(gen.tokens, non_blocking=True)
+
+    one(prompts[0])                                    # warm-up: a whole generation
+    torch.cuda.synchronize()
+    NAT.profile_start()
+    n0 = NAT.launch_count()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    e0.record(stream)
+    ids_d.copy_(prompts[1], non_blocking=True)
+    gen.prefill(ids_d)
+    e1.record(stream)
+    for step in range(1, new):
+        gen.decode(step)
+    out_h.copy_(gen.tokens, non_blocking=True)
+    e2.record(stream)
+    torch.cuda.synchronize()
+    launches = NAT.launch_count() - n0
+    prof = NAT.profile_stop()
+    total_ms = REP.max_over_ranks(e0.elapsed_time(e2), device=dev)
+    prefill_ms = e0.elapsed_time(e1)
+    decode_ms = e1.elapsed_time(e2) / (new - 1)
+    # algorithmic bytes of one decode step: the recurrent block's (16 loops, realised
+    # routing of the last step), the prelude / coda blocks' weights and caches, the head
+    D, Hkv, hd = cfg.dim, cfg.n_kv_heads, cfg.head_dim
+    lens = torch.full((B,), T0 + new - 2)
+    rec_bytes = decode_algorithmic_bytes(cfg, gen.dec_out[2].cpu(), lens)
+    Fd = cfg.dim * 4 // 3
+    block_bytes = (cfg.prelude_layers + cfg.coda_layers) * (
+        attn_weight_bytes(cfg) + 3 * D * Fd * 2 + float((lens + 1).sum()) * cache_bytes_per_key(cfg))
+    head_bytes = cfg.vocab_size * D * 2 + B * D * 2
+    step_bytes = rec_bytes + block_bytes + head_bytes
+    pk, pk_kind = peaks()
+    gbs = step_bytes / (decode_ms / 1e3) / 1e9
+    del gen, MW
+    torch.cuda.empty_cache()
+    return {"metric": "generated tokens/s (greedy, prompt pass included)", "value": B * new * world / (total_ms / 1e3),
+            "unit": "tokens/s", "ms_per_generation": total_ms, "prefill_ms": prefill_ms,
+            "decode_ms_per_token_step": decode_ms,
+            "workload": (f"{wl.name}: 1B-shaped model (dim {D}, {cfg.n_heads} heads GQA ({Hkv} kv), "
+                         f"{cfg.n_experts} routed + {cfg.n_shared_experts} shared experts top-{cfg.n_experts_per_tok}, "
+                         f"expert_dim {cfg.expert_dim}, {L} loops, {cfg.prelude_layers} prelude + {cfg.coda_layers} "
+                         f"coda dense layers, vocab {cfg.vocab_size}), batch {B} sequences, {T0}-token prompts, "
+                         f"{new} new tokens, bf16, ACT 0.99 (halting bias -30)"),
+            "e2e": {"h2d_bytes_per_generation": B * T0 * 4, "d2h_bytes_per_generation": new * B * 4},
+            "decode_roofline": {"bound": "hbm", "kernel": "whole decode step (weights, caches and head streamed)",
+                                "achieved": gbs, "peak": pk.get("hbm_gbs"), "unit": "GB/s",
+                                "frac": gbs / pk.get("hbm_gbs"), "algorithmic_bytes_per_step": step_bytes,
+                                "peak_kind": f"{pk_kind} HBM copy bandwidth"},
+            "gpu_launches": launches,
+            "kernel_ms_per_generation": {k: {"launches": v[0], "ms": v[1]} for k, v in sorted(prof.items())}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -465,6 +549,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=128)
     ap.add_argument("--no-mla-decode", action="store_true", help="skip the multi-latent-attention decode line")
+    ap.add_argument("--no-generate", action="store_true", help="skip the 1B-shaped generation line")
+    ap.add_argument("--generate-only", action="store_true", help="profiling: run only the generation line")
+    ap.add_argument("--generate-new", type=int, default=None, help="profiling: new tokens per generation")
     ap.add_argument("--decode-only", default=None,
                     choices=["rdt3b_decode", "rdt3b_mla_decode", "mla_decode_attn_small"],
                     help="profiling: run only this decode workload and print its line")
@@ -496,8 +583,9 @@ def main():
     if world > 1:
         torch.distributed.barrier()
     try:
-        if args.decode_only:
-            res = run_decode(args, rank, world, local_rank, args.decode_only)
+        if args.decode_only or args.generate_only:
+            res = (run_generate(args, rank, world, local_rank) if args.generate_only else
+                   run_decode(args, rank, world, local_rank, args.decode_only))
             if rank == 0:
                 print(json.dumps(res), flush=True)
         else:

@@ -87,7 +87,7 @@ class Workload:
     n_loops: int
     seed: int
     act_threshold: float            # <= 0: ACT off
-    kind: str = "prefill"           # "prefill" | "decode" | "model"
+    kind: str = "prefill"           # "prefill" | "decode" | "model" | "generate"
     halt_b: float = 0.0             # halting-head bias
     halt_spread: Optional[tuple] = None   # (lo, hi): per-position halting loop via logit offset
     zipf_s: Optional[float] = None  # router bias giving Zipf-like popularity
@@ -140,6 +140,15 @@ WORKLOADS = {
         attn_type="mla", kv_lora_rank=512, q_lora_rank=1536, qk_rope_head_dim=64, qk_nope_head_dim=128,
         v_head_dim=128, dtype="bf16"), batch=64, seq=1, n_loops=16, seed=5, act_threshold=0.0, kind="decode",
         cache_len=4096, decode_steps=128, device_weights=True),
+    # Greedy generation with the 1B-shaped model: the recurrent block of rdt1b_prefill, one
+    # prelude and one coda layer (the usage script's counts; the variant table gives none)
+    # and the vocabulary of the tokenizer the pages name (openai/gpt-oss-20b: 201,088
+    # tokens).  64 sequences, 128-token prompts, 128 new tokens each.
+    "rdt1b_generate": Workload("rdt1b_generate", RDTConfig(
+        vocab_size=201088, dim=2048, n_heads=16, n_kv_heads=4, max_seq_len=4096, max_loop_iters=16,
+        prelude_layers=1, coda_layers=1, n_experts=64, n_shared_experts=1, n_experts_per_tok=4,
+        expert_dim=2048, lora_rank=16, dtype="bf16"), batch=64, seq=128, n_loops=16, seed=8,
+        act_threshold=0.99, halt_b=-30.0, kind="generate", decode_steps=128, device_weights=True),
     # Profiling case for the latent attention: the attention of rdt3b_mla_decode (same
     # heads, latent widths, batch and cache length) with a small MoE and 2 loops, so that
     # well under 1 GB is held on the device.

@@ -41,11 +41,37 @@ def config_struct(cfg) -> N.rdt_config:
     return c
 
 
-def dense_config_struct(cfg) -> N.rdt_config:
-    """Config of a prelude/coda block: no routed experts, one dense SwiGLU of width 4*dim/3."""
+def dense_config_struct(cfg, hidden: Optional[int] = None) -> N.rdt_config:
+    """Config of a prelude/coda block: no routed experts, one dense SwiGLU of width 4*dim/3
+    (or `hidden`, the padded width the weights are laid out with)."""
     c = config_struct(cfg)
-    c.n_experts, c.top_k, c.n_shared_experts, c.expert_dim = 0, 0, 1, cfg.dim * 4 // 3
+    c.n_experts, c.top_k, c.n_shared_experts = 0, 0, 1
+    c.expert_dim = hidden if hidden is not None else cfg.dim * 4 // 3
     return c
+
+
+DENSE_ALIGN = 128
+
+
+def dense_padded(weights: dict) -> tuple:
+    """A prelude/coda block's dense FFN with its hidden width F rounded up to a multiple of
+    128: zero rows appended to the gate and the up half of w13 [1, 2F, D] and zero columns
+    to w2 [1, D, F].  A zero gate and up row gives silu(0) * 0 = 0 and a zero column of w2
+    adds nothing, so the block computes the same function; the padded width fits the
+    tensor-core GEMM's SwiGLU tile (128 gate + 128 up columns) and its rows are 16-byte
+    aligned for the TMA maps (4 dim / 3 seldom is either).  Done once
+    when a block is bound.  Returns (weights, padded width)."""
+    w13, w2 = weights["w13"], weights["w2"]
+    F = w2.shape[-1]
+    Fp = -(-F // DENSE_ALIGN) * DENSE_ALIGN
+    if Fp == F:
+        return weights, F
+    n13 = torch.zeros(w13.shape[0], 2 * Fp, w13.shape[2], dtype=w13.dtype, device=w13.device)
+    n13[:, :F] = w13[:, :F]
+    n13[:, Fp:Fp + F] = w13[:, F:]
+    n2 = torch.zeros(w2.shape[0], w2.shape[1], Fp, dtype=w2.dtype, device=w2.device)
+    n2[..., :F] = w2
+    return {**weights, "w13": n13, "w2": n2}, Fp
 
 
 class Weights:
@@ -228,7 +254,11 @@ class Block:
     def __init__(self, cfg, weights: dict, dense: bool = True):
         _require_cuda()
         self.cfg = cfg
-        self.cs = dense_config_struct(cfg) if dense else config_struct(cfg)
+        if dense:
+            weights, hidden = dense_padded(weights)
+            self.cs = dense_config_struct(cfg, hidden)
+        else:
+            self.cs = config_struct(cfg)
         self.w = Weights(weights, _DT[cfg.dtype][1])
 
     def workspace(self, batch: int, seq: int, max_keys: int) -> torch.Tensor:
@@ -260,7 +290,11 @@ def block_forward(cfg, weights: dict, x: torch.Tensor, batch: int, seq: int, sta
                   dense: bool = True) -> torch.Tensor:
     """rdt_block_forward: one pre-norm prelude/coda block (dense SwiGLU FFN) or a MoE block."""
     lib = _require_cuda()
-    cs = dense_config_struct(cfg) if dense else config_struct(cfg)
+    if dense:
+        weights, hidden = dense_padded(weights)
+        cs = dense_config_struct(cfg, hidden)
+    else:
+        cs = config_struct(cfg)
     w = Weights(weights, _DT[cfg.dtype][1])
     _check_act(x, "x", torch.float32, (batch * seq, cfg.dim))
     out = torch.empty_like(x)

@@ -404,6 +404,9 @@ namespace {
 int pick_bn(const GemmParams& p, int epi) {
   if (epi == EPI_SWIGLU_T) return (p.N % 128 == 0) ? 256 : 0;
   if (epi == EPI_ROUTER) return (p.N == 64 || p.N == 128) ? p.N : 0;
+  // rows that fit one 128-row tile (decode): the weights are the traffic, so the narrowest
+  // tile spreads them over the most CTAs
+  if (!p.tiles && p.M <= tc::BM && !p.vt && p.N % 64 == 0) return 64;
   if (p.N % 256 == 0) return 256;
   if (p.N % 128 == 0) return 128;
   if (p.N % 64 == 0) return 64;

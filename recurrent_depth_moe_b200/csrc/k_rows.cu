@@ -439,18 +439,35 @@ void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s)
 }
 // Greedy choice of the next token: CTA per row, argmax over the vocabulary with ties to
 // the lowest index; NaN compares below every number (a row of NaN gives 0).
-__global__ void __launch_bounds__(256) k_greedy(const float* __restrict__ logits, int vocab,
-                                               int* __restrict__ tokens, int out_ld) {
-  __shared__ float bv_s[8];
-  __shared__ int bi_s[8];
+constexpr int GREEDY_THREADS = 512;
+__global__ void __launch_bounds__(GREEDY_THREADS) k_greedy(const float* __restrict__ logits, int vocab,
+                                                          int* __restrict__ tokens, int out_ld) {
+  __shared__ float bv_s[GREEDY_THREADS / 32];
+  __shared__ int bi_s[GREEDY_THREADS / 32];
   const float* row = logits + (long long)blockIdx.x * vocab;
   float bv = -INFINITY;
   int bi = 0x7fffffff;
-  for (int v = threadIdx.x; v < vocab; v += 256) {
-    float x = row[v];
-    if (x != x) continue;
-    if (x > bv || (x == bv && v < bi)) { bv = x; bi = v; }
+  auto take = [&](float x, int v) {
+    if (x == x && (x > bv || (x == bv && v < bi))) { bv = x; bi = v; }
+  };
+  int v0 = 0;
+  if ((vocab & 3) == 0 && ((uintptr_t)row & 15) == 0) {   // 16-byte vectors, four in flight per thread
+    const float4* r4 = reinterpret_cast<const float4*>(row);
+    const int n4 = vocab >> 2;
+    for (int q = threadIdx.x; q < n4; q += 4 * GREEDY_THREADS) {
+      float4 f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) f[u] = q + u * GREEDY_THREADS < n4 ? __ldg(r4 + q + u * GREEDY_THREADS)
+                                                                   : make_float4(NAN, NAN, NAN, NAN);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = 4 * (q + u * GREEDY_THREADS);
+        take(f[u].x, v); take(f[u].y, v + 1); take(f[u].z, v + 2); take(f[u].w, v + 3);
+      }
+    }
+    v0 = vocab;
   }
+  for (int v = v0 + threadIdx.x; v < vocab; v += GREEDY_THREADS) take(row[v], v);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -461,7 +478,7 @@ __global__ void __launch_bounds__(256) k_greedy(const float* __restrict__ logits
   if (lane == 0) { bv_s[w] = bv; bi_s[w] = bi; }
   __syncthreads();
   if (threadIdx.x == 0) {
-    for (int k = 1; k < 8; ++k)
+    for (int k = 1; k < GREEDY_THREADS / 32; ++k)
       if (bv_s[k] > bv_s[0] || (bv_s[k] == bv_s[0] && bi_s[k] < bi_s[0])) { bv_s[0] = bv_s[k]; bi_s[0] = bi_s[k]; }
     tokens[(long long)blockIdx.x * out_ld] = bi_s[0] == 0x7fffffff ? 0 : bi_s[0];
   }
@@ -473,7 +490,7 @@ __global__ void k_to_model_dtype(const float* __restrict__ x, bf16* __restrict__
 }
 
 void launch_greedy(const float* logits, int n, int vocab, int* tokens, int out_ld, cudaStream_t s) {
-  k_greedy<<<n, 256, 0, s>>>(logits, vocab, tokens, out_ld);
+  k_greedy<<<n, GREEDY_THREADS, 0, s>>>(logits, vocab, tokens, out_ld);
   note_launch();
 }
 void launch_to_model_dtype(const float* x, void* out, long long n, cudaStream_t s) {

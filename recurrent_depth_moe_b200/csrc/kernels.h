@@ -11,7 +11,7 @@ struct DevStatus;
 // launches in its scope on the given stream when profiling is on).
 enum ProfClass {
   PC_PROLOGUE = 0, PC_QKV, PC_ATTN, PC_OPROJ, PC_FFN_NORM, PC_ROUTER_GEMM, PC_ROUTE, PC_EXPERT_UP,
-  PC_EXPERT_DOWN, PC_COMBINE, PC_OTHER, PC_COUNT
+  PC_EXPERT_DOWN, PC_COMBINE, PC_OTHER, PC_BLOCK, PC_HEAD, PC_TOKENS, PC_COUNT
 };
 struct ProfScope {
   ProfScope(int cls, cudaStream_t s);

@@ -16,7 +16,7 @@ void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 namespace {
 const char* kClassNames[PC_COUNT] = {"loop_prologue", "qkv_gemm_rope", "attention", "o_gemm_residual",
                                      "ffn_rmsnorm",   "router_gemm",   "route_topk_permute", "expert_up_swiglu",
-                                     "expert_down_gate", "combine_lora_inject_act", "other"};
+                                     "expert_down_gate", "combine_lora_inject_act", "other", "dense_block", "lm_head", "embed_cast_greedy"};
 struct Rec {
   int cls;
   cudaEvent_t a, b;
@@ -36,12 +36,17 @@ cudaEvent_t take_event() {
 }
 }  // namespace
 
+// Only the outermost scope of a host thread records: a whole-block scope then holds the
+// block's attention and GEMM launches once, not again under their own classes.
+static thread_local int t_scope_depth = 0;
+
 ProfScope::ProfScope(int cls, cudaStream_t s) : cls_(cls), s_(s), a_(nullptr) {
-  if (!g_prof.on) return;
+  if (t_scope_depth++ > 0 || !g_prof.on) return;
   a_ = take_event();
   if (a_) cudaEventRecord((cudaEvent_t)a_, s);
 }
 ProfScope::~ProfScope() {
+  --t_scope_depth;
   if (!g_prof.on || !a_) return;
   cudaEvent_t b = take_event();
   if (!b) {

@@ -577,6 +577,7 @@ rdt_status rdt_block_forward_cached(const rdt_config* cfg, const rdt_weights* w,
   }
   if (decode && (!cache || seq != 1)) return RDT_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
+  ProfScope ps_block(PC_BLOCK, s);
   Ctx x;
   x.c = cfg; x.w = w; x.ws = ws; x.s = s; x.dtype = cfg->dtype;
   make_layout(cfg, batch, seq, max_keys, &x.L);
@@ -620,6 +621,7 @@ rdt_status rdt_block_forward(const rdt_config* cfg, const rdt_weights* w, const 
 
 rdt_status rdt_greedy_tokens(const float* logits, int n, int vocab, int32_t* tokens, int out_ld, void* stream) {
   if (!logits || !tokens || n <= 0 || vocab <= 0 || out_ld < 1) return RDT_ERR_INVALID_ARG;
+  ProfScope ps(PC_TOKENS, (cudaStream_t)stream);
   launch_greedy(logits, n, vocab, tokens, out_ld, (cudaStream_t)stream);
   return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
 }
@@ -628,6 +630,7 @@ rdt_status rdt_to_model_dtype(const rdt_config* cfg, const float* x, void* out, 
   if (!cfg || (cfg->dtype != 0 && cfg->dtype != 1) || !x || !out || n < 0) return RDT_ERR_INVALID_ARG;
   if (n == 0) return RDT_OK;
   cudaStream_t s = (cudaStream_t)stream;
+  ProfScope ps(PC_TOKENS, s);
   if (cfg->dtype == 0) {
     if (x != out && cudaMemcpyAsync(out, x, (size_t)n * 4, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
       return RDT_ERR_CUDA;
@@ -641,6 +644,7 @@ rdt_status rdt_embed(const rdt_config* cfg, const void* table, int vocab, const 
                      void* stream) {
   if (!cfg || cfg->dim <= 0 || (cfg->dtype != 0 && cfg->dtype != 1) || !table || !ids || !out || vocab <= 0 || n <= 0)
     return RDT_ERR_INVALID_ARG;
+  ProfScope ps(PC_TOKENS, (cudaStream_t)stream);
   launch_embed(cfg->dtype, table, vocab, ids, n, cfg->dim, out, nullptr, (cudaStream_t)stream);
   return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
 }
@@ -651,6 +655,7 @@ rdt_status rdt_head_rows(const rdt_config* cfg, const float* xin, long long x_ld
   if (st != RDT_OK) return st;
   if (!xin || n <= 0 || x_ld < cfg->dim || !norm_w || !head || vocab <= 0 || !logits) return RDT_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
+  ProfScope ps(PC_HEAD, s);
   Layout L;
   make_layout(cfg, 1, n, n, &L);
   if ((st = check_ws(ws, ws_bytes, L)) != RDT_OK) return st;

@@ -46,3 +46,23 @@ def test_positions_after_a_halting_disagreement_are_left_out_of_their_sequence()
               {"cum": torch.tensor([1.1, 1.2, 1.0, 1.0, 1.0, 1.0])}]
     keep = same_halting_rows(_hw([2, 2, 2, 2, 2, 2]), _hw([2, 1, 2, 2, 2, 2]), record, thr, seq=3)
     assert keep.tolist() == [True, False, False, True, True, True]
+
+
+def test_dense_padding_keeps_the_block_function():
+    """The binding pads a dense FFN's hidden width to a multiple of 128 (SwiGLU tile, TMA rows)
+    with zero rows and columns; the SwiGLU FFN computes the same function (fp64, 4 dim / 3
+    widths of the 1B and tiny configs)."""
+    import torch.nn.functional as Fn
+    from recurrent_depth_moe_b200.api import dense_padded
+    g = torch.Generator().manual_seed(9)
+    for D in (256, 2048):
+        F = D * 4 // 3
+        w = {"w13": torch.randn(1, 2 * F, D, generator=g, dtype=torch.float64),
+             "w2": torch.randn(1, D, F, generator=g, dtype=torch.float64)}
+        p, Fp = dense_padded(w)
+        assert Fp % 128 == 0 and Fp >= F and Fp - F < 128
+        x = torch.randn(5, D, generator=g, dtype=torch.float64)
+
+        def ffn(w13, w2, h):
+            return (Fn.silu(x @ w13[0, :h].T) * (x @ w13[0, h:].T)) @ w2[0].T
+        assert torch.allclose(ffn(w["w13"], w["w2"], F), ffn(p["w13"], p["w2"], Fp), rtol=1e-12, atol=1e-12)
