@@ -45,6 +45,9 @@ struct TcArgs {
   int m_tiles;         // dense: m tiles; grouped: read from *p.n_tiles
   int b_rows_group;    // rows of B per group (grouped)
   int n_out_tile;      // output columns per tile
+  int k_splits;        // > 1: split-K, tile t covers k-blocks of split t / (m_tiles n_n)
+  int kb_split;        // k-blocks per split
+  long long split_stride;   // elements between the fp32 partials of two splits
 };
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z)); }
@@ -77,10 +80,16 @@ __device__ __forceinline__ int rope_chunk(const GemmParams& p, int c) {
   return -1;
 }
 
-struct TileInfo { int group, row0, rows, n0; };
+struct TileInfo { int group, row0, rows, n0, split; };
 
 __device__ __forceinline__ TileInfo decode_tile(const TcArgs& a, int t) {
   TileInfo ti;
+  ti.split = 0;
+  if (a.k_splits > 1) {
+    const int per = a.m_tiles * a.n_n;
+    ti.split = t / per;
+    t %= per;
+  }
   const int m_i = t / a.n_n, n_i = t % a.n_n;
   if (a.p.tiles) {
     ti.group = a.p.tiles[4 * m_i];
@@ -189,8 +198,18 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int m_tiles = p.tiles ? min(*p.n_tiles, p.max_tiles) : args.m_tiles;
-  const int total = m_tiles * args.n_n;
+  const int total = m_tiles * args.n_n * max(args.k_splits, 1);
   const int nk = p.K / BK;
+  // k-block range of a tile (all of K unless split)
+  auto k_range = [&](const TileInfo& ti, int& k0, int& k1) {
+    if (args.k_splits > 1) {
+      k0 = ti.split * args.kb_split;
+      k1 = min(nk, k0 + args.kb_split);
+    } else {
+      k0 = 0;
+      k1 = nk;
+    }
+  };
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
@@ -207,7 +226,9 @@ __global__ void __launch_bounds__(192, 1)
         b0 = gb + ti.n0;
         b1 = b0 + S::B_BOX;
       }
-      for (int ks = 0; ks < nk; ++ks) {
+      int k0, k1;
+      k_range(ti, k0, k1);
+      for (int ks = k0; ks < k1; ++ks) {
         if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
         uint8_t* sa = smem + stage * S::STAGE_BYTES;
         mbar_expect_tx(&full[stage], S::STAGE_BYTES);
@@ -229,14 +250,16 @@ __global__ void __launch_bounds__(192, 1)
       if (!(ok = mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag))) break;
       tc_fence_after();
       const uint32_t d = tmem + acc * BN;
-      for (int ks = 0; ks < nk; ++ks) {
+      int k0, k1;
+      k_range(decode_tile(args, t), k0, k1);
+      for (int ks = k0; ks < k1; ++ks) {
         if (!(ok = mbar_wait(&full[stage], phase, abort_flag))) break;
         tc_fence_after();
         uint8_t* sa = smem + stage * S::STAGE_BYTES;
         const uint64_t ad = smem_desc(sa), bd = smem_desc(sa + A_BYTES);
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)
-          umma_bf16(d, ad + 2 * k, bd + 2 * k, IDESC, (ks | k) != 0);
+          umma_bf16(d, ad + 2 * k, bd + 2 * k, IDESC, (ks != k0 || k != 0) ? 1u : 0u);
         umma_commit(&empty[stage]);
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
@@ -255,12 +278,39 @@ __global__ void __launch_bounds__(192, 1)
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const TileInfo ti = decode_tile(args, t);
+      const bool valid = rl < ti.rows;
+      const long long r = (long long)ti.row0 + rl;
+      // the residual does not depend on the accumulator: its first chunk is in flight
+      // while this tile's MMAs finish, and chunk c + 1 while chunk c is stored
+      float4 rcur[EPI == EPI_RESID_F32 ? 8 : 1], rnxt[EPI == EPI_RESID_F32 ? 8 : 1];
+      const float* rrow = (EPI == EPI_RESID_F32 && valid) ? p.resid + r * p.ld_resid + ti.n0 : nullptr;
+      if (EPI == EPI_RESID_F32 && valid && args.k_splits <= 1) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) rcur[q] = __ldg(reinterpret_cast<const float4*>(rrow) + q);
+      }
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-      const bool valid = rl < ti.rows;
-      const long long r = (long long)ti.row0 + rl;
-      if (EPI == EPI_ROUTER) {
+      if (EPI == EPI_RESID_F32 && args.k_splits <= 1) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          if (valid && c + 32 < BN) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q) rnxt[q] = __ldg(reinterpret_cast<const float4*>(rrow + c + 32) + q);
+          }
+          float v[32];
+          tmem_ld32(tbase + c, v);
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>((float*)p.C + r * p.ldc + ti.n0 + c);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[q] = make_float4(rcur[q].x + v[4 * q], rcur[q].y + v[4 * q + 1], rcur[q].z + v[4 * q + 2],
+                                   rcur[q].w + v[4 * q + 3]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) rcur[q] = rnxt[q];
+          }
+        }
+      } else if (EPI == EPI_ROUTER) {
         if (BN == 64 || BN == 128) route_row<(BN == 128 ? 128 : 64)>(p, tbase, valid, r);
       } else if (EPI == EPI_SWIGLU_T) {
 #pragma unroll 1
@@ -312,7 +362,7 @@ __global__ void __launch_bounds__(192, 1)
               for (int j = 0; j < 32; ++j) vt[(long long)j * p.vt_ld] = __float2bfloat16_rn(v[j]);
             }
           } else {
-            float* dst = (float*)p.C + r * p.ldc + col;
+            float* dst = (float*)p.C + ti.split * args.split_stride + r * p.ldc + col;
             if (EPI == EPI_RESID_F32) {
               const float4* rs4 = (const float4*)(p.resid + r * p.ld_resid + col);
 #pragma unroll
@@ -461,11 +511,72 @@ bool gemm_tc_supports(const GemmParams& p, int epi) {
   return encode_fn() != nullptr;
 }
 
+// Split-K epilogue: the sum of the fp32 partials in split order (deterministic), then the
+// GEMM's own epilogue; two columns per thread (a RoPE pair is two adjacent columns).
+__device__ __forceinline__ int rope_pair_col(const GemmParams& p, int c) {
+  for (int q = 0; q < p.n_rope; ++q) {
+    const RopeDesc& r = p.rope[q];
+    const int rel = c - r.col0;
+    if (rel < 0 || rel >= r.n_heads * r.head_stride) continue;
+    const int o = rel % r.head_stride - r.off;
+    if (o >= 0 && o < r.dim) return o >> 1;
+  }
+  return -1;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(256) k_splitk_epilogue(GemmParams p, const float* __restrict__ part, int splits,
+                                                        long long stride) {
+  const long long r = blockIdx.y;
+  const int c = 2 * (blockIdx.x * 256 + threadIdx.x);
+  if (c >= p.N) return;
+  const float* src = part + r * p.N + c;
+  float v0 = 0.f, v1 = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float2 a = *reinterpret_cast<const float2*>(src + (long long)s * stride);
+    v0 += a.x;
+    v1 += a.y;
+  }
+  if (EPI == EPI_STORE_F32) {
+    *reinterpret_cast<float2*>((float*)p.C + r * p.ldc + c) = make_float2(v0, v1);
+  } else if (EPI == EPI_RESID_F32) {
+    const float2 a = *reinterpret_cast<const float2*>(p.resid + r * p.ld_resid + c);
+    *reinterpret_cast<float2*>((float*)p.C + r * p.ldc + c) = make_float2(a.x + v0, a.y + v1);
+  } else {
+    if (EPI == EPI_ROPE_T) {
+      const int m = rope_pair_col(p, c);
+      if (m >= 0) {
+        const float2 cs = p.rope_tab[(long long)p.pos[r] * p.rope_half + m];
+        const float a0 = v0 * cs.x - v1 * cs.y, a1 = v0 * cs.y + v1 * cs.x;
+        v0 = a0;
+        v1 = a1;
+      }
+    }
+    *reinterpret_cast<__nv_bfloat162*>((bf16*)p.C + r * p.ldc + c) = __floats2bfloat162_rn(v0, v1);
+  }
+}
+
+// Splits for rows that fit one tile: enough to give every SM a tile, at least 3 k-blocks
+// each, within the caller's scratch.  1 = no split.
+static int splitk_count(const GemmParams& p, int epi, int n_tiles) {
+  if (!p.split_ws || p.tiles || p.M > tc::BM || p.vt || p.N % 2 || p.ldc % 2) return 1;
+  if (epi != EPI_STORE_F32 && epi != EPI_STORE_T && epi != EPI_RESID_F32 && epi != EPI_ROPE_T) return 1;
+  if (epi == EPI_RESID_F32 && p.ld_resid % 2) return 1;
+  const int nk = p.K / tc::BK;
+  int splits = std::min(sm_count() / std::max(n_tiles, 1), nk / 3);
+  splits = std::max(1, std::min(splits, 16));
+  while (splits > 1 && (long long)splits * p.M * p.N > p.split_ws_elems) --splits;
+  return splits;
+}
+
 int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
   const int bn = pick_bn(p, epi);
   if (!bn) return -1;
   tc::TcArgs a;
   a.p = p;
+  a.k_splits = 1;
+  a.kb_split = 0;
+  a.split_stride = 0;
   a.n_out_tile = (epi == EPI_SWIGLU_T) ? bn / 2 : bn;
   a.n_n = p.N / a.n_out_tile;
   a.m_tiles = p.tiles ? 0 : (p.M + tc::BM - 1) / tc::BM;
@@ -484,6 +595,28 @@ int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
     grid = (int)std::min<long long>(tiles, sm_count());
   }
   if (grid <= 0) return 0;
+  const int splits = splitk_count(p, epi, a.m_tiles * a.n_n);
+  if (splits > 1) {
+    // partial sums of K ranges into the scratch with the fp32 epilogue, then the real one
+    const int nk = p.K / tc::BK;
+    a.kb_split = (nk + splits - 1) / splits;
+    a.k_splits = (nk + a.kb_split - 1) / a.kb_split;
+    a.split_stride = (long long)p.M * p.N;
+    a.p.C = p.split_ws;
+    a.p.ldc = p.N;
+    grid = (int)std::min<long long>((long long)a.m_tiles * a.n_n * a.k_splits, sm_count());
+    int rc = launch_tc_bn<EPI_STORE_F32>(bn, mA, mB, a, grid, s);
+    if (rc) return rc;
+    dim3 eg((unsigned)((p.N / 2 + 255) / 256), (unsigned)p.M);
+    switch (epi) {
+      case EPI_STORE_F32: k_splitk_epilogue<EPI_STORE_F32><<<eg, 256, 0, s>>>(p, p.split_ws, a.k_splits, a.split_stride); break;
+      case EPI_STORE_T: k_splitk_epilogue<EPI_STORE_T><<<eg, 256, 0, s>>>(p, p.split_ws, a.k_splits, a.split_stride); break;
+      case EPI_RESID_F32: k_splitk_epilogue<EPI_RESID_F32><<<eg, 256, 0, s>>>(p, p.split_ws, a.k_splits, a.split_stride); break;
+      default: k_splitk_epilogue<EPI_ROPE_T><<<eg, 256, 0, s>>>(p, p.split_ws, a.k_splits, a.split_stride); break;
+    }
+    note_launch();
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  }
   int rc;
   switch (epi) {
     case EPI_STORE_F32: rc = launch_tc_bn<EPI_STORE_F32>(bn, mA, mB, a, grid, s); break;

@@ -177,6 +177,52 @@ __global__ void __launch_bounds__(128) k_route_scatter(RouteParams p) {
   }
 }
 
+// Router logits for few rows (decode), logits[m, e] = f[m, :] . Wr[e, :]: CTA per expert,
+// so the weights stream through E CTAs at once (the fused tcgen05 router would be one
+// CTA).  Warp w takes the 8 rows 8 w .. 8 w + 7 together: each 16-byte weight load
+// serves 8 rows, and the 9 loads of a step are in flight at once.
+__global__ void __launch_bounds__(256) k_router_small(const bf16* __restrict__ f, const bf16* __restrict__ wr, int M,
+                                                     int K, int E, float* __restrict__ logits) {
+  constexpr int RW = 8;
+  const int e = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bf16* w = wr + (long long)e * K;
+  for (int m0 = warp * RW; m0 < M; m0 += 8 * RW) {
+    float acc[RW];
+#pragma unroll
+    for (int i = 0; i < RW; ++i) acc[i] = 0.f;
+    for (int k = lane * 8; k < K; k += 256) {
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(w + k));
+      uint4 a[RW];
+#pragma unroll
+      for (int i = 0; i < RW; ++i)
+        a[i] = m0 + i < M ? __ldg(reinterpret_cast<const uint4*>(f + (long long)(m0 + i) * K + k)) : make_uint4(0, 0, 0, 0);
+      const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 fb = __bfloat1622float2(b2[q]);
+#pragma unroll
+        for (int i = 0; i < RW; ++i) {
+          const float2 fa = __bfloat1622float2(reinterpret_cast<const __nv_bfloat162*>(&a[i])[q]);
+          acc[i] = fmaf(fa.x, fb.x, acc[i]);
+          acc[i] = fmaf(fa.y, fb.y, acc[i]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < RW; ++i) {
+      const float t = warp_sum(acc[i]);
+      if (lane == 0 && m0 + i < M) logits[(long long)(m0 + i) * E + e] = t;
+    }
+  }
+}
+
+bool launch_router_small(const void* f, const void* wr, int M, int K, int E, float* logits, cudaStream_t s) {
+  if (K % 8 || ((uintptr_t)f & 15) || ((uintptr_t)wr & 15) || M <= 0 || E <= 0) return false;
+  k_router_small<<<E, 256, 0, s>>>((const bf16*)f, (const bf16*)wr, M, K, E, logits);
+  note_launch();
+  return true;
+}
+
 void launch_router_topk(const RouteParams& p, cudaStream_t s) {
   { k_router_topk<<<(p.N + 7) / 8, 256, 0, s>>>(p); note_launch(); }
 }

@@ -57,6 +57,9 @@ struct GemmParams {
   // EPI_ROPE_T (optional): also store the value columns [vt_col0, vt_col0 + vt_heads * vt_hd)
   // transposed: vt[((b * vt_heads + g) * vt_hd + d) * vt_ld + t] for row = b * vt_T + t
   void* vt; int vt_col0, vt_heads, vt_hd, vt_T; long long vt_ld;
+  // split-K scratch for rows that fit one tile (decode): fp32 partials [splits][M][N];
+  // nullptr = no split
+  float* split_ws; long long split_ws_elems;
   DevStatus* st;
 };
 
@@ -124,6 +127,7 @@ struct RouteParams {
   DevStatus* st;
 };
 void launch_router_topk(const RouteParams& p, cudaStream_t s);
+bool launch_router_small(const void* f, const void* wr, int M, int K, int E, float* logits, cudaStream_t s);
 void launch_route_scan(const RouteParams& p, cudaStream_t s);
 void launch_route_scatter(int dtype, const RouteParams& p, cudaStream_t s);
 

@@ -26,6 +26,7 @@ struct Layout {
   size_t run_list, run_idx, nrun, cum, halted, Avec, emb, rope, pos, p_buf, part_o, part_ml, xn, vt;
   size_t mla_ckv_all, mla_kvu_all;   // MLA with earlier cached keys: rebuilt per-head keys / values
   size_t mla_qa;                     // MLA absorbed decode: absorbed queries (0 = path not used)
+  size_t splitk; long long splitk_elems;   // split-K partials of single-tile GEMMs (decode)
   int part_dim;                      // split-KV partial width (head dim, or kv_lora_rank)
   size_t total;
   int max_tiles, max_slots, rope_dim, rope_pos, n_split;
@@ -135,6 +136,10 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
     L->part_dim = c->kv_lora_rank;
   }
   L->part_o = take(L->n_split ? (size_t)B * H * L->n_split * L->part_dim * 4 : 16);
+  if (N <= 128) {   // rows that fit one GEMM tile: the weights stream through split-K CTAs
+    L->splitk_elems = (long long)N * 16384;
+    L->splitk = take((size_t)L->splitk_elems * 4);
+  }
   L->part_ml = take(L->n_split ? (size_t)B * H * L->n_split * 2 * 4 : 16);
   L->total = off;
 }
@@ -161,6 +166,10 @@ GemmParams gemm_base(const Ctx& x) {
   memset(&g, 0, sizeof(g));
   g.st = x.st;
   g.impl = -1;
+  if (x.L.splitk) {
+    g.split_ws = at<float*>(x.ws, x.L.splitk);
+    g.split_ws_elems = x.L.splitk_elems;
+  }
   return g;
 }
 
@@ -348,8 +357,15 @@ rdt_status moe_block(Ctx& x, int N, const float* x1) {
   g.A = f; g.lda = D; g.B = w->w_router; g.ldb = D; g.M = N; g.N = E; g.K = D; g.C = logits; g.ldc = E;
   g.bias = w->router_bias; g.run_idx = at<int*>(x.ws, x.L.run_idx); g.topk = k;
   g.ids = rp.ids; g.gates = rp.gates; g.rank = rp.rank; g.counts = rp.counts;
-  const bool fused_route = gemm_pick(x.dtype, g, EPI_ROUTER) == GEMM_TC;
-  { ProfScope ps(PC_ROUTER_GEMM, x.s); RDT_TRY(launch_gemm(x.dtype, fused_route ? EPI_ROUTER : EPI_STORE_F32, g, x.s)); }
+  // few rows (decode): the logits come from a CTA per expert and top-k runs on its own
+  // kernel; otherwise the tcgen05 router GEMM routes in its epilogue
+  const bool small_router = x.dtype == 1 && N <= 128;
+  const bool fused_route = !small_router && gemm_pick(x.dtype, g, EPI_ROUTER) == GEMM_TC;
+  {
+    ProfScope ps(PC_ROUTER_GEMM, x.s);
+    if (!(small_router && launch_router_small(f, w->w_router, N, D, E, logits, x.s)))
+      RDT_TRY(launch_gemm(x.dtype, fused_route ? EPI_ROUTER : EPI_STORE_F32, g, x.s));
+  }
   {
     ProfScope ps(PC_ROUTE, x.s);
     if (!fused_route) launch_router_topk(rp, x.s);
