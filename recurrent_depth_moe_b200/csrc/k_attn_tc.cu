@@ -9,10 +9,11 @@
 //   warps 2..5  softmax of query tile 0; warps 6..9 softmax of query tile 1.
 //               Thread = query row = TMEM lane: reads its S row, masks (key j visible
 //               iff key_pos0 + j <= q_pos, "OpenMythos 분석", Core Structure causal
-//               mask), keeps a running max m and sum l in the log2 domain, writes
-//               P = exp2(s - m) as bf16 into 128B-swizzled shared memory (the A operand
-//               of the PV MMA).  The running max is raised only when it grows by more
-//               than 2^8, and only then is the O row rescaled in TMEM.
+//               mask), keeps a running max m and sum l in the log2 domain, and writes
+//               P = exp2(s - m) as bf16 back into the first 32 columns of the tile's own
+//               S buffer: the PV MMA reads its A operand from TMEM.  The running max is
+//               raised only when it grows by more than 2^8, and only then does the
+//               softmax wait for the previous PV and rescale the O row in TMEM.
 // The two query tiles share every K / V tile and their softmax groups overlap each
 // other and the tensor core.  V is consumed transposed (V^T[b][g][dim][t], written by
 // the QKV GEMM epilogue) so both MMAs read K-major operands.  Every wait is bounded.
@@ -27,15 +28,14 @@ bool tc_make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsi
 
 namespace fat {
 
-constexpr int BQ = 128, BKV = 64, HD = 128, NQ = 2, STAGES = 3;
+constexpr int BQ = 128, BKV = 64, HD = 128, NQ = 2, STAGES = 4;
 constexpr int QTILE = BQ * HD * 2;      // 32 KB: two 64-dim swizzle atoms of 16 KB
 constexpr int QHALF = QTILE / 2;
 constexpr int KTILE = BKV * HD * 2;     // 16 KB: two atoms [64 keys][64 dims] of 8 KB
 constexpr int KHALF = KTILE / 2;
 constexpr int VTILE = HD * BKV * 2;     // 16 KB: one atom [128 dims][64 keys]
-constexpr int PTILE = BQ * BKV * 2;     // 16 KB: one atom [128 queries][64 keys]
-constexpr int SMEM = NQ * QTILE + STAGES * (KTILE + VTILE) + NQ * PTILE + 1024 + 512;
-constexpr int TMEM_COLS = 512;          // S[q][buf] at (2q + buf) * 64; O[q] at 256 + 128 q
+constexpr int SMEM = NQ * QTILE + STAGES * (KTILE + VTILE) + 1024 + 512;
+constexpr int TMEM_COLS = 512;          // S[q][buf] at (2q + buf) * 64 (P in its first 32); O[q] at 256 + 128 q
 constexpr float RESCALE_LOG2 = 8.f;     // lazy rescale threshold (factor 256)
 constexpr int THREADS = 64 + NQ * 128;
 
@@ -65,8 +65,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sQ = smem;                          // [NQ] query tiles
   uint8_t* sK = sQ + NQ * QTILE;               // [STAGES]
   uint8_t* sV = sK + STAGES * KTILE;           // [STAGES]
-  uint8_t* sP = sV + STAGES * VTILE;           // [NQ]
-  uint64_t* bars = (uint64_t*)(sP + NQ * PTILE);
+  uint64_t* bars = (uint64_t*)(sV + STAGES * VTILE);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;                // [STAGES]
   uint64_t* kv_empty = kv_full + STAGES;       // [STAGES]
@@ -159,11 +158,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait(&p_full[q], jj & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t tO = tmem + 256 + q * 128;
+        const uint32_t tP = tmem + (2 * q + (jj & 1)) * BKV;   // P of tile jj, 2 bf16 per column
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t ad = smem_desc(sP + q * PTILE) + 2 * kk;
           const uint64_t bd = smem_desc(sV + st * VTILE) + 2 * kk;
-          umma_bf16(tO, ad, bd, IDESC_O, (jj > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tO, tP + 8 * kk, bd, IDESC_O, (jj > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[q]);
       }
@@ -205,7 +204,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tO = tmem + lane_base + 256 + q * 128;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint8_t* prow = sP + q * PTILE + rl * 128;
     for (int j = 0; j < ntq; ++j) {
       if (!(ok = mbar_wait(&s_full[2 * q + (j & 1)], (j >> 1) & 1, abort_flag))) break;
       tc_fence_after();
@@ -259,29 +257,30 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int k = 0; k < w; ++k) sp[k] += sp[k + w];
       l += sp[0];
-      if (j >= 1) {
-        // PV of tile j-1 done: O is stable and the P buffer is free
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // the max moved: O must hold PV of tile j-1 before it is rescaled.  pv_done can be
+        // at most one phase ahead of this wait (PV j needs this warp's arrival below)
         if (!(ok = mbar_wait(&pv_done[q], (j - 1) & 1, abort_flag))) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < HD; c += 32) {
-            float v[32];
-            tmem_ld32(tO + c, v);
+        for (int c = 0; c < HD; c += 32) {
+          float v[32];
+          tmem_ld32(tO + c, v);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] *= alpha;
-            tmem_st32(tO + c, v);
-          }
-          tmem_st_wait();
+          for (int e = 0; e < 32; ++e) v[e] *= alpha;
+          tmem_st32(tO + c, v);
         }
       }
-      // 16-byte chunk c (8 keys) of the 128-byte row goes to chunk c ^ (row & 7)
+      // P over the first 32 columns of this tile's S buffer (S is in registers already;
+      // every MMA before S of tile j, the PV that read this buffer's last P included, is
+      // complete once s_full fired)
+      {
+        float pf[32];
 #pragma unroll
-      for (int c = 0; c < BKV / 8; ++c) {
-        const int ch = c ^ (rl & 7);
-        *reinterpret_cast<uint4*>(prow + ch * 16) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        for (int c = 0; c < BKV / 2; ++c) pf[c] = __uint_as_float(pk[c]);
+        tmem_st32(tmem + lane_base + (2 * q + (j & 1)) * BKV, pf);
       }
-      fence_async_smem();
+      tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_full[q]);
     }
