@@ -116,6 +116,25 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm), "power_w_max": max(power) if power else None}
 
 
+# DRAM traffic of one full-size expert-up launch (1B shape, 16384 tokens x 5 slots), from ncu
+# dram__bytes_read.sum + dram__bytes_write.sum (1 pass; profiles/expert_up_gemm_rdt1b_small_case.md).
+# Reported only while the GEMM's sources are the ones it was captured from.
+EXPERT_UP_TRAFFIC = {"bytes": 1.43e9 + 303.23e6, "workload": "rdt1b_prefill", "n_loops": 16,
+                     "sha256": "23998a96b0d9c533a91ed917bd60185d2621b939bf0f519acb37707aad37e0b3"}
+
+
+def expert_up_traffic(wl):
+    import hashlib
+    if wl.name != EXPERT_UP_TRAFFIC["workload"] or wl.batch != 4 or wl.n_loops != EXPERT_UP_TRAFFIC["n_loops"]:
+        return None
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "recurrent_depth_moe_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("k_gemm_tc.cu", "tc_common.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return EXPERT_UP_TRAFFIC["bytes"] if h.hexdigest() == EXPERT_UP_TRAFFIC["sha256"] else None
+
+
 def expert_up_flops(wl, n_running: int) -> float:
     c = wl.cfg
     rows = n_running * (c.n_experts_per_tok + c.n_shared_experts)
@@ -300,7 +319,7 @@ def run_ours(args, wl, rank, world, local_rank):
                 "achieved": achieved_tflops, "peak": peak_t, "unit": "TFLOP/s",
                 "frac": (achieved_tflops / peak_t) if achieved_tflops else None,
                 "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)",
-                "traffic": None,
+                "traffic": expert_up_traffic(wl),
                 "flops_per_launch": expert_up_flops(wl, executed / L)}
     breakdown = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps} for k, v in sorted(prof.items())}
     res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
