@@ -142,3 +142,35 @@ def test_rdt3b_mla_decode_sequence_matches_oracle():
     assert rel_l2(d_h[b:b + 1], o_h) <= BF16_TOL
     for t in range(L):
         assert rel_l2(ckv[t, b, wl.cache_len], new_kv[t][0][0][0]) <= BF16_TOL
+
+
+def test_rdt1b_generation_teacher_forced():
+    """Generation with the 1B-shaped model (16 loops, 64 experts, 1 prelude + 1 coda layer;
+    vocabulary reduced to 4096 here, since it only sizes the embedding and the head): the
+    oracle's forward pass over the GPU's own sequence gives, at every generated step,
+    logits within the bf16 tolerance and the GPU's token as its argmax up to near-ties."""
+    wl = RI.get_workload("rdt1b_generate")
+    cfg = wl.cfg.replace(vocab_size=4096)
+    dev = torch.device("cuda")
+    MW = RI.model_weights(cfg, wl.seed, device=dev, halt_b=wl.halt_b)
+    B, T0, new, L = 2, 24, 3, wl.n_loops
+    prompt = torch.randint(0, cfg.vocab_size, (B, T0), generator=torch.Generator().manual_seed(11))
+    gen = R.Generator(cfg, MW, B, T0, new, L, wl.act_threshold)
+    gen.prefill(prompt.to(device=dev, dtype=torch.int32).contiguous())
+    logits = [gen.logits.clone()]
+    for s in range(1, new):
+        gen.decode(s)
+        logits.append(gen.logits.clone())
+    torch.cuda.synchronize()
+    toks = gen.tokens.t().cpu().long()
+    seq = torch.cat([prompt, toks], dim=1)
+    MWc = {k: ([{kk: vv.cpu() for kk, vv in blk.items()} for blk in v] if isinstance(v, list) else
+               ({kk: vv.cpu() for kk, vv in v.items()} if isinstance(v, dict) else v.cpu())) for k, v in MW.items()}
+    b = 0
+    full, _, _ = O.model_forward(cfg, MWc, seq[b:b + 1, :-1], L, wl.act_threshold)
+    for s in range(new):
+        ol = full[0, T0 - 1 + s]
+        gl = logits[s][b].cpu()
+        assert rel_l2(gl, ol) <= BF16_TOL, s
+        gap = float(ol.max() - ol[toks[b, s]])
+        assert gap <= 2e-2 * float(ol.max() - ol.min()), s
