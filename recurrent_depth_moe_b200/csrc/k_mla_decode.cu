@@ -503,11 +503,11 @@ bool mla_decode_supports(int attn_type, int dtype, int H, int kvr, int dr, int d
   return shape && dn % 8 == 0 && dn >= 8 && dn <= 256 && dv >= 1;
 }
 
-int mla_decode_splits(int B, int t_max) {
+int mla_decode_splits(int B, int t_max, int tile_keys) {
   // key ranges per sequence: fewest waves x (tiles per range + the fixed cost of a CTA:
   // its query load and partial write, about 1.5 tiles) over the SMs, one CTA each
   const int sms = tc_sm_count() > 0 ? tc_sm_count() : 148;
-  const int tiles = std::max(1, (t_max + mla::BKV - 1) / mla::BKV);
+  const int tiles = std::max(1, (t_max + tile_keys - 1) / tile_keys);
   int best = 1;
   long long best_cost = -1;
   for (int ns = 1; ns <= std::min(32, tiles); ++ns) {

@@ -105,9 +105,10 @@ struct MlaDecodeParams {
   void* qa;                                     // scratch [B][H][kvr]
   float* part_o; float* part_ml; int n_split;   // [B][H][n_split][kvr], [B][H][n_split][2]
   void* o; long long o_row;                     // attention output [B][H dv]
+  DevStatus* st;
 };
 bool mla_decode_supports(int attn_type, int dtype, int H, int kvr, int dr, int dn, int dv);
-int mla_decode_splits(int B, int t_max);
+int mla_decode_splits(int B, int t_max, int tile_keys);
 int launch_mla_decode(const MlaDecodeParams& p, cudaStream_t s);
 int tc_sm_count();
 

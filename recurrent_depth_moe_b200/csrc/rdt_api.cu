@@ -132,7 +132,7 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
   L->n_split = (T == 1) ? decode_split_count(std::max(max_keys, 1)) : 0;
   L->part_dim = 128;
   if (L->mla_qa) {
-    L->n_split = mla_decode_splits(B, std::max(max_keys, 1));
+    L->n_split = mla_decode_splits(B, std::max(max_keys, 1), 64);   // 64-key tiles
     L->part_dim = c->kv_lora_rank;
   }
   L->part_o = take(L->n_split ? (size_t)B * H * L->n_split * L->part_dim * 4 : 16);
@@ -285,7 +285,7 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
         mp.ckv = ckv_c; mp.krope = kr_c; mp.t_max = tm; mp.q_pos = pos;
         mp.qa = at<void*>(x.ws, x.L.mla_qa);
         mp.part_o = at<float*>(x.ws, x.L.part_o); mp.part_ml = at<float*>(x.ws, x.L.part_ml); mp.n_split = x.L.n_split;
-        mp.o = attn; mp.o_row = (long long)H * dv;
+        mp.o = attn; mp.o_row = (long long)H * dv; mp.st = x.st;
         ProfScope ps(PC_ATTN, x.s);
         if (launch_mla_decode(mp, x.s) != 0) return RDT_ERR_CUDA;
       } else if (decode || start_pos > 0) {
