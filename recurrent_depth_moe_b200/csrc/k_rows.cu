@@ -431,8 +431,60 @@ bool launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t 
   else { k_combine_inject_act<bf16><<<n_rows, nt, smem, s>>>(p); note_launch(); }
   return false;
 }
-void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* n_run, cudaStream_t s) {
-  { k_compact<<<1, 1024, 0, s>>>(halted, N, run_list, run_idx, n_run); note_launch(); }
+// Running-row list in two passes over CTAs of 1024 rows: each CTA counts its running rows,
+// then each CTA adds the counts of the CTAs before it (in order: the list is the same as a
+// sequential scan) and scatters its rows.  No CTA waits for another.
+__global__ void __launch_bounds__(1024) k_compact_count(const int* __restrict__ halted, int N, int* __restrict__ cta_count) {
+  __shared__ int warp_tot[32];
+  const int i = blockIdx.x * 1024 + threadIdx.x, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const unsigned m = __ballot_sync(0xffffffffu, i < N && !halted[i]);
+  if (lane == 0) warp_tot[wid] = __popc(m);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int w = 0; w < 32; ++w) tot += warp_tot[w];
+    cta_count[blockIdx.x] = tot;
+  }
+}
+__global__ void __launch_bounds__(1024) k_compact_scatter(const int* __restrict__ halted, int N,
+                                                          const int* __restrict__ cta_count, int* __restrict__ run_list,
+                                                          int* __restrict__ run_idx, int* __restrict__ n_run) {
+  __shared__ int warp_tot[32];
+  __shared__ int base;
+  const int i = blockIdx.x * 1024 + threadIdx.x, lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (threadIdx.x < 32) {
+    int b = 0;
+    for (int c = threadIdx.x; c < (int)blockIdx.x; c += 32) b += cta_count[c];
+    b = warp_sum_int(b);
+    if (threadIdx.x == 0) base = b;
+  }
+  const bool run = i < N && !halted[i];
+  const unsigned m = __ballot_sync(0xffffffffu, run);
+  if (lane == 0) warp_tot[wid] = __popc(m);
+  __syncthreads();
+  int off = base;
+  for (int w = 0; w < wid; ++w) off += warp_tot[w];
+  if (i < N) {
+    const int idx = off + __popc(m & ((1u << lane) - 1u));
+    run_idx[i] = run ? idx : -1;
+    if (run) run_list[idx] = i;
+  }
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 1023) {
+    int tot = off;
+    for (int w = wid; w < 32; ++w) tot += warp_tot[w];
+    *n_run = tot;
+  }
+}
+
+void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* n_run, int* cta_count,
+                    cudaStream_t s) {
+  const int ctas = (N + 1023) / 1024;
+  if (ctas <= 0) return;
+  if (!cta_count || ctas > 4096) { k_compact<<<1, 1024, 0, s>>>(halted, N, run_list, run_idx, n_run); note_launch(); return; }
+  k_compact_count<<<ctas, 1024, 0, s>>>(halted, N, cta_count);
+  note_launch();
+  k_compact_scatter<<<ctas, 1024, 0, s>>>(halted, N, cta_count, run_list, run_idx, n_run);
+  note_launch();
 }
 void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s) {
   { k_iota<<<(N + 255) / 256, 256, 0, s>>>(run_list, run_idx, n_run, N); note_launch(); }

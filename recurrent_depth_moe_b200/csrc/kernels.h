@@ -171,7 +171,8 @@ void launch_kv_to_cache(int dtype, const void* qkv, long long ld, int k_col, int
                         cudaStream_t s);
 // returns true when the fused next-loop prologue ran (p.next_emb set and supported)
 bool launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s);
-void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* n_run, cudaStream_t s);
+void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* n_run, int* cta_count,
+                    cudaStream_t s);
 void launch_greedy(const float* logits, int n, int vocab, int* tokens, int out_ld, cudaStream_t s);
 void launch_to_model_dtype(const float* x, void* out, long long n, cudaStream_t s);
 void launch_mla_to_cache(int dtype, const float* kv_raw, const void* krope, int kvr, int dr, const int* pos, int N,

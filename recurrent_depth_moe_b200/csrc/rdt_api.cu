@@ -23,6 +23,7 @@ struct Layout {
   // byte offsets into the workspace
   size_t status, h, combined, a, qkv, cq_raw, cq, q, kv_raw, ckv, krope, kvu, attn, x1, f, logits;
   size_t ids, gates, rank, counts, offsets, tiles, ntiles, slot_of, tok_of, gate_of, xg, u, y;
+  size_t cta_count;                  // per-CTA running-row counts of the compaction
   size_t run_list, run_idx, nrun, cum, halted, Avec, emb, rope, pos, p_buf, part_o, part_ml, xn, vt;
   size_t mla_ckv_all, mla_kvu_all;   // MLA with earlier cached keys: rebuilt per-head keys / values
   size_t mla_qa;                     // MLA absorbed decode: absorbed queries (0 = path not used)
@@ -120,6 +121,7 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
   L->run_list = take(N * 4);
   L->run_idx = take(N * 4);
   L->nrun = take(16);
+  L->cta_count = take((size_t)std::max<size_t>((N + 1023) / 1024, 1) * 4);
   L->cum = take(N * 4);
   L->halted = take(N * 4);
   L->p_buf = take(N * 4);
@@ -504,7 +506,7 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
     if (act_on && t + 1 < n_loops) {
       ProfScope ps(PC_OTHER, s);
       launch_compact(at<int*>(ws, x.L.halted), N, at<int*>(ws, x.L.run_list), at<int*>(ws, x.L.run_idx),
-                     at<int*>(ws, x.L.nrun), s);
+                     at<int*>(ws, x.L.nrun), at<int*>(ws, x.L.cta_count), s);
     }
   }
   if (cudaGetLastError() != cudaSuccess) return RDT_ERR_CUDA;
