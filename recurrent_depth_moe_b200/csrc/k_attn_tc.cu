@@ -2,18 +2,21 @@
 // head dim 128, bf16 operands, fp32 softmax and accumulation.
 //
 // One CTA per (sequence, head, pair of 128-query tiles), heaviest pairs first.
-//   warp 0      TMA: both Q tiles once; K and V^T tiles of 64 keys into a 3-stage ring
+//   warp 0      TMA: both Q tiles once; K and V^T tiles of 128 keys into a 2-stage ring
 //   warp 1      TMEM owner; lane 0 issues, per key tile j and query tile q,
-//               S_qj = Q_q K_j^T (two TMEM S buffers per query tile) and
-//               O_q += P_qj V_j (one TMEM O accumulator per query tile)
+//               O_q += P_q(j-1) V_(j-1) and then S_qj = Q_q K_j^T into the same TMEM
+//               columns (one S buffer per query tile; tcgen05 MMAs of one thread run in
+//               order, so S_qj starts after the PV that read P from those columns).
+//               Every MMA is 128 x 128 x 16: the issuing thread, not the tensor pipe, is
+//               the limit for narrower tiles.
 //   warps 2..5  softmax of query tile 0; warps 6..9 softmax of query tile 1.
 //               Thread = query row = TMEM lane: reads its S row, masks (key j visible
 //               iff key_pos0 + j <= q_pos, "OpenMythos 분석", Core Structure causal
 //               mask), keeps a running max m and sum l in the log2 domain, and writes
-//               P = exp2(s - m) as bf16 back into the first 32 columns of the tile's own
-//               S buffer: the PV MMA reads its A operand from TMEM.  The running max is
-//               raised only when it grows by more than 2^8, and only then does the
-//               softmax wait for the previous PV and rescale the O row in TMEM.
+//               P = exp2(s - m) as bf16 back into the first 64 columns of its S buffer:
+//               the PV MMA reads its A operand from TMEM.  The running max is raised only
+//               when it grows by more than 2^8, and only then is the O row rescaled (S of
+//               tile j completing means the PV of tile j-1 has too).
 // The two query tiles share every K / V tile and their softmax groups overlap each
 // other and the tensor core.  V is consumed transposed (V^T[b][g][dim][t], written by
 // the QKV GEMM epilogue) so both MMAs read K-major operands.  Every wait is bounded.
@@ -28,14 +31,15 @@ bool tc_make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsi
 
 namespace fat {
 
-constexpr int BQ = 128, BKV = 64, HD = 128, NQ = 2, STAGES = 4;
+constexpr int BQ = 128, BKV = 128, HD = 128, NQ = 2, STAGES = 2;
 constexpr int QTILE = BQ * HD * 2;      // 32 KB: two 64-dim swizzle atoms of 16 KB
 constexpr int QHALF = QTILE / 2;
-constexpr int KTILE = BKV * HD * 2;     // 16 KB: two atoms [64 keys][64 dims] of 8 KB
+constexpr int KTILE = BKV * HD * 2;     // 32 KB: two atoms [128 keys][64 dims] of 16 KB
 constexpr int KHALF = KTILE / 2;
-constexpr int VTILE = HD * BKV * 2;     // 16 KB: one atom [128 dims][64 keys]
+constexpr int VTILE = HD * BKV * 2;     // 32 KB: two atoms [128 dims][64 keys] of 16 KB
+constexpr int VHALF = VTILE / 2;
 constexpr int SMEM = NQ * QTILE + STAGES * (KTILE + VTILE) + 1024 + 512;
-constexpr int TMEM_COLS = 512;          // S[q][buf] at (2q + buf) * 64 (P in its first 32); O[q] at 256 + 128 q
+constexpr int TMEM_COLS = 512;          // S[q] at 128 q (P in its first 64); O[q] at 256 + 128 q
 constexpr float RESCALE_LOG2 = 8.f;     // lazy rescale threshold (factor 256)
 constexpr int THREADS = 64 + NQ * 128;
 
@@ -69,8 +73,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;                // [STAGES]
   uint64_t* kv_empty = kv_full + STAGES;       // [STAGES]
-  uint64_t* s_full = kv_empty + STAGES;        // [NQ][2]
-  uint64_t* p_full = s_full + 2 * NQ;          // [NQ]
+  uint64_t* s_full = kv_empty + STAGES;        // [NQ]
+  uint64_t* p_full = s_full + NQ;              // [NQ]
   uint64_t* pv_done = p_full + NQ;             // [NQ]
   uint64_t* done = pv_done + NQ;
   uint32_t* tmem_slot = (uint32_t*)(done + 1);
@@ -100,8 +104,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&kv_empty[s], 1);
     }
     for (int q = 0; q < NQ; ++q) {
-      mbar_init(&s_full[2 * q], 1);
-      mbar_init(&s_full[2 * q + 1], 1);
+      mbar_init(&s_full[q], 1);
       mbar_init(&p_full[q], 128);
       mbar_init(&pv_done[q], 1);
     }
@@ -144,50 +147,49 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_load_2d(sK + st * KTILE, &tmK, &kv_full[st], kx, ky);
       tma_load_2d(sK + st * KTILE + KHALF, &tmK, &kv_full[st], kx + 64, ky);
       tma_load_2d(sV + st * VTILE, &tmVt, &kv_full[st], j * BKV, vy);
+      tma_load_2d(sV + st * VTILE + VHALF, &tmVt, &kv_full[st], j * BKV + 64, vy);
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
     constexpr uint32_t IDESC_S = idesc_bf16(128, BKV);
     constexpr uint32_t IDESC_O = idesc_bf16(128, HD);
     bool ok = mbar_wait(q_full, 0, abort_flag);
-    auto issue_pv = [&](int jj) -> bool {
-      const int st = jj % STAGES;
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        if (jj >= nt[q]) continue;
-        if (!mbar_wait(&p_full[q], jj & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t tO = tmem + 256 + q * 128;
-        const uint32_t tP = tmem + (2 * q + (jj & 1)) * BKV;   // P of tile jj, 2 bf16 per column
-#pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t bd = smem_desc(sV + st * VTILE) + 2 * kk;
-          umma_bf16_ts(tO, tP + 8 * kk, bd, IDESC_O, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&pv_done[q]);
-      }
-      umma_commit(&kv_empty[st]);
-      return true;
-    };
-    for (int j = 0; j < nt_max && ok; ++j) {
+    // iteration j: PV of tile j - 1 then S of tile j, per query tile (j = nt_max drains)
+    for (int j = 0; j <= nt_max && ok; ++j) {
       const int st = j % STAGES;
-      if (!(ok = mbar_wait(&kv_full[st], (j / STAGES) & 1, abort_flag))) break;
-      tc_fence_after();
+      const bool load = j < nt_max;
+      if (load) {
+        if (!(ok = mbar_wait(&kv_full[st], (j / STAGES) & 1, abort_flag))) break;
+        tc_fence_after();
+      }
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
-        if (j >= nt[q]) continue;
-        const uint32_t tS = tmem + (2 * q + (j & 1)) * BKV;
+        const uint32_t tS = tmem + q * BKV;   // S of tile j; P of tile j - 1 in its first 64 columns
+        if (j >= 1 && j - 1 < nt[q]) {
+          const int pst = (j - 1) % STAGES;
+          if (!(ok = mbar_wait(&p_full[q], (j - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t tO = tmem + 256 + q * 128;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint64_t ad = smem_desc(sQ + q * QTILE + (kk >> 2) * QHALF) + 2 * (kk & 3);
-          const uint64_t bd = smem_desc(sK + st * KTILE + (kk >> 2) * KHALF) + 2 * (kk & 3);
-          umma_bf16(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < BKV / 16; ++kk) {
+            const uint64_t bd = smem_desc(sV + pst * VTILE + (kk >> 2) * VHALF) + 2 * (kk & 3);
+            umma_bf16_ts(tO, tS + 8 * kk, bd, IDESC_O, (j > 1 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&pv_done[q]);
         }
-        umma_commit(&s_full[2 * q + (j & 1)]);
+        if (load && j < nt[q]) {
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const uint64_t ad = smem_desc(sQ + q * QTILE + (kk >> 2) * QHALF) + 2 * (kk & 3);
+            const uint64_t bd = smem_desc(sK + st * KTILE + (kk >> 2) * KHALF) + 2 * (kk & 3);
+            umma_bf16(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[q]);
+        }
       }
-      if (j >= 1) ok = issue_pv(j - 1);
+      if (!ok) break;
+      if (j >= 1) umma_commit(&kv_empty[(j - 1) % STAGES]);   // K and V of tile j - 1 are consumed
     }
-    if (ok && nt_max > 0) issue_pv(nt_max - 1);
     umma_commit(done);
     mbar_wait(done, 0, abort_flag);
   } else if (warp >= 2) {
@@ -204,14 +206,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t tO = tmem + lane_base + 256 + q * 128;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    const uint32_t tS = tmem + lane_base + q * BKV;
     for (int j = 0; j < ntq; ++j) {
-      if (!(ok = mbar_wait(&s_full[2 * q + (j & 1)], (j >> 1) & 1, abort_flag))) break;
+      if (!(ok = mbar_wait(&s_full[q], j & 1, abort_flag))) break;
       tc_fence_after();
       float s[BKV];
 #pragma unroll
       for (int c = 0; c < BKV; c += 32) {
         float v[32];
-        tmem_ld32(tmem + lane_base + (2 * q + (j & 1)) * BKV + c, v);
+        tmem_ld32(tS + c, v);
 #pragma unroll
         for (int e = 0; e < 32; ++e) s[c + e] = v[e];
       }
@@ -242,15 +245,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         m_used = mx;
         l *= alpha;
       }
+      // P = 2^(s - m) as bf16 pairs over the first 64 columns of the S buffer (S is in
+      // registers already), in two halves of 64 keys
       const float base = (m_used == -INFINITY) ? 0.f : m_used;
-      uint32_t pk[BKV / 2];
       float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 partial sums, then a tree
 #pragma unroll
-      for (int c = 0; c < BKV; c += 2) {
-        const float p0 = exp2f(fmaf(s[c], a.sl2, -base)), p1 = exp2f(fmaf(s[c + 1], a.sl2, -base));
-        sp[(c >> 1) & 7] += p0 + p1;
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-        pk[c >> 1] = *reinterpret_cast<uint32_t*>(&h2);
+      for (int hh = 0; hh < 2; ++hh) {
+        float pf[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const int k = 64 * hh + c;
+          const float p0 = exp2f(fmaf(s[k], a.sl2, -base)), p1 = exp2f(fmaf(s[k + 1], a.sl2, -base));
+          sp[(c >> 1) & 7] += p0 + p1;
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          pf[c >> 1] = __uint_as_float(*reinterpret_cast<uint32_t*>(&h2));
+        }
+        tmem_st32(tS + 32 * hh, pf);
       }
 #pragma unroll
       for (int w = 4; w >= 1; w >>= 1)
@@ -258,10 +268,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int k = 0; k < w; ++k) sp[k] += sp[k + w];
       l += sp[0];
       if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // the max moved: O must hold PV of tile j-1 before it is rescaled.  pv_done can be
-        // at most one phase ahead of this wait (PV j needs this warp's arrival below)
-        if (!(ok = mbar_wait(&pv_done[q], (j - 1) & 1, abort_flag))) break;
-        tc_fence_after();
+        // the max moved: O is rescaled before this tile's PV, after P is
+        // written so the S row is no longer live (the PV of tile j - 1 is
+        // complete: it was issued before S of tile j, whose completion s_full signalled)
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
           float v[32];
@@ -270,15 +279,6 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int e = 0; e < 32; ++e) v[e] *= alpha;
           tmem_st32(tO + c, v);
         }
-      }
-      // P over the first 32 columns of this tile's S buffer (S is in registers already;
-      // every MMA before S of tile j, the PV that read this buffer's last P included, is
-      // complete once s_full fired)
-      {
-        float pf[32];
-#pragma unroll
-        for (int c = 0; c < BKV / 2; ++c) pf[c] = __uint_as_float(pk[c]);
-        tmem_st32(tmem + lane_base + (2 * q + (j & 1)) * BKV, pf);
       }
       tmem_st_wait();
       tc_fence_before();
