@@ -2,7 +2,8 @@
 // head dim 128, bf16 operands, fp32 softmax and accumulation.
 //
 // One CTA per (sequence, head, pair of 128-query tiles), heaviest pairs first.
-//   warp 0      TMA: both Q tiles once; K and V^T tiles of 128 keys into a 2-stage ring
+//   warp 0      TMA: both Q tiles once; K tiles of 128 keys into a 3-stage ring and V^T
+//               tiles into a 2-stage ring (K is freed one iteration before V)
 //   warp 1      TMEM owner; lane 0 issues, per key tile j and query tile q,
 //               O_q += P_q(j-1) V_(j-1) and then S_qj = Q_q K_j^T into the same TMEM
 //               columns (one S buffer per query tile; tcgen05 MMAs of one thread run in
@@ -31,14 +32,14 @@ bool tc_make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsi
 
 namespace fat {
 
-constexpr int BQ = 128, BKV = 128, HD = 128, NQ = 2, STAGES = 2;
+constexpr int BQ = 128, BKV = 128, HD = 128, NQ = 2, KSTAGES = 3, VSTAGES = 2;
 constexpr int QTILE = BQ * HD * 2;      // 32 KB: two 64-dim swizzle atoms of 16 KB
 constexpr int QHALF = QTILE / 2;
 constexpr int KTILE = BKV * HD * 2;     // 32 KB: two atoms [128 keys][64 dims] of 16 KB
 constexpr int KHALF = KTILE / 2;
 constexpr int VTILE = HD * BKV * 2;     // 32 KB: two atoms [128 dims][64 keys] of 16 KB
 constexpr int VHALF = VTILE / 2;
-constexpr int SMEM = NQ * QTILE + STAGES * (KTILE + VTILE) + 1024 + 512;
+constexpr int SMEM = NQ * QTILE + KSTAGES * KTILE + VSTAGES * VTILE + 1024 + 512;   // 225.5 KB
 constexpr int TMEM_COLS = 512;          // S[q] at 128 q (P in its first 64); O[q] at 256 + 128 q
 constexpr float RESCALE_LOG2 = 8.f;     // lazy rescale threshold (factor 256)
 constexpr int THREADS = 64 + NQ * 128;
@@ -67,13 +68,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;                          // [NQ] query tiles
-  uint8_t* sK = sQ + NQ * QTILE;               // [STAGES]
-  uint8_t* sV = sK + STAGES * KTILE;           // [STAGES]
-  uint64_t* bars = (uint64_t*)(sV + STAGES * VTILE);
+  uint8_t* sK = sQ + NQ * QTILE;               // [KSTAGES]
+  uint8_t* sV = sK + KSTAGES * KTILE;          // [VSTAGES]
+  uint64_t* bars = (uint64_t*)(sV + VSTAGES * VTILE);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;                // [STAGES]
-  uint64_t* kv_empty = kv_full + STAGES;       // [STAGES]
-  uint64_t* s_full = kv_empty + STAGES;        // [NQ]
+  uint64_t* k_full = bars + 1;                 // [KSTAGES]
+  uint64_t* k_empty = k_full + KSTAGES;        // [KSTAGES]
+  uint64_t* v_full = k_empty + KSTAGES;        // [VSTAGES]
+  uint64_t* v_empty = v_full + VSTAGES;        // [VSTAGES]
+  uint64_t* s_full = v_empty + VSTAGES;        // [NQ]
   uint64_t* p_full = s_full + NQ;              // [NQ]
   uint64_t* pv_done = p_full + NQ;             // [NQ]
   uint64_t* done = pv_done + NQ;
@@ -99,9 +102,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < KSTAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < VSTAGES; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int q = 0; q < NQ; ++q) {
       mbar_init(&s_full[q], 1);
@@ -140,14 +147,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int kx = a.k_col0 + g * HD;
     const int vy = (b * a.Hkv + g) * HD;
     for (int j = 0; j < nt_max; ++j) {
-      const int st = j % STAGES;
-      if (!mbar_wait(&kv_empty[st], ((j / STAGES) & 1) ^ 1, abort_flag)) break;
-      mbar_expect_tx(&kv_full[st], KTILE + VTILE);
+      const int ks = j % KSTAGES, vs = j % VSTAGES;
+      if (!mbar_wait(&k_empty[ks], ((j / KSTAGES) & 1) ^ 1, abort_flag)) break;
+      mbar_expect_tx(&k_full[ks], KTILE);
       const int ky = b * a.T + j * BKV;
-      tma_load_2d(sK + st * KTILE, &tmK, &kv_full[st], kx, ky);
-      tma_load_2d(sK + st * KTILE + KHALF, &tmK, &kv_full[st], kx + 64, ky);
-      tma_load_2d(sV + st * VTILE, &tmVt, &kv_full[st], j * BKV, vy);
-      tma_load_2d(sV + st * VTILE + VHALF, &tmVt, &kv_full[st], j * BKV + 64, vy);
+      tma_load_2d(sK + ks * KTILE, &tmK, &k_full[ks], kx, ky);
+      tma_load_2d(sK + ks * KTILE + KHALF, &tmK, &k_full[ks], kx + 64, ky);
+      if (!mbar_wait(&v_empty[vs], ((j / VSTAGES) & 1) ^ 1, abort_flag)) break;
+      mbar_expect_tx(&v_full[vs], VTILE);
+      tma_load_2d(sV + vs * VTILE, &tmVt, &v_full[vs], j * BKV, vy);
+      tma_load_2d(sV + vs * VTILE + VHALF, &tmVt, &v_full[vs], j * BKV + 64, vy);
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
@@ -156,23 +165,26 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = mbar_wait(q_full, 0, abort_flag);
     // iteration j: PV of tile j - 1 then S of tile j, per query tile (j = nt_max drains)
     for (int j = 0; j <= nt_max && ok; ++j) {
-      const int st = j % STAGES;
+      const int ks = j % KSTAGES, pvs = (j + VSTAGES - 1) % VSTAGES;   // K of tile j, V of tile j - 1
       const bool load = j < nt_max;
       if (load) {
-        if (!(ok = mbar_wait(&kv_full[st], (j / STAGES) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(&k_full[ks], (j / KSTAGES) & 1, abort_flag))) break;
+        tc_fence_after();
+      }
+      if (j >= 1) {
+        if (!(ok = mbar_wait(&v_full[pvs], ((j - 1) / VSTAGES) & 1, abort_flag))) break;
         tc_fence_after();
       }
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
         const uint32_t tS = tmem + q * BKV;   // S of tile j; P of tile j - 1 in its first 64 columns
         if (j >= 1 && j - 1 < nt[q]) {
-          const int pst = (j - 1) % STAGES;
           if (!(ok = mbar_wait(&p_full[q], (j - 1) & 1, abort_flag))) break;
           tc_fence_after();
           const uint32_t tO = tmem + 256 + q * 128;
 #pragma unroll
           for (int kk = 0; kk < BKV / 16; ++kk) {
-            const uint64_t bd = smem_desc(sV + pst * VTILE + (kk >> 2) * VHALF) + 2 * (kk & 3);
+            const uint64_t bd = smem_desc(sV + pvs * VTILE + (kk >> 2) * VHALF) + 2 * (kk & 3);
             umma_bf16_ts(tO, tS + 8 * kk, bd, IDESC_O, (j > 1 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&pv_done[q]);
@@ -181,14 +193,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint64_t ad = smem_desc(sQ + q * QTILE + (kk >> 2) * QHALF) + 2 * (kk & 3);
-            const uint64_t bd = smem_desc(sK + st * KTILE + (kk >> 2) * KHALF) + 2 * (kk & 3);
+            const uint64_t bd = smem_desc(sK + ks * KTILE + (kk >> 2) * KHALF) + 2 * (kk & 3);
             umma_bf16(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[q]);
         }
       }
       if (!ok) break;
-      if (j >= 1) umma_commit(&kv_empty[(j - 1) % STAGES]);   // K and V of tile j - 1 are consumed
+      if (load) umma_commit(&k_empty[ks]);     // K of tile j is consumed once both S MMAs finish
+      if (j >= 1) umma_commit(&v_empty[pvs]);  // V of tile j - 1 once both PV MMAs finish
     }
     umma_commit(done);
     mbar_wait(done, 0, abort_flag);
