@@ -56,6 +56,96 @@ struct Args {
 
 using namespace rdt::tc;
 
+// 32 TMEM columns of this warp's lanes into registers, no wait: the caller issues
+// tcgen05.wait::ld before it reads any of r
+__device__ __forceinline__ void tmem_ld32_nw(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the special-function unit
+__device__ __forceinline__ float ex2_sfu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x for a pair on the FMA pipe (Cody-Waite style range reduction): x = j + f with j the
+// nearest integer (added to a 1.5 * 2^23 shifter, whose low mantissa bits then hold j) and
+// f in [-1/2, 1/2]; 2^f by a cubic fitted to minimise the relative error on that interval
+// (Lawson's reweighted least squares; max relative error 7.5e-5, well inside the bf16
+// rounding that P gets); 2^j added into the exponent field.  x is clamped at -125 so the
+// exponent stays normal.  Used for a share of the exponentials so that the SFU and the
+// FMA pipe finish together.
+constexpr float EXP2_C0 = 0.99992806f, EXP2_C1 = 0.69326097f, EXP2_C2 = 0.24261114f, EXP2_C3 = 0.05517167f;
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 jf = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(jf, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+  p = __ffma2_rn(p, f, make_float2(EXP2_C1, EXP2_C1));
+  p = __ffma2_rn(p, f, make_float2(EXP2_C0, EXP2_C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// P = 2^(s * sl2 - base) for one row of BKV scores, written as bf16 pairs into the first
+// BKV / 2 TMEM columns at tS; returns the fp32 row sum.  POLY: pairs whose index has
+// (pair & 7) < 3 (3 in 8) take the FMA-pipe exponential, the rest the SFU; tiles with
+// masked keys use the SFU throughout, so masked keys (s = -inf) give exactly 0.
+template <bool POLY>
+__device__ __forceinline__ float exp_row(const float (&s)[BKV], float sl2, float base, uint32_t tS) {
+  const float2 sc = make_float2(sl2, sl2), nb = make_float2(-base, -base);
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+  for (int hh = 0; hh < BKV / 32; ++hh) {
+    uint32_t pf[16];
+#pragma unroll
+    for (int pi = 0; pi < 16; ++pi) {
+      const int k = 32 * hh + 2 * pi;
+      const float2 x = __ffma2_rn(make_float2(s[k], s[k + 1]), sc, nb);
+      float2 p;
+      if (POLY && (pi & 7) < 3) {   // pair index within the row: (16 hh + pi) & 7 = pi & 7
+        p = ex2_poly2(x);
+      } else {
+        p = make_float2(ex2_sfu(x.x), ex2_sfu(x.y));
+      }
+      acc[pi & 3] = __fadd2_rn(acc[pi & 3], p);
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(p.x, p.y);
+      pf[pi] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    tmem_st16(tS + 16 * hh, pf);
+  }
+  acc[0] = __fadd2_rn(acc[0], acc[1]);
+  acc[2] = __fadd2_rn(acc[2], acc[3]);
+  acc[0] = __fadd2_rn(acc[0], acc[2]);
+  return acc[0].x + acc[0].y;
+}
+
 __device__ __forceinline__ int visible_tiles(const Args& a, long long row_last, int q_rows) {
   if (q_rows <= 0) return 0;
   int n_vis = min(a.n_keys, a.q_pos[row_last] - a.key_pos0 + 1);
@@ -221,16 +311,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = true;
     const uint32_t tS = tmem + lane_base + q * BKV;
     for (int j = 0; j < ntq; ++j) {
-      if (!(ok = mbar_wait(&s_full[q], j & 1, abort_flag))) break;
+      // warp-uniform outcome: the TMEM loads and stores below are .sync.aligned
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s_full[q], j & 1, abort_flag)))) break;
       tc_fence_after();
+      uint32_t sr[BKV];
+#pragma unroll
+      for (int c = 0; c < BKV; c += 32) tmem_ld32_nw(tS + c, &sr[c]);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       float s[BKV];
 #pragma unroll
-      for (int c = 0; c < BKV; c += 32) {
-        float v[32];
-        tmem_ld32(tS + c, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c + e] = v[e];
-      }
+      for (int c = 0; c < BKV; ++c) s[c] = __uint_as_float(sr[c]);
       const int k0 = j * BKV;
       const int kp0 = a.key_pos0 + k0;
       const bool need_mask = (kp0 + BKV - 1 > my_pos) || (k0 + BKV > n_vis);
@@ -239,17 +329,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < BKV; ++c)
           if (kp0 + c > my_pos || k0 + c >= n_vis) s[c] = -INFINITY;
       }
-      // row max as 8 independent chains and a tree (max is exact in any order)
+      // row max: 8 independent chains of 3-input max, then a tree (exact in any order)
       float mp[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mp[k] = s[k];
+      for (int k = 0; k < 8; ++k) mp[k] = fmaxf(s[k], s[8 + k]);
 #pragma unroll
-      for (int c = 8; c < BKV; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
+      for (int c = 16; c < BKV; c += 16)
 #pragma unroll
-      for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-        for (int k = 0; k < w; ++k) mp[k] = fmaxf(mp[k], mp[k + w]);
-      const float mx = mp[0] * a.sl2;            // the scale is positive: max commutes with it
+        for (int k = 0; k < 8; ++k) mp[k] = fmax3(mp[k], s[c + k], s[c + 8 + k]);
+      mp[0] = fmax3(mp[0], mp[1], mp[2]);
+      mp[3] = fmax3(mp[3], mp[4], mp[5]);
+      mp[6] = fmaxf(mp[6], mp[7]);
+      const float mx = fmax3(mp[0], mp[3], mp[6]) * a.sl2;   // the scale is positive: max commutes with it
       float alpha = 1.f;
       if (j == 0) {
         m_used = mx;
@@ -258,32 +349,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         m_used = mx;
         l *= alpha;
       }
-      // P = 2^(s - m) as bf16 pairs over the first 64 columns of the S buffer (S is in
-      // registers already), in two halves of 64 keys
+      // P over the first 64 columns of the S buffer (S is in registers already)
       const float base = (m_used == -INFINITY) ? 0.f : m_used;
-      float sp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 8 partial sums, then a tree
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float pf[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const int k = 64 * hh + c;
-          const float p0 = exp2f(fmaf(s[k], a.sl2, -base)), p1 = exp2f(fmaf(s[k + 1], a.sl2, -base));
-          sp[(c >> 1) & 7] += p0 + p1;
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          pf[c >> 1] = __uint_as_float(*reinterpret_cast<uint32_t*>(&h2));
-        }
-        tmem_st32(tS + 32 * hh, pf);
-      }
-#pragma unroll
-      for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-        for (int k = 0; k < w; ++k) sp[k] += sp[k + w];
-      l += sp[0];
+      // exp_row stores to TMEM (.sync.aligned): the choice must be the same for the whole warp
+      l += __any_sync(0xffffffffu, need_mask) ? exp_row<false>(s, a.sl2, base, tS)
+                                              : exp_row<true>(s, a.sl2, base, tS);
       if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // the max moved: O is rescaled before this tile's PV, after P is
-        // written so the S row is no longer live (the PV of tile j - 1 is
-        // complete: it was issued before S of tile j, whose completion s_full signalled)
+        // the max moved: O is rescaled before this tile's PV, after P is written so the S
+        // row is no longer live (the PV of tile j - 1 is complete: it was issued before S
+        // of tile j, whose completion s_full signalled)
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
           float v[32];
@@ -298,7 +372,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(&p_full[q]);
     }
     // final: O / l
-    if (ok && ntq > 0 && mbar_wait(&pv_done[q], (ntq - 1) & 1, abort_flag)) {
+    if (ok && ntq > 0 && __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (ntq - 1) & 1, abort_flag))) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       bf16* orow = a.o + (row0 + rl) * a.o_row + (long long)h * HD;
