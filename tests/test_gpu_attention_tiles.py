@@ -1,0 +1,57 @@
+"""Prefill attention at sequence lengths around its 128-query / 128-key tiles (head dim
+128, bf16: the tcgen05 kernel when T is a multiple of 8, the mma.sync kernel otherwise).
+Checked for one loop, teacher-forced: from the kernel's own state entering the loop, the
+attention branch's share of the FFN input f = RMSNorm_ffn(x + Attn(RMSNorm_attn(x))), i.e.
+f minus RMSNorm_ffn(x), in the oracle and in the kernel's trace of f ("OpenMythos 분석", Core
+Structure: causal self-attention inside the pre-norm block).
+Peaky attention weights (std 0.08) so that the softmax is far from uniform."""
+import pytest
+import torch
+
+import rdt_inputs as RI
+from oracle import rdt_oracle as O
+from tests._helpers import BF16_TOL, rel_l2, to_dev
+
+pytestmark = pytest.mark.gpu
+
+R = pytest.importorskip("recurrent_depth_moe_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    R.load_library()
+
+
+# 8: one short query tile; 120 / 128 / 136: around one tile; 256 / 264: one full pair and a
+# pair plus 8 rows; 392: two pairs, the last tile 8 rows; 520: five tiles (a pair with one
+# tile); 100: not a multiple of 8 (the mma.sync kernel)
+@pytest.mark.parametrize("T", [8, 120, 128, 136, 256, 264, 392, 520, 100])
+def test_attention_tile_edges(T):
+    cfg = RI.get_workload("mid_gqa_bf16").cfg
+    W = RI.block_weights(cfg, 31, attn_std=0.08)
+    B, L = 2, 1
+    h0, e = RI.recurrent_inputs(cfg, B, T, 32)
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    tr = R.Trace.alloc(cfg, L, 0, B * T)
+    blk.forward(h0.cuda(), e.cuda(), B, T, L, 0.99, trace=tr)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    h_in = tr.h_in[0].cpu().double()
+    emb = O.loop_embedding(0, cfg.loop_dim, cfg.dim, cfg.loop_theta)
+    comb = O.rmsnorm(h_in + emb + e.double(), W["rec_norm_w"], cfg.norm_eps)
+    pos = torch.arange(B * T) % T
+    _, _, info = O.transformer_block(cfg, W, comb, B, pos, True)
+    # the attention branch's share of f: f with the branch minus f without it
+    f0 = O.rmsnorm(comb, W["ffn_norm_w"], cfg.norm_eps)
+    d_o = info["f"] - f0
+    d_k = tr.f[0].cpu().double() - f0
+    assert rel_l2(d_o, info["f"]) > 0.05, "attention barely moves f: the check would be weak"
+    for b in range(B):   # every sequence on its own
+        rows = slice(b * T, (b + 1) * T)
+        err = rel_l2(d_k[rows], d_o[rows])
+        assert err <= BF16_TOL, f"sequence {b}: relative L2 of the attention branch {err:.3e}"
+    # the last query row of each sequence sees every key: compare it on its own too
+    last = [b * T + T - 1 for b in range(B)]
+    assert rel_l2(d_k[last], d_o[last]) <= BF16_TOL
