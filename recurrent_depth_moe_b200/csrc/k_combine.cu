@@ -402,10 +402,12 @@ bool launch_combine_vpl(const CombineParams& p, int n_rows, cudaStream_t s) {
                      ((uintptr_t)p.lora_down % 16) == 0 && ((uintptr_t)p.lora_B % 16) == 0;
   const int sms = combine_sm_count();
   if (n_rows <= 2 * sms) {
-    // few rows (decode): one row group per CTA and one CTA per row (two fit an SM), so the
-    // rows spread over the SMs instead of queueing in the 8 groups of a few CTAs; the LoRA
-    // matrices are read through L1 / L2 (staging them would cost more than one row uses)
-    { k_combine_warp<T, VPL, WPR, 1, false><<<std::max(1, n_rows), WPR * 32, 0, s>>>(p); note_launch(); }
+    // few rows (decode): one CTA per row with one warp per 128 columns, so the rows spread
+    // over the SMs and each warp's chain of dependent loads is one 16-byte vector deep per
+    // array; the LoRA matrices are read through L1 / L2 (staging them would cost more than
+    // one row uses)
+    constexpr int WPR_S = VPL;
+    { k_combine_warp<T, VPL, WPR_S, 1, false><<<std::max(1, n_rows), WPR_S * 32, 0, s>>>(p); note_launch(); }
     return true;
   }
   const int grid = std::max(1, std::min((n_rows + GROUPS - 1) / GROUPS, sms));
