@@ -60,6 +60,7 @@ EXPORTS = ("rdt_workspace_size", "rdt_recurrent_forward", "rdt_recurrent_decode_
            "rdt_launch_count", "rdt_profile_start", "rdt_profile_stop")
 
 _lib = None
+_profiling = False
 
 
 def load(path: str = LIB_PATH):
@@ -122,11 +123,22 @@ def launch_count() -> int:
 
 
 def profile_start():
+    global _profiling
     check("rdt_profile_start", load().rdt_profile_start())
+    _profiling = True
+
+
+def profiling() -> bool:
+    """True between profile_start() and profile_stop(): the per-class CUDA events are
+    recorded at launch time, so callers that would replay a captured CUDA graph run
+    eagerly instead."""
+    return _profiling
 
 
 def profile_stop() -> dict:
     """{kernel class: (launches, total_ms)} recorded since profile_start()."""
+    global _profiling
+    _profiling = False
     buf = (rdt_kernel_time * 32)()
     n = load().rdt_profile_stop(buf, 32)
     if n < 0:

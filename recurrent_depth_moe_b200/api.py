@@ -395,10 +395,18 @@ class Generator:
     prelude / coda layer and per recurrent loop; every later step runs the last token
     alone at position prompt_len + step - 1 against those caches.  The next token is the
     greedy choice (rdt_greedy_tokens).  All buffers are allocated once per generator, so
-    the decode steps allocate nothing."""
+    the decode steps allocate nothing.
+
+    With cuda_graph (the default) the decode step's launches (about 20 per loop plus the
+    prelude, coda, head and greedy choice) are captured once into a CUDA graph on the
+    second decode call and replayed from then on.  Everything a step reads is at a fixed
+    address: the previous token is copied into `cur_tok` and the cache length set before
+    the replay, and the new token copied out of `cur_tok` after it.  The first decode call
+    runs eagerly (it also performs the kernels' one-time attribute setup), and so does every
+    call made while the library's profiler is recording."""
 
     def __init__(self, cfg, MW: dict, batch: int, prompt_len: int, max_new_tokens: int, n_loops: int,
-                 act_threshold: float = 0.0):
+                 act_threshold: float = 0.0, cuda_graph: bool = True):
         _require_cuda()
         self.cfg, self.MW = cfg, MW
         self.B, self.T0, self.new, self.L, self.thr = batch, prompt_len, max_new_tokens, n_loops, act_threshold
@@ -430,6 +438,11 @@ class Generator:
                         torch.empty(n_loops, B, dtype=torch.float32, device="cuda"),
                         torch.empty(n_loops, B, cfg.n_experts_per_tok, dtype=torch.int32, device="cuda"))
         self.cache_len = torch.empty(B, dtype=torch.int32, device="cuda")
+        self.cur_tok = torch.empty(B, dtype=torch.int32, device="cuda")
+        self.cuda_graph = cuda_graph
+        self._graph = None
+        self._eager_decodes = 0
+        self.graph_launches = 0      # library kernels in one replay of the captured step
 
     def _run_blocks(self, blocks, caches, x, y, seq, start_pos, cache_len):
         for blk, c in zip(blocks, caches):
@@ -457,14 +470,14 @@ class Generator:
         greedy_tokens(self.logits, out=self.tokens[0])
         return self.tokens[0]
 
-    def decode(self, step: int) -> torch.Tensor:
-        """Step `step` >= 1: the token of step - 1 at position prompt_len + step - 1."""
-        B, D = self.B, self.cfg.dim
+    def _decode_body(self, tok_in: torch.Tensor, tok_out: torch.Tensor):
+        """One decode step from the tokens in tok_in [B] to the greedy tokens in tok_out [B],
+        with the cache length already in self.cache_len."""
+        B = self.B
         lib = N.load()
-        self.cache_len.fill_(self.T0 + step - 1)
         x, y = self.xa[:B], self.xb[:B]
         rc = lib.rdt_embed(ctypes.byref(config_struct(self.cfg)), self.MW["embed"].data_ptr(),
-                           self.MW["embed"].shape[0], self.tokens[step - 1].data_ptr(), B, x.data_ptr(), _stream())
+                           self.MW["embed"].shape[0], tok_in.data_ptr(), B, x.data_ptr(), _stream())
         N.check("rdt_embed", rc)
         x, y = self._run_blocks(self.pre, self.pre_cache, x, y, 1, 0, self.cache_len)
         e = self.e[:B]
@@ -474,7 +487,25 @@ class Generator:
                             workspace=self.ws_rec_decode)
         x, y = self._run_blocks(self.coda, self.coda_cache, out[0], y, 1, 0, self.cache_len)
         head(self.cfg, x, self.MW["norm_w"], self.MW["head"], out=self.logits, workspace=self.ws_head)
-        greedy_tokens(self.logits, out=self.tokens[step])
+        greedy_tokens(self.logits, out=tok_out)
+
+    def decode(self, step: int) -> torch.Tensor:
+        """Step `step` >= 1: the token of step - 1 at position prompt_len + step - 1."""
+        self.cache_len.fill_(self.T0 + step - 1)
+        if not self.cuda_graph or N.profiling() or self._eager_decodes == 0:
+            self._decode_body(self.tokens[step - 1], self.tokens[step])
+            self._eager_decodes += 1
+            return self.tokens[step]
+        self.cur_tok.copy_(self.tokens[step - 1])
+        if self._graph is None:
+            g = torch.cuda.CUDAGraph()
+            n0 = N.launch_count()
+            with torch.cuda.graph(g):
+                self._decode_body(self.cur_tok, self.cur_tok)
+            self.graph_launches = N.launch_count() - n0
+            self._graph = g
+        self._graph.replay()
+        self.tokens[step].copy_(self.cur_tok)
         return self.tokens[step]
 
     def run(self, prompt_ids: torch.Tensor) -> torch.Tensor:

@@ -92,3 +92,28 @@ def test_generate_bf16_teacher_forced():
         gap = ol.max(-1).values - ol.gather(1, toks[:, s:s + 1])[:, 0]
         span = ol.max(-1).values - ol.min(-1).values
         assert (gap <= 2e-2 * span).all(), s
+
+
+@pytest.mark.parametrize("name", ["tiny_gqa_fp32", "tiny_mla_bf16"])
+def test_graph_replay_equals_eager(name):
+    """The Generator's CUDA-graph replay of the decode step gives the eager steps' tokens
+    and logits bit for bit (same kernels, same fixed buffers; the step's inputs are copied
+    into place before each replay)."""
+    wl = RI.get_workload(name)
+    cfg = wl.cfg
+    MW = to_dev(RI.model_weights(cfg, wl.seed))
+    prompt = torch.randint(0, cfg.vocab_size, (2, 16), generator=torch.Generator().manual_seed(9))
+    ids = prompt.to(device="cuda", dtype=torch.int32).contiguous()
+    runs = []
+    for graph in (False, True):
+        gen = R.Generator(cfg, MW, 2, 16, 8, 8, wl.act_threshold, cuda_graph=graph)
+        gen.prefill(ids)
+        logits = []
+        for s in range(1, 8):
+            gen.decode(s)
+            logits.append(gen.logits.clone())
+        torch.cuda.synchronize()
+        runs.append((gen.tokens.clone(), torch.stack(logits), gen._graph is not None, gen.graph_launches))
+    assert not runs[0][2] and runs[1][2] and runs[1][3] > 0
+    assert torch.equal(runs[0][0], runs[1][0])
+    assert torch.equal(runs[0][1], runs[1][1])
