@@ -396,7 +396,8 @@ def run_decode(args, rank, world, local_rank, name="rdt3b_decode"):
     wl = RI.get_workload(name)
     cfg = wl.cfg
     B, L, steps = wl.batch, wl.n_loops, args.decode_steps
-    t_max = wl.cache_len + steps + args.warmup
+    n_prof = min(steps, 32)                 # eager, profiled steps after the timed ones
+    t_max = wl.cache_len + args.warmup + 2 + steps + n_prof
     W = RI.block_weights(cfg, wl.seed, device=dev)
     make_cache = RI.random_kv_cache if cfg.attn_type == "gqa" else RI.random_latent_cache
     k, v = make_cache(cfg, L, B, t_max, wl.cache_len, REP.replica_input_seed(wl.seed, rank), device=dev)
@@ -411,40 +412,48 @@ def run_decode(args, rank, world, local_rank, name="rdt3b_decode"):
     clen = torch.full((B,), wl.cache_len, dtype=torch.int32, device=dev)
     out = (torch.empty(B, cfg.dim, dtype=torch.float32, device=dev), torch.empty(L, B, dtype=torch.float32, device=dev),
            torch.empty(L, B, cfg.n_experts_per_tok, dtype=torch.int32, device=dev))
+    # the step through the library's DecodeGraph: eager once, then captured and replayed
+    dg = R.DecodeGraph(blk, B, cache, clen, L, wl.act_threshold, workspace=ws, out=out)
     for st in range(args.warmup):
-        blk.decode_step(h0s[st], es[st], clen, cache, L, wl.act_threshold, out=out, workspace=ws)
-        clen.add_(1)
+        dg.step(h0s[st], es[st])
+    while dg._graph is None:                # fewer than 2 warm-up steps: capture before timing
+        dg.step(h0s[0], es[0])
     torch.cuda.synchronize()
     assert blk.read_status() == 0, "device status word set during decode warm-up"
-    lens0 = clen.clone()
     stream = torch.cuda.current_stream()
-    NAT.profile_start()
-    n0 = NAT.launch_count()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for st in range(steps):
-        blk.decode_step(h0s[args.warmup + st], es[args.warmup + st], clen, cache, L, wl.act_threshold, out=out,
-                        workspace=ws)
-        clen.add_(1)
+        dg.step(h0s[args.warmup + st], es[args.warmup + st])
     e1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    launches = NAT.launch_count() - n0
-    prof = NAT.profile_stop()
+    assert blk.read_status() == 0, "device status word set during the timed decode steps"
     ms = e0.elapsed_time(e1) / steps
     ms_max = REP.max_over_ranks(ms, device=dev)
     # algorithmic bytes of the last timed step (its routing and cache lengths)
     bytes_step = decode_algorithmic_bytes(cfg, out[2].cpu(), (clen - 1).cpu())
     pk, pk_kind = peaks()
     gbs = bytes_step / (ms / 1e3) / 1e9
-    # attention alone: the cache bytes of all timed steps over the attention kernels' time
-    keys_read = float(steps * (lens0.double() + 1).sum() + B * steps * (steps - 1) / 2) * L
-    attn_ms = prof.get("attention", (0, 0.0))[1] / steps
-    attn_bytes = keys_read / steps * cache_bytes_per_key(cfg)
+    # per-class breakdown, attention roofline and launch count: n_prof more steps, eagerly
+    # (the profiler's events are recorded at launch time, so DecodeGraph does not replay
+    # while profiling); not part of the timed numbers
+    lens0 = clen.clone()
+    NAT.profile_start()
+    n0 = NAT.launch_count()
+    for st in range(n_prof):
+        dg.step(h0s[st], es[st])
+    torch.cuda.synchronize()
+    launches = (NAT.launch_count() - n0) * steps // n_prof
+    prof = NAT.profile_stop()
+    # attention alone: the cache bytes of the profiled steps over the attention kernels' time
+    keys_read = float(n_prof * (lens0.double() + 1).sum() + B * n_prof * (n_prof - 1) / 2) * L
+    attn_ms = prof.get("attention", (0, 0.0))[1] / n_prof
+    attn_bytes = keys_read / n_prof * cache_bytes_per_key(cfg)
     attn_gbs = attn_bytes / (attn_ms / 1e3) / 1e9 if attn_ms else None
     if cfg.attn_type == "gqa":
         attn_desc = f"{cfg.n_heads} heads GQA ({cfg.n_kv_heads} kv, head dim {cfg.head_dim})"
@@ -471,8 +480,10 @@ def run_decode(args, rank, world, local_rank, name="rdt3b_decode"):
                         "frac": gbs / pk.get("hbm_gbs"), "peak_kind": f"{pk_kind} HBM copy bandwidth",
                         "algorithmic_bytes_per_step": bytes_step, "traffic": None},
            "gpu_launches": launches,
-           "kernel_ms_per_step": {k2: {"launches": v2[0], "ms_per_step": v2[1] / steps} for k2, v2 in sorted(prof.items())}}
-    del k, v, cache, W, blk, ws
+           "cuda_graph": {"decode_step_replayed": dg._graph is not None, "launches_per_step": dg.graph_launches},
+           "kernel_ms_per_step_eager": {k2: {"launches": v2[0] / n_prof, "ms_per_step": v2[1] / n_prof}
+                                        for k2, v2 in sorted(prof.items())}}
+    del k, v, cache, W, blk, ws, dg
     torch.cuda.empty_cache()
     return res
 

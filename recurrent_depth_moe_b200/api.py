@@ -248,6 +248,55 @@ class RecurrentBlock:
         return lib.rdt_read_device_status(self._ws.data_ptr(), _stream()) if self._ws is not None else N.RDT_OK
 
 
+class DecodeGraph:
+    """RecurrentBlock.decode_step replayed from a CUDA graph, for a serving loop that steps
+    the same sequences against the same caches.  Every address the captured launches use
+    is fixed: the step's h0 / e are copied into `h_in` / `e_in` before each replay, the
+    outputs land in `out`, and the cache length advances inside the graph (cache_len += 1
+    after the step, as an eager loop would do).  The first call runs eagerly (it also
+    performs the kernels' one-time attribute setup), the second captures the step once and
+    replays it, every later call replays.  Calls made while the library's profiler records
+    run eagerly, since its CUDA events are recorded at launch time."""
+
+    def __init__(self, blk: "RecurrentBlock", batch: int, cache: KVCache, cache_len: torch.Tensor, n_loops: int,
+                 act_threshold: float = 0.0, workspace: Optional[torch.Tensor] = None, out: Optional[tuple] = None):
+        cfg = blk.cfg
+        self.blk, self.B, self.cache, self.cache_len = blk, batch, cache, cache_len
+        self.L, self.thr = n_loops, act_threshold
+        self.ws = workspace if workspace is not None else blk.workspace(batch, 1, cache.t_max)
+        self.out = out if out is not None else (
+            torch.empty(batch, cfg.dim, dtype=torch.float32, device="cuda"),
+            torch.empty(n_loops, batch, dtype=torch.float32, device="cuda"),
+            torch.empty(n_loops, batch, cfg.n_experts_per_tok, dtype=torch.int32, device="cuda"))
+        self.h_in = torch.empty(batch, cfg.dim, dtype=torch.float32, device="cuda")
+        self.e_in = torch.empty(batch, cfg.dim, dtype=blk.dtype, device="cuda")
+        self._graph = None
+        self._eager = 0
+        self.graph_launches = 0      # library kernels in one replay
+
+    def _body(self, h0, e):
+        self.blk.decode_step(h0, e, self.cache_len, self.cache, self.L, self.thr, out=self.out, workspace=self.ws)
+        self.cache_len.add_(1)
+
+    def step(self, h0: torch.Tensor, e: torch.Tensor) -> tuple:
+        """One decode step of every sequence; returns (h_out, halt weights, expert ids)."""
+        if N.profiling() or self._eager == 0:
+            self._body(h0, e)
+            self._eager += 1
+            return self.out
+        self.h_in.copy_(h0)
+        self.e_in.copy_(e)
+        if self._graph is None:
+            g = torch.cuda.CUDAGraph()
+            n0 = N.launch_count()
+            with torch.cuda.graph(g):
+                self._body(self.h_in, self.e_in)
+            self.graph_launches = N.launch_count() - n0
+            self._graph = g
+        self._graph.replay()
+        return self.out
+
+
 class Block:
     """One pre-norm prelude/coda block (dense SwiGLU FFN) or MoE block bound to its weights."""
 
