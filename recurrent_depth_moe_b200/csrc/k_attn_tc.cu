@@ -14,8 +14,9 @@
 //               Thread = query row = TMEM lane: reads its S row, masks (key j visible
 //               iff key_pos0 + j <= q_pos, "OpenMythos 분석", Core Structure causal
 //               mask), keeps a running max m and sum l in the log2 domain, and writes
-//               P = exp2(s - m) as bf16 back into the first 64 columns of its S buffer:
-//               the PV MMA reads its A operand from TMEM.  The running max is raised only
+//               P = exp2(s - m) as bf16 back into the first 64 columns of its S buffer
+//               (3 in 8 of the exponentials on the FMA pipe, the rest on the SFU): the
+//               PV MMA reads its A operand from TMEM.  The running max is raised only
 //               when it grows by more than 2^8, and only then is the O row rescaled (S of
 //               tile j completing means the PV of tile j-1 has too).
 // The two query tiles share every K / V tile and their softmax groups overlap each
