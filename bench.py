@@ -119,8 +119,8 @@ class ClockSampler:
 # DRAM traffic of one full-size expert-up launch (1B shape, 16384 tokens x 5 slots), from ncu
 # dram__bytes_read.sum + dram__bytes_write.sum (1 pass; profiles/expert_up_gemm_rdt1b_small_case.md).
 # Reported only while the GEMM's sources are the ones it was captured from.
-EXPERT_UP_TRAFFIC = {"bytes": 1.43e9 + 303.23e6, "workload": "rdt1b_prefill", "n_loops": 16,
-                     "sha256": "23998a96b0d9c533a91ed917bd60185d2621b939bf0f519acb37707aad37e0b3"}
+EXPERT_UP_TRAFFIC = {"bytes": 1426189056 + 301016576, "workload": "rdt1b_prefill", "n_loops": 16,
+                     "sha256": "94721409d27298b49959cc5af1073df041ed4ea4bd4e8b9a04c45934a42826c4"}
 
 
 def expert_up_traffic(wl):

@@ -288,7 +288,9 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int q = 0; q < 8; ++q) rcur[q] = __ldg(reinterpret_cast<const float4*>(rrow) + q);
       }
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+      // warp-uniform outcome: the TMEM loads below are .sync.aligned, so a wait that gave up
+      // in some lanes only must not let the others go on to them
+      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort_flag))) break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN;
       if (EPI == EPI_RESID_F32 && args.k_splits <= 1) {
