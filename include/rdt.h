@@ -170,7 +170,13 @@ RDT_API rdt_status rdt_recurrent_forward(const rdt_config* cfg, const rdt_weight
  * generation cache): one new token per sequence b at position cache_len[b]
  * (device int32 [batch]); loop t reads and extends loop cache t (GQA or MLA).
  * The new K/V are written at cache_len[b]; the caller advances cache_len.
- * Outputs as rdt_recurrent_forward with N = batch. */
+ * Outputs as rdt_recurrent_forward with N = batch.
+ * CUDA graphs: the call only enqueues kernels and asynchronous copies on `stream`
+ * (no host synchronisation, no allocation), and every kernel argument is a function
+ * of this call's arguments, never of device data.  A stream capture of it therefore
+ * replays correctly while the arguments (pointers, sizes, n_loops, act_threshold)
+ * stay the same and the caller updates the pointed-to inputs and cache_len in place.
+ * The first call on a device sets kernel attributes once: make it before capturing. */
 RDT_API rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_weights* w,
                                      const float* h0, const void* e, int batch,
                                      const int32_t* cache_len, int n_loops, float act_threshold,
