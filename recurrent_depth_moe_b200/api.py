@@ -289,7 +289,9 @@ class DecodeGraph:
         if self._graph is None:
             g = torch.cuda.CUDAGraph()
             n0 = N.launch_count()
-            with torch.cuda.graph(g):
+            # thread-local capture: other threads of the process (a collective library's
+            # watchdog, for one) keep calling CUDA while this thread captures
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
                 self._body(self.h_in, self.e_in)
             self.graph_launches = N.launch_count() - n0
             self._graph = g
@@ -549,7 +551,9 @@ class Generator:
         if self._graph is None:
             g = torch.cuda.CUDAGraph()
             n0 = N.launch_count()
-            with torch.cuda.graph(g):
+            # thread-local capture: other threads of the process (a collective library's
+            # watchdog, for one) keep calling CUDA while this thread captures
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
                 self._decode_body(self.cur_tok, self.cur_tok)
             self.graph_launches = N.launch_count() - n0
             self._graph = g
