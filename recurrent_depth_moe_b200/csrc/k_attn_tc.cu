@@ -53,6 +53,7 @@ struct Args {
   bf16* o;
   long long o_row;         // output row stride (elements); head h at column h * 128
   int q_col0, k_col0;      // qkv columns of query head 0 and key head 0
+  DevStatus* st;           // device status word: a wait that gave up is recorded here
 };
 
 using namespace rdt::tc;
@@ -399,6 +400,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) record_status(a.st, ST_TIMEOUT, 601, blockIdx.x);
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
@@ -437,7 +439,7 @@ int launch_attention_tc(const AttnParams& p, cudaStream_t s) {
   a.q_pos = p.q_pos; a.key_pos0 = p.key_pos0; a.n_keys = p.n_keys;
   a.sl2 = p.scale * 1.4426950408889634f;
   a.o = (bf16*)p.o; a.o_row = p.o_row;
-  a.q_col0 = 0; a.k_col0 = (int)k_col0;
+  a.q_col0 = 0; a.k_col0 = (int)k_col0; a.st = p.st;
   const int n_qt = (p.T + fat::BQ - 1) / fat::BQ;
   const long long blocks = (long long)((n_qt + fat::NQ - 1) / fat::NQ) * p.B * p.H;
   if (blocks <= 0) return 0;

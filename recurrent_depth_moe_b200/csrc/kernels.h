@@ -89,6 +89,7 @@ struct AttnParams {
   float* part_o; float* part_ml; int n_split;
   // tensor-core prefill: values transposed, vt[((b * Hkv + g) * dv + d) * vt_ld + j]
   const void* vt; long long vt_ld;
+  DevStatus* st;                                        // device status word (timeouts); may be null
 };
 int launch_attention(int dtype, const AttnParams& p, cudaStream_t s);
 int launch_attention_decode(int dtype, const AttnParams& p, cudaStream_t s);

@@ -187,7 +187,7 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
   void* attn = at<void*>(x.ws, x.L.attn);
   AttnParams ap;
   memset(&ap, 0, sizeof(ap));
-  ap.B = B; ap.T = T; ap.H = H; ap.q_pos = pos;
+  ap.B = B; ap.T = T; ap.H = H; ap.q_pos = pos; ap.st = x.st;
   int dv;
   bool absorbed = false;   // MLA decode ran in the absorbed form (attention output written)
   if (c->attn_type == 0) {
