@@ -138,7 +138,14 @@ typedef struct {
 } rdt_trace;
 
 enum {
-  RDT_FLAG_TRANSFORMER_OFF = 1   /* debug: Transformer(h, e) term = 0 (pure LTI)      */
+  RDT_FLAG_TRANSFORMER_OFF = 1,  /* debug: Transformer(h, e) term = 0 (pure LTI)      */
+  /* test only (no counterpart on the pages): the call runs one tensor-core GEMM (the
+   * first attention projection of loop 0) whose TMA producer issues no loads, then
+   * returns without launching anything else; outputs are not written.  The GEMM's bounded
+   * waits run out (about 2 s), it frees its TMEM with nothing in flight, and the device
+   * status word reads RDT_ERR_DEVICE_TIMEOUT.  Needs bf16 and a tensor-core shape, else
+   * RDT_ERR_UNSUPPORTED.  Exercises the timeout path without faulting the context. */
+  RDT_FLAG_TEST_GEMM_TIMEOUT = 2
 };
 
 /* Bytes of workspace needed by rdt_recurrent_forward / rdt_recurrent_decode_step /
@@ -184,6 +191,16 @@ RDT_API rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_we
                                      const rdt_kv_cache* cache,
                                      void* ws, size_t ws_bytes, void* stream);
 
+/* rdt_recurrent_decode_step with a per-loop trace of a row range (tests: the router
+ * input f and biased logits per loop, for teacher-forced checks of the decode step's
+ * routes).  trace may be NULL, which makes it rdt_recurrent_decode_step. */
+RDT_API rdt_status rdt_recurrent_decode_step_traced(const rdt_config* cfg, const rdt_weights* w,
+                                            const float* h0, const void* e, int batch,
+                                            const int32_t* cache_len, int n_loops, float act_threshold,
+                                            float* h_out, float* halt_weights, int32_t* expert_ids,
+                                            const rdt_kv_cache* cache, const rdt_trace* trace,
+                                            void* ws, size_t ws_bytes, void* stream);
+
 /* Decode step without a caller workspace, for callers that cannot allocate device
  * memory (a warm serving loop that must not allocate, a host runtime without a CUDA
  * allocator of its own, a memory-pool budget with no room for a per-call workspace).
@@ -201,13 +218,20 @@ RDT_API rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_we
  *    any stream capture.
  *  - All calls share the one array: calls that overlap on the GPU (different streams,
  *    or other host threads) race and corrupt each other.  Each call initialises every
- *    part of the array it reads, so leftover contents of earlier calls do not matter. */
+ *    part of the array it reads, so leftover contents of earlier calls do not matter.
+ *  - The device status word lives in the array: read it with rdt_read_static_status.
+ *  - The array's address is cached per device: not usable across a cudaDeviceReset. */
 #define RDT_STATIC_SCRATCH_BYTES (32u << 20)
 RDT_API rdt_status rdt_recurrent_decode_step_static(const rdt_config* cfg, const rdt_weights* w,
                                                     const float* h0, const void* e, int batch,
                                                     const int32_t* cache_len, int n_loops, float act_threshold,
                                                     float* h_out, float* halt_weights, int32_t* expert_ids,
                                                     const rdt_kv_cache* cache, void* stream);
+
+/* Synchronise `stream`, then read and clear the device status word of the static
+ * scratch used by rdt_recurrent_decode_step_static on the current device (as
+ * rdt_read_device_status does for a caller workspace).  Allocates nothing. */
+RDT_API rdt_status rdt_read_static_status(void* stream);
 
 /* One pre-norm TransformerBlock: x_out = x1 + FFN(RMSNorm(x1)), x1 = x_in + Attn(RMSNorm(x_in)).
  * FFN is the MoE when cfg->n_experts > 0, else the dense SwiGLU in w13/w2 expert 0

@@ -16,6 +16,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "wo
 RDT_OK, RDT_ERR_INVALID_ARG, RDT_ERR_UNSUPPORTED, RDT_ERR_WORKSPACE, RDT_ERR_CUDA, RDT_ERR_DEVICE_TIMEOUT, \
     RDT_ERR_DEVICE_BOUNDS = range(7)
 RDT_FLAG_TRANSFORMER_OFF = 1
+RDT_FLAG_TEST_GEMM_TIMEOUT = 2
 
 
 class RdtError(RuntimeError):
@@ -57,7 +58,8 @@ class rdt_kernel_time(ctypes.Structure):
 EXPORTS = ("rdt_workspace_size", "rdt_recurrent_forward", "rdt_recurrent_decode_step", "rdt_block_forward",
            "rdt_block_forward_cached", "rdt_embed", "rdt_head", "rdt_head_rows", "rdt_greedy_tokens",
            "rdt_to_model_dtype", "rdt_read_device_status", "rdt_status_string", "rdt_version",
-           "rdt_launch_count", "rdt_profile_start", "rdt_profile_stop")
+           "rdt_launch_count", "rdt_profile_start", "rdt_profile_stop", "rdt_recurrent_decode_step_static",
+           "rdt_read_static_status", "rdt_recurrent_decode_step_traced")
 
 _lib = None
 _profiling = False
@@ -81,6 +83,10 @@ def load(path: str = LIB_PATH):
     lib.rdt_recurrent_decode_step.argtypes = [POINTER(rdt_config), POINTER(rdt_weights), P, P, c_int, P, c_int,
                                               c_float, P, P, P, POINTER(rdt_kv_cache), P, c_size_t, P]
     lib.rdt_recurrent_decode_step.restype = c_int
+    lib.rdt_recurrent_decode_step_traced.argtypes = [POINTER(rdt_config), POINTER(rdt_weights), P, P, c_int, P,
+                                                     c_int, c_float, P, P, P, POINTER(rdt_kv_cache),
+                                                     POINTER(rdt_trace), P, c_size_t, P]
+    lib.rdt_recurrent_decode_step_traced.restype = c_int
     lib.rdt_block_forward.argtypes = [POINTER(rdt_config), POINTER(rdt_weights), P, P, c_int, c_int, c_int, P,
                                       c_size_t, P]
     lib.rdt_block_forward.restype = c_int

@@ -222,8 +222,9 @@ class RecurrentBlock:
 
     def decode_step(self, h0: torch.Tensor, e: torch.Tensor, cache_len: torch.Tensor, cache: KVCache,
                     n_loops: int, act_threshold: float = 0.0, out: Optional[tuple] = None,
-                    workspace: Optional[torch.Tensor] = None):
-        """rdt_recurrent_decode_step: one new token per sequence at position cache_len[b]."""
+                    workspace: Optional[torch.Tensor] = None, trace: Optional[Trace] = None):
+        """rdt_recurrent_decode_step: one new token per sequence at position cache_len[b]
+        (rdt_recurrent_decode_step_traced when a trace is given)."""
         lib = N.load()
         cfg = self.cfg
         B = h0.shape[0]
@@ -236,6 +237,15 @@ class RecurrentBlock:
                    torch.empty(n_loops, B, cfg.n_experts_per_tok, dtype=torch.int32, device=h0.device))
         ws = workspace if workspace is not None else self.workspace(B, 1, cache.t_max)
         cs = cache.struct()
+        if trace is not None:
+            ts = trace.struct()
+            rc = lib.rdt_recurrent_decode_step_traced(ctypes.byref(self.cs), ctypes.byref(self.w.struct),
+                                                      h0.data_ptr(), e.data_ptr(), B, cache_len.data_ptr(), n_loops,
+                                                      float(act_threshold), out[0].data_ptr(), out[1].data_ptr(),
+                                                      out[2].data_ptr(), ctypes.byref(cs), ctypes.byref(ts),
+                                                      ws.data_ptr(), ws.numel(), _stream())
+            N.check("rdt_recurrent_decode_step_traced", rc)
+            return out
         rc = lib.rdt_recurrent_decode_step(ctypes.byref(self.cs), ctypes.byref(self.w.struct), h0.data_ptr(),
                                            e.data_ptr(), B, cache_len.data_ptr(), n_loops, float(act_threshold),
                                            out[0].data_ptr(), out[1].data_ptr(), out[2].data_ptr(),

@@ -340,12 +340,7 @@ int launch_attention_decode(int dtype, const AttnParams& p, cudaStream_t s) {
     const int ctas = p.B * (p.H / G) * n_split;
 #define RDT_DECM(GG)                                                                              \
   case GG: {                                                                                      \
-    static bool attr = false;                                                                     \
-    if (!attr) {                                                                                  \
-      if (cudaFuncSetAttribute(k_attn_decode_mma<GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                               dmma::SMEM) != cudaSuccess) return -1;                             \
-      attr = true;                                                                                \
-    }                                                                                             \
+    if (!ensure_smem_limit((const void*)k_attn_decode_mma<GG>, dmma::SMEM)) return -1;            \
     { k_attn_decode_mma<GG><<<ctas, 128, dmma::SMEM, s>>>(p, n_split, chunk); note_launch(); }   \
   } break;
     switch (G) { RDT_DECM(1) RDT_DECM(2) RDT_DECM(3) RDT_DECM(4) RDT_DECM(6) RDT_DECM(8) default: return -1; }

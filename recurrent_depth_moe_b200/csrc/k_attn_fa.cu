@@ -245,12 +245,7 @@ bool attention_fa_supports(int dtype, const AttnParams& p) {
 }
 
 int launch_attention_fa(const AttnParams& p, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(fa::k_attn_fa, cudaFuncAttributeMaxDynamicSharedMemorySize, fa::SMEM_BYTES) != cudaSuccess)
-      return -1;
-    attr = true;
-  }
+  if (!ensure_smem_limit((const void*)fa::k_attn_fa, fa::SMEM_BYTES)) return -1;
   const long long blocks = (long long)((p.T + fa::BQ - 1) / fa::BQ) * p.B * p.H;
   if (blocks <= 0) return 0;
   { fa::k_attn_fa<<<(unsigned)blocks, 128, fa::SMEM_BYTES, s>>>(p); note_launch(); }

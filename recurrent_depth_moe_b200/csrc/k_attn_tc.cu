@@ -238,6 +238,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     const int kx = a.k_col0 + g * HD;
     const int vy = (b * a.Hkv + g) * HD;
+    int k_phase[KSTAGES], v_phase[VSTAGES];   // phase of the last load issued into each stage (-1: none)
+#pragma unroll
+    for (int s = 0; s < KSTAGES; ++s) k_phase[s] = -1;
+#pragma unroll
+    for (int s = 0; s < VSTAGES; ++s) v_phase[s] = -1;
     for (int j = 0; j < nt_max; ++j) {
       const int ks = j % KSTAGES, vs = j % VSTAGES;
       if (!mbar_wait(&k_empty[ks], ((j / KSTAGES) & 1) ^ 1, abort_flag)) break;
@@ -245,11 +250,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int ky = b * a.T + j * BKV;
       tma_load_2d(sK + ks * KTILE, &tmK, &k_full[ks], kx, ky);
       tma_load_2d(sK + ks * KTILE + KHALF, &tmK, &k_full[ks], kx + 64, ky);
+      k_phase[ks] = (j / KSTAGES) & 1;
       if (!mbar_wait(&v_empty[vs], ((j / VSTAGES) & 1) ^ 1, abort_flag)) break;
       mbar_expect_tx(&v_full[vs], VTILE);
       tma_load_2d(sV + vs * VTILE, &tmVt, &v_full[vs], j * BKV, vy);
       tma_load_2d(sV + vs * VTILE + VHALF, &tmVt, &v_full[vs], j * BKV + 64, vy);
+      v_phase[vs] = (j / VSTAGES) & 1;
     }
+    // copies still in flight (an abort) land before the CTA's shared memory is released
+    if (qbytes > 0) mbar_drain(q_full, 0);
+#pragma unroll
+    for (int s = 0; s < KSTAGES; ++s)
+      if (k_phase[s] >= 0) mbar_drain(&k_full[s], (uint32_t)k_phase[s]);
+#pragma unroll
+    for (int s = 0; s < VSTAGES; ++s)
+      if (v_phase[s] >= 0) mbar_drain(&v_full[s], (uint32_t)v_phase[s]);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
     constexpr uint32_t IDESC_S = idesc_bf16(128, BKV);
@@ -295,8 +310,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (load) umma_commit(&k_empty[ks]);     // K of tile j is consumed once both S MMAs finish
       if (j >= 1) umma_commit(&v_empty[pvs]);  // V of tile j - 1 once both PV MMAs finish
     }
+    // all issued MMAs complete before TMEM is released (also after an abort)
     umma_commit(done);
-    mbar_wait(done, 0, abort_flag);
+    mbar_drain(done, 0);
   } else if (warp >= 2) {
     // ---------------- softmax of query tile q ----------------
     const int q = (warp - 2) >> 2;
@@ -419,12 +435,7 @@ bool attention_tc_supports(int dtype, const AttnParams& p) {
 }
 
 int launch_attention_tc(const AttnParams& p, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(fat::k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, fat::SMEM) != cudaSuccess)
-      return -1;
-    attr = true;
-  }
+  if (!ensure_smem_limit((const void*)fat::k_attn_tc, fat::SMEM)) return -1;
   const int Hkv = p.H / p.G;
   // Q and K live in the qkv rows [B*T, q_row]; k1 points at key head 0 inside those rows
   const long long k_col0 = ((const bf16*)p.k1 - (const bf16*)p.q);

@@ -381,16 +381,7 @@ bool launch_rmsnorm_warp(int dtype, const float* x, const float* w, void* out, i
 #undef RDT_RW
 }
 
-int combine_sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
+int combine_sm_count() { return device_sm_count(); }
 
 template <typename T, int VPL>
 bool launch_combine_vpl(const CombineParams& p, int n_rows, cudaStream_t s) {
@@ -413,13 +404,7 @@ bool launch_combine_vpl(const CombineParams& p, int n_rows, cudaStream_t s) {
   const int grid = std::max(1, std::min((n_rows + GROUPS - 1) / GROUPS, sms));
   constexpr int THREADS = GROUPS * WPR * 32;
   if (lsmem) {
-    static bool attr = false;
-    if (!attr) {
-      if (cudaFuncSetAttribute(k_combine_warp<T, VPL, WPR, GROUPS, true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024) != cudaSuccess)
-        return false;
-      attr = true;
-    }
+    if (!ensure_smem_limit((const void*)k_combine_warp<T, VPL, WPR, GROUPS, true>, 160 * 1024)) return false;
     { k_combine_warp<T, VPL, WPR, GROUPS, true><<<grid, THREADS, lbytes, s>>>(p); note_launch(); }
   } else {
     { k_combine_warp<T, VPL, WPR, GROUPS, false><<<grid, THREADS, 0, s>>>(p); note_launch(); }
@@ -428,7 +413,8 @@ bool launch_combine_vpl(const CombineParams& p, int n_rows, cudaStream_t s) {
 }
 
 bool launch_combine_warp(int dtype, const CombineParams& p, int n_rows, cudaStream_t s) {
-  if (p.D % 128 || p.r > 64 || p.k > 32) return false;
+  // one slot index per lane (combine_row): rows with more than 32 slots take the CTA-per-row kernel
+  if (p.D % 128 || p.r > 64 || p.k + p.S > 32) return false;
   const int ev = dtype == 0 ? 16 : 8;   // bytes of a 4-element vector in the model dtype
   if (!al(p.x1, 16) || !al(p.y, ev) || !al(p.h, 16) || !al(p.h_state, 16) || !al(p.h_out, 16) || !al(p.A, 16) ||
       !al(p.inj_B, 16) || !al(p.e, ev) || (p.act_on && !al(p.halt_wv, 16)) || (p.out && !al(p.out, 16)) ||

@@ -215,7 +215,12 @@ __global__ void __launch_bounds__(192, 1)
     // ---------------- TMA producer ----------------
     int stage = 0;
     uint32_t phase = 0;
-    for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+    int issued_phase[STAGES];   // phase of the last load issued into each stage (-1: none)
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s) issued_phase[s] = -1;
+    // test hook: a producer that issues nothing starves every consumer wait
+    const int n_prod = p.test_no_loads ? 0 : total;
+    for (int t = blockIdx.x; t < n_prod && !*abort_flag; t += gridDim.x) {
       const TileInfo ti = decode_tile(args, t);
       const int gb = ti.group * args.b_rows_group;
       int b0, b1;
@@ -235,9 +240,14 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_2d(sa, &tmA, &full[stage], ks * BK, ti.row0);
         tma_load_2d(sa + A_BYTES, &tmB, &full[stage], ks * BK, b0);
         if (BN > 128) tma_load_2d(sa + A_BYTES + S::B_BOX * BK * 2, &tmB, &full[stage], ks * BK, b1);
+        issued_phase[stage] = (int)phase;
         if (++stage == STAGES) { stage = 0; phase ^= 1; }
       }
     }
+    // copies still in flight (an abort) land before the CTA's shared memory is released
+#pragma unroll
+    for (int s = 0; s < STAGES; ++s)
+      if (issued_phase[s] >= 0) mbar_drain(&full[s], (uint32_t)issued_phase[s]);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
     constexpr uint32_t IDESC = idesc_bf16(BM, BN);
@@ -267,9 +277,9 @@ __global__ void __launch_bounds__(192, 1)
       umma_commit(&tfull[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
-    // all issued MMAs complete before TMEM is released
+    // all issued MMAs complete before TMEM is released (also after an abort)
     umma_commit(done);
-    mbar_wait(done, 0, abort_flag);
+    mbar_drain(done, 0);
   } else if (warp >= 2) {
     // ---------------- epilogue ----------------
     const int quarter = warp & 3;
@@ -431,16 +441,7 @@ bool make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsigne
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
+int sm_count() { return device_sm_count(); }
 
 inline bool al16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 }  // namespace
@@ -467,13 +468,7 @@ int pick_bn(const GemmParams& p, int epi) {
 
 template <int EPI, int BN>
 int launch_tc(const CUtensorMap& mA, const CUtensorMap& mB, const tc::TcArgs& a, int grid, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(tc::k_gemm_tc<EPI, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc::Shape<BN>::SMEM_BYTES) != cudaSuccess)
-      return -1;
-    attr = true;
-  }
+  if (!ensure_smem_limit((const void*)tc::k_gemm_tc<EPI, BN>, tc::Shape<BN>::SMEM_BYTES)) return -1;
   { tc::k_gemm_tc<EPI, BN><<<grid, 192, tc::Shape<BN>::SMEM_BYTES, s>>>(mA, mB, a); note_launch(); }
   return 0;
 }

@@ -485,12 +485,7 @@ namespace {
 template <int MT, int KVR, int DR>
 int launch_attn_t(const MlaDecodeParams& p, int chunk_tiles, cudaStream_t s) {
   constexpr int SMEM = mla::Shape<MT, KVR, DR>::SMEM;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(k_mla_attn<MT, KVR, DR>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
-      return -1;
-    attr = true;
-  }
+  if (!ensure_smem_limit((const void*)k_mla_attn<MT, KVR, DR>, SMEM)) return -1;
   k_mla_attn<MT, KVR, DR><<<(unsigned)(p.B * p.n_split), mla::THREADS, SMEM, s>>>(p, chunk_tiles);
   note_launch();
   return 0;

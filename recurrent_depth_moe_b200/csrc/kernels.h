@@ -7,6 +7,12 @@ namespace rdt {
 
 struct DevStatus;
 
+// Raise `kernel`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// (kernel, device); thread-safe.  Returns false if the CUDA call fails.
+bool ensure_smem_limit(const void* kernel, int bytes);
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
+
 // Kernel classes for event timing (ProfScope records a CUDA event pair around the
 // launches in its scope on the given stream when profiling is on).
 enum ProfClass {
@@ -60,6 +66,9 @@ struct GemmParams {
   // split-K scratch for rows that fit one tile (decode): fp32 partials [splits][M][N];
   // nullptr = no split
   float* split_ws; long long split_ws_elems;
+  // test only: the tensor-core producer issues no loads, so the kernel's bounded waits run
+  // out and it records a timeout (nothing is ever in flight); 0 in production
+  int test_no_loads;
   DevStatus* st;
 };
 

@@ -468,6 +468,20 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
   cp.transformer_off = transformer_off;
   cp.loop_dim = c->loop_dim; cp.w_rec = w->rec_norm_w; cp.w_attn = w->attn_norm_w; cp.eps = c->norm_eps;
   cp.combined_out = combined; cp.a_out = a;
+  if (flags & RDT_FLAG_TEST_GEMM_TIMEOUT) {
+    // the first projection of loop 0 with an idle producer; nothing reads its output
+    GemmParams g = gemm_base(x);
+    g.A = a; g.lda = D; g.M = N; g.K = D; g.test_no_loads = 1;
+    if (c->attn_type == 0) {
+      const int W = (c->n_heads + 2 * c->n_kv_heads) * (D / c->n_heads);
+      g.B = w->w_qkv; g.ldb = D; g.N = W; g.C = at<void*>(ws, x.L.qkv); g.ldc = W;
+    } else {
+      g.B = w->w_q_down; g.ldb = D; g.N = c->q_lora_rank; g.C = at<void*>(ws, x.L.cq); g.ldc = c->q_lora_rank;
+    }
+    if (gemm_pick(x.dtype, g, EPI_STORE_T) != GEMM_TC) return RDT_ERR_UNSUPPORTED;
+    RDT_TRY(launch_gemm(x.dtype, EPI_STORE_T, g, s));
+    return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
+  }
   const int emb_stride = std::max(c->loop_dim, 2);
   bool prologue_done = false;   // set when the previous loop's combine kernel computed this loop's prologue
   for (int t = 0; t < n_loops; ++t) {
@@ -574,6 +588,15 @@ rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_weights* w
                                      const rdt_kv_cache* cache, void* ws, size_t ws_bytes, void* stream) {
   return run_recurrent(cfg, w, h0, e, batch, 1, 0, cache_len, n_loops, act_threshold, nullptr, h_out, halt_weights,
                        expert_ids, cache, nullptr, 0, ws, ws_bytes, (cudaStream_t)stream, true);
+}
+
+rdt_status rdt_recurrent_decode_step_traced(const rdt_config* cfg, const rdt_weights* w, const float* h0,
+                                            const void* e, int batch, const int32_t* cache_len, int n_loops,
+                                            float act_threshold, float* h_out, float* halt_weights,
+                                            int32_t* expert_ids, const rdt_kv_cache* cache, const rdt_trace* trace,
+                                            void* ws, size_t ws_bytes, void* stream) {
+  return run_recurrent(cfg, w, h0, e, batch, 1, 0, cache_len, n_loops, act_threshold, nullptr, h_out, halt_weights,
+                       expert_ids, cache, trace, 0, ws, ws_bytes, (cudaStream_t)stream, true);
 }
 
 rdt_status rdt_block_forward_cached(const rdt_config* cfg, const rdt_weights* w, const float* x_in, float* x_out,

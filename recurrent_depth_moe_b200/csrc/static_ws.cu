@@ -22,7 +22,10 @@ static __device__ __align__(256) unsigned char g_rdt_static_scratch[RDT_STATIC_S
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices];   // device address of the array, per device (set once)
+// Device address of the array, per device, resolved on the first call with that device
+// current.  A cudaDeviceReset unloads the library's module and makes the cached address
+// stale: this path is not usable across a device reset.
+void* g_scratch_ptr[kMaxDevices];
 
 // Device address of the scratch array on the current device.  In host code the array's
 // name is only a host-side stand-in, so the real address comes from
@@ -56,4 +59,14 @@ extern "C" rdt_status rdt_recurrent_decode_step_static(const rdt_config* cfg, co
   if (st != RDT_OK) return st;
   return rdt_recurrent_decode_step(cfg, w, h0, e, batch, cache_len, n_loops, act_threshold, h_out, halt_weights,
                                    expert_ids, cache, ws, (size_t)RDT_STATIC_SCRATCH_BYTES, stream);
+}
+
+// Device status word of the static-scratch decode: the kernels record bounds violations
+// and bounded waits that gave up in the first bytes of the scratch (as they do in a
+// caller's workspace), and this reads and clears it.  Synchronises `stream`.
+extern "C" rdt_status rdt_read_static_status(void* stream) {
+  void* ws = nullptr;
+  const rdt_status st = scratch_on_current_device(&ws);
+  if (st != RDT_OK) return st;
+  return rdt_read_device_status(ws, stream);
 }

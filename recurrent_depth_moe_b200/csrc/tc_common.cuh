@@ -45,6 +45,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile
   }
   return true;
 }
+// Bounded wait that ignores the abort flag: taken on the way out, so the CTA's own
+// asynchronous operations (TMA copies it issued, MMAs it committed) finish before its
+// shared memory and TMEM are released.  False only if the limit runs out.
+__device__ __forceinline__ bool mbar_drain(uint64_t* b, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(b, parity))
+    if (clock64() - t0 > TIMEOUT_CYCLES) return false;
+  return true;
+}
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(

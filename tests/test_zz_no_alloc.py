@@ -23,6 +23,8 @@ def _lib():
     fn.argtypes = [ctypes.POINTER(N.rdt_config), ctypes.POINTER(N.rdt_weights), P, P, ctypes.c_int, P, ctypes.c_int,
                    ctypes.c_float, P, P, P, ctypes.POINTER(N.rdt_kv_cache), P]
     fn.restype = ctypes.c_int
+    lib.rdt_read_static_status.argtypes = [P]
+    lib.rdt_read_static_status.restype = ctypes.c_int
     return lib, N
 
 
@@ -56,13 +58,18 @@ def test_static_scratch_decode_matches_workspace_decode(dtype):
                                                   e.data_ptr(), B, lens.data_ptr(), L, thr, out[0].data_ptr(),
                                                   out[1].data_ptr(), out[2].data_ptr(), ctypes.byref(cs), stream)
         assert rc == 0, N.STATUS.get(rc, rc)
+        # the device status word of the static scratch: no bounds violation, no timeout
+        assert lib.rdt_read_static_status(stream) == 0
+        assert blk.read_status() == 0
         torch.cuda.synchronize()
         if dtype == "fp32":
             assert max_rel(out[0], ref[0]) <= FP32_TOL
             assert max_rel(st_cache.k, ref_cache.k) <= FP32_TOL
+            assert max_rel(st_cache.v, ref_cache.v) <= FP32_TOL
         else:
             assert rel_l2(out[0], ref[0]) <= BF16_TOL
             assert rel_l2(st_cache.k.float(), ref_cache.k.float()) <= BF16_TOL
+            assert rel_l2(st_cache.v.float(), ref_cache.v.float()) <= BF16_TOL
         assert max_rel(out[1], ref[1]) <= FP32_TOL
         assert torch.equal(out[2], ref[2])
 
