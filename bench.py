@@ -3,9 +3,13 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one full recurrent-block forward (all loops, every kernel of the path) over
-one batch of the 1B-shaped prefill workload (dim 2048, 16 heads GQA with 4 kv heads,
-64 routed + 1 shared SwiGLU experts, top-4, expert_dim 2048, lora_rank 16, 16 loops,
-batch 4 x seq 4096, bf16).  Weights and inputs are seeded synthetic draws.
+one batch of the 10B-shaped load-imbalanced prefill workload (dim 4096, 32 heads GQA with
+8 kv heads, 128 routed + 1 shared SwiGLU experts, top-8, expert_dim 5632, lora_rank 16,
+24 loops, batch 2 x seq 8192, bf16, router bias giving Zipf(1.1) expert popularity,
+per-position halting spread over 4-24 loops).  The value counts executed token-loops.
+The same line carries the 1B-shaped prefill (and its literal halting-bias variant), the
+3B-shaped KV-cached decode (GQA and MLA) and the 1B-shaped greedy generation.  Weights
+and inputs are seeded synthetic draws.
 
 Multi-GPU (torchrun, one process per GPU): each rank runs an independent replica on
 its own batch (sequences shard with no exchange); the time is the max over ranks.
@@ -35,7 +39,7 @@ from recurrent_depth_moe_b200 import replicas as REP  # noqa: E402
 
 METRIC = "recurrent-block token·loops/s prefill; decode tokens/s; % roofline, 1×B200"
 UNIT = "token·loops/s"
-WORKLOAD = "rdt1b_prefill"
+WORKLOAD = "rdt10b_prefill_zipf"
 
 
 def log(*a):
@@ -116,26 +120,26 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm), "power_w_max": max(power) if power else None}
 
 
-# DRAM traffic of one full-size expert-up launch (1B shape, 16384 tokens x 5 slots), from ncu
-# dram__bytes_read.sum + dram__bytes_write.sum (1 pass; profiles/expert_up_gemm_rdt1b_small_case.md).
-# Reported only while the GEMM's sources are the ones it was captured from.
-EXPERT_UP_TRAFFIC = {"bytes": 1426189056 + 301016576, "workload": "rdt1b_prefill", "n_loops": 16,
-                     "sha256": "94721409d27298b49959cc5af1073df041ed4ea4bd4e8b9a04c45934a42826c4"}
+# DRAM traffic of one full-size expert-up launch of a workload, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum, 1 pass), valid only while the GEMM's
+# sources are the ones it was captured from (sha256 of k_gemm_tc.cu + tc_common.cuh).
+EXPERT_UP_TRAFFIC = {}
 
 
 def expert_up_traffic(wl):
     import hashlib
-    if wl.name != EXPERT_UP_TRAFFIC["workload"] or wl.batch != 4 or wl.n_loops != EXPERT_UP_TRAFFIC["n_loops"]:
+    rec = EXPERT_UP_TRAFFIC.get(wl.name)
+    if rec is None or wl.batch != rec["batch"] or wl.n_loops != rec["n_loops"]:
         return None
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "recurrent_depth_moe_b200", "csrc")
     h = hashlib.sha256()
     for f in ("k_gemm_tc.cu", "tc_common.cuh"):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
-    return EXPERT_UP_TRAFFIC["bytes"] if h.hexdigest() == EXPERT_UP_TRAFFIC["sha256"] else None
+    return rec["bytes"] if h.hexdigest() == rec["sha256"] else None
 
 
-def expert_up_flops(wl, n_running: int) -> float:
+def expert_up_flops(wl, n_running: float) -> float:
     c = wl.cfg
     rows = n_running * (c.n_experts_per_tok + c.n_shared_experts)
     return 2.0 * rows * c.dim * 2 * c.expert_dim
@@ -145,17 +149,21 @@ def expert_up_flops(wl, n_running: int) -> float:
 # CPU oracle sample (reference arm and cpu_baseline)
 # ------------------------------------------------------------------------------------------
 
-def oracle_sample(wl, W_cpu, h0, e, positions: int, loops: int):
+ORACLE_SAMPLE = {"rdt1b_prefill": (32, 4), "rdt10b_prefill_zipf": (8, 2)}   # positions, loops per sample
+
+
+def oracle_sample(wl, W_cpu, h0, e, positions: int, loops: int, halt_off=None):
     """Time the CPU oracle on sequence 0, positions [0, positions), `loops` loops.
     Causal prefix slices are exact (attention is causal, routing per token)."""
     from oracle import rdt_oracle as O
     t0 = time.perf_counter()
-    O.recurrent_forward(wl.cfg, W_cpu, h0[:positions], e[:positions], 1, loops, wl.act_threshold)
+    O.recurrent_forward(wl.cfg, W_cpu, h0[:positions], e[:positions], 1, loops, wl.act_threshold,
+                        halt_logit_offset=None if halt_off is None else halt_off[:positions])
     dt = time.perf_counter() - t0
     return positions * loops / dt, dt
 
 
-def workload_weights(wl, device):
+def workload_weights(wl, device, halt_b=None):
     """Weights of a prefill workload (Zipf router bias and halting spread where the
     workload names them) and its per-position halting-logit offsets (or None)."""
     cfg = wl.cfg
@@ -164,7 +172,7 @@ def workload_weights(wl, device):
         W = RI.block_weights(cfg, wl.seed, device=device, router_bias=bias,
                              halt_w_std=0.0 if wl.halt_spread else None, halt_b=0.0 if wl.halt_spread else wl.halt_b)
     else:
-        W = RI.block_weights(cfg, wl.seed, device=device, halt_b=wl.halt_b)
+        W = RI.block_weights(cfg, wl.seed, device=device, halt_b=wl.halt_b if halt_b is None else halt_b)
     off = None
     if wl.halt_spread:
         off, _ = RI.halting_offsets_spread(wl.batch * wl.seq, wl.halt_spread[0], wl.halt_spread[1],
@@ -174,21 +182,25 @@ def workload_weights(wl, device):
 
 
 def run_reference(args, wl, rank, world):
+    """The oracle as it stands, on the host cores, on a bounded causal-prefix sample of the
+    workload per step.  Large workloads draw their weights with the device generator (as
+    the GPU arm does, so both see the same numbers) and copy them to the host once."""
     if rank != 0:
         return
     torch.manual_seed(0)
-    W, _ = workload_weights(wl, "cpu") if wl.cfg.n_experts <= 64 else (None, None)
-    if W is None:   # the 10B shape's expert weights (18 GB) do not fit a host sample
-        print(json.dumps({"impl": "reference", "unavailable": "10B-shaped weights exceed the host sample budget"}))
-        return
-    h0, e = RI.recurrent_inputs(wl.cfg, 1, 64, wl.seed)
-    pos, loops = 32, 4
+    dev = "cuda" if (wl.device_weights and torch.cuda.is_available()) else "cpu"
+    W, off = workload_weights(wl, dev)
+    W = {k: v.cpu() for k, v in W.items()}
+    off = None if off is None else off.cpu()
+    if dev == "cuda":
+        torch.cuda.empty_cache()
+    pos, loops = ORACLE_SAMPLE.get(wl.name, (32, 4))
+    h0, e = RI.recurrent_inputs(wl.cfg, 1, pos, wl.seed)
     for _ in range(args.warmup):
-        oracle_sample(wl, W, h0, e, pos, 1)
-    rates, total = [], 0.0
+        oracle_sample(wl, W, h0, e, pos, 1, off)
+    total = 0.0
     for _ in range(args.steps):
-        r, dt = oracle_sample(wl, W, h0, e, pos, loops)
-        rates.append(r)
+        _, dt = oracle_sample(wl, W, h0, e, pos, loops, off)
         total += dt
     value = args.steps * pos * loops / total
     cores = torch.get_num_threads()
@@ -206,7 +218,10 @@ def run_reference(args, wl, rank, world):
 # our arm
 # ------------------------------------------------------------------------------------------
 
-def run_ours(args, wl, rank, world, local_rank):
+def run_prefill(args, wl, rank, world, local_rank, *, steps=None, e2e=True, cpu_baseline=False, halt_b=None):
+    """Time `steps` recurrent-block forwards of a prefill workload (inputs resident in HBM),
+    with the per-class event profile inside the timed region; optionally the same through
+    the public API with host buffers (e2e) and the CPU oracle on a bounded sample."""
     import recurrent_depth_moe_b200 as R
     from recurrent_depth_moe_b200 import _native as NAT
     dev = torch.device("cuda", local_rank)
@@ -214,8 +229,9 @@ def run_ours(args, wl, rank, world, local_rank):
     cfg = wl.cfg
     B, T, L = wl.batch, wl.seq, wl.n_loops
     N = B * T
+    steps = steps or args.steps
     # weights: identical replica on every rank; inputs: a different batch per rank
-    W, halt_off = workload_weights(wl, dev)
+    W, halt_off = workload_weights(wl, dev, halt_b)
     h0, e = RI.recurrent_inputs(cfg, B, T, REP.replica_input_seed(wl.seed, rank), device=dev)
     blk = R.RecurrentBlock(cfg, W)
     ws = blk.workspace(B, T, T)
@@ -244,7 +260,7 @@ def run_ours(args, wl, rank, world, local_rank):
     torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
-    for _ in range(args.steps):
+    for _ in range(steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
@@ -253,7 +269,8 @@ def run_ours(args, wl, rank, world, local_rank):
     launches = NAT.launch_count() - n0
     prof = NAT.profile_stop()
     clk = clocks.stop()
-    ms = ev0.elapsed_time(ev1) / args.steps
+    assert blk.read_status() == 0, "device status word set during the timed steps"
+    ms = ev0.elapsed_time(ev1) / steps
     ms_max = REP.max_over_ranks(ms, device=dev)
 
     # executed token-loops of one step (positions that halt early run fewer loops)
@@ -262,90 +279,134 @@ def run_ours(args, wl, rank, world, local_rank):
     executed = float((last + 1).sum().item())
     executed_all = REP.sum_over_ranks(executed, device=dev)
     value = executed_all / (ms_max / 1e3)
+    ids = out[2][0].cpu()
+    load = torch.bincount(ids[ids >= 0].flatten().long(), minlength=cfg.n_experts).double()
 
-    # end to end through the public API: pinned host inputs -> device -> forward -> host outputs
-    h0_h = h0.cpu().pin_memory()
-    e_h = e.cpu().pin_memory()
-    h0_d, e_d = torch.empty_like(h0), torch.empty_like(e)
-    outs_h = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in out]
-    h2d = h0_h.numel() * h0_h.element_size() + e_h.numel() * e_h.element_size()
-    d2h = sum(o.numel() * o.element_size() for o in out)
+    res = {"value": value, "ms_per_step": ms_max, "steps": steps, "executed_token_loops_per_step": executed_all,
+           "mean_loops": executed / N, "gpu_launches": launches, "clocks": clk,
+           "expert_load_max_over_mean_loop0": float(load.max() / load.mean()),
+           "kernel_ms_per_step": {k: {"launches": v[0], "ms_per_step": v[1] / steps} for k, v in sorted(prof.items())}}
+    if e2e:
+        # end to end through the public API: pinned host inputs -> device -> forward -> host outputs
+        h0_h = h0.cpu().pin_memory()
+        e_h = e.cpu().pin_memory()
+        h0_d, e_d = torch.empty_like(h0), torch.empty_like(e)
+        outs_h = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in out]
+        h2d = h0_h.numel() * h0_h.element_size() + e_h.numel() * e_h.element_size()
+        d2h = sum(o.numel() * o.element_size() for o in out)
 
-    def e2e_step():
-        h0_d.copy_(h0_h, non_blocking=True)
-        e_d.copy_(e_h, non_blocking=True)
-        blk.forward(h0_d, e_d, B, T, L, wl.act_threshold, halt_logit_offset=halt_off, out=out, workspace=ws)
-        for oh, od in zip(outs_h, out):
-            oh.copy_(od, non_blocking=True)
+        def e2e_step():
+            h0_d.copy_(h0_h, non_blocking=True)
+            e_d.copy_(e_h, non_blocking=True)
+            blk.forward(h0_d, e_d, B, T, L, wl.act_threshold, halt_logit_offset=halt_off, out=out, workspace=ws)
+            for oh, od in zip(outs_h, out):
+                oh.copy_(od, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = REP.max_over_ranks(e0.elapsed_time(e1) / args.steps, device=dev)
-    e2e_value = executed_all / (e2e_ms / 1e3)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = REP.max_over_ranks(e0.elapsed_time(e1) / steps, device=dev)
+        res["e2e"] = {"value": executed_all / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h}
+        del h0_d, e_d, outs_h
 
-    # host copy for the CPU-oracle baseline, then free the prefill workload before the
-    # decode one (23 GB of weights and caches)
-    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and cfg.n_experts <= 64
-    W_cpu = {k: v.cpu() for k, v in W.items()} if want_cpu else None
-    h0_c, e_c = h0[:64].cpu(), e[:64].cpu()
-    del blk, ws, W, out, h0_d, e_d
+    pk, pk_kind = peaks()
+    up = prof.get("expert_up_swiglu", (0, 0.0))
+    achieved = None
+    mean_running = executed / L        # rows routed per launch, averaged over the loops
+    if up[0]:
+        achieved = expert_up_flops(wl, mean_running) / (up[1] / up[0] / 1e3) / 1e12
+    peak_t = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    res["roofline"] = {"bound": "tensor", "kernel": "expert_up_swiglu (tcgen05 grouped GEMM, SwiGLU epilogue)",
+                       "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
+                       "frac": (achieved / peak_t) if achieved else None,
+                       "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)",
+                       "traffic": expert_up_traffic(wl), "flops_per_launch": expert_up_flops(wl, mean_running)}
+    # host copy for the CPU-oracle baseline, then the GPU workload is freed
+    W_cpu = None
+    if cpu_baseline and rank == 0 and world == 1:
+        W_cpu = {k: v.cpu() for k, v in W.items()}
+        pos, loops = ORACLE_SAMPLE.get(wl.name, (32, 4))
+        h0_c, e_c = h0[:pos].cpu(), e[:pos].cpu()
+        off_c = None if halt_off is None else halt_off[:pos].cpu()
+    del blk, ws, W, out, h0, e
     torch.cuda.empty_cache()
+    if W_cpu is not None:
+        rate, dt = oracle_sample(wl, W_cpu, h0_c, e_c, pos, loops, off_c)
+        res["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
+                               "sample": f"sequence 0, positions 0-{pos - 1}, loops 0-{loops - 1} of {wl.name} "
+                                         f"(fp64 oracle, {dt:.1f} s)"}
+        del W_cpu
+    return res
+
+
+def run_ours(args, wl, rank, world, local_rank):
+    """The headline line: the largest single-GPU prefill workload (the 10B-shaped
+    load-imbalanced prefill) at the top level; the 1B-shaped prefill (with its literal
+    halting-bias variant), the 3B-shaped decode (GQA and MLA) and the 1B-shaped generation
+    alongside, with their headline figures also as flat top-level keys."""
+    head = run_prefill(args, wl, rank, world, local_rank, e2e=True, cpu_baseline=not args.no_cpu_baseline)
+    side = literal = None
+    if not args.no_secondary and wl.name != "rdt1b_prefill":
+        wl1 = RI.get_workload("rdt1b_prefill")
+        side = run_prefill(args, wl1, rank, world, local_rank, e2e=False)
+        # the literal reading of the 1B config: halting bias 0, so positions halt after 2-3 loops
+        literal = run_prefill(args, wl1, rank, world, local_rank, steps=min(args.steps, 5), e2e=False, halt_b=0.0)
     decode_res = None if args.no_decode else run_decode(args, rank, world, local_rank)
     mla_res = None if args.no_decode or args.no_mla_decode else run_decode(args, rank, world, local_rank,
                                                                              "rdt3b_mla_decode")
     gen_res = None if args.no_decode or args.no_generate else run_generate(args, rank, world, local_rank)
-
     if rank != 0:
         return
-    pk, pk_kind = peaks()
-    up = prof.get("expert_up_swiglu", (0, 0.0))
-    n_running = N  # per loop; all rows run when nothing halts early
-    achieved_tflops = None
-    if up[0]:
-        avg_ms = up[1] / up[0]
-        # rows actually routed per launch: executed token-loops / loops = mean running rows
-        mean_running = executed / L
-        achieved_tflops = expert_up_flops(wl, mean_running) / (avg_ms / 1e3) / 1e12
-    peak_t = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
-    roofline = {"bound": "tensor", "kernel": "expert_up_swiglu (tcgen05 grouped GEMM, SwiGLU epilogue)",
-                "achieved": achieved_tflops, "peak": peak_t, "unit": "TFLOP/s",
-                "frac": (achieved_tflops / peak_t) if achieved_tflops else None,
-                "peak_kind": f"{pk_kind} bf16 sustained (kernel timed inside a long step)",
-                "traffic": expert_up_traffic(wl),
-                "flops_per_launch": expert_up_flops(wl, executed / L)}
-    breakdown = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps} for k, v in sorted(prof.items())}
-    res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+    cfg = wl.cfg
+    res = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
            "vs_baseline": None, "dtype": "bf16",
            "data": "synthetic (seeded N(0,0.02) weights, unit-RMS h0/e rows)",
-           "config": {"workload": workload_desc(wl), "batch": B * world, "seq_len": T, "n_loops": L,
+           "config": {"workload": workload_desc(wl), "batch": wl.batch * world, "seq_len": wl.seq,
+                      "n_loops": wl.n_loops,
                       "parallelism": f"replicas x{world} (sequence-sharded, no collective)",
                       "l2": f"inputs larger than L2 ({3 * cfg.dim * cfg.expert_dim * (cfg.n_experts + cfg.n_shared_experts) * 2 / 1e9:.2f} GB of expert weights streamed per loop)"},
-           "executed_token_loops_per_step": executed_all,
-           "roofline": roofline, "gpu_launches": launches,
-           "kernel_ms_per_step": breakdown,
-           "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-           "clocks": clk}
-    if not args.no_decode:
+           "executed_token_loops_per_step": head["executed_token_loops_per_step"],
+           "mean_loops_per_position": head["mean_loops"],
+           "expert_load_max_over_mean_loop0": head["expert_load_max_over_mean_loop0"],
+           "roofline": head["roofline"], "expert_up_frac": head["roofline"]["frac"],
+           "gpu_launches": head["gpu_launches"], "kernel_ms_per_step": head["kernel_ms_per_step"],
+           "e2e": head["e2e"], "clocks": head["clocks"]}
+    if "cpu_baseline" in head:
+        res["cpu_baseline"] = head["cpu_baseline"]
+    if side is not None:
+        res["rdt1b_prefill"] = {"workload": workload_desc(RI.get_workload("rdt1b_prefill")), **side}
+        res["rdt1b_prefill_token_loops_per_s"] = side["value"]
+        res["rdt1b_prefill_ms_per_step"] = side["ms_per_step"]
+        res["rdt1b_expert_up_frac"] = side["roofline"]["frac"]
+    if literal is not None:
+        res["rdt1b_prefill_literal_halt_b0"] = {
+            "workload": "rdt1b_prefill with halting bias 0 (the config's literal reading: N(0, 0.02) halting "
+                        "weights, positions halt after 2-3 of the 16 loops)", **literal}
+        res["rdt1b_literal_token_loops_per_s"] = literal["value"]
+        res["rdt1b_literal_mean_loops"] = literal["mean_loops"]
+    if decode_res is not None:
         res["decode"] = decode_res
-        if mla_res is not None:
-            res["decode_mla"] = mla_res
-        if gen_res is not None:
-            res["generate"] = gen_res
-    if W_cpu is not None:
-        pos, loops = 64, 8
-        rate, dt = oracle_sample(wl, W_cpu, h0_c, e_c, pos, loops)
-        res["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": torch.get_num_threads(), "kind": "oracle",
-                               "sample": f"sequence 0, positions 0-{pos - 1}, loops 0-{loops - 1} "
-                                         f"(fp64 oracle, {dt:.1f} s)"}
+        res["decode_tokens_per_s"] = decode_res["value"]
+        res["decode_hbm_frac"] = decode_res["roofline"]["frac"]
+        res["decode_attention_hbm_frac"] = decode_res["attention_roofline"]["frac"]
+    if mla_res is not None:
+        res["decode_mla"] = mla_res
+        res["decode_mla_tokens_per_s"] = mla_res["value"]
+        res["decode_mla_hbm_frac"] = mla_res["roofline"]["frac"]
+        res["decode_mla_attention_hbm_frac"] = mla_res["attention_roofline"]["frac"]
+    if gen_res is not None:
+        res["generate"] = gen_res
+        res["generate_tokens_per_s"] = gen_res["value"]
+        res["generate_decode_hbm_frac"] = gen_res["decode_roofline"]["frac"]
     print(json.dumps(res), flush=True)
 
 
@@ -583,6 +644,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the 1B-shaped prefill lines")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=128)
     ap.add_argument("--no-mla-decode", action="store_true", help="skip the multi-latent-attention decode line")

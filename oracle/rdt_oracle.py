@@ -296,7 +296,7 @@ def recurrent_forward(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, batch: in
                       act_threshold: float, start_pos: int = 0,
                       halt_logit_offset: Optional[torch.Tensor] = None,
                       caches: Optional[list] = None, transformer_off: bool = False,
-                      record: Optional[list] = None):
+                      record: Optional[list] = None, halt_at: Optional[torch.Tensor] = None):
     """RecurrentBlock.forward ("OpenMythos 분석", "Recurrent Block") for `batch`
     sequences of T = N / batch positions each.
 
@@ -309,6 +309,10 @@ def recurrent_forward(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, batch: in
     caches: optional per-loop list of per-sequence attention caches (decode / prefix).
     transformer_off: debug switch, trans = 0 (the pure LTI recurrence).
     record: optional list that receives per-loop dicts (h_in, f, biased logits, ids, p, cum).
+    halt_at: test hook, [N] int64: -1 lets the halting rule decide; t >= 0 makes position i
+    halt at loop t (weight = the remainder there) whatever cum + p is.  Parity tests set it
+    only where the rule's outcome is decided by rounding (cum + p within the measured
+    arithmetic drift of the threshold), so both sides then follow the same discrete path.
     Returns (h_out [N, D], halt_weights [L, N], expert_ids [L, N, k], new_kv per loop)."""
     h = _d(h0).clone()
     ev = _d(e)
@@ -350,6 +354,9 @@ def recurrent_forward(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, batch: in
             p = sigmoid(z)
             last = t == n_loops - 1
             stop = (cum + p >= act_threshold) | torch.tensor(last)
+            if halt_at is not None:
+                forced = halt_at >= 0
+                stop = torch.where(forced, halt_at == t, stop) | torch.tensor(last)
             remainder = (1.0 - cum).clamp(min=0.0)
             w = torch.where(stop, remainder, p)
             w = torch.where(running, w, torch.zeros_like(w))

@@ -8,7 +8,7 @@ import torch
 
 import rdt_inputs as RI
 from oracle import rdt_oracle as O
-from tests._helpers import BF16_TOL, ID_MARGIN, rel_l2, teacher_forced_ids, topk_margin
+from tests._helpers import BF16_TOL, ID_MARGIN, halting_loop, rel_l2, teacher_forced_ids, topk_margin
 
 pytestmark = pytest.mark.gpu
 
@@ -54,6 +54,48 @@ def test_rdt1b_prefill_prefix_slice_matches_oracle():
     assert (last == L - 1).float().mean() > 0.99             # halting bias -30: nearly every row runs 16 loops
 
 
+def test_rdt1b_attention_late_key_tiles():
+    """Prefill attention at the 1B shape in the launch configuration the benchmark times
+    (4 x 4096, 16 heads, head dim 128): the last 128 query rows of sequence 0 attend to all
+    32 key tiles, so the online softmax rescales across every tile.  One loop, checked on
+    the attention branch of f = RMSNorm_ffn(x + Attn(RMSNorm_attn(x))): f minus
+    RMSNorm_ffn(x), in the kernel's trace and in the oracle (peaky attention, std 0.04)."""
+    wl = RI.get_workload("rdt1b_prefill")
+    cfg, B, T = wl.cfg, wl.batch, wl.seq
+    dev = torch.device("cuda")
+    W = RI.block_weights(cfg, wl.seed, device=dev, halt_b=wl.halt_b, attn_std=0.04)
+    h0, e = RI.recurrent_inputs(cfg, B, T, wl.seed, device=dev)
+    blk = R.RecurrentBlock(cfg, W)
+    Q = 128
+    tr = R.Trace(T - Q, Q, f=torch.zeros(1, Q, cfg.dim, dtype=torch.float32, device=dev))
+    blk.forward(h0, e, B, T, 1, wl.act_threshold, trace=tr)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    Wc = {k: W[k].cpu() for k in ("rec_norm_w", "attn_norm_w", "ffn_norm_w", "w_qkv", "w_o")}
+    eps = cfg.norm_eps
+    emb = O.loop_embedding(0, cfg.loop_dim, cfg.dim, cfg.loop_theta)
+    comb = O.rmsnorm(h0[:T].cpu().double() + emb + e[:T].cpu().double(), Wc["rec_norm_w"], eps)
+    a = O.rmsnorm(comb, Wc["attn_norm_w"], eps)
+    pos = torch.arange(T)
+    # rotated keys and values of positions 0 .. T - Q - 1 (the oracle's own, chunk by chunk:
+    # a position's key and value depend on its row alone), then the last Q queries through
+    # the oracle's cached-keys path
+    ks, vs = [], []
+    for c0 in range(0, T - Q, 128):
+        _, kc, vc = O.gqa_attention(cfg, Wc, a[c0:c0 + 128], pos[c0:c0 + 128])
+        ks.append(kc)
+        vs.append(vc)
+    cache = {"k": torch.cat(ks), "v": torch.cat(vs), "pos": pos[:T - Q]}
+    o, _, _ = O.gqa_attention(cfg, Wc, a[T - Q:], pos[T - Q:], cache)
+    f_o = O.rmsnorm(comb[T - Q:] + o, Wc["ffn_norm_w"], eps)
+    f0 = O.rmsnorm(comb[T - Q:], Wc["ffn_norm_w"], eps)
+    d_o = f_o - f0
+    d_k = tr.f[0].cpu().double() - f0
+    assert rel_l2(d_o, f_o) > 0.05, "attention barely moves f: the check would be weak"
+    err = rel_l2(d_k, d_o)
+    assert err <= BF16_TOL, f"relative L2 of the attention branch over the last key tiles {err:.3e}"
+
+
 def test_rdt3b_decode_sequences_match_oracle():
     """3B-shaped decode at full size (64 sequences, per-loop 4096-token random caches):
     sequences 0 and 37 against the oracle decode step."""
@@ -67,10 +109,14 @@ def test_rdt3b_decode_sequences_match_oracle():
     blk = R.RecurrentBlock(cfg, W)
     cache = R.KVCache(k, v)
     clen = torch.full((B,), wl.cache_len, dtype=torch.int32, device=dev)
-    d_h, d_hw, d_ids = blk.decode_step(h0, e, clen, cache, L, wl.act_threshold)
+    tr = R.Trace.alloc(cfg, L, 0, B)
+    d_h, d_hw, d_ids = blk.decode_step(h0, e, clen, cache, L, wl.act_threshold, trace=tr)
     torch.cuda.synchronize()
     assert blk.read_status() == 0
     Wc = _cpu(W)
+    # every sequence's routes in every loop, teacher-forced on the step's own router input
+    n, bad, skipped = teacher_forced_ids(cfg, Wc, tr, d_ids, L)
+    assert n > 0 and bad == 0, f"{bad} of {n} teacher-forced decode rows differ ({skipped} near-ties skipped)"
     for b in (0, 37):
         caches = [[{"k": k[t, b, :, :wl.cache_len].permute(1, 0, 2).cpu(),
                     "v": v[t, b, :, :wl.cache_len].permute(1, 0, 2).cpu(),
@@ -80,11 +126,13 @@ def test_rdt3b_decode_sequences_match_oracle():
         assert rel_l2(d_h[b:b + 1], o_h) <= BF16_TOL
 
 
-def test_rdt10b_zipf_prefill_properties():
+def test_rdt10b_zipf_prefill_matches_oracle():
     """10B-shaped load-imbalanced prefill at full size (2 x 8192, 24 loops, 128 experts
-    top-8, Zipf router bias, halting spread over 4..24 loops): every position halts at
-    exactly its drawn loop, halted positions report id -1 and zero weight, routed ids are
-    exact teacher-forced on sampled rows, and the output is finite."""
+    top-8, Zipf router bias, halting spread over 4..24 loops): rows 0..31 of sequence 0
+    against the oracle run on that causal prefix alone (all 24 loops, the same bias and
+    halting offsets); every position halts at exactly its drawn loop, halted positions
+    report id -1 and zero weight, routed ids are exact teacher-forced on the traced rows,
+    and the output is finite."""
     wl = RI.get_workload("rdt10b_prefill_zipf")
     cfg, B, T, L = wl.cfg, wl.batch, wl.seq, wl.n_loops
     N = B * T
@@ -113,6 +161,17 @@ def test_rdt10b_zipf_prefill_properties():
     # the Zipf bias makes the load imbalanced: popular experts take far more than E / k share
     counts = torch.bincount(ids_c[0][ids_c[0] >= 0].flatten(), minlength=cfg.n_experts).double()
     assert counts.max() / counts.mean() > 3.0
+    # values: the causal prefix of sequence 0 through the oracle (halting is fixed by the
+    # offsets, p_i = 0.9 / (k_i - 0.5), so both sides halt at the same loops)
+    h_p = h_out[:P].cpu()
+    Wc = _cpu(W)
+    del W, blk
+    torch.cuda.empty_cache()
+    o_h, o_hw, o_ids, _ = O.recurrent_forward(cfg, Wc, h0[:P].cpu(), e[:P].cpu(), 1, L, wl.act_threshold,
+                                              halt_logit_offset=off[:P])
+    assert torch.equal(halting_loop(o_hw), last[:P])
+    err = rel_l2(h_p, o_h)
+    assert err <= BF16_TOL, f"relative L2 of h_out over the prefix {err:.3e}"
 
 
 def test_rdt3b_mla_decode_sequence_matches_oracle():
@@ -129,11 +188,14 @@ def test_rdt3b_mla_decode_sequence_matches_oracle():
     blk = R.RecurrentBlock(cfg, W)
     cache = R.KVCache(ckv, kr)
     clen = torch.full((B,), wl.cache_len, dtype=torch.int32, device=dev)
-    d_h, d_hw, d_ids = blk.decode_step(h0, e, clen, cache, L, wl.act_threshold)
+    tr = R.Trace.alloc(cfg, L, 0, B)
+    d_h, d_hw, d_ids = blk.decode_step(h0, e, clen, cache, L, wl.act_threshold, trace=tr)
     torch.cuda.synchronize()
     assert blk.read_status() == 0
     assert torch.isfinite(d_h).all()
     Wc = _cpu(W)
+    n, bad, skipped = teacher_forced_ids(cfg, Wc, tr, d_ids, L)
+    assert n > 0 and bad == 0, f"{bad} of {n} teacher-forced decode rows differ ({skipped} near-ties skipped)"
     b = 37
     caches = [[{"c_kv": ckv[t, b, :wl.cache_len].cpu(), "k_rope": kr[t, b, :wl.cache_len].cpu(),
                 "pos": torch.arange(wl.cache_len)}] for t in range(L)]
@@ -144,18 +206,32 @@ def test_rdt3b_mla_decode_sequence_matches_oracle():
         assert rel_l2(ckv[t, b, wl.cache_len], new_kv[t][0][0][0]) <= BF16_TOL
 
 
-def test_rdt1b_generation_teacher_forced():
-    """Generation with the 1B-shaped model (16 loops, 64 experts, 1 prelude + 1 coda layer;
-    vocabulary reduced to 4096 here, since it only sizes the embedding and the head): the
-    oracle's forward pass over the GPU's own sequence gives, at every generated step,
-    logits within the bf16 tolerance and the GPU's token as its argmax up to near-ties."""
-    wl = RI.get_workload("rdt1b_generate")
-    cfg = wl.cfg.replace(vocab_size=4096)
+# model shapes of generation: (workload whose block shape is used, loops, ACT threshold,
+# halting bias).  The 1B model is the generation workload itself; the 3B and 10B models
+# take the decode and prefill workloads' block shapes with one prelude and one coda dense
+# layer (dense hidden 4 dim / 3: 4096 at dim 3072, 5461 at dim 4096, which the binding pads
+# to 5504), ACT off; the 10B model runs 4 of its loops to bound the oracle's time.
+GEN_SHAPES = {"rdt1b": ("rdt1b_generate", None, None, None), "rdt3b": ("rdt3b_decode", 16, 0.0, 0.0),
+              "rdt10b": ("rdt10b_prefill_zipf", 4, 0.0, 0.0)}
+
+
+@pytest.mark.parametrize("shape", ["rdt1b", "rdt3b", "rdt10b"])
+def test_generation_teacher_forced(shape):
+    """Generation with the 1B / 3B / 10B-shaped model (1 prelude + 1 coda layer; vocabulary
+    reduced to 4096 here, since it only sizes the embedding and the head): the oracle's
+    forward pass over the GPU's own sequence gives, at every generated step, logits within
+    the bf16 tolerance and the GPU's token as its argmax up to near-ties."""
+    name, loops, thr, halt_b = GEN_SHAPES[shape]
+    wl = RI.get_workload(name)
+    cfg = wl.cfg.replace(vocab_size=4096, prelude_layers=1, coda_layers=1)
+    L = loops or wl.n_loops
+    thr = wl.act_threshold if thr is None else thr
+    halt_b = wl.halt_b if halt_b is None else halt_b
     dev = torch.device("cuda")
-    MW = RI.model_weights(cfg, wl.seed, device=dev, halt_b=wl.halt_b)
-    B, T0, new, L = 2, 24, 3, wl.n_loops
+    MW = RI.model_weights(cfg, wl.seed, device=dev, halt_b=halt_b)
+    B, T0, new = 2, 24, 3
     prompt = torch.randint(0, cfg.vocab_size, (B, T0), generator=torch.Generator().manual_seed(11))
-    gen = R.Generator(cfg, MW, B, T0, new, L, wl.act_threshold)
+    gen = R.Generator(cfg, MW, B, T0, new, L, thr)
     gen.prefill(prompt.to(device=dev, dtype=torch.int32).contiguous())
     logits = [gen.logits.clone()]
     for s in range(1, new):
@@ -166,8 +242,10 @@ def test_rdt1b_generation_teacher_forced():
     seq = torch.cat([prompt, toks], dim=1)
     MWc = {k: ([{kk: vv.cpu() for kk, vv in blk.items()} for blk in v] if isinstance(v, list) else
                ({kk: vv.cpu() for kk, vv in v.items()} if isinstance(v, dict) else v.cpu())) for k, v in MW.items()}
+    del gen, MW
+    torch.cuda.empty_cache()
     b = 0
-    full, _, _ = O.model_forward(cfg, MWc, seq[b:b + 1, :-1], L, wl.act_threshold)
+    full, _, _ = O.model_forward(cfg, MWc, seq[b:b + 1, :-1], L, thr)
     for s in range(new):
         ol = full[0, T0 - 1 + s]
         gl = logits[s][b].cpu()

@@ -9,7 +9,7 @@ import torch
 
 import rdt_inputs as RI
 from oracle import rdt_oracle as O
-from tests._helpers import (BF16_TOL, FP32_TOL, halting_loop, max_rel, rel_l2, same_halting_rows,
+from tests._helpers import (BF16_TOL, FP32_TOL, halting_loop, max_rel, oracle_following_halts, rel_l2,
                             teacher_forced_ids, to_dev)
 
 pytestmark = pytest.mark.gpu
@@ -76,18 +76,14 @@ def test_tiny_mla_fp32_model_logits():
     assert torch.equal(rec[2].cpu().long(), o_rec[2])
 
 
-def _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, L, o_hw=None, record=None, thr=0.0, seq=0):
-    """bf16 parity, end to end: relative L2 over the rows the inputs still determine
-    (positions before the first near-threshold ACT disagreement of their sequence; any
-    disagreement away from the threshold fails); ids exact teacher-forced (the kernel's
-    own router input) wherever the top-k margin is >= 1e-3.  End-to-end routes are not
-    compared: a near-tie flip at one position changes that position's state, hence its
-    keys and values, hence every later position's attention."""
-    keep = torch.ones(h_out.shape[0], dtype=torch.bool)
-    if record is not None and thr > 0:
-        keep = same_halting_rows(hw, o_hw, record, thr, seq)
-        assert keep.float().mean() >= 0.5, "most positions follow a halting disagreement"
-    err = rel_l2(h_out.cpu()[keep], o_h[keep])
+def _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, L):
+    """bf16 parity, end to end: relative L2 over every position (the oracle follows the
+    GPU's halting loop where that decision was a near-tie, see oracle_following_halts);
+    ids exact teacher-forced (the kernel's own router input) wherever the top-k margin is
+    >= 1e-3.  End-to-end routes are not compared: a near-tie flip at one position changes
+    that position's state, hence its keys and values, hence every later position's
+    attention."""
+    err = rel_l2(h_out.cpu(), o_h)
     assert err <= BF16_TOL, f"relative L2 {err:.3e}"
     n, nbad, skipped = teacher_forced_ids(cfg, W, tr, ids, L)
     assert n > 0 and nbad == 0, f"{nbad} of {n} teacher-forced id rows differ ({skipped} near-ties skipped)"
@@ -141,9 +137,9 @@ def test_recurrent_bf16_matches_oracle(name, variant):
     h_out, hw, ids = blk.forward(h0.cuda(), e.cuda(), B, T, L, thr, trace=tr)
     torch.cuda.synchronize()
     assert blk.read_status() == 0
-    rec = []
-    o_h, o_hw, o_ids, _ = O.recurrent_forward(cfg, W, h0, e, B, L, thr, record=rec)
-    _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, L, o_hw, rec, thr, T)
+    run = lambda halt_at, rec: O.recurrent_forward(cfg, W, h0, e, B, L, thr, record=rec, halt_at=halt_at)
+    (o_h, o_hw, o_ids, _), rec, n_forced, margin = oracle_following_halts(run, hw, tr.p, thr)
+    _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, L)
     errs = _teacher_forced_states(cfg, W, tr, e, B, L, ids, hw)
     assert max(errs) <= BF16_TOL, f"per-loop teacher-forced relative L2 {errs}"
 
@@ -212,7 +208,8 @@ def test_decode_step_matches_oracle_and_prefill(dtype):
     cache = R.KVCache(k, torch.zeros_like(k))
     blk.forward(h0[keep].cuda(), e[keep].cuda(), B, T, L, thr, cache=cache)
     clen = torch.full((B,), T, dtype=torch.int32, device="cuda")
-    d_h, d_hw, d_ids = blk.decode_step(h0[last].cuda(), e[last].cuda(), clen, cache, L, thr)
+    tr = R.Trace.alloc(cfg, L, 0, B)
+    d_h, d_hw, d_ids = blk.decode_step(h0[last].cuda(), e[last].cuda(), clen, cache, L, thr, trace=tr)
     torch.cuda.synchronize()
     assert blk.read_status() == 0
     full = O.recurrent_forward(cfg, W, h0, e, B, L, thr)
@@ -221,6 +218,9 @@ def test_decode_step_matches_oracle_and_prefill(dtype):
         assert torch.equal(d_ids.cpu().long(), full[2][:, last])
     else:
         assert rel_l2(d_h, full[0][last]) <= BF16_TOL
+    # the decode step's routes, teacher-forced on its own router input
+    n, bad, skipped = teacher_forced_ids(cfg, W, tr, d_ids, L)
+    assert n > 0 and bad == 0, f"{bad} of {n} teacher-forced decode rows differ ({skipped} near-ties skipped)"
     # GPU prefill of T + 1 tokens gives the same last rows as GPU prefill + decode
     p_h, p_hw, p_ids = blk.forward(h0.cuda(), e.cuda(), B, T + 1, L, thr)
     tol = 1e-5 if dtype == "fp32" else 1e-2
@@ -268,9 +268,12 @@ def test_decode_random_cache_ragged_lengths(dtype):
     blk = R.RecurrentBlock(cfg, to_dev(W))
     cache = R.KVCache(k.cuda(), v.cuda())
     clen = torch.tensor(lens, dtype=torch.int32, device="cuda")
-    d_h, d_hw, d_ids = blk.decode_step(h0.cuda(), e.cuda(), clen, cache, L, 0.0)
+    tr = R.Trace.alloc(cfg, L, 0, B)
+    d_h, d_hw, d_ids = blk.decode_step(h0.cuda(), e.cuda(), clen, cache, L, 0.0, trace=tr)
     torch.cuda.synchronize()
     assert blk.read_status() == 0
+    n, bad, skipped = teacher_forced_ids(cfg, W, tr, d_ids, L)
+    assert n > 0 and bad == 0, f"{bad} of {n} teacher-forced decode rows differ ({skipped} near-ties skipped)"
     caches = [[{"k": k[t, b, :, :lens[b]].permute(1, 0, 2), "v": v[t, b, :, :lens[b]].permute(1, 0, 2),
                 "pos": torch.arange(lens[b])} for b in range(B)] for t in range(L)]
     o_h, o_hw, o_ids, new_kv = O.decode_step(cfg, W, h0, e, caches, lens, L, 0.0)

@@ -511,3 +511,86 @@ def test_generate_is_causally_consistent():
 def test_greedy_ties_go_to_the_lowest_index():
     x = torch.tensor([[0.5, 2.0, 2.0, -1.0], [3.0, 3.0, 3.0, 3.0]], dtype=torch.float64)
     assert O.greedy(x).tolist() == [1, 0]
+
+
+# ------------------------------------------------------------------------------------------
+# 10. model composition ("OpenMythos 분석", Core Structure): embed -> prelude -> e = x ->
+#     recurrent block -> coda -> head(norm(x)).  A block whose attention output projection
+#     is zero reduces to x + FFN(RMSNorm(x)); with its FFN down-projection zero too it is
+#     the identity.  The reduced blocks and the final norm / head are written with library
+#     routines, and the recurrent block is the (separately pinned) oracle block.
+# ------------------------------------------------------------------------------------------
+
+def _ffn_only(W):
+    """Zero the attention output projection: the block becomes x + FFN(RMSNorm(x))."""
+    return {**W, "w_o": torch.zeros_like(W["w_o"])}
+
+
+def _identity(W):
+    return {**_ffn_only(W), "w2": torch.zeros_like(W["w2"])}
+
+
+def _lib_ffn_block(W, x, eps):
+    f = Fn.rms_norm(x, (x.shape[-1],), W["ffn_norm_w"].double(), eps)
+    return x + _lib_expert(W["w13"][0], W["w2"][0], f)
+
+
+def _model_case(prelude_layers, coda_layers, seed=5):
+    cfg = tiny_cfg(prelude_layers=prelude_layers, coda_layers=coda_layers)
+    MW = RI.model_weights(cfg, seed, halt_w_std=0.2)
+    ids = torch.randint(0, cfg.vocab_size, (2, 7), generator=torch.Generator().manual_seed(seed))
+    return cfg, MW, ids
+
+
+def _lib_head(cfg, MW, x):
+    return Fn.linear(Fn.rms_norm(x, (cfg.dim,), MW["norm_w"].double(), cfg.norm_eps), MW["head"].double())
+
+
+def test_model_forward_with_identity_blocks_is_head_of_norm_of_recurrent():
+    cfg, MW, ids = _model_case(1, 1)
+    MW = {**MW, "prelude": [_identity(W) for W in MW["prelude"]], "coda": [_identity(W) for W in MW["coda"]]}
+    L, thr = 3, 0.99
+    logits, rec, e = O.model_forward(cfg, MW, ids, L, thr)
+    x = Fn.embedding(ids.reshape(-1), MW["embed"].double())
+    assert torch.equal(e, x)                                  # e is the (identity) prelude's output
+    want_rec = O.recurrent_forward(cfg, MW["recurrent"], x, x, 2, L, thr)
+    assert torch.allclose(rec[0], want_rec[0], rtol=0, atol=0) and torch.equal(rec[2], want_rec[2])
+    want = _lib_head(cfg, MW, want_rec[0]).reshape(2, 7, -1)
+    assert torch.allclose(logits, want, rtol=1e-12, atol=1e-13)
+
+
+def test_model_forward_prelude_layers_in_order_and_e_after_the_prelude():
+    cfg, MW, ids = _model_case(2, 1)
+    MW = {**MW, "prelude": [_ffn_only(W) for W in MW["prelude"]], "coda": [_identity(W) for W in MW["coda"]]}
+    L, thr = 2, 0.0
+    logits, rec, e = O.model_forward(cfg, MW, ids, L, thr)
+    x = Fn.embedding(ids.reshape(-1), MW["embed"].double())
+    for W in MW["prelude"]:                                   # layer 0, then layer 1
+        x = _lib_ffn_block(W, x, cfg.norm_eps)
+    assert torch.allclose(e, x, rtol=1e-12, atol=1e-13)
+    want_rec = O.recurrent_forward(cfg, MW["recurrent"], x, x, 2, L, thr)
+    assert torch.allclose(rec[0], want_rec[0], rtol=1e-10, atol=1e-12)
+    assert torch.allclose(logits, _lib_head(cfg, MW, want_rec[0]).reshape(2, 7, -1), rtol=1e-10, atol=1e-11)
+    # the layers do not commute: the other order gives another e
+    y = Fn.embedding(ids.reshape(-1), MW["embed"].double())
+    for W in reversed(MW["prelude"]):
+        y = _lib_ffn_block(W, y, cfg.norm_eps)
+    assert (y - x).abs().max() > 1e-6
+
+
+def test_model_forward_coda_layers_after_the_recurrent_block():
+    cfg, MW, ids = _model_case(1, 2)
+    MW = {**MW, "prelude": [_identity(W) for W in MW["prelude"]], "coda": [_ffn_only(W) for W in MW["coda"]]}
+    L, thr = 3, 0.99
+    logits, rec, e = O.model_forward(cfg, MW, ids, L, thr)
+    x = Fn.embedding(ids.reshape(-1), MW["embed"].double())
+    h = O.recurrent_forward(cfg, MW["recurrent"], x, x, 2, L, thr)[0]
+    for W in MW["coda"]:
+        h = _lib_ffn_block(W, h, cfg.norm_eps)
+    assert torch.allclose(logits, _lib_head(cfg, MW, h).reshape(2, 7, -1), rtol=1e-10, atol=1e-11)
+    # coda before the recurrent block would give other logits
+    z = x
+    for W in MW["coda"]:
+        z = _lib_ffn_block(W, z, cfg.norm_eps)
+    z = O.recurrent_forward(cfg, MW["recurrent"], z, x, 2, L, thr)[0]
+    assert (_lib_head(cfg, MW, z).reshape(2, 7, -1) - logits).abs().max() > 1e-6

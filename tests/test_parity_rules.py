@@ -1,34 +1,91 @@
 """The parity tests' rules for float-decided discrete outcomes, checked on planted cases."""
+import math
+
 import pytest
 import torch
 
-from tests._helpers import HALT_MARGIN, same_halting_rows, topk_margin
+from tests._helpers import (check_forced_halts, halt_margin, halting_loop, oracle_following_halts,
+                            topk_margin)
 
 
-def _hw(loops):
-    """ACT weights with position i halting at loop loops[i] (L = 3)."""
-    hw = torch.zeros(3, len(loops))
+def _hw(loops, L=3):
+    """ACT weights with position i halting at loop loops[i]."""
+    hw = torch.zeros(L, len(loops))
     for i, t in enumerate(loops):
         hw[: t + 1, i] = 1.0 / (t + 1)
     return hw
 
 
-def test_halting_disagreement_near_the_threshold_is_accepted():
-    thr = 0.99
-    record = [{"cum": torch.tensor([0.2, 0.6, 0.3])},
-              {"cum": torch.tensor([0.5, thr + HALT_MARGIN / 2, 0.6])},   # the oracle just reaches thr
-              {"cum": torch.tensor([1.1, 1.2, 1.0])}]
-    keep = same_halting_rows(_hw([2, 2, 2]), _hw([2, 1, 2]), record, thr)   # position 1: oracle halts at loop 1
-    assert keep.tolist() == [True, False, True]
+def test_halt_margin_is_loops_times_the_largest_drift_on_loops_run():
+    p_o = torch.full((3, 4), 0.3, dtype=torch.float64)
+    p_g = p_o.clone()
+    p_g[0, 1] += 0.002          # ran: counts
+    p_g[2, 0] += 0.5            # position 0 halted at loop 1: loop 2 is not compared
+    assert halt_margin(p_g, p_o, torch.tensor([1, 2, 2, 2])) == pytest.approx(3 * 0.002)
 
 
-def test_halting_disagreement_away_from_the_threshold_fails():
+def test_forced_halt_near_the_threshold_is_accepted():
     thr = 0.99
-    record = [{"cum": torch.tensor([0.2, 0.5, 0.3])},
-              {"cum": torch.tensor([0.5, 0.99, 0.6])},
-              {"cum": torch.tensor([1.1, 1.2, 1.0])}]
+    cum = torch.tensor([[0.2, 0.6, 0.3], [0.5, thr + 0.004, 0.6], [1.1, 1.2, 1.0]], dtype=torch.float64)
+    check_forced_halts(torch.tensor([1]), torch.tensor([1]), cum, thr, margin=0.005, n_positions=100)
+
+
+def test_forced_halt_away_from_the_threshold_fails():
+    thr = 0.99
+    cum = torch.tensor([[0.2, 0.5, 0.3], [0.5, 0.99, 0.6], [1.1, 1.2, 1.0]], dtype=torch.float64)
     with pytest.raises(AssertionError):
-        same_halting_rows(_hw([2, 0, 2]), _hw([2, 1, 2]), record, thr)   # loop 0: cum 0.5, far from 0.99
+        check_forced_halts(torch.tensor([1]), torch.tensor([0]), cum, thr, margin=0.005, n_positions=100)
+
+
+def test_too_many_forced_halts_fail():
+    thr = 0.99
+    cum = torch.full((3, 10), thr, dtype=torch.float64)
+    with pytest.raises(AssertionError):
+        check_forced_halts(torch.tensor([1, 2, 3]), torch.tensor([1, 1, 1]), cum, thr, margin=0.1, n_positions=10,
+                           max_frac=0.2)
+
+
+def test_oracle_is_rerun_on_the_gpu_halting_loop_of_a_near_tie():
+    """A planted oracle whose position 1 reaches the threshold at loop 1 by 0.001 while the
+    GPU halts it at loop 2: the helper reruns it with that halt imposed."""
+    thr, L = 0.99, 3
+    calls = []
+
+    def run(halt_at, rec):
+        calls.append(None if halt_at is None else halt_at.clone())
+        loops = [2, 1, 2] if halt_at is None else [2, int(halt_at[1]), 2]
+        p = torch.tensor([[0.3, 0.5, 0.3], [0.3, 0.491, 0.3], [0.3, 0.3, 0.3]], dtype=torch.float64)
+        cum = torch.cumsum(p, 0)
+        for t in range(L):
+            rec.append({"p": p[t], "cum": cum[t]})
+        return None, _hw(loops), None, None
+
+    p_gpu = torch.tensor([[0.3, 0.5, 0.3], [0.3, 0.4895, 0.3], [0.3, 0.3, 0.3]], dtype=torch.float64)
+    out, rec, n_forced, margin = oracle_following_halts(run, _hw([2, 2, 2]), p_gpu, thr)
+    assert n_forced == 1 and calls[0] is None and calls[1].tolist() == [-1, 2, -1]
+    assert margin == pytest.approx(3 * 0.0015)
+    assert halting_loop(out[1]).tolist() == [2, 2, 2]
+
+
+def test_oracle_halt_at_hook_imposes_the_halting_loop():
+    """The oracle's test hook: halt_at[i] = t halts position i at loop t with the remainder as
+    its weight (ACT weights still sum to one); -1 everywhere is the plain rule."""
+    import rdt_inputs as RI
+    from oracle import rdt_oracle as O
+    cfg = RI.get_workload("tiny_gqa_fp32").cfg
+    W = RI.block_weights(cfg, 3, halt_w_std=0.0, halt_b=-3.0)      # p = sigmoid(-3): no early halt
+    h0, e = RI.recurrent_inputs(cfg, 1, 6, 3)
+    L = 4
+    base = O.recurrent_forward(cfg, W, h0, e, 1, L, 0.99)
+    same = O.recurrent_forward(cfg, W, h0, e, 1, L, 0.99, halt_at=torch.full((6,), -1, dtype=torch.int64))
+    assert torch.equal(base[0], same[0]) and torch.equal(base[1], same[1])
+    assert halting_loop(base[1]).tolist() == [L - 1] * 6
+    forced = O.recurrent_forward(cfg, W, h0, e, 1, L, 0.99, halt_at=torch.tensor([-1, 1, -1, -1, 0, -1]))
+    assert halting_loop(forced[1]).tolist() == [3, 1, 3, 3, 0, 3]
+    assert torch.allclose(forced[1].sum(0), torch.ones(6, dtype=torch.float64), atol=1e-12)
+    p = 1.0 / (1.0 + math.exp(3.0))
+    assert float(forced[1][1, 1]) == pytest.approx(1.0 - p)             # remainder after one loop of p
+    assert (forced[2][2:, 1] == -1).all()                                # frozen after its halt
 
 
 def test_topk_margin_counts_order_swaps_inside_the_top_k():
@@ -36,16 +93,6 @@ def test_topk_margin_counts_order_swaps_inside_the_top_k():
     assert float(topk_margin(s, 2)[0]) == pytest.approx(5e-4)
     s = torch.tensor([[3.0, 2.0, 1.0, 0.999]], dtype=torch.float64)          # the 3rd / 4th near-tie is outside top-2 + 1
     assert float(topk_margin(s, 2)[0]) == pytest.approx(1.0)
-
-
-def test_positions_after_a_halting_disagreement_are_left_out_of_their_sequence():
-    thr = 0.99
-    # two sequences of 3 positions; position 1 of sequence 0 halts one loop apart
-    record = [{"cum": torch.tensor([0.2, 0.6, 0.3, 0.2, 0.2, 0.2])},
-              {"cum": torch.tensor([0.5, thr + HALT_MARGIN / 2, 0.6, 0.5, 0.5, 0.5])},
-              {"cum": torch.tensor([1.1, 1.2, 1.0, 1.0, 1.0, 1.0])}]
-    keep = same_halting_rows(_hw([2, 2, 2, 2, 2, 2]), _hw([2, 1, 2, 2, 2, 2]), record, thr, seq=3)
-    assert keep.tolist() == [True, False, False, True, True, True]
 
 
 def test_dense_padding_keeps_the_block_function():
