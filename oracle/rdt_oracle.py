@@ -213,24 +213,35 @@ def attention(cfg, W, a, pos, cache=None):
 # MoE
 # ------------------------------------------------------------------------------------------
 
-def router(cfg, W: dict, f: torch.Tensor):
+def router(cfg, W: dict, f: torch.Tensor, forced: Optional[torch.Tensor] = None):
     """MoEFFN router ("OpenMythos 분석", "MoE"): logits = f Wr^T, scores = softmax(logits),
-    idx = topk(logits + router_bias), gates = scores[idx] renormalised to sum 1."""
+    idx = topk(logits + router_bias), gates = scores[idx] renormalised to sum 1.
+    forced: test hook, [n, k] int64: rows with forced[i, 0] >= 0 take those experts (the
+    gates are still this router's scores at them, renormalised); parity tests impose a
+    route only where the two sides' biased logits differ enough to swap it.
+    Returns (idx, gates, logits, biased logits, the router's own idx)."""
     k = cfg.n_experts_per_tok
     logits = f @ _d(W["w_router"]).T
     scores = softmax(logits)
     biased = logits + _d(W["router_bias"])
-    idx = topk_lower_index(biased, k)
+    own = topk_lower_index(biased, k)
+    idx = own
+    if forced is not None:
+        use = forced[:, 0] >= 0
+        idx = torch.where(use[:, None], forced.to(torch.int64), own)
     g = torch.gather(scores, -1, idx)
     g = g / g.sum(dim=-1, keepdim=True)
-    return idx, g, logits, biased
+    return idx, g, logits, biased, own
 
 
-def moe_ffn(cfg, W: dict, f: torch.Tensor):
+def moe_ffn(cfg, W: dict, f: torch.Tensor, forced: Optional[torch.Tensor] = None, own: Optional[list] = None):
     """Routed top-k SwiGLU experts plus always-on shared experts (gate 1).
+    forced: test hook passed to the router; own: optional list receiving the router's own idx.
     Returns (y [n, D], idx [n, k], gates [n, k], biased logits [n, E])."""
     E, S = cfg.n_experts, cfg.n_shared_experts
-    idx, g, logits, biased = router(cfg, W, f)
+    idx, g, logits, biased, own_idx = router(cfg, W, f, forced)
+    if own is not None:
+        own.append(own_idx)
     y = torch.zeros_like(f)
     for e in torch.unique(idx).tolist():
         rows, slot = torch.nonzero(idx == e, as_tuple=True)
@@ -249,12 +260,15 @@ def dense_ffn(W: dict, f: torch.Tensor):
 # ------------------------------------------------------------------------------------------
 
 def transformer_block(cfg, W: dict, x: torch.Tensor, batch: int, pos: torch.Tensor, use_moe: bool,
-                      caches=None, row_mask: Optional[torch.Tensor] = None):
+                      caches=None, row_mask: Optional[torch.Tensor] = None,
+                      forced_ids: Optional[torch.Tensor] = None):
     """Pre-norm residual block: x1 = x + Attn(RMSNorm(x)); out = x1 + FFN(RMSNorm(x1)).
     x: [B*T, D] (sequence-major); pos: [B*T].  caches: optional per-sequence list of
     attention cache dicts (read, not modified).  row_mask (MoE only): rows whose FFN is
-    evaluated; other rows get out = x1 and expert ids -1.
-    Returns (out, x1, info) with info holding ids/gates/biased logits/new kv per sequence."""
+    evaluated; other rows get out = x1 and expert ids -1.  forced_ids: test hook, [N, k]
+    routes imposed on rows with forced_ids[i, 0] >= 0 (see router).
+    Returns (out, x1, info) with info holding ids/gates/biased logits/new kv per sequence
+    and the router's own ids ("own_ids", -1 for rows not evaluated)."""
     N, D = x.shape
     T = N // batch
     a = rmsnorm(x, W["attn_norm_w"], cfg.norm_eps)
@@ -272,15 +286,17 @@ def transformer_block(cfg, W: dict, x: torch.Tensor, batch: int, pos: torch.Tens
         return x1 + dense_ffn(W, f), x1, info
     k = cfg.n_experts_per_tok
     ids = torch.full((N, k), -1, dtype=torch.int64)
+    own_ids = torch.full((N, k), -1, dtype=torch.int64)
     gates = torch.zeros(N, k, dtype=F64)
     biased = torch.zeros(N, cfg.n_experts, dtype=F64)
     rows = torch.arange(N) if row_mask is None else torch.nonzero(row_mask, as_tuple=True)[0]
     out = x1.clone()
     if rows.numel():
-        y, idx, g, bl = moe_ffn(cfg, W, f[rows])
+        own = []
+        y, idx, g, bl = moe_ffn(cfg, W, f[rows], None if forced_ids is None else forced_ids[rows], own)
         out[rows] = x1[rows] + y
-        ids[rows], gates[rows], biased[rows] = idx, g, bl
-    info.update(ids=ids, gates=gates, biased=biased)
+        ids[rows], gates[rows], biased[rows], own_ids[rows] = idx, g, bl, own[0]
+    info.update(ids=ids, gates=gates, biased=biased, own_ids=own_ids)
     return out, x1, info
 
 
@@ -296,7 +312,8 @@ def recurrent_forward(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, batch: in
                       act_threshold: float, start_pos: int = 0,
                       halt_logit_offset: Optional[torch.Tensor] = None,
                       caches: Optional[list] = None, transformer_off: bool = False,
-                      record: Optional[list] = None, halt_at: Optional[torch.Tensor] = None):
+                      record: Optional[list] = None, halt_at: Optional[torch.Tensor] = None,
+                      route_ids: Optional[torch.Tensor] = None):
     """RecurrentBlock.forward ("OpenMythos 분석", "Recurrent Block") for `batch`
     sequences of T = N / batch positions each.
 
@@ -313,6 +330,8 @@ def recurrent_forward(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, batch: in
     halt at loop t (weight = the remainder there) whatever cum + p is.  Parity tests set it
     only where the rule's outcome is decided by rounding (cum + p within the measured
     arithmetic drift of the threshold), so both sides then follow the same discrete path.
+    route_ids: test hook, [L, N, k] int64: the routes of loop t imposed on the rows with
+    route_ids[t, i, 0] >= 0 (see router); the record keeps the router's own ids.
     Returns (h_out [N, D], halt_weights [L, N], expert_ids [L, N, k], new_kv per loop)."""
     h = _d(h0).clone()
     ev = _d(e)
@@ -339,12 +358,13 @@ def recurrent_forward(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, batch: in
             new_kv.append(None)
         else:
             trans, _, info = transformer_block(cfg, W, combined, batch, pos, True,
-                                               None if caches is None else caches[t], running)
+                                               None if caches is None else caches[t], running,
+                                               None if route_ids is None else route_ids[t])
             trans = trans + lora_delta(cfg, W, trans, t)
             expert_ids[t] = info["ids"]
             new_kv.append(info["new_kv"])
             if rec is not None:
-                rec.update(f=info["f"], biased=info["biased"], ids=info["ids"])
+                rec.update(f=info["f"], biased=info["biased"], ids=info["ids"], own_ids=info["own_ids"])
         h_new = A * h + Bv * ev + trans
         h_new[halted] = h[halted]                      # frozen rows
         if act_on:
@@ -384,16 +404,19 @@ def dense_block_forward(cfg, W: dict, x: torch.Tensor, batch: int, start_pos: in
     return out
 
 
-def model_forward(cfg, MW: dict, ids: torch.Tensor, n_loops: int, act_threshold: float):
+def model_forward(cfg, MW: dict, ids: torch.Tensor, n_loops: int, act_threshold: float,
+                  route_ids: Optional[torch.Tensor] = None, record: Optional[list] = None):
     """OpenMythos.forward ("OpenMythos 분석", "Core Structure") for ids [B, T]:
     logits = head(norm(coda(recurrent(prelude(embed(ids)), e)))).
+    route_ids / record: passed to the recurrent block (test hooks, see recurrent_forward).
     Returns (logits [B, T, V], recurrent outputs tuple, e)."""
     B, T = ids.shape
     x = _d(MW["embed"])[ids.reshape(-1)]
     for W in MW["prelude"]:
         x = dense_block_forward(cfg, W, x, B)
     e = x.clone()
-    rec = recurrent_forward(cfg, MW["recurrent"], x, e, B, n_loops, act_threshold)
+    rec = recurrent_forward(cfg, MW["recurrent"], x, e, B, n_loops, act_threshold, record=record,
+                            route_ids=route_ids)
     x = rec[0]
     for W in MW["coda"]:
         x = dense_block_forward(cfg, W, x, B)
@@ -426,12 +449,13 @@ def generate(cfg, MW: dict, prompt_ids: torch.Tensor, max_new_tokens: int, n_loo
 
 
 def decode_step(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, caches: list, cache_len: list,
-                n_loops: int, act_threshold: float = 0.0):
+                n_loops: int, act_threshold: float = 0.0, halt_logit_offset: Optional[torch.Tensor] = None):
     """One KV-cached decode step of the recurrent block ("OpenMythos 분석", "RoPE &
     generation cache"): one new token per sequence b at position cache_len[b]; loop t
     attends to its own loop cache (keys 0..cache_len[b]-1) plus the new token.
     caches[t][b] = {"k": [C_b, Hkv, hd], "v": ..., "pos": [C_b]} (GQA), or
     {"c_kv": [C_b, kv_lora_rank], "k_rope": [C_b, qk_rope_head_dim], "pos": [C_b]} (MLA).
+    halt_logit_offset: optional [B], added to the halting logit (as in recurrent_forward).
     Returns (h_out [B, D], halt_weights [L, B], expert_ids [L, B, k], new_kv)."""
     B = h0.shape[0]
     h = _d(h0).clone()
@@ -471,7 +495,10 @@ def decode_step(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, caches: list, c
         h_new = A * h + Bv * ev + trans
         h_new[halted] = h[halted]
         if act_threshold > 0:
-            p = sigmoid(h_new @ _d(W["halt_w"]) + _d(W["halt_b"])[0])
+            z = h_new @ _d(W["halt_w"]) + _d(W["halt_b"])[0]
+            if halt_logit_offset is not None:
+                z = z + _d(halt_logit_offset)
+            p = sigmoid(z)
             stop = (cum + p >= act_threshold) | torch.tensor(t == n_loops - 1)
             w = torch.where(stop, (1.0 - cum).clamp(min=0.0), p)
             w = torch.where(running, w, torch.zeros_like(w))
@@ -483,3 +510,43 @@ def decode_step(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, caches: list, c
         h_out = h_out + w[:, None] * h_new
         h = h_new
     return h_out, halt_weights, expert_ids, new_kv
+
+
+def _append_cache(cfg, cache: dict, kv, pos: int) -> dict:
+    """A sequence's loop cache extended by one position's entries (as decode_step returns
+    them: rotated key and value for GQA, c_kv and rotated k_rope for MLA)."""
+    k1, k2 = kv
+    p = torch.tensor([pos], dtype=torch.int64)
+    if cfg.attn_type == "gqa":
+        return {"k": torch.cat([_d(cache["k"]), k1], 0), "v": torch.cat([_d(cache["v"]), k2], 0),
+                "pos": torch.cat([cache["pos"].to(torch.int64), p])}
+    return {"c_kv": torch.cat([_d(cache["c_kv"]), k1], 0), "k_rope": torch.cat([_d(cache["k_rope"]), k2], 0),
+            "pos": torch.cat([cache["pos"].to(torch.int64), p])}
+
+
+def decode_tokens(cfg, W: dict, h0: torch.Tensor, e: torch.Tensor, caches: list, cache_len: list, n_loops: int,
+                  act_threshold: float = 0.0, halt_logit_offset: Optional[torch.Tensor] = None):
+    """S successive KV-cached decode steps of each of B sequences (GeekNews summary, section
+    6: continuous depth-wise batching lets each token leave the shared block at its own
+    depth and new tokens take its place; it computes exactly this).  Token n of sequence b
+    sits at position cache_len[b] + n; each step runs decode_step on that sequence alone and
+    then appends the step's keys / values of every loop -- the loops after the token halted
+    included, from its frozen state -- to the sequence's loop caches, which the next token
+    reads.  h0 [B, S, D], e [B, S, D], halt_logit_offset [B, S] or None; caches[t][b] as in
+    decode_step (not modified).
+    Returns (h_out [B, S, D], halt_weights [B, S, L], expert_ids [B, S, L, k])."""
+    B, S, D = h0.shape
+    k = cfg.n_experts_per_tok
+    h_out = torch.zeros(B, S, D, dtype=F64)
+    hw = torch.zeros(B, S, n_loops, dtype=F64)
+    ids = torch.full((B, S, n_loops, k), -1, dtype=torch.int64)
+    for b in range(B):
+        seq_caches = [caches[t][b] for t in range(n_loops)]
+        for n in range(S):
+            off = None if halt_logit_offset is None else halt_logit_offset[b, n:n + 1]
+            o_h, o_hw, o_ids, new_kv = decode_step(cfg, W, h0[b, n:n + 1], e[b, n:n + 1],
+                                                   [[c] for c in seq_caches], [cache_len[b] + n], n_loops,
+                                                   act_threshold, off)
+            h_out[b, n], hw[b, n], ids[b, n] = o_h[0], o_hw[:, 0], o_ids[:, 0]
+            seq_caches = [_append_cache(cfg, seq_caches[t], new_kv[t][0], cache_len[b] + n) for t in range(n_loops)]
+    return h_out, hw, ids

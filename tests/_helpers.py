@@ -93,6 +93,46 @@ def halting_loop(hw: torch.Tensor) -> torch.Tensor:
     return nz.max(dim=0).values
 
 
+def halting_loop_ids(ids: torch.Tensor) -> torch.Tensor:
+    """Index of the last loop a position ran its experts in, per position (ids [L, N, k]; a
+    halted position reports -1 from the next loop on).  Unlike the last non-zero ACT weight
+    this is exact even where the remainder weight at the halting loop is 0."""
+    L = ids.shape[0]
+    ran = (ids.cpu()[..., 0] >= 0).to(torch.int64) * torch.arange(L)[:, None]
+    return ran.max(dim=0).values
+
+
+def check_route_flips(ids_gpu: torch.Tensor, biased_gpu: torch.Tensor, record: list) -> int:
+    """Routes the oracle took from the GPU (route_ids) against the oracle's own top-k of the
+    same run (record[t]["own_ids"]), per loop and running row.  Top-k picks the k largest
+    biased logits ("OpenMythos 분석", MoE), so a route can differ only if some expert a the
+    oracle picked and some expert b the GPU picked (or an order inside the top k) swap
+    between the two sides' logits: with eps = max_e |l_gpu - l_oracle| of that row,
+    l_oracle[a] - l_oracle[b] <= 2 eps.  Any difference not explained so fails.
+    ids_gpu [L, N, k], biased_gpu [L, N, E] (the GPU's traced biased logits).
+    Returns the number of (loop, row) routes that differ."""
+    n = 0
+    for t, r in enumerate(record):
+        own = r["own_ids"]
+        got = ids_gpu[t].cpu().long()
+        run = (own[:, 0] >= 0) & (got[:, 0] >= 0)
+        diff = torch.nonzero((own != got).any(-1) & run)[:, 0]
+        for i in diff.tolist():
+            lo = r["biased"][i]
+            eps = float((lo - biased_gpu[t, i].cpu().double()).abs().max())
+            o, g = own[i].tolist(), got[i].tolist()
+            if set(o) != set(g):
+                pairs = [(a, b) for a in set(o) - set(g) for b in set(g) - set(o)]
+            else:   # same experts in another order: the pairs the GPU emitted in the oracle's wrong order
+                pairs = [(g[y], g[x]) for x in range(len(g)) for y in range(x + 1, len(g))
+                         if float(lo[g[x]]) < float(lo[g[y]])]
+            worst = max(float(lo[a] - lo[b]) for a, b in pairs)
+            assert worst <= 2 * eps + 1e-9, (f"loop {t} row {i}: route {g} vs the oracle's {o} with a logit "
+                                             f"gap {worst:.3e} beyond the row's drift 2 x {eps:.3e}")
+            n += 1
+    return n
+
+
 MAX_FORCED_FRAC = 0.02   # bf16: at most this share of positions may halt one loop apart from the oracle
 
 
@@ -123,7 +163,7 @@ def check_forced_halts(forced: torch.Tensor, t_star: torch.Tensor, cum_oracle: t
                            f"{dist[far].min():.3e} from the threshold (margin {margin:.3e})")
 
 
-def oracle_following_halts(run, hw_gpu: torch.Tensor, p_gpu: torch.Tensor, thr: float, max_rounds: int = 3):
+def oracle_following_halts(run, ids_gpu: torch.Tensor, p_gpu: torch.Tensor, thr: float, max_rounds: int = 10):
     """Run the oracle (`run(halt_at, record)` -> (h_out, hw, ids, kv)) so that it takes the
     GPU's halting loop at the positions where the halting decision was decided by rounding.
 
@@ -133,8 +173,9 @@ def oracle_following_halts(run, hw_gpu: torch.Tensor, p_gpu: torch.Tensor, thr: 
     halting loop imposed on the disagreeing positions (halt_at), which keeps every position
     comparable end to end.  Each imposed position must have been a near-tie: the oracle's
     cum + p within the rounding drift (halt_margin, measured on the aligned run) of thr.
+    Halting loops are read from the expert ids (halting_loop_ids).
     Returns (oracle outputs, record, number of imposed positions, margin)."""
-    hg = halting_loop(hw_gpu)
+    hg = halting_loop_ids(ids_gpu)
     N = hg.numel()
     halt_at = torch.full((N,), -1, dtype=torch.int64)
     t_star = torch.zeros(N, dtype=torch.int64)
@@ -142,7 +183,7 @@ def oracle_following_halts(run, hw_gpu: torch.Tensor, p_gpu: torch.Tensor, thr: 
     for _ in range(max_rounds):
         rec = []
         out = run(halt_at if (halt_at >= 0).any() else None, rec)
-        ho = halting_loop(out[1])
+        ho = halting_loop_ids(out[2])
         cum = torch.stack([r["cum"] for r in rec])
         if cum_first is None:
             cum_first = cum
@@ -152,7 +193,10 @@ def oracle_following_halts(run, hw_gpu: torch.Tensor, p_gpu: torch.Tensor, thr: 
         t_star[new] = torch.minimum(hg, ho)[new]
         halt_at[new] = hg[new]
     forced = torch.nonzero(halt_at >= 0)[:, 0]
-    assert torch.equal(halting_loop(out[1]), hg), "the oracle does not follow the imposed halting loops"
+    ho = halting_loop_ids(out[2])
+    left = ho != hg
+    assert not left.any(), (f"the oracle still halts {int(left.sum())} positions at another loop after imposing "
+                            f"{int((halt_at >= 0).sum())} (forced still differing: {int((left & (halt_at >= 0)).sum())})")
     margin = halt_margin(p_gpu, torch.stack([r["p"] for r in rec]), hg)
     check_forced_halts(forced, t_star[forced], cum, thr, margin, N)
     return out, rec, int(forced.numel()), margin

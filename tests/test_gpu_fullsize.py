@@ -8,7 +8,8 @@ import torch
 
 import rdt_inputs as RI
 from oracle import rdt_oracle as O
-from tests._helpers import BF16_TOL, ID_MARGIN, halting_loop, rel_l2, teacher_forced_ids, topk_margin
+from tests._helpers import (BF16_TOL, ID_MARGIN, check_route_flips, halting_loop, rel_l2, teacher_forced_ids,
+                            topk_margin)
 
 pytestmark = pytest.mark.gpu
 
@@ -42,7 +43,12 @@ def test_rdt1b_prefill_prefix_slice_matches_oracle():
     torch.cuda.synchronize()
     assert blk.read_status() == 0
     Wc = _cpu(W)
-    o_h, o_hw, o_ids, _ = O.recurrent_forward(cfg, Wc, h0[:P].cpu(), e[:P].cpu(), 1, L, wl.act_threshold)
+    # the oracle takes the GPU's routes where they differ from its own by a near-tie that the
+    # row's logit drift explains (check_route_flips), so both follow one discrete path
+    rec = []
+    o_h, o_hw, o_ids, _ = O.recurrent_forward(cfg, Wc, h0[:P].cpu(), e[:P].cpu(), 1, L, wl.act_threshold,
+                                              record=rec, route_ids=ids[:, :P].cpu().long())
+    check_route_flips(ids[:, :P], tr.biased_logits, rec)
     assert rel_l2(h_out[:P], o_h) <= BF16_TOL
     n, bad, skipped = teacher_forced_ids(cfg, Wc, tr, ids, L)
     assert n > 0 and bad == 0, f"{bad} of {n} teacher-forced rows differ ({skipped} near-ties skipped)"
@@ -167,11 +173,14 @@ def test_rdt10b_zipf_prefill_matches_oracle():
     Wc = _cpu(W)
     del W, blk
     torch.cuda.empty_cache()
+    rec = []
     o_h, o_hw, o_ids, _ = O.recurrent_forward(cfg, Wc, h0[:P].cpu(), e[:P].cpu(), 1, L, wl.act_threshold,
-                                              halt_logit_offset=off[:P])
+                                              halt_logit_offset=off[:P], record=rec,
+                                              route_ids=ids_c[:, :P].long())
+    n_flip = check_route_flips(ids_c[:, :P], tr.biased_logits, rec)
     assert torch.equal(halting_loop(o_hw), last[:P])
     err = rel_l2(h_p, o_h)
-    assert err <= BF16_TOL, f"relative L2 of h_out over the prefix {err:.3e}"
+    assert err <= BF16_TOL, f"relative L2 of h_out over the prefix {err:.3e} ({n_flip} near-tie routes aligned)"
 
 
 def test_rdt3b_mla_decode_sequence_matches_oracle():
@@ -231,12 +240,18 @@ def test_generation_teacher_forced(shape):
     MW = RI.model_weights(cfg, wl.seed, device=dev, halt_b=halt_b)
     B, T0, new = 2, 24, 3
     prompt = torch.randint(0, cfg.vocab_size, (B, T0), generator=torch.Generator().manual_seed(11))
-    gen = R.Generator(cfg, MW, B, T0, new, L, thr)
+    gen = R.Generator(cfg, MW, B, T0, new, L, thr, trace=True)
     gen.prefill(prompt.to(device=dev, dtype=torch.int32).contiguous())
+    b = 0
     logits = [gen.logits.clone()]
+    # the recurrent block's routes and biased logits of sequence b at every position
+    routes = [gen.rec_out[2][:, b * T0:(b + 1) * T0].clone()]
+    biased = [gen.trace_prefill.biased_logits[:, b * T0:(b + 1) * T0].clone()]
     for s in range(1, new):
         gen.decode(s)
         logits.append(gen.logits.clone())
+        routes.append(gen.dec_out[2][:, b:b + 1].clone())
+        biased.append(gen.trace_decode.biased_logits[:, b:b + 1].clone())
     torch.cuda.synchronize()
     toks = gen.tokens.t().cpu().long()
     seq = torch.cat([prompt, toks], dim=1)
@@ -244,8 +259,10 @@ def test_generation_teacher_forced(shape):
                ({kk: vv.cpu() for kk, vv in v.items()} if isinstance(v, dict) else v.cpu())) for k, v in MW.items()}
     del gen, MW
     torch.cuda.empty_cache()
-    b = 0
-    full, _, _ = O.model_forward(cfg, MWc, seq[b:b + 1, :-1], L, thr)
+    route_ids = torch.cat(routes, 1).cpu().long()           # [L, T0 + new - 1, k]
+    rec = []
+    full, _, _ = O.model_forward(cfg, MWc, seq[b:b + 1, :-1], L, thr, route_ids=route_ids, record=rec)
+    check_route_flips(route_ids, torch.cat(biased, 1), rec)
     for s in range(new):
         ol = full[0, T0 - 1 + s]
         gl = logits[s][b].cpu()

@@ -138,7 +138,7 @@ def test_recurrent_bf16_matches_oracle(name, variant):
     torch.cuda.synchronize()
     assert blk.read_status() == 0
     run = lambda halt_at, rec: O.recurrent_forward(cfg, W, h0, e, B, L, thr, record=rec, halt_at=halt_at)
-    (o_h, o_hw, o_ids, _), rec, n_forced, margin = oracle_following_halts(run, hw, tr.p, thr)
+    (o_h, o_hw, o_ids, _), rec, n_forced, margin = oracle_following_halts(run, ids, tr.p, thr)
     _bf16_compare(cfg, W, h_out, hw, ids, tr, o_h, L)
     errs = _teacher_forced_states(cfg, W, tr, e, B, L, ids, hw)
     assert max(errs) <= BF16_TOL, f"per-loop teacher-forced relative L2 {errs}"

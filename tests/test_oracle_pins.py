@@ -95,7 +95,7 @@ def test_router_gates_are_softmax_of_selected_logits():
     cfg = tiny_cfg()
     W = weights(cfg)
     f = torch.randn(32, cfg.dim, dtype=F64, generator=torch.Generator().manual_seed(1))
-    idx, g, logits, _ = O.router(cfg, W, f)
+    idx, g, logits, _, _ = O.router(cfg, W, f)
     sel = torch.gather(logits, 1, idx)
     assert torch.allclose(g, torch.softmax(sel, -1), atol=1e-14)
     assert torch.allclose(g.sum(-1), torch.ones(32, dtype=F64), atol=1e-14)
@@ -451,7 +451,7 @@ def test_router_bias_selects_but_does_not_weight():
     W = weights(cfg)
     W["router_bias"] = torch.tensor([0, 0, 0, 0, 0, 50.0, 0, 40.0])   # force experts 5 and 7
     f = torch.randn(16, cfg.dim, dtype=F64, generator=torch.Generator().manual_seed(18))
-    idx, g, logits, _ = O.router(cfg, W, f)
+    idx, g, logits, _, _ = O.router(cfg, W, f)
     assert (idx[:, 0] == 5).all() and (idx[:, 1] == 7).all()
     sc = torch.softmax(Fn.linear(f, W["w_router"].double()), -1)[:, [5, 7]]
     assert torch.allclose(g, sc / sc.sum(-1, keepdim=True), atol=1e-14)
@@ -594,3 +594,44 @@ def test_model_forward_coda_layers_after_the_recurrent_block():
         z = _lib_ffn_block(W, z, cfg.norm_eps)
     z = O.recurrent_forward(cfg, MW["recurrent"], z, x, 2, L, thr)[0]
     assert (_lib_head(cfg, MW, z).reshape(2, 7, -1) - logits).abs().max() > 1e-6
+
+
+# ------------------------------------------------------------------------------------------
+# 11. successive decode steps (what continuous depth-wise batching computes) equal the
+#     prefill of the token block over the same cache prefix (causality: "OpenMythos 분석",
+#     RoPE & generation cache), with tokens halting at different depths (ACT)
+# ------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("attn", ["gqa", "mla"])
+def test_decode_tokens_equal_prefill_of_the_token_block(attn):
+    name = "tiny_gqa_fp32" if attn == "gqa" else "tiny_mla_fp32"
+    cfg = RI.get_workload(name).cfg
+    W = RI.block_weights(cfg, 8, attn_std=0.08, halt_w_std=0.0, halt_b=0.0)
+    B, C, S, L, thr = 2, 5, 4, 6, 0.99
+    g = torch.Generator().manual_seed(8)
+    caches = []
+    for t in range(L):
+        per_seq = []
+        for b in range(B):
+            if attn == "gqa":
+                per_seq.append({"k": torch.randn(C, cfg.n_kv_heads, cfg.head_dim, generator=g, dtype=F64),
+                                "v": torch.randn(C, cfg.n_kv_heads, cfg.head_dim, generator=g, dtype=F64),
+                                "pos": torch.arange(C)})
+            else:
+                per_seq.append({"c_kv": torch.randn(C, cfg.kv_lora_rank, generator=g, dtype=F64),
+                                "k_rope": torch.randn(C, cfg.qk_rope_head_dim, generator=g, dtype=F64),
+                                "pos": torch.arange(C)})
+        caches.append(per_seq)
+    h0, e = RI.recurrent_inputs(cfg, B, S, 8)
+    off, kk = RI.halting_offsets_spread(B * S, 2, L, thr, 8)      # token i halts after kk[i] loops
+    D = cfg.dim
+    got_h, got_hw, got_ids = O.decode_tokens(cfg, W, h0.view(B, S, D), e.view(B, S, D), caches, [C] * B, L, thr,
+                                             off.view(B, S))
+    want_h, want_hw, want_ids, _ = O.recurrent_forward(cfg, W, h0, e, B, L, thr, start_pos=C,
+                                                       halt_logit_offset=off, caches=caches)
+    assert torch.allclose(got_h.reshape(B * S, D), want_h, rtol=1e-10, atol=1e-11)
+    assert torch.allclose(got_hw.reshape(B * S, L).T, want_hw, rtol=0, atol=1e-12)
+    assert torch.equal(got_ids.reshape(B * S, L, -1).transpose(0, 1), want_ids)
+    # the halting spread: token i's last non-zero weight is at loop kk[i] - 1
+    last = ((got_hw.reshape(B * S, L) > 0).to(torch.int64) * torch.arange(L)).max(-1).values
+    assert torch.equal(last + 1, kk) and len(set(kk.tolist())) > 1

@@ -4,8 +4,8 @@ import math
 import pytest
 import torch
 
-from tests._helpers import (check_forced_halts, halt_margin, halting_loop, oracle_following_halts,
-                            topk_margin)
+from tests._helpers import (check_forced_halts, check_route_flips, halt_margin, halting_loop, halting_loop_ids,
+                            oracle_following_halts, topk_margin)
 
 
 def _hw(loops, L=3):
@@ -45,6 +45,55 @@ def test_too_many_forced_halts_fail():
                            max_frac=0.2)
 
 
+def _ids(loops, L=3):
+    """Expert ids [L, N, 1] of positions halting at loop loops[i] (-1 after the halt)."""
+    ids = torch.full((L, len(loops), 1), -1, dtype=torch.int64)
+    for i, t in enumerate(loops):
+        ids[: t + 1, i] = 0
+    return ids
+
+
+def test_halting_loop_from_ids_is_exact_with_a_zero_remainder():
+    hw = torch.tensor([[0.6], [0.5], [0.0]])          # halts at loop 2 with remainder max(1 - 1.1, 0) = 0
+    assert halting_loop(hw).tolist() == [1]
+    assert halting_loop_ids(_ids([2])).tolist() == [2]
+
+
+def test_route_flip_within_the_row_drift_is_accepted_and_beyond_it_fails():
+    record = [{"own_ids": torch.tensor([[0, 1], [2, 3]]),
+               "biased": torch.tensor([[3.0, 2.0, 1.99, 0.0], [0.0, 0.0, 5.0, 4.0]], dtype=torch.float64)}]
+    gpu_ids = torch.tensor([[[0, 2], [2, 3]]])            # row 0: expert 2 instead of 1 (oracle gap 0.01)
+    near = torch.tensor([[[3.0, 2.0, 2.0049, 0.0], [0.0, 0.0, 5.0, 4.0]]])   # row drift 0.0051: explained
+    assert check_route_flips(gpu_ids, near, record) == 1
+    far = torch.tensor([[[3.0, 2.0, 1.9920, 0.0], [0.0, 0.0, 5.0, 4.0]]])    # drift 0.002 < gap / 2
+    with pytest.raises(AssertionError):
+        check_route_flips(gpu_ids, far, record)
+    swapped = torch.tensor([[[1, 0], [2, 3]]])           # same experts, order inverted (gap 1.0)
+    with pytest.raises(AssertionError):
+        check_route_flips(swapped, near, record)
+
+
+def test_oracle_route_hook_imposes_the_given_experts():
+    import rdt_inputs as RI
+    from oracle import rdt_oracle as O
+    cfg = RI.get_workload("tiny_gqa_fp32").cfg
+    W = RI.block_weights(cfg, 4)
+    h0, e = RI.recurrent_inputs(cfg, 1, 6, 4)
+    rec = []
+    base = O.recurrent_forward(cfg, W, h0, e, 1, 3, 0.0, record=rec)
+    same = O.recurrent_forward(cfg, W, h0, e, 1, 3, 0.0, route_ids=base[2])
+    assert torch.equal(base[0], same[0]) and torch.equal(base[2], same[2])
+    route = base[2].clone()
+    route[1, 2] = torch.tensor([7, 6])                   # loop 1, position 2: other experts
+    rec2 = []
+    moved = O.recurrent_forward(cfg, W, h0, e, 1, 3, 0.0, record=rec2, route_ids=route)
+    assert moved[2][1, 2].tolist() == [7, 6] and torch.equal(rec2[1]["own_ids"][2], base[2][1, 2])
+    assert not torch.equal(moved[0][2], base[0][2])
+    # earlier positions untouched (causal; the expert matmuls group rows differently, hence
+    # agreement to rounding rather than bit for bit)
+    assert torch.allclose(moved[0][:2], base[0][:2], rtol=1e-12, atol=1e-12)
+
+
 def test_oracle_is_rerun_on_the_gpu_halting_loop_of_a_near_tie():
     """A planted oracle whose position 1 reaches the threshold at loop 1 by 0.001 while the
     GPU halts it at loop 2: the helper reruns it with that halt imposed."""
@@ -58,10 +107,10 @@ def test_oracle_is_rerun_on_the_gpu_halting_loop_of_a_near_tie():
         cum = torch.cumsum(p, 0)
         for t in range(L):
             rec.append({"p": p[t], "cum": cum[t]})
-        return None, _hw(loops), None, None
+        return None, _hw(loops), _ids(loops), None
 
     p_gpu = torch.tensor([[0.3, 0.5, 0.3], [0.3, 0.4895, 0.3], [0.3, 0.3, 0.3]], dtype=torch.float64)
-    out, rec, n_forced, margin = oracle_following_halts(run, _hw([2, 2, 2]), p_gpu, thr)
+    out, rec, n_forced, margin = oracle_following_halts(run, _ids([2, 2, 2]), p_gpu, thr)
     assert n_forced == 1 and calls[0] is None and calls[1].tolist() == [-1, 2, -1]
     assert margin == pytest.approx(3 * 0.0015)
     assert halting_loop(out[1]).tolist() == [2, 2, 2]
