@@ -363,6 +363,7 @@ def run_ours(args, wl, rank, world, local_rank):
     mla_res = None if args.no_decode or args.no_mla_decode else run_decode(args, rank, world, local_rank,
                                                                              "rdt3b_mla_decode")
     gen_res = None if args.no_decode or args.no_generate else run_generate(args, rank, world, local_rank)
+    depth_res = None if args.no_decode or args.no_depth else run_depth_decode(args, rank, world, local_rank)
     if rank != 0:
         return
     cfg = wl.cfg
@@ -403,6 +404,11 @@ def run_ours(args, wl, rank, world, local_rank):
         res["decode_mla_tokens_per_s"] = mla_res["value"]
         res["decode_mla_hbm_frac"] = mla_res["roofline"]["frac"]
         res["decode_mla_attention_hbm_frac"] = mla_res["attention_roofline"]["frac"]
+    if depth_res is not None:
+        res["depth_batch"] = depth_res
+        res["depth_batch_tokens_per_s"] = depth_res["depth_batch_tokens_per_s"]
+        res["depth_batch_lockstep_tokens_per_s"] = depth_res["lockstep_tokens_per_s"]
+        res["depth_batch_speedup"] = depth_res["speedup"]
     if gen_res is not None:
         res["generate"] = gen_res
         res["generate_tokens_per_s"] = gen_res["value"]
@@ -549,6 +555,98 @@ def run_decode(args, rank, world, local_rank, name="rdt3b_decode"):
     return res
 
 
+def run_depth_decode(args, rank, world, local_rank, name="rdt3b_decode_halting"):
+    """Continuous depth-wise batching against lockstep decode steps on the 3B-shaped decode
+    with a 4..16-loop halting spread: 64 sequences decode S tokens each, first as S lockstep
+    steps (every step runs all 16 loops; halted rows skip the experts but keep their slot;
+    replayed from a CUDA graph), then through DepthBatch (a token leaves its slot when it
+    halts and the sequence's next token takes it; ticks replayed from a CUDA graph).  Both
+    write the same caches; the outputs are compared."""
+    import recurrent_depth_moe_b200 as R
+    from recurrent_depth_moe_b200 import _native as NAT
+    dev = torch.device("cuda", local_rank)
+    wl = RI.get_workload(name)
+    cfg = wl.cfg
+    B, L, S, thr = wl.batch, wl.n_loops, args.depth_tokens or wl.decode_steps, wl.act_threshold
+    t_max = wl.cache_len + S + 8
+    seed = REP.replica_input_seed(wl.seed, rank)
+    W = RI.block_weights(cfg, wl.seed, device=dev, halt_w_std=0.0, halt_b=0.0)
+    k, v = RI.random_kv_cache(cfg, L, B, t_max, wl.cache_len, seed, device=dev)
+    h0, e = RI.recurrent_inputs(cfg, B, S, seed, device=dev)
+    h0, e = h0.view(B, S, cfg.dim), e.view(B, S, cfg.dim)
+    off, kk = RI.halting_offsets_spread(B * S, wl.halt_spread[0], wl.halt_spread[1], thr, seed)
+    off = off.view(B, S).to(dev)
+    steps_in = [(h0[:, n].contiguous(), e[:, n].contiguous(), off[:, n].contiguous()) for n in range(S)]
+    blk = R.RecurrentBlock(cfg, W)
+    cache = R.KVCache(k, v)
+    stream = torch.cuda.current_stream()
+    # lockstep decode steps
+    clen = torch.full((B,), wl.cache_len, dtype=torch.int32, device=dev)
+    dg = R.DecodeGraph(blk, B, cache, clen, L, thr, halt_logit_offset=True)
+    for n in range(2):                       # eager step, then the captured one
+        dg.step(*steps_in[n])
+    torch.cuda.synchronize()
+    clen.fill_(wl.cache_len)
+    lock_h = torch.empty(B, S, cfg.dim, dtype=torch.float32, device=dev)
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for n in range(S):
+        lock_h[:, n].copy_(dg.step(*steps_in[n])[0])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    lock_ms = REP.max_over_ranks(e0.elapsed_time(e1), device=dev)
+    assert blk.read_status() == 0
+    # depth-batched
+    clen0 = torch.full((B,), wl.cache_len, dtype=torch.int32, device=dev)
+    db = R.DepthBatch(blk, h0, e, clen0, cache, L, thr, off)
+    check_every = 16
+    db.run(check_every=check_every, cuda_graph=True)             # warm-up (captures the tick graph)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    out = db.run(check_every=check_every, cuda_graph=True)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    depth_ms = REP.max_over_ranks(e2.elapsed_time(e3), device=dev)
+    assert db.read_status() == 0
+    ticks = db.ticks
+    diff = float((out[0] - lock_h).norm() / lock_h.norm())
+    # per-class breakdown of the depth-batched run (eager, profiled; not timed)
+    NAT.profile_start()
+    n0 = NAT.launch_count()
+    db.run(check_every=check_every)
+    torch.cuda.synchronize()
+    launches = NAT.launch_count() - n0
+    prof = NAT.profile_stop()
+    mean_loops = float(kk.double().mean())
+    tokens = B * S * world
+    res = {"metric": "decode tokens/s, continuous depth-wise batching vs lockstep steps",
+           "workload": (f"{wl.name}: 3B-shaped KV-cached decode (dim {cfg.dim}, {cfg.n_heads} heads GQA "
+                        f"({cfg.n_kv_heads} kv), {cfg.n_experts} routed + {cfg.n_shared_experts} shared experts "
+                        f"top-{cfg.n_experts_per_tok}, expert_dim {cfg.expert_dim}, {L} loops), {B} sequences "
+                        f"with {wl.cache_len}-token random caches per loop, {S} new tokens each, bf16, ACT "
+                        f"{thr} with per-token halting spread over {wl.halt_spread[0]}-{wl.halt_spread[1]} loops "
+                        f"(mean {mean_loops:.2f})"),
+           "depth_batch_tokens_per_s": tokens / (depth_ms / 1e3), "depth_batch_ms": depth_ms,
+           "depth_batch_ticks": ticks, "depth_batch_ms_per_tick": depth_ms / max(ticks, 1),
+           "lockstep_tokens_per_s": tokens / (lock_ms / 1e3), "lockstep_ms": lock_ms,
+           "lockstep_ms_per_step": lock_ms / S,
+           "speedup": lock_ms / depth_ms, "ideal_speedup": L / mean_loops,
+           "mean_loops_per_token": mean_loops, "executed_token_loops": float(kk.sum()) * world,
+           "max_rel_l2_depth_vs_lockstep_h_out": diff,
+           "cuda_graph": {"ticks_per_replay": check_every, "launches_per_replay": db.graph_launches,
+                          "lockstep_launches_per_step": dg.graph_launches},
+           "gpu_launches_eager_run": launches,
+           "kernel_ms_eager_run": {k2: {"launches": v2[0], "ms": v2[1]} for k2, v2 in sorted(prof.items())}}
+    del db, dg, cache, k, v, W, blk
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_generate(args, rank, world, local_rank):
     """1B-shaped greedy generation through the library's Generator: the prompt pass
     (embedding, prelude, 16-loop recurrent prefill filling the caches, coda, head of the
@@ -649,10 +747,14 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=128)
     ap.add_argument("--no-mla-decode", action="store_true", help="skip the multi-latent-attention decode line")
     ap.add_argument("--no-generate", action="store_true", help="skip the 1B-shaped generation line")
+    ap.add_argument("--no-depth", action="store_true", help="skip the depth-wise batching decode line")
+    ap.add_argument("--depth-only", action="store_true", help="profiling: run only the depth-wise batching line")
+    ap.add_argument("--depth-tokens", type=int, default=None, help="tokens per sequence of the depth-wise line")
     ap.add_argument("--generate-only", action="store_true", help="profiling: run only the generation line")
     ap.add_argument("--generate-new", type=int, default=None, help="profiling: new tokens per generation")
     ap.add_argument("--decode-only", default=None,
-                    choices=["rdt3b_decode", "rdt3b_mla_decode", "mla_decode_attn_small"],
+                    choices=["rdt3b_decode", "rdt3b_mla_decode", "mla_decode_attn_small", "decode_attn_small",
+                             "decode_moe_small"],
                     help="profiling: run only this decode workload and print its line")
     ap.add_argument("--workload", default=WORKLOAD, choices=["rdt1b_prefill", "rdt10b_prefill_zipf"])
     ap.add_argument("--batch", type=int, default=None, help="override the sequences per step (small profiling cases)")
@@ -682,8 +784,9 @@ def main():
     if world > 1:
         torch.distributed.barrier()
     try:
-        if args.decode_only or args.generate_only:
+        if args.decode_only or args.generate_only or args.depth_only:
             res = (run_generate(args, rank, world, local_rank) if args.generate_only else
+                   run_depth_decode(args, rank, world, local_rank) if args.depth_only else
                    run_decode(args, rank, world, local_rank, args.decode_only))
             if rank == 0:
                 print(json.dumps(res), flush=True)

@@ -191,15 +191,17 @@ RDT_API rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_we
                                      const rdt_kv_cache* cache,
                                      void* ws, size_t ws_bytes, void* stream);
 
-/* rdt_recurrent_decode_step with a per-loop trace of a row range (tests: the router
- * input f and biased logits per loop, for teacher-forced checks of the decode step's
- * routes).  trace may be NULL, which makes it rdt_recurrent_decode_step. */
-RDT_API rdt_status rdt_recurrent_decode_step_traced(const rdt_config* cfg, const rdt_weights* w,
-                                            const float* h0, const void* e, int batch,
-                                            const int32_t* cache_len, int n_loops, float act_threshold,
-                                            float* h_out, float* halt_weights, int32_t* expert_ids,
-                                            const rdt_kv_cache* cache, const rdt_trace* trace,
-                                            void* ws, size_t ws_bytes, void* stream);
+/* rdt_recurrent_decode_step with the optional arguments of rdt_recurrent_forward:
+ * halt_logit_offset (NULL or [batch] fp32 added to the halting logit) and a per-loop trace
+ * of a row range (tests: the router input f and biased logits per loop, for teacher-forced
+ * checks of the decode step's routes).  Both NULL: rdt_recurrent_decode_step. */
+RDT_API rdt_status rdt_recurrent_decode_step_ex(const rdt_config* cfg, const rdt_weights* w,
+                                        const float* h0, const void* e, int batch,
+                                        const int32_t* cache_len, int n_loops, float act_threshold,
+                                        const float* halt_logit_offset,
+                                        float* h_out, float* halt_weights, int32_t* expert_ids,
+                                        const rdt_kv_cache* cache, const rdt_trace* trace,
+                                        void* ws, size_t ws_bytes, void* stream);
 
 /* Decode step without a caller workspace, for callers that cannot allocate device
  * memory (a warm serving loop that must not allocate, a host runtime without a CUDA
@@ -232,6 +234,53 @@ RDT_API rdt_status rdt_recurrent_decode_step_static(const rdt_config* cfg, const
  * scratch used by rdt_recurrent_decode_step_static on the current device (as
  * rdt_read_device_status does for a caller workspace).  Allocates nothing. */
 RDT_API rdt_status rdt_read_static_status(void* stream);
+
+/* ---- continuous depth-wise batching of decode steps --------------------------------------
+ * GeekNews summary, section 6: with ACT ("OpenMythos 분석", ACT) a token may leave the shared
+ * block after fewer loops; continuous depth-wise batching lets it leave its batch slot there
+ * and puts new work in its place.  Here the work is decode: `batch` sequences each decode
+ * `n_tokens` tokens in order.  One slot per sequence; a tick runs the shared block once
+ * over all slots, each slot's token at its own loop (its own loop embedding, LoRA scale row,
+ * loop cache and last-loop flag).  A token that halts, or has run n_loops loops, leaves its
+ * slot: the keys / values of its remaining loops are computed from its frozen state and
+ * written into those loop caches (later tokens of the sequence attend to it there, as in a
+ * lockstep decode step), and the slot takes the sequence's next token at loop 0.  The results
+ * equal n_tokens successive rdt_recurrent_decode_step calls on each sequence (token n at
+ * position cache_len[b] + n); the work per tick stays a full batch while tokens halt early.
+ * GQA caches only (RDT_ERR_UNSUPPORTED for MLA).  All pointers are caller-owned device memory. */
+typedef struct {
+  const rdt_config* cfg;           /* host */
+  const rdt_weights* w;            /* host struct of device pointers                         */
+  const float* h0;                 /* [batch][n_tokens][D] fp32: token n of sequence b         */
+  const void* e;                   /* [batch][n_tokens][D] model dtype                         */
+  const float* halt_logit_offset;  /* NULL or [batch][n_tokens] fp32, added to the halting logit */
+  const int32_t* cache_len;        /* [batch] int32: position of token 0 of sequence b; the   */
+                                   /* tokens of b sit at cache_len[b] .. cache_len[b]+n_tokens-1 */
+  int batch, n_tokens, n_loops;
+  float act_threshold;             /* <= 0: ACT off (every token runs n_loops loops)           */
+  float* h_out;                    /* [batch][n_tokens][D] fp32                                */
+  float* halt_weights;             /* [batch][n_tokens][n_loops] fp32 (0 after a token halts)  */
+  int32_t* expert_ids;             /* [batch][n_tokens][n_loops][top_k] (-1 after it halts)    */
+  const rdt_kv_cache* cache;       /* host struct: GQA loop caches, n_loops >= n_loops, batch */
+                                   /* >= batch, t_max >= every cache_len[b] + n_tokens         */
+  void* ws; size_t ws_bytes;       /* >= rdt_depth_batch_workspace_size, 256-byte aligned;     */
+                                   /* holds the slots' state between calls                     */
+} rdt_depth_batch;
+
+/* Workspace bytes of a depth-batched decode of `batch` sequences (0 for an invalid config). */
+RDT_API size_t rdt_depth_batch_workspace_size(const rdt_config* cfg, int batch, int n_loops, int t_max);
+/* Clear the outputs and the device status word, put token 0 of every sequence in its slot. */
+RDT_API rdt_status rdt_depth_batch_begin(const rdt_depth_batch* db, void* stream);
+/* Enqueue n_ticks ticks (asynchronous; every kernel argument is a function of *db, so a
+ * stream capture of a tick replays correctly while *db stays the same).  Ticks after every
+ * token finished do no work on the outputs. */
+RDT_API rdt_status rdt_depth_batch_tick(const rdt_depth_batch* db, int n_ticks, void* stream);
+/* Synchronise `stream` and return the number of tokens not yet finished (-1: CUDA error). */
+RDT_API long long rdt_depth_batch_pending(const rdt_depth_batch* db, void* stream);
+/* begin, then ticks in chunks of check_every (reading the pending count after each chunk,
+ * which synchronises `stream`) until every token finished.  Device errors are recorded in
+ * the status word of ws (rdt_read_device_status). */
+RDT_API rdt_status rdt_depth_batch_run(const rdt_depth_batch* db, int check_every, void* stream);
 
 /* One pre-norm TransformerBlock: x_out = x1 + FFN(RMSNorm(x1)), x1 = x_in + Attn(RMSNorm(x_in)).
  * FFN is the MoE when cfg->n_experts > 0, else the dense SwiGLU in w13/w2 expert 0

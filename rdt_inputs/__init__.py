@@ -140,6 +140,15 @@ WORKLOADS = {
         attn_type="mla", kv_lora_rank=512, q_lora_rank=1536, qk_rope_head_dim=64, qk_nope_head_dim=128,
         v_head_dim=128, dtype="bf16"), batch=64, seq=1, n_loops=16, seed=5, act_threshold=0.0, kind="decode",
         cache_len=4096, decode_steps=128, device_weights=True),
+    # The 3B-shaped decode with ACT on and a per-token halting spread over 4..16 loops (zero
+    # halting head, per-token logit offsets as in the 10B prefill): the workload on which
+    # continuous depth-wise batching is compared with lockstep decode steps.  64 sequences,
+    # 64 new tokens each.
+    "rdt3b_decode_halting": Workload("rdt3b_decode_halting", RDTConfig(
+        dim=3072, n_heads=24, n_kv_heads=8, max_seq_len=4096 + 128, max_loop_iters=16,
+        n_experts=64, n_shared_experts=1, n_experts_per_tok=4, expert_dim=4096, lora_rank=16,
+        dtype="bf16"), batch=64, seq=1, n_loops=16, seed=9, act_threshold=0.99, kind="decode",
+        halt_spread=(4, 16), cache_len=4096, decode_steps=64, device_weights=True),
     # Greedy generation with the 1B-shaped model: the recurrent block of rdt1b_prefill, one
     # prelude and one coda layer (the usage script's counts; the variant table gives none)
     # and the vocabulary of the tokenizer the pages name (openai/gpt-oss-20b: 201,088
@@ -158,6 +167,22 @@ WORKLOADS = {
         attn_type="mla", kv_lora_rank=512, q_lora_rank=1536, qk_rope_head_dim=64, qk_nope_head_dim=128,
         v_head_dim=128, dtype="bf16"), batch=64, seq=1, n_loops=2, seed=6, act_threshold=0.0, kind="decode",
         cache_len=4096, decode_steps=8, device_weights=True),
+    # Profiling case for the GQA decode attention: the attention of rdt3b_decode (24 heads,
+    # 8 kv heads, 64 sequences, 4096-token caches) with a small MoE and 2 loops (about 2.2 GB
+    # of caches on the device).
+    "decode_attn_small": Workload("decode_attn_small", RDTConfig(
+        dim=3072, n_heads=24, n_kv_heads=8, max_seq_len=4096 + 128, max_loop_iters=2,
+        n_experts=8, n_shared_experts=1, n_experts_per_tok=2, expert_dim=128, lora_rank=16,
+        dtype="bf16"), batch=64, seq=1, n_loops=2, seed=10, act_threshold=0.0, kind="decode",
+        cache_len=4096, decode_steps=8, device_weights=True),
+    # Profiling case for the decode expert GEMMs and routing: the MoE of rdt3b_decode (64
+    # routed + 1 shared experts of width 4096, top-4, 64 sequences) with 1 loop and short
+    # caches (about 5 GB of expert weights on the device).
+    "decode_moe_small": Workload("decode_moe_small", RDTConfig(
+        dim=3072, n_heads=24, n_kv_heads=8, max_seq_len=512, max_loop_iters=1,
+        n_experts=64, n_shared_experts=1, n_experts_per_tok=4, expert_dim=4096, lora_rank=16,
+        dtype="bf16"), batch=64, seq=1, n_loops=1, seed=11, act_threshold=0.0, kind="decode",
+        cache_len=256, decode_steps=8, device_weights=True),
     # 10B-shaped prefill, load-imbalanced (mythos_10b: dim 4096, 128 experts, expert_dim 5632, 24 loops).
     "rdt10b_prefill_zipf": Workload("rdt10b_prefill_zipf", RDTConfig(
         dim=4096, n_heads=32, n_kv_heads=8, max_seq_len=8192, max_loop_iters=24,

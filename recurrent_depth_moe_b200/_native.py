@@ -51,6 +51,13 @@ class rdt_trace(ctypes.Structure):
                 ("biased_logits", c_void_p), ("p", c_void_p)]
 
 
+class rdt_depth_batch(ctypes.Structure):
+    _fields_ = [("cfg", POINTER(rdt_config)), ("w", POINTER(rdt_weights)), ("h0", c_void_p), ("e", c_void_p),
+                ("halt_logit_offset", c_void_p), ("cache_len", c_void_p), ("batch", c_int), ("n_tokens", c_int),
+                ("n_loops", c_int), ("act_threshold", c_float), ("h_out", c_void_p), ("halt_weights", c_void_p),
+                ("expert_ids", c_void_p), ("cache", POINTER(rdt_kv_cache)), ("ws", c_void_p), ("ws_bytes", c_size_t)]
+
+
 class rdt_kernel_time(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", c_int), ("total_ms", ctypes.c_double)]
 
@@ -59,7 +66,9 @@ EXPORTS = ("rdt_workspace_size", "rdt_recurrent_forward", "rdt_recurrent_decode_
            "rdt_block_forward_cached", "rdt_embed", "rdt_head", "rdt_head_rows", "rdt_greedy_tokens",
            "rdt_to_model_dtype", "rdt_read_device_status", "rdt_status_string", "rdt_version",
            "rdt_launch_count", "rdt_profile_start", "rdt_profile_stop", "rdt_recurrent_decode_step_static",
-           "rdt_read_static_status", "rdt_recurrent_decode_step_traced")
+           "rdt_read_static_status", "rdt_recurrent_decode_step_ex",
+           "rdt_depth_batch_workspace_size", "rdt_depth_batch_begin", "rdt_depth_batch_tick",
+           "rdt_depth_batch_pending", "rdt_depth_batch_run")
 
 _lib = None
 _profiling = False
@@ -83,10 +92,21 @@ def load(path: str = LIB_PATH):
     lib.rdt_recurrent_decode_step.argtypes = [POINTER(rdt_config), POINTER(rdt_weights), P, P, c_int, P, c_int,
                                               c_float, P, P, P, POINTER(rdt_kv_cache), P, c_size_t, P]
     lib.rdt_recurrent_decode_step.restype = c_int
-    lib.rdt_recurrent_decode_step_traced.argtypes = [POINTER(rdt_config), POINTER(rdt_weights), P, P, c_int, P,
-                                                     c_int, c_float, P, P, P, POINTER(rdt_kv_cache),
-                                                     POINTER(rdt_trace), P, c_size_t, P]
-    lib.rdt_recurrent_decode_step_traced.restype = c_int
+    lib.rdt_recurrent_decode_step_ex.argtypes = [POINTER(rdt_config), POINTER(rdt_weights), P, P, c_int, P,
+                                                 c_int, c_float, P, P, P, P, POINTER(rdt_kv_cache),
+                                                 POINTER(rdt_trace), P, c_size_t, P]
+    lib.rdt_recurrent_decode_step_ex.restype = c_int
+    lib.rdt_depth_batch_workspace_size.argtypes = [POINTER(rdt_config), c_int, c_int, c_int]
+    lib.rdt_depth_batch_workspace_size.restype = c_size_t
+    for fn in ("rdt_depth_batch_begin",):
+        getattr(lib, fn).argtypes = [POINTER(rdt_depth_batch), P]
+        getattr(lib, fn).restype = c_int
+    lib.rdt_depth_batch_tick.argtypes = [POINTER(rdt_depth_batch), c_int, P]
+    lib.rdt_depth_batch_tick.restype = c_int
+    lib.rdt_depth_batch_pending.argtypes = [POINTER(rdt_depth_batch), P]
+    lib.rdt_depth_batch_pending.restype = ctypes.c_longlong
+    lib.rdt_depth_batch_run.argtypes = [POINTER(rdt_depth_batch), c_int, P]
+    lib.rdt_depth_batch_run.restype = c_int
     lib.rdt_block_forward.argtypes = [POINTER(rdt_config), POINTER(rdt_weights), P, P, c_int, c_int, c_int, P,
                                       c_size_t, P]
     lib.rdt_block_forward.restype = c_int

@@ -222,9 +222,10 @@ class RecurrentBlock:
 
     def decode_step(self, h0: torch.Tensor, e: torch.Tensor, cache_len: torch.Tensor, cache: KVCache,
                     n_loops: int, act_threshold: float = 0.0, out: Optional[tuple] = None,
-                    workspace: Optional[torch.Tensor] = None, trace: Optional[Trace] = None):
+                    workspace: Optional[torch.Tensor] = None, trace: Optional[Trace] = None,
+                    halt_logit_offset: Optional[torch.Tensor] = None):
         """rdt_recurrent_decode_step: one new token per sequence at position cache_len[b]
-        (rdt_recurrent_decode_step_traced when a trace is given)."""
+        (rdt_recurrent_decode_step_ex when a trace or halting-logit offsets are given)."""
         lib = N.load()
         cfg = self.cfg
         B = h0.shape[0]
@@ -237,14 +238,17 @@ class RecurrentBlock:
                    torch.empty(n_loops, B, cfg.n_experts_per_tok, dtype=torch.int32, device=h0.device))
         ws = workspace if workspace is not None else self.workspace(B, 1, cache.t_max)
         cs = cache.struct()
-        if trace is not None:
-            ts = trace.struct()
-            rc = lib.rdt_recurrent_decode_step_traced(ctypes.byref(self.cs), ctypes.byref(self.w.struct),
-                                                      h0.data_ptr(), e.data_ptr(), B, cache_len.data_ptr(), n_loops,
-                                                      float(act_threshold), out[0].data_ptr(), out[1].data_ptr(),
-                                                      out[2].data_ptr(), ctypes.byref(cs), ctypes.byref(ts),
-                                                      ws.data_ptr(), ws.numel(), _stream())
-            N.check("rdt_recurrent_decode_step_traced", rc)
+        if trace is not None or halt_logit_offset is not None:
+            if halt_logit_offset is not None:
+                _check_act(halt_logit_offset, "halt_logit_offset", torch.float32, (B,))
+            ts = trace.struct() if trace is not None else None
+            rc = lib.rdt_recurrent_decode_step_ex(ctypes.byref(self.cs), ctypes.byref(self.w.struct),
+                                                  h0.data_ptr(), e.data_ptr(), B, cache_len.data_ptr(), n_loops,
+                                                  float(act_threshold), _ptr(halt_logit_offset), out[0].data_ptr(),
+                                                  out[1].data_ptr(), out[2].data_ptr(), ctypes.byref(cs),
+                                                  ctypes.byref(ts) if ts is not None else None,
+                                                  ws.data_ptr(), ws.numel(), _stream())
+            N.check("rdt_recurrent_decode_step_ex", rc)
             return out
         rc = lib.rdt_recurrent_decode_step(ctypes.byref(self.cs), ctypes.byref(self.w.struct), h0.data_ptr(),
                                            e.data_ptr(), B, cache_len.data_ptr(), n_loops, float(act_threshold),
@@ -269,7 +273,8 @@ class DecodeGraph:
     run eagerly, since its CUDA events are recorded at launch time."""
 
     def __init__(self, blk: "RecurrentBlock", batch: int, cache: KVCache, cache_len: torch.Tensor, n_loops: int,
-                 act_threshold: float = 0.0, workspace: Optional[torch.Tensor] = None, out: Optional[tuple] = None):
+                 act_threshold: float = 0.0, workspace: Optional[torch.Tensor] = None, out: Optional[tuple] = None,
+                 halt_logit_offset: bool = False):
         cfg = blk.cfg
         self.blk, self.B, self.cache, self.cache_len = blk, batch, cache, cache_len
         self.L, self.thr = n_loops, act_threshold
@@ -280,33 +285,129 @@ class DecodeGraph:
             torch.empty(n_loops, batch, cfg.n_experts_per_tok, dtype=torch.int32, device="cuda"))
         self.h_in = torch.empty(batch, cfg.dim, dtype=torch.float32, device="cuda")
         self.e_in = torch.empty(batch, cfg.dim, dtype=blk.dtype, device="cuda")
+        # per-step halting-logit offsets (copied in before each replay), when the step takes them
+        self.off_in = torch.zeros(batch, dtype=torch.float32, device="cuda") if halt_logit_offset else None
         self._graph = None
         self._eager = 0
         self.graph_launches = 0      # library kernels in one replay
 
-    def _body(self, h0, e):
-        self.blk.decode_step(h0, e, self.cache_len, self.cache, self.L, self.thr, out=self.out, workspace=self.ws)
+    def _body(self, h0, e, off=None):
+        self.blk.decode_step(h0, e, self.cache_len, self.cache, self.L, self.thr, out=self.out, workspace=self.ws,
+                             halt_logit_offset=off)
         self.cache_len.add_(1)
 
-    def step(self, h0: torch.Tensor, e: torch.Tensor) -> tuple:
+    def step(self, h0: torch.Tensor, e: torch.Tensor, halt_logit_offset: Optional[torch.Tensor] = None) -> tuple:
         """One decode step of every sequence; returns (h_out, halt weights, expert ids)."""
+        if (halt_logit_offset is None) != (self.off_in is None):
+            raise ValueError("halt_logit_offset must be given exactly when the graph was built for it")
         if N.profiling() or self._eager == 0:
-            self._body(h0, e)
+            self._body(h0, e, halt_logit_offset)
             self._eager += 1
             return self.out
         self.h_in.copy_(h0)
         self.e_in.copy_(e)
+        if self.off_in is not None:
+            self.off_in.copy_(halt_logit_offset)
         if self._graph is None:
             g = torch.cuda.CUDAGraph()
             n0 = N.launch_count()
             # thread-local capture: other threads of the process (a collective library's
             # watchdog, for one) keep calling CUDA while this thread captures
             with torch.cuda.graph(g, capture_error_mode="thread_local"):
-                self._body(self.h_in, self.e_in)
+                self._body(self.h_in, self.e_in, self.off_in)
             self.graph_launches = N.launch_count() - n0
             self._graph = g
         self._graph.replay()
         return self.out
+
+
+class DepthBatch:
+    """Continuous depth-wise batching of decode steps (rdt_depth_batch_*): `batch` sequences
+    each decode n_tokens tokens in order, one slot per sequence; every tick runs the shared
+    block once over all slots, each slot's token at its own loop, and a token that halts
+    leaves its slot to the sequence's next token (after its remaining loops' keys / values
+    are written from its frozen state).  Results equal n_tokens successive decode_step calls
+    per sequence.  h0 [B, S, D] fp32, e [B, S, D] model dtype, cache_len [B] int32 (position
+    of token 0), halt_logit_offset [B, S] fp32 or None.  Outputs: h_out [B, S, D],
+    halt_weights [B, S, L], expert_ids [B, S, L, k]."""
+
+    def __init__(self, blk: "RecurrentBlock", h0: torch.Tensor, e: torch.Tensor, cache_len: torch.Tensor,
+                 cache: KVCache, n_loops: int, act_threshold: float = 0.0,
+                 halt_logit_offset: Optional[torch.Tensor] = None, out: Optional[tuple] = None,
+                 workspace: Optional[torch.Tensor] = None):
+        lib = N.load()
+        cfg = blk.cfg
+        B, S = h0.shape[0], h0.shape[1]
+        _check_act(h0, "h0", torch.float32, (B, S, cfg.dim))
+        _check_act(e, "e", blk.dtype, (B, S, cfg.dim))
+        _check_act(cache_len, "cache_len", torch.int32, (B,))
+        if halt_logit_offset is not None:
+            _check_act(halt_logit_offset, "halt_logit_offset", torch.float32, (B, S))
+        self.blk, self.B, self.S, self.L = blk, B, S, n_loops
+        self.inputs = (h0, e, cache_len, halt_logit_offset)     # kept alive: the struct holds their addresses
+        self.out = out if out is not None else (
+            torch.empty(B, S, cfg.dim, dtype=torch.float32, device=h0.device),
+            torch.empty(B, S, n_loops, dtype=torch.float32, device=h0.device),
+            torch.empty(B, S, n_loops, cfg.n_experts_per_tok, dtype=torch.int32, device=h0.device))
+        need = int(lib.rdt_depth_batch_workspace_size(ctypes.byref(blk.cs), B, n_loops, cache.t_max))
+        if need == 0:
+            raise N.RdtError("rdt_depth_batch_workspace_size", N.RDT_ERR_INVALID_ARG)
+        self.ws = workspace if workspace is not None and workspace.numel() >= need else alloc_workspace(need)
+        self.cache, self._cs = cache, cache.struct()
+        db = N.rdt_depth_batch()
+        db.cfg, db.w = ctypes.pointer(blk.cs), ctypes.pointer(blk.w.struct)
+        db.h0, db.e, db.halt_logit_offset, db.cache_len = (h0.data_ptr(), e.data_ptr(), _ptr(halt_logit_offset),
+                                                           cache_len.data_ptr())
+        db.batch, db.n_tokens, db.n_loops, db.act_threshold = B, S, n_loops, float(act_threshold)
+        db.h_out, db.halt_weights, db.expert_ids = (o.data_ptr() for o in self.out)
+        db.cache = ctypes.pointer(self._cs)
+        db.ws, db.ws_bytes = self.ws.data_ptr(), self.ws.numel()
+        self.db = db
+        self._graph = None
+        self._graph_ticks = 0
+        self.graph_launches = 0
+        self.ticks = 0
+
+    def begin(self):
+        N.check("rdt_depth_batch_begin", N.load().rdt_depth_batch_begin(ctypes.byref(self.db), _stream()))
+        self.ticks = 0
+
+    def tick(self, n: int = 1):
+        N.check("rdt_depth_batch_tick", N.load().rdt_depth_batch_tick(ctypes.byref(self.db), n, _stream()))
+        self.ticks += n
+
+    def pending(self) -> int:
+        v = int(N.load().rdt_depth_batch_pending(ctypes.byref(self.db), _stream()))
+        if v < 0:
+            raise N.RdtError("rdt_depth_batch_pending", N.RDT_ERR_CUDA)
+        return v
+
+    def run(self, check_every: int = 8, cuda_graph: bool = False) -> tuple:
+        """All tokens: begin, then ticks in chunks of check_every until none is pending.
+        With cuda_graph the first chunk runs eagerly (kernel set-up) and later chunks replay a
+        CUDA graph of check_every ticks captured once."""
+        if not cuda_graph or N.profiling():
+            N.check("rdt_depth_batch_run", N.load().rdt_depth_batch_run(ctypes.byref(self.db), check_every,
+                                                                         _stream()))
+            return self.out
+        self.begin()
+        max_ticks = self.S * self.L
+        self.tick(min(check_every, max_ticks))
+        while self.ticks < max_ticks and self.pending() > 0:
+            if self._graph is None or self._graph_ticks != check_every:
+                g = torch.cuda.CUDAGraph()
+                n0 = N.launch_count()
+                with torch.cuda.graph(g, capture_error_mode="thread_local"):
+                    N.check("rdt_depth_batch_tick", N.load().rdt_depth_batch_tick(ctypes.byref(self.db),
+                                                                                   check_every, _stream()))
+                self.graph_launches = N.launch_count() - n0
+                self._graph, self._graph_ticks = g, check_every
+            self._graph.replay()
+            self.ticks += check_every
+        return self.out
+
+    def read_status(self) -> int:
+        return N.load().rdt_read_device_status(self.ws.data_ptr(), _stream())
 
 
 class Block:
@@ -467,7 +568,7 @@ class Generator:
     call made while the library's profiler is recording."""
 
     def __init__(self, cfg, MW: dict, batch: int, prompt_len: int, max_new_tokens: int, n_loops: int,
-                 act_threshold: float = 0.0, cuda_graph: bool = True):
+                 act_threshold: float = 0.0, cuda_graph: bool = True, trace: bool = False):
         _require_cuda()
         self.cfg, self.MW = cfg, MW
         self.B, self.T0, self.new, self.L, self.thr = batch, prompt_len, max_new_tokens, n_loops, act_threshold
@@ -501,6 +602,10 @@ class Generator:
         self.cache_len = torch.empty(B, dtype=torch.int32, device="cuda")
         self.cur_tok = torch.empty(B, dtype=torch.int32, device="cuda")
         self.cuda_graph = cuda_graph
+        # optional per-loop trace of the recurrent block (tests): every prompt row of the
+        # prefill, every sequence's row of the latest decode step
+        self.trace_prefill = Trace.alloc(cfg, n_loops, 0, B * T0) if trace else None
+        self.trace_decode = Trace.alloc(cfg, n_loops, 0, B) if trace else None
         self._graph = None
         self._eager_decodes = 0
         self.graph_launches = 0      # library kernels in one replay of the captured step
@@ -525,7 +630,7 @@ class Generator:
         x, y = self._run_blocks(self.pre, self.pre_cache, x, y, T0, 0, None)
         to_model_dtype(self.cfg, x, out=self.e)
         self.rb.forward(x, self.e, B, T0, self.L, self.thr, start_pos=0, cache=self.rec_cache, out=self.rec_out,
-                        workspace=self.ws_rec_prefill)
+                        workspace=self.ws_rec_prefill, trace=self.trace_prefill)
         x, y = self._run_blocks(self.coda, self.coda_cache, self.rec_out[0], y, T0, 0, None)
         head(self.cfg, x, self.MW["norm_w"], self.MW["head"], last_of=T0, out=self.logits, workspace=self.ws_head)
         greedy_tokens(self.logits, out=self.tokens[0])
@@ -545,7 +650,7 @@ class Generator:
         to_model_dtype(self.cfg, x, out=e)
         out = self.dec_out
         self.rb.decode_step(x, e, self.cache_len, self.rec_cache, self.L, self.thr, out=out,
-                            workspace=self.ws_rec_decode)
+                            workspace=self.ws_rec_decode, trace=self.trace_decode)
         x, y = self._run_blocks(self.coda, self.coda_cache, out[0], y, 1, 0, self.cache_len)
         head(self.cfg, x, self.MW["norm_w"], self.MW["head"], out=self.logits, workspace=self.ws_head)
         greedy_tokens(self.logits, out=tok_out)

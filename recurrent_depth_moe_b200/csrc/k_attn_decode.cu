@@ -52,8 +52,9 @@ __global__ void __launch_bounds__(128) k_attn_decode(AttnParams p, int n_split, 
     float4 v = V4<T>::ld((const T*)p.q + row * p.q_row + (long long)(g * G + h) * p.q_head + 4 * lane);
     q[h] = make_float4(v.x * p.scale, v.y * p.scale, v.z * p.scale, v.w * p.scale);
   }
-  const T* kb = (const T*)p.k1 + (long long)b * p.k1_b + (long long)g * p.k1_g + 4 * lane;
-  const T* vb = (const T*)p.v + (long long)b * p.v_b + (long long)g * p.v_g + 4 * lane;
+  const long long lp = p.row_loop ? max(p.row_loop[b], 0) : 0;
+  const T* kb = (const T*)p.k1 + lp * p.loop_k + (long long)b * p.k1_b + (long long)g * p.k1_g + 4 * lane;
+  const T* vb = (const T*)p.v + lp * p.loop_v + (long long)b * p.v_b + (long long)g * p.v_g + 4 * lane;
   float m[G], l[G];
   float4 acc[G];
 #pragma unroll
@@ -192,8 +193,11 @@ __global__ void __launch_bounds__(128) k_attn_decode_mma(AttnParams p, int n_spl
   const int j0 = split * chunk;
   const int j1 = min(j0 + chunk, n_vis);
   const int nt = j1 > j0 ? (j1 - j0 + BKV - 1) / BKV : 0;
-  const bf16* kg = (const bf16*)p.k1 + (long long)b * p.k1_b + (long long)g * p.k1_g + (long long)j0 * p.k1_j;
-  const bf16* vg = (const bf16*)p.v + (long long)b * p.v_b + (long long)g * p.v_g + (long long)j0 * p.v_j;
+  const long long lp = p.row_loop ? max(p.row_loop[b], 0) : 0;
+  const bf16* kg = (const bf16*)p.k1 + lp * p.loop_k + (long long)b * p.k1_b + (long long)g * p.k1_g +
+                   (long long)j0 * p.k1_j;
+  const bf16* vg = (const bf16*)p.v + lp * p.loop_v + (long long)b * p.v_b + (long long)g * p.v_g +
+                   (long long)j0 * p.v_j;
   if (nt > 0) {
     load_tile(Ks, kg, p.k1_j, min(BKV, j1 - j0));
     load_tile(Vs, vg, p.v_j, min(BKV, j1 - j0));

@@ -161,9 +161,14 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
   const long long rowD = (long long)i * D;
   const bool lead = (g.wr == 0);
   float4 tr[VQ];
+  // this row's loop and output row (rows at their own depth), else loop p.t and row i
+  const int t = p.t_row ? p.t_row[i] : p.t;
+  const long long wo = p.t_row ? (long long)p.out_row[i] * p.n_loops + t : (long long)t * p.N + i;
+  const long long outD = p.t_row ? (long long)p.out_row[i] * D : rowD;
   if (!p.block_only && p.halted[i]) {   // frozen row: no update, zero weight, no experts
-    if (lead && lane == 0) p.halt_w_out[(long long)p.t * p.N + i] = 0.f;
-    if (lead && lane < p.k) p.ids_out[((long long)p.t * p.N + i) * p.k + lane] = -1;
+    if (p.t_row) return;                // an idle slot: nothing to write
+    if (lead && lane == 0) p.halt_w_out[wo] = 0.f;
+    if (lead && lane < p.k) p.ids_out[wo * p.k + lane] = -1;
     if (p.next_emb) {                   // its keys / values are still recomputed next loop
 #pragma unroll
       for (int j = 0; j < VQ; ++j)
@@ -209,7 +214,7 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
     return;
   }
   if (!p.transformer_off && p.r > 0) {
-    const float* sc = p.lora_scale + (long long)min(p.t, p.max_loop_iters - 1) * p.r;
+    const float* sc = p.lora_scale + (long long)min(t, p.max_loop_iters - 1) * p.r;
     // rank in chunks of 16: partial projections of this warp's columns, one transposed warp
     // reduction, then the group sum; lane q of every warp ends with z[q0 + q]
     for (int q0 = 0; q0 < p.r; q0 += 16) {
@@ -268,7 +273,7 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
     tr[j].w += av.w * hv.w + bv.w * ev.w;
     if (p.act_on) zh += f4_dot(tr[j], __ldg(reinterpret_cast<const float4*>(p.halt_wv + d)));
   }
-  const bool last = (p.t == p.n_loops - 1);
+  const bool last = (t == p.n_loops - 1);
   float w;
   if (p.act_on) {
     zh = g.reduce1(warp_sum(zh), 16, lane);
@@ -289,7 +294,7 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
 #pragma unroll
   for (int j = 0; j < VQ; ++j) {
     const int d = 4 * lane + 128 * (j0 + j);
-    float4* ho = reinterpret_cast<float4*>(p.h_out + rowD + d);
+    float4* ho = reinterpret_cast<float4*>(p.h_out + outD + d);
     if (w != 0.f) {
       float4 o = *ho;
       o.x += w * tr[j].x; o.y += w * tr[j].y; o.z += w * tr[j].z; o.w += w * tr[j].w;
@@ -297,9 +302,8 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
     }
     *reinterpret_cast<float4*>(p.h_state + rowD + d) = tr[j];
   }
-  if (lead && lane == 0) p.halt_w_out[(long long)p.t * p.N + i] = w;
-  if (lead && lane < p.k)
-    p.ids_out[((long long)p.t * p.N + i) * p.k + lane] = p.transformer_off ? -1 : p.ids[(long long)i * p.k + lane];
+  if (lead && lane == 0) p.halt_w_out[wo] = w;
+  if (lead && lane < p.k) p.ids_out[wo * p.k + lane] = p.transformer_off ? -1 : p.ids[(long long)i * p.k + lane];
   if (p.next_emb) next_prologue<T, VQ, WPR>(p, tr, rowD, lane, j0, g);
 }
 

@@ -74,10 +74,12 @@ template <typename T>
 __global__ void k_loop_prologue(const float* __restrict__ h, const T* __restrict__ e,
                                 const float* __restrict__ emb, int loop_dim,
                                 const float* __restrict__ w_rec, const float* __restrict__ w_attn,
-                                float* __restrict__ combined, T* __restrict__ a, int D, float eps) {
+                                float* __restrict__ combined, T* __restrict__ a, int D, float eps,
+                                const int* __restrict__ row_loop, int emb_stride) {
   extern __shared__ float xs[];
   __shared__ float red[32];
   const long long row = blockIdx.x;
+  if (row_loop) emb += (long long)max(row_loop[row], 0) * emb_stride;   // this row's loop embedding
   const float* hr = h + row * D;
   const T* er = e + row * D;
   float ss = 0.f;
@@ -173,10 +175,17 @@ __global__ void k_mla_to_cache(const float* __restrict__ kv_raw, const T* __rest
 template <typename T>
 __global__ void k_kv_to_cache(const T* __restrict__ qkv, long long ld, int k_col, int v_col,
                               int Hkv, int hd, const int* __restrict__ pos, int seq, int t_max,
-                              T* __restrict__ kc, T* __restrict__ vc, DevStatus* st) {
+                              T* __restrict__ kc, T* __restrict__ vc, const int* __restrict__ row_loop,
+                              long long loop_elems, DevStatus* st) {
   const long long row = blockIdx.x;
   const int b = (int)(row / seq);
   const int p = pos[row];
+  if (row_loop) {                       // rows at their own loop depth; < 0: an idle row
+    const int lp = row_loop[row];
+    if (lp < 0) return;
+    kc += lp * loop_elems;
+    vc += lp * loop_elems;
+  }
   if (p < 0 || p >= t_max) {
     if (threadIdx.x == 0) record_status(st, ST_BOUNDS, 101, p);
     return;
@@ -207,9 +216,14 @@ __global__ void k_combine_inject_act(CombineParams p) {
   const int i = blockIdx.x;
   const int D = p.D;
   const int kS = p.k + p.S;
+  // this row's loop and output row (rows at their own depth), else loop p.t and row i
+  const int t = p.t_row ? p.t_row[i] : p.t;
+  const long long wo = p.t_row ? (long long)p.out_row[i] * p.n_loops + t : (long long)t * p.N + i;
+  const long long orow = p.t_row ? (long long)p.out_row[i] : (long long)i;
   if (!p.block_only && p.halted[i]) {   // frozen row
-    if (threadIdx.x == 0) p.halt_w_out[(long long)p.t * p.N + i] = 0.f;
-    for (int j = threadIdx.x; j < p.k; j += blockDim.x) p.ids_out[((long long)p.t * p.N + i) * p.k + j] = -1;
+    if (p.t_row) return;                // an idle slot: nothing to write
+    if (threadIdx.x == 0) p.halt_w_out[wo] = 0.f;
+    for (int j = threadIdx.x; j < p.k; j += blockDim.x) p.ids_out[wo * p.k + j] = -1;
     return;
   }
   const float* x1 = p.x1 + (long long)i * D;
@@ -235,7 +249,7 @@ __global__ void k_combine_inject_act(CombineParams p) {
   if (!p.transformer_off && p.r > 0) {
     const T* Wd = (const T*)p.lora_down;
     const T* Bl = (const T*)p.lora_B;
-    const float* sc = p.lora_scale + (long long)min(p.t, p.max_loop_iters - 1) * p.r;
+    const float* sc = p.lora_scale + (long long)min(t, p.max_loop_iters - 1) * p.r;
     for (int q = 0; q < p.r; ++q) {
       float part = 0.f;
       for (int d = threadIdx.x; d < D; d += blockDim.x) part += tr[d] * to_f(Wd[(long long)q * D + d]);
@@ -258,7 +272,7 @@ __global__ void k_combine_inject_act(CombineParams p) {
     if (p.act_on) zh += hn * p.halt_wv[d];
   }
   float w;
-  const bool last = (p.t == p.n_loops - 1);
+  const bool last = (t == p.n_loops - 1);
   if (p.act_on) {
     zh = block_sum(zh, red);
     float z = zh + p.halt_b[0] + (p.halt_off ? p.halt_off[i] : 0.f);
@@ -275,16 +289,16 @@ __global__ void k_combine_inject_act(CombineParams p) {
   } else {
     w = last ? 1.f : 0.f;
   }
-  float* ho = p.h_out + (long long)i * D;
+  float* ho = p.h_out + orow * D;
   float* hw = p.h_state + (long long)i * D;
   for (int d = threadIdx.x; d < D; d += blockDim.x) {
     float hn = tr[d];
     ho[d] += w * hn;
     hw[d] = hn;
   }
-  if (threadIdx.x == 0) p.halt_w_out[(long long)p.t * p.N + i] = w;
+  if (threadIdx.x == 0) p.halt_w_out[wo] = w;
   for (int j = threadIdx.x; j < p.k; j += blockDim.x)
-    p.ids_out[((long long)p.t * p.N + i) * p.k + j] = p.transformer_off ? -1 : p.ids[(long long)i * p.k + j];
+    p.ids_out[wo * p.k + j] = p.transformer_off ? -1 : p.ids[(long long)i * p.k + j];
 }
 
 // ------------------------------------------------------------------------------------------
@@ -372,14 +386,14 @@ void launch_positions_decode(int* pos, const int* cache_len, int B, int t_max, D
 }
 void launch_loop_prologue(int dtype, const float* h, const void* e, const float* emb, int loop_dim,
                           const float* w_rec, const float* w_attn, float* combined, void* a,
-                          int N, int D, float eps, cudaStream_t s) {
+                          int N, int D, float eps, cudaStream_t s, const int* row_loop, int emb_stride) {
   size_t smem = (size_t)D * sizeof(float);
   if (dtype == 0)
     { k_loop_prologue<float><<<N, nthreads_for(D), smem, s>>>(h, (const float*)e, emb, loop_dim, w_rec, w_attn,
-                                                           combined, (float*)a, D, eps); note_launch(); }
+                                                           combined, (float*)a, D, eps, row_loop, emb_stride); note_launch(); }
   else
     { k_loop_prologue<bf16><<<N, nthreads_for(D), smem, s>>>(h, (const bf16*)e, emb, loop_dim, w_rec, w_attn,
-                                                          combined, (bf16*)a, D, eps); note_launch(); }
+                                                          combined, (bf16*)a, D, eps, row_loop, emb_stride); note_launch(); }
 }
 bool launch_rmsnorm_warp(int dtype, const float* x, const float* w, void* out, int N, int D, float eps,
                          cudaStream_t s);
@@ -407,13 +421,13 @@ void launch_mla_kv_prep(int dtype, const float* kv_raw, int kvr, int dr, const f
 }
 void launch_kv_to_cache(int dtype, const void* qkv, long long ld, int k_col, int v_col, int Hkv, int hd,
                         const int* pos, int N, int seq, int t_max, void* kc, void* vc, DevStatus* st,
-                        cudaStream_t s) {
+                        cudaStream_t s, const int* row_loop, long long loop_elems) {
   if (dtype == 0)
     { k_kv_to_cache<float><<<N, 128, 0, s>>>((const float*)qkv, ld, k_col, v_col, Hkv, hd, pos, seq, t_max,
-                                           (float*)kc, (float*)vc, st); note_launch(); }
+                                           (float*)kc, (float*)vc, row_loop, loop_elems, st); note_launch(); }
   else
     { k_kv_to_cache<bf16><<<N, 128, 0, s>>>((const bf16*)qkv, ld, k_col, v_col, Hkv, hd, pos, seq, t_max,
-                                          (bf16*)kc, (bf16*)vc, st); note_launch(); }
+                                          (bf16*)kc, (bf16*)vc, row_loop, loop_elems, st); note_launch(); }
 }
 bool launch_combine_warp(int dtype, const CombineParams& p, int n_rows, cudaStream_t s);
 

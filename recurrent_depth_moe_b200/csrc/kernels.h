@@ -17,7 +17,7 @@ int device_sm_count();
 // launches in its scope on the given stream when profiling is on).
 enum ProfClass {
   PC_PROLOGUE = 0, PC_QKV, PC_ATTN, PC_OPROJ, PC_FFN_NORM, PC_ROUTER_GEMM, PC_ROUTE, PC_EXPERT_UP,
-  PC_EXPERT_DOWN, PC_COMBINE, PC_OTHER, PC_BLOCK, PC_HEAD, PC_TOKENS, PC_COUNT
+  PC_EXPERT_DOWN, PC_COMBINE, PC_OTHER, PC_BLOCK, PC_HEAD, PC_TOKENS, PC_DEPTH_FILL, PC_COUNT
 };
 struct ProfScope {
   ProfScope(int cls, cudaStream_t s);
@@ -98,6 +98,9 @@ struct AttnParams {
   float* part_o; float* part_ml; int n_split;
   // tensor-core prefill: values transposed, vt[((b * Hkv + g) * dv + d) * vt_ld + j]
   const void* vt; long long vt_ld;
+  // decode with rows at different loop depths: sequence b reads the loop cache
+  // max(row_loop[b], 0), i.e. k1 / v advanced by that many loop_k / loop_v elements
+  const int* row_loop; long long loop_k, loop_v;
   DevStatus* st;                                        // device status word (timeouts); may be null
 };
 int launch_attention(int dtype, const AttnParams& p, cudaStream_t s);
@@ -157,6 +160,11 @@ struct CombineParams {
   float* cum; int* halted;
   float* halt_w_out; int* ids_out; float* p_out;
   float* out;   // block_only
+  // rows at their own loop depth (continuous depth-wise batching; nullptr: every row at loop
+  // t): row i runs loop t_row[i] and its outputs go to output row out_row[i] of h_out
+  // [rows][D], halt_w_out [rows][n_loops] and ids_out [rows][n_loops][k]; halted rows are
+  // idle slots and write nothing
+  const int* t_row; const int* out_row;
   // fused prologue of loop t + 1 (warp-per-row kernel only; next_emb == nullptr: off):
   // combined = RMSNorm_rec(h_new + emb + e), a = RMSNorm_attn(combined)
   const float* next_emb; int loop_dim; const float* w_rec; const float* w_attn; float eps;
@@ -164,21 +172,46 @@ struct CombineParams {
   DevStatus* st;
 };
 
+// ------------------------------------------------------------------------------------------
+// continuous depth-wise batching of decode steps: one slot per sequence, each slot's token at
+// its own loop; finished tokens fill their remaining loops' keys / values and the slot takes
+// the sequence's next token
+// ------------------------------------------------------------------------------------------
+struct DepthParams {
+  int B, S, L, D, loop_dim, emb_stride, Hkv, hd, t_max;
+  const float* h0_seq; const void* e_seq; const float* off_seq;   // [B][S][D], [B][S][D], [B][S] or null
+  const int* cache_len0;                                           // [B] position of token 0
+  float* h; void* e_slot; float* off_slot; int* pos;               // slot state [B][D], [B][D], [B], [B]
+  int* t_row; int* tok; int* out_row; float* cum; int* halted; int* pending;
+  const float* emb_tab; const float* w_rec; const float* w_attn; float eps;   // emb_tab [L][emb_stride]
+  void* a_fill; int* pos_fill; const void* kv_fill;                // [B (L-1)][D], [B (L-1)], [B (L-1)][2 Hkv hd]
+  void* kc; void* vc; long long loop_elems;                        // GQA loop caches, elements per loop
+  DevStatus* st;
+};
+void launch_depth_start(int dtype, const DepthParams& p, cudaStream_t s);
+void launch_depth_fill_prologue(int dtype, const DepthParams& p, cudaStream_t s);
+void launch_depth_fill_store(int dtype, const DepthParams& p, cudaStream_t s);
+void launch_depth_refill(int dtype, const DepthParams& p, cudaStream_t s);
+
 void launch_lti_A(const float* log_A, const float* log_dt, float* A, int D, cudaStream_t s);
 void launch_loop_emb(float* emb, int loop_dim, int t, float theta, cudaStream_t s);
 void launch_rope_table(float2* tab, int n_pos, int dim, float theta, cudaStream_t s);
 void launch_positions(int* pos, int N, int seq, int start_pos, cudaStream_t s);
 void launch_positions_decode(int* pos, const int* cache_len, int B, int t_max, DevStatus* st, cudaStream_t s);
+// row_loop (optional): row r adds the loop embedding emb + max(row_loop[r], 0) * emb_stride
 void launch_loop_prologue(int dtype, const float* h, const void* e, const float* emb, int loop_dim,
                           const float* w_rec, const float* w_attn, float* combined, void* a,
-                          int N, int D, float eps, cudaStream_t s);
+                          int N, int D, float eps, cudaStream_t s, const int* row_loop = nullptr,
+                          int emb_stride = 0);
 void launch_rmsnorm(int in_f32, int dtype, const void* x, long long in_ld, const float* w, void* out,
                     long long out_ld, int rows, int D, float eps, cudaStream_t s);
 void launch_mla_kv_prep(int dtype, const float* kv_raw, int kvr, int dr, const float* kv_norm_w, float eps,
                         const int* pos, const float2* rope_tab, void* ckv, void* krope, int N, cudaStream_t s);
+// row_loop (optional): row r writes into the loop cache row_loop[r] (loop_elems elements per
+// loop), rows with row_loop[r] < 0 write nothing
 void launch_kv_to_cache(int dtype, const void* qkv, long long ld, int k_col, int v_col, int Hkv, int hd,
                         const int* pos, int N, int seq, int t_max, void* kc, void* vc, DevStatus* st,
-                        cudaStream_t s);
+                        cudaStream_t s, const int* row_loop = nullptr, long long loop_elems = 0);
 // returns true when the fused next-loop prologue ran (p.next_emb set and supported)
 bool launch_combine(int dtype, const CombineParams& p, int n_rows, cudaStream_t s);
 void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* n_run, int* cta_count,

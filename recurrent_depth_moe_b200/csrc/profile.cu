@@ -16,7 +16,8 @@ void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 namespace {
 const char* kClassNames[PC_COUNT] = {"loop_prologue", "qkv_gemm_rope", "attention", "o_gemm_residual",
                                      "ffn_rmsnorm",   "router_gemm",   "route_topk_permute", "expert_up_swiglu",
-                                     "expert_down_gate", "combine_lora_inject_act", "other", "dense_block", "lm_head", "embed_cast_greedy"};
+                                     "expert_down_gate", "combine_lora_inject_act", "other", "dense_block", "lm_head", "embed_cast_greedy",
+                                     "depth_kv_fill"};
 struct Rec {
   int cls;
   cudaEvent_t a, b;

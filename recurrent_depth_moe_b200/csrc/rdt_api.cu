@@ -156,6 +156,7 @@ struct Ctx {
   cudaStream_t s;
   DevStatus* st;
   int dtype;
+  const int* row_loop = nullptr;   // decode rows at their own loop depth (continuous depth-wise batching)
 };
 
 #define RDT_TRY(x)                          \
@@ -211,10 +212,16 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
     ap.scale = 1.f / sqrtf((float)hd);
     const bool use_cache = cache && cache->k;
     if (use_cache) {
-      size_t per_loop = (size_t)cache->batch * Hkv * cache->t_max * hd * es;
+      const long long loop_elems = (long long)cache->batch * Hkv * cache->t_max * hd;
+      size_t per_loop = (size_t)loop_elems * es;
       char* kc = (char*)cache->k + per_loop * loop_t;
       char* vc = (char*)cache->v + per_loop * loop_t;
-      { ProfScope ps(PC_OTHER, x.s); launch_kv_to_cache(x.dtype, qkv, W, H * hd, (H + Hkv) * hd, Hkv, hd, pos, N, T, cache->t_max, kc, vc, x.st, x.s); }
+      {
+        ProfScope ps(PC_OTHER, x.s);
+        launch_kv_to_cache(x.dtype, qkv, W, H * hd, (H + Hkv) * hd, Hkv, hd, pos, N, T, cache->t_max, kc, vc, x.st,
+                           x.s, x.row_loop, loop_elems);
+      }
+      if (x.row_loop) { ap.row_loop = x.row_loop; ap.loop_k = ap.loop_v = loop_elems; }
       if (decode || start_pos > 0) {
         long long sj = hd, sg = (long long)cache->t_max * hd, sb = (long long)Hkv * sg;
         ap.k1 = kc; ap.k1_b = sb; ap.k1_j = sj; ap.k1_g = sg;
@@ -527,6 +534,141 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
   return RDT_OK;
 }
 
+// ------------------------------------------------------------------------------------------
+// continuous depth-wise batching of decode steps
+// ------------------------------------------------------------------------------------------
+struct DepthLayout {
+  size_t t_row, tok, out_row, pending, e_slot, off_slot, emb_tab, a_fill, kv_fill, pos_fill, total;
+  int emb_stride;
+};
+
+// The decode layout of `batch` rows (one slot per sequence) followed by the slot state and
+// the fill buffers of the remaining loops of finished tokens.
+void make_depth_layout(const rdt_config* c, int B, int L, int t_max, Layout* Lo, DepthLayout* DL) {
+  make_layout(c, B, 1, t_max, Lo);
+  size_t off = Lo->total;
+  auto take = [&](size_t bytes) { size_t o = off; off += align256(bytes); return o; };
+  const size_t D = c->dim, es = esize(c), nf = (size_t)B * std::max(L - 1, 1);
+  const int hd = c->dim / c->n_heads;
+  DL->emb_stride = std::max(c->loop_dim, 2);
+  DL->t_row = take((size_t)B * 4);
+  DL->tok = take((size_t)B * 4);
+  DL->out_row = take((size_t)B * 4);
+  DL->pending = take(16);
+  DL->e_slot = take((size_t)B * D * es);
+  DL->off_slot = take((size_t)B * 4);
+  DL->emb_tab = take((size_t)L * DL->emb_stride * 4);
+  DL->a_fill = take(nf * D * es);
+  DL->kv_fill = take(nf * 2 * (size_t)c->n_kv_heads * hd * es);
+  DL->pos_fill = take(nf * 4);
+  DL->total = off;
+}
+
+struct DepthCall {
+  Ctx x;
+  DepthLayout DL;
+  DepthParams dp;
+  CombineParams cp;
+};
+
+rdt_status depth_setup(const rdt_depth_batch* db, cudaStream_t s, DepthCall* dc) {
+  if (!db) return RDT_ERR_INVALID_ARG;
+  const rdt_config* c = db->cfg;
+  const rdt_weights* w = db->w;
+  rdt_status st = check_config(c);
+  if (st != RDT_OK) return st;
+  if ((st = check_block_weights(c, w, true)) != RDT_OK) return st;
+  if (c->attn_type != 0) return RDT_ERR_UNSUPPORTED;    // GQA loop caches only
+  if (!w->rec_norm_w || !w->log_A || !w->log_dt || !w->inj_B) return RDT_ERR_INVALID_ARG;
+  if (c->lora_rank > 0 && (!w->lora_down || !w->lora_B || !w->lora_scale)) return RDT_ERR_INVALID_ARG;
+  const int B = db->batch, S = db->n_tokens, L = db->n_loops;
+  if (!db->h0 || !db->e || !db->cache_len || !db->h_out || !db->halt_weights || !db->expert_ids || !db->cache)
+    return RDT_ERR_INVALID_ARG;
+  if (B <= 0 || S <= 0 || L <= 0 || db->act_threshold != db->act_threshold) return RDT_ERR_INVALID_ARG;
+  if ((long long)B * S > (1LL << 30) || (long long)B * L > (1LL << 24)) return RDT_ERR_UNSUPPORTED;
+  const bool act_on = db->act_threshold > 0.f;
+  if (act_on && (!w->halt_w || !w->halt_b)) return RDT_ERR_INVALID_ARG;
+  const rdt_kv_cache* cache = db->cache;
+  if (!cache->k || !cache->v || cache->t_max <= 0 || cache->batch < B || cache->n_loops < L || S > cache->t_max)
+    return RDT_ERR_INVALID_ARG;
+  Ctx& x = dc->x;
+  x.c = c; x.w = w; x.ws = db->ws; x.s = s; x.dtype = c->dtype;
+  make_depth_layout(c, B, L, cache->t_max, &x.L, &dc->DL);
+  if (!db->ws || ((uintptr_t)db->ws & 255) || db->ws_bytes < dc->DL.total) return RDT_ERR_WORKSPACE;
+  x.st = at<DevStatus*>(db->ws, x.L.status);
+  const DepthLayout& DL = dc->DL;
+  void* ws = db->ws;
+  x.row_loop = at<int*>(ws, DL.t_row);
+  const int D = c->dim, hd = D / c->n_heads;
+  DepthParams& dp = dc->dp;
+  memset(&dp, 0, sizeof(dp));
+  dp.B = B; dp.S = S; dp.L = L; dp.D = D; dp.loop_dim = c->loop_dim; dp.emb_stride = DL.emb_stride;
+  dp.Hkv = c->n_kv_heads; dp.hd = hd; dp.t_max = cache->t_max;
+  dp.h0_seq = db->h0; dp.e_seq = db->e; dp.off_seq = db->halt_logit_offset; dp.cache_len0 = db->cache_len;
+  dp.h = at<float*>(ws, x.L.h); dp.e_slot = at<void*>(ws, DL.e_slot); dp.off_slot = at<float*>(ws, DL.off_slot);
+  dp.pos = at<int*>(ws, x.L.pos);
+  dp.t_row = at<int*>(ws, DL.t_row); dp.tok = at<int*>(ws, DL.tok); dp.out_row = at<int*>(ws, DL.out_row);
+  dp.cum = at<float*>(ws, x.L.cum); dp.halted = at<int*>(ws, x.L.halted); dp.pending = at<int*>(ws, DL.pending);
+  dp.emb_tab = at<float*>(ws, DL.emb_tab); dp.w_rec = w->rec_norm_w; dp.w_attn = w->attn_norm_w; dp.eps = c->norm_eps;
+  dp.a_fill = at<void*>(ws, DL.a_fill); dp.pos_fill = at<int*>(ws, DL.pos_fill); dp.kv_fill = at<void*>(ws, DL.kv_fill);
+  dp.kc = cache->k; dp.vc = cache->v;
+  dp.loop_elems = (long long)cache->batch * c->n_kv_heads * cache->t_max * hd;
+  dp.st = x.st;
+  CombineParams& cp = dc->cp;
+  cp = combine_base(x, B);
+  cp.n_loops = L; cp.act_on = act_on; cp.thr = db->act_threshold; cp.e = dp.e_slot; cp.h_out = db->h_out;
+  cp.halt_off = dp.off_slot; cp.halt_w_out = db->halt_weights; cp.ids_out = db->expert_ids;
+  cp.loop_dim = c->loop_dim; cp.w_rec = w->rec_norm_w; cp.w_attn = w->attn_norm_w; cp.eps = c->norm_eps;
+  cp.next_emb = nullptr; cp.t_row = dp.t_row; cp.out_row = dp.out_row;
+  return RDT_OK;
+}
+
+// One tick: every slot's token runs one loop at its own depth; finished tokens fill their
+// remaining loops' keys / values and their slots take the next tokens.
+rdt_status depth_tick(const rdt_depth_batch* db, DepthCall& dc) {
+  Ctx& x = dc.x;
+  const rdt_config* c = x.c;
+  const rdt_weights* w = x.w;
+  const DepthParams& dp = dc.dp;
+  const int B = dp.B, L = dp.L, D = c->dim, hd = dp.hd, Hkv = dp.Hkv, H = c->n_heads;
+  cudaStream_t s = x.s;
+  void* ws = x.ws;
+  float* combined = at<float*>(ws, x.L.combined);
+  void* a = at<void*>(ws, x.L.a);
+  float* x1 = at<float*>(ws, x.L.x1);
+  rdt_status st;
+  {
+    ProfScope ps(PC_PROLOGUE, s);
+    launch_loop_prologue(x.dtype, dp.h, dp.e_slot, dp.emb_tab, c->loop_dim, w->rec_norm_w, w->attn_norm_w,
+                         combined, a, B, D, c->norm_eps, s, dp.t_row, dp.emb_stride);
+  }
+  if ((st = attention_block(x, B, 1, combined, a, x1, db->cache, 0, 0, true)) != RDT_OK) return st;
+  if ((st = moe_block(x, B, x1)) != RDT_OK) return st;
+  { ProfScope ps(PC_COMBINE, s); launch_combine(x.dtype, dc.cp, B, s); }
+  if (L > 1) {
+    ProfScope ps(PC_DEPTH_FILL, s);
+    launch_depth_fill_prologue(x.dtype, dp, s);
+    GemmParams g;
+    memset(&g, 0, sizeof(g));
+    g.impl = -1; g.st = x.st;
+    g.A = dp.a_fill; g.lda = D;
+    g.B = (const char*)w->w_qkv + (size_t)H * hd * D * esize(c); g.ldb = D;   // the K and V rows of w_qkv
+    g.M = B * (L - 1); g.N = 2 * Hkv * hd; g.K = D;
+    g.C = const_cast<void*>(dp.kv_fill); g.ldc = 2 * Hkv * hd;
+    g.pos = dp.pos_fill; g.rope_tab = at<const float2*>(ws, x.L.rope); g.rope_half = hd / 2; g.n_rope = 1;
+    g.rope[0] = RopeDesc{0, Hkv, hd, 0, hd};
+    RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, s));
+    launch_depth_fill_store(x.dtype, dp, s);
+  }
+  {
+    ProfScope ps(PC_OTHER, s);
+    launch_depth_refill(x.dtype, dp, s);
+    launch_compact(dp.halted, B, at<int*>(ws, x.L.run_list), at<int*>(ws, x.L.run_idx), at<int*>(ws, x.L.nrun),
+                   at<int*>(ws, x.L.cta_count), s);
+  }
+  return RDT_OK;
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------------------------------
@@ -590,13 +732,13 @@ rdt_status rdt_recurrent_decode_step(const rdt_config* cfg, const rdt_weights* w
                        expert_ids, cache, nullptr, 0, ws, ws_bytes, (cudaStream_t)stream, true);
 }
 
-rdt_status rdt_recurrent_decode_step_traced(const rdt_config* cfg, const rdt_weights* w, const float* h0,
-                                            const void* e, int batch, const int32_t* cache_len, int n_loops,
-                                            float act_threshold, float* h_out, float* halt_weights,
-                                            int32_t* expert_ids, const rdt_kv_cache* cache, const rdt_trace* trace,
-                                            void* ws, size_t ws_bytes, void* stream) {
-  return run_recurrent(cfg, w, h0, e, batch, 1, 0, cache_len, n_loops, act_threshold, nullptr, h_out, halt_weights,
-                       expert_ids, cache, trace, 0, ws, ws_bytes, (cudaStream_t)stream, true);
+rdt_status rdt_recurrent_decode_step_ex(const rdt_config* cfg, const rdt_weights* w, const float* h0,
+                                        const void* e, int batch, const int32_t* cache_len, int n_loops,
+                                        float act_threshold, const float* halt_logit_offset, float* h_out,
+                                        float* halt_weights, int32_t* expert_ids, const rdt_kv_cache* cache,
+                                        const rdt_trace* trace, void* ws, size_t ws_bytes, void* stream) {
+  return run_recurrent(cfg, w, h0, e, batch, 1, 0, cache_len, n_loops, act_threshold, halt_logit_offset, h_out,
+                       halt_weights, expert_ids, cache, trace, 0, ws, ws_bytes, (cudaStream_t)stream, true);
 }
 
 rdt_status rdt_block_forward_cached(const rdt_config* cfg, const rdt_weights* w, const float* x_in, float* x_out,
@@ -714,6 +856,74 @@ rdt_status rdt_head_rows(const rdt_config* cfg, const float* xin, long long x_ld
 rdt_status rdt_head(const rdt_config* cfg, const float* xin, int n, const float* norm_w, const void* head, int vocab,
                     float* logits, void* ws, size_t ws_bytes, void* stream) {
   return rdt_head_rows(cfg, xin, cfg ? cfg->dim : 0, n, norm_w, head, vocab, logits, ws, ws_bytes, stream);
+}
+
+size_t rdt_depth_batch_workspace_size(const rdt_config* cfg, int batch, int n_loops, int t_max) {
+  if (check_config(cfg) != RDT_OK || batch <= 0 || n_loops <= 0 || t_max <= 0) return 0;
+  Layout L;
+  DepthLayout DL;
+  make_depth_layout(cfg, batch, n_loops, t_max, &L, &DL);
+  return DL.total;
+}
+
+rdt_status rdt_depth_batch_begin(const rdt_depth_batch* db, void* stream) {
+  cudaStream_t s = (cudaStream_t)stream;
+  DepthCall dc;
+  rdt_status st = depth_setup(db, s, &dc);
+  if (st != RDT_OK) return st;
+  Ctx& x = dc.x;
+  const DepthParams& dp = dc.dp;
+  const rdt_config* c = x.c;
+  const size_t rows = (size_t)dp.B * dp.S;
+  if (cudaMemsetAsync(x.st, 0, sizeof(DevStatus), s) != cudaSuccess) return RDT_ERR_CUDA;
+  if (cudaMemsetAsync(db->h_out, 0, rows * c->dim * 4, s) != cudaSuccess) return RDT_ERR_CUDA;
+  if (cudaMemsetAsync(db->halt_weights, 0, rows * dp.L * 4, s) != cudaSuccess) return RDT_ERR_CUDA;
+  if (cudaMemsetAsync(db->expert_ids, 0xFF, rows * dp.L * std::max(c->top_k, 1) * 4, s) != cudaSuccess)
+    return RDT_ERR_CUDA;                                   // every id -1 until its token runs that loop
+  launch_lti_A(x.w->log_A, x.w->log_dt, at<float*>(x.ws, x.L.Avec), c->dim, s);
+  launch_rope_table(at<float2*>(x.ws, x.L.rope), x.L.rope_pos, x.L.rope_dim, c->rope_theta, s);
+  for (int t = 0; t < dp.L; ++t) launch_loop_emb(const_cast<float*>(dp.emb_tab) + (size_t)t * dp.emb_stride,
+                                                 c->loop_dim, t, c->loop_theta, s);
+  launch_depth_start(x.dtype, dp, s);
+  launch_iota(at<int*>(x.ws, x.L.run_list), at<int*>(x.ws, x.L.run_idx), at<int*>(x.ws, x.L.nrun), dp.B, s);
+  return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
+}
+
+rdt_status rdt_depth_batch_tick(const rdt_depth_batch* db, int n_ticks, void* stream) {
+  if (n_ticks < 0) return RDT_ERR_INVALID_ARG;
+  DepthCall dc;
+  rdt_status st = depth_setup(db, (cudaStream_t)stream, &dc);
+  if (st != RDT_OK) return st;
+  for (int i = 0; i < n_ticks; ++i)
+    if ((st = depth_tick(db, dc)) != RDT_OK) return st;
+  return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
+}
+
+long long rdt_depth_batch_pending(const rdt_depth_batch* db, void* stream) {
+  cudaStream_t s = (cudaStream_t)stream;
+  DepthCall dc;
+  if (depth_setup(db, s, &dc) != RDT_OK) return -1;
+  int v = -1;
+  if (cudaMemcpyAsync(&v, (char*)db->ws + dc.DL.pending, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return -1;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return -1;
+  return v;
+}
+
+rdt_status rdt_depth_batch_run(const rdt_depth_batch* db, int check_every, void* stream) {
+  if (check_every <= 0) return RDT_ERR_INVALID_ARG;
+  rdt_status st = rdt_depth_batch_begin(db, stream);
+  if (st != RDT_OK) return st;
+  // every token runs at most n_loops ticks and a slot holds one token at a time
+  const long long max_ticks = (long long)db->n_tokens * db->n_loops;
+  for (long long done = 0; done < max_ticks; done += check_every) {
+    const int n = (int)std::min<long long>(check_every, max_ticks - done);
+    if ((st = rdt_depth_batch_tick(db, n, stream)) != RDT_OK) return st;
+    const long long left = rdt_depth_batch_pending(db, stream);
+    if (left < 0) return RDT_ERR_CUDA;
+    if (left == 0) return RDT_OK;
+  }
+  return rdt_depth_batch_pending(db, stream) == 0 ? RDT_OK : RDT_ERR_CUDA;
 }
 
 rdt_status rdt_read_device_status(void* ws, void* stream) {
