@@ -57,13 +57,17 @@ def peaks():
 def workload_desc(wl):
     c = wl.cfg
     shape = {"rdt1b_prefill": "1B-shaped recurrent block prefill",
-             "rdt10b_prefill_zipf": "10B-shaped load-imbalanced recurrent block prefill"}.get(wl.name, wl.name)
+             "rdt10b_prefill_zipf": "10B-shaped load-imbalanced recurrent block prefill",
+             "rdt3b_mla_prefill": "3B-shaped MLA recurrent block prefill"}.get(wl.name, wl.name)
+    attn = (f"{c.n_heads} heads GQA ({c.n_kv_heads} kv)" if c.attn_type == "gqa" else
+            f"{c.n_heads} heads MLA (kv_lora_rank {c.kv_lora_rank}, q_lora_rank {c.q_lora_rank}, nope "
+            f"{c.qk_nope_head_dim}, rope {c.qk_rope_head_dim}, v {c.v_head_dim})")
     extra = ""
     if wl.zipf_s:
         extra += f", Zipf(s={wl.zipf_s}) router bias"
     if wl.halt_spread:
         extra += f", halting spread over {wl.halt_spread[0]}-{wl.halt_spread[1]} loops"
-    return (f"{wl.name}: {shape}, dim {c.dim}, {c.n_heads} heads GQA ({c.n_kv_heads} kv), "
+    return (f"{wl.name}: {shape}, dim {c.dim}, {attn}, "
             f"{c.n_experts} routed + {c.n_shared_experts} shared SwiGLU experts top-{c.n_experts_per_tok}, "
             f"expert_dim {c.expert_dim}, lora_rank {c.lora_rank}, {wl.n_loops} loops, batch {wl.batch} x seq {wl.seq}, "
             f"{c.dtype}, ACT {wl.act_threshold} (halting bias {wl.halt_b}){extra}")
@@ -137,6 +141,16 @@ def expert_up_traffic(wl):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return rec["bytes"] if h.hexdigest() == rec["sha256"] else None
+
+
+def attention_flops(cfg, B: int, T: int) -> float:
+    """Causal prefill attention per launch: per (sequence, head) S = Q K^T and O = P V over the
+    T^2 / 2 visible (query, key) pairs, 2 FLOPs per multiply-add: (score dim + value dim) T^2."""
+    if cfg.attn_type == "gqa":
+        dqk = dv = cfg.head_dim
+    else:
+        dqk, dv = cfg.qk_nope_head_dim + cfg.qk_rope_head_dim, cfg.v_head_dim
+    return float(B) * cfg.n_heads * (dqk + dv) * T * T
 
 
 def expert_up_flops(wl, n_running: float) -> float:
@@ -324,6 +338,14 @@ def run_prefill(args, wl, rank, world, local_rank, *, steps=None, e2e=True, cpu_
     if up[0]:
         achieved = expert_up_flops(wl, mean_running) / (up[1] / up[0] / 1e3) / 1e12
     peak_t = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    att = prof.get("attention", (0, 0.0))
+    if att[0]:
+        att_tf = attention_flops(cfg, B, T) / (att[1] / att[0] / 1e3) / 1e12
+        res["attention_roofline"] = {
+            "bound": "tensor", "achieved": att_tf, "peak": peak_t, "unit": "TFLOP/s", "frac": att_tf / peak_t,
+            "flops_per_launch": attention_flops(cfg, B, T), "ms_per_launch": att[1] / att[0],
+            "kernel": ("k_attn_tc (tcgen05, GQA)" if cfg.attn_type == "gqa" else
+                       "k_attn_tc (tcgen05, MLA: keys [k_nope | k_rope], values read in place)")}
     res["roofline"] = {"bound": "tensor", "kernel": "expert_up_swiglu (tcgen05 grouped GEMM, SwiGLU epilogue)",
                        "achieved": achieved, "peak": peak_t, "unit": "TFLOP/s",
                        "frac": (achieved / peak_t) if achieved else None,
@@ -359,6 +381,10 @@ def run_ours(args, wl, rank, world, local_rank):
         side = run_prefill(args, wl1, rank, world, local_rank, e2e=False)
         # the literal reading of the 1B config: halting bias 0, so positions halt after 2-3 loops
         literal = run_prefill(args, wl1, rank, world, local_rank, steps=min(args.steps, 5), e2e=False, halt_b=0.0)
+    mla_prefill = None
+    if not args.no_secondary:
+        mla_prefill = run_prefill(args, RI.get_workload("rdt3b_mla_prefill"), rank, world, local_rank,
+                                  steps=min(args.steps, 5), e2e=False)
     decode_res = None if args.no_decode else run_decode(args, rank, world, local_rank)
     mla_res = None if args.no_decode or args.no_mla_decode else run_decode(args, rank, world, local_rank,
                                                                              "rdt3b_mla_decode")
@@ -394,6 +420,16 @@ def run_ours(args, wl, rank, world, local_rank):
                         "weights, positions halt after 2-3 of the 16 loops)", **literal}
         res["rdt1b_literal_token_loops_per_s"] = literal["value"]
         res["rdt1b_literal_mean_loops"] = literal["mean_loops"]
+    if "attention_roofline" in head:
+        res["attention_frac"] = head["attention_roofline"]["frac"]
+    if side is not None and "attention_roofline" in side:
+        res["rdt1b_attention_frac"] = side["attention_roofline"]["frac"]
+    if mla_prefill is not None:
+        res["rdt3b_mla_prefill"] = {"workload": workload_desc(RI.get_workload("rdt3b_mla_prefill")), **mla_prefill}
+        res["rdt3b_mla_prefill_token_loops_per_s"] = mla_prefill["value"]
+        if "attention_roofline" in mla_prefill:
+            res["mla_prefill_attention_tflops"] = mla_prefill["attention_roofline"]["achieved"]
+            res["mla_prefill_attention_frac"] = mla_prefill["attention_roofline"]["frac"]
     if decode_res is not None:
         res["decode"] = decode_res
         res["decode_tokens_per_s"] = decode_res["value"]

@@ -140,6 +140,14 @@ WORKLOADS = {
         attn_type="mla", kv_lora_rank=512, q_lora_rank=1536, qk_rope_head_dim=64, qk_nope_head_dim=128,
         v_head_dim=128, dtype="bf16"), batch=64, seq=1, n_loops=16, seed=5, act_threshold=0.0, kind="decode",
         cache_len=4096, decode_steps=128, device_weights=True),
+    # MLA prefill at the 3B MLA shape (the widths of rdt3b_mla_decode): 1 x 4096, 16 loops,
+    # halting bias -30 as in the 1B prefill; the workload of the tensor-core MLA prefill line.
+    "rdt3b_mla_prefill": Workload("rdt3b_mla_prefill", RDTConfig(
+        dim=3072, n_heads=24, n_kv_heads=24, max_seq_len=4096, max_loop_iters=16,
+        n_experts=64, n_shared_experts=1, n_experts_per_tok=4, expert_dim=4096, lora_rank=16,
+        attn_type="mla", kv_lora_rank=512, q_lora_rank=1536, qk_rope_head_dim=64, qk_nope_head_dim=128,
+        v_head_dim=128, dtype="bf16"), batch=1, seq=4096, n_loops=16, seed=12, act_threshold=0.99, halt_b=-30.0,
+        device_weights=True),
     # The 3B-shaped decode with ACT on and a per-token halting spread over 4..16 loops (zero
     # halting head, per-token logit offsets as in the 10B prefill): the workload on which
     # continuous depth-wise batching is compared with lockstep decode steps.  64 sequences,

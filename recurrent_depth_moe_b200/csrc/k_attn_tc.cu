@@ -33,17 +33,31 @@ bool tc_make_map(CUtensorMap* m, const void* base, unsigned long long rows, unsi
 
 namespace fat {
 
-constexpr int BQ = 128, BKV = 128, HD = 128, NQ = 2, KSTAGES = 3, VSTAGES = 2;
-constexpr int QTILE = BQ * HD * 2;      // 32 KB: two 64-dim swizzle atoms of 16 KB
-constexpr int QHALF = QTILE / 2;
-constexpr int KTILE = BKV * HD * 2;     // 32 KB: two atoms [128 keys][64 dims] of 16 KB
-constexpr int KHALF = KTILE / 2;
-constexpr int VTILE = HD * BKV * 2;     // 32 KB: two atoms [128 dims][64 keys] of 16 KB
+constexpr int BQ = 128, BKV = 128, HD = 128;   // query / key tile rows; value (and GQA key) head dim
+constexpr int BOX = BQ * 64 * 2;                 // 16 KB: one TMA box [128 rows][64 dims], SW128
+constexpr int VTILE = HD * BKV * 2;              // 32 KB: two boxes of values
 constexpr int VHALF = VTILE / 2;
-constexpr int SMEM = NQ * QTILE + KSTAGES * KTILE + VSTAGES * VTILE + 1024 + 512;   // 225.5 KB
-constexpr int TMEM_COLS = 512;          // S[q] at 128 q (P in its first 64); O[q] at 256 + 128 q
-constexpr float RESCALE_LOG2 = 8.f;     // lazy rescale threshold (factor 256)
-constexpr int THREADS = 64 + NQ * 128;
+constexpr float RESCALE_LOG2 = 8.f;              // lazy rescale threshold (factor 256)
+
+// Kernel variants: HQK = score head dim (query and key), NQ = query tiles per CTA, MLA = keys
+// from the per-head k_nope columns plus the head-shared k_rope, values read in place
+// (MN-major B operand) instead of a transposed copy.
+//   GQA: HQK 128, NQ 2, keys and values^T from the QKV projection (3 K stages, 225.5 KB)
+//   MLA: HQK 192 (nope 128 + rope 64), NQ 1, keys [k_nope | k_rope], values from the per-head
+//        [k_nope | v] rows (2 K stages, 209.5 KB)
+template <int HQK_, int NQ_, bool MLA_>
+struct Cfg {
+  static constexpr int HQK = HQK_, NQ = NQ_;
+  static constexpr bool MLA = MLA_;
+  static constexpr int NBOX = HQK / 64;                  // 64-dim boxes per query / key row
+  static constexpr int QTILE = BQ * HQK * 2, KTILE = BKV * HQK * 2;
+  static constexpr int KSTAGES = MLA ? 2 : 3, VSTAGES = 2;
+  static constexpr int SMEM = NQ * QTILE + KSTAGES * KTILE + VSTAGES * VTILE + 1024 + 512;
+  static constexpr int TMEM_COLS = NQ == 2 ? 512 : 256;  // S[q] at BKV q (P in its first 64); O[q] at BKV NQ + 128 q
+  static constexpr int THREADS = 64 + NQ * 128;
+};
+using CfgGqa = Cfg<128, 2, false>;
+using CfgMla = Cfg<192, 1, true>;
 
 struct Args {
   int B, T, H, G, Hkv;
@@ -52,7 +66,9 @@ struct Args {
   float sl2;               // softmax scale * log2(e)
   bf16* o;
   long long o_row;         // output row stride (elements); head h at column h * 128
-  int q_col0, k_col0;      // qkv columns of query head 0 and key head 0
+  int q_col0, k_col0;      // GQA: qkv columns of query head 0 and key head 0
+  int q_head, k_head;      // columns between heads: queries; keys / values (MLA: nope + v)
+  int v_col0;              // MLA: column of the values inside a head's [k_nope | v] row
   DevStatus* st;           // device status word: a wait that gave up is recorded here
 };
 
@@ -154,9 +170,14 @@ __device__ __forceinline__ int visible_tiles(const Args& a, long long row_last, 
   return n_vis > 0 ? (n_vis + BKV - 1) / BKV : 0;
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+// tmQ: query rows; tmK: key rows (GQA qkv / MLA k_nope); tmKR: MLA k_rope rows (unused for
+// GQA); tmV: GQA values transposed [b][g][dim][t], MLA the [k_nope | v] rows.
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmVt, const Args a) {
+              const __grid_constant__ CUtensorMap tmKR, const __grid_constant__ CUtensorMap tmV, const Args a) {
+  constexpr int NQ = C::NQ, QTILE = C::QTILE, KTILE = C::KTILE, KSTAGES = C::KSTAGES, VSTAGES = C::VSTAGES;
+  constexpr int TMEM_COLS = C::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sQ = smem;                          // [NQ] query tiles
@@ -228,16 +249,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
     for (int q = 0; q < NQ; ++q) qbytes += q_rows[q] > 0 ? QTILE : 0;
     mbar_expect_tx(q_full, qbytes);
-    const int qx = a.q_col0 + h * HD;
+    const int qx = a.q_col0 + h * a.q_head;
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
       if (q_rows[q] <= 0) continue;
       const int qy = b * a.T + q0[q];
-      tma_load_2d(sQ + q * QTILE, &tmQ, q_full, qx, qy);
-      tma_load_2d(sQ + q * QTILE + QHALF, &tmQ, q_full, qx + 64, qy);
+#pragma unroll
+      for (int kb = 0; kb < C::NBOX; ++kb) tma_load_2d(sQ + q * QTILE + kb * BOX, &tmQ, q_full, qx + 64 * kb, qy);
     }
-    const int kx = a.k_col0 + g * HD;
-    const int vy = (b * a.Hkv + g) * HD;
+    const int kx = a.k_col0 + g * a.k_head;
+    const int vy = (b * a.Hkv + g) * HD;          // GQA: the head's value rows of V^T
+    const int vx = g * a.k_head + a.v_col0;       // MLA: the head's value columns
     int k_phase[KSTAGES], v_phase[VSTAGES];   // phase of the last load issued into each stage (-1: none)
 #pragma unroll
     for (int s = 0; s < KSTAGES; ++s) k_phase[s] = -1;
@@ -248,13 +270,24 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!mbar_wait(&k_empty[ks], ((j / KSTAGES) & 1) ^ 1, abort_flag)) break;
       mbar_expect_tx(&k_full[ks], KTILE);
       const int ky = b * a.T + j * BKV;
-      tma_load_2d(sK + ks * KTILE, &tmK, &k_full[ks], kx, ky);
-      tma_load_2d(sK + ks * KTILE + KHALF, &tmK, &k_full[ks], kx + 64, ky);
+      if (C::MLA) {                               // [k_nope (2 boxes) | k_rope (1 box, shared by the heads)]
+        tma_load_2d(sK + ks * KTILE, &tmK, &k_full[ks], kx, ky);
+        tma_load_2d(sK + ks * KTILE + BOX, &tmK, &k_full[ks], kx + 64, ky);
+        tma_load_2d(sK + ks * KTILE + 2 * BOX, &tmKR, &k_full[ks], 0, ky);
+      } else {
+#pragma unroll
+        for (int kb = 0; kb < C::NBOX; ++kb) tma_load_2d(sK + ks * KTILE + kb * BOX, &tmK, &k_full[ks], kx + 64 * kb, ky);
+      }
       k_phase[ks] = (j / KSTAGES) & 1;
       if (!mbar_wait(&v_empty[vs], ((j / VSTAGES) & 1) ^ 1, abort_flag)) break;
       mbar_expect_tx(&v_full[vs], VTILE);
-      tma_load_2d(sV + vs * VTILE, &tmVt, &v_full[vs], j * BKV, vy);
-      tma_load_2d(sV + vs * VTILE + VHALF, &tmVt, &v_full[vs], j * BKV + 64, vy);
+      if (C::MLA) {                               // [128 keys][64 dims] boxes: an MN-major B operand
+        tma_load_2d(sV + vs * VTILE, &tmV, &v_full[vs], vx, ky);
+        tma_load_2d(sV + vs * VTILE + VHALF, &tmV, &v_full[vs], vx + 64, ky);
+      } else {                                    // [128 dims][64 keys] boxes: K-major
+        tma_load_2d(sV + vs * VTILE, &tmV, &v_full[vs], j * BKV, vy);
+        tma_load_2d(sV + vs * VTILE + VHALF, &tmV, &v_full[vs], j * BKV + 64, vy);
+      }
       v_phase[vs] = (j / VSTAGES) & 1;
     }
     // copies still in flight (an abort) land before the CTA's shared memory is released
@@ -268,7 +301,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
     constexpr uint32_t IDESC_S = idesc_bf16(128, BKV);
-    constexpr uint32_t IDESC_O = idesc_bf16(128, HD);
+    constexpr uint32_t IDESC_O = idesc_bf16_mn(128, HD, false, C::MLA);   // MLA values: B MN-major
     bool ok = mbar_wait(q_full, 0, abort_flag);
     // iteration j: PV of tile j - 1 then S of tile j, per query tile (j = nt_max drains)
     for (int j = 0; j <= nt_max && ok; ++j) {
@@ -288,19 +321,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (j >= 1 && j - 1 < nt[q]) {
           if (!(ok = mbar_wait(&p_full[q], (j - 1) & 1, abort_flag))) break;
           tc_fence_after();
-          const uint32_t tO = tmem + 256 + q * 128;
+          const uint32_t tO = tmem + NQ * BKV + q * 128;
 #pragma unroll
           for (int kk = 0; kk < BKV / 16; ++kk) {
-            const uint64_t bd = smem_desc(sV + pvs * VTILE + (kk >> 2) * VHALF) + 2 * (kk & 3);
+            const uint64_t bd = C::MLA ? smem_desc_mn(sV + pvs * VTILE + kk * 2048, VHALF)   // 16 keys = 2 atoms
+                                       : smem_desc(sV + pvs * VTILE + (kk >> 2) * VHALF) + 2 * (kk & 3);
             umma_bf16_ts(tO, tS + 8 * kk, bd, IDESC_O, (j > 1 || kk > 0) ? 1u : 0u);
           }
           umma_commit(&pv_done[q]);
         }
         if (load && j < nt[q]) {
 #pragma unroll
-          for (int kk = 0; kk < HD / 16; ++kk) {
-            const uint64_t ad = smem_desc(sQ + q * QTILE + (kk >> 2) * QHALF) + 2 * (kk & 3);
-            const uint64_t bd = smem_desc(sK + ks * KTILE + (kk >> 2) * KHALF) + 2 * (kk & 3);
+          for (int kk = 0; kk < C::HQK / 16; ++kk) {
+            const uint64_t ad = smem_desc(sQ + q * QTILE + (kk >> 2) * BOX) + 2 * (kk & 3);
+            const uint64_t bd = smem_desc(sK + ks * KTILE + (kk >> 2) * BOX) + 2 * (kk & 3);
             umma_bf16(tS, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
           }
           umma_commit(&s_full[q]);
@@ -324,7 +358,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int my_pos = row_valid ? a.q_pos[row0 + rl] : -1;
     const int n_vis = row_valid ? min(a.n_keys, a.q_pos[row0 + q_rows[q] - 1] - a.key_pos0 + 1) : 0;
     const int ntq = nt[q];
-    const uint32_t tO = tmem + lane_base + 256 + q * 128;
+    const uint32_t tO = tmem + lane_base + NQ * BKV + q * 128;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     const uint32_t tS = tmem + lane_base + q * BKV;
@@ -434,8 +468,31 @@ bool attention_tc_supports(int dtype, const AttnParams& p) {
          ((uintptr_t)p.o & 15) == 0;
 }
 
+// The MLA prefill of a bf16 block with nope 128, rope 64 and value 128 (the DeepSeek-V2
+// widths) whose keys are this call's rows: k_nope / v in the per-head [k_nope | v] rows of
+// k1 (= v - dn), k_rope in k2, one row per position.
+bool attention_tc_mla_supports(int dtype, const AttnParams& p) {
+  const long long kvw = p.k1_j;
+  return dtype == 1 && p.dn == 128 && p.dr == 64 && p.dv == 128 && p.G == 1 && p.k2 && !p.n_keys_dev &&
+         p.n_keys == p.T && p.q_head == 192 && p.q_row == (long long)p.H * 192 && p.k1_g == 256 &&
+         kvw == (long long)p.H * 256 && p.k1_b == (long long)p.T * kvw && p.k2_j == 64 &&
+         p.k2_b == (long long)p.T * 64 && p.v == (const void*)((const bf16*)p.k1 + 128) && p.v_j == kvw &&
+         p.v_g == 256 && p.v_b == p.k1_b && p.o_row % 8 == 0 && ((uintptr_t)p.q & 15) == 0 &&
+         ((uintptr_t)p.k1 & 15) == 0 && ((uintptr_t)p.k2 & 15) == 0 && ((uintptr_t)p.o & 15) == 0;
+}
+
+template <class C>
+static int launch_attn_tc_t(const CUtensorMap& mQ, const CUtensorMap& mK, const CUtensorMap& mKR,
+                            const CUtensorMap& mV, const fat::Args& a, cudaStream_t s) {
+  if (!ensure_smem_limit((const void*)fat::k_attn_tc<C>, C::SMEM)) return -1;
+  const int n_qt = (a.T + fat::BQ - 1) / fat::BQ;
+  const long long blocks = (long long)((n_qt + C::NQ - 1) / C::NQ) * a.B * a.H;
+  if (blocks <= 0) return 0;
+  { fat::k_attn_tc<C><<<(unsigned)blocks, C::THREADS, C::SMEM, s>>>(mQ, mK, mKR, mV, a); note_launch(); }
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
 int launch_attention_tc(const AttnParams& p, cudaStream_t s) {
-  if (!ensure_smem_limit((const void*)fat::k_attn_tc, fat::SMEM)) return -1;
   const int Hkv = p.H / p.G;
   // Q and K live in the qkv rows [B*T, q_row]; k1 points at key head 0 inside those rows
   const long long k_col0 = ((const bf16*)p.k1 - (const bf16*)p.q);
@@ -450,12 +507,25 @@ int launch_attention_tc(const AttnParams& p, cudaStream_t s) {
   a.q_pos = p.q_pos; a.key_pos0 = p.key_pos0; a.n_keys = p.n_keys;
   a.sl2 = p.scale * 1.4426950408889634f;
   a.o = (bf16*)p.o; a.o_row = p.o_row;
-  a.q_col0 = 0; a.k_col0 = (int)k_col0; a.st = p.st;
-  const int n_qt = (p.T + fat::BQ - 1) / fat::BQ;
-  const long long blocks = (long long)((n_qt + fat::NQ - 1) / fat::NQ) * p.B * p.H;
-  if (blocks <= 0) return 0;
-  { fat::k_attn_tc<<<(unsigned)blocks, fat::THREADS, fat::SMEM, s>>>(mQ, mK, mVt, a); note_launch(); }
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  a.q_col0 = 0; a.k_col0 = (int)k_col0; a.q_head = fat::HD; a.k_head = fat::HD; a.v_col0 = 0; a.st = p.st;
+  return launch_attn_tc_t<fat::CfgGqa>(mQ, mK, mK, mVt, a, s);
+}
+
+int launch_attention_tc_mla(const AttnParams& p, cudaStream_t s) {
+  CUtensorMap mQ, mK, mKR, mV;
+  const unsigned long long rows = (unsigned long long)p.B * p.T;
+  const unsigned long long kvw = (unsigned long long)p.k1_j;
+  if (!tc_make_map(&mQ, p.q, rows, (unsigned long long)p.q_row, p.q_row, fat::BQ)) return -1;
+  if (!tc_make_map(&mK, p.k1, rows, kvw, kvw, fat::BKV)) return -1;     // k_nope and v columns
+  if (!tc_make_map(&mKR, p.k2, rows, 64, 64, fat::BKV)) return -1;
+  mV = mK;
+  fat::Args a;
+  a.B = p.B; a.T = p.T; a.H = p.H; a.G = 1; a.Hkv = p.H;
+  a.q_pos = p.q_pos; a.key_pos0 = p.key_pos0; a.n_keys = p.n_keys;
+  a.sl2 = p.scale * 1.4426950408889634f;
+  a.o = (bf16*)p.o; a.o_row = p.o_row;
+  a.q_col0 = 0; a.k_col0 = 0; a.q_head = 192; a.k_head = 256; a.v_col0 = 128; a.st = p.st;
+  return launch_attn_tc_t<fat::CfgMla>(mQ, mK, mKR, mV, a, s);
 }
 
 }  // namespace rdt

@@ -683,6 +683,8 @@ bool attention_fa_supports(int dtype, const AttnParams& p);
 int launch_attention_fa(const AttnParams& p, cudaStream_t s);
 bool attention_tc_supports(int dtype, const AttnParams& p);
 int launch_attention_tc(const AttnParams& p, cudaStream_t s);
+bool attention_tc_mla_supports(int dtype, const AttnParams& p);
+int launch_attention_tc_mla(const AttnParams& p, cudaStream_t s);
 
 int gemm_tile_m(GemmImpl impl) { return impl == GEMM_TC ? 128 : 64; }
 GemmImpl gemm_pick(int dtype, const GemmParams& p, int epi) {
@@ -697,6 +699,7 @@ int launch_gemm(int dtype, int epi, const GemmParams& p, cudaStream_t s) {
 int launch_attention(int dtype, const AttnParams& p, cudaStream_t s) {
   if (p.part_o && p.T == 1 && launch_attention_decode(dtype, p, s) == 0) return 0;
   if (attention_tc_supports(dtype, p)) return launch_attention_tc(p, s);
+  if (attention_tc_mla_supports(dtype, p)) return launch_attention_tc_mla(p, s);
   if (attention_fa_supports(dtype, p)) return launch_attention_fa(p, s);
   return launch_attention_simt(dtype, p, s);
 }

@@ -74,9 +74,26 @@ __device__ __forceinline__ uint64_t smem_desc(const void* p) {
   return d;
 }
 
+// MN-major, 128-byte-swizzled operand tile (the rows of the stored tile run along K, 128
+// bytes = 64 elements of M or N each): the next 64 elements of M / N start lbo bytes further
+// on (the next TMA box), the next 8 rows of K 1024 bytes further on.
+__device__ __forceinline__ uint64_t smem_desc_mn(const void* p, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_u32(p) >> 4) & 0x3FFF);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;    // leading byte offset: the next 64 M / N elements
+  d |= (uint64_t)(1024 >> 4) << 32;              // stride byte offset: the next 8 rows of K
+  d |= (uint64_t)1 << 46;                        // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                        // SWIZZLE_128B
+  return d;
+}
+
 // kind::f16 instruction descriptor: bf16 A/B, fp32 D, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// The same with A (transpose A, bit 15) or B (transpose B, bit 16) MN-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_mn(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_bf16(M, N) | (a_mn ? (1u << 15) : 0u) | (b_mn ? (1u << 16) : 0u);
 }
 
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {

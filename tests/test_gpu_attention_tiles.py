@@ -55,3 +55,40 @@ def test_attention_tile_edges(T):
     # the last query row of each sequence sees every key: compare it on its own too
     last = [b * T + T - 1 for b in range(B)]
     assert rel_l2(d_k[last], d_o[last]) <= BF16_TOL
+
+
+def _mla_wide(H=24):
+    # DeepSeek-V2 head widths (nope 128, rope 64, value 128, kv_lora_rank 512): the
+    # tensor-core MLA prefill kernel's shape
+    return RI.RDTConfig(dim=1536, n_heads=H, n_kv_heads=H, max_seq_len=1024, max_loop_iters=2, n_experts=8,
+                        n_shared_experts=1, n_experts_per_tok=2, expert_dim=128, lora_rank=8, attn_type="mla",
+                        kv_lora_rank=512, q_lora_rank=256, qk_rope_head_dim=64, qk_nope_head_dim=128,
+                        v_head_dim=128, dtype="bf16")
+
+
+# MLA prefill on the tensor cores (one 128-query tile per CTA, keys [k_nope | shared k_rope],
+# values read in place): around one tile, several tiles with a ragged last one
+@pytest.mark.parametrize("T", [8, 128, 136, 300, 520])
+def test_mla_attention_tile_edges(T):
+    cfg = _mla_wide()
+    W = RI.block_weights(cfg, 33, attn_std=0.05)
+    B, L = 2, 1
+    h0, e = RI.recurrent_inputs(cfg, B, T, 34)
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    tr = R.Trace.alloc(cfg, L, 0, B * T)
+    blk.forward(h0.cuda(), e.cuda(), B, T, L, 0.99, trace=tr)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    h_in = tr.h_in[0].cpu().double()
+    emb = O.loop_embedding(0, cfg.loop_dim, cfg.dim, cfg.loop_theta)
+    comb = O.rmsnorm(h_in + emb + e.double(), W["rec_norm_w"], cfg.norm_eps)
+    pos = torch.arange(B * T) % T
+    _, _, info = O.transformer_block(cfg, W, comb, B, pos, True)
+    f0 = O.rmsnorm(comb, W["ffn_norm_w"], cfg.norm_eps)
+    d_o = info["f"] - f0
+    d_k = tr.f[0].cpu().double() - f0
+    assert rel_l2(d_o, info["f"]) > 0.05, "attention barely moves f: the check would be weak"
+    for b in range(B):
+        rows = slice(b * T, (b + 1) * T)
+        err = rel_l2(d_k[rows], d_o[rows])
+        assert err <= BF16_TOL, f"sequence {b}: relative L2 of the MLA attention branch {err:.3e}"

@@ -102,6 +102,53 @@ def test_rdt1b_attention_late_key_tiles():
     assert err <= BF16_TOL, f"relative L2 of the attention branch over the last key tiles {err:.3e}"
 
 
+def test_rdt3b_mla_prefill_prefix_and_late_key_tiles():
+    """MLA prefill on the tensor cores at the 3B MLA shape (24 heads, nope 128 + rope 64,
+    value 128, kv_lora_rank 512), 1 x 4096, one loop: rows 0..63 against the oracle run on
+    that causal prefix, and the attention branch of f for the last 128 query rows, which see
+    all 32 key tiles (keys and values of the earlier positions through the oracle's own
+    latent-cache path)."""
+    wl = RI.get_workload("rdt3b_mla_decode")
+    cfg = wl.cfg
+    B, T = 1, 4096
+    dev = torch.device("cuda")
+    W = RI.block_weights(cfg, wl.seed, device=dev, attn_std=0.03)
+    h0, e = RI.recurrent_inputs(cfg, B, T, wl.seed, device=dev)
+    blk = R.RecurrentBlock(cfg, W)
+    Q, P = 128, 64
+    tp = R.Trace.alloc(cfg, 1, 0, P)                          # the prefix rows: routes checked
+    h_out, hw, ids = blk.forward(h0, e, B, T, 1, 0.0, trace=tp)
+    h_out, ids = h_out.clone(), ids.clone()
+    tr = R.Trace(T - Q, Q, f=torch.zeros(1, Q, cfg.dim, dtype=torch.float32, device=dev))
+    blk.forward(h0, e, B, T, 1, 0.0, trace=tr)                # the last rows: attention branch
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    Wc = _cpu(W)
+    rec = []
+    o_h, _, _, _ = O.recurrent_forward(cfg, Wc, h0[:P].cpu(), e[:P].cpu(), 1, 1, 0.0, record=rec,
+                                       route_ids=ids[:, :P].cpu().long())
+    check_route_flips(ids[:, :P], tp.biased_logits, rec)
+    assert rel_l2(h_out[:P], o_h) <= BF16_TOL
+    eps = cfg.norm_eps
+    emb = O.loop_embedding(0, cfg.loop_dim, cfg.dim, cfg.loop_theta)
+    comb = O.rmsnorm(h0.cpu().double() + emb + e.cpu().double(), Wc["rec_norm_w"], eps)
+    a = O.rmsnorm(comb, Wc["attn_norm_w"], eps)
+    pos = torch.arange(T)
+    ck, kr = [], []
+    for c0 in range(0, T - Q, 128):
+        _, c, r = O.mla_attention(cfg, Wc, a[c0:c0 + 128], pos[c0:c0 + 128])
+        ck.append(c)
+        kr.append(r)
+    cache = {"c_kv": torch.cat(ck), "k_rope": torch.cat(kr), "pos": pos[:T - Q]}
+    o, _, _ = O.mla_attention(cfg, Wc, a[T - Q:], pos[T - Q:], cache)
+    f_o = O.rmsnorm(comb[T - Q:] + o, Wc["ffn_norm_w"], eps)
+    f0 = O.rmsnorm(comb[T - Q:], Wc["ffn_norm_w"], eps)
+    d_o, d_k = f_o - f0, tr.f[0].cpu().double() - f0
+    assert rel_l2(d_o, f_o) > 0.05, "attention barely moves f: the check would be weak"
+    err = rel_l2(d_k, d_o)
+    assert err <= BF16_TOL, f"relative L2 of the MLA attention branch over the last key tiles {err:.3e}"
+
+
 def test_rdt3b_decode_sequences_match_oracle():
     """3B-shaped decode at full size (64 sequences, per-loop 4096-token random caches):
     sequences 0 and 37 against the oracle decode step."""

@@ -140,7 +140,7 @@ def _wide(H):
                         v_head_dim=128, dtype="bf16")
 
 
-@pytest.mark.parametrize("H", [16, 24])
+@pytest.mark.parametrize("H", [8, 16, 24, 32])
 def test_mla_absorbed_decode_wide_latent_ragged(H):
     """Absorbed decode at kv_lora_rank 512 against the oracle's decode step, with ragged
     cache lengths: several key ranges, a tile-aligned length + 1, an empty cache (the new
