@@ -48,6 +48,7 @@ struct TcArgs {
   int k_splits;        // > 1: split-K, tile t covers k-blocks of split t / (m_tiles n_n)
   int kb_split;        // k-blocks per split
   long long split_stride;   // elements between the fp32 partials of two splits
+  int group_m;         // row tiles per rasterization group (1: column tile fastest)
 };
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z)); }
@@ -82,15 +83,25 @@ __device__ __forceinline__ int rope_chunk(const GemmParams& p, int c) {
 
 struct TileInfo { int group, row0, rows, n0, split; };
 
-__device__ __forceinline__ TileInfo decode_tile(const TcArgs& a, int t) {
+// Tiles are walked in groups of group_m row tiles: inside a group the row tile varies
+// fastest, then the column tile.  The CTAs in flight at any moment then cover a few column
+// tiles of up to group_m row tiles, so each weight tile (B) is read from DRAM once per group
+// and the group's activation rows (A) stay in L2 across its column tiles.  With the column
+// tile fastest (group_m = 1), an expert holding many row tiles -- a popular expert under a
+// skewed router -- has its whole weight slab swept once per wave of CTAs, which only L2 can
+// absorb when the slab is small; the host picks group_m from the slab size.
+__device__ __forceinline__ TileInfo decode_tile(const TcArgs& a, int t, int m_tiles) {
   TileInfo ti;
   ti.split = 0;
   if (a.k_splits > 1) {
-    const int per = a.m_tiles * a.n_n;
+    const int per = m_tiles * a.n_n;
     ti.split = t / per;
     t %= per;
   }
-  const int m_i = t / a.n_n, n_i = t % a.n_n;
+  const int per_group = a.group_m * a.n_n;
+  const int gm0 = (t / per_group) * a.group_m, r = t % per_group;
+  const int gsz = min(a.group_m, m_tiles - gm0);   // the last group may hold fewer row tiles
+  const int m_i = gm0 + r % gsz, n_i = r / gsz;
   if (a.p.tiles) {
     ti.group = a.p.tiles[4 * m_i];
     ti.row0 = a.p.tiles[4 * m_i + 1];
@@ -221,7 +232,7 @@ __global__ void __launch_bounds__(192, 1)
     // test hook: a producer that issues nothing starves every consumer wait
     const int n_prod = p.test_no_loads ? 0 : total;
     for (int t = blockIdx.x; t < n_prod && !*abort_flag; t += gridDim.x) {
-      const TileInfo ti = decode_tile(args, t);
+      const TileInfo ti = decode_tile(args, t, m_tiles);
       const int gb = ti.group * args.b_rows_group;
       int b0, b1;
       if (EPI == EPI_SWIGLU_T) {
@@ -261,7 +272,7 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const uint32_t d = tmem + acc * BN;
       int k0, k1;
-      k_range(decode_tile(args, t), k0, k1);
+      k_range(decode_tile(args, t, m_tiles), k0, k1);
       for (int ks = k0; ks < k1; ++ks) {
         if (!(ok = mbar_wait(&full[stage], phase, abort_flag))) break;
         tc_fence_after();
@@ -287,7 +298,7 @@ __global__ void __launch_bounds__(192, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const TileInfo ti = decode_tile(args, t);
+      const TileInfo ti = decode_tile(args, t, m_tiles);
       const bool valid = rl < ti.rows;
       const long long r = (long long)ti.row0 + rl;
       // the residual does not depend on the accumulator: its first chunk is in flight
@@ -578,6 +589,12 @@ int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
   a.n_n = p.N / a.n_out_tile;
   a.m_tiles = p.tiles ? 0 : (p.M + tc::BM - 1) / tc::BM;
   a.b_rows_group = p.tiles ? (int)(p.b_group_stride / p.ldb) : 0;
+  // weight bytes one row tile sweeps (SwiGLU: gate and up rows): group the row tiles when
+  // that slab would not stay resident in L2 between the waves of CTAs
+  {
+    const long long slab = (long long)((epi == EPI_SWIGLU_T) ? 2 * p.N : p.N) * p.K * 2;
+    a.group_m = slab > (32ll << 20) ? 16 : 1;
+  }
   // B map extent: the caller's b_rows (all groups' rows), else N rows (SwiGLU: gate then up rows)
   CUtensorMap mA, mB;
   if (!make_map(&mA, p.A, (unsigned long long)p.M, p.K, p.lda, 128)) return -1;
