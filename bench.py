@@ -127,7 +127,15 @@ class ClockSampler:
 # DRAM traffic of one full-size expert-up launch of a workload, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum, 1 pass), valid only while the GEMM's
 # sources are the ones it was captured from (sha256 of k_gemm_tc.cu + tc_common.cuh).
-EXPERT_UP_TRAFFIC = {}
+EXPERT_UP_TRAFFIC = {
+    # mean over the 16 expert-up launches of one step (ncu --metrics dram__bytes_read.sum,
+    # dram__bytes_write.sum on the default prefill command of each workload)
+    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1725410640,
+                      "sha256": "fb6cfa4e868a79ba0fc49f384df30a91cae47fde4f3a40f321a57eb4bb85a665"},
+    # mean over the 24 expert-up launches of one step
+    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13139956576,
+                            "sha256": "fb6cfa4e868a79ba0fc49f384df30a91cae47fde4f3a40f321a57eb4bb85a665"},
+}
 
 
 def expert_up_traffic(wl):
