@@ -171,7 +171,9 @@ def expert_up_flops(wl, n_running: float) -> float:
 # CPU oracle sample (reference arm and cpu_baseline)
 # ------------------------------------------------------------------------------------------
 
-ORACLE_SAMPLE = {"rdt1b_prefill": (32, 4), "rdt10b_prefill_zipf": (8, 2)}   # positions, loops per sample
+ORACLE_SAMPLE = {"rdt1b_prefill": (32, 4), "rdt10b_prefill_zipf": (8, 2)}   # positions, loops per reference step
+# the cpu_baseline leg of the default line: one sample of about 10-15 s of host work
+CPU_BASELINE_SAMPLE = {"rdt1b_prefill": (128, 16), "rdt10b_prefill_zipf": (16, 6)}
 
 
 def oracle_sample(wl, W_cpu, h0, e, positions: int, loops: int, halt_off=None):
@@ -363,7 +365,7 @@ def run_prefill(args, wl, rank, world, local_rank, *, steps=None, e2e=True, cpu_
     W_cpu = None
     if cpu_baseline and rank == 0 and world == 1:
         W_cpu = {k: v.cpu() for k, v in W.items()}
-        pos, loops = ORACLE_SAMPLE.get(wl.name, (32, 4))
+        pos, loops = CPU_BASELINE_SAMPLE.get(wl.name, (32, 4))
         h0_c, e_c = h0[:pos].cpu(), e[:pos].cpu()
         off_c = None if halt_off is None else halt_off[:pos].cpu()
     del blk, ws, W, out, h0, e

@@ -389,9 +389,11 @@ int combine_sm_count() { return device_sm_count(); }
 
 template <typename T, int VPL>
 bool launch_combine_vpl(const CombineParams& p, int n_rows, cudaStream_t s) {
-  // rows split over 4 warps when the width allows (32 warps per SM, 16-register rows)
-  constexpr int WPR = (VPL % 4 == 0) ? 4 : ((VPL % 2 == 0) ? 2 : 1);
-  constexpr int GROUPS = 8;
+  // a row's columns split over warps so that each lane holds at most 4 float4 of a row
+  // (16 registers per row array: wider rows spilled at the 64-register limit of 1024
+  // threads), and about 32 warps per SM
+  constexpr int WPR = (VPL >= 16 && VPL % 4 == 0) ? VPL / 4 : ((VPL % 4 == 0) ? 4 : ((VPL % 2 == 0) ? 2 : 1));
+  constexpr int GROUPS = (32 / WPR) < 8 ? (32 / WPR) : 8;
   const size_t lbytes = (size_t)2 * p.r * p.D * sizeof(T);
   const bool lsmem = p.r > 0 && lbytes <= 160 * 1024 && (((size_t)p.r * p.D * sizeof(T)) % 16) == 0 &&
                      ((uintptr_t)p.lora_down % 16) == 0 && ((uintptr_t)p.lora_B % 16) == 0;
