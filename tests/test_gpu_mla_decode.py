@@ -132,15 +132,15 @@ def test_mla_chunked_prefill_reads_the_latent_cache(dtype):
 
 
 def _wide(H):
-    # DeepSeek-V2 latent widths (kv_lora_rank 512, rope 64); H 16 fills one 16-row MMA
-    # tile, H 24 two tiles with 8 padded rows
+    # DeepSeek-V2 latent widths (kv_lora_rank 512, rope 64); the heads are the 8-wide MMA
+    # columns: H 4, 12 and 20 leave padded columns inside a tile, H 32 fills four
     return RI.RDTConfig(dim=1536, n_heads=H, n_kv_heads=H, max_seq_len=1024, max_loop_iters=4, n_experts=8,
                         n_shared_experts=1, n_experts_per_tok=2, expert_dim=128, lora_rank=8, attn_type="mla",
                         kv_lora_rank=512, q_lora_rank=256, qk_rope_head_dim=64, qk_nope_head_dim=128,
                         v_head_dim=128, dtype="bf16")
 
 
-@pytest.mark.parametrize("H", [8, 16, 24, 32])
+@pytest.mark.parametrize("H", [4, 8, 12, 16, 20, 24, 32])
 def test_mla_absorbed_decode_wide_latent_ragged(H):
     """Absorbed decode at kv_lora_rank 512 against the oracle's decode step, with ragged
     cache lengths: several key ranges, a tile-aligned length + 1, an empty cache (the new
