@@ -5,10 +5,12 @@
 // One slot per sequence.  A tick runs the shared block once over all slots, each slot's
 // token at its own loop t_row[slot] (per-row loop embedding, LoRA scale row, loop cache and
 // last-loop flag).  After the tick, a token that halted (or ran its last loop) leaves:
+//   k_depth_fill_list      the (slot, loop) rows to fill this tick, compacted, and their
+//                          128-row GEMM tiles,
 //   k_depth_fill_prologue  the attention input of its remaining loops u > t_row, from its
 //                          frozen state (the loop embedding changes with u, the state not),
 //   fill GEMM (host side)  their keys / values (K/V rows of the QKV weight, RoPE at the
-//                          token's position),
+//                          token's position), over the device tile list of the fill rows,
 //   k_depth_fill_store     those keys / values into the loop caches u at the position,
 // so later tokens of its sequence find it at every loop, exactly as when the token stays
 // frozen in a lockstep step; then k_depth_refill puts the sequence's next token in the
@@ -51,23 +53,61 @@ __device__ __forceinline__ bool slot_finished(const DepthParams& p, int b) {
   return t >= 0 && (p.halted[b] || t == p.L - 1);
 }
 
-// Row r = b (L - 1) + (u - 1), u = 1 .. L - 1: the attention input of loop u for the token
-// that just left slot b at loop t_row[b] < u, from its frozen state:
-//   a = RMSNorm_attn(RMSNorm_rec(h + emb_u + e)).  Other rows are zero.
+// The fill rows of this tick, in slot order: for each finished slot b, its loops
+// u = t_row[b] + 1 .. L - 1.  One CTA: per-thread slot ranges, a block scan of their row
+// counts, then the list, its length and its GEMM row tiles (fill_tile_m rows each).
+constexpr int FILL_THREADS = 256;
+__global__ void __launch_bounds__(FILL_THREADS) k_depth_fill_list(DepthParams p) {
+  __shared__ int sums[FILL_THREADS];
+  const int t = threadIdx.x;
+  const int per = (p.B + FILL_THREADS - 1) / FILL_THREADS;
+  const int b0 = min(p.B, t * per), b1 = min(p.B, b0 + per);
+  int n = 0;
+  for (int b = b0; b < b1; ++b)
+    if (slot_finished(p, b)) n += p.L - 1 - p.t_row[b];
+  sums[t] = n;
+  __syncthreads();
+  for (int off = 1; off < FILL_THREADS; off <<= 1) {   // inclusive scan
+    const int v = t >= off ? sums[t - off] : 0;
+    __syncthreads();
+    sums[t] += v;
+    __syncthreads();
+  }
+  int r = sums[t] - n;
+  for (int b = b0; b < b1; ++b) {
+    if (!slot_finished(p, b)) continue;
+    for (int u = p.t_row[b] + 1; u < p.L; ++u, ++r) {
+      p.fill_b[r] = b;
+      p.fill_u[r] = u;
+    }
+  }
+  const int total = sums[FILL_THREADS - 1], tm = p.fill_tile_m;
+  const int ntiles = (total + tm - 1) / tm;
+  if (t == 0) {
+    *p.fill_n = total;
+    *p.fill_ntiles = ntiles;
+  }
+  for (int i = t; i < ntiles; i += FILL_THREADS) {
+    p.fill_tiles[4 * i] = 0;
+    p.fill_tiles[4 * i + 1] = tm * i;
+    p.fill_tiles[4 * i + 2] = min(tm, total - tm * i);
+    p.fill_tiles[4 * i + 3] = 0;
+  }
+}
+
+// Fill row r (slot b = fill_b[r], loop u = fill_u[r] > t_row[b]): the attention input of
+// loop u for the token that just left slot b, from its frozen state:
+//   a = RMSNorm_attn(RMSNorm_rec(h + emb_u + e)).  CTAs past the list's length return.
 template <typename T>
 __global__ void k_depth_fill_prologue(DepthParams p) {
   extern __shared__ float xs[];
   __shared__ float red[32];
   const int r = blockIdx.x;
-  const int b = r / (p.L - 1), u = r % (p.L - 1) + 1;
+  if (r >= *p.fill_n) return;
+  const int b = p.fill_b[r], u = p.fill_u[r];
   const long long D = p.D;
   T* a = (T*)p.a_fill + (long long)r * D;
-  const bool valid = slot_finished(p, b) && u > p.t_row[b];
-  if (threadIdx.x == 0) p.pos_fill[r] = valid ? p.pos[b] : 0;
-  if (!valid) {
-    for (long long d = threadIdx.x; d < D; d += blockDim.x) a[d] = from_f<T>(0.f);
-    return;
-  }
+  if (threadIdx.x == 0) p.pos_fill[r] = p.pos[b];
   const float* h = p.h + b * D;
   const T* e = (const T*)p.e_slot + b * D;
   const float* emb = p.emb_tab + (long long)u * p.emb_stride;
@@ -92,12 +132,12 @@ __global__ void k_depth_fill_prologue(DepthParams p) {
 }
 
 // The filled keys / values (kv_fill row r: Hkv hd rotated key columns, then Hkv hd value
-// columns) into loop cache u of sequence b at the token's position.
+// columns) into loop cache u = fill_u[r] of sequence b = fill_b[r] at the token's position.
 template <typename T>
 __global__ void k_depth_fill_store(DepthParams p) {
   const int r = blockIdx.x;
-  const int b = r / (p.L - 1), u = r % (p.L - 1) + 1;
-  if (!(slot_finished(p, b) && u > p.t_row[b])) return;
+  if (r >= *p.fill_n) return;
+  const int b = p.fill_b[r], u = p.fill_u[r];
   const int pos = p.pos[b];
   if (pos < 0 || pos >= p.t_max) {
     if (threadIdx.x == 0) record_status(p.st, ST_BOUNDS, 702, pos);
@@ -161,6 +201,10 @@ static inline int depth_threads(int D) { return D >= 2048 ? 256 : 128; }
 void launch_depth_start(int dtype, const DepthParams& p, cudaStream_t s) {
   if (dtype == 0) { k_depth_start<float><<<p.B, depth_threads(p.D), 0, s>>>(p); note_launch(); }
   else { k_depth_start<bf16><<<p.B, depth_threads(p.D), 0, s>>>(p); note_launch(); }
+}
+void launch_depth_fill_list(const DepthParams& p, cudaStream_t s) {
+  k_depth_fill_list<<<1, FILL_THREADS, 0, s>>>(p);
+  note_launch();
 }
 void launch_depth_fill_prologue(int dtype, const DepthParams& p, cudaStream_t s) {
   const size_t smem = (size_t)p.D * sizeof(float);

@@ -495,6 +495,11 @@ void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* 
   const int ctas = (N + 1023) / 1024;
   if (ctas <= 0) return;
   if (!cta_count || ctas > 4096) { k_compact<<<1, 1024, 0, s>>>(halted, N, run_list, run_idx, n_run); note_launch(); return; }
+  if (ctas == 1) {   // one CTA of ceil(N / 32) warps does it in a single launch
+    k_compact<<<1, (N + 31) / 32 * 32, 0, s>>>(halted, N, run_list, run_idx, n_run);
+    note_launch();
+    return;
+  }
   k_compact_count<<<ctas, 1024, 0, s>>>(halted, N, cta_count);
   note_launch();
   k_compact_scatter<<<ctas, 1024, 0, s>>>(halted, N, cta_count, run_list, run_idx, n_run);

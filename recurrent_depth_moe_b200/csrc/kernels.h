@@ -185,10 +185,13 @@ struct DepthParams {
   int* t_row; int* tok; int* out_row; float* cum; int* halted; int* pending;
   const float* emb_tab; const float* w_rec; const float* w_attn; float eps;   // emb_tab [L][emb_stride]
   void* a_fill; int* pos_fill; const void* kv_fill;                // [B (L-1)][D], [B (L-1)], [B (L-1)][2 Hkv hd]
+  int* fill_b; int* fill_u; int* fill_n;                           // fill row r = (slot fill_b[r], loop fill_u[r]), r < *fill_n
+  int* fill_tiles; int* fill_ntiles; int fill_tile_m;              // GEMM row tiles of the fill rows {0, row0, rows, 0}
   void* kc; void* vc; long long loop_elems;                        // GQA loop caches, elements per loop
   DevStatus* st;
 };
 void launch_depth_start(int dtype, const DepthParams& p, cudaStream_t s);
+void launch_depth_fill_list(const DepthParams& p, cudaStream_t s);
 void launch_depth_fill_prologue(int dtype, const DepthParams& p, cudaStream_t s);
 void launch_depth_fill_store(int dtype, const DepthParams& p, cudaStream_t s);
 void launch_depth_refill(int dtype, const DepthParams& p, cudaStream_t s);

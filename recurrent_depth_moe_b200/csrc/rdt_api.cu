@@ -538,8 +538,9 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
 // continuous depth-wise batching of decode steps
 // ------------------------------------------------------------------------------------------
 struct DepthLayout {
-  size_t t_row, tok, out_row, pending, e_slot, off_slot, emb_tab, a_fill, kv_fill, pos_fill, total;
-  int emb_stride;
+  size_t t_row, tok, out_row, pending, e_slot, off_slot, emb_tab, a_fill, kv_fill, pos_fill;
+  size_t fill_b, fill_u, fill_n, fill_tiles, fill_ntiles, total;
+  int emb_stride, fill_max_tiles;
 };
 
 // The decode layout of `batch` rows (one slot per sequence) followed by the slot state and
@@ -561,6 +562,12 @@ void make_depth_layout(const rdt_config* c, int B, int L, int t_max, Layout* Lo,
   DL->a_fill = take(nf * D * es);
   DL->kv_fill = take(nf * 2 * (size_t)c->n_kv_heads * hd * es);
   DL->pos_fill = take(nf * 4);
+  DL->fill_b = take(nf * 4);
+  DL->fill_u = take(nf * 4);
+  DL->fill_n = take(16);
+  DL->fill_max_tiles = (int)((nf + 63) / 64);   // the smaller of the two GEMM row tiles
+  DL->fill_tiles = take((size_t)DL->fill_max_tiles * 16);
+  DL->fill_ntiles = take(16);
   DL->total = off;
 }
 
@@ -611,6 +618,8 @@ rdt_status depth_setup(const rdt_depth_batch* db, cudaStream_t s, DepthCall* dc)
   dp.cum = at<float*>(ws, x.L.cum); dp.halted = at<int*>(ws, x.L.halted); dp.pending = at<int*>(ws, DL.pending);
   dp.emb_tab = at<float*>(ws, DL.emb_tab); dp.w_rec = w->rec_norm_w; dp.w_attn = w->attn_norm_w; dp.eps = c->norm_eps;
   dp.a_fill = at<void*>(ws, DL.a_fill); dp.pos_fill = at<int*>(ws, DL.pos_fill); dp.kv_fill = at<void*>(ws, DL.kv_fill);
+  dp.fill_b = at<int*>(ws, DL.fill_b); dp.fill_u = at<int*>(ws, DL.fill_u); dp.fill_n = at<int*>(ws, DL.fill_n);
+  dp.fill_tiles = at<int*>(ws, DL.fill_tiles); dp.fill_ntiles = at<int*>(ws, DL.fill_ntiles);
   dp.kc = cache->k; dp.vc = cache->v;
   dp.loop_elems = (long long)cache->batch * c->n_kv_heads * cache->t_max * hd;
   dp.st = x.st;
@@ -647,18 +656,24 @@ rdt_status depth_tick(const rdt_depth_batch* db, DepthCall& dc) {
   { ProfScope ps(PC_COMBINE, s); launch_combine(x.dtype, dc.cp, B, s); }
   if (L > 1) {
     ProfScope ps(PC_DEPTH_FILL, s);
-    launch_depth_fill_prologue(x.dtype, dp, s);
+    // the fill rows are compacted on the device; the GEMM runs over their row tiles only
     GemmParams g;
     memset(&g, 0, sizeof(g));
     g.impl = -1; g.st = x.st;
     g.A = dp.a_fill; g.lda = D;
     g.B = (const char*)w->w_qkv + (size_t)H * hd * D * esize(c); g.ldb = D;   // the K and V rows of w_qkv
     g.M = B * (L - 1); g.N = 2 * Hkv * hd; g.K = D;
+    g.tiles = dp.fill_tiles; g.n_tiles = dp.fill_ntiles; g.b_group_stride = 0; g.b_rows = g.N;
     g.C = const_cast<void*>(dp.kv_fill); g.ldc = 2 * Hkv * hd;
     g.pos = dp.pos_fill; g.rope_tab = at<const float2*>(ws, x.L.rope); g.rope_half = hd / 2; g.n_rope = 1;
     g.rope[0] = RopeDesc{0, Hkv, hd, 0, hd};
+    DepthParams fp = dp;
+    fp.fill_tile_m = gemm_tile_m(gemm_pick(x.dtype, g, EPI_ROPE_T));
+    g.max_tiles = (g.M + fp.fill_tile_m - 1) / fp.fill_tile_m;
+    launch_depth_fill_list(fp, s);
+    launch_depth_fill_prologue(x.dtype, fp, s);
     RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, s));
-    launch_depth_fill_store(x.dtype, dp, s);
+    launch_depth_fill_store(x.dtype, fp, s);
   }
   {
     ProfScope ps(PC_OTHER, s);
