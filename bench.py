@@ -130,11 +130,11 @@ class ClockSampler:
 EXPERT_UP_TRAFFIC = {
     # mean over the 16 expert-up launches of one step (ncu --metrics dram__bytes_read.sum,
     # dram__bytes_write.sum on the default prefill command of each workload)
-    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1725410640,
-                      "sha256": "fb6cfa4e868a79ba0fc49f384df30a91cae47fde4f3a40f321a57eb4bb85a665"},
+    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1726496704,
+                      "sha256": "b3e2ce69381eaa13db7926a715461cc13dfe0e4aefe8fec5807d68b3ab0ba3e3"},
     # mean over the 24 expert-up launches of one step
-    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13139956576,
-                            "sha256": "fb6cfa4e868a79ba0fc49f384df30a91cae47fde4f3a40f321a57eb4bb85a665"},
+    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13075452053,
+                            "sha256": "b3e2ce69381eaa13db7926a715461cc13dfe0e4aefe8fec5807d68b3ab0ba3e3"},
 }
 
 

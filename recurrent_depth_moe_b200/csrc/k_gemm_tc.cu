@@ -469,8 +469,11 @@ int pick_bn(const GemmParams& p, int epi) {
   if (epi == EPI_SWIGLU_T) return (p.N % 128 == 0) ? 256 : 0;
   if (epi == EPI_ROUTER) return (p.N == 64 || p.N == 128) ? p.N : 0;
   // rows that fit one 128-row tile (decode): the weights are the traffic, so the narrowest
-  // tile spreads them over the most CTAs
-  if (!p.tiles && p.M <= tc::BM && !p.vt && p.N % 64 == 0) return 64;
+  // tile spreads them over the most CTAs -- unless N is so wide that every CTA gets many
+  // tiles anyway (the vocabulary head): then 128-wide tiles halve the re-reads of the
+  // shared activation rows, which cross L2 once per tile
+  if (!p.tiles && p.M <= tc::BM && !p.vt && p.N % 64 == 0)
+    return (p.N % 128 == 0 && p.N / 64 >= 16 * sm_count()) ? 128 : 64;
   if (p.N % 256 == 0) return 256;
   if (p.N % 128 == 0) return 128;
   if (p.N % 64 == 0) return 64;
