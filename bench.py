@@ -161,6 +161,18 @@ def attention_flops(cfg, B: int, T: int) -> float:
     return float(B) * cfg.n_heads * (dqk + dv) * T * T
 
 
+def attention_flops_executed(cfg, last: torch.Tensor, T: int) -> float:
+    """Causal prefill attention of the rows that run, summed over the loops: a row at position
+    p running loop t attends to p + 1 keys, (score dim + value dim) * 2 FLOPs per head and key
+    (a halted row's query is not computed).  last[i] = the last loop row i ran."""
+    if cfg.attn_type == "gqa":
+        dqk = dv = cfg.head_dim
+    else:
+        dqk, dv = cfg.qk_nope_head_dim + cfg.qk_rope_head_dim, cfg.v_head_dim
+    pos = torch.arange(last.numel(), device=last.device) % T
+    return float(2.0 * cfg.n_heads * (dqk + dv) * ((last + 1).double() * (pos + 1).double()).sum().item())
+
+
 def expert_up_flops(wl, n_running: float) -> float:
     c = wl.cfg
     rows = n_running * (c.n_experts_per_tok + c.n_shared_experts)
@@ -382,10 +394,11 @@ def run_prefill(args, wl, rank, world, local_rank, *, steps=None, e2e=True, cpu_
     peak_t = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
     att = prof.get("attention", (0, 0.0))
     if att[0]:
-        att_tf = attention_flops(cfg, B, T) / (att[1] / att[0] / 1e3) / 1e12
+        att_flops = attention_flops_executed(cfg, last, T) / L   # per launch, the loops' average
+        att_tf = att_flops / (att[1] / att[0] / 1e3) / 1e12
         res["attention_roofline"] = {
             "bound": "tensor", "achieved": att_tf, "peak": peak_t, "unit": "TFLOP/s", "frac": att_tf / peak_t,
-            "flops_per_launch": attention_flops(cfg, B, T), "ms_per_launch": att[1] / att[0],
+            "flops_per_launch": att_flops, "ms_per_launch": att[1] / att[0],
             "kernel": ("k_attn_tc (tcgen05, GQA)" if cfg.attn_type == "gqa" else
                        "k_attn_tc (tcgen05, MLA: keys [k_nope | k_rope], values read in place)")}
     res["roofline"] = {"bound": "tensor", "kernel": "expert_up_swiglu (tcgen05 grouped GEMM, SwiGLU epilogue)",

@@ -69,8 +69,17 @@ struct Args {
   int q_col0, k_col0;      // GQA: qkv columns of query head 0 and key head 0
   int q_head, k_head;      // columns between heads: queries; keys / values (MLA: nope + v)
   int v_col0;              // MLA: column of the values inside a head's [k_nope | v] row
+  // compact queries (or nullptr): the query / output rows of sequence b are the compact rows
+  // seq_off[b] .. seq_off[b + 1]; compact row r sits at position q_pos[run_list[r]]
+  const int* seq_off;
+  const int* run_list;
   DevStatus* st;           // device status word: a wait that gave up is recorded here
 };
+
+// position of query row idx (a batch row, or a compact row in compact mode)
+__device__ __forceinline__ int query_pos(const Args& a, long long idx) {
+  return a.run_list ? a.q_pos[a.run_list[idx]] : a.q_pos[idx];
+}
 
 using namespace rdt::tc;
 
@@ -132,10 +141,11 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
 }
 
 // P = 2^(s * sl2 - base) for one row of BKV scores, written as bf16 pairs into the first
-// BKV / 2 TMEM columns at tS; returns the fp32 row sum.  POLY: pairs whose index has
-// (pair & 7) < 3 (3 in 8) take the FMA-pipe exponential, the rest the SFU; tiles with
-// masked keys use the SFU throughout, so masked keys (s = -inf) give exactly 0.
-template <bool POLY>
+// BKV / 2 TMEM columns at tS; returns the fp32 row sum.  Pairs whose index has
+// (pair & 7) < 3 (3 in 8) take the FMA-pipe exponential, the rest the SFU; a masked key
+// (s = -inf) gives exactly 0 on either.  The choice depends on the column alone, so a row's
+// P does not depend on which other rows share its warp (compact query tiles keep causal
+// results bit-identical).
 __device__ __forceinline__ float exp_row(const float (&s)[BKV], float sl2, float base, uint32_t tS) {
   const float2 sc = make_float2(sl2, sl2), nb = make_float2(-base, -base);
   float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -147,8 +157,10 @@ __device__ __forceinline__ float exp_row(const float (&s)[BKV], float sl2, float
       const int k = 32 * hh + 2 * pi;
       const float2 x = __ffma2_rn(make_float2(s[k], s[k + 1]), sc, nb);
       float2 p;
-      if (POLY && (pi & 7) < 3) {   // pair index within the row: (16 hh + pi) & 7 = pi & 7
+      if ((pi & 7) < 3) {   // pair index within the row: (16 hh + pi) & 7 = pi & 7
         p = ex2_poly2(x);
+        if (s[k] == -INFINITY) p.x = 0.f;
+        if (s[k + 1] == -INFINITY) p.y = 0.f;
       } else {
         p = make_float2(ex2_sfu(x.x), ex2_sfu(x.y));
       }
@@ -166,7 +178,7 @@ __device__ __forceinline__ float exp_row(const float (&s)[BKV], float sl2, float
 
 __device__ __forceinline__ int visible_tiles(const Args& a, long long row_last, int q_rows) {
   if (q_rows <= 0) return 0;
-  int n_vis = min(a.n_keys, a.q_pos[row_last] - a.key_pos0 + 1);
+  int n_vis = min(a.n_keys, query_pos(a, row_last) - a.key_pos0 + 1);
   return n_vis > 0 ? (n_vis + BKV - 1) / BKV : 0;
 }
 
@@ -203,13 +215,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int pair = n_pairs - 1 - (int)(blockIdx.x / BH);    // heaviest pairs first
   const int bh = blockIdx.x % BH;
   const int b = bh / a.H, h = bh % a.H, g = h / a.G;
+  // this sequence's query rows: rows b T .. b T + T - 1, or its compact rows
+  const long long qbase = a.seq_off ? (long long)a.seq_off[b] : (long long)b * a.T;
+  const int n_rows = a.seq_off ? a.seq_off[b + 1] - a.seq_off[b] : a.T;
   int q0[NQ], q_rows[NQ], nt[NQ];
   int nt_max = 0;
 #pragma unroll
   for (int q = 0; q < NQ; ++q) {
     q0[q] = (pair * NQ + q) * BQ;
-    q_rows[q] = max(0, min(BQ, a.T - q0[q]));
-    nt[q] = visible_tiles(a, (long long)b * a.T + q0[q] + q_rows[q] - 1, q_rows[q]);
+    q_rows[q] = max(0, min(BQ, n_rows - q0[q]));
+    nt[q] = visible_tiles(a, qbase + q0[q] + q_rows[q] - 1, q_rows[q]);
     nt_max = max(nt_max, nt[q]);
   }
 
@@ -253,7 +268,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
       if (q_rows[q] <= 0) continue;
-      const int qy = b * a.T + q0[q];
+      const int qy = (int)(qbase + q0[q]);
 #pragma unroll
       for (int kb = 0; kb < C::NBOX; ++kb) tma_load_2d(sQ + q * QTILE + kb * BOX, &tmQ, q_full, qx + 64 * kb, qy);
     }
@@ -353,10 +368,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int quarter = warp & 3;
     const int rl = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const long long row0 = (long long)b * a.T + q0[q];
+    const long long row0 = qbase + q0[q];
     const bool row_valid = rl < q_rows[q];
-    const int my_pos = row_valid ? a.q_pos[row0 + rl] : -1;
-    const int n_vis = row_valid ? min(a.n_keys, a.q_pos[row0 + q_rows[q] - 1] - a.key_pos0 + 1) : 0;
+    const int my_pos = row_valid ? query_pos(a, row0 + rl) : -1;
+    const int n_vis = row_valid ? min(a.n_keys, query_pos(a, row0 + q_rows[q] - 1) - a.key_pos0 + 1) : 0;
     const int ntq = nt[q];
     const uint32_t tO = tmem + lane_base + NQ * BKV + q * 128;
     float m_used = -INFINITY, l = 0.f;
@@ -403,9 +418,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       // P over the first 64 columns of the S buffer (S is in registers already)
       const float base = (m_used == -INFINITY) ? 0.f : m_used;
-      // exp_row stores to TMEM (.sync.aligned): the choice must be the same for the whole warp
-      l += __any_sync(0xffffffffu, need_mask) ? exp_row<false>(s, a.sl2, base, tS)
-                                              : exp_row<true>(s, a.sl2, base, tS);
+      l += exp_row(s, a.sl2, base, tS);
       if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // the max moved: O is rescaled before this tile's PV, after P is written so the S
         // row is no longer live (the PV of tile j - 1 is complete: it was issued before S
@@ -462,10 +475,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 // The prefill attention of a bf16 GQA block with head dim 128 can run here when the
 // values were also written transposed (p.vt) and rows are 16-byte aligned.
 bool attention_tc_supports(int dtype, const AttnParams& p) {
+  // keys in the QKV rows: the same rows as the queries, or (compact queries) their own rows
+  const bool keys = p.seq_off ? (p.run_list && p.k1_j % 8 == 0 && p.k1_b == (long long)p.T * p.k1_j &&
+                                 ((uintptr_t)p.k1 & 15) == 0 && p.q_row == (long long)p.H * 128)
+                              : (p.k1_j == p.q_row && p.k1_b == (long long)p.T * p.q_row);
   return dtype == 1 && p.vt && p.dn == 128 && p.dr == 0 && p.dv == 128 && !p.n_keys_dev && p.T % 8 == 0 &&
-         p.vt_ld == p.T && p.q_row % 8 == 0 && p.k1_j == p.q_row && p.k1_b == (long long)p.T * p.q_row &&
-         p.o_row % 8 == 0 && ((uintptr_t)p.q & 15) == 0 && ((uintptr_t)p.vt & 15) == 0 &&
-         ((uintptr_t)p.o & 15) == 0;
+         p.vt_ld == p.T && p.q_row % 8 == 0 && keys && p.o_row % 8 == 0 && ((uintptr_t)p.q & 15) == 0 &&
+         ((uintptr_t)p.vt & 15) == 0 && ((uintptr_t)p.o & 15) == 0;
 }
 
 // The MLA prefill of a bf16 block with nope 128, rope 64 and value 128 (the DeepSeek-V2
@@ -494,12 +510,18 @@ static int launch_attn_tc_t(const CUtensorMap& mQ, const CUtensorMap& mK, const 
 
 int launch_attention_tc(const AttnParams& p, cudaStream_t s) {
   const int Hkv = p.H / p.G;
-  // Q and K live in the qkv rows [B*T, q_row]; k1 points at key head 0 inside those rows
-  const long long k_col0 = ((const bf16*)p.k1 - (const bf16*)p.q);
   CUtensorMap mQ, mK, mVt;
   const unsigned long long rows = (unsigned long long)p.B * p.T;
+  long long k_col0 = 0;
   if (!tc_make_map(&mQ, p.q, rows, (unsigned long long)p.q_row, p.q_row, fat::BQ)) return -1;
-  if (!tc_make_map(&mK, p.q, rows, (unsigned long long)p.q_row, p.q_row, fat::BKV)) return -1;
+  if (p.seq_off) {
+    // compact queries in their own buffer; the keys: Hkv heads from key head 0 of the QKV rows
+    if (!tc_make_map(&mK, p.k1, rows, (unsigned long long)Hkv * fat::HD, p.k1_j, fat::BKV)) return -1;
+  } else {
+    // Q and K live in the qkv rows [B*T, q_row]; k1 points at key head 0 inside those rows
+    k_col0 = ((const bf16*)p.k1 - (const bf16*)p.q);
+    if (!tc_make_map(&mK, p.q, rows, (unsigned long long)p.q_row, p.q_row, fat::BKV)) return -1;
+  }
   if (!tc_make_map(&mVt, p.vt, (unsigned long long)p.B * Hkv * fat::HD, (unsigned long long)p.T, p.vt_ld, fat::HD))
     return -1;
   fat::Args a;
@@ -508,6 +530,7 @@ int launch_attention_tc(const AttnParams& p, cudaStream_t s) {
   a.sl2 = p.scale * 1.4426950408889634f;
   a.o = (bf16*)p.o; a.o_row = p.o_row;
   a.q_col0 = 0; a.k_col0 = (int)k_col0; a.q_head = fat::HD; a.k_head = fat::HD; a.v_col0 = 0; a.st = p.st;
+  a.seq_off = p.seq_off; a.run_list = p.seq_off ? p.run_list : nullptr;
   return launch_attn_tc_t<fat::CfgGqa>(mQ, mK, mK, mVt, a, s);
 }
 
@@ -525,6 +548,7 @@ int launch_attention_tc_mla(const AttnParams& p, cudaStream_t s) {
   a.sl2 = p.scale * 1.4426950408889634f;
   a.o = (bf16*)p.o; a.o_row = p.o_row;
   a.q_col0 = 0; a.k_col0 = 0; a.q_head = 192; a.k_head = 256; a.v_col0 = 128; a.st = p.st;
+  a.seq_off = nullptr; a.run_list = nullptr;
   return launch_attn_tc_t<fat::CfgMla>(mQ, mK, mKR, mV, a, s);
 }
 

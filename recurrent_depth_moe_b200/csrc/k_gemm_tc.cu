@@ -301,10 +301,12 @@ __global__ void __launch_bounds__(192, 1)
       const TileInfo ti = decode_tile(args, t, m_tiles);
       const bool valid = rl < ti.rows;
       const long long r = (long long)ti.row0 + rl;
+      // output / residual row (EPI_RESID_F32 with a row map: the product's rows are compact)
+      const long long ro = (EPI == EPI_RESID_F32 && p.row_map && valid) ? (long long)p.row_map[r] : r;
       // the residual does not depend on the accumulator: its first chunk is in flight
       // while this tile's MMAs finish, and chunk c + 1 while chunk c is stored
       float4 rcur[EPI == EPI_RESID_F32 ? 8 : 1], rnxt[EPI == EPI_RESID_F32 ? 8 : 1];
-      const float* rrow = (EPI == EPI_RESID_F32 && valid) ? p.resid + r * p.ld_resid + ti.n0 : nullptr;
+      const float* rrow = (EPI == EPI_RESID_F32 && valid) ? p.resid + ro * p.ld_resid + ti.n0 : nullptr;
       if (EPI == EPI_RESID_F32 && valid && args.k_splits <= 1) {
 #pragma unroll
         for (int q = 0; q < 8; ++q) rcur[q] = __ldg(reinterpret_cast<const float4*>(rrow) + q);
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(192, 1)
           float v[32];
           tmem_ld32(tbase + c, v);
           if (valid) {
-            float4* dst = reinterpret_cast<float4*>((float*)p.C + r * p.ldc + ti.n0 + c);
+            float4* dst = reinterpret_cast<float4*>((float*)p.C + ro * p.ldc + ti.n0 + c);
 #pragma unroll
             for (int q = 0; q < 8; ++q)
               dst[q] = make_float4(rcur[q].x + v[4 * q], rcur[q].y + v[4 * q + 1], rcur[q].z + v[4 * q + 2],
@@ -519,6 +521,7 @@ bool gemm_tc_supports(const GemmParams& p, int epi) {
   if (epi == EPI_ROUTER && (!p.bias || !p.ids || !p.gates || !p.rank || !p.counts || p.topk < 1 || p.topk > 32))
     return false;
   if (p.tiles && (p.b_group_stride % p.ldb || p.b_rows <= 0)) return false;
+  if (p.row_map && (epi != EPI_RESID_F32 || !p.tiles)) return false;   // compact rows: tile list, no split
   return encode_fn() != nullptr;
 }
 

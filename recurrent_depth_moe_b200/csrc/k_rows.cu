@@ -505,6 +505,54 @@ void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* 
   k_compact_scatter<<<ctas, 1024, 0, s>>>(halted, N, cta_count, run_list, run_idx, n_run);
   note_launch();
 }
+// seq_off[b] = number of running rows before sequence b (run_list is in row order, so a
+// lower bound of b T), and the 128-row tiles of the compact rows.
+__global__ void k_compact_meta(const int* __restrict__ run_list, const int* __restrict__ n_run_p, int B, int T,
+                               int* __restrict__ seq_off, int* __restrict__ tiles, int* __restrict__ n_tiles) {
+  const int n_run = *n_run_p;
+  for (int b = threadIdx.x; b <= B; b += blockDim.x) {
+    const long long key = (long long)b * T;
+    int lo = 0, hi = n_run;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if ((long long)run_list[mid] < key) lo = mid + 1;
+      else hi = mid;
+    }
+    seq_off[b] = lo;
+  }
+  const int nt = (n_run + 127) / 128;
+  if (threadIdx.x == 0) *n_tiles = nt;
+  for (int i = threadIdx.x; i < nt; i += blockDim.x) {
+    tiles[4 * i] = 0;
+    tiles[4 * i + 1] = 128 * i;
+    tiles[4 * i + 2] = min(128, n_run - 128 * i);
+    tiles[4 * i + 3] = 0;
+  }
+}
+void launch_compact_meta(const int* run_list, const int* n_run, int B, int T, int* seq_off, int* tiles,
+                         int* n_tiles, cudaStream_t s) {
+  k_compact_meta<<<1, 1024, 0, s>>>(run_list, n_run, B, T, seq_off, tiles, n_tiles);
+  note_launch();
+}
+
+// dst[r] = src[run_list[r]] for the compact rows r < n_run (16-byte vectors; CTAs past
+// n_run return)
+__global__ void __launch_bounds__(128) k_gather_rows(const uint8_t* __restrict__ src, long long src_ld,
+                                                     uint8_t* __restrict__ dst, long long dst_ld, long long nv,
+                                                     const int* __restrict__ run_list, const int* __restrict__ n_run) {
+  const int r = blockIdx.x;
+  if (r >= *n_run) return;
+  const int4* s4 = reinterpret_cast<const int4*>(src + (long long)run_list[r] * src_ld);
+  int4* d4 = reinterpret_cast<int4*>(dst + (long long)r * dst_ld);
+  for (long long v = threadIdx.x; v < nv; v += blockDim.x) d4[v] = __ldg(s4 + v);
+}
+void launch_gather_rows(const void* src, long long src_ld, void* dst, long long dst_ld, long long bytes,
+                        const int* run_list, const int* n_run, int N, cudaStream_t s) {
+  if (N <= 0) return;
+  k_gather_rows<<<N, 128, 0, s>>>((const uint8_t*)src, src_ld, (uint8_t*)dst, dst_ld, bytes / 16, run_list, n_run);
+  note_launch();
+}
+
 void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s) {
   { k_iota<<<(N + 255) / 256, 256, 0, s>>>(run_list, run_idx, n_run, N); note_launch(); }
 }

@@ -69,6 +69,9 @@ struct GemmParams {
   // test only: the tensor-core producer issues no loads, so the kernel's bounded waits run
   // out and it records a timeout (nothing is ever in flight); 0 in production
   int test_no_loads;
+  // EPI_RESID_F32 (optional): row r of the product is written to, and takes its residual
+  // from, row row_map[r] of C / resid
+  const int* row_map;
   DevStatus* st;
 };
 
@@ -101,10 +104,15 @@ struct AttnParams {
   // decode with rows at different loop depths: sequence b reads the loop cache
   // max(row_loop[b], 0), i.e. k1 / v advanced by that many loop_k / loop_v elements
   const int* row_loop; long long loop_k, loop_v;
+  // compact queries (tensor-core prefill): q holds only the running rows, in row order, and
+  // o receives them in the same order; sequence b's rows are q[seq_off[b] .. seq_off[b + 1])
+  // and compact row r is row run_list[r] of the batch (its position q_pos[run_list[r]])
+  const int* seq_off; const int* run_list;
   DevStatus* st;                                        // device status word (timeouts); may be null
 };
 int launch_attention(int dtype, const AttnParams& p, cudaStream_t s);
 int launch_attention_decode(int dtype, const AttnParams& p, cudaStream_t s);
+bool attention_tc_supports(int dtype, const AttnParams& p);   // the tensor-core prefill kernel takes p
 
 // MLA decode on the latent cache, weight-absorbed (bf16): q absorption, split-KV latent
 // attention over all heads of a sequence, range merge + value absorption into o.
@@ -224,6 +232,13 @@ void launch_to_model_dtype(const float* x, void* out, long long n, cudaStream_t 
 void launch_mla_to_cache(int dtype, const float* kv_raw, const void* krope, int kvr, int dr, const int* pos, int N,
                          int seq, int t_max, void* ckv_c, void* kr_c, DevStatus* st, cudaStream_t s);
 void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s);
+// Compact running rows: per-sequence offsets of run_list (seq_off[b] = first compact index
+// of sequence b's rows, [B + 1]) and the 128-row tiles of the n_run compact rows.
+void launch_compact_meta(const int* run_list, const int* n_run, int B, int T, int* seq_off, int* tiles,
+                         int* n_tiles, cudaStream_t s);
+// dst[r] = src[run_list[r]] for r < n_run: `bytes` per row (a multiple of 16), row strides in bytes
+void launch_gather_rows(const void* src, long long src_ld, void* dst, long long dst_ld, long long bytes,
+                        const int* run_list, const int* n_run, int N, cudaStream_t s);
 void launch_embed(int dtype, const void* table, int vocab, const int* ids, int n, int D, float* out,
                   DevStatus* st, cudaStream_t s);
 void launch_trace_rows(int src_is_model_dtype, int dtype, const void* src, int W, int row0, int n,

@@ -28,6 +28,7 @@ struct Layout {
   size_t mla_ckv_all, mla_kvu_all;   // MLA with earlier cached keys: rebuilt per-head keys / values
   size_t mla_qa;                     // MLA absorbed decode: absorbed queries (0 = path not used)
   size_t splitk; long long splitk_elems;   // split-K partials of single-tile GEMMs (decode)
+  size_t qc, seq_off, otiles, ontiles;     // compact queries of the running rows (GQA prefill; 0 = unused)
   int part_dim;                      // split-KV partial width (head dim, or kv_lora_rank)
   size_t total;
   int max_tiles, max_slots, rope_dim, rope_pos, n_split;
@@ -79,6 +80,12 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
     L->vt = take(N * (size_t)c->n_kv_heads * hd * es);   // values transposed per sequence
     dv = hd;
     L->rope_dim = hd;
+    if (T > 1 && c->dtype == 1) {   // prefill: the running rows' queries, gathered, and their tiles
+      L->qc = take(N * (size_t)H * hd * es);
+      L->seq_off = take((size_t)(B + 1) * 4);
+      L->otiles = take(((N + 127) / 128) * 16);
+      L->ontiles = take(16);
+    }
   } else {
     int dn = c->qk_nope_head_dim, dr = c->qk_rope_head_dim;
     dv = c->v_head_dim;
@@ -157,6 +164,7 @@ struct Ctx {
   DevStatus* st;
   int dtype;
   const int* row_loop = nullptr;   // decode rows at their own loop depth (continuous depth-wise batching)
+  bool compact_q = false;          // prefill with ACT: attention queries and O projection on the running rows
 };
 
 #define RDT_TRY(x)                          \
@@ -319,10 +327,37 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
     ap.scale = 1.f / sqrtf((float)(dn + dr));
   }
   ap.o = attn; ap.o_row = (long long)H * dv; ap.o_head = dv;
-  if (!absorbed) { ProfScope ps(PC_ATTN, x.s); RDT_TRY(launch_attention(x.dtype, ap, x.s)); }
   GemmParams g = gemm_base(x);
   g.A = attn; g.lda = (long long)H * dv; g.B = w->w_o; g.ldb = (long long)H * dv; g.M = N; g.N = D; g.K = H * dv;
   g.C = x1; g.ldc = D; g.resid = combined; g.ld_resid = D;
+  // Prefill with ACT: only the running rows need an attention output and x1 (a halted row
+  // keeps its state; its keys / values, written above, stay context for the others).  The
+  // running rows' queries are gathered (compact, in row order), the attention runs over them
+  // and the O projection over their tiles, writing x1 back through the row map.
+  if (x.compact_q && c->attn_type == 0 && x.L.qc && ap.vt) {
+    AttnParams cq = ap;
+    const int hd = dv;
+    cq.q = at<void*>(x.ws, x.L.qc); cq.q_row = (long long)H * hd;
+    cq.seq_off = at<const int*>(x.ws, x.L.seq_off); cq.run_list = at<const int*>(x.ws, x.L.run_list);
+    GemmParams gc = g;
+    gc.tiles = at<const int*>(x.ws, x.L.otiles); gc.n_tiles = at<const int*>(x.ws, x.L.ontiles);
+    gc.max_tiles = (N + 127) / 128; gc.b_group_stride = 0; gc.b_rows = D;
+    gc.row_map = at<const int*>(x.ws, x.L.run_list);
+    if (attention_tc_supports(x.dtype, cq) && gemm_pick(x.dtype, gc, EPI_RESID_F32) == GEMM_TC) {
+      const int* nrun = at<const int*>(x.ws, x.L.nrun);
+      {
+        ProfScope ps(PC_OTHER, x.s);
+        launch_compact_meta(cq.run_list, nrun, B, T, at<int*>(x.ws, x.L.seq_off), at<int*>(x.ws, x.L.otiles),
+                            at<int*>(x.ws, x.L.ontiles), x.s);
+        launch_gather_rows(ap.q, ap.q_row * es, at<void*>(x.ws, x.L.qc), cq.q_row * es, cq.q_row * es, cq.run_list,
+                           nrun, N, x.s);
+      }
+      { ProfScope ps(PC_ATTN, x.s); RDT_TRY(launch_attention(x.dtype, cq, x.s)); }
+      { ProfScope ps(PC_OPROJ, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_RESID_F32, gc, x.s)); }
+      return RDT_OK;
+    }
+  }
+  if (!absorbed) { ProfScope ps(PC_ATTN, x.s); RDT_TRY(launch_attention(x.dtype, ap, x.s)); }
   { ProfScope ps(PC_OPROJ, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_RESID_F32, g, x.s)); }
   return RDT_OK;
 }
@@ -449,6 +484,9 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
   x.c = c; x.w = w; x.ws = ws; x.s = s; x.dtype = c->dtype;
   make_layout(c, B, T, max_keys, &x.L);
   if ((st = check_ws(ws, ws_bytes, x.L)) != RDT_OK) return st;
+  // halted rows drop out of the attention queries and the O projection (prefill with ACT,
+  // keys from this call's rows)
+  x.compact_q = act_on && !decode && !(cache && cache->k && start_pos > 0);
   x.st = at<DevStatus*>(ws, x.L.status);
   const int N = B * T, D = c->dim, E = c->n_experts;
   const bool transformer_off = (flags & RDT_FLAG_TRANSFORMER_OFF) != 0;
