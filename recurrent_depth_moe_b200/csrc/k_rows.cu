@@ -506,10 +506,12 @@ void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* 
   note_launch();
 }
 // seq_off[b] = number of running rows before sequence b (run_list is in row order, so a
-// lower bound of b T), and the 128-row tiles of the compact rows.
+// lower bound of b T), the compact rows' positions and their 128-row tiles.
 __global__ void k_compact_meta(const int* __restrict__ run_list, const int* __restrict__ n_run_p, int B, int T,
-                               int* __restrict__ seq_off, int* __restrict__ tiles, int* __restrict__ n_tiles) {
+                               const int* __restrict__ pos, int* __restrict__ seq_off, int* __restrict__ pos_c,
+                               int* __restrict__ tiles, int* __restrict__ n_tiles) {
   const int n_run = *n_run_p;
+  for (int r = threadIdx.x; r < n_run; r += blockDim.x) pos_c[r] = pos[run_list[r]];
   for (int b = threadIdx.x; b <= B; b += blockDim.x) {
     const long long key = (long long)b * T;
     int lo = 0, hi = n_run;
@@ -529,9 +531,9 @@ __global__ void k_compact_meta(const int* __restrict__ run_list, const int* __re
     tiles[4 * i + 3] = 0;
   }
 }
-void launch_compact_meta(const int* run_list, const int* n_run, int B, int T, int* seq_off, int* tiles,
-                         int* n_tiles, cudaStream_t s) {
-  k_compact_meta<<<1, 1024, 0, s>>>(run_list, n_run, B, T, seq_off, tiles, n_tiles);
+void launch_compact_meta(const int* run_list, const int* n_run, int B, int T, const int* pos, int* seq_off,
+                         int* pos_c, int* tiles, int* n_tiles, cudaStream_t s) {
+  k_compact_meta<<<1, 1024, 0, s>>>(run_list, n_run, B, T, pos, seq_off, pos_c, tiles, n_tiles);
   note_launch();
 }
 

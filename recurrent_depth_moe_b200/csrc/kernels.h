@@ -233,9 +233,10 @@ void launch_mla_to_cache(int dtype, const float* kv_raw, const void* krope, int 
                          int seq, int t_max, void* ckv_c, void* kr_c, DevStatus* st, cudaStream_t s);
 void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s);
 // Compact running rows: per-sequence offsets of run_list (seq_off[b] = first compact index
-// of sequence b's rows, [B + 1]) and the 128-row tiles of the n_run compact rows.
-void launch_compact_meta(const int* run_list, const int* n_run, int B, int T, int* seq_off, int* tiles,
-                         int* n_tiles, cudaStream_t s);
+// of sequence b's rows, [B + 1]), their positions pos_c[r] = pos[run_list[r]], and the
+// 128-row tiles of the n_run compact rows.
+void launch_compact_meta(const int* run_list, const int* n_run, int B, int T, const int* pos, int* seq_off,
+                         int* pos_c, int* tiles, int* n_tiles, cudaStream_t s);
 // dst[r] = src[run_list[r]] for r < n_run: `bytes` per row (a multiple of 16), row strides in bytes
 void launch_gather_rows(const void* src, long long src_ld, void* dst, long long dst_ld, long long bytes,
                         const int* run_list, const int* n_run, int N, cudaStream_t s);

@@ -28,7 +28,7 @@ struct Layout {
   size_t mla_ckv_all, mla_kvu_all;   // MLA with earlier cached keys: rebuilt per-head keys / values
   size_t mla_qa;                     // MLA absorbed decode: absorbed queries (0 = path not used)
   size_t splitk; long long splitk_elems;   // split-K partials of single-tile GEMMs (decode)
-  size_t qc, seq_off, otiles, ontiles;     // compact queries of the running rows (GQA prefill; 0 = unused)
+  size_t qc, seq_off, pos_c, otiles, ontiles;   // compact queries of the running rows (GQA prefill; 0 = unused)
   int part_dim;                      // split-KV partial width (head dim, or kv_lora_rank)
   size_t total;
   int max_tiles, max_slots, rope_dim, rope_pos, n_split;
@@ -83,6 +83,7 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
     if (T > 1 && c->dtype == 1) {   // prefill: the running rows' queries, gathered, and their tiles
       L->qc = take(N * (size_t)H * hd * es);
       L->seq_off = take((size_t)(B + 1) * 4);
+      L->pos_c = take(N * 4);
       L->otiles = take(((N + 127) / 128) * 16);
       L->ontiles = take(16);
     }
@@ -215,8 +216,45 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
       if (gemm_pick(x.dtype, g, EPI_ROPE_T) != GEMM_TC) { g.vt = nullptr; want_vt = false; }
     }
     ap.vt = want_vt ? g.vt : nullptr; ap.vt_ld = T;
-    { ProfScope ps(PC_QKV, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, x.s)); }
-    ap.q = qkv; ap.q_row = W; ap.q_head = hd; ap.dn = hd; ap.dr = 0; ap.dv = hd; ap.G = H / Hkv;
+    // Compact queries (prefill with ACT on the tensor-core attention): keys / values for every
+    // row, queries only for the running rows, gathered in row order (their `a` rows into the
+    // f buffer, free until the MoE) and projected into their own buffer with RoPE at their
+    // positions.
+    bool compact = false;
+    GemmParams gq, gkv;
+    if (x.compact_q && want_vt && x.L.qc) {
+      gkv = g;
+      gkv.B = (const char*)w->w_qkv + (size_t)H * hd * D * es; gkv.N = 2 * Hkv * hd;
+      gkv.C = (char*)qkv + (size_t)H * hd * es; gkv.n_rope = 1; gkv.rope[0] = RopeDesc{0, Hkv, hd, 0, hd};
+      gkv.vt_col0 = Hkv * hd;
+      gq = gemm_base(x);
+      gq.A = at<void*>(x.ws, x.L.f); gq.lda = D; gq.B = w->w_qkv; gq.ldb = D; gq.M = N; gq.N = H * hd; gq.K = D;
+      gq.tiles = at<const int*>(x.ws, x.L.otiles); gq.n_tiles = at<const int*>(x.ws, x.L.ontiles);
+      gq.max_tiles = (N + 127) / 128; gq.b_group_stride = 0; gq.b_rows = (long long)H * hd;
+      gq.C = at<void*>(x.ws, x.L.qc); gq.ldc = (long long)H * hd; gq.pos = at<const int*>(x.ws, x.L.pos_c);
+      gq.rope_tab = tab; gq.rope_half = hd / 2; gq.n_rope = 1; gq.rope[0] = RopeDesc{0, H, hd, 0, hd};
+      compact = gemm_pick(x.dtype, gkv, EPI_ROPE_T) == GEMM_TC && gemm_pick(x.dtype, gq, EPI_ROPE_T) == GEMM_TC;
+    }
+    if (compact) {
+      const int* run_list = at<const int*>(x.ws, x.L.run_list);
+      const int* nrun = at<const int*>(x.ws, x.L.nrun);
+      {
+        ProfScope ps(PC_OTHER, x.s);
+        launch_compact_meta(run_list, nrun, B, T, pos, at<int*>(x.ws, x.L.seq_off), at<int*>(x.ws, x.L.pos_c),
+                            at<int*>(x.ws, x.L.otiles), at<int*>(x.ws, x.L.ontiles), x.s);
+        launch_gather_rows(a, (long long)D * es, at<void*>(x.ws, x.L.f), (long long)D * es, (long long)D * es,
+                           run_list, nrun, N, x.s);
+      }
+      ProfScope ps(PC_QKV, x.s);
+      RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, gkv, x.s));
+      RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, gq, x.s));
+      ap.q = at<void*>(x.ws, x.L.qc); ap.q_row = (long long)H * hd;
+      ap.seq_off = at<const int*>(x.ws, x.L.seq_off); ap.run_list = run_list;
+    } else {
+      { ProfScope ps(PC_QKV, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, g, x.s)); }
+      ap.q = qkv; ap.q_row = W;
+    }
+    ap.q_head = hd; ap.dn = hd; ap.dr = 0; ap.dv = hd; ap.G = H / Hkv;
     ap.scale = 1.f / sqrtf((float)hd);
     const bool use_cache = cache && cache->k;
     if (use_cache) {
@@ -330,32 +368,18 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
   GemmParams g = gemm_base(x);
   g.A = attn; g.lda = (long long)H * dv; g.B = w->w_o; g.ldb = (long long)H * dv; g.M = N; g.N = D; g.K = H * dv;
   g.C = x1; g.ldc = D; g.resid = combined; g.ld_resid = D;
-  // Prefill with ACT: only the running rows need an attention output and x1 (a halted row
-  // keeps its state; its keys / values, written above, stay context for the others).  The
-  // running rows' queries are gathered (compact, in row order), the attention runs over them
-  // and the O projection over their tiles, writing x1 back through the row map.
-  if (x.compact_q && c->attn_type == 0 && x.L.qc && ap.vt) {
-    AttnParams cq = ap;
-    const int hd = dv;
-    cq.q = at<void*>(x.ws, x.L.qc); cq.q_row = (long long)H * hd;
-    cq.seq_off = at<const int*>(x.ws, x.L.seq_off); cq.run_list = at<const int*>(x.ws, x.L.run_list);
+  // Compact queries: only the running rows get an attention output and x1 (a halted row keeps
+  // its state); the O projection runs over their tiles and writes x1 through the row map.
+  if (ap.seq_off) {
     GemmParams gc = g;
     gc.tiles = at<const int*>(x.ws, x.L.otiles); gc.n_tiles = at<const int*>(x.ws, x.L.ontiles);
     gc.max_tiles = (N + 127) / 128; gc.b_group_stride = 0; gc.b_rows = D;
-    gc.row_map = at<const int*>(x.ws, x.L.run_list);
-    if (attention_tc_supports(x.dtype, cq) && gemm_pick(x.dtype, gc, EPI_RESID_F32) == GEMM_TC) {
-      const int* nrun = at<const int*>(x.ws, x.L.nrun);
-      {
-        ProfScope ps(PC_OTHER, x.s);
-        launch_compact_meta(cq.run_list, nrun, B, T, at<int*>(x.ws, x.L.seq_off), at<int*>(x.ws, x.L.otiles),
-                            at<int*>(x.ws, x.L.ontiles), x.s);
-        launch_gather_rows(ap.q, ap.q_row * es, at<void*>(x.ws, x.L.qc), cq.q_row * es, cq.q_row * es, cq.run_list,
-                           nrun, N, x.s);
-      }
-      { ProfScope ps(PC_ATTN, x.s); RDT_TRY(launch_attention(x.dtype, cq, x.s)); }
-      { ProfScope ps(PC_OPROJ, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_RESID_F32, gc, x.s)); }
-      return RDT_OK;
-    }
+    gc.row_map = ap.run_list;
+    if (!attention_tc_supports(x.dtype, ap) || gemm_pick(x.dtype, gc, EPI_RESID_F32) != GEMM_TC)
+      return RDT_ERR_UNSUPPORTED;   // the shapes were checked before the queries were made compact
+    { ProfScope ps(PC_ATTN, x.s); RDT_TRY(launch_attention(x.dtype, ap, x.s)); }
+    { ProfScope ps(PC_OPROJ, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_RESID_F32, gc, x.s)); }
+    return RDT_OK;
   }
   if (!absorbed) { ProfScope ps(PC_ATTN, x.s); RDT_TRY(launch_attention(x.dtype, ap, x.s)); }
   { ProfScope ps(PC_OPROJ, x.s); RDT_TRY(launch_gemm(x.dtype, EPI_RESID_F32, g, x.s)); }
