@@ -341,12 +341,18 @@ __global__ void __launch_bounds__(GROUPS * WPR * 32, 1) k_combine_warp(CombinePa
     combine_row<T, VPL, WPR>(p, i, lane, g, zs[grp], Wd, Bl);
 }
 
-// out = RMSNorm(x) * w for fp32 rows of width D = 128 * VPL, one warp per row.
+// out = RMSNorm(x) * w for fp32 rows of width D = 128 * VPL, one warp per row; with a row
+// list, only rows rows[0 .. *n_rows) (the other rows are left as they are).
 template <typename T, int VPL>
 __global__ void __launch_bounds__(256) k_rmsnorm_warp(const float* __restrict__ x, const float* __restrict__ w,
-                                                      T* __restrict__ out, int N, int D, float eps) {
+                                                      T* __restrict__ out, int N, int D, float eps,
+                                                      const int* __restrict__ rows, const int* __restrict__ n_rows) {
   const int lane = threadIdx.x & 31;
-  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (rows) {
+    if (i >= *n_rows) return;
+    i = rows[i];
+  }
   if (i >= N) return;
   const long long rowD = (long long)i * D;
   float4 v[VPL];
@@ -370,13 +376,13 @@ __global__ void __launch_bounds__(256) k_rmsnorm_warp(const float* __restrict__ 
 static inline bool al(const void* q, int b) { return ((uintptr_t)q % b) == 0; }
 
 bool launch_rmsnorm_warp(int dtype, const float* x, const float* w, void* out, int N, int D, float eps,
-                         cudaStream_t s) {
+                         cudaStream_t s, const int* rows, const int* n_rows) {
   if (D % 128 || !al(x, 16) || !al(w, 16) || !al(out, dtype == 0 ? 16 : 8)) return false;
   const unsigned blocks = (unsigned)((N + 7) / 8);
 #define RDT_RW(V)                                                                                             \
   case V:                                                                                                     \
-    if (dtype == 0) { k_rmsnorm_warp<float, V><<<blocks, 256, 0, s>>>(x, w, (float*)out, N, D, eps); note_launch(); } \
-    else { k_rmsnorm_warp<bf16, V><<<blocks, 256, 0, s>>>(x, w, (bf16*)out, N, D, eps); note_launch(); }    \
+    if (dtype == 0) { k_rmsnorm_warp<float, V><<<blocks, 256, 0, s>>>(x, w, (float*)out, N, D, eps, rows, n_rows); note_launch(); } \
+    else { k_rmsnorm_warp<bf16, V><<<blocks, 256, 0, s>>>(x, w, (bf16*)out, N, D, eps, rows, n_rows); note_launch(); }    \
     return true;
   switch (D / 128) {
     RDT_RW(1) RDT_RW(2) RDT_RW(4) RDT_RW(8) RDT_RW(12) RDT_RW(16) RDT_RW(24) RDT_RW(32)

@@ -396,7 +396,14 @@ void launch_loop_prologue(int dtype, const float* h, const void* e, const float*
                                                           combined, (bf16*)a, D, eps, row_loop, emb_stride); note_launch(); }
 }
 bool launch_rmsnorm_warp(int dtype, const float* x, const float* w, void* out, int N, int D, float eps,
-                         cudaStream_t s);
+                         cudaStream_t s, const int* rows = nullptr, const int* n_rows = nullptr);
+
+// RMSNorm of the running rows only (row list run_list[0 .. *n_run)), fp32 input rows of
+// width D; false when the shape needs the all-rows kernel
+bool launch_rmsnorm_rows(int dtype, const float* x, const float* w, void* out, int N, int D, float eps,
+                         const int* run_list, const int* n_run, cudaStream_t s) {
+  return launch_rmsnorm_warp(dtype, x, w, out, N, D, eps, s, run_list, n_run);
+}
 
 void launch_rmsnorm(int in_f32, int dtype, const void* x, long long in_ld, const float* w, void* out,
                     long long out_ld, int rows, int D, float eps, cudaStream_t s) {
@@ -506,12 +513,10 @@ void launch_compact(const int* halted, int N, int* run_list, int* run_idx, int* 
   note_launch();
 }
 // seq_off[b] = number of running rows before sequence b (run_list is in row order, so a
-// lower bound of b T), the compact rows' positions and their 128-row tiles.
+// lower bound of b T), and the 128-row tiles of the compact rows.
 __global__ void k_compact_meta(const int* __restrict__ run_list, const int* __restrict__ n_run_p, int B, int T,
-                               const int* __restrict__ pos, int* __restrict__ seq_off, int* __restrict__ pos_c,
-                               int* __restrict__ tiles, int* __restrict__ n_tiles) {
+                               int* __restrict__ seq_off, int* __restrict__ tiles, int* __restrict__ n_tiles) {
   const int n_run = *n_run_p;
-  for (int r = threadIdx.x; r < n_run; r += blockDim.x) pos_c[r] = pos[run_list[r]];
   for (int b = threadIdx.x; b <= B; b += blockDim.x) {
     const long long key = (long long)b * T;
     int lo = 0, hi = n_run;
@@ -531,27 +536,44 @@ __global__ void k_compact_meta(const int* __restrict__ run_list, const int* __re
     tiles[4 * i + 3] = 0;
   }
 }
-void launch_compact_meta(const int* run_list, const int* n_run, int B, int T, const int* pos, int* seq_off,
-                         int* pos_c, int* tiles, int* n_tiles, cudaStream_t s) {
-  k_compact_meta<<<1, 1024, 0, s>>>(run_list, n_run, B, T, pos, seq_off, pos_c, tiles, n_tiles);
+void launch_compact_meta(const int* run_list, const int* n_run, int B, int T, int* seq_off, int* tiles,
+                         int* n_tiles, cudaStream_t s) {
+  k_compact_meta<<<1, 1024, 0, s>>>(run_list, n_run, B, T, seq_off, tiles, n_tiles);
   note_launch();
 }
 
-// dst[r] = src[run_list[r]] for the compact rows r < n_run (16-byte vectors; CTAs past
-// n_run return)
-__global__ void __launch_bounds__(128) k_gather_rows(const uint8_t* __restrict__ src, long long src_ld,
-                                                     uint8_t* __restrict__ dst, long long dst_ld, long long nv,
-                                                     const int* __restrict__ run_list, const int* __restrict__ n_run) {
-  const int r = blockIdx.x;
-  if (r >= *n_run) return;
-  const int4* s4 = reinterpret_cast<const int4*>(src + (long long)run_list[r] * src_ld);
-  int4* d4 = reinterpret_cast<int4*>(dst + (long long)r * dst_ld);
-  for (long long v = threadIdx.x; v < nv; v += blockDim.x) d4[v] = __ldg(s4 + v);
+// dst[r] = src[run_list[r]] for the compact rows r < n_run: a warp per row (rows strided over
+// the grid's warps), 16-byte vectors, four loads in flight per lane; with pos_c, also the
+// compact rows' positions pos_c[r] = pos[run_list[r]]
+__global__ void __launch_bounds__(256) k_gather_rows(const uint8_t* __restrict__ src, long long src_ld,
+                                                     uint8_t* __restrict__ dst, long long dst_ld, int nv,
+                                                     const int* __restrict__ run_list, const int* __restrict__ n_run,
+                                                     const int* __restrict__ pos, int* __restrict__ pos_c) {
+  const int lane = threadIdx.x & 31;
+  const int n = *n_run;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < n; r += warps) {
+    const int i = run_list[r];
+    if (pos_c && lane == 0) pos_c[r] = pos[i];
+    const int4* s4 = reinterpret_cast<const int4*>(src + (long long)i * src_ld);
+    int4* d4 = reinterpret_cast<int4*>(dst + (long long)r * dst_ld);
+    for (int v0 = lane; v0 < nv; v0 += 128) {
+      int4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v0 + 32 * u < nv) v[u] = __ldg(s4 + v0 + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (v0 + 32 * u < nv) d4[v0 + 32 * u] = v[u];
+    }
+  }
 }
 void launch_gather_rows(const void* src, long long src_ld, void* dst, long long dst_ld, long long bytes,
-                        const int* run_list, const int* n_run, int N, cudaStream_t s) {
+                        const int* run_list, const int* n_run, int N, cudaStream_t s, const int* pos, int* pos_c) {
   if (N <= 0) return;
-  k_gather_rows<<<N, 128, 0, s>>>((const uint8_t*)src, src_ld, (uint8_t*)dst, dst_ld, bytes / 16, run_list, n_run);
+  const int grid = (int)std::min<long long>((N + 7) / 8, 8LL * device_sm_count());
+  k_gather_rows<<<std::max(grid, 1), 256, 0, s>>>((const uint8_t*)src, src_ld, (uint8_t*)dst, dst_ld,
+                                                  (int)(bytes / 16), run_list, n_run, pos, pos_c);
   note_launch();
 }
 

@@ -214,6 +214,8 @@ void launch_loop_prologue(int dtype, const float* h, const void* e, const float*
                           const float* w_rec, const float* w_attn, float* combined, void* a,
                           int N, int D, float eps, cudaStream_t s, const int* row_loop = nullptr,
                           int emb_stride = 0);
+bool launch_rmsnorm_rows(int dtype, const float* x, const float* w, void* out, int N, int D, float eps,
+                         const int* run_list, const int* n_run, cudaStream_t s);   // running rows only
 void launch_rmsnorm(int in_f32, int dtype, const void* x, long long in_ld, const float* w, void* out,
                     long long out_ld, int rows, int D, float eps, cudaStream_t s);
 void launch_mla_kv_prep(int dtype, const float* kv_raw, int kvr, int dr, const float* kv_norm_w, float eps,
@@ -233,13 +235,14 @@ void launch_mla_to_cache(int dtype, const float* kv_raw, const void* krope, int 
                          int seq, int t_max, void* ckv_c, void* kr_c, DevStatus* st, cudaStream_t s);
 void launch_iota(int* run_list, int* run_idx, int* n_run, int N, cudaStream_t s);
 // Compact running rows: per-sequence offsets of run_list (seq_off[b] = first compact index
-// of sequence b's rows, [B + 1]), their positions pos_c[r] = pos[run_list[r]], and the
-// 128-row tiles of the n_run compact rows.
-void launch_compact_meta(const int* run_list, const int* n_run, int B, int T, const int* pos, int* seq_off,
-                         int* pos_c, int* tiles, int* n_tiles, cudaStream_t s);
-// dst[r] = src[run_list[r]] for r < n_run: `bytes` per row (a multiple of 16), row strides in bytes
+// of sequence b's rows, [B + 1]) and the 128-row tiles of the n_run compact rows.
+void launch_compact_meta(const int* run_list, const int* n_run, int B, int T, int* seq_off, int* tiles,
+                         int* n_tiles, cudaStream_t s);
+// dst[r] = src[run_list[r]] for r < n_run: `bytes` per row (a multiple of 16), row strides in
+// bytes; with pos_c also pos_c[r] = pos[run_list[r]]
 void launch_gather_rows(const void* src, long long src_ld, void* dst, long long dst_ld, long long bytes,
-                        const int* run_list, const int* n_run, int N, cudaStream_t s);
+                        const int* run_list, const int* n_run, int N, cudaStream_t s, const int* pos = nullptr,
+                        int* pos_c = nullptr);
 void launch_embed(int dtype, const void* table, int vocab, const int* ids, int n, int D, float* out,
                   DevStatus* st, cudaStream_t s);
 void launch_trace_rows(int src_is_model_dtype, int dtype, const void* src, int W, int row0, int n,

@@ -222,7 +222,7 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
     // positions.
     bool compact = false;
     GemmParams gq, gkv;
-    if (x.compact_q && want_vt && x.L.qc) {
+    if (x.compact_q && loop_t > 0 && want_vt && x.L.qc) {   // loop 0 runs every row
       gkv = g;
       gkv.B = (const char*)w->w_qkv + (size_t)H * hd * D * es; gkv.N = 2 * Hkv * hd;
       gkv.C = (char*)qkv + (size_t)H * hd * es; gkv.n_rope = 1; gkv.rope[0] = RopeDesc{0, Hkv, hd, 0, hd};
@@ -240,10 +240,10 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
       const int* nrun = at<const int*>(x.ws, x.L.nrun);
       {
         ProfScope ps(PC_OTHER, x.s);
-        launch_compact_meta(run_list, nrun, B, T, pos, at<int*>(x.ws, x.L.seq_off), at<int*>(x.ws, x.L.pos_c),
-                            at<int*>(x.ws, x.L.otiles), at<int*>(x.ws, x.L.ontiles), x.s);
+        launch_compact_meta(run_list, nrun, B, T, at<int*>(x.ws, x.L.seq_off), at<int*>(x.ws, x.L.otiles),
+                            at<int*>(x.ws, x.L.ontiles), x.s);
         launch_gather_rows(a, (long long)D * es, at<void*>(x.ws, x.L.f), (long long)D * es, (long long)D * es,
-                           run_list, nrun, N, x.s);
+                           run_list, nrun, N, x.s, pos, at<int*>(x.ws, x.L.pos_c));
       }
       ProfScope ps(PC_QKV, x.s);
       RDT_TRY(launch_gemm(x.dtype, EPI_ROPE_T, gkv, x.s));
@@ -392,7 +392,13 @@ rdt_status moe_block(Ctx& x, int N, const float* x1) {
   const rdt_weights* w = x.w;
   const int D = c->dim, E = c->n_experts, k = c->top_k, S = c->n_shared_experts, F = c->expert_dim;
   void* f = at<void*>(x.ws, x.L.f);
-  { ProfScope ps(PC_FFN_NORM, x.s); launch_rmsnorm(1, x.dtype, x1, D, w->ffn_norm_w, f, D, N, D, c->norm_eps, x.s); }
+  {
+    // the router and the experts read f of the running rows only
+    ProfScope ps(PC_FFN_NORM, x.s);
+    if (!launch_rmsnorm_rows(x.dtype, x1, w->ffn_norm_w, f, N, D, c->norm_eps, at<const int*>(x.ws, x.L.run_list),
+                             at<const int*>(x.ws, x.L.nrun), x.s))
+      launch_rmsnorm(1, x.dtype, x1, D, w->ffn_norm_w, f, D, N, D, c->norm_eps, x.s);
+  }
   float* logits = at<float*>(x.ws, x.L.logits);
   RouteParams rp;
   memset(&rp, 0, sizeof(rp));
