@@ -151,16 +151,6 @@ def expert_up_traffic(wl):
     return rec["bytes"] if h.hexdigest() == rec["sha256"] else None
 
 
-def attention_flops(cfg, B: int, T: int) -> float:
-    """Causal prefill attention per launch: per (sequence, head) S = Q K^T and O = P V over the
-    T^2 / 2 visible (query, key) pairs, 2 FLOPs per multiply-add: (score dim + value dim) T^2."""
-    if cfg.attn_type == "gqa":
-        dqk = dv = cfg.head_dim
-    else:
-        dqk, dv = cfg.qk_nope_head_dim + cfg.qk_rope_head_dim, cfg.v_head_dim
-    return float(B) * cfg.n_heads * (dqk + dv) * T * T
-
-
 def attention_flops_executed(cfg, last: torch.Tensor, T: int) -> float:
     """Causal prefill attention of the rows that run, summed over the loops: a row at position
     p running loop t attends to p + 1 keys, (score dim + value dim) * 2 FLOPs per head and key

@@ -62,3 +62,21 @@ def test_decode_bytes_follow_the_realised_routing():
     ids2 = ids.clone()
     ids2[1, 0] = -1
     assert bench.decode_algorithmic_bytes(cfg, ids2, lens) == got
+
+
+def test_attention_flops_count_the_keys_each_running_row_sees():
+    """Brute force over (loop, row, key): a row at position p that runs loop t sees keys
+    0 .. p; each (query, key) pair costs (score dim + value dim) multiply-adds per head."""
+    for name in ("mid_gqa_bf16", "tiny_mla_bf16"):
+        cfg = RI.get_workload(name).cfg
+        T, L = 5, 3
+        last = torch.tensor([2, 0, 1, 2, 2, 0, 0, 1, 2, 1])    # two sequences of 5; last loop each row ran
+        d = (2 * cfg.head_dim) if cfg.attn_type == "gqa" else \
+            (cfg.qk_nope_head_dim + cfg.qk_rope_head_dim + cfg.v_head_dim)
+        want = 0
+        for t in range(L):
+            for i in range(last.numel()):
+                if t <= int(last[i]):
+                    for key in range(i % T + 1):
+                        want += 2 * cfg.n_heads * d
+        assert bench.attention_flops_executed(cfg, last, T) == float(want), name
