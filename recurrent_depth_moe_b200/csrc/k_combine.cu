@@ -308,9 +308,9 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
 }
 
 // Persistent: GROUPS row groups of WPR warps per CTA, one CTA per SM, rows strided over
-// the grid.  With LSMEM the LoRA matrices (2 r D elements) are staged in shared memory once
+// the grid.  With LSMEM the LoRA matrices (2 r D elements, or the down one alone) are staged in shared memory once
 // per CTA, so the rank-r projections read shared memory instead of L2.
-template <typename T, int VPL, int WPR, int GROUPS, bool LSMEM>
+template <typename T, int VPL, int WPR, int GROUPS, int LSMEM>
 __global__ void __launch_bounds__(GROUPS * WPR * 32, 1) k_combine_warp(CombineParams p) {
   extern __shared__ __align__(16) uint8_t csm[];
   __shared__ float zs[GROUPS][64];
@@ -324,6 +324,7 @@ __global__ void __launch_bounds__(GROUPS * WPR * 32, 1) k_combine_warp(CombinePa
   const T* Wd = (const T*)p.lora_down;
   const T* Bl = (const T*)p.lora_B;
   if (LSMEM && p.r > 0 && !p.transformer_off && !p.block_only) {
+    // LSMEM 1: both matrices in shared memory; 2: the down projection only (both do not fit)
     const size_t bytes = (size_t)p.r * p.D * sizeof(T);
     const int4* gs0 = reinterpret_cast<const int4*>(p.lora_down);
     const int4* gs1 = reinterpret_cast<const int4*>(p.lora_B);
@@ -331,11 +332,11 @@ __global__ void __launch_bounds__(GROUPS * WPR * 32, 1) k_combine_warp(CombinePa
     int4* d1 = reinterpret_cast<int4*>(csm + bytes);
     for (size_t v = threadIdx.x; v < bytes / 16; v += blockDim.x) {
       d0[v] = __ldg(gs0 + v);
-      d1[v] = __ldg(gs1 + v);
+      if (LSMEM == 1) d1[v] = __ldg(gs1 + v);
     }
     __syncthreads();
     Wd = reinterpret_cast<const T*>(csm);
-    Bl = reinterpret_cast<const T*>(csm + bytes);
+    if (LSMEM == 1) Bl = reinterpret_cast<const T*>(csm + bytes);
   }
   for (int i = blockIdx.x * GROUPS + grp; i < p.N; i += gridDim.x * GROUPS)
     combine_row<T, VPL, WPR>(p, i, lane, g, zs[grp], Wd, Bl);
@@ -400,9 +401,12 @@ bool launch_combine_vpl(const CombineParams& p, int n_rows, cudaStream_t s) {
   // threads), and about 32 warps per SM
   constexpr int WPR = (VPL >= 16 && VPL % 4 == 0) ? VPL / 4 : ((VPL % 4 == 0) ? 4 : ((VPL % 2 == 0) ? 2 : 1));
   constexpr int GROUPS = (32 / WPR) < 8 ? (32 / WPR) : 8;
-  const size_t lbytes = (size_t)2 * p.r * p.D * sizeof(T);
-  const bool lsmem = p.r > 0 && lbytes <= 160 * 1024 && (((size_t)p.r * p.D * sizeof(T)) % 16) == 0 &&
-                     ((uintptr_t)p.lora_down % 16) == 0 && ((uintptr_t)p.lora_B % 16) == 0;
+  // LoRA matrices in shared memory: both when they fit in 160 KB, else the down projection
+  // alone when it fits in 200 KB (the row group's per-row reads of it then stay on the SM)
+  const size_t one = (size_t)p.r * p.D * sizeof(T);
+  const bool al_ok = p.r > 0 && (one % 16) == 0 && ((uintptr_t)p.lora_down % 16) == 0 && ((uintptr_t)p.lora_B % 16) == 0;
+  const int lsmem = !al_ok ? 0 : (2 * one <= 160 * 1024 ? 1 : (one <= 200 * 1024 ? 2 : 0));
+  const size_t lbytes = lsmem == 1 ? 2 * one : one;
   const int sms = combine_sm_count();
   if (n_rows <= 2 * sms) {
     // few rows (decode): one CTA per row with one warp per 128 columns, so the rows spread
@@ -410,16 +414,19 @@ bool launch_combine_vpl(const CombineParams& p, int n_rows, cudaStream_t s) {
     // array; the LoRA matrices are read through L1 / L2 (staging them would cost more than
     // one row uses)
     constexpr int WPR_S = VPL;
-    { k_combine_warp<T, VPL, WPR_S, 1, false><<<std::max(1, n_rows), WPR_S * 32, 0, s>>>(p); note_launch(); }
+    { k_combine_warp<T, VPL, WPR_S, 1, 0><<<std::max(1, n_rows), WPR_S * 32, 0, s>>>(p); note_launch(); }
     return true;
   }
   const int grid = std::max(1, std::min((n_rows + GROUPS - 1) / GROUPS, sms));
   constexpr int THREADS = GROUPS * WPR * 32;
-  if (lsmem) {
-    if (!ensure_smem_limit((const void*)k_combine_warp<T, VPL, WPR, GROUPS, true>, 160 * 1024)) return false;
-    { k_combine_warp<T, VPL, WPR, GROUPS, true><<<grid, THREADS, lbytes, s>>>(p); note_launch(); }
+  if (lsmem == 1) {
+    if (!ensure_smem_limit((const void*)k_combine_warp<T, VPL, WPR, GROUPS, 1>, 160 * 1024)) return false;
+    { k_combine_warp<T, VPL, WPR, GROUPS, 1><<<grid, THREADS, lbytes, s>>>(p); note_launch(); }
+  } else if (lsmem == 2) {
+    if (!ensure_smem_limit((const void*)k_combine_warp<T, VPL, WPR, GROUPS, 2>, 200 * 1024)) return false;
+    { k_combine_warp<T, VPL, WPR, GROUPS, 2><<<grid, THREADS, lbytes, s>>>(p); note_launch(); }
   } else {
-    { k_combine_warp<T, VPL, WPR, GROUPS, false><<<grid, THREADS, 0, s>>>(p); note_launch(); }
+    { k_combine_warp<T, VPL, WPR, GROUPS, 0><<<grid, THREADS, 0, s>>>(p); note_launch(); }
   }
   return true;
 }
