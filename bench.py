@@ -610,7 +610,7 @@ def run_decode(args, rank, world, local_rank, name="rdt3b_decode"):
         attn_desc = (f"{cfg.n_heads} heads MLA (kv_lora_rank {cfg.kv_lora_rank}, q_lora_rank {cfg.q_lora_rank}, "
                      f"rope {cfg.qk_rope_head_dim}, nope {cfg.qk_nope_head_dim}, v {cfg.v_head_dim}; latent cache, "
                      f"absorbed)")
-        attn_kernel = "k_mla_q_absorb + k_mla_attn + k_mla_out (split-KV latent attention, mma.sync)"
+        attn_kernel = "k_mla_q_absorb + k_mla_attn_tc + k_mla_out (split-KV latent attention; tcgen05 at kv_lora_rank 512)"
     res = {"metric": "decode tokens/s", "value": B * world / (ms_max / 1e3), "unit": "tokens/s",
            "ms_per_step": ms_max, "steps": steps,
            "workload": (f"{wl.name}: 3B-shaped KV-cached decode, dim {cfg.dim}, {attn_desc}, "

@@ -17,8 +17,10 @@
 // The attention kernel streams the cache once: (kvr + dr) * 2 bytes per visible key.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 #include <algorithm>
+#include <mutex>
 
 namespace rdt {
 
@@ -603,6 +605,488 @@ __global__ void __launch_bounds__(256) k_mla_out(MlaDecodeParams p) {
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// k_mla_attn_tc: the latent attention of kv_lora_rank 512 / rope 64 on the tcgen05 tensor
+// cores (same partials as k_mla_attn).  Per (sequence, key range) CTA, tiles of 128 keys:
+//   S^T[key, head]   = C Qa^T (latent) and R Qr^T (rope)     M = 128 keys, N = 32 heads
+//   U^T[dim, head]  += C^T P'^T                               M = 128 dims (x 4), N = 32
+// with C the tile's latent rows [128 keys][512], R its rope rows [128][64], Qa / Qr the
+// absorbed and rope query rows of the sequence (heads past H are zero) and P' = p r_j.
+// Two TMA streams (no multicast), each with its own producer warp and ring, so that the
+// cache keeps streaming while a tile waits for its softmax:
+//   warp 0: the score chunks (four 128-dim latent chunks and the rope chunk of each tile,
+//           32 KB slots) from HBM;
+//   warp 2: the value chunks (the same latent rows again, [64 keys][128 dims] per 16 KB
+//           slot), L2 hits since the score pass read them a tile earlier.
+// Warps 7..10 (thread = key) read each latent score chunk from shared memory as well and
+// sum the key's squares, giving r_j = 1 / sqrt(mean(c_j^2) + eps) per tile; a score slot
+// is free once the MMAs and these four warps are done with it.  Warp 1 owns TMEM and
+// issues the score MMAs, up to three tiles ahead of the softmax (four S buffers in TMEM),
+// so the HBM stream never waits for a softmax; warp 11 issues the value product of each
+// tile after its softmax.  Warps 3..6 (thread = key = TMEM lane) stage the query, then per tile read
+// the scores and the key's r_j, mask, take the per-head
+// tile maximum across the 128 keys, keep a lazy running maximum per head (raised only when
+// a score exceeds it by more than 2^8; then the l sums and U^T are rescaled), and write P'
+// [head][key] (double-buffered) as the B operand of the value product.  At the end they
+// write the unnormalised U rows and (m, l) per head.  Every wait is bounded; a wait that
+// gives up aborts the CTA after its copies and MMAs have drained.
+namespace mtc {
+constexpr int BK = 128, NP = 32, KVR = 512, DR = 64;
+constexpr int BOX = BK * 128;                 // 16 KB: [128 keys][64 dims] bf16, 128-byte swizzle
+constexpr int SSLOT = 2 * BOX, NS = 3;        // score ring: a 128-dim latent chunk or the rope chunk
+constexpr int VBOX = 64 * 128;                // 8 KB: [64 keys][64 dims]
+constexpr int VSLOT = 2 * VBOX, NV = 4;       // value ring: [64 keys][128 dims]
+constexpr int QBOX = NP * 128;                // 4 KB: [32 heads][64 dims] (or [32 heads][64 keys] of P')
+constexpr int NQB = (KVR + DR) / 64;          // 8 latent + 1 rope query boxes
+constexpr int PBUF = 2 * QBOX;                // P' [32 heads][128 keys]
+constexpr int V_OFF = NS * SSLOT, Q_OFF = V_OFF + NV * VSLOT, P_OFF = Q_OFF + NQB * QBOX, BAR_OFF = P_OFF + 2 * PBUF;
+constexpr int NSB = 4, NRB = 8;               // S buffers in TMEM; r_j buffers
+constexpr int SMEM = BAR_OFF + 2048 + NRB * BK * 4 + 1024;   // barriers, reduction scratch, r_j, alignment slack
+constexpr int THREADS = 384;                  // warps: 0 score loads, 1 score MMAs, 2 value loads, 3..6 softmax,
+                                              // 7..10 sums of squares, 11 value MMAs
+constexpr int SMX0 = 96, SSQ0 = 224;          // first softmax / sum-of-squares thread
+constexpr int TMEM_COLS = 512;                // S buffer sb at 64 sb: latent +0, rope +32; U^T at 256 + 32 q
+constexpr int T_U = NSB * 64;
+constexpr float RESCALE_LOG2 = 8.f;
+constexpr unsigned FULL = 0xffffffffu;
+
+// 3-D tile load with an L2 eviction-priority policy (createpolicy): the score pass keeps
+// its lines (evict_last) for the value pass, which reads them for the last time (evict_first).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(tc::smem_u32(dst)),
+      "l"((uint64_t)map), "r"(tc::smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tmem_ld32_raw(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+// Barrier `id` over n threads that also ANDs a predicate across them (every thread gets the
+// same answer, so all leave a loop together).
+__device__ __forceinline__ bool bar_and(bool v, int id, int n) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+// Transposed warp reductions of 32 columns (31 shuffles): lane l ends with the reduction of
+// column l over the warp's lanes.
+template <bool MAX>
+__device__ __forceinline__ float warp_reduce32(const float (&v)[32], int lane) {
+  auto op = [](float x, float y) { return MAX ? fmaxf(x, y) : x + y; };
+  float a[16], b[8], c[4], d[2];
+  bool hi = lane & 16;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a[i] = op(hi ? v[i + 16] : v[i], __shfl_xor_sync(FULL, hi ? v[i] : v[i + 16], 16));
+  hi = lane & 8;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) b[i] = op(hi ? a[i + 8] : a[i], __shfl_xor_sync(FULL, hi ? a[i] : a[i + 8], 8));
+  hi = lane & 4;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = op(hi ? b[i + 4] : b[i], __shfl_xor_sync(FULL, hi ? b[i] : b[i + 4], 4));
+  hi = lane & 2;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) d[i] = op(hi ? c[i + 2] : c[i], __shfl_xor_sync(FULL, hi ? c[i] : c[i + 2], 2));
+  hi = lane & 1;
+  return op(hi ? d[1] : d[0], __shfl_xor_sync(FULL, hi ? d[0] : d[1], 1));
+}
+// A ring of n slots fed by one producer thread and drained by the MMA thread (in order).
+struct Ring {
+  uint64_t* full;
+  uint64_t* empty;
+  int n, c;
+};
+}  // namespace mtc
+
+__global__ void __launch_bounds__(mtc::THREADS, 1)
+    k_mla_attn_tc(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmR,
+                  const __grid_constant__ CUtensorMap tmV, const MlaDecodeParams p, int chunk_tiles) {
+  using namespace tc;
+  using namespace mtc;
+  extern __shared__ uint8_t mtc_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)mtc_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sring = sm;
+  uint8_t* vring = sm + V_OFF;
+  uint8_t* sQ = sm + Q_OFF;
+  uint8_t* sP = sm + P_OFF;
+  uint64_t* sfull = (uint64_t*)(sm + BAR_OFF);
+  uint64_t* sempty = sfull + NS;
+  uint64_t* vfull = sempty + NS;
+  uint64_t* vempty = vfull + NV;
+  uint64_t* q_ready = vempty + NV;
+  uint64_t* s_full = q_ready + 1;    // [NSB] scores of tile t in TMEM buffer t % NSB
+  uint64_t* s_free = s_full + NSB;   // [NSB] the softmax has read them
+  uint64_t* r_ready = s_free + NSB;  // [NRB] r_j of tile t in buffer t % NRB
+  uint64_t* p_full = r_ready + NRB;  // [2] P' of tile t written into buffer t & 1 (one barrier per
+                                     // buffer: the softmax runs ahead of the MMA thread's waits)
+  uint64_t* pv_done = p_full + 2;    // [2] value product of tile t (P' buffer t & 1) complete
+  uint64_t* done = pv_done + 2;       // [2] each MMA issuer's MMAs complete
+  uint32_t* tmem_slot = (uint32_t*)(sm + BAR_OFF + 512);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  float* red = (float*)(sm + BAR_OFF + 1024);   // [2][4][32]
+  float* rbuf = (float*)(sm + BAR_OFF + 2048);  // [NRB][128]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x % p.n_split, b = blockIdx.x / p.n_split;
+  const int n_vis = min(p.q_pos[b] + 1, p.t_max);            // keys 0 .. cache_len[b]
+  const int j0 = split * chunk_tiles * BK;
+  const int j1 = min(j0 + chunk_tiles * BK, n_vis);
+  const int nt = j1 > j0 ? (j1 - j0 + BK - 1) / BK : 0;
+  // first key of tile t: a ragged last tile is moved back to end at j1 (keys before its
+  // nominal start are masked; before key 0 the copy reads zeros)
+  auto tile_start = [&](int t) { const int k = j0 + t * BK; return k + BK <= j1 ? k : j1 - BK; };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&sempty[i], 1 + 4);   // the MMAs' commit and the four sum-of-squares warps
+    }
+    for (int i = 0; i < NV; ++i) {
+      mbar_init(&vfull[i], 1);
+      mbar_init(&vempty[i], 1);
+    }
+    mbar_init(q_ready, 128);
+    for (int i = 0; i < NSB; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 128);
+    }
+    for (int i = 0; i < NRB; ++i) mbar_init(&r_ready[i], 128);
+    mbar_init(&p_full[0], 128);
+    mbar_init(&p_full[1], 128);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
+    mbar_init(&done[0], 1);
+    mbar_init(&done[1], 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if ((warp == 0 || warp == 2) && lane == 0 && nt > 0) {
+    // ---------------- TMA producers: chunks in the order the MMAs consume them ----------------
+    const bool score = warp == 0;
+    Ring rg{score ? sfull : vfull, score ? sempty : vempty, score ? NS : NV, 0};
+    const uint64_t pol = score ? policy_evict_last() : policy_evict_first();
+    int phase[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) phase[i] = -1;
+    auto get = [&](uint32_t bytes) -> int {
+      const int s = rg.c % rg.n;
+      if (!mbar_wait(&rg.empty[s], ((rg.c / rg.n) & 1) ^ 1, abort_flag)) return -1;
+      mbar_expect_tx(&rg.full[s], bytes);
+      phase[s] = (rg.c / rg.n) & 1;
+      ++rg.c;
+      return s;
+    };
+    bool ok = true;
+    for (int t = 0; t < nt && ok; ++t) {
+      const int ks = tile_start(t);
+      if (score) {
+        for (int i = 0; i < 4 && ok; ++i) {
+          const int s = get(SSLOT);
+          if (!(ok = s >= 0)) break;
+          tma_load_3d(sring + s * SSLOT, &tmC, &sfull[s], 128 * i, ks, b, pol);
+          tma_load_3d(sring + s * SSLOT + BOX, &tmC, &sfull[s], 128 * i + 64, ks, b, pol);
+        }
+        if (!ok) break;
+        const int s = get(BOX);
+        if (!(ok = s >= 0)) break;
+        tma_load_3d(sring + s * SSLOT, &tmR, &sfull[s], 0, ks, b, pol);
+      } else {
+        for (int i = 0; i < 4 && ok; ++i)
+          for (int kh = 0; kh < 2 && ok; ++kh) {
+            const int s = get(VSLOT);
+            if (!(ok = s >= 0)) break;
+            tma_load_3d(vring + s * VSLOT, &tmV, &vfull[s], 128 * i, ks + 64 * kh, b, pol);
+            tma_load_3d(vring + s * VSLOT + VBOX, &tmV, &vfull[s], 128 * i + 64, ks + 64 * kh, b, pol);
+          }
+      }
+    }
+    // copies still in flight (an abort) land before the CTA's shared memory is released
+    for (int i = 0; i < rg.n; ++i)
+      if (phase[i] >= 0) mbar_drain(&rg.full[i], (uint32_t)phase[i]);
+  } else if ((warp == 1 || warp == 11) && lane == 0) {
+    // ---------------- MMA issuers: warp 1 the scores, warp 11 the value products ----------------
+    // (separate threads, so neither stream waits behind the other's memory latency; they
+    // write disjoint TMEM columns and each commit tracks its own thread's MMAs)
+    const bool score = warp == 1;
+    if (nt > 0) {
+      constexpr uint32_t ID_S = idesc_bf16(BK, NP);
+      constexpr uint32_t ID_U = idesc_bf16_mn(128, NP, true, false);   // A = C^T: MN-major
+      Ring r = score ? Ring{sfull, sempty, NS, 0} : Ring{vfull, vempty, NV, 0};
+      auto take = [&]() -> int {
+        const int s = r.c % r.n;
+        if (!mbar_wait(&r.full[s], (r.c / r.n) & 1, abort_flag)) return -1;
+        tc_fence_after();
+        ++r.c;
+        return s;
+      };
+      bool ok = true;
+      if (score) {
+        ok = mbar_wait(q_ready, 0, abort_flag);
+        tc_fence_after();
+        // the scores of tile t into TMEM buffer t % NSB once the softmax has read tile t - NSB
+        for (int t = 0; t < nt && ok; ++t) {
+          const int sb = t % NSB;
+          if (t >= NSB && !(ok = mbar_wait(&s_free[sb], ((t / NSB) - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t tS = tmem + 64 * sb;
+          for (int i = 0; i < 4 && ok; ++i) {
+            const int s = take();
+            if (!(ok = s >= 0)) break;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t a = smem_desc(sring + s * SSLOT + (kk >> 2) * BOX) + 2 * (kk & 3);
+              const uint64_t bq = smem_desc(sQ + (2 * i + (kk >> 2)) * QBOX) + 2 * (kk & 3);
+              umma_bf16(tS, a, bq, ID_S, (i > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&sempty[s]);
+          }
+          if (!ok) break;
+          const int s = take();
+          if (!(ok = s >= 0)) break;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tS + 32, smem_desc(sring + s * SSLOT) + 2 * kk, smem_desc(sQ + 8 * QBOX) + 2 * kk, ID_S,
+                      kk > 0 ? 1u : 0u);
+          umma_commit(&sempty[s]);
+          umma_commit(&s_full[sb]);
+        }
+      } else {
+        // the value product of tile t once its P' is written
+        for (int t = 0; t < nt && ok; ++t) {
+          if (!(ok = mbar_wait(&p_full[t & 1], (t >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint8_t* pb = sP + (t & 1) * PBUF;
+          for (int i = 0; i < 4 && ok; ++i)
+            for (int kh = 0; kh < 2; ++kh) {
+              const int s = take();
+              if (!(ok = s >= 0)) break;
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t a = smem_desc_mn(vring + s * VSLOT + kk * 2048, VBOX);   // 16 keys = 2 KB
+                const uint64_t bp = smem_desc(pb + kh * QBOX) + 2 * kk;
+                umma_bf16(tmem + T_U + 32 * i, a, bp, ID_U, (t > 0 || kh > 0 || kk > 0) ? 1u : 0u);
+              }
+              umma_commit(&vempty[s]);
+            }
+          if (ok) umma_commit(&pv_done[t & 1]);
+        }
+      }
+    }
+    // all issued MMAs complete before TMEM is released (also after an abort)
+    umma_commit(&done[score ? 0 : 1]);
+    mbar_drain(&done[score ? 0 : 1], 0);
+  } else if (warp >= 3 && warp <= 6) {
+    // ---------------- softmax: thread = key kl of the tile = TMEM lane ----------------
+    const int quarter = warp & 3, kl = quarter * 32 + lane, st = threadIdx.x - SMX0;
+    const uint32_t lb = (uint32_t)(quarter * 32) << 16;
+    if (nt > 0) {
+      // query rows [32 heads][576] in the 128-byte-swizzled K-major layout; heads past H zero
+      for (int i = st; i < NP * 72; i += 128) {
+        const int n = i / 72, u = i % 72;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (n < p.H) {
+          if (u < 64) v = *reinterpret_cast<const uint4*>((const bf16*)p.qa + ((long long)b * p.H + n) * KVR + 8 * u);
+          else
+            v = *reinterpret_cast<const uint4*>((const bf16*)p.q + (long long)b * p.q_row + (long long)n * p.q_head +
+                                                p.dn + 8 * (u - 64));
+        }
+        *reinterpret_cast<uint4*>(sQ + (u >> 3) * QBOX + n * 128 + (((u & 7) ^ (n & 7)) << 4)) = v;
+      }
+      fence_async_smem();
+      mbar_arrive(q_ready);
+    }
+    const float lg2s = p.scale * 1.4426950408889634f;   // scores in log2 units
+    float m_run = -INFINITY;                             // running maximum of head `lane`
+    float lp[NP];                                        // this key's share of l, per head
+#pragma unroll
+    for (int h = 0; h < NP; ++h) lp[h] = 0.f;
+    bool ok = true;
+    for (int t = 0; t < nt; ++t) {
+      const int sb = t & 1, tb = t % NSB;
+      ok = bar_and(mbar_wait(&s_full[tb], (t / NSB) & 1, abort_flag) &&
+                       mbar_wait(&r_ready[t % NRB], (t / NRB) & 1, abort_flag),
+                   1, 128);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tS = tmem + lb + 64 * tb;
+      uint32_t rl[32], rr[32];
+      tmem_ld32_raw(tS, rl);
+      tmem_ld32_raw(tS + 32, rr);
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(&s_free[tb]);                  // the scores of tile t + NSB may land there
+      const float r = rbuf[(t % NRB) * BK + kl];
+      const int kabs = tile_start(t) + kl;
+      const bool valid = kabs >= j0 + t * BK && kabs < j1;
+      float s[NP];
+#pragma unroll
+      for (int h = 0; h < NP; ++h)
+        s[h] = (valid && h < p.H) ? (__uint_as_float(rl[h]) * r + __uint_as_float(rr[h])) * lg2s : -INFINITY;
+      // the tile's maximum per head over its 128 keys (lane h of every warp: head h)
+      red[(sb * 4 + quarter) * 32 + lane] = warp_reduce32<true>(s, lane);
+      bar_sync(1, 128);
+      const float* rs = red + sb * 128;
+      const float mt = fmaxf(fmaxf(rs[lane], rs[32 + lane]), fmaxf(rs[64 + lane], rs[96 + lane]));
+      float corr = 1.f;
+      if (mt > m_run + RESCALE_LOG2) {
+        corr = exp2f(m_run - mt);
+        m_run = mt;
+      }
+      const bool resc = t > 0 && __any_sync(FULL, corr != 1.f);   // the same in every warp
+      const float base = (m_run == -INFINITY) ? 0.f : m_run;
+      float pr[NP];
+#pragma unroll
+      for (int h = 0; h < NP; ++h) pr[h] = exp2f(s[h] - __shfl_sync(FULL, base, h));
+      if (resc) {
+#pragma unroll
+        for (int h = 0; h < NP; ++h) lp[h] *= __shfl_sync(FULL, corr, h);
+      }
+#pragma unroll
+      for (int h = 0; h < NP; ++h) lp[h] += pr[h];
+      // P' buffer t & 1 was read by the value product of tile t - 2; a rescale of U^T waits
+      // for that of tile t - 1
+      bool w = t < 2 || mbar_wait(&pv_done[sb], ((t >> 1) - 1) & 1, abort_flag);
+      if (w && resc) w = mbar_wait(&pv_done[sb ^ 1], ((t - 1) >> 1) & 1, abort_flag);
+      ok = bar_and(w, 1, 128);
+      if (!ok) break;
+      tc_fence_after();
+      if (resc) {
+        float cf[NP];
+#pragma unroll
+        for (int h = 0; h < NP; ++h) cf[h] = __shfl_sync(FULL, corr, h);
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          float v[32];
+          tmem_ld32(tmem + lb + T_U + 32 * q, v);
+#pragma unroll
+          for (int h = 0; h < NP; ++h) v[h] *= cf[h];
+          tmem_st32(tmem + lb + T_U + 32 * q, v);
+        }
+        tmem_st_wait();
+      }
+      // P'[head][key] = p r_j (the value side sums p r_j c_j), K-major with 128-byte swizzle
+      uint8_t* pcol = sP + sb * PBUF + (kl >> 6) * QBOX + (kl & 7) * 2;
+      const int unit = (kl & 63) >> 3;
+#pragma unroll
+      for (int h = 0; h < NP; ++h)
+        *reinterpret_cast<bf16*>(pcol + h * 128 + ((unit ^ (h & 7)) << 4)) = __float2bfloat16_rn(pr[h] * r);
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[sb]);
+    }
+    // ---- the range's partials: U rows (unnormalised), m (log2 units) and l per head
+    if (ok && nt > 0) ok = bar_and(mbar_wait(&pv_done[(nt - 1) & 1], ((nt - 1) >> 1) & 1, abort_flag), 1, 128);
+    if (ok) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        float v[32];
+        if (nt > 0) {
+          tmem_ld32(tmem + lb + T_U + 32 * q, v);
+        } else {
+#pragma unroll
+          for (int h = 0; h < NP; ++h) v[h] = 0.f;
+        }
+        const int c = 128 * q + kl;
+#pragma unroll
+        for (int h = 0; h < NP; ++h)
+          if (h < p.H) p.part_o[(((long long)b * p.H + h) * p.n_split + split) * KVR + c] = v[h];
+      }
+      const float lw = warp_reduce32<false>(lp, lane);
+      bar_sync(1, 128);   // the last tile's reads of red are done
+      red[quarter * 32 + lane] = lw;
+      bar_sync(1, 128);
+      if (quarter == 0 && lane < p.H) {
+        const long long slot = ((long long)b * p.H + lane) * p.n_split + split;
+        p.part_ml[2 * slot] = m_run;
+        p.part_ml[2 * slot + 1] = red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane];
+      }
+    }
+  } else if (warp >= 7 && warp <= 10) {
+    // ---------------- sums of squares: thread = key kl of the tile ----------------
+    const int kl = threadIdx.x - SSQ0;
+    int c = 0;
+    bool ok = true;
+    for (int t = 0; t < nt && ok; ++t) {
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      for (int ch = 0; ch < 5; ++ch) {          // the tile's four latent chunks, then its rope chunk
+        const int s = c % NS;
+        if (!(ok = mbar_wait(&sfull[s], (c / NS) & 1, abort_flag))) break;
+        if (ch < 4) {
+          const uint8_t* row = sring + s * SSLOT + kl * 128;
+#pragma unroll
+          for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const uint4 v = *reinterpret_cast<const uint4*>(row + bx * BOX + ((u ^ (kl & 7)) << 4));
+              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
+                acc[2 * e] = fmaf(lo, lo, acc[2 * e]);
+                acc[2 * e + 1] = fmaf(hi, hi, acc[2 * e + 1]);
+              }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[s]);
+        ++c;
+        if (ch == 3) {
+          const float ssq = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+          rbuf[(t % NRB) * BK + kl] = rsqrtf(ssq * (1.f / KVR) + p.eps);
+          mbar_arrive(&r_ready[t % NRB]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) record_status(p.st, ST_TIMEOUT, 611, blockIdx.x);
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS) : "memory");
+  }
+}
+
 namespace {
 template <int NTH, int KVR, int DR>
 int launch_attn_t(const MlaDecodeParams& p, cudaStream_t s) {
@@ -634,6 +1118,56 @@ int launch_out_t(const MlaDecodeParams& p, cudaStream_t s) {
   note_launch();
   return 0;
 }
+
+// 3-D bf16 map [d2][d1][d0] (row stride s1 bytes, plane stride s2 bytes), box {64, box1, 1},
+// 128-byte swizzle; coordinates outside the tensor read zeros.
+typedef CUresult (*EncodeTiled3Fn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+bool make_map3(CUtensorMap* m, const void* base, unsigned long long d0, unsigned long long d1, unsigned long long d2,
+               unsigned long long s1, unsigned long long s2, unsigned box1) {
+  static EncodeTiled3Fn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiled3Fn)ptr;
+  });
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {64, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool mla_tc_shape(int H, int kvr, int dr, int t_max) {
+  return kvr == mtc::KVR && dr == mtc::DR && H >= 1 && H <= mtc::NP && t_max >= mtc::BK;
+}
+
+// 1: not this kernel's shape or layout (the caller takes the mma.sync kernel), 0: launched,
+// -1: error.
+int launch_attn_tc(const MlaDecodeParams& p, cudaStream_t s) {
+  if (!mla_tc_shape(p.H, p.kvr, p.dr, p.t_max)) return 1;
+  auto a16 = [](const void* q) { return ((uintptr_t)q & 15) == 0; };
+  if (!a16(p.ckv) || !a16(p.krope) || !a16(p.qa) || !a16(p.q) || p.q_row % 8 || p.q_head % 8 || p.dn % 8) return 1;
+  CUtensorMap mC, mR;
+  const unsigned long long tm = (unsigned long long)p.t_max, B = (unsigned long long)p.B;
+  if (!make_map3(&mC, p.ckv, mtc::KVR, tm, B, mtc::KVR * 2ull, tm * mtc::KVR * 2ull, mtc::BK)) return 1;
+  if (!make_map3(&mR, p.krope, mtc::DR, tm, B, mtc::DR * 2ull, tm * mtc::DR * 2ull, mtc::BK)) return 1;
+  CUtensorMap mV;   // the value chunks: [64 keys][64 dims] boxes of the latent cache
+  if (!make_map3(&mV, p.ckv, mtc::KVR, tm, B, mtc::KVR * 2ull, tm * mtc::KVR * 2ull, 64)) return 1;
+  if (!ensure_smem_limit((const void*)k_mla_attn_tc, mtc::SMEM)) return -1;
+  const int tiles = (p.t_max + mtc::BK - 1) / mtc::BK;
+  const int chunk_tiles = (tiles + p.n_split - 1) / p.n_split;
+  k_mla_attn_tc<<<(unsigned)(p.B * p.n_split), mtc::THREADS, mtc::SMEM, s>>>(mC, mR, mV, p, chunk_tiles);
+  note_launch();
+  return 0;
+}
 }  // namespace
 
 bool mla_decode_supports(int attn_type, int dtype, int H, int kvr, int dr, int dn, int dv) {
@@ -642,12 +1176,25 @@ bool mla_decode_supports(int attn_type, int dtype, int H, int kvr, int dr, int d
   return shape && dn % 8 == 0 && dn >= 8 && dn <= 256 && dv >= 1;
 }
 
-int mla_decode_splits(int B, int H, int t_max) {
+int mla_decode_splits(int B, int H, int kvr, int dr, int t_max) {
+  const int sms = tc_sm_count() > 0 ? tc_sm_count() : 148;
+  if (mla_tc_shape(H, kvr, dr, t_max)) {
+    // tensor-core kernel: one CTA per SM, 128-key tiles; fewest waves x (tiles per range +
+    // about 2 tiles of fixed cost: the query staging, the first scores, the partial write)
+    const int tiles = (t_max + mtc::BK - 1) / mtc::BK;
+    int best = 1;
+    long long best_cost = -1;
+    for (int ns = 1; ns <= std::min(32, tiles); ++ns) {
+      const long long waves = ((long long)B * ns + sms - 1) / sms;
+      const long long cost = waves * ((tiles + ns - 1) / ns + 2);
+      if (best_cost < 0 || cost < best_cost) { best_cost = cost; best = ns; }
+    }
+    return best;
+  }
   // key ranges per sequence: fewest waves x (tiles per range + the fixed cost of a CTA:
   // its query load and partial write, about 1.5 tiles) over the CTA slots of the SMs
   const int kg = mla::kg_for((std::max(H, 1) + 7) / 8);
   const int tile_keys = 32 * kg, per_sm = 3 - kg;
-  const int sms = tc_sm_count() > 0 ? tc_sm_count() : 148;
   const int tiles = std::max(1, (t_max + tile_keys - 1) / tile_keys);
   int best = 1;
   long long best_cost = -1;
@@ -670,7 +1217,10 @@ int launch_mla_decode(const MlaDecodeParams& p, cudaStream_t s) {
   int rc = -1;
   if (p.kvr == 32 && p.dr == 16) rc = launch_attn_h<32, 16>(p, s);
   else if (p.kvr == 128 && p.dr == 32) rc = launch_attn_h<128, 32>(p, s);
-  else if (p.kvr == 512 && p.dr == 64) rc = launch_attn_h<512, 64>(p, s);
+  else if (p.kvr == 512 && p.dr == 64) {
+    rc = launch_attn_tc(p, s);
+    if (rc > 0) rc = launch_attn_h<512, 64>(p, s);
+  }
   if (rc) return rc;
   if (p.kvr == 32) rc = launch_out_t<32>(p, s);
   else if (p.kvr == 128) rc = launch_out_t<128>(p, s);

@@ -129,7 +129,7 @@ struct MlaDecodeParams {
   DevStatus* st;
 };
 bool mla_decode_supports(int attn_type, int dtype, int H, int kvr, int dr, int dn, int dv);
-int mla_decode_splits(int B, int H, int t_max);   // key ranges per sequence (part_o slots)
+int mla_decode_splits(int B, int H, int kvr, int dr, int t_max);   // key ranges per sequence (part_o slots)
 int launch_mla_decode(const MlaDecodeParams& p, cudaStream_t s);
 int tc_sm_count();
 

@@ -142,7 +142,7 @@ void make_layout(const rdt_config* c, int B, int T, int max_keys, Layout* L) {
   L->n_split = (T == 1) ? decode_split_count(std::max(max_keys, 1)) : 0;
   L->part_dim = 128;
   if (L->mla_qa) {
-    L->n_split = mla_decode_splits(B, H, std::max(max_keys, 1));
+    L->n_split = mla_decode_splits(B, H, c->kv_lora_rank, c->qk_rope_head_dim, std::max(max_keys, 1));
     L->part_dim = c->kv_lora_rank;
   }
   L->part_o = take(L->n_split ? (size_t)B * H * L->n_split * L->part_dim * 4 : 16);
