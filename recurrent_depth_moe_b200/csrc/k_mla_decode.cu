@@ -660,6 +660,13 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       "l"((uint64_t)map), "r"(tc::smem_u32(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
       : "memory");
 }
+// (d0, d1) += (a0^2, a1^2) as one packed fp32x2 FMA (two independent fma.rn).
+__device__ __forceinline__ void sq2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n\t.reg .b64 a, c;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 c, {%0, %1};\n\t"
+      "fma.rn.f32x2 c, a, a, c;\n\tmov.b64 {%0, %1}, c;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
@@ -1060,11 +1067,8 @@ __global__ void __launch_bounds__(mtc::THREADS, 1)
               const uint4 v = *reinterpret_cast<const uint4*>(row + bx * BOX + ((u ^ (kl & 7)) << 4));
               const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const float lo = __uint_as_float(w[e] << 16), hi = __uint_as_float(w[e] & 0xffff0000u);
-                acc[2 * e] = fmaf(lo, lo, acc[2 * e]);
-                acc[2 * e + 1] = fmaf(hi, hi, acc[2 * e + 1]);
-              }
+              for (int e = 0; e < 4; ++e)
+                sq2(acc[2 * e], acc[2 * e + 1], __uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
             }
         }
         __syncwarp();
