@@ -145,10 +145,21 @@ def test_mla_absorbed_decode_wide_latent_ragged(H):
     """Absorbed decode at kv_lora_rank 512 against the oracle's decode step, with ragged
     cache lengths: several key ranges, a tile-aligned length + 1, an empty cache (the new
     token alone) and a single cached token."""
+    _wide_case(H, 720, [300, 700, 64, 0, 1])
+
+
+@pytest.mark.parametrize("t_max,lens", [(100, [99, 40, 0]), (128, [127, 5, 64])])
+def test_mla_absorbed_decode_wide_latent_short_caches(t_max, lens):
+    """Caches shorter than one 128-key tile (the mma.sync kernel at kv_lora_rank 512) and
+    exactly one tile (the tensor-core kernel: a full tile, and short sequences whose tile
+    starts before key 0 and reads zeros there)."""
+    _wide_case(24, t_max, lens)
+
+
+def _wide_case(H, t_max, lens):
     cfg = _wide(H)
     W = RI.block_weights(cfg, 60 + H, attn_std=0.05)
-    B, L, t_max = 5, 2, 720
-    lens = [300, 700, 64, 0, 1]
+    B, L = len(lens), 2
     ckv, kr = RI.random_latent_cache(cfg, L, B, t_max, max(lens), 61)
     for b, n in enumerate(lens):
         ckv[:, b, n:] = 0
