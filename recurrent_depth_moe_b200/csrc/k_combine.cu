@@ -32,6 +32,24 @@ template <> struct Vec4<bf16> {
 };
 
 __device__ __forceinline__ float4 f4_add(float4 a, float4 b) { return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w); }
+// Packed fp32x2 arithmetic (two independent fp32 operations per instruction).
+__device__ __forceinline__ float4 f4_add2(float4 a, float4 b) {
+  const float2 lo = __fadd2_rn(make_float2(a.x, a.y), make_float2(b.x, b.y));
+  const float2 hi = __fadd2_rn(make_float2(a.z, a.w), make_float2(b.z, b.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+// a + s b, elementwise
+__device__ __forceinline__ float4 f4_fma2(float s, float4 b, float4 a) {
+  const float2 lo = __ffma2_rn(make_float2(s, s), make_float2(b.x, b.y), make_float2(a.x, a.y));
+  const float2 hi = __ffma2_rn(make_float2(s, s), make_float2(b.z, b.w), make_float2(a.z, a.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+// a + b c, elementwise
+__device__ __forceinline__ float4 f4_fmav2(float4 b, float4 c, float4 a) {
+  const float2 lo = __ffma2_rn(make_float2(b.x, b.y), make_float2(c.x, c.y), make_float2(a.x, a.y));
+  const float2 hi = __ffma2_rn(make_float2(b.z, b.w), make_float2(c.z, c.w), make_float2(a.z, a.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
 template <typename T> __device__ __forceinline__ void store4(T* p, float4 v);
 template <> __device__ __forceinline__ void store4<float>(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
 template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float4 v) {
@@ -204,7 +222,7 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
         const int c = 128 * (j0 + j);
         const float4 a0 = s0 >= 0 ? Vec4<T>::load(y0 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
         const float4 a1 = s1 >= 0 ? Vec4<T>::load(y1 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-        tr[j] = f4_add(tr[j], f4_add(a0, a1));
+        tr[j] = f4_add2(tr[j], f4_add2(a0, a1));
       }
     }
   }
@@ -219,15 +237,31 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
     // reduction, then the group sum; lane q of every warp ends with z[q0 + q]
     for (int q0 = 0; q0 < p.r; q0 += 16) {
       const int nq = min(16, p.r - q0);
+      // ranks q and q + 1 share one packed FMA per element: (part_q, part_q+1) += t (w_q, w_q+1)
+      float2 part2[8];
+#pragma unroll
+      for (int q = 0; q < 16; q += 2) {
+        part2[q / 2] = make_float2(0.f, 0.f);
+        if (q < nq) {
+          const T* w0 = Wd + (long long)(q0 + q) * D + 4 * lane;
+          const T* w1 = w0 + (q + 1 < nq ? D : 0);   // (the odd rank past nq is discarded below)
+#pragma unroll
+          for (int j = 0; j < VQ; ++j) {
+            const float4 a = ld4<T>(w0 + 128 * (j0 + j)), b = ld4<T>(w1 + 128 * (j0 + j)), t = tr[j];
+            float2 acc = part2[q / 2];
+            acc = __ffma2_rn(make_float2(t.x, t.x), make_float2(a.x, b.x), acc);
+            acc = __ffma2_rn(make_float2(t.y, t.y), make_float2(a.y, b.y), acc);
+            acc = __ffma2_rn(make_float2(t.z, t.z), make_float2(a.z, b.z), acc);
+            acc = __ffma2_rn(make_float2(t.w, t.w), make_float2(a.w, b.w), acc);
+            part2[q / 2] = acc;
+          }
+        }
+      }
       float part[16];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        part[q] = 0.f;
-        if (q < nq) {
-          const T* w = Wd + (long long)(q0 + q) * D + 4 * lane;
-#pragma unroll
-          for (int j = 0; j < VQ; ++j) part[q] += f4_dot(tr[j], ld4<T>(w + 128 * (j0 + j)));
-        }
+      for (int q = 0; q < 16; q += 2) {
+        part[q] = part2[q / 2].x;
+        part[q + 1] = (q + 1 < nq) ? part2[q / 2].y : 0.f;
       }
       const float ws = warp_sum16(part, lane);           // sum of part[lane >> 1]
       if (WPR == 1) {
@@ -250,10 +284,7 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
       const T* bq = Bl + (long long)q * D + 4 * lane;
       const float zv = z[q];
 #pragma unroll
-      for (int j = 0; j < VQ; ++j) {
-        float4 v = ld4<T>(bq + 128 * (j0 + j));
-        tr[j].x += zv * v.x; tr[j].y += zv * v.y; tr[j].z += zv * v.z; tr[j].w += zv * v.w;
-      }
+      for (int j = 0; j < VQ; ++j) tr[j] = f4_fma2(zv, ld4<T>(bq + 128 * (j0 + j)), tr[j]);
     }
     __syncwarp();
   }
@@ -267,10 +298,7 @@ __device__ __forceinline__ void combine_row(const CombineParams& p, int i, int l
     float4 av = __ldg(reinterpret_cast<const float4*>(p.A + d));
     float4 bv = __ldg(reinterpret_cast<const float4*>(p.inj_B + d));
     float4 ev = Vec4<T>::load(er + 128 * (j0 + j));
-    tr[j].x += av.x * hv.x + bv.x * ev.x;
-    tr[j].y += av.y * hv.y + bv.y * ev.y;
-    tr[j].z += av.z * hv.z + bv.z * ev.z;
-    tr[j].w += av.w * hv.w + bv.w * ev.w;
+    tr[j] = f4_fmav2(bv, ev, f4_fmav2(av, hv, tr[j]));
     if (p.act_on) zh += f4_dot(tr[j], __ldg(reinterpret_cast<const float4*>(p.halt_wv + d)));
   }
   const bool last = (t == p.n_loops - 1);
