@@ -840,6 +840,8 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD, choices=["rdt1b_prefill", "rdt10b_prefill_zipf"])
     ap.add_argument("--batch", type=int, default=None, help="override the sequences per step (small profiling cases)")
     ap.add_argument("--loops", type=int, default=None, help="override n_loops (small profiling cases)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override the routed expert count (small profiling cases: the same row shapes in a few GB)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         log("warm-up raised to 3 steps")
@@ -848,9 +850,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     wl = RI.get_workload(args.workload)
-    if args.batch or args.loops:
+    if args.batch or args.loops or args.experts:
         import dataclasses
-        wl = dataclasses.replace(wl, batch=args.batch or wl.batch, n_loops=args.loops or wl.n_loops)
+        wl = dataclasses.replace(wl, batch=args.batch or wl.batch, n_loops=args.loops or wl.n_loops,
+                                 cfg=wl.cfg.replace(n_experts=args.experts) if args.experts else wl.cfg)
     if args.impl == "reference":
         run_reference(args, wl, rank, world)
         return
