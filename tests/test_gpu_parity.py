@@ -50,6 +50,36 @@ def test_recurrent_fp32_matches_oracle(name):
     assert torch.equal(ids.cpu().long(), o_ids)
 
 
+@pytest.mark.parametrize("dim,rank", [(512, 5), (4096, 4), (4096, 8), (4096, 16)])
+def test_combine_lora_staging_modes_fp32(dim, rank):
+    """The combine kernel's LoRA paths ("OpenMythos 분석", Recurrent Block: the depth-wise LoRA
+    of the transformer output) at row widths 512 and 4096 in fp32: both matrices staged in
+    shared memory (rank 5 at 512, odd, so the last pair of ranks has one live rank; rank 4 at
+    4096), the down projection alone (rank 8 at 4096: 128 KB) and neither (rank 16: 256 KB
+    each).  320 rows take the persistent row-group kernel; halting rows freeze along the way.
+    Max relative error <= 1e-4 against the oracle, ids exact.  The attention and halting
+    weights' scale shrinks as 1 / sqrt(dim) so that the query-key and halting logits keep one
+    scale at every width: unscaled, at dim 4096 the oracle's own steps taken in fp32 already
+    drift 2.7e-4 from fp64, past what a 1e-4 bar can separate from a fault; scaled, the drift
+    is below 4e-5 on h_out and the halting weights at every case here."""
+    cfg = RI.RDTConfig(dim=dim, n_heads=dim // 128, n_kv_heads=max(dim // 512, 1), max_seq_len=512,
+                       max_loop_iters=4, n_experts=8, n_shared_experts=1, n_experts_per_tok=2, expert_dim=128,
+                       lora_rank=rank, dtype="fp32")
+    sc = math.sqrt(512 / dim)
+    W = RI.block_weights(cfg, 300 + rank, attn_std=0.08 * sc, halt_w_std=0.2 * sc, lora_scale_std=1.0)
+    B, T, L, thr = 1, 320, 3, 0.99
+    h0, e = RI.recurrent_inputs(cfg, B, T, 301)
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    h_out, hw, ids = blk.forward(h0.cuda(), e.cuda(), B, T, L, thr)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    o_h, o_hw, o_ids, _ = O.recurrent_forward(cfg, W, h0, e, B, L, thr)
+    assert max_rel(h_out, o_h) <= FP32_TOL
+    assert max_rel(hw, o_hw) <= FP32_TOL
+    assert torch.equal(ids.cpu().long(), o_ids)
+    assert (halting_loop(o_hw) < L - 1).any(), "some rows halt before the last loop"
+
+
 def test_tiny_gqa_fp32_model_logits():
     """The usage script's tiny GQA model end to end: logits (2, 16, 1000)."""
     wl = RI.get_workload("tiny_gqa_fp32")
