@@ -156,11 +156,22 @@ def test_mla_absorbed_decode_wide_latent_short_caches(t_max, lens):
     _wide_case(24, t_max, lens)
 
 
-def _wide_case(H, t_max, lens):
+def test_mla_absorbed_decode_rescales_as_rope_scores_grow():
+    """The tensor-core latent attention with a running maximum that keeps rising: k_rope is
+    scaled by 1 + j / 32 at position j (the latent part is scale-free: its RMSNorm factor r_j
+    cancels any scaling of c_j), so the rope scores grow along the cache and pass the previous
+    maximum by more than the lazy-rescale threshold (2^8) tile after tile; the rescales of the
+    running sums and of U^T in TMEM must hold."""
+    _wide_case(24, 720, [700, 300, 129, 1], rope_growth=True)
+
+
+def _wide_case(H, t_max, lens, rope_growth=False):
     cfg = _wide(H)
     W = RI.block_weights(cfg, 60 + H, attn_std=0.05)
     B, L = len(lens), 2
     ckv, kr = RI.random_latent_cache(cfg, L, B, t_max, max(lens), 61)
+    if rope_growth:
+        kr = kr * (1.0 + torch.arange(t_max, dtype=torch.float64) / 32).to(kr.dtype)[None, None, :, None]
     for b, n in enumerate(lens):
         ckv[:, b, n:] = 0
         kr[:, b, n:] = 0

@@ -282,6 +282,44 @@ def test_invalid_arguments_return_errors():
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_decode_rescales_as_key_scores_grow(dtype):
+    """Decode attention whose running maximum keeps rising: the cached keys are scaled by
+    1 + j / 32 at position j (fp32), so a query's largest score grows about 30-fold along a
+    1000-key cache and passes the previous maximum by more than the lazy-rescale threshold
+    (2^8) on 6-9 of its 16 tiles; every rescale of the running sum and output must hold.
+    bf16 takes 1 + j / 160 (3-4 raises, scores up to about 30): at scores near 100 the bf16
+    rounding of the query alone moves a score by about 0.2, which the 2e-2 bar would not
+    separate from a fault.  Ragged lengths (1000, 600, 129 keys) put the growth in one key
+    range and across ranges."""
+    cfg = RI.RDTConfig(dim=768, n_heads=6, n_kv_heads=2, max_seq_len=1100, max_loop_iters=2, n_experts=8,
+                       n_shared_experts=1, n_experts_per_tok=2, expert_dim=128, lora_rank=8, dtype=dtype)
+    W = RI.block_weights(cfg, 24, attn_std=0.05)
+    B, L, t_max = 3, 2, 1100
+    lens = [1000, 600, 129]
+    k, v = RI.random_kv_cache(cfg, L, B, t_max, max(lens), 25)
+    grow = (1.0 + torch.arange(t_max, dtype=torch.float64) / (32 if dtype == "fp32" else 160)).to(k.dtype)
+    k = k * grow[None, None, None, :, None]
+    for b, n in enumerate(lens):
+        k[:, b, :, n:] = 0
+        v[:, b, :, n:] = 0
+    h0, e = RI.decode_inputs(cfg, B, 0, 26)
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    cache = R.KVCache(k.cuda(), v.cuda())
+    clen = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    d_h, d_hw, d_ids = blk.decode_step(h0.cuda(), e.cuda(), clen, cache, L, 0.0)
+    torch.cuda.synchronize()
+    assert blk.read_status() == 0
+    caches = [[{"k": k[t, b, :, :lens[b]].permute(1, 0, 2), "v": v[t, b, :, :lens[b]].permute(1, 0, 2),
+                "pos": torch.arange(lens[b])} for b in range(B)] for t in range(L)]
+    o_h, o_hw, o_ids, _ = O.decode_step(cfg, W, h0, e, caches, lens, L, 0.0)
+    if dtype == "fp32":
+        assert max_rel(d_h, o_h) <= FP32_TOL
+    else:
+        for b in range(B):
+            assert rel_l2(d_h[b], o_h[b]) <= BF16_TOL, b
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 def test_decode_random_cache_ragged_lengths(dtype):
     """Decode step against random per-loop caches (the 3B decode workload's structure:
     GQA group 3, one cache per loop) with a different cache length per sequence."""
