@@ -145,7 +145,15 @@ enum {
    * waits run out (about 2 s), it frees its TMEM with nothing in flight, and the device
    * status word reads RDT_ERR_DEVICE_TIMEOUT.  Needs bf16 and a tensor-core shape, else
    * RDT_ERR_UNSUPPORTED.  Exercises the timeout path without faulting the context. */
-  RDT_FLAG_TEST_GEMM_TIMEOUT = 2
+  RDT_FLAG_TEST_GEMM_TIMEOUT = 2,
+  /* test only (no counterpart on the pages): a one-token call on an MLA latent cache runs
+   * loop 0 up to its absorbed latent attention, launches that attention on the tensor
+   * cores with its TMA producers idle, and returns without launching anything else;
+   * outputs are not written.  The attention's bounded waits run out (about 2 s), every
+   * warp role leaves with nothing in flight, TMEM is freed, and the device status word
+   * reads RDT_ERR_DEVICE_TIMEOUT.  Needs bf16, kv_lora_rank 512, rope 64, H <= 32 and a
+   * cache of at least 128 positions (the tensor-core kernel), else RDT_ERR_UNSUPPORTED. */
+  RDT_FLAG_TEST_MLA_ATTN_TIMEOUT = 4
 };
 
 /* Bytes of workspace needed by rdt_recurrent_forward / rdt_recurrent_decode_step /

@@ -17,6 +17,7 @@ RDT_OK, RDT_ERR_INVALID_ARG, RDT_ERR_UNSUPPORTED, RDT_ERR_WORKSPACE, RDT_ERR_CUD
     RDT_ERR_DEVICE_BOUNDS = range(7)
 RDT_FLAG_TRANSFORMER_OFF = 1
 RDT_FLAG_TEST_GEMM_TIMEOUT = 2
+RDT_FLAG_TEST_MLA_ATTN_TIMEOUT = 4
 
 
 class RdtError(RuntimeError):

@@ -821,7 +821,8 @@ __global__ void __launch_bounds__(mtc::THREADS, 1)
       return s;
     };
     bool ok = true;
-    for (int t = 0; t < nt && ok; ++t) {
+    const int n_load = p.test_no_loads ? 0 : nt;   // test only: idle producers, so the waits run out
+    for (int t = 0; t < n_load && ok; ++t) {
       const int ks = tile_start(t);
       if (score) {
         for (int i = 0; i < 4 && ok; ++i) {
@@ -1213,6 +1214,7 @@ int mla_decode_splits(int B, int H, int kvr, int dr, int t_max) {
 int launch_mla_decode(const MlaDecodeParams& p, cudaStream_t s) {
   if (p.B <= 0) return 0;
   if (p.n_split < 1 || p.n_split > 32) return -1;
+  if (p.test_no_loads) return launch_attn_tc(p, s) == 0 ? 0 : -1;   // test only: the attention alone
   {
     dim3 grid((unsigned)p.H, (unsigned)((p.kvr + qab::BC - 1) / qab::BC), (unsigned)((p.B + qab::BB - 1) / qab::BB));
     k_mla_q_absorb<<<grid, 128, 0, s>>>(p);

@@ -127,6 +127,7 @@ struct MlaDecodeParams {
   float* part_o; float* part_ml; int n_split;   // [B][H][n_split][kvr], [B][H][n_split][2]
   void* o; long long o_row;                     // attention output [B][H dv]
   DevStatus* st;
+  int test_no_loads;                            // test only: the tensor-core attention alone, producers idle
 };
 bool mla_decode_supports(int attn_type, int dtype, int H, int kvr, int dr, int dn, int dv);
 int mla_decode_splits(int B, int H, int kvr, int dr, int t_max);   // key ranges per sequence (part_o slots)

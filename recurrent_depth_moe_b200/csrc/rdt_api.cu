@@ -166,6 +166,8 @@ struct Ctx {
   int dtype;
   const int* row_loop = nullptr;   // decode rows at their own loop depth (continuous depth-wise batching)
   bool compact_q = false;          // prefill with ACT: attention queries and O projection on the running rows
+  bool test_mla_timeout = false;   // test only: RDT_FLAG_TEST_MLA_ATTN_TIMEOUT
+  bool test_mla_done = false;      // ... and its attention was launched
 };
 
 #define RDT_TRY(x)                          \
@@ -341,6 +343,11 @@ rdt_status attention_block(Ctx& x, int B, int T, const float* combined, const vo
         mp.qa = at<void*>(x.ws, x.L.mla_qa);
         mp.part_o = at<float*>(x.ws, x.L.part_o); mp.part_ml = at<float*>(x.ws, x.L.part_ml); mp.n_split = x.L.n_split;
         mp.o = attn; mp.o_row = (long long)H * dv; mp.st = x.st;
+        if (x.test_mla_timeout) {   // the tensor-core attention alone, its producers idle
+          mp.test_no_loads = 1;
+          x.test_mla_done = launch_mla_decode(mp, x.s) == 0;
+          return x.test_mla_done ? RDT_OK : RDT_ERR_UNSUPPORTED;
+        }
         ProfScope ps(PC_ATTN, x.s);
         if (launch_mla_decode(mp, x.s) != 0) return RDT_ERR_CUDA;
       } else if (decode || start_pos > 0) {
@@ -543,6 +550,7 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
   cp.transformer_off = transformer_off;
   cp.loop_dim = c->loop_dim; cp.w_rec = w->rec_norm_w; cp.w_attn = w->attn_norm_w; cp.eps = c->norm_eps;
   cp.combined_out = combined; cp.a_out = a;
+  x.test_mla_timeout = (flags & RDT_FLAG_TEST_MLA_ATTN_TIMEOUT) != 0;
   if (flags & RDT_FLAG_TEST_GEMM_TIMEOUT) {
     // the first projection of loop 0 with an idle producer; nothing reads its output
     GemmParams g = gemm_base(x);
@@ -572,6 +580,10 @@ rdt_status run_recurrent(const rdt_config* c, const rdt_weights* w, const float*
     }
     if (!transformer_off) {
       if ((st = attention_block(x, B, T, combined, a, x1, cache, t, start_pos, decode)) != RDT_OK) return st;
+      if (x.test_mla_timeout) {
+        if (!x.test_mla_done) return RDT_ERR_UNSUPPORTED;
+        return cudaGetLastError() == cudaSuccess ? RDT_OK : RDT_ERR_CUDA;
+      }
       if ((st = moe_block(x, N, x1)) != RDT_OK) return st;
       if (trace && trace->f)
         launch_trace_rows(1, x.dtype, at<void*>(ws, x.L.f), D, trace->row0, trace->n_rows, nullptr,

@@ -47,6 +47,41 @@ def test_gemm_timeout_is_recorded_and_the_context_stays_usable():
     assert rel_l2(h, oh) <= BF16_TOL
 
 
+def test_mla_attention_timeout_is_recorded_and_the_context_stays_usable():
+    """The tensor-core MLA latent attention with its TMA producers idle (test flag): its
+    score-MMA thread's bounded wait gives up, every other warp role sees the abort and
+    leaves with nothing in flight, TMEM is freed, and the status word reads
+    RDT_ERR_DEVICE_TIMEOUT; a normal decode step in the same process then matches the
+    oracle ("OpenMythos 분석", MLA)."""
+    from recurrent_depth_moe_b200 import _native as N
+    cfg = RI.RDTConfig(dim=1536, n_heads=24, n_kv_heads=24, max_seq_len=1024, max_loop_iters=4, n_experts=8,
+                       n_shared_experts=1, n_experts_per_tok=2, expert_dim=128, lora_rank=8, attn_type="mla",
+                       kv_lora_rank=512, q_lora_rank=256, qk_rope_head_dim=64, qk_nope_head_dim=128,
+                       v_head_dim=128, dtype="bf16")
+    W = RI.block_weights(cfg, 71, attn_std=0.05)
+    B, L, t_max, n = 2, 2, 720, 700
+    ckv, kr = RI.random_latent_cache(cfg, L, B, t_max, n, 72)
+    h0, e = RI.decode_inputs(cfg, B, 0, 73)
+    blk = R.RecurrentBlock(cfg, to_dev(W))
+    cache = R.KVCache(ckv.cuda(), kr.cuda())
+    blk.forward(h0.cuda(), e.cuda(), B, 1, L, 0.0, start_pos=n, cache=cache, flags=N.RDT_FLAG_TEST_MLA_ATTN_TIMEOUT)
+    torch.cuda.synchronize()
+    assert blk.read_status() == N.RDT_ERR_DEVICE_TIMEOUT
+    assert blk.read_status() == N.RDT_OK                 # reading clears the word
+    # the same process, the same block: a normal decode step is unaffected (the flagged call
+    # wrote this step's latent entries at position n; the decode step rewrites them)
+    cache = R.KVCache(ckv.cuda(), kr.cuda())
+    clen = torch.full((B,), n, dtype=torch.int32, device="cuda")
+    d_h, _, _ = blk.decode_step(h0.cuda(), e.cuda(), clen, cache, L, 0.0)
+    torch.cuda.synchronize()
+    assert blk.read_status() == N.RDT_OK
+    caches = [[{"c_kv": ckv[t, b, :n], "k_rope": kr[t, b, :n], "pos": torch.arange(n)} for b in range(B)]
+              for t in range(L)]
+    o_h, _, _, _ = O.decode_step(cfg, W, h0, e, caches, [n] * B, L, 0.0)
+    for b in range(B):
+        assert rel_l2(d_h[b], o_h[b]) <= BF16_TOL, b
+
+
 def test_decode_position_out_of_range_is_recorded_and_clamped():
     from recurrent_depth_moe_b200 import _native as N
     cfg = RI.RDTConfig(dim=512, n_heads=4, n_kv_heads=2, max_seq_len=96, max_loop_iters=2, n_experts=8,
