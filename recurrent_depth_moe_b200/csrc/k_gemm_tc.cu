@@ -13,9 +13,11 @@
 //
 // Warp roles (192 threads): warp 0 lane 0 issues TMA loads; warp 1 owns TMEM
 // (alloc / dealloc) and lane 0 issues the MMAs; warps 2..5 are the epilogue, each
-// reading its 32-lane quarter of the accumulator with tcgen05.ld.  The accumulator
-// is double-buffered in TMEM (2 x BN columns) so the epilogue of one tile overlaps
-// the MMAs of the next.  Every mbarrier wait is bounded: on timeout the CTA records
+// reading its 32-lane quarter of the accumulator with tcgen05.ld (one row per lane).
+// The bf16 and residual epilogues pass each 32 x 32 chunk through shared memory, so
+// their global loads and stores cover whole row pieces rather than 16 bytes of 32
+// rows.  The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue
+// of one tile overlaps the MMAs of the next.  Every mbarrier wait is bounded: on timeout the CTA records
 // RDT_ERR_DEVICE_TIMEOUT in the status word and leaves its loops.
 #include "common.cuh"
 #include "kernels.h"
@@ -30,11 +32,19 @@ namespace tc {
 
 constexpr int BM = 128, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
+// Epilogue staging in shared memory, one [32 rows][pitch] block per epilogue warp: fp32 rows
+// of the residual epilogue (pitch 36 floats) or bf16 rows of the stores (pitch 20 words).  Both
+// pitches keep the row-per-lane writes and the row-piece-per-lane reads free of bank conflicts.
+constexpr int RS_LD = 36, BS_LD = 20, RS_BYTES = 4 * 32 * RS_LD * 4;
 
 template <int BN> struct Shape {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  // the fp32 residual and the bf16 epilogues add the per-warp staging blocks
+  static constexpr int smem_bytes(int epi) {
+    return SMEM_BYTES + (epi == EPI_ROUTER || epi == EPI_STORE_F32 ? 0 : RS_BYTES);
+  }
   static constexpr int TMEM_COLS = 2 * BN < 32 ? 32 : 2 * BN;   // power of two >= 32
   static constexpr int B_BOX = BN > 128 ? 128 : BN;             // rows per TMA box
 };
@@ -53,7 +63,13 @@ struct TcArgs {
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z)); }
 
-__device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
+// A warp's 32 rows x 32 columns (lane k holds row k in v) to bf16 rows base + k ld, line-wise:
+// the rows pass through the warp's staging block, then lane l stores 16 bytes of row
+// 8 i + l % 8 (i = 0..3), so each store instruction writes eight whole 64-byte row pieces
+// instead of sixteen bytes of 32 rows.  Rows k >= n_valid are not written.  Every lane of
+// the warp takes part.
+__device__ __forceinline__ void store_rows_bf16x32(uint32_t* stg, int lane, const float (&v)[32], bf16* base,
+                                                   long long ld, int n_valid) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     uint4 u;
@@ -63,8 +79,16 @@ __device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
       __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * q + 2 * j], v[8 * q + 2 * j + 1]);
       w[j] = *reinterpret_cast<uint32_t*>(&h2);
     }
-    reinterpret_cast<uint4*>(dst)[q] = u;
+    *reinterpret_cast<uint4*>(stg + lane * BS_LD + 4 * q) = u;
   }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = 8 * i + (lane & 7), k = lane >> 3;
+    const uint4 u = *reinterpret_cast<const uint4*>(stg + row * BS_LD + 4 * k);
+    if (row < n_valid) *reinterpret_cast<uint4*>(base + row * ld + 8 * k) = u;
+  }
+  __syncwarp();
 }
 
 // RoPE pair index of the first column of a 32-column chunk, or -1 when the chunk is
@@ -182,6 +206,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* done = tempty + 2;
   uint32_t* tmem_slot = (uint32_t*)(done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+  float* epi_stage = (float*)(smem + STAGES * S::STAGE_BYTES + 256);   // RS_BYTES, not for the router
   const GemmParams& p = args.p;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -301,39 +326,59 @@ __global__ void __launch_bounds__(192, 1)
       const TileInfo ti = decode_tile(args, t, m_tiles);
       const bool valid = rl < ti.rows;
       const long long r = (long long)ti.row0 + rl;
-      // output / residual row (EPI_RESID_F32 with a row map: the product's rows are compact)
-      const long long ro = (EPI == EPI_RESID_F32 && p.row_map && valid) ? (long long)p.row_map[r] : r;
-      // the residual does not depend on the accumulator: its first chunk is in flight
-      // while this tile's MMAs finish, and chunk c + 1 while chunk c is stored
-      float4 rcur[EPI == EPI_RESID_F32 ? 8 : 1], rnxt[EPI == EPI_RESID_F32 ? 8 : 1];
-      const float* rrow = (EPI == EPI_RESID_F32 && valid) ? p.resid + ro * p.ld_resid + ti.n0 : nullptr;
-      if (EPI == EPI_RESID_F32 && valid && args.k_splits <= 1) {
+      // fp32 residual epilogue, line-wise: a warp's 32 rows x 32 columns pass through shared
+      // memory, so lane l handles row 4i + l / 8, columns 4 (l % 8) .. + 3 of instruction i and
+      // every residual load and output store covers whole 128-byte lines.  Output / residual
+      // rows go through the row map when the product's rows are compact.  The residual does
+      // not depend on the accumulator: its first chunk is in flight while this tile's MMAs
+      // finish, and chunk c + 1 while chunk c is stored.
+      constexpr bool RES = (EPI == EPI_RESID_F32);
+      long long ro_i[RES ? 8 : 1];
+      bool ok_i[RES ? 8 : 1];
+      float4 rcur[RES ? 8 : 1], rnxt[RES ? 8 : 1];
+      const int c4 = 4 * (lane & 7);
+      if (RES && args.k_splits <= 1) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) rcur[q] = __ldg(reinterpret_cast<const float4*>(rrow) + q);
+        for (int i = 0; i < 8; ++i) {
+          const int rw = quarter * 32 + 4 * i + (lane >> 3);
+          ok_i[i] = rw < ti.rows;
+          const long long rr = (long long)ti.row0 + rw;
+          ro_i[i] = ok_i[i] ? (p.row_map ? (long long)p.row_map[rr] : rr) : 0;
+          if (ok_i[i]) rcur[i] = __ldg(reinterpret_cast<const float4*>(p.resid + ro_i[i] * p.ld_resid + ti.n0 + c4));
+        }
       }
       // warp-uniform outcome: the TMEM loads below are .sync.aligned, so a wait that gave up
       // in some lanes only must not let the others go on to them
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, abort_flag))) break;
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(quarter * 32) << 16) + acc * BN;
-      if (EPI == EPI_RESID_F32 && args.k_splits <= 1) {
+      uint32_t* const bstg = reinterpret_cast<uint32_t*>(epi_stage) + (warp - 2) * 32 * BS_LD;
+      if (RES && args.k_splits <= 1) {
+        float* stg = epi_stage + (warp - 2) * 32 * RS_LD;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
-          if (valid && c + 32 < BN) {
+          if (c + 32 < BN) {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) rnxt[q] = __ldg(reinterpret_cast<const float4*>(rrow + c + 32) + q);
+            for (int i = 0; i < 8; ++i)
+              if (ok_i[i])
+                rnxt[i] = __ldg(reinterpret_cast<const float4*>(p.resid + ro_i[i] * p.ld_resid + ti.n0 + c + 32 + c4));
           }
           float v[32];
           tmem_ld32(tbase + c, v);
-          if (valid) {
-            float4* dst = reinterpret_cast<float4*>((float*)p.C + ro * p.ldc + ti.n0 + c);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              dst[q] = make_float4(rcur[q].x + v[4 * q], rcur[q].y + v[4 * q + 1], rcur[q].z + v[4 * q + 2],
-                                   rcur[q].w + v[4 * q + 3]);
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(stg + lane * RS_LD + 4 * q) =
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          __syncwarp();
 #pragma unroll
-            for (int q = 0; q < 8; ++q) rcur[q] = rnxt[q];
+          for (int i = 0; i < 8; ++i) {
+            const float4 a = *reinterpret_cast<const float4*>(stg + (4 * i + (lane >> 3)) * RS_LD + c4);
+            if (ok_i[i])
+              *reinterpret_cast<float4*>((float*)p.C + ro_i[i] * p.ldc + ti.n0 + c + c4) =
+                  make_float4(rcur[i].x + a.x, rcur[i].y + a.y, rcur[i].z + a.z, rcur[i].w + a.w);
+            rcur[i] = rnxt[i];
           }
+          __syncwarp();
         }
       } else if (EPI == EPI_ROUTER) {
         if (BN == 64 || BN == 128) route_row<(BN == 128 ? 128 : 64)>(p, tbase, valid, r);
@@ -345,23 +390,24 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld32(tbase + BN / 2 + c, u);
 #pragma unroll
           for (int j = 0; j < 32; ++j) g[j] = silu_f(g[j]) * u[j];
-          if (valid) store_bf16x32((bf16*)p.C + r * p.ldc + ti.n0 + c, g);
+          store_rows_bf16x32(bstg, lane, g, (bf16*)p.C + (long long)(ti.row0 + quarter * 32) * p.ldc + ti.n0 + c,
+                             p.ldc, ti.rows - quarter * 32);
         }
       } else {
         const float rs = (EPI == EPI_GATE_T && valid) ? p.row_scale[r] : 0.f;
         const int pos = (EPI == EPI_ROPE_T && valid) ? p.pos[r] : 0;
+        bf16* const crow0 = (bf16*)p.C + (long long)(ti.row0 + quarter * 32) * p.ldc;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           float v[32];
           tmem_ld32(tbase + c, v);
-          if (!valid) continue;
           const int col = ti.n0 + c;
           if (EPI == EPI_STORE_T) {
-            store_bf16x32((bf16*)p.C + r * p.ldc + col, v);
+            store_rows_bf16x32(bstg, lane, v, crow0 + col, p.ldc, ti.rows - quarter * 32);
           } else if (EPI == EPI_GATE_T) {
 #pragma unroll
             for (int q = 0; q < 32; ++q) v[q] *= rs;
-            store_bf16x32((bf16*)p.C + r * p.ldc + col, v);
+            store_rows_bf16x32(bstg, lane, v, crow0 + col, p.ldc, ti.rows - quarter * 32);
           } else if (EPI == EPI_ROPE_T) {
             const int m0 = rope_chunk(p, col);
             if (m0 >= 0) {
@@ -376,8 +422,8 @@ __global__ void __launch_bounds__(192, 1)
                 v[4 * q + 3] = b0 * cs.w + b1 * cs.z;
               }
             }
-            store_bf16x32((bf16*)p.C + r * p.ldc + col, v);
-            if (p.vt && col >= p.vt_col0 && col < p.vt_col0 + p.vt_heads * p.vt_hd) {
+            store_rows_bf16x32(bstg, lane, v, crow0 + col, p.ldc, ti.rows - quarter * 32);
+            if (valid && p.vt && col >= p.vt_col0 && col < p.vt_col0 + p.vt_heads * p.vt_hd) {
               // transposed copy of the values: for each dim, the warp's 32 rows are 32
               // consecutive positions, so every store instruction writes 64 contiguous bytes
               const int vc = col - p.vt_col0, g = vc / p.vt_hd, d0 = vc % p.vt_hd;
@@ -386,7 +432,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
               for (int j = 0; j < 32; ++j) vt[(long long)j * p.vt_ld] = __float2bfloat16_rn(v[j]);
             }
-          } else {
+          } else if (valid) {
             float* dst = (float*)p.C + ti.split * args.split_stride + r * p.ldc + col;
             if (EPI == EPI_RESID_F32) {
               const float4* rs4 = (const float4*)(p.resid + r * p.ld_resid + col);
@@ -484,8 +530,9 @@ int pick_bn(const GemmParams& p, int epi) {
 
 template <int EPI, int BN>
 int launch_tc(const CUtensorMap& mA, const CUtensorMap& mB, const tc::TcArgs& a, int grid, cudaStream_t s) {
-  if (!ensure_smem_limit((const void*)tc::k_gemm_tc<EPI, BN>, tc::Shape<BN>::SMEM_BYTES)) return -1;
-  { tc::k_gemm_tc<EPI, BN><<<grid, 192, tc::Shape<BN>::SMEM_BYTES, s>>>(mA, mB, a); note_launch(); }
+  constexpr int smem = tc::Shape<BN>::smem_bytes(EPI);
+  if (!ensure_smem_limit((const void*)tc::k_gemm_tc<EPI, BN>, smem)) return -1;
+  { tc::k_gemm_tc<EPI, BN><<<grid, 192, smem, s>>>(mA, mB, a); note_launch(); }
   return 0;
 }
 
