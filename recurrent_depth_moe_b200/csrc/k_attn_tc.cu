@@ -440,24 +440,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (ok && ntq > 0 && __all_sync(0xffffffffu, mbar_wait(&pv_done[q], (ntq - 1) & 1, abort_flag))) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      bf16* orow = a.o + (row0 + rl) * a.o_row + (long long)h * HD;
+      // line-wise through shared memory: this query tile's Q block is free now (the last PV
+      // completing means every S MMA that read it has completed too)
+      uint32_t* stg = reinterpret_cast<uint32_t*>(sQ + q * QTILE) + quarter * 32 * BS_LD;
+      bf16* obase = a.o + (row0 + quarter * 32) * a.o_row + (long long)h * HD;
 #pragma unroll 1
       for (int c = 0; c < HD; c += 32) {
         float v[32];
         tmem_ld32(tO + c, v);
-        if (row_valid) {
 #pragma unroll
-          for (int e0 = 0; e0 < 32; e0 += 8) {
-            uint4 u;
-            uint32_t* w = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(v[e0 + 2 * e] * inv, v[e0 + 2 * e + 1] * inv);
-              w[e] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-            *reinterpret_cast<uint4*>(orow + c + e0) = u;
-          }
-        }
+        for (int e = 0; e < 32; ++e) v[e] *= inv;
+        store_rows_bf16x32(stg, lane, v, obase + c, a.o_row, q_rows[q] - quarter * 32);
       }
     }
   }

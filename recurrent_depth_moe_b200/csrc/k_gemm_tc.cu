@@ -33,9 +33,10 @@ namespace tc {
 constexpr int BM = 128, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
 // Epilogue staging in shared memory, one [32 rows][pitch] block per epilogue warp: fp32 rows
-// of the residual epilogue (pitch 36 floats) or bf16 rows of the stores (pitch 20 words).  Both
-// pitches keep the row-per-lane writes and the row-piece-per-lane reads free of bank conflicts.
-constexpr int RS_LD = 36, BS_LD = 20, RS_BYTES = 4 * 32 * RS_LD * 4;
+// of the residual epilogue (pitch 36 floats, which keeps the row-per-lane writes and the
+// line-per-8-lanes reads free of bank conflicts) or bf16 rows of the stores
+// (store_rows_bf16x32, pitch BS_LD words).
+constexpr int RS_LD = 36, RS_BYTES = 4 * 32 * RS_LD * 4;
 
 template <int BN> struct Shape {
   static constexpr int B_BYTES = BN * BK * 2;
@@ -62,34 +63,6 @@ struct TcArgs {
 };
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z)); }
-
-// A warp's 32 rows x 32 columns (lane k holds row k in v) to bf16 rows base + k ld, line-wise:
-// the rows pass through the warp's staging block, then lane l stores 16 bytes of row
-// 8 i + l % 8 (i = 0..3), so each store instruction writes eight whole 64-byte row pieces
-// instead of sixteen bytes of 32 rows.  Rows k >= n_valid are not written.  Every lane of
-// the warp takes part.
-__device__ __forceinline__ void store_rows_bf16x32(uint32_t* stg, int lane, const float (&v)[32], bf16* base,
-                                                   long long ld, int n_valid) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 u;
-    uint32_t* w = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * q + 2 * j], v[8 * q + 2 * j + 1]);
-      w[j] = *reinterpret_cast<uint32_t*>(&h2);
-    }
-    *reinterpret_cast<uint4*>(stg + lane * BS_LD + 4 * q) = u;
-  }
-  __syncwarp();
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int row = 8 * i + (lane & 7), k = lane >> 3;
-    const uint4 u = *reinterpret_cast<const uint4*>(stg + row * BS_LD + 4 * k);
-    if (row < n_valid) *reinterpret_cast<uint4*>(base + row * ld + 8 * k) = u;
-  }
-  __syncwarp();
-}
 
 // RoPE pair index of the first column of a 32-column chunk, or -1 when the chunk is
 // not rotated.  Descriptors are 32-column aligned (checked on the host), so a chunk is

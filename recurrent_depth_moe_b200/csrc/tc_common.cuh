@@ -1,6 +1,7 @@
 // sm_100a building blocks shared by the tensor-core kernels: mbarriers with bounded
 // waits, TMA tile loads (no multicast), tcgen05 MMA / commit / fences, TMEM loads and
-// stores, and the K-major 128-byte-swizzle shared-memory descriptor.
+// stores, the K-major 128-byte-swizzle shared-memory descriptor, and the line-wise store of
+// a warp's accumulator rows.
 #pragma once
 #include "common.cuh"
 #include <cuda.h>
@@ -155,6 +156,38 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+constexpr int BS_LD = 20;
+
+// A warp's 32 rows x 32 columns (lane k holds row k in v, as tcgen05.ld gives them) to bf16
+// rows base + k ld, line-wise: the rows pass through the warp's staging block in shared
+// memory (32 x BS_LD words; the pitch of 20 words keeps the row-per-lane writes and the
+// eight-rows-per-phase reads free of bank conflicts), then lane l stores 16 bytes of row
+// 8 i + l % 8 (i = 0..3), so each store instruction writes eight whole 64-byte row pieces
+// instead of sixteen bytes of 32 rows.  Rows k >= n_valid are not written.  Every lane of
+// the warp takes part.
+__device__ __forceinline__ void store_rows_bf16x32(uint32_t* stg, int lane, const float (&v)[32], bf16* base,
+                                                   long long ld, int n_valid) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 u;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * q + 2 * j], v[8 * q + 2 * j + 1]);
+      w[j] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    *reinterpret_cast<uint4*>(stg + lane * BS_LD + 4 * q) = u;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = 8 * i + (lane & 7), k = lane >> 3;
+    const uint4 u = *reinterpret_cast<const uint4*>(stg + row * BS_LD + 4 * k);
+    if (row < n_valid) *reinterpret_cast<uint4*>(base + row * ld + 8 * k) = u;
+  }
+  __syncwarp();
+}
 
 // generic-proxy shared-memory writes -> visible to the tensor core (async proxy)
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
