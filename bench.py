@@ -130,11 +130,11 @@ class ClockSampler:
 EXPERT_UP_TRAFFIC = {
     # mean over the 16 expert-up launches of one step (ncu --metrics dram__bytes_read.sum,
     # dram__bytes_write.sum on the default prefill command of each workload)
-    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1726028688,
-                      "sha256": "b30f748765052c8d24f148a2449ab0e5685bc432a1f69a610c7e59fcaa377ce6"},
+    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1732270432,
+                      "sha256": "23bcbda33009eccb937cd51cdd9bbc6480e8e26c731bb3e97085bfc76652df69"},
     # mean over the 24 expert-up launches of one step
-    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13132007115,
-                            "sha256": "b30f748765052c8d24f148a2449ab0e5685bc432a1f69a610c7e59fcaa377ce6"},
+    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13174255317,
+                            "sha256": "23bcbda33009eccb937cd51cdd9bbc6480e8e26c731bb3e97085bfc76652df69"},
 }
 
 
