@@ -30,7 +30,7 @@
 namespace rdt {
 namespace tc {
 
-constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int BM = 128, BK = 64;
 constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
 // Epilogue staging in shared memory, one [32 rows][pitch] block per epilogue warp: fp32 rows
 // of the residual epilogue (pitch 36 floats, which keeps the row-per-lane writes and the
@@ -41,6 +41,10 @@ constexpr int RS_LD = 36, RS_BYTES = 4 * 32 * RS_LD * 4;
 template <int BN> struct Shape {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  // ring depth: 192 KB of stages at every width, so the narrow tiles of the decode-sized GEMMs
+  // (one 128-row tile of activations, the weights streaming through) keep as many weight bytes
+  // in flight per CTA as the wide ones
+  static constexpr int STAGES = BN == 64 ? 8 : (BN == 128 ? 6 : 4);
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
   // the fp32 residual and the bf16 epilogues add the per-warp staging blocks
   static constexpr int smem_bytes(int epi) {
@@ -172,19 +176,19 @@ __global__ void __launch_bounds__(192, 1)
   using S = Shape<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = (uint64_t*)(smem + STAGES * S::STAGE_BYTES);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint64_t* full = (uint64_t*)(smem + S::STAGES * S::STAGE_BYTES);
+  uint64_t* empty = full + S::STAGES;
+  uint64_t* tfull = empty + S::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* done = tempty + 2;
   uint32_t* tmem_slot = (uint32_t*)(done + 1);
   volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
-  float* epi_stage = (float*)(smem + STAGES * S::STAGE_BYTES + 256);   // RS_BYTES, not for the router
+  float* epi_stage = (float*)(smem + S::STAGES * S::STAGE_BYTES + 256);   // RS_BYTES, not for the router
   const GemmParams& p = args.p;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < S::STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -224,9 +228,9 @@ __global__ void __launch_bounds__(192, 1)
     // ---------------- TMA producer ----------------
     int stage = 0;
     uint32_t phase = 0;
-    int issued_phase[STAGES];   // phase of the last load issued into each stage (-1: none)
+    int issued_phase[S::STAGES];   // phase of the last load issued into each stage (-1: none)
 #pragma unroll
-    for (int s = 0; s < STAGES; ++s) issued_phase[s] = -1;
+    for (int s = 0; s < S::STAGES; ++s) issued_phase[s] = -1;
     // test hook: a producer that issues nothing starves every consumer wait
     const int n_prod = p.test_no_loads ? 0 : total;
     for (int t = blockIdx.x; t < n_prod && !*abort_flag; t += gridDim.x) {
@@ -250,12 +254,12 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_2d(sa + A_BYTES, &tmB, &full[stage], ks * BK, b0);
         if (BN > 128) tma_load_2d(sa + A_BYTES + S::B_BOX * BK * 2, &tmB, &full[stage], ks * BK, b1);
         issued_phase[stage] = (int)phase;
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
       }
     }
     // copies still in flight (an abort) land before the CTA's shared memory is released
 #pragma unroll
-    for (int s = 0; s < STAGES; ++s)
+    for (int s = 0; s < S::STAGES; ++s)
       if (issued_phase[s] >= 0) mbar_drain(&full[s], (uint32_t)issued_phase[s]);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
@@ -280,7 +284,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int k = 0; k < BK / 16; ++k)
           umma_bf16(d, ad + 2 * k, bd + 2 * k, IDESC, (ks != k0 || k != 0) ? 1u : 0u);
         umma_commit(&empty[stage]);
-        if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
       }
       if (!ok) break;
       umma_commit(&tfull[acc]);
