@@ -130,11 +130,11 @@ class ClockSampler:
 EXPERT_UP_TRAFFIC = {
     # mean over the 16 expert-up launches of one step (ncu --metrics dram__bytes_read.sum,
     # dram__bytes_write.sum on the default prefill command of each workload)
-    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1732270432,
-                      "sha256": "23bcbda33009eccb937cd51cdd9bbc6480e8e26c731bb3e97085bfc76652df69"},
+    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1731794720,
+                      "sha256": "1e9ea0f858ecf6481f2e13e6334bd480b6d009242981ac2c5f19199fb3142e65"},
     # mean over the 24 expert-up launches of one step
-    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13174255317,
-                            "sha256": "23bcbda33009eccb937cd51cdd9bbc6480e8e26c731bb3e97085bfc76652df69"},
+    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13112710581,
+                            "sha256": "1e9ea0f858ecf6481f2e13e6334bd480b6d009242981ac2c5f19199fb3142e65"},
 }
 
 
