@@ -130,11 +130,11 @@ class ClockSampler:
 EXPERT_UP_TRAFFIC = {
     # mean over the 16 expert-up launches of one step (ncu --metrics dram__bytes_read.sum,
     # dram__bytes_write.sum on the default prefill command of each workload)
-    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1731794720,
-                      "sha256": "1e9ea0f858ecf6481f2e13e6334bd480b6d009242981ac2c5f19199fb3142e65"},
+    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1737749824,
+                      "sha256": "df1cac22764788a47b78f30edf7294d9509a1a92409480fd8eb99635e1bb2d35"},
     # mean over the 24 expert-up launches of one step
-    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13112710581,
-                            "sha256": "1e9ea0f858ecf6481f2e13e6334bd480b6d009242981ac2c5f19199fb3142e65"},
+    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13719101781,
+                            "sha256": "df1cac22764788a47b78f30edf7294d9509a1a92409480fd8eb99635e1bb2d35"},
 }
 
 

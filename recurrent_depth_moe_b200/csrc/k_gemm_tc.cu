@@ -31,6 +31,21 @@ namespace rdt {
 namespace tc {
 
 constexpr int BM = 128, BK = 64;
+// Decode-sized grouped expert GEMMs (EPI_SWIGLU_T / EPI_GATE_T at BN = 256 over a tile list of
+// at most TR_SLOTS slot rows; their tiles hold at most TR_ROWS rows each) run with the tokens on
+// the MMA's N side: the stage holds the same
+// boxes (128 token rows, then 256 weight rows), but each MMA takes a 128-row weight box as A and
+// the token box as B, D^T[weight row, token] = W . X^T, with N = the tile's rows rounded up to
+// 16.  An MMA's time follows N (M = 64 costs as much as M = 128; N = 16 / 64 / 128 take about
+// 36 / 48 / 64 cycles against 128 for the full 128 x 256 tile), so an expert segment's last,
+// partial tile costs about its own rows, and decode tiles of a few rows free their stages
+// sooner (3B decode step 17.24 -> 15.97 ms).  Prefill keeps the tokens on M: there the partial
+// tiles in this form measured slower (10B step +1.5%), and full tiles would read the token
+// operand twice (two 128-wide MMAs), a third more shared-memory traffic than one 256-wide MMA.
+//   SwiGLU: gate box -> D_gate, up box -> D_up (128 output columns, N tokens each); the lane of
+//           an output column forms silu(gate) * up for its tokens.
+//   gate:   the two 128-row boxes of W2 -> two accumulators (256 output columns).
+constexpr int TR_ROWS = 64, TR_SLOTS = 1024;
 constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
 // Epilogue staging in shared memory, one [32 rows][pitch] block per epilogue warp: fp32 rows
 // of the residual epilogue (pitch 36 floats, which keeps the row-per-lane writes and the
@@ -64,6 +79,7 @@ struct TcArgs {
   int kb_split;        // k-blocks per split
   long long split_stride;   // elements between the fp32 partials of two splits
   int group_m;         // row tiles per rasterization group (1: column tile fastest)
+  int tr_rows;         // tiles of at most this many rows take the tokens-on-N form (0: none)
 };
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.f + __expf(-z)); }
@@ -269,20 +285,36 @@ __global__ void __launch_bounds__(192, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
+    constexpr bool TRC = (EPI == EPI_SWIGLU_T || EPI == EPI_GATE_T) && BN == 256;
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       if (!(ok = mbar_wait(&tempty[acc], acc_phase ^ 1, abort_flag))) break;
       tc_fence_after();
       const uint32_t d = tmem + acc * BN;
+      const TileInfo ti = decode_tile(args, t, m_tiles);
+      // tokens on N for a small tile of a tile list: its rows rounded up to 16 (N = 16..64)
+      const bool TR = TRC && ti.rows <= args.tr_rows;
+      const uint32_t idesc_tr = idesc_bf16(128, TR ? ((max(ti.rows, 1) + 15) & ~15) : 16);
       int k0, k1;
-      k_range(decode_tile(args, t, m_tiles), k0, k1);
+      k_range(ti, k0, k1);
       for (int ks = k0; ks < k1; ++ks) {
         if (!(ok = mbar_wait(&full[stage], phase, abort_flag))) break;
         tc_fence_after();
         uint8_t* sa = smem + stage * S::STAGE_BYTES;
         const uint64_t ad = smem_desc(sa), bd = smem_desc(sa + A_BYTES);
+        if (TR) {
+          // A = a 128-row weight box, B = the token box; the two boxes into their own accumulators
+          const uint64_t wd1 = smem_desc(sa + A_BYTES + S::B_BOX * BK * 2);
 #pragma unroll
-        for (int k = 0; k < BK / 16; ++k)
-          umma_bf16(d, ad + 2 * k, bd + 2 * k, IDESC, (ks != k0 || k != 0) ? 1u : 0u);
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint32_t accum = (ks != k0 || k != 0) ? 1u : 0u;
+            umma_bf16(d, bd + 2 * k, ad + 2 * k, idesc_tr, accum);
+            umma_bf16(d + 128, wd1 + 2 * k, ad + 2 * k, idesc_tr, accum);
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_bf16(d, ad + 2 * k, bd + 2 * k, IDESC, (ks != k0 || k != 0) ? 1u : 0u);
+        }
         umma_commit(&empty[stage]);
         if (++stage == S::STAGES) { stage = 0; phase ^= 1; }
       }
@@ -356,6 +388,39 @@ __global__ void __launch_bounds__(192, 1)
             rcur[i] = rnxt[i];
           }
           __syncwarp();
+        }
+      } else if ((EPI == EPI_SWIGLU_T || EPI == EPI_GATE_T) && BN == 256 && ti.rows <= args.tr_rows) {
+        // tokens on N: lane = output column (weight row of the box), TMEM columns = the tile's
+        // tokens; for a token the warp's 32 lanes write 32 consecutive columns (64 contiguous bytes)
+        const int n_tok = ti.rows;
+        const int j = quarter * 32 + lane;
+#pragma unroll 1
+        for (int c = 0; c < n_tok; c += 32) {
+          float g[32];
+          tmem_ld32(tbase + c, g);
+          if (EPI == EPI_SWIGLU_T) {
+            float u[32];
+            tmem_ld32(tbase + 128 + c, u);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
+            bf16* col = (bf16*)p.C + (long long)(ti.row0 + c) * p.ldc + ti.n0 + j;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c + i < n_tok) col[(long long)i * p.ldc] = __float2bfloat16_rn(g[i]);
+          } else {
+            float u[32];
+            tmem_ld32(tbase + 128 + c, u);
+            const float gs = (c + lane < n_tok) ? p.row_scale[ti.row0 + c + lane] : 0.f;   // lane i: token c + i
+            bf16* col = (bf16*)p.C + (long long)(ti.row0 + c) * p.ldc + ti.n0 + j;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float s = __shfl_sync(0xffffffffu, gs, i);
+              if (c + i < n_tok) {
+                col[(long long)i * p.ldc] = __float2bfloat16_rn(g[i] * s);
+                col[(long long)i * p.ldc + 128] = __float2bfloat16_rn(u[i] * s);
+              }
+            }
+          }
         }
       } else if (EPI == EPI_ROUTER) {
         if (BN == 64 || BN == 128) route_row<(BN == 128 ? 128 : 64)>(p, tbase, valid, r);
@@ -617,6 +682,7 @@ int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
   a.split_stride = 0;
   a.n_out_tile = (epi == EPI_SWIGLU_T) ? bn / 2 : bn;
   a.n_n = p.N / a.n_out_tile;
+  a.tr_rows = (p.tiles && p.M <= tc::TR_SLOTS && bn == 256 && (epi == EPI_SWIGLU_T || epi == EPI_GATE_T)) ? tc::TR_ROWS : 0;
   a.m_tiles = p.tiles ? 0 : (p.M + tc::BM - 1) / tc::BM;
   a.b_rows_group = p.tiles ? (int)(p.b_group_stride / p.ldb) : 0;
   // weight bytes one row tile sweeps (SwiGLU: gate and up rows): group the row tiles when
