@@ -130,11 +130,11 @@ class ClockSampler:
 EXPERT_UP_TRAFFIC = {
     # mean over the 16 expert-up launches of one step (ncu --metrics dram__bytes_read.sum,
     # dram__bytes_write.sum on the default prefill command of each workload)
-    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1737749824,
-                      "sha256": "df1cac22764788a47b78f30edf7294d9509a1a92409480fd8eb99635e1bb2d35"},
+    "rdt1b_prefill": {"batch": 4, "n_loops": 16, "bytes": 1738791616,
+                      "sha256": "20988b66acaa3c9ae7884b4054f06d19dff31b3b5c797b65bf83a17772fb436f"},
     # mean over the 24 expert-up launches of one step
-    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13719101781,
-                            "sha256": "df1cac22764788a47b78f30edf7294d9509a1a92409480fd8eb99635e1bb2d35"},
+    "rdt10b_prefill_zipf": {"batch": 2, "n_loops": 24, "bytes": 13418124843,
+                            "sha256": "20988b66acaa3c9ae7884b4054f06d19dff31b3b5c797b65bf83a17772fb436f"},
 }
 
 

@@ -31,9 +31,9 @@ namespace rdt {
 namespace tc {
 
 constexpr int BM = 128, BK = 64;
-// Decode-sized grouped expert GEMMs (EPI_SWIGLU_T / EPI_GATE_T at BN = 256 over a tile list of
-// at most TR_SLOTS slot rows; their tiles hold at most TR_ROWS rows each) run with the tokens on
-// the MMA's N side: the stage holds the same
+// Decode-sized grouped expert GEMMs (EPI_SWIGLU_T / EPI_GATE_T at BN = 256 over a tile list
+// with at most TR_ROWS slot rows per expert on average) run their tiles of at most TR_ROWS rows
+// with the tokens on the MMA's N side: the stage holds the same
 // boxes (128 token rows, then 256 weight rows), but each MMA takes a 128-row weight box as A and
 // the token box as B, D^T[weight row, token] = W . X^T, with N = the tile's rows rounded up to
 // 16.  An MMA's time follows N (M = 64 costs as much as M = 128; N = 16 / 64 / 128 take about
@@ -45,7 +45,7 @@ constexpr int BM = 128, BK = 64;
 //   SwiGLU: gate box -> D_gate, up box -> D_up (128 output columns, N tokens each); the lane of
 //           an output column forms silu(gate) * up for its tokens.
 //   gate:   the two 128-row boxes of W2 -> two accumulators (256 output columns).
-constexpr int TR_ROWS = 64, TR_SLOTS = 1024;
+constexpr int TR_ROWS = 64;
 constexpr int A_BYTES = BM * BK * 2;                 // 16 KB
 // Epilogue staging in shared memory, one [32 rows][pitch] block per epilogue warp: fp32 rows
 // of the residual epilogue (pitch 36 floats, which keeps the row-per-lane writes and the
@@ -682,7 +682,15 @@ int launch_gemm_tc(int epi, const GemmParams& p, cudaStream_t s) {
   a.split_stride = 0;
   a.n_out_tile = (epi == EPI_SWIGLU_T) ? bn / 2 : bn;
   a.n_n = p.N / a.n_out_tile;
-  a.tr_rows = (p.tiles && p.M <= tc::TR_SLOTS && bn == 256 && (epi == EPI_SWIGLU_T || epi == EPI_GATE_T)) ? tc::TR_ROWS : 0;
+  {
+    // decode-sized: at most TR_ROWS slot rows per weight group (expert) on average
+    const long long rows_group = (p.tiles && p.ldb > 0) ? p.b_group_stride / p.ldb : 0;
+    const long long groups = rows_group > 0 ? p.b_rows / rows_group : 0;
+    a.tr_rows = (groups > 0 && p.M <= (long long)tc::TR_ROWS * groups && bn == 256 &&
+                 (epi == EPI_SWIGLU_T || epi == EPI_GATE_T))
+                    ? tc::TR_ROWS
+                    : 0;
+  }
   a.m_tiles = p.tiles ? 0 : (p.M + tc::BM - 1) / tc::BM;
   a.b_rows_group = p.tiles ? (int)(p.b_group_stride / p.ldb) : 0;
   // weight bytes one row tile sweeps (SwiGLU: gate and up rows): group the row tiles when
